@@ -1,0 +1,372 @@
+/*
+ * trace_oracle.c -- CPU oracle for TRACE rollout-guided NVFP4 rounding.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, obviously correct
+ * statement of what the GPU path computes.  Only the tests, the smoke check
+ * and the benchmark's CPU-baseline leg load it.  It shares no code, header,
+ * table or helper with the CUDA library, and it never calls it.
+ *
+ * Source of the method: the rcap.io post "TRACE: Rollout-Guided
+ * Quantization-Aware Training for FP4" (2026-10-06):
+ *   - section "rollout-guided rounding": pick, of the two FP4 codewords
+ *     around the training value, the one that agrees with what the rollout
+ *     produced;
+ *   - section "compact cache": keep one mantissa bit per element plus the
+ *     scale metadata;
+ *   - the pseudocode listing: capture (fp4_quantize, low_bits) and the QAT
+ *     forward (z = clip(x/s,-6,6), reconstruct_from_mantissa, fp4_bracket,
+ *     argmin, straight_through_estimator).
+ * The NVFP4 arithmetic (16-element blocks, E4M3 block scales, an fp32
+ * per-tensor scale amax/(6*448), the E2M1 grid {0,.5,1,1.5,2,3,4,6}) is the
+ * format the post's rollout runs in; the pages name NVFP4 but do not spell
+ * it out, so the readings taken here are listed at each step.
+ *
+ * Every floating-point operation below is ONE IEEE-754 binary32 operation
+ * with round-to-nearest-even.  Build with -ffp-contract=off and without
+ * -ffast-math so that the compiler fuses nothing.
+ *
+ * Parity pins: every function here is pinned by tests in tests/ against
+ * brute force (exhaustive nearest-codeword and nearest-E4M3 searches in exact
+ * rationals), library routines (torch bf16 and float8_e4m3fn conversion,
+ * numpy float32 arithmetic), closed forms and the worked straddle example.
+ */
+#include <assert.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* E2M1 magnitudes, indexed by the 3-bit magnitude code. */
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+/* ------------------------------------------------------------------ */
+/* Scalar format helpers                                               */
+/* ------------------------------------------------------------------ */
+
+/* bf16 -> fp32: the bf16 bits are the top half of the fp32 bits (exact). */
+float oracle_bf16_to_f32(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+/* fp32 -> bf16, round to nearest, ties to even, on the 16 dropped bits of
+ * the significand (sign-magnitude, so the same rule holds for negatives;
+ * overflow rounds to infinity as IEEE does).  Finite inputs only. */
+uint16_t oracle_f32_to_bf16(float f) {
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  uint32_t sign = u & 0x80000000u;
+  uint32_t mag = u & 0x7FFFFFFFu;
+  assert(mag <= 0x7F7FFFFFu); /* finite */
+  uint32_t keep = mag >> 16;
+  uint32_t dropped = mag & 0xFFFFu;
+  if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u))) keep += 1u;
+  return (uint16_t)((sign >> 16) | keep);
+}
+
+/* E4M3 (the "fn" variant: bias 7, no infinities, 0x7F/0xFF are NaN) -> fp32. */
+float oracle_e4m3_to_f32(uint8_t b) {
+  int s = (b >> 7) & 1;
+  int e = (b >> 3) & 0xF;
+  int m = b & 7;
+  float v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexpf((float)m, -9);          /* subnormal: m * 2^-9 */
+  else
+    v = ldexpf(1.0f + (float)m / 8.0f, e - 7);
+  return s ? -v : v;
+}
+
+/* Non-negative fp32 -> E4M3, round to nearest with ties to the even
+ * mantissa, saturating: anything that rounds above 448 becomes 448 (0x7E).
+ * Textbook route: split t = f * 2^E with f in [1,2), round (f-1)*8 to an
+ * integer (a carry bumps the exponent); below 2^-6 the grid is m * 2^-9. */
+uint8_t oracle_f32_to_e4m3(float t) {
+  assert(!(t < 0.0f) && !isnan(t));
+  if (t >= 448.0f) return 0x7E;
+  if (t < ldexpf(1.0f, -6)) {
+    double q = nearbyint((double)t * 512.0); /* exact scaling, RNE */
+    return (uint8_t)q;                       /* q == 8 is 2^-6 = 0x08 */
+  }
+  int E;
+  double f = frexp((double)t, &E); /* t = f * 2^E, f in [0.5,1) */
+  f *= 2.0;
+  E -= 1;                          /* f in [1,2) */
+  double q = nearbyint((f - 1.0) * 8.0); /* exact: f has 24 bits */
+  if (q == 8.0) {
+    q = 0.0;
+    E += 1;
+  }
+  int code = ((E + 7) << 3) | (int)q;
+  if (code > 0x7E) code = 0x7E;
+  return (uint8_t)code;
+}
+
+/* Round a clipped magnitude a in [0,6] to the E2M1 grid, ties toward the
+ * code whose mantissa bit (its least significant bit) is 0.  The midpoints
+ * 0.25, 1.25, 2.5 and 5 therefore go down (to codes 0,2,4,6), and 0.75, 1.75
+ * and 3.5 go up (to codes 2,4,6). */
+int oracle_e2m1_rtn(float a) {
+  assert(a >= 0.0f && a <= 6.0f);
+  if (a <= 0.25f) return 0;
+  if (a < 0.75f) return 1;
+  if (a <= 1.25f) return 2;
+  if (a < 1.75f) return 3;
+  if (a <= 2.5f) return 4;
+  if (a < 3.5f) return 5;
+  if (a <= 5.0f) return 6;
+  return 7;
+}
+
+/* fp4_bracket for a clipped magnitude a in [0,6]: the largest codeword <= a
+ * and the smallest >= a.  They coincide when a is itself a codeword. */
+void oracle_e2m1_bracket(float a, int* lo, int* hi) {
+  assert(a >= 0.0f && a <= 6.0f);
+  int l = 0;
+  for (int k = 0; k < 8; ++k)
+    if (kE2M1[k] <= a) l = k;
+  int h = 7;
+  for (int k = 7; k >= 0; --k)
+    if (kE2M1[k] >= a) h = k;
+  *lo = l;
+  *hi = h;
+}
+
+/* The guided choice for one site (QAT forward in the pseudocode listing).
+ * a: |z| after clipping; bit: the cached mantissa bit of the rollout code.
+ * reconstruct_from_mantissa: read as "the bracket member whose mantissa bit
+ * equals the cached bit" -- on the E2M1 code ladder neighbours alternate
+ * that bit, so exactly one member qualifies; when the bracket collapses it
+ * is its single member.  The argmin over the bracket is then taken as the
+ * listing writes it.  Returns the magnitude code of q*. */
+int oracle_guided_code(float a, int bit) {
+  int lo, hi;
+  oracle_e2m1_bracket(a, &lo, &hi);
+  if (lo == hi) return lo;
+  int q_hat = ((lo & 1) == (bit & 1)) ? lo : hi;
+  float d_lo = fabsf(kE2M1[lo] - kE2M1[q_hat]);
+  float d_hi = fabsf(kE2M1[hi] - kE2M1[q_hat]);
+  return (d_lo <= d_hi) ? lo : hi;
+}
+
+/* Dequantised output for a signed code: bf16( (VAL[c] * sbv) * s_g ).
+ * VAL[c] * sbv is exact (at most 2 x 4 significant bits), so the only
+ * roundings are one fp32 multiply and the fp32 -> bf16 step. */
+uint16_t oracle_dequant_bf16(int code, int negative, float sbv, float s_g) {
+  float m = kE2M1[code] * sbv;
+  float v = m * s_g;
+  if (negative) v = -v;
+  return oracle_f32_to_bf16(v);
+}
+
+/* ------------------------------------------------------------------ */
+/* Scale computation shared by capture (rollout) and the comparators    */
+/* ------------------------------------------------------------------ */
+
+/* Global scale of one group: s_g = amax / (6*448), or 1 when amax is 0. */
+float oracle_global_scale(float amax) {
+  if (amax == 0.0f) return 1.0f;
+  return amax / 2688.0f;
+}
+
+/* Block scale: t = bmax / (6 * s_g), then E4M3 with RNE and saturation. */
+uint8_t oracle_block_scale(float bmax, float s_g) {
+  float den6 = 6.0f * s_g;
+  float t = bmax / den6;
+  return oracle_f32_to_e4m3(t);
+}
+
+/* z for one element: x / (s_g * sbv); a zero denominator makes the whole
+ * block a zero block, where z keeps only the sign of x. */
+static float scaled_z(float x, float s_g, float sbv) {
+  float d = s_g * sbv;
+  if (d == 0.0f) return copysignf(0.0f, x);
+  return x / d;
+}
+
+/* Group of a row: offsets[g] <= row < offsets[g+1] (linear search). */
+static int group_of_row(int64_t row, int32_t G, const int64_t* offs) {
+  if (G == 1 || offs == 0) return 0;
+  for (int g = 0; g < G; ++g)
+    if (row >= offs[g] && row < offs[g + 1]) return g;
+  assert(0 && "row outside the group offsets");
+  return -1;
+}
+
+static void check_offsets(int64_t rows, int32_t G, const int64_t* offs) {
+  if (G == 1 || offs == 0) return;
+  assert(offs[0] == 0 && offs[G] == rows);
+  for (int g = 0; g < G; ++g) assert(offs[g] <= offs[g + 1]);
+}
+
+/* The global scale of every row, from the per-group scales. */
+static float* expand_row_scales(int64_t rows, int32_t G, const int64_t* offs,
+                                const float* gscale) {
+  float* r = (float*)malloc((size_t)(rows > 0 ? rows : 1) * sizeof(float));
+  assert(r);
+  for (int64_t i = 0; i < rows; ++i) r[i] = gscale[group_of_row(i, G, offs)];
+  return r;
+}
+
+/* ------------------------------------------------------------------ */
+/* The four operations of the hot path                                 */
+/* ------------------------------------------------------------------ */
+
+/* Steps 1-2 of capture: amax = max |x| over the rows of each group. */
+void oracle_group_amax(const uint16_t* x, int64_t rows, int64_t cols,
+                       int32_t G, const int64_t* offs, float* amax) {
+  assert(G >= 1);
+  check_offsets(rows, G, offs);
+  for (int g = 0; g < G; ++g) {
+    int64_t r0 = (G == 1 || !offs) ? 0 : offs[g];
+    int64_t r1 = (G == 1 || !offs) ? rows : offs[g + 1];
+    float m = 0.0f;
+    for (int64_t i = r0 * cols; i < r1 * cols; ++i) {
+      float a = fabsf(oracle_bf16_to_f32(x[i]));
+      assert(isfinite(a));
+      if (a > m) m = a;
+    }
+    amax[g] = m;
+  }
+}
+
+/* Steps 3-6 of capture for rows whose global scales are known:
+ *   codes : N/2 bytes, element 2k in the low nibble of byte k, 2k+1 high;
+ *           a code is sign<<3 | magnitude code.
+ *   mbits : N/32 words, element i at bit (i & 31) of word (i >> 5).
+ *   scales: N/16 E4M3 bytes, row-major [rows, cols/16]. */
+void oracle_capture_rows(const uint16_t* x, int64_t rows, int64_t cols,
+                         const float* row_gscale, uint8_t* codes,
+                         uint32_t* mbits, uint8_t* scales) {
+  assert(cols % 32 == 0);
+  int64_t n = rows * cols;
+  memset(codes, 0, (size_t)(n / 2));
+  memset(mbits, 0, (size_t)(n / 32) * sizeof(uint32_t));
+  for (int64_t b = 0; b < n / 16; ++b) {
+    float s_g = row_gscale[(b * 16) / cols];
+    float bmax = 0.0f;
+    for (int j = 0; j < 16; ++j) {
+      float a = fabsf(oracle_bf16_to_f32(x[b * 16 + j]));
+      if (a > bmax) bmax = a;
+    }
+    uint8_t sb = oracle_block_scale(bmax, s_g);
+    scales[b] = sb;
+    float sbv = oracle_e4m3_to_f32(sb);
+    for (int j = 0; j < 16; ++j) {
+      int64_t i = b * 16 + j;
+      float z = scaled_z(oracle_bf16_to_f32(x[i]), s_g, sbv);
+      float a = fabsf(z);
+      if (a > 6.0f) a = 6.0f; /* clip(z, -6, 6) */
+      int c = oracle_e2m1_rtn(a);
+      int code = (signbit(z) ? 8 : 0) | c;
+      codes[i / 2] |= (uint8_t)(code << (4 * (i & 1)));
+      mbits[i / 32] |= (uint32_t)(c & 1) << (i & 31); /* low_bits(q_roll, 1) */
+    }
+  }
+}
+
+/* Rollout capture (pseudocode: q_roll = fp4_quantize(x_rollout, scale_roll);
+ * cache = (low_bits(q_roll, b=1), scale_roll)).  gscale: G fp32 scales. */
+void oracle_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
+                    const int64_t* offs, uint8_t* codes, uint32_t* mbits,
+                    uint8_t* scales, float* gscale) {
+  assert(cols % 32 == 0 && G >= 1);
+  float* amax = (float*)malloc((size_t)G * sizeof(float));
+  assert(amax);
+  oracle_group_amax(x, rows, cols, G, offs, amax);
+  for (int g = 0; g < G; ++g) gscale[g] = oracle_global_scale(amax[g]);
+  free(amax);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  oracle_capture_rows(x, rows, cols, rs, codes, mbits, scales);
+  free(rs);
+}
+
+/* One fake-quant forward over rows with given scales.  guided != 0 uses the
+ * cached mantissa bits (TRACE); guided == 0 is plain round-to-nearest (the
+ * vanilla QAT comparator).  mask: bit i set when |z_i| <= 6, z taken before
+ * clipping (straight-through estimator support).  sites: optional signed
+ * code per element. */
+static void fake_quant(const uint16_t* x, int64_t rows, int64_t cols,
+                       const float* row_gscale, const uint32_t* mbits,
+                       const uint8_t* scales, uint16_t* out, uint32_t* mask,
+                       uint8_t* sites, int guided) {
+  assert(cols % 32 == 0);
+  int64_t n = rows * cols;
+  if (mask) memset(mask, 0, (size_t)(n / 32) * sizeof(uint32_t));
+  for (int64_t b = 0; b < n / 16; ++b) {
+    float s_g = row_gscale[(b * 16) / cols];
+    float sbv = oracle_e4m3_to_f32(scales[b]);
+    for (int j = 0; j < 16; ++j) {
+      int64_t i = b * 16 + j;
+      float xv = oracle_bf16_to_f32(x[i]);
+      assert(isfinite(xv));
+      float z = scaled_z(xv, s_g, sbv);
+      float a = fabsf(z);
+      if (mask && a <= 6.0f) mask[i / 32] |= 1u << (i & 31);
+      if (a > 6.0f) a = 6.0f;
+      int c;
+      if (guided)
+        c = oracle_guided_code(a, (int)((mbits[i / 32] >> (i & 31)) & 1u));
+      else
+        c = oracle_e2m1_rtn(a);
+      if (out) out[i] = oracle_dequant_bf16(c, signbit(z) != 0, sbv, s_g);
+      if (sites) sites[i] = (uint8_t)((signbit(z) ? 8 : 0) | c);
+    }
+  }
+}
+
+/* Guided QAT forward for rows with known global scales (row_gscale[r]);
+ * mbits == NULL gives the round-to-nearest comparator instead. */
+void oracle_fake_quant_rows(const uint16_t* x, int64_t rows, int64_t cols,
+                            const float* row_gscale, const uint32_t* mbits,
+                            const uint8_t* scales, uint16_t* out,
+                            uint32_t* mask) {
+  fake_quant(x, rows, cols, row_gscale, mbits, scales, out, mask, 0, mbits != 0);
+}
+
+/* Guided QAT forward on x_train with the rollout's cache (pseudocode:
+ * z = clip(x_train/s); bracket; pick by the cached bit; s * q_star). */
+void oracle_guided_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                       int32_t G, const int64_t* offs, const uint32_t* mbits,
+                       const uint8_t* scales, const float* gscale,
+                       uint16_t* out, uint32_t* mask) {
+  check_offsets(rows, G, offs);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  fake_quant(x_train, rows, cols, rs, mbits, scales, out, mask, 0, 1);
+  free(rs);
+}
+
+/* Plain round-to-nearest fake-quant with the given scales (comparator). */
+void oracle_rtn_fwd(const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
+                    const int64_t* offs, const uint8_t* scales,
+                    const float* gscale, uint16_t* out, uint32_t* mask) {
+  check_offsets(rows, G, offs);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  fake_quant(x, rows, cols, rs, 0, scales, out, mask, 0, 0);
+  free(rs);
+}
+
+/* Diagnostic: the signed code (sign<<3 | magnitude code) that the guided
+ * forward (mbits != NULL) or the round-to-nearest forward (mbits == NULL)
+ * picks at every site, one byte per element.  Used to check the per-site
+ * properties the post states for rollout-guided rounding. */
+void oracle_fake_quant_codes(const uint16_t* x, int64_t rows, int64_t cols,
+                             int32_t G, const int64_t* offs,
+                             const uint32_t* mbits, const uint8_t* scales,
+                             const float* gscale, uint8_t* sites) {
+  check_offsets(rows, G, offs);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  fake_quant(x, rows, cols, rs, mbits, scales, 0, 0, sites, mbits != 0);
+  free(rs);
+}
+
+/* Masked straight-through estimator backward: the gradient passes where the
+ * mask bit is set and is +0.0 elsewhere. */
+void oracle_fq_bwd(const uint16_t* grad_out, const uint32_t* mask, int64_t n,
+                   uint16_t* grad_in) {
+  for (int64_t i = 0; i < n; ++i)
+    grad_in[i] = ((mask[i / 32] >> (i & 31)) & 1u) ? grad_out[i] : (uint16_t)0;
+}

@@ -1,0 +1,163 @@
+"""Brute-force restatement of the NVFP4 rounding decisions, for pinning the
+oracle on tiny inputs.
+
+Nothing here shares an algorithm with ``oracle/trace_oracle.c``: every
+rounding decision is an exhaustive search over the candidate values in exact
+rational arithmetic (``fractions.Fraction``), where the oracle uses threshold
+comparisons and exponent/mantissa arithmetic.  The fp32 operations the format
+prescribes (a division, a product) are taken from numpy float32 arithmetic,
+which is IEEE-754 binary32 with round-to-nearest-even; fp32 -> bf16 is
+torch's CPU conversion (round to nearest even).
+"""
+from __future__ import annotations
+
+from fractions import Fraction
+
+import numpy as np
+import torch
+
+# The signed E2M1 grid as (value, magnitude code).  The mantissa bit of a
+# codeword is the lowest bit of its magnitude code.
+_MAGS = [Fraction(0), Fraction(1, 2), Fraction(1), Fraction(3, 2), Fraction(2),
+         Fraction(3), Fraction(4), Fraction(6)]
+SIGNED_GRID = sorted({(s * m, c) for c, m in enumerate(_MAGS) for s in (1, -1)},
+                     key=lambda t: t[0])
+# +0 and -0 are one point of the grid.
+SIGNED_GRID = [g for i, g in enumerate(SIGNED_GRID) if i == 0 or g[0] != SIGNED_GRID[i - 1][0]]
+
+
+def e4m3_value(byte: int) -> Fraction:
+    """Exact value of a non-negative finite E4M3 (fn) byte 0x00..0x7E."""
+    assert 0 <= byte <= 0x7E
+    e, m = byte >> 3, byte & 7
+    if e == 0:
+        return Fraction(m, 512)
+    return Fraction(8 + m, 8) * (Fraction(2) ** (e - 7))
+
+
+E4M3_TABLE = [(e4m3_value(b), b) for b in range(0x7F)]
+
+
+def brute_e4m3(t: float) -> int:
+    """Nearest E4M3 byte to t >= 0 by exhaustive search; ties to the even
+    mantissa; values beyond 448 saturate to 448."""
+    tq = Fraction(float(np.float32(t)))
+    best = None
+    for v, b in E4M3_TABLE:
+        d = abs(tq - v)
+        if best is None or d < best[0] or (d == best[0] and (b & 1) == 0):
+            best = (d, b)
+    return best[1]
+
+
+def brute_rtn(z: Fraction) -> tuple[Fraction, int]:
+    """Clip z to [-6,6], then nearest signed codeword by exhaustive search;
+    ties go to the codeword whose mantissa bit is 0."""
+    zc = max(Fraction(-6), min(Fraction(6), z))
+    best = None
+    for v, c in SIGNED_GRID:
+        d = abs(zc - v)
+        if best is None or d < best[0] or (d == best[0] and (c & 1) == 0):
+            best = (d, v, c)
+    return best[1], best[2]
+
+
+def brute_bracket(z: Fraction) -> tuple[tuple[Fraction, int], tuple[Fraction, int]]:
+    """The two signed codewords around clip(z): the largest <= and the
+    smallest >=, by exhaustive search."""
+    zc = max(Fraction(-6), min(Fraction(6), z))
+    below = max((g for g in SIGNED_GRID if g[0] <= zc), key=lambda g: g[0])
+    above = min((g for g in SIGNED_GRID if g[0] >= zc), key=lambda g: g[0])
+    return below, above
+
+
+def brute_guided(z: Fraction, bit: int) -> tuple[Fraction, int]:
+    """Of the bracket around clip(z), the member whose mantissa bit equals
+    ``bit``; a collapsed bracket gives its single member."""
+    lo, hi = brute_bracket(z)
+    if lo[0] == hi[0]:
+        return lo
+    return lo if (lo[1] & 1) == bit else hi
+
+
+def f32(x) -> np.float32:
+    return np.float32(x)
+
+
+def bf16_bits_to_float(h: int) -> float:
+    return float(np.array([h << 16], dtype=np.uint32).view(np.float32)[0])
+
+
+def float_to_bf16_bits(v: np.float32) -> int:
+    t = torch.tensor([float(v)], dtype=torch.float32).to(torch.bfloat16)
+    return int(t.view(torch.int16).item()) & 0xFFFF
+
+
+def _signed_code(value: Fraction, mag_code: int, z_negative: bool) -> int:
+    neg = value < 0 or (value == 0 and z_negative)
+    return (8 if neg else 0) | mag_code
+
+
+def brute_pipeline(x_roll: np.ndarray, x_train: np.ndarray, grad: np.ndarray):
+    """Capture on x_roll, guided and RTN fake-quant on x_train, STE backward,
+    for one group, by brute force.  Inputs are bf16 bit arrays [rows, cols].
+    Returns a dict of the same arrays the oracle produces."""
+    rows, cols = x_roll.shape
+    n = rows * cols
+    xr = [bf16_bits_to_float(int(h)) for h in x_roll.reshape(-1)]
+    xt = [bf16_bits_to_float(int(h)) for h in x_train.reshape(-1)]
+    amax = max(abs(v) for v in xr)
+    s_g = f32(1.0) if amax == 0 else f32(amax) / f32(2688.0)
+    den6 = f32(6.0) * s_g
+    codes = np.zeros(n // 2, np.uint8)
+    mbits = np.zeros(n // 32, np.uint32)
+    scales = np.zeros(n // 16, np.uint8)
+    out_g = np.zeros(n, np.uint16)
+    out_r = np.zeros(n, np.uint16)
+    mask = np.zeros(n // 32, np.uint32)
+
+    def zval(x: float, d: np.float32) -> tuple[Fraction, bool]:
+        if d == 0:
+            return Fraction(0), np.signbit(np.float32(x))
+        z = f32(x) / d
+        return Fraction(float(z)), bool(np.signbit(z))
+
+    def deq(value: Fraction, z_negative: bool, sbv: Fraction) -> int:
+        exact = abs(value) * sbv * Fraction(float(s_g))
+        v = f32(float(exact))          # exact product has <= 30 bits: one rounding
+        if value < 0 or (value == 0 and z_negative):
+            v = -v
+        return float_to_bf16_bits(v)
+
+    for b in range(n // 16):
+        blk = range(16 * b, 16 * b + 16)
+        bmax = max(abs(xr[i]) for i in blk)
+        t = f32(bmax) / den6
+        sb = brute_e4m3(float(t))
+        scales[b] = sb
+        sbv = e4m3_value(sb)
+        d = s_g * f32(float(sbv))
+        for i in blk:
+            z, neg = zval(xr[i], d)
+            v, c = brute_rtn(z)
+            codes[i // 2] |= _signed_code(v, c, neg) << (4 * (i & 1))
+            mbits[i // 32] |= (c & 1) << (i & 31)
+    for b in range(n // 16):
+        sbv = e4m3_value(int(scales[b]))
+        d = s_g * f32(float(sbv))
+        for i in range(16 * b, 16 * b + 16):
+            z, neg = zval(xt[i], d)
+            if abs(z) <= 6:
+                mask[i // 32] |= 1 << (i & 31)
+            bit = (int(mbits[i // 32]) >> (i & 31)) & 1
+            vg, _ = brute_guided(z, bit)
+            vr, _ = brute_rtn(z)
+            out_g[i] = deq(vg, neg, sbv)
+            out_r[i] = deq(vr, neg, sbv)
+    g = grad.reshape(-1)
+    gin = np.array([g[i] if (mask[i // 32] >> (i & 31)) & 1 else 0 for i in range(n)],
+                   dtype=np.uint16)
+    return dict(codes=codes, mbits=mbits, scales=scales.reshape(rows, cols // 16),
+                gscale=np.array([s_g], np.float32), out_guided=out_g.reshape(rows, cols),
+                out_rtn=out_r.reshape(rows, cols), mask=mask,
+                grad_in=gin.reshape(rows, cols))
