@@ -1,0 +1,415 @@
+#!/usr/bin/env python
+"""Throughput of the TRACE capture + guided NVFP4 fake-quant hot path on B200.
+
+One step = one pass of the whole path over one synthetic activation site:
+  rollout capture of x_roll  (3 launches: zero accumulators, grid amax, quantise
+                              -> FP4 codes + compact cache of mantissa bits and scales)
+  guided fake-quant forward of x_train with that cache (bf16 out + STE mask)
+  masked straight-through backward of an upstream gradient
+  round-to-nearest fake-quant forward of x_train (the vanilla-QAT comparator)
+
+Workload: the Qwen3-30B-A3B-shaped attention-input site, bf16 [16384, 2048],
+lognormal channel scales, 1% outlier channels x100, 0.5% relative training
+noise (seeded, synthetic).  L2 is flushed (256 MiB write) before every step.
+
+The reported value is algorithmic bytes / time (GB/s): every input read once
+and every output written once per kernel, x_roll read twice by capture (its
+two passes).  Per-element bytes: capture 4.6875, guided 4.3125, backward
+4.125, RTN 4.1875 (+4 bytes per group).  elem/s and the fraction of the
+measured HBM copy bandwidth are reported beside it.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl trace|reference]
+Under torchrun every rank runs its own site (weak scaling, no collective on
+the data path); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "capture & guided fake-quant fwd GB/s (elem/s) and % of B200 HBM roofline"
+ROWS, COLS = 16384, 2048
+WORKLOAD = "attn_in [16384 x 2048] bf16, Qwen3-30B-A3B-shaped attention-input site"
+BYTES_PER_ELEM = {"capture": 4.6875, "guided_fwd": 4.3125, "ste_bwd": 4.125, "rtn_fwd": 4.1875}
+KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<true>",
+                "ste_bwd": "k_ste_bwd", "rtn_fwd": "k_fake_quant<false>"}
+LAUNCHES_PER_STEP = 6  # zero + amax + capture, guided, bwd, rtn
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+CSRC = os.path.join(ROOT, "fp4_quantization_aware_trace_b200", "csrc", "trace_fp4.cu")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["trace", "reference"], default="trace")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU work budget of the oracle baseline leg")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_from_profiles(kernel_key: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or
+    None when the summary is missing or the source changed since."""
+    src_hash = hashlib.sha256(open(CSRC, "rb").read()).hexdigest()[:16]
+    path = os.path.join(PROFILE_DIR, f"{kernel_key}_attn_in_16384x2048.md")
+    if not os.path.exists(path):
+        return None
+    txt = open(path).read()
+    h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
+    if not h or not t or h.group(1) != src_hash:
+        return None
+    return int(t.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return None
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            try:
+                sm.append(float(f[1]))
+                mx = max(mx, float(f[2]))
+            except (ValueError, IndexError):
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def max_over_ranks(values, pg, device):
+    """Element-wise max of per-rank device timings (one all-reduce after the
+    timed region; identity with a single process)."""
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if pg is not None:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_gbs(world: int, n_per_rank: int, bytes_per_elem: float, ms_per_step: float) -> float:
+    """Whole-job algorithmic GB/s: every rank processes its own site of
+    n_per_rank elements per step; the step time is the slowest rank's."""
+    return world * n_per_rank * bytes_per_elem / (ms_per_step * 1e-3) / 1e9
+
+
+def site_seed(rank: int) -> int:
+    """Seed of rank r's site: rank 0 is the workload's own seed (1)."""
+    return 1 + 1000 * rank
+
+
+def make_site(rank: int, device):
+    from fp4_quantization_aware_trace_b200 import inputs
+    return inputs.attention_input(seed=site_seed(rank), rows=ROWS, cols=COLS, device=device)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs (reported baseline / reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_step(oracle, xr, xt, g):
+    codes, mbits, scales, gscale = oracle.capture(xr)
+    out, mask = oracle.guided_fwd(xt, mbits, scales, gscale)
+    oracle.fq_bwd(g, mask)
+    oracle.rtn_fwd(xt, scales, gscale)
+
+
+def cpu_oracle_rate(site, budget_s: float, rows: int | None = None):
+    """Time the oracle, as it stands, on host copies of the workload (or its
+    first `rows` rows); returns (GB/s, elem/s, seconds, sample text)."""
+    import oracle
+    from fp4_quantization_aware_trace_b200 import inputs
+    oracle.build()
+    xr, xt, g = (inputs.bits(t) for t in (site.x_roll, site.x_train, site.grad))
+    if rows is not None:
+        xr, xt, g = xr[:rows].copy(), xt[:rows].copy(), g[:rows].copy()
+    n = xr.size
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(oracle, xr, xt, g)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    per = el / passes
+    bpe = sum(BYTES_PER_ELEM.values())
+    sample = (f"{passes} full step(s) (capture+guided+bwd+rtn) over the first {xr.shape[0]} of "
+              f"{ROWS} rows [{xr.shape[0]} x {COLS}] of the same site, single-threaded C oracle")
+    return n * bpe / per / 1e9, n / per, per, sample
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    site = make_site(0, "cpu")
+    import oracle
+    from fp4_quantization_aware_trace_b200 import inputs
+    oracle.build()
+    sample_rows = 4096
+    xr, xt, g = (inputs.bits(t)[:sample_rows].copy() for t in (site.x_roll, site.x_train, site.grad))
+    n = xr.size
+    for _ in range(args.warmup):
+        oracle_step(oracle, xr, xt, g)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(oracle, xr, xt, g)
+    el = time.perf_counter() - t0
+    bpe = sum(BYTES_PER_ELEM.values())
+    value = n * bpe * args.steps / el / 1e9
+    sample = f"each step: the first {sample_rows} of {ROWS} rows [{sample_rows} x {COLS}]"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "elem_per_s": round(n * args.steps / el, 1),
+        "config": {"workload": WORKLOAD, "rows": sample_rows, "cols": COLS, "groups": 1,
+                   "step": "capture + guided fwd + STE bwd + RTN fwd", "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_trace(args):
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    from fp4_quantization_aware_trace_b200 import ops
+    ops.library()
+
+    site = make_site(rank, dev)
+    xr, xt, g = site.x_roll, site.x_train, site.grad
+    n = xr.numel()
+    cap, ws = ops.alloc_capture(ROWS, COLS, 1, dev)
+    out = torch.empty_like(xt)
+    mask = torch.empty(n // 32, dtype=torch.int32, device=dev)
+    gin = torch.empty_like(g)
+    out_r = torch.empty_like(xt)
+    mask_r = torch.empty_like(mask)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        ops.capture(xr, None, cap, ws, stream)
+        if ev: ev[1].record(stream)
+        ops.guided_fq_fwd(xt, cap, out, mask, stream)
+        if ev: ev[2].record(stream)
+        ops.fq_bwd(g, mask, gin, stream)
+        if ev: ev[3].record(stream)
+        ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, None, out_r, mask_r, stream)
+        if ev: ev[4].record(stream)
+
+    for i in range(max(args.warmup, 3)):
+        flush.fill_(i & 0xFF)
+        step()
+    torch.cuda.synchronize()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        if pg: pg.barrier()
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush.fill_((k + 7) & 0xFF)
+            step(events[k])
+        torch.cuda.synchronize()
+        if pg: pg.barrier()
+    clocks = clk.summary()
+
+    names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
+    per_kernel = {nm: 0.0 for nm in names}
+    total_ms = 0.0
+    for ev in events:
+        total_ms += ev[0].elapsed_time(ev[4])
+        for i, nm in enumerate(names):
+            per_kernel[nm] += ev[i].elapsed_time(ev[i + 1])
+    t_max = max_over_ranks([total_ms] + [per_kernel[nm] for nm in names], pg, dev)
+    total_ms = t_max[0]
+    per_kernel = {nm: t_max[i + 1] for i, nm in enumerate(names)}
+
+    ms_step = total_ms / args.steps
+    bpe = sum(BYTES_PER_ELEM.values())
+    value = job_gbs(world, n, bpe, ms_step)
+    hbm, peak_kind = measured_peaks()
+    kern = {}
+    for nm in names:
+        ms = per_kernel[nm] / args.steps
+        kern[nm] = {"kernel": KERNEL_NAMES[nm], "us": round(ms * 1e3, 2),
+                    "gbs": round(n * BYTES_PER_ELEM[nm] / (ms * 1e-3) / 1e9, 1),
+                    "elem_per_s": round(n / (ms * 1e-3), 1)}
+        kern[nm]["frac_of_hbm"] = round(kern[nm]["gbs"] / hbm, 4)
+    # dominant single-launch kernel (capture is three launches: listed, not chosen)
+    dom = max(["guided_fwd", "ste_bwd", "rtn_fwd"], key=lambda nm: per_kernel[nm])
+    dom_bytes = n * BYTES_PER_ELEM[dom]
+    achieved = kern[dom]["gbs"]
+    traffic = traffic_from_profiles({"guided_fwd": "k_fake_quant_guided", "rtn_fwd": "k_fake_quant_rtn",
+                                     "ste_bwd": "k_ste_bwd"}[dom])
+
+    # --- end-to-end through the C ABI with pinned host buffers -------------
+    e2e = None
+    if not args.no_e2e:
+        hx = [t.cpu().pin_memory() for t in (xr, xt, g)]
+        houts = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
+                 for t in (cap.codes, cap.mbits, cap.scales, cap.gscale, out, mask, gin, out_r, mask_r)]
+        douts = [cap.codes, cap.mbits, cap.scales, cap.gscale, out, mask, gin, out_r, mask_r]
+
+        def e2e_step():
+            xr.copy_(hx[0], non_blocking=True)
+            xt.copy_(hx[1], non_blocking=True)
+            g.copy_(hx[2], non_blocking=True)
+            step()
+            for h, d in zip(houts, douts):
+                h.copy_(d, non_blocking=True)
+
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if pg: pg.barrier()
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], pg, dev)[0] / args.steps
+        h2d = sum(h.numel() * h.element_size() for h in hx)
+        d2h = sum(h.numel() * h.element_size() for h in houts)
+        e2e = {"value": round(job_gbs(world, n, bpe, e2e_ms), 3), "unit": "GB/s",
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "elem_per_s": round(world * n / (e2e_ms * 1e-3), 1)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, eps, per, sample = cpu_oracle_rate(site, args.cpu_seconds)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": sample, "elem_per_s": round(eps, 1), "s_per_step": round(per, 3)}
+
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "elem_per_s": round(world * n / (ms_step * 1e-3), 1),
+        "frac_of_hbm": round(value / world / hbm, 4),
+        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "groups": 1,
+                   "step": "capture + guided fwd + STE bwd + RTN fwd",
+                   "l2": "flushed before every step (256 MiB write)",
+                   "parallelism": f"{world} independent sites, one per GPU (no collective)"},
+        "kernels": kern,
+        "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
+                     "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic,
+                     "algorithmic_bytes": int(dom_bytes)},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_trace(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,231 @@
+"""Thin ctypes binding of libtrace_fp4.so (C ABI in include/trace_fp4.h).
+
+Argument marshalling only: every step of the path runs in the library's
+CUDA kernels.  Tensors must be CUDA tensors; bf16 data is passed by pointer
+as raw 16-bit words.  Calls are asynchronous on the given stream (default:
+torch's current stream).  If the library is missing or fails to load, the
+first call raises -- there is no fallback of any kind.
+
+Method: rcap.io post "TRACE: Rollout-Guided Quantization-Aware Training for
+FP4" -- rollout capture of the compact cache (1 mantissa bit + scales), the
+guided QAT fake-quant forward and its straight-through backward.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libtrace_fp4.so")
+_lock = threading.Lock()
+_lib = None
+
+TRACE_OK = 0
+
+
+class TraceError(RuntimeError):
+    pass
+
+
+def library() -> ctypes.CDLL:
+    """Load libtrace_fp4.so (raises if it is missing: build it with
+    ``python -c 'import __graft_entry__ as g; g.build()'``)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise TraceError(f"{LIB_PATH} is missing: the CUDA library has not been built")
+        lib = ctypes.CDLL(LIB_PATH)
+        P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+        lib.trace_strerror.argtypes = [ctypes.c_int]
+        lib.trace_strerror.restype = ctypes.c_char_p
+        lib.trace_abi_version.argtypes = []
+        lib.trace_abi_version.restype = ctypes.c_int
+        lib.trace_capture_workspace_bytes.argtypes = [i64, i64, i32]
+        lib.trace_capture_workspace_bytes.restype = sz
+        lib.trace_capture.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, sz, P]
+        lib.trace_capture.restype = ctypes.c_int
+        lib.trace_guided_fq_fwd.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, P]
+        lib.trace_guided_fq_fwd.restype = ctypes.c_int
+        lib.trace_fq_bwd.argtypes = [P, P, i64, P, P]
+        lib.trace_fq_bwd.restype = ctypes.c_int
+        lib.trace_rtn_fq_fwd.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
+        lib.trace_rtn_fq_fwd.restype = ctypes.c_int
+        lib.trace_copy_bf16.argtypes = [P, P, i64, P]
+        lib.trace_copy_bf16.restype = ctypes.c_int
+        _lib = lib
+        return lib
+
+
+def _check(status: int, what: str) -> None:
+    if status != TRACE_OK:
+        msg = library().trace_strerror(status).decode()
+        raise TraceError(f"{what}: status {status} ({msg})")
+
+
+def _p(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise TraceError("tensors passed to libtrace_fp4 must be CUDA tensors")
+    if not t.is_contiguous():
+        raise TraceError("tensors passed to libtrace_fp4 must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _groups(offsets: torch.Tensor | None) -> int:
+    if offsets is None:
+        return 1
+    if offsets.dtype != torch.int64:
+        raise TraceError("group offsets must be int64")
+    return int(offsets.numel()) - 1
+
+
+# ---------------------------------------------------------------------------
+# Raw C-ABI calls, same names and argument order as include/trace_fp4.h
+# ---------------------------------------------------------------------------
+
+def trace_capture_workspace_bytes(rows: int, cols: int, num_groups: int) -> int:
+    return int(library().trace_capture_workspace_bytes(rows, cols, num_groups))
+
+
+def trace_capture(x, rows, cols, num_groups, offsets, codes, mbits, scales, gscale,
+                  workspace, workspace_bytes, stream=None) -> None:
+    _check(library().trace_capture(_p(x), rows, cols, num_groups, _p(offsets), _p(codes),
+                                   _p(mbits), _p(scales), _p(gscale), _p(workspace),
+                                   workspace_bytes, _stream(stream)), "trace_capture")
+
+
+def trace_guided_fq_fwd(x_train, rows, cols, num_groups, offsets, mbits, scales, gscale,
+                        out, ste_mask, stream=None) -> None:
+    _check(library().trace_guided_fq_fwd(_p(x_train), rows, cols, num_groups, _p(offsets),
+                                         _p(mbits), _p(scales), _p(gscale), _p(out),
+                                         _p(ste_mask), _stream(stream)), "trace_guided_fq_fwd")
+
+
+def trace_fq_bwd(grad_out, ste_mask, numel, grad_in, stream=None) -> None:
+    _check(library().trace_fq_bwd(_p(grad_out), _p(ste_mask), numel, _p(grad_in),
+                                  _stream(stream)), "trace_fq_bwd")
+
+
+def trace_rtn_fq_fwd(x, rows, cols, num_groups, offsets, scales, gscale, out, ste_mask,
+                     stream=None) -> None:
+    _check(library().trace_rtn_fq_fwd(_p(x), rows, cols, num_groups, _p(offsets), _p(scales),
+                                      _p(gscale), _p(out), _p(ste_mask), _stream(stream)),
+           "trace_rtn_fq_fwd")
+
+
+def trace_copy_bf16(src, dst, numel, stream=None) -> None:
+    _check(library().trace_copy_bf16(_p(src), _p(dst), numel, _stream(stream)), "trace_copy_bf16")
+
+
+# ---------------------------------------------------------------------------
+# Convenience wrappers that allocate their outputs (still no arithmetic here)
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Capture:
+    """What one capture site records: the rollout's full FP4 codes (for its
+    own FP4 GEMM) and the compact cache (mbits + scales + gscale)."""
+    codes: torch.Tensor    # uint8 [N/2]
+    mbits: torch.Tensor    # int32 words [N/32] (bit patterns; uint32 ABI)
+    scales: torch.Tensor   # uint8 [rows, cols/16] E4M3
+    gscale: torch.Tensor   # float32 [G]
+    offsets: torch.Tensor | None = None
+
+    def cache_nbytes(self) -> int:
+        """Bytes of the compact cache (mantissa bits + block and global scales)."""
+        return self.mbits.numel() * 4 + self.scales.numel() + self.gscale.numel() * 4
+
+
+def _bf16_2d(x: torch.Tensor) -> tuple[int, int]:
+    if x.dtype != torch.bfloat16:
+        raise TraceError("activations must be bf16")
+    if x.dim() != 2:
+        raise TraceError("activations must be 2-D [rows, cols]")
+    return int(x.shape[0]), int(x.shape[1])
+
+
+def alloc_capture(rows: int, cols: int, num_groups: int = 1, device="cuda",
+                  offsets: torch.Tensor | None = None) -> tuple[Capture, torch.Tensor]:
+    """Allocate capture outputs and the workspace (torch device memory)."""
+    n = rows * cols
+    cap = Capture(codes=torch.empty(n // 2, dtype=torch.uint8, device=device),
+                  mbits=torch.empty(n // 32, dtype=torch.int32, device=device),
+                  scales=torch.empty(rows, cols // 16, dtype=torch.uint8, device=device),
+                  gscale=torch.empty(num_groups, dtype=torch.float32, device=device),
+                  offsets=offsets)
+    ws = torch.empty(max(trace_capture_workspace_bytes(rows, cols, num_groups), 256),
+                     dtype=torch.uint8, device=device)
+    return cap, ws
+
+
+def capture(x: torch.Tensor, offsets: torch.Tensor | None = None, out: Capture | None = None,
+            workspace: torch.Tensor | None = None, stream=None) -> Capture:
+    """Rollout capture of one site (x bf16 [rows, cols]; offsets int64 [G+1])."""
+    rows, cols = _bf16_2d(x)
+    G = _groups(offsets)
+    if out is None or workspace is None:
+        out, workspace = alloc_capture(rows, cols, G, x.device, offsets)
+    trace_capture(x, rows, cols, G, offsets, out.codes, out.mbits, out.scales, out.gscale,
+                  workspace, workspace.numel(), stream)
+    return out
+
+
+def guided_fq_fwd(x_train: torch.Tensor, cache: Capture, out: torch.Tensor | None = None,
+                  mask: torch.Tensor | None = None, stream=None):
+    """Guided fake-quant forward with a rollout cache.  Returns (out, mask)."""
+    rows, cols = _bf16_2d(x_train)
+    out = torch.empty_like(x_train) if out is None else out
+    mask = torch.empty(rows * cols // 32, dtype=torch.int32, device=x_train.device) if mask is None else mask
+    trace_guided_fq_fwd(x_train, rows, cols, _groups(cache.offsets), cache.offsets, cache.mbits,
+                        cache.scales, cache.gscale, out, mask, stream)
+    return out, mask
+
+
+def rtn_fq_fwd(x: torch.Tensor, scales: torch.Tensor, gscale: torch.Tensor,
+               offsets: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               mask: torch.Tensor | None = None, stream=None):
+    """Round-to-nearest fake-quant with given scales.  Returns (out, mask)."""
+    rows, cols = _bf16_2d(x)
+    out = torch.empty_like(x) if out is None else out
+    mask = torch.empty(rows * cols // 32, dtype=torch.int32, device=x.device) if mask is None else mask
+    trace_rtn_fq_fwd(x, rows, cols, _groups(offsets), offsets, scales, gscale, out, mask, stream)
+    return out, mask
+
+
+def fq_bwd(grad_out: torch.Tensor, mask: torch.Tensor, out: torch.Tensor | None = None,
+           stream=None) -> torch.Tensor:
+    """Masked straight-through backward."""
+    if grad_out.dtype != torch.bfloat16:
+        raise TraceError("gradients must be bf16")
+    out = torch.empty_like(grad_out) if out is None else out
+    trace_fq_bwd(grad_out, mask, grad_out.numel(), out, stream)
+    return out
+
+
+class GuidedFakeQuant(torch.autograd.Function):
+    """Autograd wrapper: forward = guided fake-quant with the rollout cache,
+    backward = masked straight-through estimator (both in the library)."""
+
+    @staticmethod
+    def forward(ctx, x_train, cache: Capture):
+        out, mask = guided_fq_fwd(x_train, cache)
+        ctx.save_for_backward(mask)
+        return out
+
+    @staticmethod
+    def backward(ctx, grad):
+        (mask,) = ctx.saved_tensors
+        return fq_bwd(grad.contiguous(), mask), None

@@ -1,0 +1,150 @@
+/*
+ * trace_fp4.h -- C ABI of the B200 (sm_100a) TRACE rollout-guided NVFP4
+ * rounding library (libtrace_fp4.so).
+ *
+ * The method is the one the rcap.io post "TRACE: Rollout-Guided
+ * Quantization-Aware Training for FP4" (2026-10-06) describes: during the
+ * rollout, every quantisation site records a compact cache (one mantissa bit
+ * per element plus the scale metadata; section "compact cache" and the
+ * capture half of the pseudocode listing); during the QAT forward on the
+ * paired training activation, each element is rounded to whichever of its
+ * two neighbouring FP4 codewords agrees with the rollout (section
+ * "rollout-guided rounding" and the QAT-forward half of the listing), and the
+ * straight-through estimator passes the gradient back.
+ *
+ * Number format (NVFP4, as the post's rollout uses it):
+ *   - x is bf16, row-major [rows, cols], cols a multiple of 32;
+ *   - one fp32 global scale per group: s_g = amax / (6*448), or 1 if amax = 0;
+ *   - one E4M3 block scale per 16 consecutive elements of a row:
+ *     s_b = E4M3(bmax / (6*s_g)), round to nearest even, saturating at 448;
+ *   - z = x / (s_g*s_b) (a zero denominator gives z = +-0), clipped to [-6,6],
+ *     on the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6}; code = sign<<3 | magnitude
+ *     code 0..7; the mantissa bit of a code is its lowest bit.
+ *
+ * Layouts (N = rows*cols, element i = row*cols + col):
+ *   codes   : uint8[N/2]; byte k holds element 2k in its low nibble and
+ *             element 2k+1 in its high nibble.
+ *   mbits   : uint32[N/32]; element i is bit (i & 31) of word (i >> 5).
+ *   scales  : uint8[rows, cols/16] E4M3 bytes, row-major (linear, not the
+ *             swizzled layout of a block-scaled GEMM).
+ *   gscale  : float[G], one per group.
+ *   ste_mask: uint32[N/32], same packing as mbits; bit set where |z| <= 6
+ *             (z before clipping).
+ *   Groups: G >= 1 contiguous row ranges (e.g. the experts of a MoE layer),
+ *   given as int64 device offsets [G+1] with offsets[0] = 0,
+ *   offsets[G] = rows, non-decreasing (empty groups allowed).  NULL offsets
+ *   mean G == 1.
+ *
+ * Ownership and execution: every pointer except `stream` is a DEVICE
+ * pointer owned by the caller; the library never allocates, frees or
+ * synchronises.  All calls are asynchronous on `stream` (a cudaStream_t
+ * passed as void*, NULL = the legacy default stream).  The library holds no
+ * mutable global state apart from a per-device cache of the SM count, so it
+ * may be called from several host threads.
+ *
+ * Errors: arguments are checked on the host before anything is enqueued; a
+ * failed check returns its code and enqueues nothing.  A launch failure
+ * returns TRACE_ERR_CUDA.  Device-side preconditions that the host cannot
+ * see are stated per call; breaking them gives unspecified results (never an
+ * out-of-bounds access in this library's kernels, apart from reading the
+ * offsets array itself, which must hold G+1 entries).
+ *   - inputs are finite bf16 (no NaN or infinity);
+ *   - scale bytes passed to the forward kernels are non-negative finite E4M3
+ *     (0x00..0x7E) and global scales finite and positive, as capture writes;
+ *   - the group offsets satisfy the rules above.
+ * Limits: N/8 < 2^32 (N < 2^35 elements per call).
+ */
+#ifndef TRACE_FP4_H
+#define TRACE_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TRACE_OK = 0,
+  TRACE_ERR_NULL = 1,      /* a required pointer is NULL */
+  TRACE_ERR_SHAPE = 2,     /* rows < 0, cols <= 0, cols % 32, G < 1, size limit */
+  TRACE_ERR_ALIGN = 3,     /* a pointer is not aligned as the call requires */
+  TRACE_ERR_WORKSPACE = 4, /* workspace smaller than the query returned */
+  TRACE_ERR_CUDA = 5       /* a CUDA runtime call or launch failed */
+} trace_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* trace_strerror(int status);
+
+/* ABI version of this header (bumped on any incompatible change). */
+#define TRACE_ABI_VERSION 1
+int trace_abi_version(void);
+
+/* Bytes of device workspace that trace_capture needs for G groups: the
+ * per-group amax accumulators (4 bytes each, rounded up to 256).  Returns 0
+ * when the shape is invalid. */
+size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols,
+                                     int32_t num_groups);
+
+/* Rollout capture: fp4_quantize(x_rollout) plus low_bits(q_roll, 1) and the
+ * scales (the capture half of the post's pseudocode listing; the compact
+ * cache is mbits + scales + gscale, 1.5 bits per element).
+ *   x       : bf16 [rows, cols], 16-byte aligned.
+ *   codes   : out, uint8[N/2], 16-byte aligned (the full NVFP4 codes, for the
+ *             rollout's own FP4 GEMM).
+ *   mbits   : out, uint32[N/32], 16-byte aligned.
+ *   scales  : out, uint8[N/16], 16-byte aligned.
+ *   gscale  : out, float[G], 4-byte aligned.
+ *   workspace: device scratch of at least trace_capture_workspace_bytes()
+ *             bytes, 256-byte aligned; its contents on entry do not matter.
+ * Launches three kernels (zero the accumulators, grid amax, quantise). */
+int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
+                  int32_t num_groups, const int64_t* group_row_offsets,
+                  uint8_t* codes, uint32_t* mbits, uint8_t* scales,
+                  float* gscale, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* Guided QAT fake-quant forward (the QAT-forward half of the listing):
+ * z = clip(x_train / (s_g*s_b), -6, 6) with the ROLLOUT's scales; of the two
+ * codewords bracketing z (one, if z is a codeword) take the one whose
+ * mantissa bit equals the cached bit; out = bf16((q* * s_b) * s_g) with the
+ * sign of z (fp32 product, round to nearest even into bf16); ste_mask bit =
+ * |z| <= 6.
+ *   x_train : bf16 [rows, cols], 16-byte aligned.
+ *   mbits, scales, gscale: the rollout's compact cache (capture's outputs).
+ *   out     : out, bf16 [rows, cols], 16-byte aligned; may alias x_train.
+ *   ste_mask: out, uint32[N/32], 16-byte aligned. */
+int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                        int32_t num_groups, const int64_t* group_row_offsets,
+                        const uint32_t* mbits, const uint8_t* scales,
+                        const float* gscale, uint16_t* out, uint32_t* ste_mask,
+                        void* stream);
+
+/* Masked straight-through-estimator backward:
+ * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
+ *   grad_out, grad_in: bf16 [numel], 16-byte aligned; may alias.
+ *   ste_mask: uint32[numel/32], 16-byte aligned.  numel % 32 == 0. */
+int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask,
+                 int64_t numel, uint16_t* grad_in, void* stream);
+
+/* Plain round-to-nearest fake-quant with given scales (the vanilla QAT
+ * comparator the post measures TRACE against): as trace_guided_fq_fwd with
+ * q* replaced by round-to-nearest (ties to the even code).  Vanilla QAT
+ * with the training side's own scales is trace_capture(x) followed by this
+ * call with the scales it wrote. */
+int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                     int32_t num_groups, const int64_t* group_row_offsets,
+                     const uint8_t* scales, const float* gscale, uint16_t* out,
+                     uint32_t* ste_mask, void* stream);
+
+/* Plain bf16 copy (dst = src) with the same load/store path as the kernels
+ * above: the measured-bandwidth yardstick for the roofline.  Not part of the
+ * method.  16-byte aligned, numel % 8 == 0, no overlap. */
+int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel,
+                    void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRACE_FP4_H */

@@ -1,0 +1,99 @@
+"""The C-ABI library loads without a GPU, exports every function that
+include/*.h declares, and rejects bad arguments on the host before touching
+CUDA (no compute call is made here)."""
+from __future__ import annotations
+
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from fp4_quantization_aware_trace_b200 import _build, ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    _build.build()
+    return ops.library()
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(trace_\w+)\s*\(", src, re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_header_declares_the_abi():
+    names = _declared()
+    for n in ("trace_capture", "trace_guided_fq_fwd", "trace_fq_bwd", "trace_rtn_fq_fwd",
+              "trace_capture_workspace_bytes", "trace_strerror", "trace_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", ops.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    missing = _declared() - exported
+    assert not missing, missing
+    for n in _declared():
+        assert hasattr(lib, n)
+
+
+def test_version_and_strings(lib):
+    assert lib.trace_abi_version() == 1
+    for st in range(6):
+        assert lib.trace_strerror(st)
+    assert b"unknown" in lib.trace_strerror(99)
+
+
+def test_workspace_query(lib):
+    assert ops.trace_capture_workspace_bytes(16, 32, 1) == 256
+    assert ops.trace_capture_workspace_bytes(16, 32, 64) == 256
+    assert ops.trace_capture_workspace_bytes(16, 32, 65) == 512
+    assert ops.trace_capture_workspace_bytes(16, 33, 1) == 0
+    assert ops.trace_capture_workspace_bytes(16, 32, 0) == 0
+
+
+def test_host_argument_checks(lib):
+    P = ctypes.c_void_p
+    a = P(1 << 20)          # aligned fake pointers: never dereferenced
+    odd = P((1 << 20) + 2)
+    # shape errors come first
+    assert lib.trace_capture(a, 4, 48, 1, None, a, a, a, a, a, 256, None) == 2
+    assert lib.trace_capture(a, -1, 32, 1, None, a, a, a, a, a, 256, None) == 2
+    assert lib.trace_capture(a, 4, 32, 0, None, a, a, a, a, a, 256, None) == 2
+    assert lib.trace_capture(a, 1 << 33, 32, 1, None, a, a, a, a, a, 256, None) == 2
+    # NULLs
+    assert lib.trace_capture(None, 4, 32, 1, None, a, a, a, a, a, 256, None) == 1
+    assert lib.trace_capture(a, 4, 32, 3, None, a, a, a, a, a, 256, None) == 1
+    assert lib.trace_guided_fq_fwd(a, 4, 32, 1, None, None, a, a, a, a, None) == 1
+    assert lib.trace_rtn_fq_fwd(a, 4, 32, 1, None, a, a, None, a, None) == 1
+    assert lib.trace_fq_bwd(a, None, 32, a, None) == 1
+    # alignment
+    assert lib.trace_capture(odd, 4, 32, 1, None, a, a, a, a, a, 256, None) == 3
+    assert lib.trace_guided_fq_fwd(a, 4, 32, 1, None, a, a, a, odd, a, None) == 3
+    assert lib.trace_fq_bwd(a, a, 32, odd, None) == 3
+    assert lib.trace_copy_bf16(a, odd, 8, None) == 3
+    # workspace
+    assert lib.trace_capture(a, 4, 32, 1, None, a, a, a, a, a, 255, None) == 4
+    assert lib.trace_capture(a, 4, 32, 65, a, a, a, a, a, a, 256, None) == 4
+    # sizes
+    assert lib.trace_fq_bwd(a, a, 40, a, None) == 2
+    assert lib.trace_copy_bf16(a, a, 12, None) == 2
+
+
+def test_binding_rejects_host_tensors(lib):
+    import torch
+    x = torch.zeros(4, 32, dtype=torch.bfloat16)
+    with pytest.raises(ops.TraceError):
+        ops.fq_bwd(x, torch.zeros(4, dtype=torch.int32))

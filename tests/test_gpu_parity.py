@@ -1,0 +1,358 @@
+"""Bit-exact parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every output -- FP4 codes, mantissa bits, E4M3 block scales, global scales,
+dequantised bf16 outputs, STE masks and STE gradients -- must match the
+oracle bit for bit (tolerance 0 ULP): the format fixes every rounding.
+
+Workloads are the seeded synthetic sites of
+``fp4_quantization_aware_trace_b200.inputs``; full tensors go through the
+oracle where it finishes in seconds, and the largest ones are checked on
+sampled rows, with the global scales computed by the oracle over the whole
+tensor.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+from fp4_quantization_aware_trace_b200 import inputs, ops
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _u(t: torch.Tensor) -> np.ndarray:
+    """device tensor -> host numpy array of its raw bits"""
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.int32:
+        return t.numpy().view(np.uint32)
+    if t.dtype == torch.float32:
+        return t.numpy()
+    return t.numpy()
+
+
+def _eq(name, got, ref):
+    got = np.asarray(got).reshape(-1)
+    ref = np.asarray(ref).reshape(-1)
+    assert got.shape == ref.shape, f"{name}: shape {got.shape} vs {ref.shape}"
+    if got.dtype == np.float32:
+        got, ref = got.view(np.uint32), ref.view(np.uint32)
+    bad = np.flatnonzero(got != ref)
+    assert bad.size == 0, (f"{name}: {bad.size} mismatches, first at {bad[:8].tolist()}: "
+                           f"got {got[bad[:8]].tolist()} ref {ref[bad[:8]].tolist()}")
+
+
+def _offs_np(site):
+    return None if site.offsets is None else site.offsets.cpu().numpy()
+
+
+def run_gpu(site: inputs.Site):
+    """capture(x_roll) -> guided(x_train) -> bwd(grad), plus RTN(x_train)."""
+    xr = site.x_roll.to(DEV).contiguous()
+    xt = site.x_train.to(DEV).contiguous()
+    g = site.grad.to(DEV).contiguous()
+    offs = None if site.offsets is None else site.offsets.to(DEV)
+    cap = ops.capture(xr, offs)
+    out, mask = ops.guided_fq_fwd(xt, cap)
+    gin = ops.fq_bwd(g, mask)
+    out_r, mask_r = ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, offs)
+    torch.cuda.synchronize()
+    return dict(codes=_u(cap.codes), mbits=_u(cap.mbits), scales=_u(cap.scales),
+                gscale=_u(cap.gscale), out=_u(out), mask=_u(mask), grad_in=_u(gin),
+                out_rtn=_u(out_r), mask_rtn=_u(mask_r))
+
+
+def run_oracle(oracle_mod, site: inputs.Site):
+    xr, xt, g = inputs.bits(site.x_roll), inputs.bits(site.x_train), inputs.bits(site.grad)
+    G, offs = site.num_groups, _offs_np(site)
+    codes, mbits, scales, gscale = oracle_mod.capture(xr, G, offs)
+    out, mask = oracle_mod.guided_fwd(xt, mbits, scales, gscale, G, offs)
+    out_r, mask_r = oracle_mod.rtn_fwd(xt, scales, gscale, G, offs)
+    gin = oracle_mod.fq_bwd(g, mask)
+    return dict(codes=codes, mbits=mbits, scales=scales, gscale=gscale, out=out, mask=mask,
+                grad_in=gin, out_rtn=out_r, mask_rtn=mask_r)
+
+
+def check_full(oracle_mod, site):
+    got, ref = run_gpu(site), run_oracle(oracle_mod, site)
+    for k in ref:
+        _eq(f"{site.name}.{k}", got[k], ref[k])
+    return got, ref
+
+
+def check_sampled_rows(oracle_mod, site, rows_idx):
+    """Parity on sampled rows of a tensor too large for the whole-tensor
+    oracle: the oracle computes the per-group amax over the full tensor,
+    then captures and fake-quantises the sampled rows on its own."""
+    got = run_gpu(site)
+    xr, xt, g = inputs.bits(site.x_roll), inputs.bits(site.x_train), inputs.bits(site.grad)
+    R, C = xr.shape
+    G, offs = site.num_groups, _offs_np(site)
+    amax = oracle_mod.group_amax(xr, G, offs)
+    gs = np.array([oracle_mod.global_scale(float(a)) for a in amax], np.float32)
+    _eq(f"{site.name}.gscale", got["gscale"], gs)
+    row_g = np.full(R, gs[0], np.float32) if G == 1 else np.repeat(gs, np.diff(offs))
+    rows_idx = np.asarray(sorted(set(int(r) for r in rows_idx)))
+    rg = np.ascontiguousarray(row_g[rows_idx], np.float32)
+    codes, mbits, scales = oracle_mod.capture_rows(xr[rows_idx], rg)
+    out, mask = oracle_mod.fake_quant_rows(xt[rows_idx], rg, scales, mbits)
+    out_r, mask_r = oracle_mod.fake_quant_rows(xt[rows_idx], rg, scales, None)
+    gin = oracle_mod.fq_bwd(np.ascontiguousarray(g[rows_idx]), mask)
+    _eq(f"{site.name}.codes", got["codes"].reshape(R, C // 2)[rows_idx], codes)
+    _eq(f"{site.name}.mbits", got["mbits"].reshape(R, C // 32)[rows_idx], mbits)
+    _eq(f"{site.name}.scales", got["scales"].reshape(R, C // 16)[rows_idx], scales)
+    _eq(f"{site.name}.out", got["out"].reshape(R, C)[rows_idx], out)
+    _eq(f"{site.name}.mask", got["mask"].reshape(R, C // 32)[rows_idx], mask)
+    _eq(f"{site.name}.out_rtn", got["out_rtn"].reshape(R, C)[rows_idx], out_r)
+    _eq(f"{site.name}.mask_rtn", got["mask_rtn"].reshape(R, C // 32)[rows_idx], mask_r)
+    _eq(f"{site.name}.grad_in", got["grad_in"].reshape(R, C)[rows_idx], gin)
+
+
+def _sample_rows(R, k=96, seed=0):
+    rng = np.random.default_rng(seed)
+    return np.concatenate([[0, 1, R // 2, R - 2, R - 1], rng.integers(0, R, k)])
+
+
+# ---------------------------------------------------------------------------
+# Small cases: several tiles, ragged tails, groups, edge cases
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (3, 32), (37, 96), (129, 160), (1000, 64),
+                                       (513, 2048), (4099, 128)])
+def test_parity_small_shapes(oracle_mod, rows, cols):
+    check_full(oracle_mod, inputs.tiny_site(rows * 7 + cols, rows, cols, eps=0.02))
+
+
+def test_parity_cfg1_single_activation(oracle_mod):
+    check_full(oracle_mod, inputs.single_activation(0))
+
+
+def test_parity_ragged_groups(oracle_mod):
+    s = inputs.tiny_site(5, 777, 96, eps=0.01)
+    x = s.x_roll.float()
+    x[100:300] *= 1e4
+    x[500:520] *= 1e-6
+    s.x_roll = x.to(torch.bfloat16)
+    s.x_train = (s.x_roll.float() * 1.003).to(torch.bfloat16)
+    s.offsets = torch.tensor([0, 0, 1, 100, 300, 300, 301, 520, 777, 777], dtype=torch.int64)
+    got, ref = check_full(oracle_mod, s)
+    assert got["gscale"][0] == 1.0 and got["gscale"][4] == 1.0
+
+
+def test_parity_many_small_groups(oracle_mod):
+    s = inputs.tiny_site(6, 2000, 64)
+    x = s.x_roll.float() * torch.exp(torch.linspace(-20, 20, 2000))[:, None]
+    s.x_roll = x.to(torch.bfloat16)
+    s.x_train = inputs._perturb(s.x_roll, 0.005, inputs._gen(1, "cpu"))
+    s.offsets = torch.cat([torch.arange(0, 2000, 3, dtype=torch.int64), torch.tensor([2000])])
+    check_full(oracle_mod, s)
+
+
+def test_parity_empty_and_zero(oracle_mod):
+    # rows == 0: only the global scales are written (amax 0 -> 1.0)
+    x = torch.empty(0, 64, dtype=torch.bfloat16, device=DEV)
+    offs = torch.tensor([0, 0, 0], dtype=torch.int64, device=DEV)
+    cap = ops.capture(x, offs)
+    out, mask = ops.guided_fq_fwd(x, cap)
+    torch.cuda.synchronize()
+    assert cap.gscale.cpu().tolist() == [1.0, 1.0] and out.numel() == 0
+    # all-zero tensor with negative zeros: zero blocks everywhere
+    z = torch.zeros(64, 64)
+    z[::2, 1::3] = -0.0
+    s = inputs.Site("zeros", z.to(torch.bfloat16), z.to(torch.bfloat16),
+                    torch.ones(64, 64).to(torch.bfloat16))
+    got, _ = check_full(oracle_mod, s)
+    assert np.all(got["mask"] == 0xFFFFFFFF)
+
+
+def test_parity_special_values(oracle_mod):
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((64, 256)).astype(np.float32)
+    x[0, :16] = 0.0                              # zero block
+    x[1, :16] = 1e-39 * rng.standard_normal(16)  # subnormal block
+    x[2, :] *= 1e30                              # large rows
+    x[3, 5] = 3.3e38                             # near the bf16 maximum
+    x[4, :32] = 2.0 ** -133                      # smallest subnormal
+    x[5, :] = np.tile([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0], 32)
+    x[6, :] *= 1e-30
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    s = inputs.Site("special", xb, (xb.float() * 1.01).to(torch.bfloat16),
+                    torch.from_numpy(rng.standard_normal((64, 256)).astype(np.float32)).to(torch.bfloat16))
+    check_full(oracle_mod, s)
+    s2 = inputs.Site("special_tiny", (xb.float() * 1e-30).to(torch.bfloat16), s.x_train, s.grad)
+    check_full(oracle_mod, s2)
+
+
+def test_guided_equals_rollout_rtn_when_same_input(oracle_mod):
+    s = inputs.attention_input(seed=4, rows=512)
+    s.x_train = s.x_roll.clone()
+    got, _ = check_full(oracle_mod, s)
+    assert np.array_equal(got["out"], got["out_rtn"])
+
+
+# ---------------------------------------------------------------------------
+# Exhaustive sweeps over bf16 inputs and scale choices
+# ---------------------------------------------------------------------------
+
+def _all_finite_bf16():
+    p = np.arange(1 << 16, dtype=np.uint32)
+    p = p[((p >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    pad = (-p.size) % 256
+    return np.concatenate([p, np.zeros(pad, np.uint16)]).reshape(-1, 256)
+
+
+@pytest.mark.parametrize("bit", [0, 1])
+def test_exhaustive_bf16_fake_quant(oracle_mod, bit):
+    """All finite bf16 patterns x every E4M3 block scale x several global
+    scales (power of two, full-mantissa, subnormal, huge) through the guided
+    and round-to-nearest forwards."""
+    pats = _all_finite_bf16()                     # [255, 256]
+    gs_vals = np.array([1.0, 0.3712345, 2.0 ** -10, 7.1e-3, 2.0 ** -140, 1.9e30],
+                       np.float32)
+    sbytes = np.arange(0x7F, dtype=np.uint8)
+    slab = pats.shape[0]
+    x = np.tile(pats, (len(sbytes) * len(gs_vals), 1))
+    R, C = x.shape
+    scales = np.repeat(np.tile(np.repeat(sbytes, slab), len(gs_vals)), C // 16).reshape(R, C // 16)
+    offs = np.arange(0, R + 1, slab * len(sbytes), dtype=np.int64)
+    G = len(gs_vals)
+    mbits = np.full(R * C // 32, 0xFFFFFFFF if bit else 0, np.uint32)
+
+    xd = inputs.from_bits(x, DEV)
+    sc = torch.from_numpy(scales).to(DEV)
+    gs = torch.from_numpy(gs_vals).to(DEV)
+    od = torch.from_numpy(offs).to(DEV)
+    mb = torch.from_numpy(mbits.view(np.int32)).to(DEV)
+    cache = ops.Capture(codes=None, mbits=mb, scales=sc, gscale=gs, offsets=od)
+    out, mask = ops.guided_fq_fwd(xd, cache)
+    out_r, mask_r = ops.rtn_fq_fwd(xd, sc, gs, od)
+    torch.cuda.synchronize()
+    ref, ref_m = oracle_mod.guided_fwd(x, mbits, scales, gs_vals, G, offs)
+    _eq("guided_out", _u(out), ref)
+    _eq("guided_mask", _u(mask), ref_m)
+    ref_r, ref_rm = oracle_mod.rtn_fwd(x, scales, gs_vals, G, offs)
+    _eq("rtn_out", _u(out_r), ref_r)
+    _eq("rtn_mask", _u(mask_r), ref_rm)
+
+
+def test_exhaustive_bf16_capture(oracle_mod):
+    """All finite bf16 patterns through capture, in groups whose amax puts
+    them in different parts of the scale range, and with every block holding
+    one pattern next to a fixed maximum (every E4M3 rounding case of t)."""
+    pats = _all_finite_bf16()
+    R = pats.shape[0]
+    rows = [pats]
+    # each pattern p as the max of its own block, next to small values
+    p = np.arange(1, 0x7F80, dtype=np.uint16)
+    blocks = np.zeros((p.size, 16), np.uint16)
+    blocks[:, 0] = p
+    blocks[:, 1:] = (p[:, None] >> 1) & 0x7FFF
+    blocks = np.concatenate([blocks, np.zeros(((-blocks.size) % (256 * 16) // 16, 16), np.uint16)])
+    rows.append(blocks.reshape(-1, 256))
+    x = np.concatenate(rows + [pats & 0x3FFF, pats & 0x1FFF])
+    offs = np.array([0, R, R + rows[1].shape[0], R + rows[1].shape[0] + R, x.shape[0]], np.int64)
+    s = inputs.Site("sweep", inputs.from_bits(x), inputs.from_bits(x), inputs.from_bits(x),
+                    torch.from_numpy(offs))
+    check_full(oracle_mod, s)
+
+
+# ---------------------------------------------------------------------------
+# The workloads at their full sizes
+# ---------------------------------------------------------------------------
+
+def test_parity_cfg2_attention_input_full(oracle_mod):
+    check_full(oracle_mod, inputs.attention_input(device=DEV))
+
+
+@pytest.mark.parametrize("which", ["k", "v"])
+def test_parity_cfg4_kv_cache_full(oracle_mod, which):
+    check_full(oracle_mod, inputs.kv_cache(device=DEV, which=which))
+
+
+@pytest.mark.parametrize("cols,name", [(2048, "expert_up_in"), (768, "expert_down_in")])
+def test_parity_cfg3_moe_experts(oracle_mod, cols, name):
+    s = inputs.moe_experts(seed=2 if cols == 2048 else 12, cols=cols, device=DEV, name=name)
+    if cols == 768:
+        check_full(oracle_mod, s)
+    else:
+        check_sampled_rows(oracle_mod, s, _sample_rows(s.x_roll.shape[0], 256, 3))
+
+
+@pytest.mark.parametrize("layer,site", [(20, 0), (31, 2), (39, 3)])
+def test_parity_cfg5_layer_sweep_sampled(oracle_mod, layer, site):
+    s = inputs.layer_sweep_site(layer, site, device=DEV)
+    check_sampled_rows(oracle_mod, s, _sample_rows(s.x_roll.shape[0], 64, layer))
+
+
+# ---------------------------------------------------------------------------
+# Buffer discipline: aliasing, canaries, argument errors
+# ---------------------------------------------------------------------------
+
+def test_inplace_aliasing(oracle_mod):
+    s = inputs.tiny_site(3, 300, 128)
+    xr, xt = s.x_roll.to(DEV), s.x_train.to(DEV)
+    cap = ops.capture(xr)
+    ref, _ = ops.guided_fq_fwd(xt, cap)
+    buf = xt.clone()
+    ops.guided_fq_fwd(buf, cap, out=buf)
+    g = s.grad.to(DEV)
+    _, mask = ops.guided_fq_fwd(xt, cap)
+    gref = ops.fq_bwd(g, mask)
+    gbuf = g.clone()
+    ops.fq_bwd(gbuf, mask, out=gbuf)
+    torch.cuda.synchronize()
+    assert torch.equal(buf.view(torch.int16), ref.view(torch.int16))
+    assert torch.equal(gbuf.view(torch.int16), gref.view(torch.int16))
+
+
+def test_canaries_untouched():
+    """Outputs padded with 4 KiB sentinels on both sides: no call writes
+    outside its buffers (odd row counts, several group counts)."""
+    PAD = 4096
+    for rows, cols, offs in [(37, 96, None), (257, 64, [0, 100, 100, 257]),
+                             (1001, 32, list(range(0, 1001, 7)) + [1001])]:
+        s = inputs.tiny_site(rows, rows, cols)
+        n = rows * cols
+        o = None if offs is None else torch.tensor(offs, dtype=torch.int64, device=DEV)
+        G = 1 if offs is None else len(offs) - 1
+
+        def padded(nbytes):
+            b = torch.full((nbytes + 2 * PAD,), 0xA5, dtype=torch.uint8, device=DEV)
+            return b, b[PAD:PAD + nbytes]
+
+        bufs = {k: padded(v) for k, v in dict(codes=n // 2, mbits=n // 8, scales=n // 16,
+                                                 gscale=4 * G, out=2 * n, mask=n // 8,
+                                                 gin=2 * n).items()}
+        v = {k: b[1] for k, b in bufs.items()}
+        ws = torch.empty(ops.trace_capture_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=DEV)
+        xr, xt, g = s.x_roll.to(DEV), s.x_train.to(DEV), s.grad.to(DEV)
+        ops.trace_capture(xr, rows, cols, G, o, v["codes"], v["mbits"], v["scales"], v["gscale"],
+                          ws, ws.numel())
+        ops.trace_guided_fq_fwd(xt, rows, cols, G, o, v["mbits"], v["scales"], v["gscale"],
+                                v["out"], v["mask"])
+        ops.trace_rtn_fq_fwd(xt, rows, cols, G, o, v["scales"], v["gscale"], v["out"], v["mask"])
+        ops.trace_fq_bwd(g, v["mask"], n, v["gin"])
+        torch.cuda.synchronize()
+        for k, (b, _) in bufs.items():
+            assert torch.all(b[:PAD] == 0xA5) and torch.all(b[-PAD:] == 0xA5), k
+
+
+def test_argument_errors_enqueue_nothing():
+    lib = ops.library()
+    x = torch.zeros(64, 64, dtype=torch.bfloat16, device=DEV)
+    cap, ws = ops.alloc_capture(64, 64)
+    P = lambda t, off=0: __import__("ctypes").c_void_p(t.data_ptr() + off)
+    assert lib.trace_capture(P(x), 64, 48, 1, None, P(cap.codes), P(cap.mbits), P(cap.scales),
+                             P(cap.gscale), P(ws), ws.numel(), None) == 2
+    assert lib.trace_capture(P(x, 2), 64, 64, 1, None, P(cap.codes), P(cap.mbits), P(cap.scales),
+                             P(cap.gscale), P(ws), ws.numel(), None) == 3
+    assert lib.trace_capture(P(x), 64, 64, 1, None, P(cap.codes), P(cap.mbits), P(cap.scales),
+                             P(cap.gscale), P(ws), 0, None) == 4
+    assert lib.trace_capture(P(x), 64, 64, 2, None, P(cap.codes), P(cap.mbits), P(cap.scales),
+                             P(cap.gscale), P(ws), ws.numel(), None) == 1
+    assert lib.trace_fq_bwd(P(x), P(cap.mbits), 48, P(x), None) == 2
+    torch.cuda.synchronize()
