@@ -335,6 +335,25 @@ def run_trace(args):
     traffic = traffic_from_profiles({"guided_fwd": "k_fake_quant_guided", "rtn_fwd": "k_fake_quant_rtn",
                                      "ste_bwd": "k_ste_bwd"}[dom])
 
+    # --- yardstick: the library's plain copy kernel on the same bytes -------
+    ysrc = torch.empty(n, dtype=torch.bfloat16, device=dev).fill_(1.0)
+    ydst = torch.empty_like(ysrc)
+    yev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    for i in range(3):
+        flush.fill_(i)
+        ops.trace_copy_bf16(ysrc, ydst, n, stream)
+    for k in range(args.steps):
+        flush.fill_((k + 3) & 0xFF)
+        yev[k][0].record(stream)
+        ops.trace_copy_bf16(ysrc, ydst, n, stream)
+        yev[k][1].record(stream)
+    torch.cuda.synchronize()
+    y_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in yev) / args.steps], pg, dev)[0]
+    yardstick = {"kernel": "k_copy", "bytes": 4 * n, "us": round(y_ms * 1e3, 2),
+                 "gbs": round(4 * n / (y_ms * 1e-3) / 1e9, 1)}
+    del ysrc, ydst
+
     # --- end-to-end through the C ABI with pinned host buffers -------------
     e2e = None
     if not args.no_e2e:
@@ -391,6 +410,7 @@ def run_trace(args):
                    "l2": "flushed before every step (256 MiB write)",
                    "parallelism": f"{world} independent sites, one per GPU (no collective)"},
         "kernels": kern,
+        "yardstick": yardstick,
         "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
                      "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": round(achieved / hbm, 4), "traffic": traffic,

@@ -9,29 +9,37 @@
 // the layouts are documented in include/trace_fp4.h.
 //
 // Design (everything here is HBM-bound elementwise work; no tensor cores):
-//   * x is streamed as 16-byte vectors of 8 bf16; a CTA of 256 threads works
-//     on tiles of 1024 vectors (16 KiB), 4 vectors per thread with all loads
-//     issued before any use; each CTA owns one contiguous range of tiles and
-//     the grid is a multiple of the SM count.  Two neighbouring lanes hold
-//     the two halves of a 16-element scale block.
+//   * One thread owns one 16-element scale block: a single 32-byte load
+//     (ld.global.v8) brings it in, so a warp reads 1 KiB contiguous per
+//     instruction and the per-block work (scale decode, reciprocal) is done
+//     once.  A CTA of 256 threads works on tiles of 512 blocks, two blocks per
+//     thread with all loads issued before any use; each CTA owns one
+//     contiguous range of tiles and the grid is a multiple of the SM count.
 //   * Capture is a two-pass grid amax: kernel 1 reduces max|x| per group
 //     (shared-memory table per CTA, one global atomicMax per group per CTA
 //     into a zeroed workspace); kernel 2 walks the same tiles in REVERSE
 //     order, so it starts on the data kernel 1 touched last and finds much of
 //     x still in the 126 MB L2.
-//   * Division-free fast path.  z = fl(x / d) (d = fl(s_g * s_b)) is needed
-//     only through comparisons with the codewords, the midpoints and 6, all
-//     of which have their low 21 fp32 bits zero.  za = fl(|x| * fl(1/d)) is
-//     within 6 units in the last place of fl(|x|/d); when za is more than 16
-//     units away from every number whose low 21 bits are zero, za and
-//     fl(|x|/d) fall strictly inside the same interval between critical
-//     points, so every decision taken on za is the one the exact quotient
-//     gives.  The rest (za near a critical point, tiny quotients, zero
-//     blocks, scales outside [2^-120, 2^120]) takes the exact path, which
-//     divides with IEEE round-to-nearest (__fdiv_rn), as the format states.
-//   * Outputs: codes as one 32-bit store per vector, mantissa bits and STE
-//     mask as one byte per vector (lane l writes byte l: a warp fills one
-//     32-byte sector), block scales as one byte per block.
+//   * Exact quotient without a division per element: with r = RN(1/d),
+//     q0 = RN(x*r), e = RN(x - q0*d) (one FMA) and z = RN(q0 + e*r) (one FMA)
+//     is the correctly rounded x/d for every bf16 x and fp32 d whose
+//     quotient is a normal number -- the correction step of Markstein
+//     (IBM J. Res. Dev. 34(1), 1990), established here by exhaustive check of
+//     all 2^31 pairs of bf16 and fp32 significands in both result binades
+//     (tests/test_kernel_math.py).  Two elements go through each
+//     packed fp32x2 instruction (mul/fma .f32x2, sm_100).
+//   * Rounding on the E2M1 grid without a table: with M = 2^22 * max(1, 2^E)
+//     (E the binade of a = min(|z|,6)), a + M rounded down / up lands on
+//     M + floor / M + ceiling of a on the grid (spacing 0.5 below 2, 1 in
+//     [2,4), 2 in [4,8)), and the lowest bit of the sum is the mantissa bit
+//     of that codeword.  The guided choice is "the neighbour whose bit equals
+//     the cached bit"; when a is a codeword both roundings agree, which is
+//     the collapsed bracket.  Round-to-nearest uses the hardware
+//     cvt.rn.satfinite.e2m1x2.f32 (ties to the even code).
+//   * Anything outside the fast path's assumptions -- zero blocks, scales d
+//     outside [2^-100, 2^100], guided elements whose quotient is below
+//     2^-126 (where "exactly zero" decides the bracket) -- goes through an
+//     exact per-element path that divides with IEEE round-to-nearest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -41,28 +49,24 @@
 
 namespace {
 
+typedef unsigned long long u64;
+
 constexpr int kThreads = 256;
-constexpr int kVecPerThread = 4;
-constexpr int kTileVecs = kThreads * kVecPerThread;  // 1024 vectors = 8192 elements
+constexpr int kBlkPerThread = 2;
+constexpr int kTileBlks = kThreads * kBlkPerThread;  // 512 blocks = 8192 elements
 constexpr int kCtasPerSm = 4;
 constexpr int kAmaxTable = 256;  // groups per CTA kept in shared memory
 
-// Critical-point window, in fp32 units in the last place (see header).
-constexpr uint32_t kNearWin = 16u;
-constexpr uint32_t kLow21 = 0x1FFFFFu;
-constexpr uint32_t kSix = 0x40C00000u;        // 6.0f
-constexpr uint32_t kTinyZ = 0x0D800000u;      // 2^-100
-constexpr uint32_t kDMin = 0x03800000u;       // 2^-120
-constexpr uint32_t kDMax = 0x7B800000u;       // 2^120
+constexpr uint32_t kDMin = 0x0D800000u;  // 2^-100: fast path needs d in [2^-100, 2^100]
+constexpr uint32_t kDMax = 0x71800000u;  // 2^100
 
 // ---------------------------------------------------------------------------
 // Fast unsigned 32-bit division by a runtime constant (Granlund & Montgomery,
 // "Division by invariant integers using multiplication", PLDI 1994, the
-// round-up method with the add-back step), used to map a vector index to its
-// row when there are several groups.
+// round-up method with the add-back step): block index -> row.
 // ---------------------------------------------------------------------------
 struct FastDiv {
-  uint32_t d, m, s;  // s = ceil(log2 d); d == 1 handled separately
+  uint32_t d, m, s;  // s = ceil(log2 d); d <= 1 handled separately
 };
 
 FastDiv make_fastdiv(uint32_t d) {
@@ -82,22 +86,97 @@ __device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
 }
 
 // ---------------------------------------------------------------------------
-// Number-format helpers (hardware conversions from the public PTX ISA).
+// Memory access (public PTX ISA: 32-byte vector loads/stores on sm_100)
+// ---------------------------------------------------------------------------
+struct V8 {
+  uint32_t w[8];
+};
+
+// One 16-element bf16 block; read once, not kept in L1.
+__device__ __forceinline__ V8 ld_block_stream(const void* p) {
+  V8 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                 "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_block(void* p, const V8& v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+               "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+               "r"(v.w[7])
+               : "memory");
+}
+
+__device__ __forceinline__ V8 zero_block() {
+  V8 v;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v.w[k] = 0u;
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Packed fp32x2 arithmetic (public PTX ISA, sm_100: mul/fma/add/sub .f32x2)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ u64 pk(float lo, float hi) {
+  u64 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk(u64 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+  u64 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+  u64 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ u64 add_rm2(u64 a, u64 b) {
+  u64 r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ u64 add_rp2(u64 a, u64 b) {
+  u64 r;
+  asm("add.rp.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
+  u64 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Number-format helpers (hardware conversions from the public PTX ISA)
 // ---------------------------------------------------------------------------
 
-// Eight fp32 magnitudes -> eight E2M1 codes (round to nearest even, satfinite)
-// packed as nibbles: element j in bits [4j, 4j+4).
-__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&z)[8]) {
+// Two fp32 -> one byte of two E2M1 codes (round to nearest even, satfinite):
+// lo in bits 0-3, hi in bits 4-7; the sign of each input is kept.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+      "cvt.u16.u8 %0, b;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte of two E2M1 codes -> f16x2 (exact): lo code in the low half.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.u8.u32 b, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
       : "=r"(r)
-      : "f"(z[0]), "f"(z[1]), "f"(z[2]), "f"(z[3]), "f"(z[4]), "f"(z[5]),
-        "f"(z[6]), "f"(z[7]));
+      : "r"(byte));
   return r;
 }
 
@@ -116,41 +195,25 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
-__device__ __forceinline__ uint32_t f32_to_bf16_bits(float f) {
-  return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(f));
+// Two fp32 -> bf16x2 (round to nearest even): lo in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// |x| of the 8 elements of a vector as fp32.
-__device__ __forceinline__ void abs8(const uint4& v, float (&a)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+// max|x| over a block as bf16 bits (integer order = magnitude order).
+__device__ __forceinline__ uint32_t absmax_block(const V8& v) {
+  uint32_t m = __vmaxu2(v.w[0] & 0x7FFF7FFFu, v.w[1] & 0x7FFF7FFFu);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    a[2 * k] = __uint_as_float((w[k] << 16) & 0x7FFF0000u);
-    a[2 * k + 1] = __uint_as_float(w[k] & 0x7FFF0000u);
-  }
-}
-
-// Sign bits of the 8 elements: bit j = sign of element j.
-__device__ __forceinline__ uint32_t signs8(const uint4& v) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-  uint32_t s = 0;
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    s |= (((w[k] >> 15) & 1u) | ((w[k] >> 30) & 2u)) << (2 * k);
-  return s;
-}
-
-// max|x| of the 8 elements as bf16 bits (integer order = magnitude order).
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4& v) {
-  uint32_t m = __vmaxu2(__vmaxu2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                        __vmaxu2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+  for (int k = 2; k < 8; ++k) m = __vmaxu2(m, v.w[k] & 0x7FFF7FFFu);
   return max(m & 0xFFFFu, m >> 16);
 }
 
-// Bit j of the result = bit 4j of n (gathers the lowest bit of each nibble).
+// Bit j of the result = bit 4j of n (the lowest bit of each nibble).
 __device__ __forceinline__ uint32_t nibble_lsbs(uint32_t n) {
   uint32_t c = n & 0x11111111u;
   c = (c | (c >> 3)) & 0x03030303u;
@@ -158,10 +221,41 @@ __device__ __forceinline__ uint32_t nibble_lsbs(uint32_t n) {
   return (c | (c >> 12)) & 0xFFu;
 }
 
-// True when za (bits zb) is within kNearWin ulps of a number whose low 21
-// bits are zero (every codeword, midpoint and 6 is such a number).
-__device__ __forceinline__ bool near_critical(uint32_t zb) {
-  return ((zb + kNearWin) & kLow21) < 2u * kNearWin;
+// Per-block constants of the fast path.
+struct BlkK {
+  u64 rr;    // (r, r), r = RN(1/d)
+  u64 ndd;   // (-d, -d)
+  u64 sbv2;  // (s_b, s_b)
+  u64 sg2;   // (s_g, s_g)
+  uint32_t tiny_b;  // |x| bits below this may give a quotient below 2^-126
+};
+
+__device__ __forceinline__ BlkK make_blk(float d, float sbv, float s_g) {
+  BlkK k;
+  const float r = __frcp_rn(d);
+  k.rr = pk(r, r);
+  k.ndd = pk(-d, -d);
+  k.sbv2 = pk(sbv, sbv);
+  k.sg2 = pk(s_g, s_g);
+  k.tiny_b = max(__float_as_uint(__fmul_rn(d, 0x1p-125f)), 1u);
+  return k;
+}
+
+__device__ __forceinline__ bool fast_scale(float d) {
+  const uint32_t db = __float_as_uint(d);
+  return db >= kDMin && db <= kDMax;
+}
+
+// Correctly rounded quotients of a pair: (lo, hi) / d.
+__device__ __forceinline__ u64 quot2(u64 xx, const BlkK& k) {
+  const u64 q0 = mul2(xx, k.rr);
+  const u64 e = fma2(q0, k.ndd, xx);
+  return fma2(e, k.rr, q0);
+}
+
+// Magic addend of the grid rounding for a = min(|z|, 6).
+__device__ __forceinline__ float grid_magic(float a) {
+  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
 }
 
 // ---- exact path: the format's steps with an IEEE division -----------------
@@ -173,12 +267,12 @@ struct Exact {
   bool in;     // |z| <= 6 (STE mask)
 };
 
-__device__ __noinline__ Exact exact_site(float xf, float d) {
-  float z = (d == 0.0f) ? copysignf(0.0f, xf) : __fdiv_rn(xf, d);
-  float a = fabsf(z);
+__device__ __forceinline__ Exact exact_site(float xf, float d) {
+  const float z = (d == 0.0f) ? copysignf(0.0f, xf) : __fdiv_rn(xf, d);
+  const float a = fabsf(z);
   Exact e;
   e.in = a <= 6.0f;
-  float c = fminf(a, 6.0f);
+  const float c = fminf(a, 6.0f);
   e.rtn = (c <= 0.25f) ? 0 : (c < 0.75f) ? 1 : (c <= 1.25f) ? 2 : (c < 1.75f) ? 3
         : (c <= 2.5f) ? 4 : (c < 3.5f) ? 5 : (c <= 5.0f) ? 6 : 7;
   e.floor = (c < 0.5f) ? 0 : (c < 1.0f) ? 1 : (c < 1.5f) ? 2 : (c < 2.0f) ? 3
@@ -195,20 +289,43 @@ __device__ __forceinline__ float e2m1_value(int c) {
   return c >= 2 ? __uint_as_float((uint32_t)(c + 252) << 22) : (c == 1 ? 0.5f : 0.0f);
 }
 
-// bf16 magnitude of q * s for code c: bf16((VAL[c] * sbv) * s_g).
-__device__ __forceinline__ uint32_t dequant_exact(int c, float sbv, float s_g) {
-  return f32_to_bf16_bits(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g));
+// Capture of one block on the exact path: 16 codes (sign<<3 | rtn).
+__device__ __noinline__ void capture_block_exact(V8 v, float d, uint32_t* code_lo,
+                                                 uint32_t* code_hi) {
+  uint32_t c[2] = {0u, 0u};
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t w = v.w[j >> 1];
+    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+    const Exact e = exact_site(xf, d);
+    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
+    c[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << (4 * (j & 7));
+  }
+  *code_lo = c[0];
+  *code_hi = c[1];
 }
 
-// Per-block dequant table for the fast path: for c >= 1 the magnitude is a
-// power of two times bf16(s_g*sbv) (even codes and code 1) or times
-// bf16((1.5*sbv)*s_g) (odd codes >= 3); both products are one fp32 rounding
-// of the exact value, and scaling by 2^j commutes with both roundings while
-// the result stays normal, which d in [2^-120, 2^120] guarantees.
-__device__ __forceinline__ uint32_t dequant_fast(uint32_t c, uint32_t b1, uint32_t b15) {
-  uint32_t base = ((c & 1u) && c >= 3u) ? b15 : b1;
-  uint32_t r = base + (((c >> 1) - 1u) << 7);
-  return c == 0u ? 0u : (r & 0xFFFFu);
+// Fake-quant of one block on the exact path: bf16 outputs and STE mask.
+__device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, float s_g,
+                                                    uint32_t bits16, bool guided, V8* out,
+                                                    uint32_t* mask16) {
+  uint32_t m = 0u;
+  for (int k = 0; k < 8; ++k) out->w[k] = 0u;
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t w = v.w[j >> 1];
+    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+    const Exact e = exact_site(xf, d);
+    int c = e.rtn;
+    if (guided) {
+      const int bit = (int)((bits16 >> j) & 1u);
+      c = e.exact ? e.floor : e.floor + ((e.floor ^ bit) & 1);
+    }
+    const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
+        __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
+    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
+    out->w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
+    m |= (uint32_t)e.in << j;
+  }
+  *mask16 = m;
 }
 
 // ---------------------------------------------------------------------------
@@ -229,11 +346,17 @@ struct GroupCursor {
   }
   // returns true when the group changed
   __device__ __forceinline__ bool seek(uint32_t row) {
-    if (G == 1) { if (g == 0 && lo == 0u) return false; g = 0; lo = 0u; hi = 0xFFFFFFFFu; return true; }
+    if (G == 1) {
+      if (lo == 0u) return false;
+      g = 0;
+      lo = 0u;
+      hi = 0xFFFFFFFFu;
+      return true;
+    }
     if (row >= lo && row < hi) return false;
     int a = 0, b = G;  // last g with offs[g] <= row
     while (b - a > 1) {
-      int m = (a + b) >> 1;
+      const int m = (a + b) >> 1;
       if ((uint64_t)offs[m] <= row) a = m; else b = m;
     }
     g = a;
@@ -244,14 +367,14 @@ struct GroupCursor {
 };
 
 struct Shape {
-  uint32_t nvec;    // N / 8
-  uint32_t ntiles;  // ceil(nvec / kTileVecs)
-  FastDiv vpr;      // vectors per row
+  uint32_t nblk;    // N / 16
+  uint32_t ntiles;  // ceil(nblk / kTileBlks)
+  FastDiv bpr;      // blocks per row
   int G;
 };
 
 __device__ __forceinline__ void cta_tile_range(const Shape& sh, uint32_t& t0, uint32_t& t1) {
-  uint64_t P = gridDim.x, c = blockIdx.x;
+  const uint64_t P = gridDim.x, c = blockIdx.x;
   t0 = (uint32_t)((uint64_t)sh.ntiles * c / P);
   t1 = (uint32_t)((uint64_t)sh.ntiles * (c + 1) / P);
 }
@@ -267,21 +390,19 @@ __global__ void k_zero_u32(uint32_t* p, int n) {
 // Kernel 1: per-group amax (bits of max|x| as bf16, kept as u32 so that
 // atomicMax orders them as magnitudes).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_amax(const uint4* __restrict__ x, Shape sh,
-                                                   const int64_t* __restrict__ offs,
-                                                   uint32_t* __restrict__ amax) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_amax(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+           uint32_t* __restrict__ amax) {
   __shared__ uint32_t table[kAmaxTable];
   __shared__ int g_first_s;
   uint32_t t0, t1;
   cta_tile_range(sh, t0, t1);
   if (t0 >= t1) return;
-  const uint32_t v_first = t0 * kTileVecs;
-  const uint32_t v_last = min(t1 * kTileVecs, sh.nvec) - 1u;
 
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (threadIdx.x == 0) {
-    gc.seek(fastdiv(v_first, sh.vpr));
+    gc.seek(fastdiv(t0 * kTileBlks, sh.bpr));
     g_first_s = gc.g;
   }
   for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
@@ -293,34 +414,37 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_amax(const uint4* __re
   int run_g = -1;
   auto flush = [&](int g, uint32_t val) {
     if (g < 0 || val == 0u) return;
-    int slot = g - g_first;
+    const int slot = g - g_first;
     if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
     else atomicMax(&amax[g], val);
   };
 
   for (uint32_t t = t0; t < t1; ++t) {
-    uint4 v[kVecPerThread];
-    const uint32_t base = t * kTileVecs + threadIdx.x;
+    V8 v[kBlkPerThread];
+    const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      uint32_t vi = base + u * kThreads;
-      v[u] = vi < sh.nvec ? __ldg(x + vi) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
     }
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      uint32_t vi = base + u * kThreads;
-      if (vi >= sh.nvec) continue;
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b >= sh.nblk) continue;
       if (sh.G > 1) {
-        gc.seek(fastdiv(vi, sh.vpr));
-        if (gc.g != run_g) { flush(run_g, run); run = 0u; run_g = gc.g; }
+        gc.seek(fastdiv(b, sh.bpr));
+        if (gc.g != run_g) {
+          flush(run_g, run);
+          run = 0u;
+          run_g = gc.g;
+        }
       } else {
         run_g = 0;
       }
-      run = max(run, absmax8_bits(v[u]));
+      run = max(run, absmax_block(v[u]));
     }
   }
   if (sh.G == 1) {
-    // whole CTA feeds one accumulator: warp reduce, then shared, then global
     for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
     if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
   } else {
@@ -328,99 +452,105 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_amax(const uint4* __re
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
-    uint32_t val = table[i];
+    const uint32_t val = table[i];
     if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
   }
 }
 
-// Global scale from the amax bits: s_g = amax / 2688, or 1 for amax = 0.
-__device__ __forceinline__ float global_scale_from(uint32_t amax_bits) {
-  float a = __uint_as_float(amax_bits << 16);
-  return amax_bits == 0u ? 1.0f : __fdiv_rn(a, 2688.0f);
+// Per-group constants of capture.
+struct GroupK {
+  float s_g;    // amax / 2688, or 1
+  float den6;   // RN(6 * s_g)
+  float r6;     // RN(1 / den6)
+  bool fast6;   // den6 in the range where bmax/den6 may use the FMA quotient
+};
+
+__device__ __forceinline__ GroupK group_consts(uint32_t amax_bits) {
+  GroupK k;
+  const float a = __uint_as_float(amax_bits << 16);
+  k.s_g = amax_bits == 0u ? 1.0f : __fdiv_rn(a, 2688.0f);
+  k.den6 = __fmul_rn(6.0f, k.s_g);
+  k.fast6 = fast_scale(k.den6);
+  k.r6 = k.fast6 ? __frcp_rn(k.den6) : 0.0f;
+  return k;
 }
 
 // ---------------------------------------------------------------------------
 // Kernel 2: capture.  Per 16-element block: E4M3 scale; per element: the
 // round-to-nearest code and its mantissa bit.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_capture(const uint4* __restrict__ x, Shape sh,
-                                                      const int64_t* __restrict__ offs,
-                                                      const uint32_t* __restrict__ amax,
-                                                      uint32_t* __restrict__ codes,
-                                                      uint8_t* __restrict__ mbits,
-                                                      uint8_t* __restrict__ scales,
-                                                      float* __restrict__ gscale) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+              const uint32_t* __restrict__ amax, u64* __restrict__ codes,
+              uint16_t* __restrict__ mbits, uint8_t* __restrict__ scales,
+              float* __restrict__ gscale) {
   // global scales of all groups (any CTA may write them; all write the same)
   for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
-    gscale[g] = global_scale_from(amax[g]);
+    gscale[g] = group_consts(amax[g]).s_g;
 
   uint32_t t0, t1;
   cta_tile_range(sh, t0, t1);
   GroupCursor gc;
   gc.init(offs, sh.G);
-  float s_g = 1.0f, den6 = 6.0f;
-  const bool odd_lane = threadIdx.x & 1;
+  GroupK gk = group_consts(0u);
 
   for (uint32_t tt = t1; tt > t0; --tt) {  // reverse order: L2 reuse after k_amax
     const uint32_t t = tt - 1u;
-    uint4 v[kVecPerThread];
-    const uint32_t base = t * kTileVecs + threadIdx.x;
+    V8 v[kBlkPerThread];
+    const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      uint32_t vi = base + u * kThreads;
-      v[u] = vi < sh.nvec ? __ldcs(x + vi) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
     }
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      const bool valid = vi < sh.nvec;
-      if (valid && gc.seek(sh.G > 1 ? fastdiv(vi, sh.vpr) : 0u)) {
-        s_g = global_scale_from(__ldg(amax + gc.g));
-        den6 = __fmul_rn(6.0f, s_g);
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b >= sh.nblk) continue;
+      if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) gk = group_consts(__ldg(amax + gc.g));
+      // block scale: t = bmax / RN(6 s_g), E4M3 round-to-nearest-even, satfinite
+      const float bmax = __uint_as_float(absmax_block(v[u]) << 16);
+      float tq;
+      if (gk.fast6) {
+        const float q0 = __fmul_rn(bmax, gk.r6);
+        tq = __fmaf_rn(__fmaf_rn(q0, -gk.den6, bmax), gk.r6, q0);
+      } else {
+        tq = __fdiv_rn(bmax, gk.den6);
       }
-      // block max over the lane pair holding the 16-element block
-      uint32_t m = absmax8_bits(v[u]);
-      m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      if (!valid) continue;
-      const float bmax = __uint_as_float(m << 16);
-      const uint32_t sb = cvt_e4m3(__fdiv_rn(bmax, den6));
-      const float sbv = e4m3_to_f32(sb);
-      const float d = __fmul_rn(s_g, sbv);
-      const uint32_t db = __float_as_uint(d);
-      const bool fast_blk = db >= kDMin && db <= kDMax;
-      const float r = fast_blk ? __frcp_rn(d) : 0.0f;
-
-      float a[8], za[8];
-      abs8(v[u], a);
-      uint32_t slow = fast_blk ? 0u : 0xFFu;
+      const uint32_t sb = cvt_e4m3(tq);
+      const float d = __fmul_rn(gk.s_g, e4m3_to_f32(sb));
+      uint32_t c0, c1;
+      if (d == 0.0f) {
+        // zero block: z = +-0, code = sign only
+        c0 = c1 = 0u;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        za[j] = __fmul_rn(a[j], r);
-        const uint32_t zb = __float_as_uint(za[j]);
-        const bool hard = (a[j] != 0.0f) && (near_critical(zb) || zb < kTinyZ);
-        slow |= (uint32_t)hard << j;
-      }
-      uint32_t code = cvt_e2m1x8(za);
-      if (slow) {
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
-          if (!((slow >> j) & 1u)) continue;
-          const float xf = (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
-          const Exact e = exact_site(xf, d);
-          code = (code & ~(0xFu << (4 * j))) | ((uint32_t)e.rtn << (4 * j));
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t w = v[u].w[k];
+          const uint32_t nib = (((w >> 15) & 1u) << 3) | ((w >> 31) << 7);
+          if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
         }
-      }
-      const uint32_t mb = nibble_lsbs(code);
-      // sign bit of every nibble = sign of x (z = x/d keeps it, zeros too)
-      const uint32_t sg = signs8(v[u]);
-      uint32_t sgn = 0u;
+      } else if (fast_scale(d)) {
+        const BlkK bk = make_blk(d, 0.0f, 0.0f);
+        uint32_t c[2] = {0u, 0u};
 #pragma unroll
-      for (int j = 0; j < 8; ++j) sgn |= ((sg >> j) & 1u) << (4 * j + 3);
-      code |= sgn;
-      codes[vi] = code;
-      mbits[vi] = (uint8_t)mb;
-      if (!odd_lane) scales[vi >> 1] = (uint8_t)sb;
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t w = v[u].w[k];
+          const float xl = bf16_lo(w), xh = bf16_hi(w);
+          float zl, zh;
+          upk(quot2(pk(xl, xh), bk), zl, zh);
+          // the code carries the sign of x (also for zeros and underflows)
+          zl = __uint_as_float((__float_as_uint(zl) & 0x7FFFFFFFu) | (__float_as_uint(xl) & 0x80000000u));
+          zh = __uint_as_float((__float_as_uint(zh) & 0x7FFFFFFFu) | (w & 0x80000000u));
+          c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+        }
+        c0 = c[0];
+        c1 = c[1];
+      } else {
+        capture_block_exact(v[u], d, &c0, &c1);
+      }
+      codes[b] = ((u64)c1 << 32) | c0;
+      mbits[b] = (uint16_t)(nibble_lsbs(c0) | (nibble_lsbs(c1) << 8));
+      scales[b] = (uint8_t)sb;
     }
   }
 }
@@ -431,13 +561,41 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_capture(const uint4* _
 // round to nearest.  Writes bf16 q*·s and the STE mask.
 // ---------------------------------------------------------------------------
 template <bool GUIDED>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_fake_quant(const uint4* __restrict__ x, Shape sh,
-                                                         const int64_t* __restrict__ offs,
-                                                         const uint8_t* __restrict__ mbits,
-                                                         const uint8_t* __restrict__ scales,
-                                                         const float* __restrict__ gscale,
-                                                         uint4* __restrict__ out,
-                                                         uint8_t* __restrict__ mask) {
+__device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const BlkK& k,
+                                            uint32_t& m2, bool& slow) {
+  const uint32_t axl_b = (w << 16) & 0x7FFF0000u, axh_b = w & 0x7FFF0000u;
+  const u64 xx = pk(__uint_as_float(axl_b), __uint_as_float(axh_b));
+  float zl, zh;
+  upk(quot2(xx, k), zl, zh);  // >= 0; +inf/NaN only where |x|/d overflows
+  m2 = (uint32_t)(zl <= 6.0f) | ((uint32_t)(zh <= 6.0f) << 1);
+  const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);  // NaN -> 6
+  float ql, qh;
+  if (GUIDED) {
+    slow |= (axl_b - 1u < k.tiny_b - 1u) | (axh_b - 1u < k.tiny_b - 1u);
+    const u64 MM = pk(grid_magic(al), grid_magic(ah));
+    const u64 aa = pk(al, ah);
+    float lol, loh, hil, hih;
+    upk(add_rm2(aa, MM), lol, loh);
+    upk(add_rp2(aa, MM), hil, hih);
+    const float tl = ((__float_as_uint(lol) ^ bits2) & 1u) ? hil : lol;
+    const float th = ((__float_as_uint(loh) ^ (bits2 >> 1)) & 1u) ? hih : loh;
+    upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
+  } else {
+    // round to nearest on the grid (ties to the even code), then dequantise
+    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
+    const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    const float vh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    upk(mul2(mul2(pk(vl, vh), k.sbv2), k.sg2), ql, qh);
+  }
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+template <bool GUIDED>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+                 const uint16_t* __restrict__ mbits, const uint8_t* __restrict__ scales,
+                 const float* __restrict__ gscale, V8* __restrict__ out,
+                 uint16_t* __restrict__ mask) {
   uint32_t t0, t1;
   cta_tile_range(sh, t0, t1);
   GroupCursor gc;
@@ -445,84 +603,45 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_fake_quant(const uint4
   float s_g = 1.0f;
 
   for (uint32_t t = t0; t < t1; ++t) {
-    uint4 v[kVecPerThread];
-    uint32_t bits[kVecPerThread], sbs[kVecPerThread];
-    const uint32_t base = t * kTileVecs + threadIdx.x;
+    V8 v[kBlkPerThread];
+    uint32_t bits[kBlkPerThread], sbs[kBlkPerThread];
+    const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      const bool valid = vi < sh.nvec;
-      v[u] = valid ? __ldcs(x + vi) : make_uint4(0u, 0u, 0u, 0u);
-      bits[u] = (GUIDED && valid) ? (uint32_t)__ldcs(mbits + vi) : 0u;
-      sbs[u] = valid ? (uint32_t)__ldcs(scales + (vi >> 1)) : 0u;
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      const bool valid = b < sh.nblk;
+      v[u] = valid ? ld_block_stream(x + b) : zero_block();
+      bits[u] = (GUIDED && valid) ? (uint32_t)__ldcs(mbits + b) : 0u;
+      sbs[u] = valid ? (uint32_t)__ldcs(scales + b) : 0u;
     }
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      if (vi >= sh.nvec) continue;
-      if (gc.seek(sh.G > 1 ? fastdiv(vi, sh.vpr) : 0u)) s_g = __ldg(gscale + gc.g);
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b >= sh.nblk) continue;
+      if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
       const float sbv = e4m3_to_f32(sbs[u]);
       const float d = __fmul_rn(s_g, sbv);
-      const uint32_t db = __float_as_uint(d);
-      const bool fast_blk = db >= kDMin && db <= kDMax;
-      const float r = fast_blk ? __frcp_rn(d) : 0.0f;
-      const uint32_t b1 = f32_to_bf16_bits(d);
-      const uint32_t b15 = f32_to_bf16_bits(__fmul_rn(__fmul_rn(1.5f, sbv), s_g));
-
-      float a[8], za[8];
-      abs8(v[u], a);
-      uint32_t slow = fast_blk ? 0u : 0xFFu;
-      uint32_t inmask = 0u;
-      uint32_t c[8];
+      V8 o;
+      uint32_t m = 0u;
+      bool slow = !fast_scale(d);
+      if (d == 0.0f) {
+        // zero block: z = +-0, output +-0, mask set
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        za[j] = __fmul_rn(a[j], r);
-        const uint32_t zb = __float_as_uint(za[j]);
-        const bool hard = (a[j] != 0.0f) && (near_critical(zb) || zb < kTinyZ);
-        slow |= (uint32_t)hard << j;
-        inmask |= (uint32_t)(zb <= kSix) << j;
-        if (GUIDED) {
-          const int tq = (int)(zb >> 22) - 252;
-          const uint32_t k = (uint32_t)(min(max(tq, 0), 7) + (tq == 0));
-          const bool exact = (zb == 0u) || (zb > kSix);
-          const uint32_t bit = (bits[u] >> j) & 1u;
-          c[j] = exact ? k : k + ((k ^ bit) & 1u);
+        for (int k = 0; k < 8; ++k) o.w[k] = v[u].w[k] & 0x80008000u;
+        m = 0xFFFFu;
+        slow = false;
+      } else if (!slow) {
+        const BlkK bk = make_blk(d, sbv, s_g);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          uint32_t m2;
+          o.w[k] = fq_pair<GUIDED>(v[u].w[k], bits[u] >> (2 * k), bk, m2, slow);
+          m |= m2 << (2 * k);
         }
       }
-      if (!GUIDED) {
-        const uint32_t code = cvt_e2m1x8(za);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) c[j] = (code >> (4 * j)) & 0xFu;
-      }
-      uint32_t o[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = dequant_fast(c[j], b1, b15);
-      if (slow) {
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll 1
-        for (int j = 0; j < 8; ++j) {
-          if (!((slow >> j) & 1u)) continue;
-          const float xf = (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
-          const Exact e = exact_site(xf, d);
-          int cs;
-          if (GUIDED) {
-            const int bit = (bits[u] >> j) & 1;
-            cs = e.exact ? e.floor : e.floor + ((e.floor ^ bit) & 1);
-          } else {
-            cs = e.rtn;
-          }
-          inmask = (inmask & ~(1u << j)) | ((uint32_t)e.in << j);
-          o[j] = dequant_exact(cs, sbv, s_g);
-        }
-      }
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      uint4 res;
-      res.x = (o[0] | (o[1] << 16)) | (w[0] & 0x80008000u);
-      res.y = (o[2] | (o[3] << 16)) | (w[1] & 0x80008000u);
-      res.z = (o[4] | (o[5] << 16)) | (w[2] & 0x80008000u);
-      res.w = (o[6] | (o[7] << 16)) | (w[3] & 0x80008000u);
-      out[vi] = res;
-      mask[vi] = (uint8_t)inmask;
+      if (slow) fake_quant_block_exact(v[u], d, sbv, s_g, bits[u], GUIDED, &o, &m);
+      st_block(out + b, o);
+      mask[b] = (uint16_t)m;
     }
   }
 }
@@ -530,37 +649,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_fake_quant(const uint4
 // ---------------------------------------------------------------------------
 // Kernel 4: masked straight-through backward.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_ste_bwd(const uint4* __restrict__ g, Shape sh,
-                                                      const uint8_t* __restrict__ mask,
-                                                      uint4* __restrict__ gin) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint16_t* __restrict__ mask,
+              V8* __restrict__ gin) {
   uint32_t t0, t1;
   cta_tile_range(sh, t0, t1);
   for (uint32_t t = t0; t < t1; ++t) {
-    uint4 v[kVecPerThread];
-    uint32_t m[kVecPerThread];
-    const uint32_t base = t * kTileVecs + threadIdx.x;
+    V8 v[kBlkPerThread];
+    uint32_t m[kBlkPerThread];
+    const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      const bool valid = vi < sh.nvec;
-      v[u] = valid ? __ldcs(g + vi) : make_uint4(0u, 0u, 0u, 0u);
-      m[u] = valid ? (uint32_t)__ldcs(mask + vi) : 0u;
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      const bool valid = b < sh.nblk;
+      v[u] = valid ? ld_block_stream(g + b) : zero_block();
+      m[u] = valid ? (uint32_t)__ldcs(mask + b) : 0u;
     }
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      if (vi >= sh.nvec) continue;
-      const uint32_t b = m[u];
-      // bit pair (2k, 2k+1) -> half-word keep masks of word k
-      auto keep = [&](int k) {
-        return (((b >> (2 * k)) & 1u) ? 0x0000FFFFu : 0u) | (((b >> (2 * k + 1)) & 1u) ? 0xFFFF0000u : 0u);
-      };
-      uint4 r;
-      r.x = v[u].x & keep(0);
-      r.y = v[u].y & keep(1);
-      r.z = v[u].z & keep(2);
-      r.w = v[u].w & keep(3);
-      gin[vi] = r;
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b >= sh.nblk) continue;
+      V8 r;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        // bits (2k, 2k+1) -> keep masks of the two halves of word k
+        const uint32_t keep = (((m[u] >> (2 * k)) & 1u) * 0x0000FFFFu) |
+                              (((m[u] >> (2 * k + 1)) & 1u) * 0xFFFF0000u);
+        r.w[k] = v[u].w[k] & keep;
+      }
+      st_block(gin + b, r);
     }
   }
 }
@@ -568,22 +685,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) k_ste_bwd(const uint4* _
 // ---------------------------------------------------------------------------
 // Kernel 6: plain copy with the same access pattern (bandwidth yardstick).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) k_copy(const uint4* __restrict__ s, Shape sh,
-                                                   uint4* __restrict__ d) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_copy(const V8* __restrict__ s, Shape sh, V8* __restrict__ d) {
   uint32_t t0, t1;
   cta_tile_range(sh, t0, t1);
   for (uint32_t t = t0; t < t1; ++t) {
-    uint4 v[kVecPerThread];
-    const uint32_t base = t * kTileVecs + threadIdx.x;
+    V8 v[kBlkPerThread];
+    const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      v[u] = vi < sh.nvec ? __ldcs(s + vi) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(s + b) : zero_block();
     }
 #pragma unroll
-    for (int u = 0; u < kVecPerThread; ++u) {
-      const uint32_t vi = base + u * kThreads;
-      if (vi < sh.nvec) d[vi] = v[u];
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b < sh.nblk) st_block(d + b, v[u]);
     }
   }
 }
@@ -610,16 +727,16 @@ int check_shape(int64_t rows, int64_t cols, int32_t G, const int64_t* offs) {
   if (rows < 0 || cols <= 0 || cols % 32 != 0 || G < 1) return TRACE_ERR_SHAPE;
   if (G > 1 && offs == nullptr) return TRACE_ERR_NULL;
   const long double n = (long double)rows * (long double)cols;
-  if (n / 8 >= 4294967296.0L - (long double)kTileVecs) return TRACE_ERR_SHAPE;
+  if (n / 16 >= 4294967296.0L - (long double)kTileBlks) return TRACE_ERR_SHAPE;
   return TRACE_OK;
 }
 
 Shape make_shape(int64_t rows, int64_t cols, int32_t G) {
   Shape sh;
   const uint64_t n = (uint64_t)rows * (uint64_t)cols;
-  sh.nvec = (uint32_t)(n / 8);
-  sh.ntiles = (uint32_t)((sh.nvec + kTileVecs - 1) / kTileVecs);
-  sh.vpr = make_fastdiv((uint32_t)(cols / 8));
+  sh.nblk = (uint32_t)(n / 16);
+  sh.ntiles = (uint32_t)(((uint64_t)sh.nblk + kTileBlks - 1) / kTileBlks);
+  sh.bpr = make_fastdiv((uint32_t)(cols / 16));
   sh.G = G;
   return sh;
 }
@@ -643,7 +760,7 @@ const char* trace_strerror(int status) {
   switch (status) {
     case TRACE_OK: return "ok";
     case TRACE_ERR_NULL: return "a required pointer is NULL";
-    case TRACE_ERR_SHAPE: return "invalid shape (rows < 0, cols <= 0, cols % 32 != 0, groups < 1, or N/8 >= 2^32)";
+    case TRACE_ERR_SHAPE: return "invalid shape (rows < 0, cols <= 0, cols % 32 != 0, groups < 1, or N/16 >= 2^32)";
     case TRACE_ERR_ALIGN: return "a pointer is not aligned as the call requires";
     case TRACE_ERR_WORKSPACE: return "workspace smaller than trace_capture_workspace_bytes()";
     case TRACE_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
@@ -668,7 +785,7 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_gro
   // empty tensors may be NULL
   const bool empty = rows == 0;
   if ((!empty && (!x || !codes || !mbits || !scales)) || !gscale || !workspace) return TRACE_ERR_NULL;
-  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(mbits, 16) || !aligned(scales, 16) ||
+  if (!aligned(x, 32) || !aligned(codes, 16) || !aligned(mbits, 16) || !aligned(scales, 16) ||
       !aligned(gscale, 4) || !aligned(workspace, 256))
     return TRACE_ERR_ALIGN;
   if (workspace_bytes < trace_capture_workspace_bytes(rows, cols, num_groups)) return TRACE_ERR_WORKSPACE;
@@ -680,9 +797,9 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_gro
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
   const int zg = (num_groups + kThreads - 1) / kThreads;
   k_zero_u32<<<zg < 1024 ? zg : 1024, kThreads, 0, s>>>(amax, num_groups);
-  if (sh.nvec > 0) k_amax<<<grid, kThreads, 0, s>>>((const uint4*)x, sh, offs, amax);
-  k_capture<<<grid, kThreads, 0, s>>>((const uint4*)x, sh, offs, amax, (uint32_t*)codes,
-                                      (uint8_t*)mbits, scales, gscale);
+  if (sh.nblk > 0) k_amax<<<grid, kThreads, 0, s>>>((const V8*)x, sh, offs, amax);
+  k_capture<<<grid, kThreads, 0, s>>>((const V8*)x, sh, offs, amax, (u64*)codes,
+                                      (uint16_t*)mbits, scales, gscale);
   return launched();
 }
 
@@ -693,21 +810,21 @@ static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64
   if (st) return st;
   if (rows == 0) return TRACE_OK;  // nothing to do; empty tensors may have NULL data
   if (!x || (guided && !mbits) || !scales || !gscale || !out || !mask) return TRACE_ERR_NULL;
-  if (!aligned(x, 16) || (guided && !aligned(mbits, 16)) || !aligned(scales, 16) ||
-      !aligned(gscale, 4) || !aligned(out, 16) || !aligned(mask, 16))
+  if (!aligned(x, 32) || (guided && !aligned(mbits, 16)) || !aligned(scales, 16) ||
+      !aligned(gscale, 4) || !aligned(out, 32) || !aligned(mask, 16))
     return TRACE_ERR_ALIGN;
   const Shape sh = make_shape(rows, cols, G);
-  if (sh.nvec == 0) return TRACE_OK;
+  if (sh.nblk == 0) return TRACE_OK;
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* o = G > 1 ? offs : nullptr;
   if (guided)
-    k_fake_quant<true><<<grid, kThreads, 0, s>>>((const uint4*)x, sh, o, (const uint8_t*)mbits,
-                                                 scales, gscale, (uint4*)out, (uint8_t*)mask);
+    k_fake_quant<true><<<grid, kThreads, 0, s>>>((const V8*)x, sh, o, (const uint16_t*)mbits,
+                                                 scales, gscale, (V8*)out, (uint16_t*)mask);
   else
-    k_fake_quant<false><<<grid, kThreads, 0, s>>>((const uint4*)x, sh, o, nullptr, scales, gscale,
-                                                  (uint4*)out, (uint8_t*)mask);
+    k_fake_quant<false><<<grid, kThreads, 0, s>>>((const V8*)x, sh, o, nullptr, scales, gscale,
+                                                  (V8*)out, (uint16_t*)mask);
   return launched();
 }
 
@@ -729,34 +846,32 @@ int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,
                  uint16_t* grad_in, void* stream) {
   if (numel < 0 || numel % 32 != 0) return TRACE_ERR_SHAPE;
-  if ((long double)numel / 8 >= 4294967296.0L - (long double)kTileVecs) return TRACE_ERR_SHAPE;
+  if ((long double)numel / 16 >= 4294967296.0L - (long double)kTileBlks) return TRACE_ERR_SHAPE;
   if (numel == 0) return TRACE_OK;
   if (!grad_out || !ste_mask || !grad_in) return TRACE_ERR_NULL;
-  if (!aligned(grad_out, 16) || !aligned(ste_mask, 16) || !aligned(grad_in, 16)) return TRACE_ERR_ALIGN;
+  if (!aligned(grad_out, 32) || !aligned(ste_mask, 16) || !aligned(grad_in, 32)) return TRACE_ERR_ALIGN;
   const Shape sh = make_shape(numel / 32, 32, 1);
-  if (sh.nvec == 0) return TRACE_OK;
   int grid, st;
   if ((st = grid_for(sh, &grid))) return st;
-  k_ste_bwd<<<grid, kThreads, 0, (cudaStream_t)stream>>>((const uint4*)grad_out, sh,
-                                                         (const uint8_t*)ste_mask, (uint4*)grad_in);
+  k_ste_bwd<<<grid, kThreads, 0, (cudaStream_t)stream>>>((const V8*)grad_out, sh,
+                                                         (const uint16_t*)ste_mask, (V8*)grad_in);
   return launched();
 }
 
 int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* stream) {
-  if (numel < 0 || numel % 8 != 0) return TRACE_ERR_SHAPE;
-  if ((long double)numel / 8 >= 4294967296.0L - (long double)kTileVecs) return TRACE_ERR_SHAPE;
+  if (numel < 0 || numel % 16 != 0) return TRACE_ERR_SHAPE;
+  if ((long double)numel / 16 >= 4294967296.0L - (long double)kTileBlks) return TRACE_ERR_SHAPE;
   if (numel == 0) return TRACE_OK;
   if (!src || !dst) return TRACE_ERR_NULL;
-  if (!aligned(src, 16) || !aligned(dst, 16)) return TRACE_ERR_ALIGN;
+  if (!aligned(src, 32) || !aligned(dst, 32)) return TRACE_ERR_ALIGN;
   Shape sh;
-  sh.nvec = (uint32_t)(numel / 8);
-  sh.ntiles = (sh.nvec + kTileVecs - 1) / kTileVecs;
-  sh.vpr = make_fastdiv(1);
+  sh.nblk = (uint32_t)(numel / 16);
+  sh.ntiles = (uint32_t)(((uint64_t)sh.nblk + kTileBlks - 1) / kTileBlks);
+  sh.bpr = make_fastdiv(1);
   sh.G = 1;
-  if (sh.nvec == 0) return TRACE_OK;
   int grid, st;
   if ((st = grid_for(sh, &grid))) return st;
-  k_copy<<<grid, kThreads, 0, (cudaStream_t)stream>>>((const uint4*)src, sh, (uint4*)dst);
+  k_copy<<<grid, kThreads, 0, (cudaStream_t)stream>>>((const V8*)src, sh, (V8*)dst);
   return launched();
 }
 

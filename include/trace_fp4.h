@@ -52,7 +52,8 @@
  *   - scale bytes passed to the forward kernels are non-negative finite E4M3
  *     (0x00..0x7E) and global scales finite and positive, as capture writes;
  *   - the group offsets satisfy the rules above.
- * Limits: N/8 < 2^32 (N < 2^35 elements per call).
+ * Limits: N/16 < 2^32 - 512 (N < 2^36 elements per call).  With rows == 0
+ * (numel == 0) the data pointers may be NULL.
  */
 #ifndef TRACE_FP4_H
 #define TRACE_FP4_H
@@ -89,7 +90,7 @@ size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols,
 /* Rollout capture: fp4_quantize(x_rollout) plus low_bits(q_roll, 1) and the
  * scales (the capture half of the post's pseudocode listing; the compact
  * cache is mbits + scales + gscale, 1.5 bits per element).
- *   x       : bf16 [rows, cols], 16-byte aligned.
+ *   x       : bf16 [rows, cols], 32-byte aligned.
  *   codes   : out, uint8[N/2], 16-byte aligned (the full NVFP4 codes, for the
  *             rollout's own FP4 GEMM).
  *   mbits   : out, uint32[N/32], 16-byte aligned.
@@ -110,9 +111,9 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
  * mantissa bit equals the cached bit; out = bf16((q* * s_b) * s_g) with the
  * sign of z (fp32 product, round to nearest even into bf16); ste_mask bit =
  * |z| <= 6.
- *   x_train : bf16 [rows, cols], 16-byte aligned.
+ *   x_train : bf16 [rows, cols], 32-byte aligned.
  *   mbits, scales, gscale: the rollout's compact cache (capture's outputs).
- *   out     : out, bf16 [rows, cols], 16-byte aligned; may alias x_train.
+ *   out     : out, bf16 [rows, cols], 32-byte aligned; may alias x_train.
  *   ste_mask: out, uint32[N/32], 16-byte aligned. */
 int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
                         int32_t num_groups, const int64_t* group_row_offsets,
@@ -122,7 +123,7 @@ int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
 
 /* Masked straight-through-estimator backward:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
- *   grad_out, grad_in: bf16 [numel], 16-byte aligned; may alias.
+ *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.
  *   ste_mask: uint32[numel/32], 16-byte aligned.  numel % 32 == 0. */
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask,
                  int64_t numel, uint16_t* grad_in, void* stream);
@@ -139,7 +140,7 @@ int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
 
 /* Plain bf16 copy (dst = src) with the same load/store path as the kernels
  * above: the measured-bandwidth yardstick for the roofline.  Not part of the
- * method.  16-byte aligned, numel % 8 == 0, no overlap. */
+ * method.  32-byte aligned, numel % 16 == 0, no overlap. */
 int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel,
                     void* stream);
 

@@ -83,7 +83,7 @@ def test_host_argument_checks(lib):
     assert lib.trace_capture(odd, 4, 32, 1, None, a, a, a, a, a, 256, None) == 3
     assert lib.trace_guided_fq_fwd(a, 4, 32, 1, None, a, a, a, odd, a, None) == 3
     assert lib.trace_fq_bwd(a, a, 32, odd, None) == 3
-    assert lib.trace_copy_bf16(a, odd, 8, None) == 3
+    assert lib.trace_copy_bf16(a, odd, 16, None) == 3
     # workspace
     assert lib.trace_capture(a, 4, 32, 1, None, a, a, a, a, a, 255, None) == 4
     assert lib.trace_capture(a, 4, 32, 65, a, a, a, a, a, a, 256, None) == 4
