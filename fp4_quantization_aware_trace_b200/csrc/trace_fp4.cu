@@ -13,33 +13,45 @@
 //     (ld.global.v8) brings it in, so a warp reads 1 KiB contiguous per
 //     instruction and the per-block work (scale decode, reciprocal) is done
 //     once.  A CTA of 256 threads works on tiles of 512 blocks, two blocks per
-//     thread with all loads issued before any use; each CTA owns one
-//     contiguous range of tiles and the grid is a multiple of the SM count.
+//     thread with all loads issued before any use.  The grid is 32 CTAs per
+//     SM (about one tile per CTA at the 64 MiB sizes), striding over tiles
+//     beyond that: oversubscribing lets the block scheduler balance the tail,
+//     which measured faster on B200 than persistent per-CTA ranges.
 //   * Capture is a two-pass grid amax: kernel 1 reduces max|x| per group
 //     (shared-memory table per CTA, one global atomicMax per group per CTA
-//     into a zeroed workspace); kernel 2 walks the same tiles in REVERSE
-//     order, so it starts on the data kernel 1 touched last and finds much of
-//     x still in the 126 MB L2.
+//     into a zeroed workspace); kernel 2 walks the tiles in REVERSE order, so
+//     it starts on the data kernel 1 touched last and finds much of x still
+//     in the 126 MB L2.
 //   * Exact quotient without a division per element: with r = RN(1/d),
 //     q0 = RN(x*r), e = RN(x - q0*d) (one FMA) and z = RN(q0 + e*r) (one FMA)
 //     is the correctly rounded x/d for every bf16 x and fp32 d whose
-//     quotient is a normal number -- the correction step of Markstein
-//     (IBM J. Res. Dev. 34(1), 1990), established here by exhaustive check of
-//     all 2^31 pairs of bf16 and fp32 significands in both result binades
-//     (tests/test_kernel_math.py).  Two elements go through each
-//     packed fp32x2 instruction (mul/fma .f32x2, sm_100).
+//     quotient is a normal number and whose remainder is representable --
+//     the correction step of Markstein (IBM J. Res. Dev. 34(1), 1990),
+//     established here by exhaustive check of all 2^31 pairs of bf16 and fp32
+//     significands in both result binades (tests/test_kernel_math.py).
+//     Capture and round-to-nearest only need the exact quotient from 0.25 up
+//     (x >= 2^-92 when d >= 2^-90, where the remainder is exact; below
+//     0.25 every decision is "code 0", and the sign comes from x).  The
+//     guided path also needs "exactly zero" to be exact, so it divides
+//     |x| * 2^64: for d in [2^-90, 2^16] every nonzero bf16 then has a
+//     normal quotient and a normal remainder, and fl(x/d) itself is nonzero
+//     (x/d >= 2^-133 / 2^16 = 2^-149), so the scaled quotient is zero exactly
+//     when fl(x/d) is; the codeword found is scaled back by folding 2^-64
+//     into s_b.  Two elements go through each
+//     packed fp32x2 instruction (mul/fma/add .f32x2, sm_100).
 //   * Rounding on the E2M1 grid without a table: with M = 2^22 * max(1, 2^E)
-//     (E the binade of a = min(|z|,6)), a + M rounded down / up lands on
+//     (E the binade of a = min(|z|,6); everything times 2^64 on the guided
+//     path), a + M rounded down / up lands on
 //     M + floor / M + ceiling of a on the grid (spacing 0.5 below 2, 1 in
 //     [2,4), 2 in [4,8)), and the lowest bit of the sum is the mantissa bit
 //     of that codeword.  The guided choice is "the neighbour whose bit equals
 //     the cached bit"; when a is a codeword both roundings agree, which is
 //     the collapsed bracket.  Round-to-nearest uses the hardware
 //     cvt.rn.satfinite.e2m1x2.f32 (ties to the even code).
-//   * Anything outside the fast path's assumptions -- zero blocks, scales d
-//     outside [2^-100, 2^100], guided elements whose quotient is below
-//     2^-126 (where "exactly zero" decides the bracket) -- goes through an
-//     exact per-element path that divides with IEEE round-to-nearest.
+//   * Zero blocks (d = 0) take a short path (every z is +-0); blocks with d
+//     outside [2^-90, 2^100] ([2^-90, 2^16] for the guided forward) go
+//     through an exact per-element path that divides with IEEE
+//     round-to-nearest.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -54,11 +66,17 @@ typedef unsigned long long u64;
 constexpr int kThreads = 256;
 constexpr int kBlkPerThread = 2;
 constexpr int kTileBlks = kThreads * kBlkPerThread;  // 512 blocks = 8192 elements
-constexpr int kCtasPerSm = 4;
+constexpr int kCtasPerSm = 4;    // resident CTAs per SM the register budget allows
+constexpr int kGridPerSm = 32;   // CTAs launched per SM: about one tile each
 constexpr int kAmaxTable = 256;  // groups per CTA kept in shared memory
 
-constexpr uint32_t kDMin = 0x0D800000u;  // 2^-100: fast path needs d in [2^-100, 2^100]
-constexpr uint32_t kDMax = 0x71800000u;  // 2^100
+constexpr uint32_t kDMin = 0x12800000u;     // 2^-90: fast paths need d >= 2^-90
+constexpr uint32_t kDMax = 0x71800000u;     // 2^100: capture / round-to-nearest
+constexpr uint32_t kDMaxExactZ = 0x47800000u;  // 2^16: guided (see below)
+// The guided path divides |x| * 2^64: every nonzero bf16 then has a normal
+// quotient and an exactly representable remainder for d in the fast range.
+constexpr float kXs = 0x1p64f;
+constexpr float kSixS = 0x1p64f * 6.0f;
 
 // ---------------------------------------------------------------------------
 // Fast unsigned 32-bit division by a runtime constant (Granlund & Montgomery,
@@ -225,9 +243,8 @@ __device__ __forceinline__ uint32_t nibble_lsbs(uint32_t n) {
 struct BlkK {
   u64 rr;    // (r, r), r = RN(1/d)
   u64 ndd;   // (-d, -d)
-  u64 sbv2;  // (s_b, s_b)
+  u64 sbv2;  // (s_b, s_b), times 2^-64 on the guided path
   u64 sg2;   // (s_g, s_g)
-  uint32_t tiny_b;  // |x| bits below this may give a quotient below 2^-126
 };
 
 __device__ __forceinline__ BlkK make_blk(float d, float sbv, float s_g) {
@@ -237,13 +254,19 @@ __device__ __forceinline__ BlkK make_blk(float d, float sbv, float s_g) {
   k.ndd = pk(-d, -d);
   k.sbv2 = pk(sbv, sbv);
   k.sg2 = pk(s_g, s_g);
-  k.tiny_b = max(__float_as_uint(__fmul_rn(d, 0x1p-125f)), 1u);
   return k;
 }
 
-__device__ __forceinline__ bool fast_scale(float d) {
+// 0xFFFFFFFF when a <= b (false for NaN), else 0.
+__device__ __forceinline__ uint32_t le_mask(float a, float b) {
+  uint32_t r;
+  asm("set.le.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ bool fast_scale(float d, uint32_t dmax_bits = kDMax) {
   const uint32_t db = __float_as_uint(d);
-  return db >= kDMin && db <= kDMax;
+  return db >= kDMin && db <= dmax_bits;
 }
 
 // Correctly rounded quotients of a pair: (lo, hi) / d.
@@ -253,9 +276,10 @@ __device__ __forceinline__ u64 quot2(u64 xx, const BlkK& k) {
   return fma2(e, k.rr, q0);
 }
 
-// Magic addend of the grid rounding for a = min(|z|, 6).
-__device__ __forceinline__ float grid_magic(float a) {
-  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
+// Magic addend of the grid rounding for a = min(|z|, 6) * 2^64:
+// M = 2^86 * max(1, 2^E), E the binade of a / 2^64.
+__device__ __forceinline__ float grid_magic_s(float a_s) {
+  return __uint_as_float(max((__float_as_uint(a_s) & 0x7F800000u) + 0x0B000000u, 0x6A800000u));
 }
 
 // ---- exact path: the format's steps with an IEEE division -----------------
@@ -373,12 +397,6 @@ struct Shape {
   int G;
 };
 
-__device__ __forceinline__ void cta_tile_range(const Shape& sh, uint32_t& t0, uint32_t& t1) {
-  const uint64_t P = gridDim.x, c = blockIdx.x;
-  t0 = (uint32_t)((uint64_t)sh.ntiles * c / P);
-  t1 = (uint32_t)((uint64_t)sh.ntiles * (c + 1) / P);
-}
-
 // ---------------------------------------------------------------------------
 // Kernel 0: zero the per-group amax accumulators.
 // ---------------------------------------------------------------------------
@@ -395,14 +413,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
            uint32_t* __restrict__ amax) {
   __shared__ uint32_t table[kAmaxTable];
   __shared__ int g_first_s;
-  uint32_t t0, t1;
-  cta_tile_range(sh, t0, t1);
-  if (t0 >= t1) return;
+  if (blockIdx.x >= sh.ntiles) return;
 
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (threadIdx.x == 0) {
-    gc.seek(fastdiv(t0 * kTileBlks, sh.bpr));
+    gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
     g_first_s = gc.g;
   }
   for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
@@ -419,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     else atomicMax(&amax[g], val);
   };
 
-  for (uint32_t t = t0; t < t1; ++t) {
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     V8 v[kBlkPerThread];
     const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
@@ -488,14 +504,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
     gscale[g] = group_consts(amax[g]).s_g;
 
-  uint32_t t0, t1;
-  cta_tile_range(sh, t0, t1);
   GroupCursor gc;
   gc.init(offs, sh.G);
   GroupK gk = group_consts(0u);
 
-  for (uint32_t tt = t1; tt > t0; --tt) {  // reverse order: L2 reuse after k_amax
-    const uint32_t t = tt - 1u;
+  // tiles in reverse order: k_amax read the high tiles last, so they are the
+  // most likely to be still in L2
+  for (uint32_t i = blockIdx.x; i < sh.ntiles; i += gridDim.x) {
+    const uint32_t t = sh.ntiles - 1u - i;
     V8 v[kBlkPerThread];
     const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
@@ -562,25 +578,29 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // ---------------------------------------------------------------------------
 template <bool GUIDED>
 __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const BlkK& k,
-                                            uint32_t& m2, bool& slow) {
-  const uint32_t axl_b = (w << 16) & 0x7FFF0000u, axh_b = w & 0x7FFF0000u;
-  const u64 xx = pk(__uint_as_float(axl_b), __uint_as_float(axh_b));
-  float zl, zh;
-  upk(quot2(xx, k), zl, zh);  // >= 0; +inf/NaN only where |x|/d overflows
-  m2 = (uint32_t)(zl <= 6.0f) | ((uint32_t)(zh <= 6.0f) << 1);
-  const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);  // NaN -> 6
+                                            uint32_t& m2) {
+  const u64 xx = pk(__uint_as_float((w << 16) & 0x7FFF0000u), __uint_as_float(w & 0x7FFF0000u));
   float ql, qh;
   if (GUIDED) {
-    slow |= (axl_b - 1u < k.tiny_b - 1u) | (axh_b - 1u < k.tiny_b - 1u);
-    const u64 MM = pk(grid_magic(al), grid_magic(ah));
+    // z * 2^64 (exact, >= 0; +inf/NaN only where |x|/d overflows)
+    float zl, zh;
+    upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
+    m2 = (le_mask(zl, kSixS) & 1u) | (le_mask(zh, kSixS) & 2u);
+    const float al = fminf(zl, kSixS), ah = fminf(zh, kSixS);  // NaN -> 6 * 2^64
+    const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
     const u64 aa = pk(al, ah);
     float lol, loh, hil, hih;
     upk(add_rm2(aa, MM), lol, loh);
     upk(add_rp2(aa, MM), hil, hih);
+    // of floor / ceiling, the one whose mantissa bit is the cached bit
     const float tl = ((__float_as_uint(lol) ^ bits2) & 1u) ? hil : lol;
-    const float th = ((__float_as_uint(loh) ^ (bits2 >> 1)) & 1u) ? hih : loh;
+    const float th = (((__float_as_uint(loh) << 1) ^ bits2) & 2u) ? hih : loh;
     upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
   } else {
+    float zl, zh;
+    upk(quot2(xx, k), zl, zh);
+    m2 = (le_mask(zl, 6.0f) & 1u) | (le_mask(zh, 6.0f) & 2u);
+    const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);  // NaN -> 6
     // round to nearest on the grid (ties to the even code), then dequantise
     const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
     const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
@@ -596,13 +616,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                  const uint16_t* __restrict__ mbits, const uint8_t* __restrict__ scales,
                  const float* __restrict__ gscale, V8* __restrict__ out,
                  uint16_t* __restrict__ mask) {
-  uint32_t t0, t1;
-  cta_tile_range(sh, t0, t1);
   GroupCursor gc;
   gc.init(offs, sh.G);
   float s_g = 1.0f;
 
-  for (uint32_t t = t0; t < t1; ++t) {
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     V8 v[kBlkPerThread];
     uint32_t bits[kBlkPerThread], sbs[kBlkPerThread];
     const uint32_t base = t * kTileBlks + threadIdx.x;
@@ -623,23 +641,22 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       const float d = __fmul_rn(s_g, sbv);
       V8 o;
       uint32_t m = 0u;
-      bool slow = !fast_scale(d);
       if (d == 0.0f) {
         // zero block: z = +-0, output +-0, mask set
 #pragma unroll
         for (int k = 0; k < 8; ++k) o.w[k] = v[u].w[k] & 0x80008000u;
         m = 0xFFFFu;
-        slow = false;
-      } else if (!slow) {
-        const BlkK bk = make_blk(d, sbv, s_g);
+      } else if (fast_scale(d, GUIDED ? kDMaxExactZ : kDMax)) {
+        const BlkK bk = make_blk(d, GUIDED ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
           uint32_t m2;
-          o.w[k] = fq_pair<GUIDED>(v[u].w[k], bits[u] >> (2 * k), bk, m2, slow);
+          o.w[k] = fq_pair<GUIDED>(v[u].w[k], bits[u] >> (2 * k), bk, m2);
           m |= m2 << (2 * k);
         }
+      } else {
+        fake_quant_block_exact(v[u], d, sbv, s_g, bits[u], GUIDED, &o, &m);
       }
-      if (slow) fake_quant_block_exact(v[u], d, sbv, s_g, bits[u], GUIDED, &o, &m);
       st_block(out + b, o);
       mask[b] = (uint16_t)m;
     }
@@ -652,9 +669,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint16_t* __restrict__ mask,
               V8* __restrict__ gin) {
-  uint32_t t0, t1;
-  cta_tile_range(sh, t0, t1);
-  for (uint32_t t = t0; t < t1; ++t) {
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     V8 v[kBlkPerThread];
     uint32_t m[kBlkPerThread];
     const uint32_t base = t * kTileBlks + threadIdx.x;
@@ -687,9 +702,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_copy(const V8* __restrict__ s, Shape sh, V8* __restrict__ d) {
-  uint32_t t0, t1;
-  cta_tile_range(sh, t0, t1);
-  for (uint32_t t = t0; t < t1; ++t) {
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     V8 v[kBlkPerThread];
     const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
@@ -744,7 +757,7 @@ Shape make_shape(int64_t rows, int64_t cols, int32_t G) {
 int grid_for(const Shape& sh, int* grid) {
   const int sms = sm_count();
   if (sms <= 0) return TRACE_ERR_CUDA;
-  uint32_t g = (uint32_t)sms * kCtasPerSm;
+  uint32_t g = (uint32_t)sms * kGridPerSm;
   if (sh.ntiles < g) g = sh.ntiles;
   *grid = (int)(g > 0 ? g : 1);
   return TRACE_OK;

@@ -208,10 +208,15 @@ def _all_finite_bf16():
 @pytest.mark.parametrize("bit", [0, 1])
 def test_exhaustive_bf16_fake_quant(oracle_mod, bit):
     """All finite bf16 patterns x every E4M3 block scale x several global
-    scales (power of two, full-mantissa, subnormal, huge) through the guided
-    and round-to-nearest forwards."""
+    scales (power of two, full-mantissa, subnormal, huge, and around the
+    edges of the kernels' fast range) through the guided and round-to-nearest
+    forwards."""
     pats = _all_finite_bf16()                     # [255, 256]
-    gs_vals = np.array([1.0, 0.3712345, 2.0 ** -10, 7.1e-3, 2.0 ** -140, 1.9e30],
+    # includes scales at the edges of the kernels' fast ranges (d from 2^-90
+    # to 2^16 for the guided forward, to 2^100 otherwise) and beyond them,
+    # with every bf16 input, subnormals included
+    gs_vals = np.array([1.0, 0.3712345, 2.0 ** -10, 7.1e-3, 2.0 ** -140, 1.9e30,
+                        2.0 ** 30, 1.37 * 2.0 ** -80, 3.1e10, 2.0 ** 9, 911.0],
                        np.float32)
     sbytes = np.arange(0x7F, dtype=np.uint8)
     slab = pats.shape[0]
