@@ -79,6 +79,19 @@ constexpr float kXs = 0x1p64f;
 constexpr float kSixS = 0x1p64f * 6.0f;
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch (sm_90+): every kernel waits for the
+// previous kernel in the stream to complete before it reads any global
+// memory, then lets the next kernel start launching.  Launched with the
+// programmatic-serialization attribute, a kernel's launch and prologue
+// overlap the tail of the one before it; launched without it, both
+// instructions are no-ops.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Fast unsigned 32-bit division by a runtime constant (Granlund & Montgomery,
 // "Division by invariant integers using multiplication", PLDI 1994, the
 // round-up method with the add-back step): block index -> row.
@@ -401,6 +414,7 @@ struct Shape {
 // Kernel 0: zero the per-group amax accumulators.
 // ---------------------------------------------------------------------------
 __global__ void k_zero_u32(uint32_t* p, int n) {
+  pdl_begin();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0u;
 }
 
@@ -413,6 +427,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
            uint32_t* __restrict__ amax) {
   __shared__ uint32_t table[kAmaxTable];
   __shared__ int g_first_s;
+  pdl_begin();
   if (blockIdx.x >= sh.ntiles) return;
 
   GroupCursor gc;
@@ -500,6 +515,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
               const uint32_t* __restrict__ amax, u64* __restrict__ codes,
               uint16_t* __restrict__ mbits, uint8_t* __restrict__ scales,
               float* __restrict__ gscale) {
+  pdl_begin();
   // global scales of all groups (any CTA may write them; all write the same)
   for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
     gscale[g] = group_consts(amax[g]).s_g;
@@ -579,28 +595,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 template <bool GUIDED>
 __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const BlkK& k,
                                             uint32_t& m2) {
-  const u64 xx = pk(__uint_as_float((w << 16) & 0x7FFF0000u), __uint_as_float(w & 0x7FFF0000u));
+  // signed x; only |z| is used below (sign of the output comes from w)
+  const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
   float ql, qh;
   if (GUIDED) {
-    // z * 2^64 (exact, >= 0; +inf/NaN only where |x|/d overflows)
+    // z * 2^64 (exact; +-inf/NaN only where |x|/d overflows)
     float zl, zh;
     upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
-    m2 = (le_mask(zl, kSixS) & 1u) | (le_mask(zh, kSixS) & 2u);
-    const float al = fminf(zl, kSixS), ah = fminf(zh, kSixS);  // NaN -> 6 * 2^64
+    m2 = (le_mask(fabsf(zl), kSixS) & 1u) | (le_mask(fabsf(zh), kSixS) & 2u);
+    const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
     const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
     const u64 aa = pk(al, ah);
     float lol, loh, hil, hih;
     upk(add_rm2(aa, MM), lol, loh);
     upk(add_rp2(aa, MM), hil, hih);
-    // of floor / ceiling, the one whose mantissa bit is the cached bit
-    const float tl = ((__float_as_uint(lol) ^ bits2) & 1u) ? hil : lol;
-    const float th = (((__float_as_uint(loh) << 1) ^ bits2) & 2u) ? hih : loh;
+    // of floor / ceiling, the one whose mantissa bit is the cached bit: the
+    // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
+    // bit of the floor sum is its codeword's mantissa bit
+    const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+    const float tl = __uint_as_float(lb + ((lb ^ bits2) & (__float_as_uint(hil) - lb)));
+    const float th = __uint_as_float(hb + ((hb ^ (bits2 >> 1)) & (__float_as_uint(hih) - hb)));
     upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
   } else {
     float zl, zh;
     upk(quot2(xx, k), zl, zh);
-    m2 = (le_mask(zl, 6.0f) & 1u) | (le_mask(zh, 6.0f) & 2u);
-    const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);  // NaN -> 6
+    m2 = (le_mask(fabsf(zl), 6.0f) & 1u) | (le_mask(fabsf(zh), 6.0f) & 2u);
+    const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
     // round to nearest on the grid (ties to the even code), then dequantise
     const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
     const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
@@ -616,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                  const uint16_t* __restrict__ mbits, const uint8_t* __restrict__ scales,
                  const float* __restrict__ gscale, V8* __restrict__ out,
                  uint16_t* __restrict__ mask) {
+  pdl_begin();
   GroupCursor gc;
   gc.init(offs, sh.G);
   float s_g = 1.0f;
@@ -669,6 +690,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint16_t* __restrict__ mask,
               V8* __restrict__ gin) {
+  pdl_begin();
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     V8 v[kBlkPerThread];
     uint32_t m[kBlkPerThread];
@@ -702,6 +724,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_copy(const V8* __restrict__ s, Shape sh, V8* __restrict__ d) {
+  pdl_begin();
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     V8 v[kBlkPerThread];
     const uint32_t base = t * kTileBlks + threadIdx.x;
@@ -763,7 +786,24 @@ int grid_for(const Shape& sh, int* grid) {
   return TRACE_OK;
 }
 
-int launched() { return cudaGetLastError() == cudaSuccess ? TRACE_OK : TRACE_ERR_CUDA; }
+// Launch with programmatic stream serialization (see pdl_begin): the kernel
+// may begin launching while the previous kernel in the stream finishes; it
+// waits for it before touching memory.
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? TRACE_OK
+                                                                                      : TRACE_ERR_CUDA;
+}
 
 }  // namespace
 
@@ -809,11 +849,10 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_gro
   uint32_t* amax = (uint32_t*)workspace;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
   const int zg = (num_groups + kThreads - 1) / kThreads;
-  k_zero_u32<<<zg < 1024 ? zg : 1024, kThreads, 0, s>>>(amax, num_groups);
-  if (sh.nblk > 0) k_amax<<<grid, kThreads, 0, s>>>((const V8*)x, sh, offs, amax);
-  k_capture<<<grid, kThreads, 0, s>>>((const V8*)x, sh, offs, amax, (u64*)codes,
-                                      (uint16_t*)mbits, scales, gscale);
-  return launched();
+  if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups))) return st;
+  if (sh.nblk > 0 && (st = launch(k_amax, grid, s, (const V8*)x, sh, offs, amax))) return st;
+  return launch(k_capture, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax, (u64*)codes,
+                (uint16_t*)mbits, scales, gscale);
 }
 
 static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
@@ -833,12 +872,10 @@ static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* o = G > 1 ? offs : nullptr;
   if (guided)
-    k_fake_quant<true><<<grid, kThreads, 0, s>>>((const V8*)x, sh, o, (const uint16_t*)mbits,
-                                                 scales, gscale, (V8*)out, (uint16_t*)mask);
-  else
-    k_fake_quant<false><<<grid, kThreads, 0, s>>>((const V8*)x, sh, o, nullptr, scales, gscale,
-                                                  (V8*)out, (uint16_t*)mask);
-  return launched();
+    return launch(k_fake_quant<true>, grid, s, (const V8*)x, sh, o, (const uint16_t*)mbits, scales,
+                  gscale, (V8*)out, (uint16_t*)mask);
+  return launch(k_fake_quant<false>, grid, s, (const V8*)x, sh, o, (const uint16_t*)nullptr, scales,
+                gscale, (V8*)out, (uint16_t*)mask);
 }
 
 int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols, int32_t num_groups,
@@ -866,9 +903,8 @@ int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t num
   const Shape sh = make_shape(numel / 32, 32, 1);
   int grid, st;
   if ((st = grid_for(sh, &grid))) return st;
-  k_ste_bwd<<<grid, kThreads, 0, (cudaStream_t)stream>>>((const V8*)grad_out, sh,
-                                                         (const uint16_t*)ste_mask, (V8*)grad_in);
-  return launched();
+  return launch(k_ste_bwd, grid, (cudaStream_t)stream, (const V8*)grad_out, sh,
+                (const uint16_t*)ste_mask, (V8*)grad_in);
 }
 
 int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* stream) {
@@ -884,8 +920,7 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* str
   sh.G = 1;
   int grid, st;
   if ((st = grid_for(sh, &grid))) return st;
-  k_copy<<<grid, kThreads, 0, (cudaStream_t)stream>>>((const V8*)src, sh, (V8*)dst);
-  return launched();
+  return launch(k_copy, grid, (cudaStream_t)stream, (const V8*)src, sh, (V8*)dst);
 }
 
 }  // extern "C"
