@@ -923,4 +923,38 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* str
   return launch(k_copy, grid, (cudaStream_t)stream, (const V8*)src, sh, (V8*)dst);
 }
 
+
+// ---------------------------------------------------------------------------
+// Capture without a caller-provided workspace.
+//
+// Some callers cannot hand the library a scratch buffer: a host program whose
+// device memory is carved up once at start-up and may not grow afterwards, or
+// a thin binding that only forwards the tensors it was given and has no
+// allocator to call.  This entry point therefore keeps the amax accumulators
+// that trace_capture takes as `workspace` in a fixed array that lives in the
+// library itself, one copy per GPU, for the life of the process.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint32_t g_capture_scratch[TRACE_STATIC_MAX_GROUPS];
+
+static void* g_capture_scratch_addr[kMaxDevices];  // per device; benign race (same value)
+
+int trace_capture_static_ws(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
+                            const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
+                            uint8_t* scales, float* gscale, void* stream) {
+  if (num_groups > TRACE_STATIC_MAX_GROUPS) return TRACE_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TRACE_ERR_CUDA;
+  void* ws = g_capture_scratch_addr[dev];
+  if (ws == nullptr) {
+    // first call on this device: the host-side name of the array is only a
+    // stand-in, so ask the runtime for its address on the current device
+    if (cudaGetSymbolAddress(&ws, g_capture_scratch) != cudaSuccess || ws == nullptr)
+      return TRACE_ERR_CUDA;
+    g_capture_scratch_addr[dev] = ws;
+  }
+  // the accumulators are zeroed by the capture's first kernel on every call
+  return trace_capture(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,
+                       ws, sizeof(g_capture_scratch), stream);
+}
+
 }  // extern "C"

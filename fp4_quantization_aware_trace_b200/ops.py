@@ -58,6 +58,8 @@ def library() -> ctypes.CDLL:
         lib.trace_rtn_fq_fwd.restype = ctypes.c_int
         lib.trace_copy_bf16.argtypes = [P, P, i64, P]
         lib.trace_copy_bf16.restype = ctypes.c_int
+        lib.trace_capture_static_ws.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
+        lib.trace_capture_static_ws.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -124,6 +126,19 @@ def trace_rtn_fq_fwd(x, rows, cols, num_groups, offsets, scales, gscale, out, st
     _check(library().trace_rtn_fq_fwd(_p(x), rows, cols, num_groups, _p(offsets), _p(scales),
                                       _p(gscale), _p(out), _p(ste_mask), _stream(stream)),
            "trace_rtn_fq_fwd")
+
+
+def trace_capture_static_ws(x, rows, cols, num_groups, offsets, codes, mbits, scales, gscale,
+                            stream=None) -> None:
+    """trace_capture for callers that cannot supply a workspace: the library
+    keeps the scratch in a fixed per-GPU array (at most
+    TRACE_STATIC_MAX_GROUPS groups; calls must not overlap on the GPU)."""
+    _check(library().trace_capture_static_ws(_p(x), rows, cols, num_groups, _p(offsets),
+                                             _p(codes), _p(mbits), _p(scales), _p(gscale),
+                                             _stream(stream)), "trace_capture_static_ws")
+
+
+TRACE_STATIC_MAX_GROUPS = 4096
 
 
 def trace_copy_bf16(src, dst, numel, stream=None) -> None:

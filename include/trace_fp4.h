@@ -144,6 +144,31 @@ int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
 int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel,
                     void* stream);
 
+/* Rollout capture for callers that cannot provide a workspace.  The paper
+ * has no counterpart: this is a calling convention, not a step of the method.
+ * Who needs it: a caller that may not allocate device memory when it calls
+ * the library -- e.g. a host program whose device memory is fixed at
+ * start-up, or a binding that can only pass along the buffers it was given.
+ * Instead of a `workspace` argument, the amax accumulators live in a static
+ * array inside the library: TRACE_STATIC_MAX_GROUPS uint32 (16 KiB) per GPU
+ * that loads the library, kept until the process exits.
+ *   Arguments and outputs are those of trace_capture without `workspace`.
+ *   num_groups > TRACE_STATIC_MAX_GROUPS: returns TRACE_ERR_WORKSPACE and
+ *   enqueues nothing.
+ *   The first call on each device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  Nothing here calls cudaMalloc or cudaFree.
+ *   Every call on a device shares the one array (its contents are zeroed at
+ *   the start of each call): two calls that may run at the same time on the
+ *   GPU -- e.g. on streams with no ordering between them -- race on it and
+ *   give wrong results; order them (one stream, or events). */
+#define TRACE_STATIC_MAX_GROUPS 4096
+int trace_capture_static_ws(const uint16_t* x, int64_t rows, int64_t cols,
+                            int32_t num_groups,
+                            const int64_t* group_row_offsets, uint8_t* codes,
+                            uint32_t* mbits, uint8_t* scales, float* gscale,
+                            void* stream);
+
 #ifdef __cplusplus
 }
 #endif
