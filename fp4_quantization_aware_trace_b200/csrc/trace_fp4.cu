@@ -510,10 +510,58 @@ __device__ __forceinline__ GroupK group_consts(uint32_t amax_bits) {
 // Kernel 2: capture.  Per 16-element block: E4M3 scale; per element: the
 // round-to-nearest code and its mantissa bit.
 // ---------------------------------------------------------------------------
+// One block: returns its E4M3 scale byte, writes its 16 codes to c0 (elements
+// 0-7) and c1 (8-15).
+__device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk, uint32_t& c0,
+                                                  uint32_t& c1) {
+  // block scale: t = bmax / RN(6 s_g), E4M3 round-to-nearest-even, satfinite
+  const float bmax = __uint_as_float(absmax_block(v) << 16);
+  float tq;
+  if (gk.fast6) {
+    const float q0 = __fmul_rn(bmax, gk.r6);
+    tq = __fmaf_rn(__fmaf_rn(q0, -gk.den6, bmax), gk.r6, q0);
+  } else {
+    tq = __fdiv_rn(bmax, gk.den6);
+  }
+  const uint32_t sb = cvt_e4m3(tq);
+  const float d = __fmul_rn(gk.s_g, e4m3_to_f32(sb));
+  if (d == 0.0f) {
+    // zero block: z = +-0, code = sign only
+    c0 = c1 = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = v.w[k];
+      const uint32_t nib = (((w >> 15) & 1u) << 3) | ((w >> 31) << 7);
+      if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
+    }
+  } else if (fast_scale(d)) {
+    const BlkK bk = make_blk(d, 0.0f, 0.0f);
+    uint32_t c[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = v.w[k];
+      const float xl = bf16_lo(w), xh = bf16_hi(w);
+      float zl, zh;
+      upk(quot2(pk(xl, xh), bk), zl, zh);
+      // the code carries the sign of x (also for zeros and underflows)
+      zl = __uint_as_float((__float_as_uint(zl) & 0x7FFFFFFFu) | (__float_as_uint(xl) & 0x80000000u));
+      zh = __uint_as_float((__float_as_uint(zh) & 0x7FFFFFFFu) | (w & 0x80000000u));
+      c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+    }
+    c0 = c[0];
+    c1 = c[1];
+  } else {
+    capture_block_exact(v, d, &c0, &c1);
+  }
+  return sb;
+}
+
+// Each thread owns two adjacent blocks: one 16-byte store of codes, one
+// 32-bit store of mantissa bits, one 16-bit store of scales.
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-              const uint32_t* __restrict__ amax, u64* __restrict__ codes,
-              uint16_t* __restrict__ mbits, uint8_t* __restrict__ scales,
+              const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
+              uint32_t* __restrict__ mbits, uint16_t* __restrict__ scales,
               float* __restrict__ gscale) {
   pdl_begin();
   // global scales of all groups (any CTA may write them; all write the same)
@@ -528,62 +576,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   // most likely to be still in L2
   for (uint32_t i = blockIdx.x; i < sh.ntiles; i += gridDim.x) {
     const uint32_t t = sh.ntiles - 1u - i;
-    V8 v[kBlkPerThread];
-    const uint32_t base = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
-    }
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      if (b >= sh.nblk) continue;
-      if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) gk = group_consts(__ldg(amax + gc.g));
-      // block scale: t = bmax / RN(6 s_g), E4M3 round-to-nearest-even, satfinite
-      const float bmax = __uint_as_float(absmax_block(v[u]) << 16);
-      float tq;
-      if (gk.fast6) {
-        const float q0 = __fmul_rn(bmax, gk.r6);
-        tq = __fmaf_rn(__fmaf_rn(q0, -gk.den6, bmax), gk.r6, q0);
-      } else {
-        tq = __fdiv_rn(bmax, gk.den6);
-      }
-      const uint32_t sb = cvt_e4m3(tq);
-      const float d = __fmul_rn(gk.s_g, e4m3_to_f32(sb));
-      uint32_t c0, c1;
-      if (d == 0.0f) {
-        // zero block: z = +-0, code = sign only
-        c0 = c1 = 0u;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t w = v[u].w[k];
-          const uint32_t nib = (((w >> 15) & 1u) << 3) | ((w >> 31) << 7);
-          if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
-        }
-      } else if (fast_scale(d)) {
-        const BlkK bk = make_blk(d, 0.0f, 0.0f);
-        uint32_t c[2] = {0u, 0u};
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const uint32_t w = v[u].w[k];
-          const float xl = bf16_lo(w), xh = bf16_hi(w);
-          float zl, zh;
-          upk(quot2(pk(xl, xh), bk), zl, zh);
-          // the code carries the sign of x (also for zeros and underflows)
-          zl = __uint_as_float((__float_as_uint(zl) & 0x7FFFFFFFu) | (__float_as_uint(xl) & 0x80000000u));
-          zh = __uint_as_float((__float_as_uint(zh) & 0x7FFFFFFFu) | (w & 0x80000000u));
-          c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
-        }
-        c0 = c[0];
-        c1 = c[1];
-      } else {
-        capture_block_exact(v[u], d, &c0, &c1);
-      }
-      codes[b] = ((u64)c1 << 32) | c0;
-      mbits[b] = (uint16_t)(nibble_lsbs(c0) | (nibble_lsbs(c1) << 8));
-      scales[b] = (uint8_t)sb;
-    }
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    // both blocks of the pair are in the same row (cols is a multiple of 32)
+    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) gk = group_consts(__ldg(amax + gc.g));
+    uint4 c;
+    const uint32_t s0 = capture_block(v0, gk, c.x, c.y);
+    const uint32_t s1 = capture_block(v1, gk, c.z, c.w);
+    codes[b >> 1] = c;
+    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
+                    (nibble_lsbs(c.w) << 24);
+    scales[b >> 1] = (uint16_t)(s0 | (s1 << 8));
   }
 }
 
@@ -594,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // ---------------------------------------------------------------------------
 template <bool GUIDED>
 __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const BlkK& k,
-                                            uint32_t& m2) {
+                                            uint32_t& m, int pos) {
   // signed x; only |z| is used below (sign of the output comes from w)
   const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
   float ql, qh;
@@ -602,7 +606,7 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const Bl
     // z * 2^64 (exact; +-inf/NaN only where |x|/d overflows)
     float zl, zh;
     upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
-    m2 = (le_mask(fabsf(zl), kSixS) & 1u) | (le_mask(fabsf(zh), kSixS) & 2u);
+    m |= (le_mask(fabsf(zl), kSixS) & (1u << pos)) | (le_mask(fabsf(zh), kSixS) & (2u << pos));
     const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
     const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
     const u64 aa = pk(al, ah);
@@ -619,7 +623,7 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const Bl
   } else {
     float zl, zh;
     upk(quot2(xx, k), zl, zh);
-    m2 = (le_mask(fabsf(zl), 6.0f) & 1u) | (le_mask(fabsf(zh), 6.0f) & 2u);
+    m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
     const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
     // round to nearest on the grid (ties to the even code), then dequantise
     const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
@@ -630,57 +634,56 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const Bl
   return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
 }
 
+// One 16-element block of the fake-quant forward: bf16 outputs and 16 mask
+// bits (in the low half of the returned mask).
+template <bool GUIDED>
+__device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, float sbv,
+                                                 float s_g, V8& o, uint32_t& m) {
+  const float d = __fmul_rn(s_g, sbv);
+  m = 0u;
+  if (d == 0.0f) {
+    // zero block: z = +-0, output +-0, mask set
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o.w[k] = v.w[k] & 0x80008000u;
+    m = 0xFFFFu;
+  } else if (fast_scale(d, GUIDED ? kDMaxExactZ : kDMax)) {
+    const BlkK bk = make_blk(d, GUIDED ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o.w[k] = fq_pair<GUIDED>(v.w[k], bits16 >> (2 * k), bk, m, 2 * k);
+  } else {
+    fake_quant_block_exact(v, d, sbv, s_g, bits16, GUIDED, &o, &m);
+  }
+}
+
+// Each thread owns two adjacent blocks, so their mantissa bits, scales and
+// mask move as one 32-bit / 16-bit / 32-bit access.
 template <bool GUIDED>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-                 const uint16_t* __restrict__ mbits, const uint8_t* __restrict__ scales,
+                 const uint32_t* __restrict__ mbits, const uint16_t* __restrict__ scales,
                  const float* __restrict__ gscale, V8* __restrict__ out,
-                 uint16_t* __restrict__ mask) {
+                 uint32_t* __restrict__ mask) {
   pdl_begin();
   GroupCursor gc;
   gc.init(offs, sh.G);
   float s_g = 1.0f;
 
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    V8 v[kBlkPerThread];
-    uint32_t bits[kBlkPerThread], sbs[kBlkPerThread];
-    const uint32_t base = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      const bool valid = b < sh.nblk;
-      v[u] = valid ? ld_block_stream(x + b) : zero_block();
-      bits[u] = (GUIDED && valid) ? (uint32_t)__ldcs(mbits + b) : 0u;
-      sbs[u] = valid ? (uint32_t)__ldcs(scales + b) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      if (b >= sh.nblk) continue;
-      if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
-      const float sbv = e4m3_to_f32(sbs[u]);
-      const float d = __fmul_rn(s_g, sbv);
-      V8 o;
-      uint32_t m = 0u;
-      if (d == 0.0f) {
-        // zero block: z = +-0, output +-0, mask set
-#pragma unroll
-        for (int k = 0; k < 8; ++k) o.w[k] = v[u].w[k] & 0x80008000u;
-        m = 0xFFFFu;
-      } else if (fast_scale(d, GUIDED ? kDMaxExactZ : kDMax)) {
-        const BlkK bk = make_blk(d, GUIDED ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          uint32_t m2;
-          o.w[k] = fq_pair<GUIDED>(v[u].w[k], bits[u] >> (2 * k), bk, m2);
-          m |= m2 << (2 * k);
-        }
-      } else {
-        fake_quant_block_exact(v[u], d, sbv, s_g, bits[u], GUIDED, &o, &m);
-      }
-      st_block(out + b, o);
-      mask[b] = (uint16_t)m;
-    }
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = GUIDED ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint32_t sb2 = __ldcs(scales + (b >> 1));
+    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
+    V8 o;
+    uint32_t m0, m1;
+    fake_quant_block<GUIDED>(v0, bits & 0xFFFFu, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
+    st_block(out + b, o);
+    // a row holds a whole number of 32-element words, so both blocks of the
+    // pair are in the same row and group
+    fake_quant_block<GUIDED>(v1, bits >> 16, e4m3_to_f32(sb2 >> 8), s_g, o, m1);
+    st_block(out + b + 1, o);
+    mask[b >> 1] = m0 | (m1 << 16);
   }
 }
 
@@ -688,34 +691,25 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // Kernel 4: masked straight-through backward.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint16_t* __restrict__ mask,
+    k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint32_t* __restrict__ mask,
               V8* __restrict__ gin) {
   pdl_begin();
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    V8 v[kBlkPerThread];
-    uint32_t m[kBlkPerThread];
-    const uint32_t base = t * kTileBlks + threadIdx.x;
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // two adjacent blocks
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(g + b), v1 = ld_block_stream(g + b + 1);
+    const uint32_t m = __ldcs(mask + (b >> 1));
+    V8 r0, r1;
 #pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      const bool valid = b < sh.nblk;
-      v[u] = valid ? ld_block_stream(g + b) : zero_block();
-      m[u] = valid ? (uint32_t)__ldcs(mask + b) : 0u;
+    for (int k = 0; k < 8; ++k) {
+      // bits (2k, 2k+1) -> keep masks of the two halves of word k
+      r0.w[k] = v0.w[k] & ((((m >> (2 * k)) & 1u) * 0x0000FFFFu) |
+                           (((m >> (2 * k + 1)) & 1u) * 0xFFFF0000u));
+      r1.w[k] = v1.w[k] & ((((m >> (2 * k + 16)) & 1u) * 0x0000FFFFu) |
+                           (((m >> (2 * k + 17)) & 1u) * 0xFFFF0000u));
     }
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      if (b >= sh.nblk) continue;
-      V8 r;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        // bits (2k, 2k+1) -> keep masks of the two halves of word k
-        const uint32_t keep = (((m[u] >> (2 * k)) & 1u) * 0x0000FFFFu) |
-                              (((m[u] >> (2 * k + 1)) & 1u) * 0xFFFF0000u);
-        r.w[k] = v[u].w[k] & keep;
-      }
-      st_block(gin + b, r);
-    }
+    st_block(gin + b, r0);
+    st_block(gin + b + 1, r1);
   }
 }
 
@@ -851,8 +845,8 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_gro
   const int zg = (num_groups + kThreads - 1) / kThreads;
   if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups))) return st;
   if (sh.nblk > 0 && (st = launch(k_amax, grid, s, (const V8*)x, sh, offs, amax))) return st;
-  return launch(k_capture, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax, (u64*)codes,
-                (uint16_t*)mbits, scales, gscale);
+  return launch(k_capture, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax, (uint4*)codes,
+                (uint32_t*)mbits, (uint16_t*)scales, gscale);
 }
 
 static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
@@ -872,10 +866,10 @@ static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* o = G > 1 ? offs : nullptr;
   if (guided)
-    return launch(k_fake_quant<true>, grid, s, (const V8*)x, sh, o, (const uint16_t*)mbits, scales,
-                  gscale, (V8*)out, (uint16_t*)mask);
-  return launch(k_fake_quant<false>, grid, s, (const V8*)x, sh, o, (const uint16_t*)nullptr, scales,
-                gscale, (V8*)out, (uint16_t*)mask);
+    return launch(k_fake_quant<true>, grid, s, (const V8*)x, sh, o, (const uint32_t*)mbits,
+                  (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
+  return launch(k_fake_quant<false>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
+                (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
 }
 
 int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols, int32_t num_groups,
@@ -904,7 +898,7 @@ int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t num
   int grid, st;
   if ((st = grid_for(sh, &grid))) return st;
   return launch(k_ste_bwd, grid, (cudaStream_t)stream, (const V8*)grad_out, sh,
-                (const uint16_t*)ste_mask, (V8*)grad_in);
+                (const uint32_t*)ste_mask, (V8*)grad_in);
 }
 
 int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* stream) {
