@@ -19,8 +19,11 @@ two passes).  Per-element bytes: capture 4.6875, guided 4.3125, backward
 measured HBM copy bandwidth are reported beside it.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl trace|reference]
-Under torchrun every rank runs its own site (weak scaling, no collective on
-the data path); rank 0 prints one JSON line.
+                       [--config 1..5]
+--config picks another of the five workloads for the same measurement (a step
+then covers every tensor of the workload; the headline is --config 2, the
+default).  Under torchrun every rank runs its own sites (weak scaling, no
+collective on the data path); rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -63,6 +66,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline leg")
+    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5],
+                    help="workload: 1 single activation, 2 attention input (default, the "
+                         "headline), 3 MoE experts, 4 KV cache, 5 later-half layer sweep")
     return ap.parse_args()
 
 
@@ -176,6 +182,33 @@ def make_site(rank: int, device):
     return inputs.attention_input(seed=site_seed(rank), rows=ROWS, cols=COLS, device=device)
 
 
+def make_workload(cfg: int, rank: int, device):
+    """(workload name, sites) of a configuration; rank r shifts every seed."""
+    from fp4_quantization_aware_trace_b200 import inputs
+    off = 1000 * rank
+    if cfg == 1:
+        return ("single activation [256 x 2048] bf16, 8 outlier channels x50",
+                [inputs.single_activation(0 + off, device=device)])
+    if cfg == 2:
+        return WORKLOAD, [make_site(rank, device)]
+    if cfg == 3:
+        return ("MoE experts: 128 experts x 512 tokens, up-proj input [65536 x 2048] and "
+                "down-proj input [65536 x 768] bf16, one group per expert",
+                [inputs.moe_experts(2 + off, cols=2048, device=device, name="expert_up_in"),
+                 inputs.moe_experts(12 + off, cols=768, device=device, name="expert_down_in")])
+    if cfg == 4:
+        return ("FP4 KV cache: K and V [32768 tokens, 4 heads, 128] bf16 as [131072 x 128]",
+                [inputs.kv_cache(3 + off, device=device, which="k"),
+                 inputs.kv_cache(3 + off, device=device, which="v")])
+    sites = [inputs.layer_sweep_site(layer, k, device=device)
+             for layer in (20, 21) for k in range(4)]
+    if rank:
+        sites = [inputs.layer_sweep_site(20 + 2 * rank + layer % 2, k, device=device)
+                 for layer in (20, 21) for k in range(4)]
+    return ("later-half layer sweep: 8 of the 80 sites (layers 20-21 x qkv-in, o-in, up-in, "
+            "down-in), each [65536 x 4096] bf16", sites)
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle legs (reported baseline / reference arm)
 # ---------------------------------------------------------------------------
@@ -267,30 +300,41 @@ def run_trace(args):
     from fp4_quantization_aware_trace_b200 import ops
     ops.library()
 
-    site = make_site(rank, dev)
-    xr, xt, g = site.x_roll, site.x_train, site.grad
-    n = xr.numel()
-    cap, ws = ops.alloc_capture(ROWS, COLS, 1, dev)
-    out = torch.empty_like(xt)
-    mask = torch.empty(n // 32, dtype=torch.int32, device=dev)
-    gin = torch.empty_like(g)
-    out_r = torch.empty_like(xt)
-    mask_r = torch.empty_like(mask)
+    workload, sites = make_workload(args.config, rank, dev)
+    work = []
+    for site in sites:
+        R, C = site.x_roll.shape
+        offs = None if site.offsets is None else site.offsets.to(dev)
+        cap, ws = ops.alloc_capture(R, C, site.num_groups, dev, offs)
+        w = dict(site=site, xr=site.x_roll.contiguous(), xt=site.x_train.contiguous(),
+                 g=site.grad.contiguous(), offs=offs, cap=cap, ws=ws,
+                 out=torch.empty_like(site.x_train), gin=torch.empty_like(site.grad),
+                 out_r=torch.empty_like(site.x_train),
+                 mask=torch.empty(R * C // 32, dtype=torch.int32, device=dev),
+                 mask_r=torch.empty(R * C // 32, dtype=torch.int32, device=dev))
+        work.append(w)
+    n = sum(w["xr"].numel() for w in work)
+    groups = [w["site"].num_groups for w in work]
+    shapes = [list(w["xr"].shape) for w in work]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(ev=None, dom=None):
-        if ev: ev[0].record(stream)
-        ops.capture(xr, None, cap, ws, stream)
-        if ev: ev[1].record(stream)
-        if dom: dom[0].record(stream)
-        ops.guided_fq_fwd(xt, cap, out, mask, stream)
-        if ev: ev[2].record(stream)
-        if dom: dom[1].record(stream)
-        ops.fq_bwd(g, mask, gin, stream)
-        if ev: ev[3].record(stream)
-        ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, None, out_r, mask_r, stream)
-        if ev: ev[4].record(stream)
+        for i, w in enumerate(work):
+            e = ev[i] if ev else None
+            d = dom[i] if dom else None
+            if e: e[0].record(stream)
+            ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], stream)
+            if e: e[1].record(stream)
+            if d: d[0].record(stream)
+            ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], stream)
+            if e: e[2].record(stream)
+            if d: d[1].record(stream)
+            ops.fq_bwd(w["g"], w["mask"], w["gin"], stream)
+            if e: e[3].record(stream)
+            ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                           w["mask_r"], stream)
+            if e: e[4].record(stream)
 
     for i in range(max(args.warmup, 3)):
         flush.fill_(i & 0xFF)
@@ -303,11 +347,12 @@ def run_trace(args):
                for _ in range(args.steps)]
     # the dominant kernel (guided forward) is also bracketed inside the timed
     # steps, for the roofline's achieved bandwidth
-    dom_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(args.steps)]
+    dom_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in work] for _ in range(args.steps)]
     # per-kernel breakdown: events between the calls (which can delay the
     # next launch a little, so these durations are slightly pessimistic)
-    kern_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    kern_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
+               for _ in range(args.steps)]
     with ClockSampler(local) as clk:
         if pg: pg.barrier()
         torch.cuda.synchronize()
@@ -327,10 +372,11 @@ def run_trace(args):
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
     per_kernel = {nm: 0.0 for nm in names}
     total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
-    dom_ms = sum(a.elapsed_time(b) for a, b in dom_ev)
-    for ev in kern_ev:
-        for i, nm in enumerate(names):
-            per_kernel[nm] += ev[i].elapsed_time(ev[i + 1])
+    dom_ms = sum(a.elapsed_time(b) for per in dom_ev for a, b in per)
+    for per in kern_ev:
+        for ev in per:
+            for i, nm in enumerate(names):
+                per_kernel[nm] += ev[i].elapsed_time(ev[i + 1])
     t_max = max_over_ranks([total_ms, dom_ms] + [per_kernel[nm] for nm in names], pg, dev)
     total_ms, dom_ms = t_max[0], t_max[1]
     per_kernel = {nm: t_max[i + 2] for i, nm in enumerate(names)}
@@ -355,38 +401,38 @@ def run_trace(args):
     traffic = traffic_from_profiles("k_fake_quant_guided")
 
     # --- yardstick: the library's plain copy kernel on the same bytes -------
-    ysrc = torch.empty(n, dtype=torch.bfloat16, device=dev).fill_(1.0)
+    ny = max(w["xr"].numel() for w in work)
+    ysrc = torch.empty(ny, dtype=torch.bfloat16, device=dev).fill_(1.0)
     ydst = torch.empty_like(ysrc)
     yev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for i in range(3):
         flush.fill_(i)
-        ops.trace_copy_bf16(ysrc, ydst, n, stream)
+        ops.trace_copy_bf16(ysrc, ydst, ny, stream)
     for k in range(args.steps):
         flush.fill_((k + 3) & 0xFF)
         yev[k][0].record(stream)
-        ops.trace_copy_bf16(ysrc, ydst, n, stream)
+        ops.trace_copy_bf16(ysrc, ydst, ny, stream)
         yev[k][1].record(stream)
     torch.cuda.synchronize()
     y_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in yev) / args.steps], pg, dev)[0]
-    yardstick = {"kernel": "k_copy", "bytes": 4 * n, "us": round(y_ms * 1e3, 2),
-                 "gbs": round(4 * n / (y_ms * 1e-3) / 1e9, 1)}
+    yardstick = {"kernel": "k_copy", "bytes": 4 * ny, "us": round(y_ms * 1e3, 2),
+                 "gbs": round(4 * ny / (y_ms * 1e-3) / 1e9, 1)}
     del ysrc, ydst
 
     # --- end-to-end through the C ABI with pinned host buffers -------------
     e2e = None
-    if not args.no_e2e:
-        hx = [t.cpu().pin_memory() for t in (xr, xt, g)]
-        houts = [torch.empty(t.shape, dtype=t.dtype).pin_memory()
-                 for t in (cap.codes, cap.mbits, cap.scales, cap.gscale, out, mask, gin, out_r, mask_r)]
-        douts = [cap.codes, cap.mbits, cap.scales, cap.gscale, out, mask, gin, out_r, mask_r]
+    if not args.no_e2e and args.config == 2:
+        ins = [(w[k], w[k].cpu().pin_memory()) for w in work for k in ("xr", "xt", "g")]
+        outs = [(d, torch.empty(d.shape, dtype=d.dtype).pin_memory()) for w in work
+                for d in (w["cap"].codes, w["cap"].mbits, w["cap"].scales, w["cap"].gscale,
+                          w["out"], w["mask"], w["gin"], w["out_r"], w["mask_r"])]
 
         def e2e_step():
-            xr.copy_(hx[0], non_blocking=True)
-            xt.copy_(hx[1], non_blocking=True)
-            g.copy_(hx[2], non_blocking=True)
+            for d, h in ins:
+                d.copy_(h, non_blocking=True)
             step()
-            for h, d in zip(houts, douts):
+            for d, h in outs:
                 h.copy_(d, non_blocking=True)
 
         for _ in range(3):
@@ -400,15 +446,15 @@ def run_trace(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks([e0.elapsed_time(e1)], pg, dev)[0] / args.steps
-        h2d = sum(h.numel() * h.element_size() for h in hx)
-        d2h = sum(h.numel() * h.element_size() for h in houts)
+        h2d = sum(h.numel() * h.element_size() for _, h in ins)
+        d2h = sum(h.numel() * h.element_size() for _, h in outs)
         e2e = {"value": round(job_gbs(world, n, bpe, e2e_ms), 3), "unit": "GB/s",
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "elem_per_s": round(world * n / (e2e_ms * 1e-3), 1)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, eps, per, sample = cpu_oracle_rate(site, args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
+        gbs, eps, per, sample = cpu_oracle_rate(work[0]["site"], args.cpu_seconds)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": sample, "elem_per_s": round(eps, 1), "s_per_step": round(per, 3)}
 
@@ -424,7 +470,7 @@ def run_trace(args):
         "data": "synthetic",
         "elem_per_s": round(world * n / (ms_step * 1e-3), 1),
         "frac_of_hbm": round(value / world / hbm, 4),
-        "config": {"workload": WORKLOAD, "rows": ROWS, "cols": COLS, "groups": 1,
+        "config": {"workload": workload, "shapes": shapes, "groups": groups,
                    "step": "capture + guided fwd + STE bwd + RTN fwd",
                    "l2": "flushed before every step (256 MiB write)",
                    "parallelism": f"{world} independent sites, one per GPU (no collective)"},
@@ -437,7 +483,7 @@ def run_trace(args):
                      "algorithmic_bytes": int(dom_bytes)},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * len(work) * args.steps,
         "timing": ("value: events around each step only; kernels: a second, untimed pass of "
                    "the same steps with events between the calls"),
         "clocks": clocks,
