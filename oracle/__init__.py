@@ -90,6 +90,14 @@ def _load():
         lib.oracle_fake_quant_rows.restype = None
         lib.oracle_fake_quant_codes.argtypes = [P, i64, i64, i32, P, P, P, P, P]
         lib.oracle_fake_quant_codes.restype = None
+        lib.oracle_full_guided_code.argtypes = [f32, ctypes.c_int]
+        lib.oracle_full_guided_code.restype = ctypes.c_int
+        lib.oracle_full_guided_fwd.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
+        lib.oracle_full_guided_fwd.restype = None
+        lib.oracle_full_guided_codes.argtypes = [P, i64, i64, i32, P, P, P, P, P]
+        lib.oracle_full_guided_codes.restype = None
+        lib.oracle_full_guided_rows.argtypes = [P, i64, i64, P, P, P, P, P]
+        lib.oracle_full_guided_rows.restype = None
         _lib = lib
         return lib
 
@@ -296,3 +304,54 @@ def unpack_bits(words: np.ndarray) -> np.ndarray:
     """Packed u32 bit words -> one 0/1 byte per element (layout helper)."""
     w = np.asarray(words, dtype=np.uint32).view(np.uint8)
     return np.unpackbits(w, bitorder="little")
+
+
+# -- full-information guidance (the cache keeps the whole rollout code) ------
+
+def full_guided_code(z: float, roll_code: int) -> int:
+    """Magnitude code of q* for unclipped z and a signed rollout code."""
+    return _load().oracle_full_guided_code(z, roll_code)
+
+
+def full_guided_fwd(x_train, rcodes, scales, gscale, num_groups: int = 1, offsets=None):
+    """Full-information guided forward.  Returns (out, mask)."""
+    x = _as_bf16_bits(x_train)
+    rows, cols = x.shape
+    o = _offsets(offsets, num_groups, rows)
+    rcodes = np.ascontiguousarray(rcodes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    gscale = np.ascontiguousarray(gscale, dtype=np.float32)
+    assert rcodes.size == rows * cols // 2 and scales.size == rows * cols // 16
+    out = np.zeros((rows, cols), np.uint16)
+    mask = np.zeros(rows * cols // 32, np.uint32)
+    _load().oracle_full_guided_fwd(_ptr(x), rows, cols, num_groups, _ptr(o), _ptr(rcodes),
+                                   _ptr(scales), _ptr(gscale), _ptr(out), _ptr(mask))
+    return out, mask
+
+
+def full_guided_codes(x, rcodes, scales, gscale, num_groups: int = 1, offsets=None):
+    """Signed code picked at every site by full-information guidance."""
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    o = _offsets(offsets, num_groups, rows)
+    sites = np.zeros((rows, cols), np.uint8)
+    _load().oracle_full_guided_codes(_ptr(x), rows, cols, num_groups, _ptr(o),
+                                     _ptr(np.ascontiguousarray(rcodes, dtype=np.uint8)),
+                                     _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
+                                     _ptr(np.ascontiguousarray(gscale, dtype=np.float32)),
+                                     _ptr(sites))
+    return sites
+
+
+def full_guided_rows(x, row_gscale, scales, rcodes):
+    """Full-information guided forward for rows with known global scales."""
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    rg = np.ascontiguousarray(row_gscale, dtype=np.float32)
+    out = np.zeros((rows, cols), np.uint16)
+    mask = np.zeros(rows * cols // 32, np.uint32)
+    _load().oracle_full_guided_rows(_ptr(x), rows, cols, _ptr(rg),
+                                    _ptr(np.ascontiguousarray(rcodes, dtype=np.uint8)),
+                                    _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
+                                    _ptr(out), _ptr(mask))
+    return out, mask

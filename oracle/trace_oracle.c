@@ -152,6 +152,27 @@ int oracle_guided_code(float a, int bit) {
   return (d_lo <= d_hi) ? lo : hi;
 }
 
+/* Full-information guidance (the upper bound the post's layer ablation
+ * compares the 1-bit cache against): the cache holds the whole rollout code,
+ * and q* is the argmin of the listing taken with the exact rollout codeword:
+ * of the two codewords bracketing z (one when z is a codeword), the one
+ * nearest to q_roll.  z: the unclipped scaled value; roll_code: sign<<3 |
+ * magnitude.  Returns the magnitude code of q*; its sign is that of z (both
+ * bracket members lie on z's side of zero).  No tie is possible: q_roll is a
+ * codeword, so it is either a bracket member or strictly nearer one end. */
+int oracle_full_guided_code(float z, int roll_code) {
+  float a = fabsf(z);
+  if (a > 6.0f) a = 6.0f;
+  int lo, hi;
+  oracle_e2m1_bracket(a, &lo, &hi);
+  /* the bracket of z on the signed grid */
+  const float s = signbit(z) ? -1.0f : 1.0f;
+  const float q_lo = s * kE2M1[lo], q_hi = s * kE2M1[hi];
+  const float q_roll = ((roll_code & 8) ? -1.0f : 1.0f) * kE2M1[roll_code & 7];
+  const float d_lo = fabsf(q_lo - q_roll), d_hi = fabsf(q_hi - q_roll);
+  return (d_hi < d_lo) ? hi : lo;
+}
+
 /* Dequantised output for a signed code: bf16( (VAL[c] * sbv) * s_g ).
  * VAL[c] * sbv is exact (at most 2 x 4 significant bits), so the only
  * roundings are one fp32 multiply and the fp32 -> bf16 step. */
@@ -289,10 +310,13 @@ void oracle_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
  * vanilla QAT comparator).  mask: bit i set when |z_i| <= 6, z taken before
  * clipping (straight-through estimator support).  sites: optional signed
  * code per element. */
+enum { FQ_RTN = 0, FQ_GUIDED = 1, FQ_FULL = 2 };
+
 static void fake_quant(const uint16_t* x, int64_t rows, int64_t cols,
                        const float* row_gscale, const uint32_t* mbits,
-                       const uint8_t* scales, uint16_t* out, uint32_t* mask,
-                       uint8_t* sites, int guided) {
+                       const uint8_t* rcodes, const uint8_t* scales,
+                       uint16_t* out, uint32_t* mask, uint8_t* sites,
+                       int mode) {
   assert(cols % 32 == 0);
   int64_t n = rows * cols;
   if (mask) memset(mask, 0, (size_t)(n / 32) * sizeof(uint32_t));
@@ -308,8 +332,10 @@ static void fake_quant(const uint16_t* x, int64_t rows, int64_t cols,
       if (mask && a <= 6.0f) mask[i / 32] |= 1u << (i & 31);
       if (a > 6.0f) a = 6.0f;
       int c;
-      if (guided)
+      if (mode == FQ_GUIDED)
         c = oracle_guided_code(a, (int)((mbits[i / 32] >> (i & 31)) & 1u));
+      else if (mode == FQ_FULL)
+        c = oracle_full_guided_code(z, (rcodes[i / 2] >> (4 * (i & 1))) & 0xF);
       else
         c = oracle_e2m1_rtn(a);
       if (out) out[i] = oracle_dequant_bf16(c, signbit(z) != 0, sbv, s_g);
@@ -324,7 +350,8 @@ void oracle_fake_quant_rows(const uint16_t* x, int64_t rows, int64_t cols,
                             const float* row_gscale, const uint32_t* mbits,
                             const uint8_t* scales, uint16_t* out,
                             uint32_t* mask) {
-  fake_quant(x, rows, cols, row_gscale, mbits, scales, out, mask, 0, mbits != 0);
+  fake_quant(x, rows, cols, row_gscale, mbits, 0, scales, out, mask, 0,
+             mbits != 0 ? FQ_GUIDED : FQ_RTN);
 }
 
 /* Guided QAT forward on x_train with the rollout's cache (pseudocode:
@@ -335,7 +362,7 @@ void oracle_guided_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
                        uint16_t* out, uint32_t* mask) {
   check_offsets(rows, G, offs);
   float* rs = expand_row_scales(rows, G, offs, gscale);
-  fake_quant(x_train, rows, cols, rs, mbits, scales, out, mask, 0, 1);
+  fake_quant(x_train, rows, cols, rs, mbits, 0, scales, out, mask, 0, FQ_GUIDED);
   free(rs);
 }
 
@@ -345,7 +372,7 @@ void oracle_rtn_fwd(const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
                     const float* gscale, uint16_t* out, uint32_t* mask) {
   check_offsets(rows, G, offs);
   float* rs = expand_row_scales(rows, G, offs, gscale);
-  fake_quant(x, rows, cols, rs, 0, scales, out, mask, 0, 0);
+  fake_quant(x, rows, cols, rs, 0, 0, scales, out, mask, 0, FQ_RTN);
   free(rs);
 }
 
@@ -359,8 +386,40 @@ void oracle_fake_quant_codes(const uint16_t* x, int64_t rows, int64_t cols,
                              const float* gscale, uint8_t* sites) {
   check_offsets(rows, G, offs);
   float* rs = expand_row_scales(rows, G, offs, gscale);
-  fake_quant(x, rows, cols, rs, mbits, scales, 0, 0, sites, mbits != 0);
+  fake_quant(x, rows, cols, rs, mbits, 0, scales, 0, 0, sites,
+             mbits != 0 ? FQ_GUIDED : FQ_RTN);
   free(rs);
+}
+
+/* Full-information guided forward on x_train with the rollout's full codes
+ * (capture's `codes` output) and scales. */
+void oracle_full_guided_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                            int32_t G, const int64_t* offs, const uint8_t* rcodes,
+                            const uint8_t* scales, const float* gscale,
+                            uint16_t* out, uint32_t* mask) {
+  check_offsets(rows, G, offs);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  fake_quant(x_train, rows, cols, rs, 0, rcodes, scales, out, mask, 0, FQ_FULL);
+  free(rs);
+}
+
+/* Signed code picked at every site by full-information guidance. */
+void oracle_full_guided_codes(const uint16_t* x, int64_t rows, int64_t cols,
+                              int32_t G, const int64_t* offs,
+                              const uint8_t* rcodes, const uint8_t* scales,
+                              const float* gscale, uint8_t* sites) {
+  check_offsets(rows, G, offs);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  fake_quant(x, rows, cols, rs, 0, rcodes, scales, 0, 0, sites, FQ_FULL);
+  free(rs);
+}
+
+/* Full-information guided forward for rows with known global scales. */
+void oracle_full_guided_rows(const uint16_t* x, int64_t rows, int64_t cols,
+                             const float* row_gscale, const uint8_t* rcodes,
+                             const uint8_t* scales, uint16_t* out,
+                             uint32_t* mask) {
+  fake_quant(x, rows, cols, row_gscale, 0, rcodes, scales, out, mask, 0, FQ_FULL);
 }
 
 /* Masked straight-through estimator backward: the gradient passes where the

@@ -161,3 +161,12 @@ def brute_pipeline(x_roll: np.ndarray, x_train: np.ndarray, grad: np.ndarray):
                 gscale=np.array([s_g], np.float32), out_guided=out_g.reshape(rows, cols),
                 out_rtn=out_r.reshape(rows, cols), mask=mask,
                 grad_in=gin.reshape(rows, cols))
+
+
+def brute_full_guided(z: Fraction, roll_value: Fraction) -> tuple[Fraction, int]:
+    """Of the bracket around clip(z), the member nearest to the rollout
+    codeword value, by exhaustive comparison (no tie can occur)."""
+    lo, hi = brute_bracket(z)
+    dl, dh = abs(lo[0] - roll_value), abs(hi[0] - roll_value)
+    assert lo[0] == hi[0] or dl != dh
+    return hi if dh < dl else lo

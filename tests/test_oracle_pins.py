@@ -441,3 +441,86 @@ def test_ste_backward_definition(oracle_mod):
     gin = oracle_mod.fq_bwd(g, mask)
     keep = oracle_mod.unpack_bits(mask).astype(bool)
     assert np.array_equal(gin[keep], g[keep]) and np.all(gin[~keep] == 0)
+
+
+# --------------------------------------------------------------------------
+# Full-information guidance (the cache keeps the whole rollout code)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("sign", [1, -1])
+def test_full_guided_choice_vs_bruteforce(oracle_mod, sign):
+    rolls = [c for c in range(16)]
+    for a in _z_lattice():
+        z = sign * a
+        for rc in rolls:
+            rv = Fraction(E2M1[rc & 7]) * (-1 if rc & 8 else 1)
+            v, c = bf.brute_full_guided(Fraction(z), rv)
+            got = oracle_mod.full_guided_code(z, rc)
+            assert got == c and Fraction(E2M1[got]) == abs(v), (z, rc)
+
+
+def test_full_guidance_guarantee_holds_everywhere(oracle_mod):
+    """With the whole rollout code, |q* - q_roll| <= |RTN(z) - q_roll| at
+    every site (the per-site guarantee of rollout-guided rounding), also
+    where the training value has moved past the neighbouring codewords; it
+    agrees with 1-bit guidance wherever q_roll lies in the bracket."""
+    s = inputs.tiny_site(17, 96, 512, eps=0.25)     # large drift on purpose
+    xr, xt = inputs.bits(s.x_roll), inputs.bits(s.x_train)
+    codes, mbits, scales, gscale = oracle_mod.capture(xr)
+    q_roll = oracle_mod.unpack_codes(codes)
+    q_full = oracle_mod.full_guided_codes(xt, codes, scales, gscale).reshape(-1)
+    q_bit = oracle_mod.fake_quant_codes(xt, scales, gscale, mbits).reshape(-1)
+    q_rtn = oracle_mod.fake_quant_codes(xt, scales, gscale, None).reshape(-1)
+    vr, vf, vb, vn = (_signed_value(c) for c in (q_roll, q_full, q_bit, q_rtn))
+    assert np.all(np.abs(vf - vr) <= np.abs(vn - vr))
+    violated = np.abs(vb - vr) > np.abs(vn - vr)      # where 1 bit is not enough
+    assert violated.sum() > 0                         # the drift produces some
+    # q_roll lies in the bracket exactly where full guidance reproduces it;
+    # there the 1-bit choice reproduces it too
+    in_bracket = vf == vr
+    assert np.all(vb[in_bracket] == vr[in_bracket])
+    assert np.count_nonzero(vf != vr) <= np.count_nonzero(vb != vr)
+
+
+def test_full_guidance_equals_rollout_when_inputs_equal(oracle_mod):
+    s = inputs.single_activation(0, rows=32, cols=256)
+    xr = inputs.bits(s.x_roll)
+    codes, mbits, scales, gscale = oracle_mod.capture(xr)
+    q = oracle_mod.full_guided_codes(xr, codes, scales, gscale).reshape(-1)
+    assert np.array_equal(q, oracle_mod.unpack_codes(codes))
+    out_f, mask_f = oracle_mod.full_guided_fwd(xr, codes, scales, gscale)
+    out_r, mask_r = oracle_mod.rtn_fwd(xr, scales, gscale)
+    assert np.array_equal(out_f, out_r) and np.array_equal(mask_f, mask_r)
+
+
+def test_full_guided_pipeline_vs_bruteforce(oracle_mod):
+    """Whole full-information forward on tiny inputs against brute force:
+    exhaustive bracket and nearest-member search, numpy fp32, torch bf16."""
+    for xr, xt, g in _tiny_cases()[:5]:
+        ref = bf.brute_pipeline(xr, xt, g)
+        codes, mbits, scales, gscale = oracle_mod.capture(xr)
+        rows, cols = xr.shape
+        q_roll = oracle_mod.unpack_codes(codes)
+        out, mask = oracle_mod.full_guided_fwd(xt, codes, scales, gscale)
+        assert np.array_equal(mask, ref["mask"])
+        xtf = [bf.bf16_bits_to_float(int(h)) for h in xt.reshape(-1)]
+        s_g = np.float32(gscale[0])
+        expect = np.zeros(rows * cols, np.uint16)
+        for b in range(rows * cols // 16):
+            sbv = bf.e4m3_value(int(scales.reshape(-1)[b]))
+            d = s_g * np.float32(float(sbv))
+            for i in range(16 * b, 16 * b + 16):
+                if d == 0:
+                    z, neg = Fraction(0), bool(np.signbit(np.float32(xtf[i])))
+                else:
+                    zf = np.float32(xtf[i]) / d
+                    z, neg = Fraction(float(zf)), bool(np.signbit(zf))
+                rc = int(q_roll[i])
+                rv = Fraction(E2M1[rc & 7]) * (-1 if rc & 8 else 1)
+                v, _ = bf.brute_full_guided(z, rv)
+                exact = abs(v) * sbv * Fraction(float(s_g))
+                f = np.float32(float(exact))
+                if v < 0 or (v == 0 and neg):
+                    f = -f
+                expect[i] = bf.float_to_bf16_bits(f)
+        assert np.array_equal(out.reshape(-1), expect)
