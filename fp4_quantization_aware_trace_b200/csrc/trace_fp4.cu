@@ -342,9 +342,11 @@ __device__ __noinline__ void capture_block_exact(V8 v, float d, uint32_t* code_l
 }
 
 // Fake-quant of one block on the exact path: bf16 outputs and STE mask.
+// mode: 0 round-to-nearest, 1 1-bit guided (bits16), 2 full-information
+// guided (rollout codes c0: elements 0-7, c1: 8-15).
 __device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, float s_g,
-                                                    uint32_t bits16, bool guided, V8* out,
-                                                    uint32_t* mask16) {
+                                                    uint32_t bits16, uint32_t c0, uint32_t c1,
+                                                    int mode, V8* out, uint32_t* mask16) {
   uint32_t m = 0u;
   for (int k = 0; k < 8; ++k) out->w[k] = 0u;
   for (int j = 0; j < 16; ++j) {
@@ -352,9 +354,17 @@ __device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, fl
     const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
     const Exact e = exact_site(xf, d);
     int c = e.rtn;
-    if (guided) {
+    if (mode == 1) {
       const int bit = (int)((bits16 >> j) & 1u);
       c = e.exact ? e.floor : e.floor + ((e.floor ^ bit) & 1);
+    } else if (mode == 2) {
+      // nearest of floor / ceiling to the rollout value on z's side of zero
+      const uint32_t rc = ((j < 8 ? c0 : c1) >> (4 * (j & 7))) & 0xFu;
+      float q = e2m1_value((int)(rc & 7u));
+      const bool neg_roll = (rc & 8u) != 0u, neg_z = ((w >> ((j & 1) ? 31 : 15)) & 1u) != 0u;
+      if (neg_roll != neg_z) q = -q;
+      const int hi = e.exact ? e.floor : e.floor + 1;
+      c = (q > e2m1_value(e.floor)) ? hi : e.floor;
     }
     const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
         __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
@@ -592,17 +602,25 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
-// Kernel 3/5: fake-quant forward with given scales.  GUIDED: pick, of the
-// bracket around z, the member whose mantissa bit is the cached bit; else
-// round to nearest.  Writes bf16 q*·s and the STE mask.
+// Kernel 3/5: fake-quant forward with given scales: bf16 q*·s and the STE
+// mask, q* chosen by round-to-nearest, by the cached mantissa bit, or by the
+// whole rollout code.
 // ---------------------------------------------------------------------------
-template <bool GUIDED>
-__device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const BlkK& k,
+// Fake-quant modes: round to nearest (vanilla QAT), 1-bit guided (TRACE's
+// compact cache), full-information guided (the cache keeps the whole code).
+enum FqMode { kRtn = 0, kGuided = 1, kFull = 2 };
+
+// Two elements (one bf16x2 word w) of the fake-quant forward.  `side` carries
+// the guidance of the pair: MODE kGuided -- the cached bits of the two
+// elements in bits 0 and 1; kFull -- the rollout's two 4-bit codes (low
+// nibble first).  Mask bits go to positions pos, pos + 1 of m.
+template <int MODE>
+__device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const BlkK& k,
                                             uint32_t& m, int pos) {
   // signed x; only |z| is used below (sign of the output comes from w)
   const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
   float ql, qh;
-  if (GUIDED) {
+  if (MODE != kRtn) {
     // z * 2^64 (exact; +-inf/NaN only where |x|/d overflows)
     float zl, zh;
     upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
@@ -613,13 +631,31 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const Bl
     float lol, loh, hil, hih;
     upk(add_rm2(aa, MM), lol, loh);
     upk(add_rp2(aa, MM), hil, hih);
-    // of floor / ceiling, the one whose mantissa bit is the cached bit: the
-    // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
-    // bit of the floor sum is its codeword's mantissa bit
-    const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-    const float tl = __uint_as_float(lb + ((lb ^ bits2) & (__float_as_uint(hil) - lb)));
-    const float th = __uint_as_float(hb + ((hb ^ (bits2 >> 1)) & (__float_as_uint(hih) - hb)));
-    upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
+    if (MODE == kGuided) {
+      // of floor / ceiling, the one whose mantissa bit is the cached bit: the
+      // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
+      // bit of the floor sum is its codeword's mantissa bit
+      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+      const float tl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+      const float th = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+      upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
+    } else {
+      // of floor / ceiling, the one nearest the rollout codeword: the
+      // rollout value reflected to z's side of zero picks the ceiling
+      // exactly when it lies above the floor (no codeword lies between)
+      float fl, fh, cl, ch;
+      upk(sub2(pk(lol, loh), MM), fl, fh);
+      upk(sub2(pk(hil, hih), MM), cl, ch);
+      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
+      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+      upk(mul2(pk(rl, rh), pk(kXs, kXs)), rl, rh);
+      const float tl = rl > fl ? cl : fl;
+      const float th = rh > fh ? ch : fh;
+      upk(mul2(mul2(pk(tl, th), k.sbv2), k.sg2), ql, qh);
+    }
   } else {
     float zl, zh;
     upk(quot2(xx, k), zl, zh);
@@ -635,10 +671,12 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t bits2, const Bl
 }
 
 // One 16-element block of the fake-quant forward: bf16 outputs and 16 mask
-// bits (in the low half of the returned mask).
-template <bool GUIDED>
-__device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, float sbv,
-                                                 float s_g, V8& o, uint32_t& m) {
+// bits.  side: kGuided -- the block's 16 cached bits; kFull -- its 16
+// rollout codes (c0: elements 0-7, c1: 8-15).
+template <int MODE>
+__device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, uint32_t c0,
+                                                 uint32_t c1, float sbv, float s_g, V8& o,
+                                                 uint32_t& m) {
   const float d = __fmul_rn(s_g, sbv);
   m = 0u;
   if (d == 0.0f) {
@@ -646,23 +684,28 @@ __device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, f
 #pragma unroll
     for (int k = 0; k < 8; ++k) o.w[k] = v.w[k] & 0x80008000u;
     m = 0xFFFFu;
-  } else if (fast_scale(d, GUIDED ? kDMaxExactZ : kDMax)) {
-    const BlkK bk = make_blk(d, GUIDED ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
+  } else if (fast_scale(d, MODE != kRtn ? kDMaxExactZ : kDMax)) {
+    const BlkK bk = make_blk(d, MODE != kRtn ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) o.w[k] = fq_pair<GUIDED>(v.w[k], bits16 >> (2 * k), bk, m, 2 * k);
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits16 >> (2 * k)
+                          : MODE == kFull ? ((k < 4 ? c0 : c1) >> (8 * (k & 3))) : 0u;
+      o.w[k] = fq_pair<MODE>(v.w[k], side, bk, m, 2 * k);
+    }
   } else {
-    fake_quant_block_exact(v, d, sbv, s_g, bits16, GUIDED, &o, &m);
+    fake_quant_block_exact(v, d, sbv, s_g, bits16, c0, c1, MODE, &o, &m);
   }
 }
 
 // Each thread owns two adjacent blocks, so their mantissa bits, scales and
-// mask move as one 32-bit / 16-bit / 32-bit access.
-template <bool GUIDED>
+// mask move as one 32-bit / 16-bit / 32-bit access (the full codes as one
+// 16-byte access).
+template <int MODE>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-                 const uint32_t* __restrict__ mbits, const uint16_t* __restrict__ scales,
-                 const float* __restrict__ gscale, V8* __restrict__ out,
-                 uint32_t* __restrict__ mask) {
+                 const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
+                 const uint16_t* __restrict__ scales, const float* __restrict__ gscale,
+                 V8* __restrict__ out, uint32_t* __restrict__ mask) {
   pdl_begin();
   GroupCursor gc;
   gc.init(offs, sh.G);
@@ -672,16 +715,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
     if (b >= sh.nblk) continue;
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const uint32_t bits = GUIDED ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t sb2 = __ldcs(scales + (b >> 1));
     if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
     V8 o;
     uint32_t m0, m1;
-    fake_quant_block<GUIDED>(v0, bits & 0xFFFFu, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
+    fake_quant_block<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
     st_block(out + b, o);
     // a row holds a whole number of 32-element words, so both blocks of the
     // pair are in the same row and group
-    fake_quant_block<GUIDED>(v1, bits >> 16, e4m3_to_f32(sb2 >> 8), s_g, o, m1);
+    fake_quant_block<MODE>(v1, bits >> 16, rc.z, rc.w, e4m3_to_f32(sb2 >> 8), s_g, o, m1);
     st_block(out + b + 1, o);
     mask[b >> 1] = m0 | (m1 << 16);
   }
@@ -849,15 +893,19 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_gro
                 (uint32_t*)mbits, (uint16_t*)scales, gscale);
 }
 
-static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
-                             const int64_t* offs, const uint32_t* mbits, const uint8_t* scales,
-                             const float* gscale, uint16_t* out, uint32_t* mask, void* stream) {
+static int fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
+                             const int64_t* offs, const uint32_t* mbits, const uint8_t* rcodes,
+                             const uint8_t* scales, const float* gscale, uint16_t* out,
+                             uint32_t* mask, void* stream) {
   int st = check_shape(rows, cols, G, offs);
   if (st) return st;
   if (rows == 0) return TRACE_OK;  // nothing to do; empty tensors may have NULL data
-  if (!x || (guided && !mbits) || !scales || !gscale || !out || !mask) return TRACE_ERR_NULL;
-  if (!aligned(x, 32) || (guided && !aligned(mbits, 16)) || !aligned(scales, 16) ||
-      !aligned(gscale, 4) || !aligned(out, 32) || !aligned(mask, 16))
+  if (!x || (mode == kGuided && !mbits) || (mode == kFull && !rcodes) || !scales || !gscale ||
+      !out || !mask)
+    return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || (mode == kGuided && !aligned(mbits, 16)) ||
+      (mode == kFull && !aligned(rcodes, 16)) || !aligned(scales, 16) || !aligned(gscale, 4) ||
+      !aligned(out, 32) || !aligned(mask, 16))
     return TRACE_ERR_ALIGN;
   const Shape sh = make_shape(rows, cols, G);
   if (sh.nblk == 0) return TRACE_OK;
@@ -865,26 +913,37 @@ static int fake_quant_launch(bool guided, const uint16_t* x, int64_t rows, int64
   if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* o = G > 1 ? offs : nullptr;
-  if (guided)
-    return launch(k_fake_quant<true>, grid, s, (const V8*)x, sh, o, (const uint32_t*)mbits,
-                  (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
-  return launch(k_fake_quant<false>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
-                (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
+  if (mode == kGuided)
+    return launch(k_fake_quant<kGuided>, grid, s, (const V8*)x, sh, o, (const uint32_t*)mbits,
+                  (const uint4*)nullptr, (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
+  if (mode == kFull)
+    return launch(k_fake_quant<kFull>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
+                  (const uint4*)rcodes, (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
+  return launch(k_fake_quant<kRtn>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
+                (const uint4*)nullptr, (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
 }
 
 int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols, int32_t num_groups,
                         const int64_t* group_row_offsets, const uint32_t* mbits,
                         const uint8_t* scales, const float* gscale, uint16_t* out,
                         uint32_t* ste_mask, void* stream) {
-  return fake_quant_launch(true, x_train, rows, cols, num_groups, group_row_offsets, mbits, scales,
-                           gscale, out, ste_mask, stream);
+  return fake_quant_launch(kGuided, x_train, rows, cols, num_groups, group_row_offsets, mbits,
+                           nullptr, scales, gscale, out, ste_mask, stream);
 }
 
 int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                      const int64_t* group_row_offsets, const uint8_t* scales, const float* gscale,
                      uint16_t* out, uint32_t* ste_mask, void* stream) {
-  return fake_quant_launch(false, x, rows, cols, num_groups, group_row_offsets, nullptr, scales,
-                           gscale, out, ste_mask, stream);
+  return fake_quant_launch(kRtn, x, rows, cols, num_groups, group_row_offsets, nullptr, nullptr,
+                           scales, gscale, out, ste_mask, stream);
+}
+
+int trace_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                             int32_t num_groups, const int64_t* group_row_offsets,
+                             const uint8_t* codes, const uint8_t* scales, const float* gscale,
+                             uint16_t* out, uint32_t* ste_mask, void* stream) {
+  return fake_quant_launch(kFull, x_train, rows, cols, num_groups, group_row_offsets, nullptr,
+                           codes, scales, gscale, out, ste_mask, stream);
 }
 
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,

@@ -58,6 +58,8 @@ def library() -> ctypes.CDLL:
         lib.trace_rtn_fq_fwd.restype = ctypes.c_int
         lib.trace_copy_bf16.argtypes = [P, P, i64, P]
         lib.trace_copy_bf16.restype = ctypes.c_int
+        lib.trace_full_guided_fq_fwd.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, P]
+        lib.trace_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_capture_static_ws.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
         lib.trace_capture_static_ws.restype = ctypes.c_int
         _lib = lib
@@ -114,6 +116,14 @@ def trace_guided_fq_fwd(x_train, rows, cols, num_groups, offsets, mbits, scales,
     _check(library().trace_guided_fq_fwd(_p(x_train), rows, cols, num_groups, _p(offsets),
                                          _p(mbits), _p(scales), _p(gscale), _p(out),
                                          _p(ste_mask), _stream(stream)), "trace_guided_fq_fwd")
+
+
+def trace_full_guided_fq_fwd(x_train, rows, cols, num_groups, offsets, codes, scales, gscale,
+                             out, ste_mask, stream=None) -> None:
+    _check(library().trace_full_guided_fq_fwd(_p(x_train), rows, cols, num_groups, _p(offsets),
+                                              _p(codes), _p(scales), _p(gscale), _p(out),
+                                              _p(ste_mask), _stream(stream)),
+           "trace_full_guided_fq_fwd")
 
 
 def trace_fq_bwd(grad_out, ste_mask, numel, grad_in, stream=None) -> None:
@@ -206,6 +216,18 @@ def guided_fq_fwd(x_train: torch.Tensor, cache: Capture, out: torch.Tensor | Non
     mask = torch.empty(rows * cols // 32, dtype=torch.int32, device=x_train.device) if mask is None else mask
     trace_guided_fq_fwd(x_train, rows, cols, _groups(cache.offsets), cache.offsets, cache.mbits,
                         cache.scales, cache.gscale, out, mask, stream)
+    return out, mask
+
+
+def full_guided_fq_fwd(x_train: torch.Tensor, cache: Capture, out: torch.Tensor | None = None,
+                       mask: torch.Tensor | None = None, stream=None):
+    """Full-information guided forward (the cache keeps the rollout's whole
+    codes).  Returns (out, mask)."""
+    rows, cols = _bf16_2d(x_train)
+    out = torch.empty_like(x_train) if out is None else out
+    mask = torch.empty(rows * cols // 32, dtype=torch.int32, device=x_train.device) if mask is None else mask
+    trace_full_guided_fq_fwd(x_train, rows, cols, _groups(cache.offsets), cache.offsets, cache.codes,
+                             cache.scales, cache.gscale, out, mask, stream)
     return out, mask
 
 

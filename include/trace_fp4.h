@@ -121,6 +121,24 @@ int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
                         const float* gscale, uint16_t* out, uint32_t* ste_mask,
                         void* stream);
 
+/* Full-information guided fake-quant forward: the upper bound the post's
+ * ablation compares the 1-bit cache against ("keeping only 1 mantissa bit ...
+ * is close to full-information guidance", results list).  The cache keeps
+ * the rollout's whole 4-bit code, and q* is the listing's argmin taken with
+ * the exact rollout codeword: of the two codewords bracketing z (one if z is
+ * a codeword), the one nearest q_roll.  This makes the per-site guarantee of
+ * the rollout-guided-rounding paragraph exact: |q* - q_roll| <=
+ * |RTN(z) - q_roll| everywhere.  As trace_guided_fq_fwd, except:
+ *   codes: the rollout's packed 4-bit codes (capture's `codes` output),
+ *          uint8[N/2], 16-byte aligned (read 0.5 byte per element instead of
+ *          0.125 for the bits). */
+int trace_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows,
+                             int64_t cols, int32_t num_groups,
+                             const int64_t* group_row_offsets,
+                             const uint8_t* codes, const uint8_t* scales,
+                             const float* gscale, uint16_t* out,
+                             uint32_t* ste_mask, void* stream);
+
 /* Masked straight-through-estimator backward:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
  *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.

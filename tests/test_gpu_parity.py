@@ -60,10 +60,11 @@ def run_gpu(site: inputs.Site):
     out, mask = ops.guided_fq_fwd(xt, cap)
     gin = ops.fq_bwd(g, mask)
     out_r, mask_r = ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, offs)
+    out_f, mask_f = ops.full_guided_fq_fwd(xt, cap)
     torch.cuda.synchronize()
     return dict(codes=_u(cap.codes), mbits=_u(cap.mbits), scales=_u(cap.scales),
                 gscale=_u(cap.gscale), out=_u(out), mask=_u(mask), grad_in=_u(gin),
-                out_rtn=_u(out_r), mask_rtn=_u(mask_r))
+                out_rtn=_u(out_r), mask_rtn=_u(mask_r), out_full=_u(out_f), mask_full=_u(mask_f))
 
 
 def run_oracle(oracle_mod, site: inputs.Site):
@@ -72,9 +73,10 @@ def run_oracle(oracle_mod, site: inputs.Site):
     codes, mbits, scales, gscale = oracle_mod.capture(xr, G, offs)
     out, mask = oracle_mod.guided_fwd(xt, mbits, scales, gscale, G, offs)
     out_r, mask_r = oracle_mod.rtn_fwd(xt, scales, gscale, G, offs)
+    out_f, mask_f = oracle_mod.full_guided_fwd(xt, codes, scales, gscale, G, offs)
     gin = oracle_mod.fq_bwd(g, mask)
     return dict(codes=codes, mbits=mbits, scales=scales, gscale=gscale, out=out, mask=mask,
-                grad_in=gin, out_rtn=out_r, mask_rtn=mask_r)
+                grad_in=gin, out_rtn=out_r, mask_rtn=mask_r, out_full=out_f, mask_full=mask_f)
 
 
 def check_full(oracle_mod, site):
@@ -101,6 +103,7 @@ def check_sampled_rows(oracle_mod, site, rows_idx):
     codes, mbits, scales = oracle_mod.capture_rows(xr[rows_idx], rg)
     out, mask = oracle_mod.fake_quant_rows(xt[rows_idx], rg, scales, mbits)
     out_r, mask_r = oracle_mod.fake_quant_rows(xt[rows_idx], rg, scales, None)
+    out_f, mask_f = oracle_mod.full_guided_rows(xt[rows_idx], rg, scales, codes)
     gin = oracle_mod.fq_bwd(np.ascontiguousarray(g[rows_idx]), mask)
     _eq(f"{site.name}.codes", got["codes"].reshape(R, C // 2)[rows_idx], codes)
     _eq(f"{site.name}.mbits", got["mbits"].reshape(R, C // 32)[rows_idx], mbits)
@@ -110,6 +113,8 @@ def check_sampled_rows(oracle_mod, site, rows_idx):
     _eq(f"{site.name}.out_rtn", got["out_rtn"].reshape(R, C)[rows_idx], out_r)
     _eq(f"{site.name}.mask_rtn", got["mask_rtn"].reshape(R, C // 32)[rows_idx], mask_r)
     _eq(f"{site.name}.grad_in", got["grad_in"].reshape(R, C)[rows_idx], gin)
+    _eq(f"{site.name}.out_full", got["out_full"].reshape(R, C)[rows_idx], out_f)
+    _eq(f"{site.name}.mask_full", got["mask_full"].reshape(R, C // 32)[rows_idx], mask_f)
 
 
 def _sample_rows(R, k=96, seed=0):
@@ -242,6 +247,34 @@ def test_exhaustive_bf16_fake_quant(oracle_mod, bit):
     ref_r, ref_rm = oracle_mod.rtn_fwd(x, scales, gs_vals, G, offs)
     _eq("rtn_out", _u(out_r), ref_r)
     _eq("rtn_mask", _u(mask_r), ref_rm)
+
+
+def test_exhaustive_bf16_full_guided(oracle_mod):
+    """Full-information guidance: every finite bf16 pattern against every
+    signed rollout code (cycled across the slabs), every E4M3 block scale and
+    the same global scales as the bit-guided sweep."""
+    pats = _all_finite_bf16()
+    gs_vals = np.array([1.0, 0.3712345, 2.0 ** -140, 1.9e30, 2.0 ** 9, 911.0], np.float32)
+    sbytes = np.arange(0x7F, dtype=np.uint8)
+    slab = pats.shape[0]
+    x = np.tile(pats, (len(sbytes) * len(gs_vals), 1))
+    R, C = x.shape
+    scales = np.repeat(np.tile(np.repeat(sbytes, slab), len(gs_vals)), C // 16).reshape(R, C // 16)
+    offs = np.arange(0, R + 1, slab * len(sbytes), dtype=np.int64)
+    G = len(gs_vals)
+    idx = np.arange(R * C, dtype=np.int64)
+    nib = ((idx + idx // (slab * C)) % 16).astype(np.uint8)
+    rcodes = (nib[0::2] | (nib[1::2] << 4)).astype(np.uint8)
+    xd = inputs.from_bits(x, DEV)
+    cache = ops.Capture(codes=torch.from_numpy(rcodes).to(DEV), mbits=None,
+                        scales=torch.from_numpy(scales).to(DEV),
+                        gscale=torch.from_numpy(gs_vals).to(DEV),
+                        offsets=torch.from_numpy(offs).to(DEV))
+    out, mask = ops.full_guided_fq_fwd(xd, cache)
+    torch.cuda.synchronize()
+    ref, ref_m = oracle_mod.full_guided_fwd(x, rcodes, scales, gs_vals, G, offs)
+    _eq("full_out", _u(out), ref)
+    _eq("full_mask", _u(mask), ref_m)
 
 
 def test_exhaustive_bf16_capture(oracle_mod):
