@@ -369,6 +369,19 @@ def run_trace(args):
         step(kern_ev[k])
     torch.cuda.synchronize()
 
+    # the next row built beyond the step: full-information guidance (the
+    # cache keeps the rollout's whole codes), timed alone the same way
+    full_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in work] for _ in range(args.steps)]
+    for k in range(args.steps):
+        flush.fill_((k + 13) & 0xFF)
+        for i, w in enumerate(work):
+            full_ev[k][i][0].record(stream)
+            ops.full_guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], stream)
+            full_ev[k][i][1].record(stream)
+    torch.cuda.synchronize()
+    full_ms = max_over_ranks([sum(a.elapsed_time(b) for per in full_ev for a, b in per)], pg, dev)[0]
+
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
     per_kernel = {nm: 0.0 for nm in names}
     total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
@@ -392,6 +405,12 @@ def run_trace(args):
                     "gbs": round(n * BYTES_PER_ELEM[nm] / (ms * 1e-3) / 1e9, 1),
                     "elem_per_s": round(n / (ms * 1e-3), 1)}
         kern[nm]["frac_of_hbm"] = round(kern[nm]["gbs"] / hbm, 4)
+    fms = full_ms / args.steps
+    next_rows = {"full_guided_fwd": {
+        "kernel": "k_fake_quant<kFull>", "us": round(fms * 1e3, 2),
+        "gbs": round(n * 4.6875 / (fms * 1e-3) / 1e9, 1),
+        "frac_of_hbm": round(n * 4.6875 / (fms * 1e-3) / 1e9 / hbm, 4),
+        "bytes_per_elem": 4.6875}}
     # dominant kernel: the guided forward (the largest single launch of the
     # step), timed inside the timed steps
     dom = "guided_fwd"
@@ -476,6 +495,7 @@ def run_trace(args):
                    "parallelism": f"{world} independent sites, one per GPU (no collective)"},
         "kernels": kern,
         "yardstick": yardstick,
+        "next_rows": next_rows,
         "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
                      "us_per_launch": round(dom_us, 2),
                      "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
