@@ -98,6 +98,8 @@ def _load():
         lib.oracle_full_guided_codes.restype = None
         lib.oracle_full_guided_rows.argtypes = [P, i64, i64, P, P, P, P, P]
         lib.oracle_full_guided_rows.restype = None
+        lib.oracle_mismatch_histogram.argtypes = [P, i64, i64, i32, P, P, P, P, P]
+        lib.oracle_mismatch_histogram.restype = None
         _lib = lib
         return lib
 
@@ -355,3 +357,21 @@ def full_guided_rows(x, row_gscale, scales, rcodes):
                                     _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
                                     _ptr(out), _ptr(mask))
     return out, mask
+
+
+# -- mismatch diagnostic ------------------------------------------------------
+
+def mismatch_histogram(x_train, rcodes, scales, gscale, num_groups: int = 1, offsets=None):
+    """uint64[3, 15]: ladder distance from the rollout code of the training
+    side's RTN (row 0), 1-bit guided (row 1) and full-information guided
+    (row 2) codes."""
+    x = _as_bf16_bits(x_train)
+    rows, cols = x.shape
+    o = _offsets(offsets, num_groups, rows)
+    hist = np.zeros(45, np.uint64)
+    _load().oracle_mismatch_histogram(_ptr(x), rows, cols, num_groups, _ptr(o),
+                                      _ptr(np.ascontiguousarray(rcodes, dtype=np.uint8)),
+                                      _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
+                                      _ptr(np.ascontiguousarray(gscale, dtype=np.float32)),
+                                      _ptr(hist))
+    return hist.reshape(3, 15)

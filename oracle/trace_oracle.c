@@ -422,6 +422,51 @@ void oracle_full_guided_rows(const uint16_t* x, int64_t rows, int64_t cols,
   fake_quant(x, rows, cols, row_gscale, 0, rcodes, scales, out, mask, 0, FQ_FULL);
 }
 
+/* Position of a signed code on the signed E2M1 ladder: -7..7 (+0 and -0
+ * are one point). */
+static int ladder(int code) {
+  const int mag = code & 7;
+  return (code & 8) ? -mag : mag;
+}
+
+/* Mismatch diagnostic (the compact-cache paragraph: most sites where the two
+ * paths disagree differ by one adjacent codebook entry).  For every element
+ * of x_train, with the rollout's scales, three training-side codes are
+ * compared with the rollout's code q_roll (capture's `codes`): round to
+ * nearest, 1-bit guided (the bit is q_roll's mantissa bit), and
+ * full-information guided.  hist[k*15 + d] counts the elements whose code k
+ * (0 RTN, 1 guided, 2 full) sits d ladder steps from q_roll.  The counts are
+ * added to hist. */
+void oracle_mismatch_histogram(const uint16_t* x, int64_t rows, int64_t cols,
+                               int32_t G, const int64_t* offs,
+                               const uint8_t* rcodes, const uint8_t* scales,
+                               const float* gscale, uint64_t* hist) {
+  assert(cols % 32 == 0);
+  check_offsets(rows, G, offs);
+  float* rs = expand_row_scales(rows, G, offs, gscale);
+  const int64_t n = rows * cols;
+  for (int64_t b = 0; b < n / 16; ++b) {
+    const float s_g = rs[(b * 16) / cols];
+    const float sbv = oracle_e4m3_to_f32(scales[b]);
+    for (int j = 0; j < 16; ++j) {
+      const int64_t i = b * 16 + j;
+      const float z = scaled_z(oracle_bf16_to_f32(x[i]), s_g, sbv);
+      float a = fabsf(z);
+      if (a > 6.0f) a = 6.0f;
+      const int rc = (rcodes[i / 2] >> (4 * (i & 1))) & 0xF;
+      const int sz = signbit(z) ? 8 : 0;
+      const int c_rtn = sz | oracle_e2m1_rtn(a);
+      const int c_gd = sz | oracle_guided_code(a, rc & 1);
+      const int c_full = sz | oracle_full_guided_code(z, rc);
+      const int lr = ladder(rc);
+      hist[0 * 15 + abs(ladder(c_rtn) - lr)] += 1;
+      hist[1 * 15 + abs(ladder(c_gd) - lr)] += 1;
+      hist[2 * 15 + abs(ladder(c_full) - lr)] += 1;
+    }
+  }
+  free(rs);
+}
+
 /* Masked straight-through estimator backward: the gradient passes where the
  * mask bit is set and is +0.0 elsewhere. */
 void oracle_fq_bwd(const uint16_t* grad_out, const uint32_t* mask, int64_t n,

@@ -524,3 +524,61 @@ def test_full_guided_pipeline_vs_bruteforce(oracle_mod):
                     f = -f
                 expect[i] = bf.float_to_bf16_bits(f)
         assert np.array_equal(out.reshape(-1), expect)
+
+
+# --------------------------------------------------------------------------
+# Mismatch diagnostic (compact-cache paragraph: mismatched sites are mostly
+# one adjacent codeword apart)
+# --------------------------------------------------------------------------
+
+def _ladder(c):
+    c = np.asarray(c, np.int64)
+    return np.where(c & 8, -(c & 7), c & 7)
+
+
+def test_mismatch_histogram_vs_codes(oracle_mod):
+    """The histogram counts the ladder distances of the per-site codes the
+    other oracle entry points pick (and brute force on a tiny input)."""
+    s = inputs.tiny_site(23, 64, 256, eps=0.05)
+    xr, xt = inputs.bits(s.x_roll), inputs.bits(s.x_train)
+    codes, mbits, scales, gscale = oracle_mod.capture(xr)
+    hist = oracle_mod.mismatch_histogram(xt, codes, scales, gscale)
+    q_roll = oracle_mod.unpack_codes(codes)
+    q = [oracle_mod.fake_quant_codes(xt, scales, gscale, None).reshape(-1),
+         oracle_mod.fake_quant_codes(xt, scales, gscale, mbits).reshape(-1),
+         oracle_mod.full_guided_codes(xt, codes, scales, gscale).reshape(-1)]
+    for k in range(3):
+        d = np.abs(_ladder(q[k]) - _ladder(q_roll))
+        assert np.array_equal(hist[k], np.bincount(d, minlength=15))
+    assert np.all(hist.sum(axis=1) == xr.size)
+    # brute force on the special tiny case
+    xr2, xt2, g2 = _special_tiny()
+    ref = bf.brute_pipeline(xr2, xt2, g2)
+    c2, m2, sc2, gs2 = oracle_mod.capture(xr2)
+    h2 = oracle_mod.mismatch_histogram(xt2, c2, sc2, gs2)
+    out_g = torch.from_numpy(ref["out_guided"].view(np.int16)).view(torch.bfloat16).float().numpy().reshape(-1)
+    out_r = torch.from_numpy(ref["out_rtn"].view(np.int16)).view(torch.bfloat16).float().numpy().reshape(-1)
+    qr = oracle_mod.unpack_codes(c2)
+    sbv = np.repeat([float(bf.e4m3_value(int(b))) for b in sc2.reshape(-1)], 16)
+    d = sbv * float(gs2[0])
+    lr = _ladder(qr)
+    grid = np.array(E2M1)
+    for k, o in ((0, out_r), (1, out_g)):
+        mag = np.where(d > 0, np.abs(o) / np.where(d > 0, d, 1), 0)
+        code = np.array([int(np.argmin(np.abs(grid - m))) for m in mag])
+        lad = np.where(np.signbit(o), -code, code)
+        assert np.array_equal(h2[k], np.bincount(np.abs(lad - lr), minlength=15))
+
+
+def test_mismatch_dominance_and_identity(oracle_mod):
+    """Full guidance is at least as close as RTN at every site, so its
+    cumulative histogram dominates; identical inputs give all-zero
+    distances."""
+    s = inputs.tiny_site(29, 64, 512, eps=0.2)
+    xr, xt = inputs.bits(s.x_roll), inputs.bits(s.x_train)
+    codes, mbits, scales, gscale = oracle_mod.capture(xr)
+    h = oracle_mod.mismatch_histogram(xt, codes, scales, gscale).astype(np.int64)
+    assert np.all(np.cumsum(h[2]) >= np.cumsum(h[0]))
+    assert h[0, 1:].sum() > h[2, 1:].sum()
+    h0 = oracle_mod.mismatch_histogram(xr, codes, scales, gscale)
+    assert np.all(h0[:, 0] == xr.size) and np.all(h0[:, 1:] == 0)
