@@ -62,6 +62,8 @@ def library() -> ctypes.CDLL:
         lib.trace_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_capture_static_ws.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
         lib.trace_capture_static_ws.restype = ctypes.c_int
+        lib.trace_mismatch_histogram.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
+        lib.trace_mismatch_histogram.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -149,6 +151,13 @@ def trace_capture_static_ws(x, rows, cols, num_groups, offsets, codes, mbits, sc
 
 
 TRACE_STATIC_MAX_GROUPS = 4096
+
+
+def trace_mismatch_histogram(x_train, rows, cols, num_groups, offsets, codes, scales, gscale,
+                             hist, stream=None) -> None:
+    _check(library().trace_mismatch_histogram(_p(x_train), rows, cols, num_groups, _p(offsets),
+                                              _p(codes), _p(scales), _p(gscale), _p(hist),
+                                              _stream(stream)), "trace_mismatch_histogram")
 
 
 def trace_copy_bf16(src, dst, numel, stream=None) -> None:
@@ -250,6 +259,25 @@ def fq_bwd(grad_out: torch.Tensor, mask: torch.Tensor, out: torch.Tensor | None 
     out = torch.empty_like(grad_out) if out is None else out
     trace_fq_bwd(grad_out, mask, grad_out.numel(), out, stream)
     return out
+
+
+MISMATCH_RULES = ("rtn", "guided_1bit", "full_guided")
+MISMATCH_BINS = 15
+
+
+def mismatch_histogram(x_train: torch.Tensor, cache: Capture, hist: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """Add the ladder-distance counts of x_train against the rollout cache
+    into hist (int64 [3, 15], the uint64 counts' bits; zeros if None).  Row k
+    is the rule MISMATCH_RULES[k]; column d counts the elements d codewords
+    from the rollout's code."""
+    rows, cols = _bf16_2d(x_train)
+    if hist is None:
+        hist = torch.zeros(len(MISMATCH_RULES), MISMATCH_BINS, dtype=torch.int64,
+                           device=x_train.device)
+    trace_mismatch_histogram(x_train, rows, cols, _groups(cache.offsets), cache.offsets,
+                             cache.codes, cache.scales, cache.gscale, hist, stream)
+    return hist
 
 
 class GuidedFakeQuant(torch.autograd.Function):

@@ -139,6 +139,33 @@ int trace_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows,
                              const float* gscale, uint16_t* out,
                              uint32_t* ste_mask, void* stream);
 
+/* Mismatch diagnostic: how far the training side's FP4 codes land from the
+ * rollout's (the compact-cache paragraph reports that nearly all sites where
+ * the two sides disagree differ by one adjacent codebook entry).  For every
+ * element, z is formed from x_train with the ROLLOUT's scales, and three
+ * codes are taken: round to nearest (as trace_rtn_fq_fwd), 1-bit guided (as
+ * trace_guided_fq_fwd, with the mantissa bit of the rollout's code) and
+ * full-information guided (as trace_full_guided_fq_fwd).  Each code's
+ * distance to the rollout's code q_roll is counted on the signed E2M1 ladder
+ * -6, -4, ..., -0.5, 0, 0.5, ..., 6 (15 points; +0 and -0 are one point), so
+ * distances are 0..14:
+ *   hist[k*15 + d] += number of elements whose rule-k code lies d ladder
+ *   steps from q_roll; k = 0 round to nearest, 1 1-bit guided, 2 full.
+ * The counts are ADDED to hist (zero it first; summing several sites into
+ * one histogram is allowed).  Row k = 2, bin 0 counts the sites where q_roll
+ * is in the bracket of z_train; all other sites have q_roll outside it.
+ *   x_train : bf16 [rows, cols], 32-byte aligned.
+ *   codes, scales, gscale: the rollout's capture outputs (codes uint8[N/2],
+ *             16-byte aligned).
+ *   hist    : in/out, uint64[45], 8-byte aligned; NULL is an error even when
+ *             rows == 0 (then nothing is added). */
+int trace_mismatch_histogram(const uint16_t* x_train, int64_t rows,
+                             int64_t cols, int32_t num_groups,
+                             const int64_t* group_row_offsets,
+                             const uint8_t* codes, const uint8_t* scales,
+                             const float* gscale, uint64_t* hist,
+                             void* stream);
+
 /* Masked straight-through-estimator backward:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
  *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.
