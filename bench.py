@@ -47,8 +47,8 @@ METRIC = "capture & guided fake-quant fwd GB/s (elem/s) and % of B200 HBM roofli
 ROWS, COLS = 16384, 2048
 WORKLOAD = "attn_in [16384 x 2048] bf16, Qwen3-30B-A3B-shaped attention-input site"
 BYTES_PER_ELEM = {"capture": 4.6875, "guided_fwd": 4.3125, "ste_bwd": 4.125, "rtn_fwd": 4.1875}
-KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<true>",
-                "ste_bwd": "k_ste_bwd", "rtn_fwd": "k_fake_quant<false>"}
+KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<1> (1-bit guided)",
+                "ste_bwd": "k_ste_bwd", "rtn_fwd": "k_fake_quant<0> (round to nearest)"}
 LAUNCHES_PER_STEP = 6  # zero + amax + capture, guided, bwd, rtn
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
@@ -402,6 +402,33 @@ def run_trace(args):
     hist_ms = max_over_ranks([sum(a.elapsed_time(b) for per in hist_ev for a, b in per)], pg, dev)[0]
     hist_counts = hist.cpu().tolist()
 
+    # the cache tier: every site's compact cache captured into one record and
+    # copied to pinned host memory on a copy stream while the compute stream
+    # goes on; timed from the first capture to the end of the last copy
+    from fp4_quantization_aware_trace_b200 import cache_tier
+    # one device record per site: a smaller ring throttles the captures to
+    # the copy engine (its back-pressure), which is not what is timed here
+    tier = cache_tier.CacheTier(num_layers=1, keep=1, device=dev, ring=len(work))
+    for i, w in enumerate(work):  # untimed: allocates records and host buffers
+        tier.capture(("site", i), 0, w["xr"], w["offs"], w["cap"].codes, stream)
+    torch.cuda.synchronize()
+    tier_ev = []
+    for k in range(args.steps):
+        flush.fill_((k + 41) & 0xFF)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record(stream)
+        for i, w in enumerate(work):
+            tier.capture(("site", i), 0, w["xr"], w["offs"], w["cap"].codes, stream)
+        ev[1].record(stream)
+        ev[2].record(tier.copy_stream)
+        tier_ev.append(ev)
+    torch.cuda.synchronize()
+    tier_compute_ms = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in tier_ev)], pg, dev)[0]
+    tier_total_ms = max_over_ranks([sum(e[0].elapsed_time(e[2]) for e in tier_ev)], pg, dev)[0]
+    rec_bytes = sum(cache_tier.RecordLayout.of(*w["xr"].shape, w["site"].num_groups).nbytes
+                    for w in work)
+    del tier
+
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
     per_kernel = {nm: 0.0 for nm in names}
     total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
@@ -442,6 +469,16 @@ def run_trace(args):
         "disagree_frac": [round(1.0 - r[0] / tot, 6) for r in hist_counts],
         "adjacent_frac_of_disagreements": [round(r[1] / max(1, tot - r[0]), 6) for r in hist_counts],
         "counts": hist_counts}
+    cms, tms = tier_compute_ms / args.steps, tier_total_ms / args.steps
+    next_rows["cache_tier"] = {
+        "what": "capture of every site into one compact record + one D2H copy per site to pinned "
+                "host memory on a copy stream",
+        "record_bytes_per_step": rec_bytes, "ring_slots": len(work),
+        "bits_per_elem": round(8 * rec_bytes / n, 4),
+        "capture_only_us": round(per_kernel["capture"] * 1e3 / args.steps, 2),
+        "compute_stream_us": round(cms * 1e3, 2),
+        "until_last_copy_us": round(tms * 1e3, 2),
+        "d2h_gbs": round(rec_bytes / (tms * 1e-3) / 1e9, 2)}
     # dominant kernel: the guided forward (the largest single launch of the
     # step), timed inside the timed steps
     dom = "guided_fwd"

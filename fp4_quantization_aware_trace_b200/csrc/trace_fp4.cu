@@ -1056,6 +1056,21 @@ size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols, int32_t num_gro
   return ((size_t)num_groups * 4u + 255u) / 256u * 256u;
 }
 
+size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
+                                size_t* mbits_offset, size_t* scales_offset,
+                                size_t* gscale_offset) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0 || num_groups < 1) return 0;
+  const long double nl = (long double)rows * (long double)cols;
+  if (nl / 16 >= 4294967296.0L - (long double)kTileBlks) return 0;
+  const size_t n = (size_t)rows * (size_t)cols;
+  auto up16 = [](size_t v) { return (v + 15u) / 16u * 16u; };
+  const size_t om = 0, os = up16(n / 8), og = up16(os + n / 16);
+  if (mbits_offset) *mbits_offset = om;
+  if (scales_offset) *scales_offset = os;
+  if (gscale_offset) *gscale_offset = og;
+  return up16(og + 4u * (size_t)num_groups);
+}
+
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                   const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
                   uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,

@@ -64,6 +64,8 @@ def library() -> ctypes.CDLL:
         lib.trace_capture_static_ws.restype = ctypes.c_int
         lib.trace_mismatch_histogram.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
         lib.trace_mismatch_histogram.restype = ctypes.c_int
+        lib.trace_cache_record_bytes.argtypes = [i64, i64, i32, P, P, P]
+        lib.trace_cache_record_bytes.restype = sz
         _lib = lib
         return lib
 
@@ -104,6 +106,15 @@ def _groups(offsets: torch.Tensor | None) -> int:
 
 def trace_capture_workspace_bytes(rows: int, cols: int, num_groups: int) -> int:
     return int(library().trace_capture_workspace_bytes(rows, cols, num_groups))
+
+
+def trace_cache_record_bytes(rows: int, cols: int, num_groups: int) -> tuple[int, int, int, int]:
+    """(record bytes, mbits offset, scales offset, gscale offset); record
+    bytes is 0 for an invalid shape."""
+    om, os_, og = ctypes.c_size_t(0), ctypes.c_size_t(0), ctypes.c_size_t(0)
+    nb = library().trace_cache_record_bytes(rows, cols, num_groups, ctypes.byref(om),
+                                            ctypes.byref(os_), ctypes.byref(og))
+    return int(nb), om.value, os_.value, og.value
 
 
 def trace_capture(x, rows, cols, num_groups, offsets, codes, mbits, scales, gscale,

@@ -87,6 +87,22 @@ int trace_abi_version(void);
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols,
                                      int32_t num_groups);
 
+/* Layout of one site's compact-cache record: the mantissa bits, block
+ * scales and global scales of a capture in ONE contiguous buffer, so that a
+ * cache tier moves a site with a single copy each way (the post's "cache
+ * tier that holds" the per-site records, stack-and-caveats list).  Host
+ * function; touches no device.
+ *   Returns the record's size in bytes (a multiple of 16), or 0 for an
+ *   invalid shape (the rules of trace_capture).  Writes the byte offsets of
+ *   mbits (uint32[N/32]), scales (uint8[N/16]) and gscale (float[G]) inside
+ *   the record to the non-NULL out-pointers; each offset is a multiple of 16,
+ *   so a record whose base is 16-byte aligned satisfies every alignment the
+ *   calls below ask of these arrays.  Size: N/8 + N/16 + 4G bytes plus at
+ *   most 45 bytes of padding, i.e. 1.5 bits per element. */
+size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
+                                size_t* mbits_offset, size_t* scales_offset,
+                                size_t* gscale_offset);
+
 /* Rollout capture: fp4_quantize(x_rollout) plus low_bits(q_roll, 1) and the
  * scales (the capture half of the post's pseudocode listing; the compact
  * cache is mbits + scales + gscale, 1.5 bits per element).
