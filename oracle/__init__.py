@@ -100,6 +100,20 @@ def _load():
         lib.oracle_full_guided_rows.restype = None
         lib.oracle_mismatch_histogram.argtypes = [P, i64, i64, i32, P, P, P, P, P]
         lib.oracle_mismatch_histogram.restype = None
+        lib.oracle_e8m0_to_f32.argtypes = [ctypes.c_uint8]
+        lib.oracle_e8m0_to_f32.restype = ctypes.c_float
+        lib.oracle_mx_scale.argtypes = [ctypes.c_float]
+        lib.oracle_mx_scale.restype = ctypes.c_uint8
+        lib.oracle_mx_capture.argtypes = [P, i64, i64, P, P, P]
+        lib.oracle_mx_capture.restype = None
+        lib.oracle_mx_guided_fwd.argtypes = [P, i64, i64, P, P, P, P]
+        lib.oracle_mx_guided_fwd.restype = None
+        lib.oracle_mx_rtn_fwd.argtypes = [P, i64, i64, P, P, P]
+        lib.oracle_mx_rtn_fwd.restype = None
+        lib.oracle_mx_full_guided_fwd.argtypes = [P, i64, i64, P, P, P, P]
+        lib.oracle_mx_full_guided_fwd.restype = None
+        lib.oracle_mx_fake_quant_codes.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int]
+        lib.oracle_mx_fake_quant_codes.restype = None
         _lib = lib
         return lib
 
@@ -375,3 +389,67 @@ def mismatch_histogram(x_train, rcodes, scales, gscale, num_groups: int = 1, off
                                       _ptr(np.ascontiguousarray(gscale, dtype=np.float32)),
                                       _ptr(hist))
     return hist.reshape(3, 15)
+
+
+# -- MXFP4 variant ------------------------------------------------------------
+
+def e8m0_to_f32(b: int) -> float:
+    return float(_load().oracle_e8m0_to_f32(int(b)))
+
+
+def mx_scale(amax: float) -> int:
+    return int(_load().oracle_mx_scale(float(amax)))
+
+
+def mx_capture(x_roll):
+    """(codes uint8[N/2], mbits uint32[N/32], scales uint8[rows, cols/32])."""
+    x = _as_bf16_bits(x_roll)
+    rows, cols = x.shape
+    n = rows * cols
+    codes = np.zeros(n // 2, np.uint8)
+    mbits = np.zeros(n // 32, np.uint32)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    _load().oracle_mx_capture(_ptr(x), rows, cols, _ptr(codes), _ptr(mbits), _ptr(scales))
+    return codes, mbits, scales
+
+
+def _mx_fwd(fn, x, extra, scales):
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    out = np.zeros((rows, cols), np.uint16)
+    mask = np.zeros(rows * cols // 32, np.uint32)
+    args = [_ptr(x), rows, cols]
+    if extra is not None:
+        args.append(_ptr(extra))
+    args += [_ptr(np.ascontiguousarray(scales, dtype=np.uint8)), _ptr(out), _ptr(mask)]
+    fn(*args)
+    return out, mask
+
+
+def mx_guided_fwd(x_train, mbits, scales):
+    return _mx_fwd(_load().oracle_mx_guided_fwd, x_train,
+                   np.ascontiguousarray(mbits, dtype=np.uint32), scales)
+
+
+def mx_rtn_fwd(x, scales):
+    return _mx_fwd(_load().oracle_mx_rtn_fwd, x, None, scales)
+
+
+def mx_full_guided_fwd(x_train, rcodes, scales):
+    return _mx_fwd(_load().oracle_mx_full_guided_fwd, x_train,
+                   np.ascontiguousarray(rcodes, dtype=np.uint8), scales)
+
+
+def mx_fake_quant_codes(x, scales, mbits=None, rcodes=None):
+    """Signed code per element: RTN (both None), 1-bit guided (mbits) or
+    full-information guided (rcodes)."""
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    sites = np.zeros(rows * cols, np.uint8)
+    mode = 1 if mbits is not None else (2 if rcodes is not None else 0)
+    mb = None if mbits is None else np.ascontiguousarray(mbits, dtype=np.uint32)
+    rc = None if rcodes is None else np.ascontiguousarray(rcodes, dtype=np.uint8)
+    _load().oracle_mx_fake_quant_codes(_ptr(x), rows, cols, _ptr(mb), _ptr(rc),
+                                       _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
+                                       _ptr(sites), mode)
+    return sites.reshape(rows, cols)

@@ -21,6 +21,10 @@
  * format the post's rollout runs in; the pages name NVFP4 but do not spell
  * it out, so the readings taken here are listed at each step.
  *
+ * The MXFP4 variant at the end of the file (the post's results list: the
+ * method carries over to MXFP4 W4A4) swaps the scale step for the OCP
+ * Microscaling one; the rounding rules on the E2M1 grid are unchanged.
+ *
  * Every floating-point operation below is ONE IEEE-754 binary32 operation
  * with round-to-nearest-even.  Build with -ffp-contract=off and without
  * -ffast-math so that the compiler fuses nothing.
@@ -473,4 +477,124 @@ void oracle_fq_bwd(const uint16_t* grad_out, const uint32_t* mask, int64_t n,
                    uint16_t* grad_in) {
   for (int64_t i = 0; i < n; ++i)
     grad_in[i] = ((mask[i / 32] >> (i & 31)) & 1u) ? grad_out[i] : (uint16_t)0;
+}
+
+/* ------------------------------------------------------------------ */
+/* MXFP4 variant                                                        */
+/*                                                                      */
+/* The pages say only that the method carries over to MXFP4 and that    */
+/* MX scales are powers of two.  The format is the OCP Microscaling one: */
+/* 32-element blocks along a row, one E8M0 scale X = 2^e per block with  */
+/* e = floor(log2(max|x|)) - 2 (2 is the exponent of E2M1's largest      */
+/* value 6 = 1.5 * 2^2), clamped to E8M0's range [-127, 127]; an         */
+/* all-zero block takes e = -127; there is no per-tensor scale.  Then    */
+/* z = x / X, and clipping, rounding, the cached bit, the STE mask and   */
+/* dequantisation q * X are those of the NVFP4 path.                     */
+/* ------------------------------------------------------------------ */
+
+/* E8M0 byte -> 2^(b - 127) (exact; 2^-127 is an fp32 subnormal). */
+float oracle_e8m0_to_f32(uint8_t b) {
+  assert(b != 0xFF); /* the NaN encoding is never produced */
+  return ldexpf(1.0f, (int)b - 127);
+}
+
+/* E8M0 scale byte of a block whose largest magnitude is amax. */
+uint8_t oracle_mx_scale(float amax) {
+  int e = -127;
+  if (amax != 0.0f) {
+    int k;
+    (void)frexpf(amax, &k); /* amax = m * 2^k, m in [0.5, 1): floor(log2) = k-1 */
+    e = (k - 1) - 2;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+  }
+  return (uint8_t)(e + 127);
+}
+
+/* MX capture: codes, mantissa bits (layouts as oracle_capture_rows) and one
+ * E8M0 byte per 32 elements, row-major [rows, cols/32]. */
+void oracle_mx_capture(const uint16_t* x, int64_t rows, int64_t cols,
+                       uint8_t* codes, uint32_t* mbits, uint8_t* scales) {
+  assert(cols % 32 == 0);
+  const int64_t n = rows * cols;
+  memset(codes, 0, (size_t)(n / 2));
+  memset(mbits, 0, (size_t)(n / 32) * sizeof(uint32_t));
+  for (int64_t b = 0; b < n / 32; ++b) {
+    float bmax = 0.0f;
+    for (int j = 0; j < 32; ++j) {
+      const float a = fabsf(oracle_bf16_to_f32(x[b * 32 + j]));
+      if (a > bmax) bmax = a;
+    }
+    scales[b] = oracle_mx_scale(bmax);
+    const float X = oracle_e8m0_to_f32(scales[b]);
+    for (int j = 0; j < 32; ++j) {
+      const int64_t i = b * 32 + j;
+      const float z = oracle_bf16_to_f32(x[i]) / X;
+      float a = fabsf(z);
+      if (a > 6.0f) a = 6.0f;
+      const int c = oracle_e2m1_rtn(a);
+      codes[i / 2] |= (uint8_t)(((signbit(z) ? 8 : 0) | c) << (4 * (i & 1)));
+      mbits[i / 32] |= (uint32_t)(c & 1) << (i & 31);
+    }
+  }
+}
+
+/* MX fake-quant forward with given E8M0 scales; mode as fake_quant(). */
+static void mx_fake_quant(const uint16_t* x, int64_t rows, int64_t cols,
+                          const uint32_t* mbits, const uint8_t* rcodes,
+                          const uint8_t* scales, uint16_t* out, uint32_t* mask,
+                          uint8_t* sites, int mode) {
+  assert(cols % 32 == 0);
+  const int64_t n = rows * cols;
+  if (mask) memset(mask, 0, (size_t)(n / 32) * sizeof(uint32_t));
+  for (int64_t b = 0; b < n / 32; ++b) {
+    const float X = oracle_e8m0_to_f32(scales[b]);
+    for (int j = 0; j < 32; ++j) {
+      const int64_t i = b * 32 + j;
+      const float xv = oracle_bf16_to_f32(x[i]);
+      assert(isfinite(xv));
+      const float z = xv / X;
+      float a = fabsf(z);
+      if (mask && a <= 6.0f) mask[i / 32] |= 1u << (i & 31);
+      if (a > 6.0f) a = 6.0f;
+      int c;
+      if (mode == FQ_GUIDED)
+        c = oracle_guided_code(a, (int)((mbits[i / 32] >> (i & 31)) & 1u));
+      else if (mode == FQ_FULL)
+        c = oracle_full_guided_code(z, (rcodes[i / 2] >> (4 * (i & 1))) & 0xF);
+      else
+        c = oracle_e2m1_rtn(a);
+      if (out) {
+        float v = kE2M1[c] * X; /* exact: at most 2 significant bits */
+        if (signbit(z)) v = -v;
+        out[i] = oracle_f32_to_bf16(v);
+      }
+      if (sites) sites[i] = (uint8_t)((signbit(z) ? 8 : 0) | c);
+    }
+  }
+}
+
+void oracle_mx_guided_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                          const uint32_t* mbits, const uint8_t* scales,
+                          uint16_t* out, uint32_t* mask) {
+  mx_fake_quant(x_train, rows, cols, mbits, 0, scales, out, mask, 0, FQ_GUIDED);
+}
+
+void oracle_mx_rtn_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                       const uint8_t* scales, uint16_t* out, uint32_t* mask) {
+  mx_fake_quant(x, rows, cols, 0, 0, scales, out, mask, 0, FQ_RTN);
+}
+
+void oracle_mx_full_guided_fwd(const uint16_t* x_train, int64_t rows,
+                               int64_t cols, const uint8_t* rcodes,
+                               const uint8_t* scales, uint16_t* out,
+                               uint32_t* mask) {
+  mx_fake_quant(x_train, rows, cols, 0, rcodes, scales, out, mask, 0, FQ_FULL);
+}
+
+/* Per-element signed codes of an MX fake-quant (mode as fake_quant()). */
+void oracle_mx_fake_quant_codes(const uint16_t* x, int64_t rows, int64_t cols,
+                                const uint32_t* mbits, const uint8_t* rcodes,
+                                const uint8_t* scales, uint8_t* sites, int mode) {
+  mx_fake_quant(x, rows, cols, mbits, rcodes, scales, 0, 0, sites, mode);
 }

@@ -170,3 +170,71 @@ def brute_full_guided(z: Fraction, roll_value: Fraction) -> tuple[Fraction, int]
     dl, dh = abs(lo[0] - roll_value), abs(hi[0] - roll_value)
     assert lo[0] == hi[0] or dl != dh
     return hi if dh < dl else lo
+
+
+# ---------------------------------------------------------------------------
+# MXFP4 variant: 32-element blocks, E8M0 power-of-two scales, no global scale
+# ---------------------------------------------------------------------------
+
+def e8m0_value(byte: int) -> Fraction:
+    assert 0 <= byte <= 254
+    return Fraction(2) ** (byte - 127)
+
+
+def brute_mx_scale(amax: Fraction) -> int:
+    """The E8M0 byte whose value X puts amax / X in [4, 8) (the binade of
+    E2M1's largest value), by search over all bytes; the smallest byte when
+    amax is too small for any (or zero)."""
+    if amax == 0:
+        return 0
+    hits = [b for b in range(255) if 4 <= amax / e8m0_value(b) < 8]
+    assert len(hits) <= 1
+    return hits[0] if hits else 0
+
+
+def brute_mx_pipeline(x_roll: np.ndarray, x_train: np.ndarray):
+    """MX capture on x_roll, then 1-bit guided, round-to-nearest and full
+    guided fake-quant of x_train, by brute force (bf16 bit arrays)."""
+    rows, cols = x_roll.shape
+    n = rows * cols
+    xr = [bf16_bits_to_float(int(h)) for h in x_roll.reshape(-1)]
+    xt = [bf16_bits_to_float(int(h)) for h in x_train.reshape(-1)]
+    codes = np.zeros(n // 2, np.uint8)
+    mbits = np.zeros(n // 32, np.uint32)
+    scales = np.zeros(n // 32, np.uint8)
+    outs = {k: np.zeros(n, np.uint16) for k in ("out_guided", "out_rtn", "out_full")}
+    mask = np.zeros(n // 32, np.uint32)
+
+    def zval(x: float, X: np.float32):
+        z = f32(x) / X
+        return Fraction(float(z)), bool(np.signbit(z))
+
+    def deq(value: Fraction, neg: bool, X: Fraction) -> int:
+        v = f32(float(abs(value) * X))   # exact
+        if value < 0 or (value == 0 and neg):
+            v = -v
+        return float_to_bf16_bits(v)
+
+    for b in range(n // 32):
+        blk = range(32 * b, 32 * b + 32)
+        sb = brute_mx_scale(max(Fraction(abs(xr[i])) for i in blk))
+        scales[b] = sb
+        Xq = e8m0_value(sb)
+        X = f32(float(Xq))
+        for i in blk:
+            z, neg = zval(xr[i], X)
+            v, c = brute_rtn(z)
+            codes[i // 2] |= _signed_code(v, c, neg) << (4 * (i & 1))
+            mbits[i // 32] |= (c & 1) << (i & 31)
+        for i in blk:
+            z, neg = zval(xt[i], X)
+            if abs(z) <= 6:
+                mask[i // 32] |= 1 << (i & 31)
+            bit = (int(mbits[i // 32]) >> (i & 31)) & 1
+            rc = (int(codes[i // 2]) >> (4 * (i & 1))) & 0xF
+            rv = _MAGS[rc & 7] * (-1 if rc & 8 else 1)
+            outs["out_guided"][i] = deq(brute_guided(z, bit)[0], neg, Xq)
+            outs["out_rtn"][i] = deq(brute_rtn(z)[0], neg, Xq)
+            outs["out_full"][i] = deq(brute_full_guided(z, rv)[0], neg, Xq)
+    return dict(codes=codes, mbits=mbits, scales=scales.reshape(rows, cols // 32), mask=mask,
+                **{k: v.reshape(rows, cols) for k, v in outs.items()})

@@ -582,3 +582,83 @@ def test_mismatch_dominance_and_identity(oracle_mod):
     assert h[0, 1:].sum() > h[2, 1:].sum()
     h0 = oracle_mod.mismatch_histogram(xr, codes, scales, gscale)
     assert np.all(h0[:, 0] == xr.size) and np.all(h0[:, 1:] == 0)
+
+
+# --------------------------------------------------------------------------
+# MXFP4 variant (results list: the method carries over to MXFP4 W4A4; the
+# scale step is the OCP Microscaling one, the E2M1 rounding is unchanged)
+# --------------------------------------------------------------------------
+
+def test_e8m0_decode_vs_exact_and_torch(oracle_mod):
+    b = np.arange(255, dtype=np.uint8)
+    got = np.array([oracle_mod.e8m0_to_f32(int(v)) for v in b], np.float32)
+    exact = [bf.e8m0_value(int(v)) for v in b]
+    assert all(Fraction(float(g)) == e for g, e in zip(got, exact))
+    if hasattr(torch, "float8_e8m0fnu"):
+        t = torch.from_numpy(b).view(torch.float8_e8m0fnu).float().numpy()
+        assert np.array_equal(t.view(np.uint32), got.view(np.uint32))
+
+
+def test_mx_scale_vs_bruteforce(oracle_mod):
+    """Every bf16 magnitude pattern as a block maximum: the E8M0 byte puts
+    amax / X in [4, 8) (E2M1's top binade), clamped at 2^-127."""
+    pats = np.arange(0x7F80, dtype=np.uint32)
+    vals = (pats << 16).view(np.float32)
+    for a in vals[::7].tolist() + [0.0, 2.0 ** -133, 2.0 ** -125, 2.0 ** -124, 3.3e38, 8.0, 7.99, 4.0]:
+        a = float(np.float32(a))
+        assert oracle_mod.mx_scale(a) == bf.brute_mx_scale(Fraction(a)), a
+
+
+@pytest.mark.parametrize("case", range(7))
+def test_mx_pipeline_vs_bruteforce(oracle_mod, case):
+    xr, xt, _ = _tiny_cases()[case]
+    ref = bf.brute_mx_pipeline(xr, xt)
+    codes, mbits, scales = oracle_mod.mx_capture(xr)
+    assert np.array_equal(scales, ref["scales"])
+    assert np.array_equal(codes, ref["codes"])
+    assert np.array_equal(mbits, ref["mbits"])
+    out, mask = oracle_mod.mx_guided_fwd(xt, mbits, scales)
+    assert np.array_equal(mask, ref["mask"]) and np.array_equal(out, ref["out_guided"])
+    out_r, mask_r = oracle_mod.mx_rtn_fwd(xt, scales)
+    assert np.array_equal(mask_r, ref["mask"]) and np.array_equal(out_r, ref["out_rtn"])
+    out_f, mask_f = oracle_mod.mx_full_guided_fwd(xt, codes, scales)
+    assert np.array_equal(mask_f, ref["mask"]) and np.array_equal(out_f, ref["out_full"])
+
+
+def test_mx_scale_invariance_and_identity(oracle_mod):
+    """x * 2^k shifts every E8M0 byte by k and leaves the codes alone (no
+    clamping and no underflow in range); guided on x_roll itself returns the
+    rollout's codes; codes decode to the outputs."""
+    s = inputs.tiny_site(41, 16, 256, eps=0.02, outliers=False)
+    xr = inputs.bits(s.x_roll)
+    codes, mbits, scales = oracle_mod.mx_capture(xr)
+    for k in (-20, 7):
+        xk = inputs.bits((s.x_roll.float() * 2.0 ** k).to(torch.bfloat16))
+        ck, mk, sk = oracle_mod.mx_capture(xk)
+        assert np.array_equal(sk.astype(int), scales.astype(int) + k)
+        assert np.array_equal(ck, codes) and np.array_equal(mk, mbits)
+    q = oracle_mod.mx_fake_quant_codes(xr, scales, mbits=mbits).reshape(-1)
+    assert np.array_equal(q, oracle_mod.unpack_codes(codes))
+    q_full = oracle_mod.mx_fake_quant_codes(xr, scales, rcodes=codes).reshape(-1)
+    assert np.array_equal(q_full, q)
+    out, _ = oracle_mod.mx_guided_fwd(xr, mbits, scales)
+    mag = np.array(E2M1)[q & 7] * np.repeat([oracle_mod.e8m0_to_f32(int(b)) for b in scales.reshape(-1)], 32)
+    val = np.where(q & 8, -mag, mag).astype(np.float32)
+    exp = inputs.bits(torch.from_numpy(val).to(torch.bfloat16).reshape(xr.shape))
+    assert np.array_equal(out, exp)
+
+
+def test_mx_rtn_error_bound(oracle_mod):
+    """Inside the block's range, RTN lands within half a grid gap of z; the
+    top binade can clip (amax / X up to 8 > 6)."""
+    s = inputs.tiny_site(43, 32, 256, eps=0.0)
+    xr = inputs.bits(s.x_roll)
+    _, _, scales = oracle_mod.mx_capture(xr)
+    q = oracle_mod.mx_fake_quant_codes(xr, scales).reshape(-1)
+    X = np.repeat([oracle_mod.e8m0_to_f32(int(b)) for b in scales.reshape(-1)], 32)
+    z = np.abs(s.x_roll.float().numpy().reshape(-1)) / X
+    v = np.array(E2M1)[q & 7]
+    gap = np.where(v < 2, 0.5, np.where(v < 4, 1.0, 2.0))
+    inside = z <= 6
+    assert np.all(np.abs(z[inside] - v[inside]) <= gap[inside] / 2 + 1e-7)
+    assert np.all(v[~inside] == 6.0) and np.all(z[~inside] < 8)
