@@ -414,6 +414,8 @@ def run_trace(args):
     torch.cuda.synchronize()
     tier_ev = []
     for k in range(args.steps):
+        # each step starts with an idle copy engine (no backlog from the last)
+        torch.cuda.synchronize()
         flush.fill_((k + 41) & 0xFF)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         ev[0].record(stream)
@@ -428,6 +430,35 @@ def run_trace(args):
     rec_bytes = sum(cache_tier.RecordLayout.of(*w["xr"].shape, w["site"].num_groups).nbytes
                     for w in work)
     del tier
+
+    # the MXFP4 variant on the same sites: capture, 1-bit guided, RTN and
+    # full-guided forwards, each launch timed on its own
+    mxc = [ops.mx_capture(w["xr"], stream=stream) for w in work]
+
+    def mx_pass(evs):
+        for i, w in enumerate(work):
+            ev = evs[i] if evs is not None else None
+            if ev: ev[0].record(stream)
+            ops.mx_capture(w["xr"], mxc[i], stream)
+            if ev: ev[1].record(stream)
+            ops.mx_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
+            if ev: ev[2].record(stream)
+            ops.mx_rtn_fq_fwd(w["xt"], mxc[i].scales, w["out_r"], w["mask_r"], stream)
+            if ev: ev[3].record(stream)
+            ops.mx_full_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
+            if ev: ev[4].record(stream)
+
+    mx_pass(None)  # untimed: first launches
+    mx_ev = []
+    for k in range(args.steps):
+        flush.fill_((k + 53) & 0xFF)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
+        mx_pass(evs)
+        mx_ev.append(evs)
+    torch.cuda.synchronize()
+    mx_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in mx_ev for i in range(len(work)))
+             for j in range(4)]
+    mx_ms = max_over_ranks(mx_ms, pg, dev)
 
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
     per_kernel = {nm: 0.0 for nm in names}
@@ -469,6 +500,16 @@ def run_trace(args):
         "disagree_frac": [round(1.0 - r[0] / tot, 6) for r in hist_counts],
         "adjacent_frac_of_disagreements": [round(r[1] / max(1, tot - r[0]), 6) for r in hist_counts],
         "counts": hist_counts}
+    mx_rows = {}
+    for j, (nm, kn, bpe) in enumerate([("capture", "k_mx_capture", 2.65625),
+                                       ("guided_fwd", "k_mx_fake_quant<1>", 4.28125),
+                                       ("rtn_fwd", "k_mx_fake_quant<0>", 4.15625),
+                                       ("full_guided_fwd", "k_mx_fake_quant<2>", 4.65625)]):
+        ms = mx_ms[j] / args.steps
+        mx_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": bpe,
+                       "gbs": round(n * bpe / (ms * 1e-3) / 1e9, 1),
+                       "frac_of_hbm": round(n * bpe / (ms * 1e-3) / 1e9 / hbm, 4)}
+    next_rows["mxfp4"] = mx_rows
     cms, tms = tier_compute_ms / args.steps, tier_total_ms / args.steps
     next_rows["cache_tier"] = {
         "what": "capture of every site into one compact record + one D2H copy per site to pinned "

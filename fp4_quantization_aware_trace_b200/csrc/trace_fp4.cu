@@ -948,6 +948,152 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
+// Kernels 8-9: the MXFP4 variant (the post's results list: the method carries
+// over to MXFP4).  OCP Microscaling scales: one E8M0 byte per 32 elements of
+// a row, X = 2^e with e = floor(log2 max|x|) - 2 clamped at -127, and no
+// global scale.  A thread's pair of 16-element blocks is exactly one MX
+// block.  Dividing by a power of two is exact up to the one rounding of the
+// result, so z = x * 2^-e matches z = fl(x / X) with no correction step and
+// no exact path; the E2M1 decisions are those of the NVFP4 kernels.
+// ---------------------------------------------------------------------------
+
+// 2^k as fp32 for k in [-127, 127] (2^-127 is a subnormal).
+__device__ __forceinline__ float pow2f(int k) {
+  return __uint_as_float(k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00800000u >> (-126 - k));
+}
+
+// E8M0 exponent of a block whose max|x| has the bf16 bits amax (sign
+// cleared): floor(log2 amax) - 2, at least -127 (a bf16 amax stays below
+// 2^128, so the top of the range is never reached); -127 for an all-zero
+// block.
+__device__ __forceinline__ int mx_exp(uint32_t amax) {
+  if (amax == 0u) return -127;
+  const int e = (int)(amax >> 7);
+  const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;  // bf16 subnormal: m * 2^-133
+  return max(fl - 2, -127);
+}
+
+// Magic addend of the grid rounding for a = min(|z|, 6) (unscaled):
+// M = 2^22 * max(1, 2^E).
+__device__ __forceinline__ float grid_magic(float a) {
+  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
+}
+
+// Codes of one 16-element block: c0 elements 0-7, c1 elements 8-15.
+__device__ __forceinline__ void mx_codes_block(const V8& v, u64 inv2, uint32_t& c0, uint32_t& c1) {
+  uint32_t c[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w = v.w[k];
+    float zl, zh;
+    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+    // |z| < 8 from the block's own maximum; the conversion saturates past 6
+    // and keeps the sign of x, also on zeros
+    c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+  }
+  c0 = c[0];
+  c1 = c[1];
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx_capture(const V8* __restrict__ x, Shape sh, uint4* __restrict__ codes,
+                 uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const int e = mx_exp(max(absmax_block(v0), absmax_block(v1)));
+    const float inv = pow2f(-e);
+    const u64 inv2 = pk(inv, inv);
+    uint4 c;
+    mx_codes_block(v0, inv2, c.x, c.y);
+    mx_codes_block(v1, inv2, c.z, c.w);
+    codes[b >> 1] = c;
+    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
+                    (nibble_lsbs(c.w) << 24);
+    scales[b >> 1] = (uint8_t)(e + 127);
+  }
+}
+
+// Two elements of the MX fake-quant forward (side as fq_pair).
+template <int MODE>
+__device__ __forceinline__ uint32_t mx_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
+                                               uint32_t& m, int pos) {
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
+  m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
+  const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
+  float tl, th;  // chosen codeword value
+  if (MODE == kRtn) {
+    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
+    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+  } else {
+    const u64 MM = pk(grid_magic(al), grid_magic(ah));
+    const u64 aa = pk(al, ah);
+    float lol, loh, hil, hih;
+    upk(add_rm2(aa, MM), lol, loh);
+    upk(add_rp2(aa, MM), hil, hih);
+    if (MODE == kGuided) {
+      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+      upk(sub2(pk(sl, sh), MM), tl, th);
+    } else {
+      float fl, fh, cl, ch;
+      upk(sub2(pk(lol, loh), MM), fl, fh);
+      upk(sub2(pk(hil, hih), MM), cl, ch);
+      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
+      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+      tl = rl > fl ? cl : fl;
+      th = rh > fh ? ch : fh;
+    }
+  }
+  float ql, qh;
+  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
+                    const uint4* __restrict__ rcodes, const uint8_t* __restrict__ scales,
+                    V8* __restrict__ out, uint32_t* __restrict__ mask) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
+    const int e = (int)__ldcs(scales + (b >> 1)) - 127;
+    const float inv = pow2f(-e), X = pow2f(e);
+    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
+    uint32_t m = 0u;
+    V8 o;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
+                          : MODE == kFull ? ((k < 4 ? rc.x : rc.y) >> (8 * (k & 3))) : 0u;
+      o.w[k] = mx_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
+    }
+    st_block(out + b, o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
+                          : MODE == kFull ? ((k < 4 ? rc.z : rc.w) >> (8 * (k & 3))) : 0u;
+      o.w[k] = mx_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
+    }
+    st_block(out + b + 1, o);
+    mask[b >> 1] = m;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Kernel 6: plain copy with the same access pattern (bandwidth yardstick).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -1169,6 +1315,66 @@ int trace_mismatch_histogram(const uint16_t* x_train, int64_t rows, int64_t cols
   return launch(k_mismatch_hist, grid, (cudaStream_t)stream, (const V8*)x_train, sh,
                 num_groups > 1 ? group_row_offsets : nullptr, (const uint4*)codes,
                 (const uint16_t*)scales, gscale, (unsigned long long*)hist);
+}
+
+int trace_mx_capture(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                     uint32_t* mbits, uint8_t* scales, void* stream) {
+  int st = check_shape(rows, cols, 1, nullptr);
+  if (st) return st;
+  if (rows == 0) return TRACE_OK;
+  if (!x || !codes || !mbits || !scales) return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || !aligned(codes, 16) || !aligned(mbits, 4)) return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, 1);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  return launch(k_mx_capture, grid, (cudaStream_t)stream, (const V8*)x, sh, (uint4*)codes, mbits,
+                scales);
+}
+
+static int mx_fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64_t cols,
+                                const uint32_t* mbits, const uint8_t* rcodes,
+                                const uint8_t* scales, uint16_t* out, uint32_t* mask,
+                                void* stream) {
+  int st = check_shape(rows, cols, 1, nullptr);
+  if (st) return st;
+  if (rows == 0) return TRACE_OK;
+  if (!x || (mode == kGuided && !mbits) || (mode == kFull && !rcodes) || !scales || !out || !mask)
+    return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || (mode == kGuided && !aligned(mbits, 4)) ||
+      (mode == kFull && !aligned(rcodes, 16)) || !aligned(out, 32) || !aligned(mask, 4))
+    return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, 1);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (mode == kGuided)
+    return launch(k_mx_fake_quant<kGuided>, grid, s, (const V8*)x, sh, mbits, (const uint4*)nullptr,
+                  scales, (V8*)out, mask);
+  if (mode == kFull)
+    return launch(k_mx_fake_quant<kFull>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
+                  (const uint4*)rcodes, scales, (V8*)out, mask);
+  return launch(k_mx_fake_quant<kRtn>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
+                (const uint4*)nullptr, scales, (V8*)out, mask);
+}
+
+int trace_mx_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                           const uint32_t* mbits, const uint8_t* scales, uint16_t* out,
+                           uint32_t* ste_mask, void* stream) {
+  return mx_fake_quant_launch(kGuided, x_train, rows, cols, mbits, nullptr, scales, out, ste_mask,
+                              stream);
+}
+
+int trace_mx_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                                const uint8_t* codes, const uint8_t* scales, uint16_t* out,
+                                uint32_t* ste_mask, void* stream) {
+  return mx_fake_quant_launch(kFull, x_train, rows, cols, nullptr, codes, scales, out, ste_mask,
+                              stream);
+}
+
+int trace_mx_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* scales,
+                        uint16_t* out, uint32_t* ste_mask, void* stream) {
+  return mx_fake_quant_launch(kRtn, x, rows, cols, nullptr, nullptr, scales, out, ste_mask,
+                              stream);
 }
 
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,

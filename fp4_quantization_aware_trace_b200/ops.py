@@ -66,6 +66,14 @@ def library() -> ctypes.CDLL:
         lib.trace_mismatch_histogram.restype = ctypes.c_int
         lib.trace_cache_record_bytes.argtypes = [i64, i64, i32, P, P, P]
         lib.trace_cache_record_bytes.restype = sz
+        lib.trace_mx_capture.argtypes = [P, i64, i64, P, P, P, P]
+        lib.trace_mx_capture.restype = ctypes.c_int
+        lib.trace_mx_guided_fq_fwd.argtypes = [P, i64, i64, P, P, P, P, P]
+        lib.trace_mx_guided_fq_fwd.restype = ctypes.c_int
+        lib.trace_mx_full_guided_fq_fwd.argtypes = [P, i64, i64, P, P, P, P, P]
+        lib.trace_mx_full_guided_fq_fwd.restype = ctypes.c_int
+        lib.trace_mx_rtn_fq_fwd.argtypes = [P, i64, i64, P, P, P, P]
+        lib.trace_mx_rtn_fq_fwd.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -270,6 +278,82 @@ def fq_bwd(grad_out: torch.Tensor, mask: torch.Tensor, out: torch.Tensor | None 
     out = torch.empty_like(grad_out) if out is None else out
     trace_fq_bwd(grad_out, mask, grad_out.numel(), out, stream)
     return out
+
+
+def trace_mx_capture(x, rows, cols, codes, mbits, scales, stream=None) -> None:
+    _check(library().trace_mx_capture(_p(x), rows, cols, _p(codes), _p(mbits), _p(scales),
+                                      _stream(stream)), "trace_mx_capture")
+
+
+def trace_mx_guided_fq_fwd(x_train, rows, cols, mbits, scales, out, ste_mask, stream=None) -> None:
+    _check(library().trace_mx_guided_fq_fwd(_p(x_train), rows, cols, _p(mbits), _p(scales),
+                                            _p(out), _p(ste_mask), _stream(stream)),
+           "trace_mx_guided_fq_fwd")
+
+
+def trace_mx_full_guided_fq_fwd(x_train, rows, cols, codes, scales, out, ste_mask,
+                                stream=None) -> None:
+    _check(library().trace_mx_full_guided_fq_fwd(_p(x_train), rows, cols, _p(codes), _p(scales),
+                                                 _p(out), _p(ste_mask), _stream(stream)),
+           "trace_mx_full_guided_fq_fwd")
+
+
+def trace_mx_rtn_fq_fwd(x, rows, cols, scales, out, ste_mask, stream=None) -> None:
+    _check(library().trace_mx_rtn_fq_fwd(_p(x), rows, cols, _p(scales), _p(out), _p(ste_mask),
+                                         _stream(stream)), "trace_mx_rtn_fq_fwd")
+
+
+@dataclasses.dataclass
+class MxCapture:
+    """One MXFP4 capture site: full codes plus the compact cache (mantissa
+    bits + E8M0 block scales, 1.25 bits per element)."""
+    codes: torch.Tensor    # uint8 [N/2]
+    mbits: torch.Tensor    # int32 words [N/32]
+    scales: torch.Tensor   # uint8 [rows, cols/32] E8M0
+
+    def cache_nbytes(self) -> int:
+        return self.mbits.numel() * 4 + self.scales.numel()
+
+
+def mx_capture(x: torch.Tensor, out: MxCapture | None = None, stream=None) -> MxCapture:
+    """MXFP4 rollout capture of one site (x bf16 [rows, cols])."""
+    rows, cols = _bf16_2d(x)
+    n = rows * cols
+    if out is None:
+        out = MxCapture(codes=torch.empty(n // 2, dtype=torch.uint8, device=x.device),
+                        mbits=torch.empty(n // 32, dtype=torch.int32, device=x.device),
+                        scales=torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device))
+    trace_mx_capture(x, rows, cols, out.codes, out.mbits, out.scales, stream)
+    return out
+
+
+def _fq_outputs(x, out, mask):
+    rows, cols = _bf16_2d(x)
+    out = torch.empty_like(x) if out is None else out
+    mask = torch.empty(rows * cols // 32, dtype=torch.int32, device=x.device) if mask is None else mask
+    return rows, cols, out, mask
+
+
+def mx_guided_fq_fwd(x_train: torch.Tensor, cache: MxCapture, out=None, mask=None, stream=None):
+    """MXFP4 1-bit guided forward.  Returns (out, mask)."""
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    trace_mx_guided_fq_fwd(x_train, rows, cols, cache.mbits, cache.scales, out, mask, stream)
+    return out, mask
+
+
+def mx_full_guided_fq_fwd(x_train: torch.Tensor, cache: MxCapture, out=None, mask=None,
+                          stream=None):
+    """MXFP4 full-information guided forward.  Returns (out, mask)."""
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    trace_mx_full_guided_fq_fwd(x_train, rows, cols, cache.codes, cache.scales, out, mask, stream)
+    return out, mask
+
+
+def mx_rtn_fq_fwd(x: torch.Tensor, scales: torch.Tensor, out=None, mask=None, stream=None):
+    """MXFP4 round-to-nearest fake-quant with given E8M0 scales."""
+    rows, cols, out, mask = _fq_outputs(x, out, mask)
+    trace_mx_rtn_fq_fwd(x, rows, cols, scales, out, mask, stream)
+    return out, mask
 
 
 MISMATCH_RULES = ("rtn", "guided_1bit", "full_guided")

@@ -182,6 +182,36 @@ int trace_mismatch_histogram(const uint16_t* x_train, int64_t rows,
                              const float* gscale, uint64_t* hist,
                              void* stream);
 
+/* ---- MXFP4 variant ------------------------------------------------------
+ * The post's results list reports that the method carries over to MXFP4.
+ * The pages give no MX arithmetic beyond power-of-two scales, so the format
+ * is the OCP Microscaling one: 32-element blocks along a row, one E8M0 scale
+ * byte b per block, X = 2^(b-127), chosen as 2^(floor(log2 max|x|) - 2)
+ * (2 is the exponent of E2M1's largest value 6) and clamped at 2^-127 (an
+ * all-zero block gets b = 0); no global scale, no groups.  z = x / X, and
+ * the rest -- clip, E2M1 rounding, cached bit, STE mask (|z| <= 6),
+ * out = bf16(q* * X) -- is as in the NVFP4 calls above.
+ *   scales: uint8[rows, cols/32] E8M0 bytes, row-major, no alignment
+ *           requirement.  Capture writes 0..252 (a bf16 maximum stays below
+ *           2^128); bytes passed to the forwards must be 0..252 too, since
+ *           6 * 2^126 and above overflow the bf16 output.
+ *   codes, mbits, ste_mask: layouts as above; x/out 32-byte aligned, codes
+ *   16-byte, mbits and ste_mask 4-byte aligned.  trace_fq_bwd serves both
+ *   formats.  The compact MX cache is mbits + scales: 1.25 bits/element. */
+int trace_mx_capture(const uint16_t* x, int64_t rows, int64_t cols,
+                     uint8_t* codes, uint32_t* mbits, uint8_t* scales,
+                     void* stream);
+int trace_mx_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                           const uint32_t* mbits, const uint8_t* scales,
+                           uint16_t* out, uint32_t* ste_mask, void* stream);
+int trace_mx_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows,
+                                int64_t cols, const uint8_t* codes,
+                                const uint8_t* scales, uint16_t* out,
+                                uint32_t* ste_mask, void* stream);
+int trace_mx_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                        const uint8_t* scales, uint16_t* out,
+                        uint32_t* ste_mask, void* stream);
+
 /* Masked straight-through-estimator backward:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
  *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.
