@@ -114,6 +114,10 @@ def _load():
         lib.oracle_mx_full_guided_fwd.restype = None
         lib.oracle_mx_fake_quant_codes.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int]
         lib.oracle_mx_fake_quant_codes.restype = None
+        lib.oracle_swizzled_scale_bytes.argtypes = [i64, i64]
+        lib.oracle_swizzled_scale_bytes.restype = i64
+        lib.oracle_swizzle_scales.argtypes = [P, i64, i64, P]
+        lib.oracle_swizzle_scales.restype = None
         _lib = lib
         return lib
 
@@ -453,3 +457,19 @@ def mx_fake_quant_codes(x, scales, mbits=None, rcodes=None):
                                        _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
                                        _ptr(sites), mode)
     return sites.reshape(rows, cols)
+
+
+# -- block-scale layout of a block-scaled FP4 GEMM ------------------------------
+
+def swizzled_scale_bytes(rows: int, scols: int) -> int:
+    return int(_load().oracle_swizzled_scale_bytes(rows, scols))
+
+
+def swizzle_scales(scales) -> np.ndarray:
+    """Row-major scales [rows, scols] (uint8) -> the 128 x 4 tiled layout
+    (uint8, padding bytes 0)."""
+    lin = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, scols = lin.shape
+    out = np.zeros(swizzled_scale_bytes(rows, scols), np.uint8)
+    _load().oracle_swizzle_scales(_ptr(lin), rows, scols, _ptr(out))
+    return out

@@ -598,3 +598,38 @@ void oracle_mx_fake_quant_codes(const uint16_t* x, int64_t rows, int64_t cols,
                                 const uint8_t* scales, uint8_t* sites, int mode) {
   mx_fake_quant(x, rows, cols, mbits, rcodes, scales, 0, 0, sites, mode);
 }
+
+/* ------------------------------------------------------------------ */
+/* Block-scale layout of a block-scaled FP4 GEMM                        */
+/*                                                                      */
+/* The abstract on the thelatestinai.com TRACE page credits NVFP4 with  */
+/* FP4 GEMMs that run W4A4 natively.  A tcgen05 block-scaled FP4 GEMM    */
+/* reads its block scales not                                            */
+/* row-major but in 128 x 4 tiles: the [rows, scols] scale matrix is     */
+/* padded to whole tiles (rows to a multiple of 128, scale columns to a  */
+/* multiple of 4), the tiles are stored one after another in row-major   */
+/* tile order, and inside a 512-byte tile the entry of row r and column  */
+/* c sits at 16 * (r mod 32) + 4 * (r div 32) + c.  The layout is the     */
+/* same for E4M3 scales of 16-element blocks and E8M0 scales of          */
+/* 32-element blocks.                                                    */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of the tiled layout of a [rows, scols] scale matrix. */
+int64_t oracle_swizzled_scale_bytes(int64_t rows, int64_t scols) {
+  const int64_t rt = (rows + 127) / 128, ct = (scols + 3) / 4;
+  return rt * ct * 512;
+}
+
+/* Row-major scales [rows, scols] -> the tiled layout (padding bytes 0). */
+void oracle_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t scols,
+                           uint8_t* out) {
+  const int64_t ct = (scols + 3) / 4;
+  memset(out, 0, (size_t)oracle_swizzled_scale_bytes(rows, scols));
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < scols; ++c) {
+      const int64_t tile = (r / 128) * ct + c / 4;
+      const int64_t rr = r % 128, cc = c % 4;
+      out[tile * 512 + 16 * (rr % 32) + 4 * (rr / 32) + cc] = lin[r * scols + c];
+    }
+  }
+}

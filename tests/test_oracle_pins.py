@@ -662,3 +662,29 @@ def test_mx_rtn_error_bound(oracle_mod):
     inside = z <= 6
     assert np.all(np.abs(z[inside] - v[inside]) <= gap[inside] / 2 + 1e-7)
     assert np.all(v[~inside] == 6.0) and np.all(z[~inside] < 8)
+
+
+# --------------------------------------------------------------------------
+# Block-scale layout of a block-scaled FP4 GEMM (128 x 4 tiles)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,scols", [(1, 1), (5, 6), (128, 4), (130, 5), (300, 64), (257, 129)])
+def test_swizzle_scales_vs_library(oracle_mod, rows, scols):
+    """Against vllm's row-major -> 128x4 scale swizzle (a torch routine that
+    runs on the CPU; it is written for E8M0 scales of 32-element blocks and
+    the layout depends only on the scale matrix's shape)."""
+    mx = pytest.importorskip("vllm.model_executor.layers.quantization.utils.mxfp8_utils")
+    rng = np.random.default_rng(rows * 1000 + scols)
+    lin = rng.integers(1, 256, (rows, scols), dtype=np.uint8)
+    ref = mx.swizzle_mxfp8_scale(torch.from_numpy(lin), rows, scols * 32).reshape(-1).numpy()
+    got = oracle_mod.swizzle_scales(lin)
+    assert got.shape == ref.shape and np.array_equal(got, ref)
+
+
+def test_swizzle_scales_is_a_padded_permutation(oracle_mod):
+    rows, scols = 300, 37
+    lin = (np.arange(rows * scols) % 251 + 1).astype(np.uint8).reshape(rows, scols)
+    got = oracle_mod.swizzle_scales(lin)
+    assert got.size == 384 * 40
+    assert np.count_nonzero(got) == rows * scols
+    assert np.array_equal(np.sort(got[got != 0]), np.sort(lin.reshape(-1)))
