@@ -448,6 +448,36 @@ def run_trace(args):
             ops.mx_full_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
             if ev: ev[4].record(stream)
 
+    # capture and guided forward with the scales in the 128 x 4 tiled layout
+    # of a block-scaled FP4 GEMM
+    tcap = [ops.capture_tiled(w["xr"], w["offs"], stream) for w in work]
+    tws = [w["ws"] for w in work]
+
+    def tiled_pass(evs):
+        for i, w in enumerate(work):
+            R, C = w["xr"].shape
+            G = w["site"].num_groups
+            ev = evs[i] if evs is not None else None
+            if ev: ev[0].record(stream)
+            ops.trace_capture_ex(w["xr"], R, C, G, w["offs"], tcap[i].codes, tcap[i].mbits,
+                                 tcap[i].scales, tcap[i].gscale, tws[i], tws[i].numel(),
+                                 ops.TRACE_SCALES_TILED_128x4, stream)
+            if ev: ev[1].record(stream)
+            ops.fq_fwd_tiled(ops.TRACE_RULE_GUIDED, w["xt"], tcap[i], w["out"], w["mask"], stream)
+            if ev: ev[2].record(stream)
+
+    tiled_pass(None)
+    tl_ev = []
+    for k in range(args.steps):
+        flush.fill_((k + 67) & 0xFF)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in work]
+        tiled_pass(evs)
+        tl_ev.append(evs)
+    torch.cuda.synchronize()
+    tl_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in tl_ev for i in range(len(work)))
+             for j in range(2)]
+    tl_ms = max_over_ranks(tl_ms, pg, dev)
+
     mx_pass(None)  # untimed: first launches
     mx_ev = []
     for k in range(args.steps):
@@ -510,6 +540,12 @@ def run_trace(args):
                        "gbs": round(n * bpe / (ms * 1e-3) / 1e9, 1),
                        "frac_of_hbm": round(n * bpe / (ms * 1e-3) / 1e9 / hbm, 4)}
     next_rows["mxfp4"] = mx_rows
+    next_rows["tiled_scales"] = {
+        nm: {"kernel": kn, "us": round(tl_ms[j] / args.steps * 1e3, 2), "bytes_per_elem": bpe,
+             "gbs": round(n * bpe / (tl_ms[j] / args.steps * 1e-3) / 1e9, 1),
+             "frac_of_hbm": round(n * bpe / (tl_ms[j] / args.steps * 1e-3) / 1e9 / hbm, 4)}
+        for j, (nm, kn, bpe) in enumerate([("capture", "k_amax + k_capture<true>", 4.6875),
+                                           ("guided_fwd", "k_fake_quant<1, true>", 4.3125)])}
     cms, tms = tier_compute_ms / args.steps, tier_total_ms / args.steps
     next_rows["cache_tier"] = {
         "what": "capture of every site into one compact record + one D2H copy per site to pinned "

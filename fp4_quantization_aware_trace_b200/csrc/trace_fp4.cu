@@ -418,7 +418,17 @@ struct Shape {
   uint32_t ntiles;  // ceil(nblk / kTileBlks)
   FastDiv bpr;      // blocks per row
   int G;
+  uint32_t sw_ct;   // tiled scale layout: 128 x 4 tiles per row of tiles
 };
+
+// Byte offset of the scale at (row, col) in the tiled layout a block-scaled
+// FP4 GEMM reads: the scale matrix cut into 128-row x 4-column tiles of 512
+// bytes, stored in row-major tile order (ct tiles per row of tiles); inside
+// a tile, row r and column c sit at 16 (r mod 32) + 4 (r div 32) + c.
+__device__ __forceinline__ size_t tiled_scale_offset(uint32_t row, uint32_t col, uint32_t ct) {
+  return ((size_t)(row >> 7) * ct + (col >> 2)) * 512u + ((row & 31u) << 4) +
+         (((row >> 5) & 3u) << 2) + (col & 3u);
+}
 
 // ---------------------------------------------------------------------------
 // Kernel 0: zero the per-group amax accumulators.
@@ -568,10 +578,12 @@ __device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk,
 
 // Each thread owns two adjacent blocks: one 16-byte store of codes, one
 // 32-bit store of mantissa bits, one 16-bit store of scales.
+// SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
+template <bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
               const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
-              uint32_t* __restrict__ mbits, uint16_t* __restrict__ scales,
+              uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales,
               float* __restrict__ gscale) {
   pdl_begin();
   // global scales of all groups (any CTA may write them; all write the same)
@@ -590,14 +602,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (b >= sh.nblk) continue;
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     // both blocks of the pair are in the same row (cols is a multiple of 32)
-    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) gk = group_consts(__ldg(amax + gc.g));
+    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+    if (gc.seek(row)) gk = group_consts(__ldg(amax + gc.g));
     uint4 c;
     const uint32_t s0 = capture_block(v0, gk, c.x, c.y);
     const uint32_t s1 = capture_block(v1, gk, c.z, c.w);
     codes[b >> 1] = c;
     mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
                     (nibble_lsbs(c.w) << 24);
-    scales[b >> 1] = (uint16_t)(s0 | (s1 << 8));
+    const uint16_t sv = (uint16_t)(s0 | (s1 << 8));
+    if (SW)  // the pair's two columns are neighbours inside one tile
+      *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
+    else
+      reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
   }
 }
 
@@ -700,11 +717,11 @@ __device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, u
 // Each thread owns two adjacent blocks, so their mantissa bits, scales and
 // mask move as one 32-bit / 16-bit / 32-bit access (the full codes as one
 // 16-byte access).
-template <int MODE>
+template <int MODE, bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
                  const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
-                 const uint16_t* __restrict__ scales, const float* __restrict__ gscale,
+                 const uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                  V8* __restrict__ out, uint32_t* __restrict__ mask) {
   pdl_begin();
   GroupCursor gc;
@@ -717,8 +734,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
     const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t sb2 = __ldcs(scales + (b >> 1));
-    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
+    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+    const uint32_t sb2 =
+        SW ? __ldcs(reinterpret_cast<const unsigned short*>(
+                 scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
+           : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
+    if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
     V8 o;
     uint32_t m0, m1;
     fake_quant_block<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
@@ -995,6 +1016,7 @@ __device__ __forceinline__ void mx_codes_block(const V8& v, u64 inv2, uint32_t& 
   c1 = c[1];
 }
 
+template <bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mx_capture(const V8* __restrict__ x, Shape sh, uint4* __restrict__ codes,
                  uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
@@ -1012,7 +1034,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     codes[b >> 1] = c;
     mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
                     (nibble_lsbs(c.w) << 24);
-    scales[b >> 1] = (uint8_t)(e + 127);
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      scales[tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct)] = (uint8_t)(e + 127);
+    } else {
+      scales[b >> 1] = (uint8_t)(e + 127);
+    }
   }
 }
 
@@ -1058,7 +1085,7 @@ __device__ __forceinline__ uint32_t mx_fq_pair(uint32_t w, uint32_t side, u64 in
   return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
 }
 
-template <int MODE>
+template <int MODE, bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mx_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
                     const uint4* __restrict__ rcodes, const uint8_t* __restrict__ scales,
@@ -1070,7 +1097,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
     const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
-    const int e = (int)__ldcs(scales + (b >> 1)) - 127;
+    size_t so = b >> 1;
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
+    }
+    const int e = (int)__ldcs(scales + so) - 127;
     const float inv = pow2f(-e), X = pow2f(e);
     const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
     uint32_t m = 0u;
@@ -1148,6 +1180,7 @@ Shape make_shape(int64_t rows, int64_t cols, int32_t G) {
   sh.ntiles = (uint32_t)(((uint64_t)sh.nblk + kTileBlks - 1) / kTileBlks);
   sh.bpr = make_fastdiv((uint32_t)(cols / 16));
   sh.G = G;
+  sh.sw_ct = (uint32_t)((cols / 16 + 3) / 4);  // NVFP4: cols/16 scale columns
   return sh;
 }
 
@@ -1177,6 +1210,35 @@ int launch(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? TRACE_OK
                                                                                       : TRACE_ERR_CUDA;
+}
+
+template <bool SW>
+int fake_quant_dispatch(int mode, int grid, cudaStream_t s, const uint16_t* x,
+                               const Shape& sh, const int64_t* o, const uint32_t* mbits,
+                               const uint8_t* rcodes, const uint8_t* scales, const float* gscale,
+                               uint16_t* out, uint32_t* mask) {
+  if (mode == kGuided)
+    return launch(k_fake_quant<kGuided, SW>, grid, s, (const V8*)x, sh, o, mbits,
+                  (const uint4*)nullptr, scales, gscale, (V8*)out, mask);
+  if (mode == kFull)
+    return launch(k_fake_quant<kFull, SW>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
+                  (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
+  return launch(k_fake_quant<kRtn, SW>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
+                (const uint4*)nullptr, scales, gscale, (V8*)out, mask);
+}
+
+template <bool SW>
+int mx_fake_quant_dispatch(int mode, int grid, cudaStream_t s, const uint16_t* x,
+                                  const Shape& sh, const uint32_t* mbits, const uint8_t* rcodes,
+                                  const uint8_t* scales, uint16_t* out, uint32_t* mask) {
+  if (mode == kGuided)
+    return launch(k_mx_fake_quant<kGuided, SW>, grid, s, (const V8*)x, sh, mbits,
+                  (const uint4*)nullptr, scales, (V8*)out, mask);
+  if (mode == kFull)
+    return launch(k_mx_fake_quant<kFull, SW>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
+                  (const uint4*)rcodes, scales, (V8*)out, mask);
+  return launch(k_mx_fake_quant<kRtn, SW>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
+                (const uint4*)nullptr, scales, (V8*)out, mask);
 }
 
 }  // namespace
@@ -1217,10 +1279,10 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
   return up16(og + 4u * (size_t)num_groups);
 }
 
-int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
-                  const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
-                  uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
-                  void* stream) {
+static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
+                        const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
+                        uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
+                        bool tiled, void* stream) {
   int st = check_shape(rows, cols, num_groups, group_row_offsets);
   if (st) return st;
   // with no rows only the global scales are written; the data pointers of
@@ -1240,14 +1302,26 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_gro
   const int zg = (num_groups + kThreads - 1) / kThreads;
   if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups))) return st;
   if (sh.nblk > 0 && (st = launch(k_amax, grid, s, (const V8*)x, sh, offs, amax))) return st;
-  return launch(k_capture, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax, (uint4*)codes,
-                (uint32_t*)mbits, (uint16_t*)scales, gscale);
+  if (tiled)
+    return launch(k_capture<true>, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax,
+                  (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+  return launch(k_capture<false>, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax,
+                (uint4*)codes, (uint32_t*)mbits, scales, gscale);
 }
+
+int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
+                  const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
+                  uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
+                  void* stream) {
+  return capture_impl(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,
+                      workspace, workspace_bytes, false, stream);
+}
+
 
 static int fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64_t cols, int32_t G,
                              const int64_t* offs, const uint32_t* mbits, const uint8_t* rcodes,
                              const uint8_t* scales, const float* gscale, uint16_t* out,
-                             uint32_t* mask, void* stream) {
+                             uint32_t* mask, void* stream, bool tiled = false) {
   int st = check_shape(rows, cols, G, offs);
   if (st) return st;
   if (rows == 0) return TRACE_OK;  // nothing to do; empty tensors may have NULL data
@@ -1264,14 +1338,10 @@ static int fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64_t 
   if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* o = G > 1 ? offs : nullptr;
-  if (mode == kGuided)
-    return launch(k_fake_quant<kGuided>, grid, s, (const V8*)x, sh, o, (const uint32_t*)mbits,
-                  (const uint4*)nullptr, (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
-  if (mode == kFull)
-    return launch(k_fake_quant<kFull>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
-                  (const uint4*)rcodes, (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
-  return launch(k_fake_quant<kRtn>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
-                (const uint4*)nullptr, (const uint16_t*)scales, gscale, (V8*)out, (uint32_t*)mask);
+  return tiled ? fake_quant_dispatch<true>(mode, grid, s, x, sh, o, mbits, rcodes, scales, gscale,
+                                           out, mask)
+               : fake_quant_dispatch<false>(mode, grid, s, x, sh, o, mbits, rcodes, scales,
+                                            gscale, out, mask);
 }
 
 int trace_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols, int32_t num_groups,
@@ -1317,24 +1387,34 @@ int trace_mismatch_histogram(const uint16_t* x_train, int64_t rows, int64_t cols
                 (const uint16_t*)scales, gscale, (unsigned long long*)hist);
 }
 
-int trace_mx_capture(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
-                     uint32_t* mbits, uint8_t* scales, void* stream) {
+static int mx_capture_impl(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                           uint32_t* mbits, uint8_t* scales, bool tiled, void* stream) {
   int st = check_shape(rows, cols, 1, nullptr);
   if (st) return st;
   if (rows == 0) return TRACE_OK;
   if (!x || !codes || !mbits || !scales) return TRACE_ERR_NULL;
   if (!aligned(x, 32) || !aligned(codes, 16) || !aligned(mbits, 4)) return TRACE_ERR_ALIGN;
-  const Shape sh = make_shape(rows, cols, 1);
+  Shape sh = make_shape(rows, cols, 1);
+  sh.sw_ct = (uint32_t)((cols / 32 + 3) / 4);  // cols/32 E8M0 scale columns
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
-  return launch(k_mx_capture, grid, (cudaStream_t)stream, (const V8*)x, sh, (uint4*)codes, mbits,
-                scales);
+  if (tiled)
+    return launch(k_mx_capture<true>, grid, (cudaStream_t)stream, (const V8*)x, sh, (uint4*)codes,
+                  mbits, scales);
+  return launch(k_mx_capture<false>, grid, (cudaStream_t)stream, (const V8*)x, sh, (uint4*)codes,
+                mbits, scales);
 }
+
+int trace_mx_capture(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                     uint32_t* mbits, uint8_t* scales, void* stream) {
+  return mx_capture_impl(x, rows, cols, codes, mbits, scales, false, stream);
+}
+
 
 static int mx_fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64_t cols,
                                 const uint32_t* mbits, const uint8_t* rcodes,
                                 const uint8_t* scales, uint16_t* out, uint32_t* mask,
-                                void* stream) {
+                                void* stream, bool tiled = false) {
   int st = check_shape(rows, cols, 1, nullptr);
   if (st) return st;
   if (rows == 0) return TRACE_OK;
@@ -1343,18 +1423,14 @@ static int mx_fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64
   if (!aligned(x, 32) || (mode == kGuided && !aligned(mbits, 4)) ||
       (mode == kFull && !aligned(rcodes, 16)) || !aligned(out, 32) || !aligned(mask, 4))
     return TRACE_ERR_ALIGN;
-  const Shape sh = make_shape(rows, cols, 1);
+  Shape sh = make_shape(rows, cols, 1);
+  sh.sw_ct = (uint32_t)((cols / 32 + 3) / 4);
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  if (mode == kGuided)
-    return launch(k_mx_fake_quant<kGuided>, grid, s, (const V8*)x, sh, mbits, (const uint4*)nullptr,
-                  scales, (V8*)out, mask);
-  if (mode == kFull)
-    return launch(k_mx_fake_quant<kFull>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
-                  (const uint4*)rcodes, scales, (V8*)out, mask);
-  return launch(k_mx_fake_quant<kRtn>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
-                (const uint4*)nullptr, scales, (V8*)out, mask);
+  return tiled ? mx_fake_quant_dispatch<true>(mode, grid, s, x, sh, mbits, rcodes, scales, out, mask)
+               : mx_fake_quant_dispatch<false>(mode, grid, s, x, sh, mbits, rcodes, scales, out,
+                                               mask);
 }
 
 int trace_mx_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
@@ -1375,6 +1451,54 @@ int trace_mx_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols, const uin
                         uint16_t* out, uint32_t* ste_mask, void* stream) {
   return mx_fake_quant_launch(kRtn, x, rows, cols, nullptr, nullptr, scales, out, ste_mask,
                               stream);
+}
+
+size_t trace_scale_bytes(int64_t rows, int64_t cols, int32_t block_size, int32_t scale_layout) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0 || (block_size != 16 && block_size != 32)) return 0;
+  const int64_t scols = cols / block_size;
+  if (scale_layout == TRACE_SCALES_ROW_MAJOR) return (size_t)(rows * scols);
+  if (scale_layout != TRACE_SCALES_TILED_128x4) return 0;
+  return (size_t)((rows + 127) / 128) * (size_t)((scols + 3) / 4) * 512u;
+}
+
+static bool valid_layout(int32_t layout) {
+  return layout == TRACE_SCALES_ROW_MAJOR || layout == TRACE_SCALES_TILED_128x4;
+}
+
+int trace_capture_ex(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
+                     const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
+                     uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
+                     int32_t scale_layout, void* stream) {
+  if (!valid_layout(scale_layout)) return TRACE_ERR_SHAPE;
+  return capture_impl(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,
+                      workspace, workspace_bytes, scale_layout == TRACE_SCALES_TILED_128x4, stream);
+}
+
+int trace_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows, int64_t cols,
+                    int32_t num_groups, const int64_t* group_row_offsets, const uint32_t* mbits,
+                    const uint8_t* codes, const uint8_t* scales, const float* gscale, uint16_t* out,
+                    uint32_t* ste_mask, int32_t scale_layout, void* stream) {
+  if (!valid_layout(scale_layout) || rule < TRACE_RULE_RTN || rule > TRACE_RULE_FULL)
+    return TRACE_ERR_SHAPE;
+  return fake_quant_launch(rule, x_train, rows, cols, num_groups, group_row_offsets, mbits, codes,
+                           scales, gscale, out, ste_mask, stream,
+                           scale_layout == TRACE_SCALES_TILED_128x4);
+}
+
+int trace_mx_capture_ex(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                        uint32_t* mbits, uint8_t* scales, int32_t scale_layout, void* stream) {
+  if (!valid_layout(scale_layout)) return TRACE_ERR_SHAPE;
+  return mx_capture_impl(x, rows, cols, codes, mbits, scales,
+                         scale_layout == TRACE_SCALES_TILED_128x4, stream);
+}
+
+int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows, int64_t cols,
+                       const uint32_t* mbits, const uint8_t* codes, const uint8_t* scales,
+                       uint16_t* out, uint32_t* ste_mask, int32_t scale_layout, void* stream) {
+  if (!valid_layout(scale_layout) || rule < TRACE_RULE_RTN || rule > TRACE_RULE_FULL)
+    return TRACE_ERR_SHAPE;
+  return mx_fake_quant_launch(rule, x_train, rows, cols, mbits, codes, scales, out, ste_mask,
+                              stream, scale_layout == TRACE_SCALES_TILED_128x4);
 }
 
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,
@@ -1402,6 +1526,7 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* str
   sh.ntiles = (uint32_t)(((uint64_t)sh.nblk + kTileBlks - 1) / kTileBlks);
   sh.bpr = make_fastdiv(1);
   sh.G = 1;
+  sh.sw_ct = 1;
   int grid, st;
   if ((st = grid_for(sh, &grid))) return st;
   return launch(k_copy, grid, (cudaStream_t)stream, (const V8*)src, sh, (V8*)dst);

@@ -74,6 +74,16 @@ def library() -> ctypes.CDLL:
         lib.trace_mx_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_mx_rtn_fq_fwd.argtypes = [P, i64, i64, P, P, P, P]
         lib.trace_mx_rtn_fq_fwd.restype = ctypes.c_int
+        lib.trace_scale_bytes.argtypes = [i64, i64, i32, i32]
+        lib.trace_scale_bytes.restype = sz
+        lib.trace_capture_ex.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, sz, i32, P]
+        lib.trace_capture_ex.restype = ctypes.c_int
+        lib.trace_fq_fwd_ex.argtypes = [i32, P, i64, i64, i32, P, P, P, P, P, P, P, i32, P]
+        lib.trace_fq_fwd_ex.restype = ctypes.c_int
+        lib.trace_mx_capture_ex.argtypes = [P, i64, i64, P, P, P, i32, P]
+        lib.trace_mx_capture_ex.restype = ctypes.c_int
+        lib.trace_mx_fq_fwd_ex.argtypes = [i32, P, i64, i64, P, P, P, P, P, i32, P]
+        lib.trace_mx_fq_fwd_ex.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -353,6 +363,88 @@ def mx_rtn_fq_fwd(x: torch.Tensor, scales: torch.Tensor, out=None, mask=None, st
     """MXFP4 round-to-nearest fake-quant with given E8M0 scales."""
     rows, cols, out, mask = _fq_outputs(x, out, mask)
     trace_mx_rtn_fq_fwd(x, rows, cols, scales, out, mask, stream)
+    return out, mask
+
+
+# scale layouts and rounding rules of the _ex calls
+TRACE_SCALES_ROW_MAJOR, TRACE_SCALES_TILED_128x4 = 0, 1
+TRACE_RULE_RTN, TRACE_RULE_GUIDED, TRACE_RULE_FULL = 0, 1, 2
+
+
+def trace_scale_bytes(rows: int, cols: int, block_size: int, scale_layout: int) -> int:
+    return int(library().trace_scale_bytes(rows, cols, block_size, scale_layout))
+
+
+def trace_capture_ex(x, rows, cols, num_groups, offsets, codes, mbits, scales, gscale, workspace,
+                     workspace_bytes, scale_layout, stream=None) -> None:
+    _check(library().trace_capture_ex(_p(x), rows, cols, num_groups, _p(offsets), _p(codes),
+                                      _p(mbits), _p(scales), _p(gscale), _p(workspace),
+                                      workspace_bytes, scale_layout, _stream(stream)),
+           "trace_capture_ex")
+
+
+def trace_fq_fwd_ex(rule, x_train, rows, cols, num_groups, offsets, mbits, codes, scales, gscale,
+                    out, ste_mask, scale_layout, stream=None) -> None:
+    _check(library().trace_fq_fwd_ex(rule, _p(x_train), rows, cols, num_groups, _p(offsets),
+                                     _p(mbits), _p(codes), _p(scales), _p(gscale), _p(out),
+                                     _p(ste_mask), scale_layout, _stream(stream)), "trace_fq_fwd_ex")
+
+
+def trace_mx_capture_ex(x, rows, cols, codes, mbits, scales, scale_layout, stream=None) -> None:
+    _check(library().trace_mx_capture_ex(_p(x), rows, cols, _p(codes), _p(mbits), _p(scales),
+                                         scale_layout, _stream(stream)), "trace_mx_capture_ex")
+
+
+def trace_mx_fq_fwd_ex(rule, x_train, rows, cols, mbits, codes, scales, out, ste_mask,
+                       scale_layout, stream=None) -> None:
+    _check(library().trace_mx_fq_fwd_ex(rule, _p(x_train), rows, cols, _p(mbits), _p(codes),
+                                        _p(scales), _p(out), _p(ste_mask), scale_layout,
+                                        _stream(stream)), "trace_mx_fq_fwd_ex")
+
+
+def capture_tiled(x: torch.Tensor, offsets: torch.Tensor | None = None, stream=None) -> Capture:
+    """NVFP4 capture with the scales in the 128 x 4 tiled layout of a
+    block-scaled FP4 GEMM (Capture.scales is then a flat uint8 tensor of
+    trace_scale_bytes(...) bytes, padding zeroed)."""
+    rows, cols = _bf16_2d(x)
+    G = _groups(offsets)
+    cap, ws = alloc_capture(rows, cols, G, x.device, offsets)
+    cap.scales = torch.zeros(trace_scale_bytes(rows, cols, 16, TRACE_SCALES_TILED_128x4),
+                             dtype=torch.uint8, device=x.device)
+    trace_capture_ex(x, rows, cols, G, offsets, cap.codes, cap.mbits, cap.scales, cap.gscale, ws,
+                     ws.numel(), TRACE_SCALES_TILED_128x4, stream)
+    return cap
+
+
+def fq_fwd_tiled(rule: int, x_train: torch.Tensor, cache: Capture, out=None, mask=None,
+                 stream=None):
+    """NVFP4 forward (rule TRACE_RULE_*) reading tiled scales.  Returns (out, mask)."""
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    trace_fq_fwd_ex(rule, x_train, rows, cols, _groups(cache.offsets), cache.offsets, cache.mbits,
+                    cache.codes, cache.scales, cache.gscale, out, mask, TRACE_SCALES_TILED_128x4,
+                    stream)
+    return out, mask
+
+
+def mx_capture_tiled(x: torch.Tensor, stream=None) -> MxCapture:
+    """MXFP4 capture with the E8M0 scales in the 128 x 4 tiled layout."""
+    rows, cols = _bf16_2d(x)
+    n = rows * cols
+    cap = MxCapture(codes=torch.empty(n // 2, dtype=torch.uint8, device=x.device),
+                    mbits=torch.empty(n // 32, dtype=torch.int32, device=x.device),
+                    scales=torch.zeros(trace_scale_bytes(rows, cols, 32, TRACE_SCALES_TILED_128x4),
+                                       dtype=torch.uint8, device=x.device))
+    trace_mx_capture_ex(x, rows, cols, cap.codes, cap.mbits, cap.scales, TRACE_SCALES_TILED_128x4,
+                        stream)
+    return cap
+
+
+def mx_fq_fwd_tiled(rule: int, x_train: torch.Tensor, cache: MxCapture, out=None, mask=None,
+                    stream=None):
+    """MXFP4 forward (rule TRACE_RULE_*) reading tiled scales."""
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    trace_mx_fq_fwd_ex(rule, x_train, rows, cols, cache.mbits, cache.codes, cache.scales, out,
+                       mask, TRACE_SCALES_TILED_128x4, stream)
     return out, mask
 
 

@@ -212,6 +212,54 @@ int trace_mx_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
                         const uint8_t* scales, uint16_t* out,
                         uint32_t* ste_mask, void* stream);
 
+/* ---- Block-scale layout of a block-scaled FP4 GEMM ------------------------
+ * The abstract on the thelatestinai.com TRACE page credits NVFP4 with FP4
+ * GEMMs that run W4A4 natively.  The rollout's own FP4 GEMM (a tcgen05
+ * block-scaled MMA) reads the block scales in a tiled layout rather than
+ * row-major; these entry points let capture write them in that layout
+ * directly (no separate reformatting pass over the scales) and let the
+ * forwards read it.  Layout TRACE_SCALES_TILED_128x4: the [rows, scols]
+ * scale matrix (scols = cols/16 E4M3 scales, or cols/32 E8M0 scales for
+ * MXFP4) is cut into 128-row x 4-column tiles of 512 bytes, stored in
+ * row-major tile order; inside a tile the scale of row r and column c is at
+ * byte 16*(r % 32) + 4*(r / 32) + c.  Rows are padded to a multiple of 128
+ * and scale columns to a multiple of 4; the kernels never write or read the
+ * padding (zero it once if the GEMM reads it).
+ *   rule: TRACE_RULE_RTN (trace_rtn_fq_fwd), TRACE_RULE_GUIDED
+ *         (trace_guided_fq_fwd: mbits), TRACE_RULE_FULL
+ *         (trace_full_guided_fq_fwd: codes); the pointer the rule does not
+ *         read may be NULL.
+ *   Everything else as the calls without _ex (which are scale_layout =
+ *   TRACE_SCALES_ROW_MAJOR).  An unknown layout or rule returns
+ *   TRACE_ERR_SHAPE.  The mismatch histogram and the cache record take
+ *   row-major scales only. */
+typedef enum { TRACE_SCALES_ROW_MAJOR = 0, TRACE_SCALES_TILED_128x4 = 1 } trace_scale_layout;
+typedef enum { TRACE_RULE_RTN = 0, TRACE_RULE_GUIDED = 1, TRACE_RULE_FULL = 2 } trace_rule;
+
+/* Bytes of the scale array for block_size 16 (NVFP4) or 32 (MXFP4) in a
+ * layout (padding included); 0 for an invalid argument.  Host only. */
+size_t trace_scale_bytes(int64_t rows, int64_t cols, int32_t block_size,
+                         int32_t scale_layout);
+int trace_capture_ex(const uint16_t* x, int64_t rows, int64_t cols,
+                     int32_t num_groups, const int64_t* group_row_offsets,
+                     uint8_t* codes, uint32_t* mbits, uint8_t* scales,
+                     float* gscale, void* workspace, size_t workspace_bytes,
+                     int32_t scale_layout, void* stream);
+int trace_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows,
+                    int64_t cols, int32_t num_groups,
+                    const int64_t* group_row_offsets, const uint32_t* mbits,
+                    const uint8_t* codes, const uint8_t* scales,
+                    const float* gscale, uint16_t* out, uint32_t* ste_mask,
+                    int32_t scale_layout, void* stream);
+int trace_mx_capture_ex(const uint16_t* x, int64_t rows, int64_t cols,
+                        uint8_t* codes, uint32_t* mbits, uint8_t* scales,
+                        int32_t scale_layout, void* stream);
+int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows,
+                       int64_t cols, const uint32_t* mbits,
+                       const uint8_t* codes, const uint8_t* scales,
+                       uint16_t* out, uint32_t* ste_mask, int32_t scale_layout,
+                       void* stream);
+
 /* Masked straight-through-estimator backward:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
  *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.

@@ -97,3 +97,14 @@ def test_binding_rejects_host_tensors(lib):
     x = torch.zeros(4, 32, dtype=torch.bfloat16)
     with pytest.raises(ops.TraceError):
         ops.fq_bwd(x, torch.zeros(4, dtype=torch.int32))
+
+
+def test_scale_bytes_query(lib):
+    """Host-only size query of the scale layouts (no GPU needed)."""
+    assert lib.trace_scale_bytes(300, 2048, 16, 0) == 300 * 128
+    assert lib.trace_scale_bytes(300, 2048, 16, 1) == 3 * 32 * 512
+    assert lib.trace_scale_bytes(300, 2048, 32, 1) == 3 * 16 * 512
+    assert lib.trace_scale_bytes(1, 32, 16, 1) == 512
+    assert lib.trace_scale_bytes(1, 32, 32, 0) == 1
+    for bad in [(4, 48, 16, 0), (4, 64, 8, 0), (4, 64, 16, 2), (-1, 64, 16, 0)]:
+        assert lib.trace_scale_bytes(*bad) == 0
