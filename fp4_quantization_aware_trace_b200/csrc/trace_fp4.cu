@@ -1465,6 +1465,46 @@ static bool valid_layout(int32_t layout) {
   return layout == TRACE_SCALES_ROW_MAJOR || layout == TRACE_SCALES_TILED_128x4;
 }
 
+int trace_capture_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
+                       const int64_t* group_row_offsets, uint32_t* amax, void* stream) {
+  int st = check_shape(rows, cols, num_groups, group_row_offsets);
+  if (st) return st;
+  if ((rows > 0 && !x) || !amax) return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || !aligned(amax, 4)) return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, num_groups);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int zg = (num_groups + kThreads - 1) / kThreads;
+  if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups))) return st;
+  if (sh.nblk == 0) return TRACE_OK;
+  return launch(k_amax, grid, s, (const V8*)x, sh, num_groups > 1 ? group_row_offsets : nullptr,
+                amax);
+}
+
+int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
+                            const int64_t* group_row_offsets, const uint32_t* amax,
+                            uint8_t* codes, uint32_t* mbits, uint8_t* scales, float* gscale,
+                            int32_t scale_layout, void* stream) {
+  int st = check_shape(rows, cols, num_groups, group_row_offsets);
+  if (st) return st;
+  if (!valid_layout(scale_layout)) return TRACE_ERR_SHAPE;
+  if ((rows > 0 && (!x || !codes || !mbits || !scales)) || !gscale || !amax) return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || !aligned(codes, 16) || !aligned(mbits, 16) || !aligned(scales, 16) ||
+      !aligned(gscale, 4) || !aligned(amax, 4))
+    return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, num_groups);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
+  if (scale_layout == TRACE_SCALES_TILED_128x4)
+    return launch(k_capture<true>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes, mbits,
+                  scales, gscale);
+  return launch(k_capture<false>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes, mbits,
+                scales, gscale);
+}
+
 int trace_capture_ex(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                      const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
                      uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,

@@ -84,6 +84,10 @@ def library() -> ctypes.CDLL:
         lib.trace_mx_capture_ex.restype = ctypes.c_int
         lib.trace_mx_fq_fwd_ex.argtypes = [i32, P, i64, i64, P, P, P, P, P, i32, P]
         lib.trace_mx_fq_fwd_ex.restype = ctypes.c_int
+        lib.trace_capture_amax.argtypes = [P, i64, i64, i32, P, P, P]
+        lib.trace_capture_amax.restype = ctypes.c_int
+        lib.trace_capture_with_amax.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, i32, P]
+        lib.trace_capture_with_amax.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -446,6 +450,41 @@ def mx_fq_fwd_tiled(rule: int, x_train: torch.Tensor, cache: MxCapture, out=None
     trace_mx_fq_fwd_ex(rule, x_train, rows, cols, cache.mbits, cache.codes, cache.scales, out,
                        mask, TRACE_SCALES_TILED_128x4, stream)
     return out, mask
+
+
+def trace_capture_amax(x, rows, cols, num_groups, offsets, amax, stream=None) -> None:
+    _check(library().trace_capture_amax(_p(x), rows, cols, num_groups, _p(offsets), _p(amax),
+                                        _stream(stream)), "trace_capture_amax")
+
+
+def trace_capture_with_amax(x, rows, cols, num_groups, offsets, amax, codes, mbits, scales,
+                            gscale, scale_layout=0, stream=None) -> None:
+    _check(library().trace_capture_with_amax(_p(x), rows, cols, num_groups, _p(offsets), _p(amax),
+                                             _p(codes), _p(mbits), _p(scales), _p(gscale),
+                                             scale_layout, _stream(stream)),
+           "trace_capture_with_amax")
+
+
+def capture_sharded(x: torch.Tensor, offsets: torch.Tensor | None = None, group=None,
+                    stream=None) -> Capture:
+    """Capture of this rank's row shard of a tensor whose rows are spread
+    over the ranks of `group` (torch.distributed; None = no reduction): the
+    per-group amax is all-reduced (MAX) between the two passes, so every
+    rank ends with the global scales of the whole tensor.  The one
+    collective moves 4 bytes per group."""
+    rows, cols = _bf16_2d(x)
+    G = _groups(offsets)
+    cap, _ = alloc_capture(rows, cols, G, x.device, offsets)
+    amax = torch.empty(G, dtype=torch.int32, device=x.device)
+    trace_capture_amax(x, rows, cols, G, offsets, amax, stream)
+    if group is not None:
+        import torch.distributed as dist
+        s = torch.cuda.current_stream(x.device) if stream is None else stream
+        with torch.cuda.stream(s):
+            dist.all_reduce(amax, op=dist.ReduceOp.MAX, group=group)
+    trace_capture_with_amax(x, rows, cols, G, offsets, amax, cap.codes, cap.mbits, cap.scales,
+                            cap.gscale, TRACE_SCALES_ROW_MAJOR, stream)
+    return cap
 
 
 MISMATCH_RULES = ("rtn", "guided_1bit", "full_guided")

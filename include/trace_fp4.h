@@ -260,6 +260,30 @@ int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows,
                        uint16_t* out, uint32_t* ste_mask, int32_t scale_layout,
                        void* stream);
 
+/* ---- Capture of a row-sharded tensor -------------------------------------
+ * When one tensor's rows are spread over several GPUs, its global scale
+ * needs the maximum over every shard.  Capture's two passes are then called
+ * separately around an all-reduce(MAX) of the G accumulators (4 bytes per
+ * group; as uint32 the bf16 bit patterns of non-negative values order like
+ * the values, so an integer MAX reduction is exact):
+ *   trace_capture_amax: zeroes amax[G] and writes max|x| per group over
+ *     this shard's rows (bf16 bits in uint32; a group with no rows here
+ *     stays 0).  amax: device uint32[G], 4-byte aligned.
+ *   trace_capture_with_amax: the quantisation pass of trace_capture with
+ *     the given (reduced) amax: gscale[g] = amax/2688 or 1, scales, codes,
+ *     mbits.  scale_layout as trace_capture_ex.
+ * On one GPU, trace_capture_amax followed by trace_capture_with_amax equals
+ * trace_capture.  Group offsets are this shard's, over its own rows. */
+int trace_capture_amax(const uint16_t* x, int64_t rows, int64_t cols,
+                       int32_t num_groups, const int64_t* group_row_offsets,
+                       uint32_t* amax, void* stream);
+int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols,
+                            int32_t num_groups,
+                            const int64_t* group_row_offsets,
+                            const uint32_t* amax, uint8_t* codes,
+                            uint32_t* mbits, uint8_t* scales, float* gscale,
+                            int32_t scale_layout, void* stream);
+
 /* Masked straight-through-estimator backward:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
  *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.

@@ -60,3 +60,44 @@ def test_job_value_counts_every_rank():
     assert bench.job_gbs(4, 1000, 17.3125, 2.0) == pytest.approx(4 * one)
     assert bench.job_gbs(2, 1000, 17.3125, 4.0) == pytest.approx(one)
     assert bench.max_over_ranks([1.5, 2.5], None, "cpu") == [1.5, 2.5]
+
+
+def _amax_worker(rank, world, port, q):
+    """Each rank holds a row shard; the per-group amax (bf16 bit patterns in
+    int32, as trace_capture_amax writes them) is all-reduced with MAX."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import numpy as np
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(100 + rank)
+        vals = np.abs(rng.standard_normal(7).astype(np.float32)) * 10.0 ** rng.integers(-30, 30, 7)
+        vals[rank] = 0.0                                     # a group empty on this shard
+        bits = torch.from_numpy(vals).to(torch.bfloat16).view(torch.int16).to(torch.int32)
+        local = bits.clone()
+        dist.all_reduce(bits, op=dist.ReduceOp.MAX)
+        allv = [torch.zeros(7, dtype=torch.int32) for _ in range(world)]
+        dist.all_gather(allv, local)
+        q.put((rank, bits.tolist(), [a.tolist() for a in allv]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_sharded_amax_reduction():
+    """The one collective of a row-sharded capture: MAX over the bf16 bit
+    patterns equals the bit pattern of the largest magnitude, on every rank."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_amax_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, red, allv in res:
+        for g in range(7):
+            mags = [torch.tensor([a[g]], dtype=torch.int32).to(torch.int16).view(torch.bfloat16).float().item()
+                    for a in allv]
+            want = torch.tensor([max(mags)]).to(torch.bfloat16).view(torch.int16).item()
+            assert red[g] == want

@@ -148,3 +148,43 @@ def test_ex_argument_errors():
     assert lib.trace_scale_bytes(4, 64, 8, 0) == 0 and lib.trace_scale_bytes(4, 64, 16, 5) == 0
     torch.cuda.synchronize()
     assert int(mask.abs().sum()) == 0
+
+
+def test_row_sharded_capture_matches_whole(oracle_mod):
+    """Three row shards of one grouped tensor, captured with the two-pass
+    entry points around a MAX reduction of the per-group amax (done here
+    with torch.maximum on one GPU, as the all-reduce would across GPUs):
+    every shard's outputs equal the oracle's capture of the whole tensor."""
+    s = inputs.tiny_site(21, 600, 256, eps=0.01)
+    x = s.x_roll.float()
+    x[100:250] *= 1e3
+    s.x_roll = x.to(torch.bfloat16)
+    offs = np.array([0, 150, 150, 420, 600], np.int64)
+    G = 4
+    cuts = [0, 200, 333, 600]
+    xd = s.x_roll.to(DEV)
+    amaxes, shards = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        lo = np.clip(offs - a, 0, b - a)
+        o = torch.from_numpy(lo).to(DEV)
+        am = torch.empty(G, dtype=torch.int32, device=DEV)
+        ops.trace_capture_amax(xd[a:b], b - a, 256, G, o, am)
+        amaxes.append(am)
+        shards.append((a, b, o))
+    red = torch.stack(amaxes).max(dim=0).values
+    codes, mbits, scales, gscale = oracle_mod.capture(inputs.bits(s.x_roll), G, offs)
+    for a, b, o in shards:
+        cap, _ = ops.alloc_capture(b - a, 256, G, DEV, o)
+        ops.trace_capture_with_amax(xd[a:b], b - a, 256, G, o, red, cap.codes, cap.mbits,
+                                    cap.scales, cap.gscale)
+        torch.cuda.synchronize()
+        _eq("gscale", _u(cap.gscale).view(np.uint32), gscale.view(np.uint32))
+        _eq("codes", _u(cap.codes), codes[a * 128:b * 128])
+        _eq("mbits", _u(cap.mbits), mbits[a * 8:b * 8])
+        _eq("scales", _u(cap.scales), scales[a:b])
+    # one GPU, no process group: the sharded helper is a whole capture
+    one = ops.capture_sharded(xd, torch.from_numpy(offs).to(DEV))
+    torch.cuda.synchronize()
+    _eq("sharded helper codes", _u(one.codes), codes)
+    _eq("sharded helper scales", _u(one.scales), scales)
+    _eq("sharded helper gscale", _u(one.gscale).view(np.uint32), gscale.view(np.uint32))
