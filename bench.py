@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["trace", "reference"], default="trace")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="time the step as separate launches instead of a CUDA-graph replay")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline leg")
@@ -319,27 +321,46 @@ def run_trace(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None, dom=None):
+    def step(ev=None, dom=None, s=None):
+        s = stream if s is None else s
         for i, w in enumerate(work):
             e = ev[i] if ev else None
             d = dom[i] if dom else None
-            if e: e[0].record(stream)
-            ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], stream)
-            if e: e[1].record(stream)
-            if d: d[0].record(stream)
-            ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], stream)
-            if e: e[2].record(stream)
-            if d: d[1].record(stream)
-            ops.fq_bwd(w["g"], w["mask"], w["gin"], stream)
-            if e: e[3].record(stream)
+            if e: e[0].record(s)
+            ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], s)
+            if e: e[1].record(s)
+            if d: d[0].record(s)
+            ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], s)
+            if e: e[2].record(s)
+            if d: d[1].record(s)
+            ops.fq_bwd(w["g"], w["mask"], w["gin"], s)
+            if e: e[3].record(s)
             ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
-                           w["mask_r"], stream)
-            if e: e[4].record(stream)
+                           w["mask_r"], s)
+            if e: e[4].record(s)
 
     for i in range(max(args.warmup, 3)):
         flush.fill_(i & 0xFF)
         step()
     torch.cuda.synchronize()
+
+    # the step captured once as a CUDA graph (all sites, every kernel of the
+    # path) and replayed per step: one graph launch instead of 6 launches per
+    # site, and no per-launch submission gap between the kernels
+    gph, graph_error = None, None
+    if not args.eager:
+        try:
+            gph = torch.cuda.CUDAGraph()
+            cs = torch.cuda.Stream()
+            cs.wait_stream(stream)
+            with torch.cuda.graph(gph, stream=cs):
+                step(s=cs)
+            torch.cuda.synchronize()
+            for _ in range(max(args.warmup, 3)):
+                gph.replay()
+            torch.cuda.synchronize()
+        except Exception as exc:  # fall back to separate launches, and say so
+            gph, graph_error = None, f"{type(exc).__name__}: {exc}"[:200]
 
     # timed region: one event pair around every step (nothing between the
     # kernels, so each launch can overlap the tail of the previous one)
@@ -353,17 +374,37 @@ def run_trace(args):
     # next launch a little, so these durations are slightly pessimistic)
     kern_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
                for _ in range(args.steps)]
+    eager_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
     with ClockSampler(local) as clk:
+        # timed region 1 (the value): the step, graph-replayed (or eager)
         if pg: pg.barrier()
         torch.cuda.synchronize()
         for k in range(args.steps):
             flush.fill_((k + 7) & 0xFF)
             step_ev[k][0].record(stream)
-            step(dom=dom_ev[k])
+            if gph is not None:
+                gph.replay()
+            else:
+                step(dom=dom_ev[k])
             step_ev[k][1].record(stream)
         torch.cuda.synchronize()
         if pg: pg.barrier()
+        # timed region 2: the same step as separate launches, with the
+        # dominant kernel bracketed by events on its stream (the roofline)
+        if gph is not None:
+            if pg: pg.barrier()
+            torch.cuda.synchronize()
+            for k in range(args.steps):
+                flush.fill_((k + 5) & 0xFF)
+                eager_ev[k][0].record(stream)
+                step(dom=dom_ev[k])
+                eager_ev[k][1].record(stream)
+            torch.cuda.synchronize()
+            if pg: pg.barrier()
     clocks = clk.summary()
+    if gph is not None:
+        del gph
     for k in range(args.steps):          # breakdown pass, outside the timed region
         flush.fill_((k + 11) & 0xFF)
         step(kern_ev[k])
@@ -493,6 +534,9 @@ def run_trace(args):
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
     per_kernel = {nm: 0.0 for nm in names}
     total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    eager_ms = (sum(a.elapsed_time(b) for a, b in eager_ev) if graph_error is None and not args.eager
+                else total_ms)
+    eager_ms = max_over_ranks([eager_ms], pg, dev)[0]
     dom_ms = sum(a.elapsed_time(b) for per in dom_ev for a, b in per)
     for per in kern_ev:
         for ev in per:
@@ -531,20 +575,20 @@ def run_trace(args):
         "adjacent_frac_of_disagreements": [round(r[1] / max(1, tot - r[0]), 6) for r in hist_counts],
         "counts": hist_counts}
     mx_rows = {}
-    for j, (nm, kn, bpe) in enumerate([("capture", "k_mx_capture", 2.65625),
+    for j, (nm, kn, b_k) in enumerate([("capture", "k_mx_capture", 2.65625),
                                        ("guided_fwd", "k_mx_fake_quant<1>", 4.28125),
                                        ("rtn_fwd", "k_mx_fake_quant<0>", 4.15625),
                                        ("full_guided_fwd", "k_mx_fake_quant<2>", 4.65625)]):
         ms = mx_ms[j] / args.steps
-        mx_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": bpe,
-                       "gbs": round(n * bpe / (ms * 1e-3) / 1e9, 1),
-                       "frac_of_hbm": round(n * bpe / (ms * 1e-3) / 1e9 / hbm, 4)}
+        mx_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": b_k,
+                       "gbs": round(n * b_k / (ms * 1e-3) / 1e9, 1),
+                       "frac_of_hbm": round(n * b_k / (ms * 1e-3) / 1e9 / hbm, 4)}
     next_rows["mxfp4"] = mx_rows
     next_rows["tiled_scales"] = {
-        nm: {"kernel": kn, "us": round(tl_ms[j] / args.steps * 1e3, 2), "bytes_per_elem": bpe,
-             "gbs": round(n * bpe / (tl_ms[j] / args.steps * 1e-3) / 1e9, 1),
-             "frac_of_hbm": round(n * bpe / (tl_ms[j] / args.steps * 1e-3) / 1e9 / hbm, 4)}
-        for j, (nm, kn, bpe) in enumerate([("capture", "k_amax + k_capture<true>", 4.6875),
+        nm: {"kernel": kn, "us": round(tl_ms[j] / args.steps * 1e3, 2), "bytes_per_elem": b_k,
+             "gbs": round(n * b_k / (tl_ms[j] / args.steps * 1e-3) / 1e9, 1),
+             "frac_of_hbm": round(n * b_k / (tl_ms[j] / args.steps * 1e-3) / 1e9 / hbm, 4)}
+        for j, (nm, kn, b_k) in enumerate([("capture", "k_amax + k_capture<true>", 4.6875),
                                            ("guided_fwd", "k_fake_quant<1, true>", 4.3125)])}
     cms, tms = tier_compute_ms / args.steps, tier_total_ms / args.steps
     next_rows["cache_tier"] = {
@@ -637,6 +681,9 @@ def run_trace(args):
         "config": {"workload": workload, "shapes": shapes, "groups": groups,
                    "step": "capture + guided fwd + STE bwd + RTN fwd",
                    "l2": "flushed before every step (256 MiB write)",
+                   "launch": ("CUDA graph of the whole step, captured once and replayed"
+                              if graph_error is None and not args.eager else
+                              "separate launches (programmatic stream serialization)"),
                    "parallelism": f"{world} independent sites, one per GPU (no collective)"},
         "kernels": kern,
         "yardstick": yardstick,
@@ -649,8 +696,11 @@ def run_trace(args):
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": LAUNCHES_PER_STEP * len(work) * args.steps,
-        "timing": ("value: events around each step only; kernels: a second, untimed pass of "
-                   "the same steps with events between the calls"),
+        "eager_ms_per_step": round(eager_ms / args.steps, 5),
+        "graph_error": graph_error,
+        "timing": ("value: events around each step (graph replay) only; roofline: events around "
+                   "the guided forward in a second timed pass of eager steps; kernels: a third, "
+                   "untimed pass with events between the calls"),
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -394,3 +394,41 @@ def test_argument_errors_enqueue_nothing():
                              P(cap.gscale), P(ws), ws.numel(), None) == 1
     assert lib.trace_fq_bwd(P(x), P(cap.mbits), 48, P(x), None) == 2
     torch.cuda.synchronize()
+
+
+def test_step_in_a_cuda_graph(oracle_mod):
+    """The library's launches (with programmatic stream serialization) can be
+    captured into a CUDA graph: a captured capture -> guided -> bwd -> RTN step
+    replays to the oracle's outputs, also on new inputs copied into the same
+    buffers."""
+    s = inputs.tiny_site(61, 640, 512, eps=0.01)
+    xr, xt, g = (t.to(DEV) for t in (s.x_roll, s.x_train, s.grad))
+    cap, ws = ops.alloc_capture(640, 512)
+    out = torch.empty_like(xt)
+    mask = torch.empty(640 * 512 // 32, dtype=torch.int32, device=DEV)
+    gin = torch.empty_like(g)
+    out_r = torch.empty_like(xt)
+    mask_r = torch.empty_like(mask)
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph, stream=cs):
+        ops.capture(xr, None, cap, ws, cs)
+        ops.guided_fq_fwd(xt, cap, out, mask, cs)
+        ops.fq_bwd(g, mask, gin, cs)
+        ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, None, out_r, mask_r, cs)
+    for seed in (61, 62):
+        if seed == 62:
+            s = inputs.tiny_site(seed, 640, 512, eps=0.03)
+            xr.copy_(s.x_roll.to(DEV))
+            xt.copy_(s.x_train.to(DEV))
+            g.copy_(s.grad.to(DEV))
+        gph.replay()
+        torch.cuda.synchronize()
+        ref = run_oracle(oracle_mod, s)
+        got = dict(codes=_u(cap.codes), mbits=_u(cap.mbits), scales=_u(cap.scales),
+                   gscale=_u(cap.gscale), out=_u(out), mask=_u(mask), grad_in=_u(gin),
+                   out_rtn=_u(out_r), mask_rtn=_u(mask_r))
+        for k in got:
+            _eq(f"graph.{seed}.{k}", got[k], ref[k])
+    del gph
