@@ -695,7 +695,10 @@ def run_trace(args):
                      "algorithmic_bytes": int(dom_bytes)},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": LAUNCHES_PER_STEP * len(work) * args.steps,
+        # the graph replays launch the same kernels as separate steps do;
+        # with the graph there is also the eager pass for the roofline
+        "gpu_launches": LAUNCHES_PER_STEP * len(work) * args.steps *
+                        (2 if graph_error is None and not args.eager else 1),
         "eager_ms_per_step": round(eager_ms / args.steps, 5),
         "graph_error": graph_error,
         "timing": ("value: events around each step (graph replay) only; roofline: events around "
