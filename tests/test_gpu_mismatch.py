@@ -165,6 +165,12 @@ def test_hist_cfg2_full(oracle_mod):
     # use the rollout agree with it more often than round to nearest
     assert got[0, 1] > 0 and got[0, 2:].sum() < got[0, 1] // 100
     assert got[1, 0] > got[0, 0] and got[2, 0] >= got[1, 0]
+    # at 0.5% drift q_roll always lies in the bracket of z_train: leaving it
+    # takes a relative move of at least 1/7 (from just under the midpoint
+    # 1.75 up to the codeword 2, or 3.5 up to 4), about 29 standard
+    # deviations here; full guidance then reproduces every rollout code, and
+    # so does the 1-bit cache
+    assert got[2, 0] == got[2].sum() and got[1, 0] == got[1].sum()
 
 
 def test_hist_cfg3_and_cfg4(oracle_mod):
@@ -199,6 +205,7 @@ def test_hist_cfg5_sampled_and_additive(oracle_mod, layer, site):
     rg = np.full(rows_idx.size, gs[0], np.float32)
     codes, _, scales = oracle_mod.capture_rows(xr_b[rows_idx], rg)
     ref = oracle_mod.mismatch_histogram(np.ascontiguousarray(xt_b[rows_idx]), codes, scales, gs)
+    assert whole[2, 0] == R * C          # no q_roll outside its bracket at 0.5% drift
     acc.zero_()
     for r in rows_idx:
         x1, c1 = _row_slices(xt, cap, int(r), int(r) + 1, 0)
