@@ -63,6 +63,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["trace", "reference"], default="trace")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=8,
+                    help="row chunks of the host-to-host step (copies overlap compute)")
     ap.add_argument("--eager", action="store_true",
                     help="time the step as separate launches instead of a CUDA-graph replay")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -631,17 +633,22 @@ def run_trace(args):
     # --- end-to-end through the C ABI with pinned host buffers -------------
     e2e = None
     if not args.no_e2e and args.config == 2:
-        ins = [(w[k], w[k].cpu().pin_memory()) for w in work for k in ("xr", "xt", "g")]
-        outs = [(d, torch.empty(d.shape, dtype=d.dtype).pin_memory()) for w in work
-                for d in (w["cap"].codes, w["cap"].mbits, w["cap"].scales, w["cap"].gscale,
-                          w["out"], w["mask"], w["gin"], w["out_r"], w["mask_r"])]
+        # through the public host-to-host API: inputs from pinned host memory,
+        # every output back to it, the copies overlapped with the kernels in
+        # row chunks (host_step.HostStep)
+        from fp4_quantization_aware_trace_b200 import host_step
+        hs = []
+        for w in work:
+            R, C = w["xr"].shape
+            offs_h = None if w["offs"] is None else w["offs"].cpu()
+            h = host_step.HostStep(R, C, offs_h, chunks=args.e2e_chunks, device=dev)
+            hs.append((h, [w[k].cpu().pin_memory() for k in ("xr", "xt", "g")], h.alloc_host()))
+        ins = [t for _, i, _ in hs for t in i]
+        outs = [t for _, _, o in hs for t in o.values()]
 
         def e2e_step():
-            for d, h in ins:
-                d.copy_(h, non_blocking=True)
-            step()
-            for d, h in outs:
-                h.copy_(d, non_blocking=True)
+            for h, (xr_h, xt_h, g_h), out_h in hs:
+                h.run(xr_h, xt_h, g_h, out_h, stream)
 
         for _ in range(3):
             e2e_step()
@@ -654,10 +661,11 @@ def run_trace(args):
         e1.record(stream)
         torch.cuda.synchronize()
         e2e_ms = max_over_ranks([e0.elapsed_time(e1)], pg, dev)[0] / args.steps
-        h2d = sum(h.numel() * h.element_size() for _, h in ins)
-        d2h = sum(h.numel() * h.element_size() for _, h in outs)
+        h2d = sum(t.numel() * t.element_size() for t in ins)
+        d2h = sum(t.numel() * t.element_size() for t in outs)
         e2e = {"value": round(job_gbs(world, n, bpe, e2e_ms), 3), "unit": "GB/s",
                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "api": f"host_step.HostStep.run, {len(hs[0][0].cuts)} row chunks",
                "elem_per_s": round(world * n / (e2e_ms * 1e-3), 1)}
 
     cpu = None

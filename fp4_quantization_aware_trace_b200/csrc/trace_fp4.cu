@@ -1490,6 +1490,21 @@ int trace_capture_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t nu
                 amax);
 }
 
+int trace_capture_amax_accumulate(const uint16_t* x, int64_t rows, int64_t cols,
+                                  int32_t num_groups, const int64_t* group_row_offsets,
+                                  uint32_t* amax, void* stream) {
+  int st = check_shape(rows, cols, num_groups, group_row_offsets);
+  if (st) return st;
+  if ((rows > 0 && !x) || !amax) return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || !aligned(amax, 4)) return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, num_groups);
+  if (sh.nblk == 0) return TRACE_OK;
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  return launch(k_amax, grid, (cudaStream_t)stream, (const V8*)x, sh,
+                num_groups > 1 ? group_row_offsets : nullptr, amax);
+}
+
 int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                             const int64_t* group_row_offsets, const uint32_t* amax,
                             uint8_t* codes, uint32_t* mbits, uint8_t* scales, float* gscale,

@@ -86,6 +86,8 @@ def library() -> ctypes.CDLL:
         lib.trace_mx_fq_fwd_ex.restype = ctypes.c_int
         lib.trace_capture_amax.argtypes = [P, i64, i64, i32, P, P, P]
         lib.trace_capture_amax.restype = ctypes.c_int
+        lib.trace_capture_amax_accumulate.argtypes = [P, i64, i64, i32, P, P, P]
+        lib.trace_capture_amax_accumulate.restype = ctypes.c_int
         lib.trace_capture_with_amax.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, i32, P]
         lib.trace_capture_with_amax.restype = ctypes.c_int
         _lib = lib
@@ -455,6 +457,12 @@ def mx_fq_fwd_tiled(rule: int, x_train: torch.Tensor, cache: MxCapture, out=None
 def trace_capture_amax(x, rows, cols, num_groups, offsets, amax, stream=None) -> None:
     _check(library().trace_capture_amax(_p(x), rows, cols, num_groups, _p(offsets), _p(amax),
                                         _stream(stream)), "trace_capture_amax")
+
+
+def trace_capture_amax_accumulate(x, rows, cols, num_groups, offsets, amax, stream=None) -> None:
+    _check(library().trace_capture_amax_accumulate(_p(x), rows, cols, num_groups, _p(offsets),
+                                                   _p(amax), _stream(stream)),
+           "trace_capture_amax_accumulate")
 
 
 def trace_capture_with_amax(x, rows, cols, num_groups, offsets, amax, codes, mbits, scales,

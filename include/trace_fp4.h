@@ -272,11 +272,20 @@ int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows,
  *   trace_capture_with_amax: the quantisation pass of trace_capture with
  *     the given (reduced) amax: gscale[g] = amax/2688 or 1, scales, codes,
  *     mbits.  scale_layout as trace_capture_ex.
+ *   trace_capture_amax_accumulate: as trace_capture_amax without the
+ *     zeroing: max-accumulates this part's maxima into amax, so a tensor that
+ *     arrives in row chunks (e.g. copied from the host chunk by chunk) gets
+ *     its whole-tensor amax from one trace_capture_amax on the first chunk
+ *     and this call on the others.
  * On one GPU, trace_capture_amax followed by trace_capture_with_amax equals
  * trace_capture.  Group offsets are this shard's, over its own rows. */
 int trace_capture_amax(const uint16_t* x, int64_t rows, int64_t cols,
                        int32_t num_groups, const int64_t* group_row_offsets,
                        uint32_t* amax, void* stream);
+int trace_capture_amax_accumulate(const uint16_t* x, int64_t rows,
+                                  int64_t cols, int32_t num_groups,
+                                  const int64_t* group_row_offsets,
+                                  uint32_t* amax, void* stream);
 int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols,
                             int32_t num_groups,
                             const int64_t* group_row_offsets,

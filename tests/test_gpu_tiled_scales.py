@@ -188,3 +188,36 @@ def test_row_sharded_capture_matches_whole(oracle_mod):
     _eq("sharded helper codes", _u(one.codes), codes)
     _eq("sharded helper scales", _u(one.scales), scales)
     _eq("sharded helper gscale", _u(one.gscale).view(np.uint32), gscale.view(np.uint32))
+
+
+@pytest.mark.parametrize("rows,cols,chunks,grouped", [(600, 256, 4, True), (1000, 96, 3, False),
+                                                       (16384, 2048, 4, False)])
+def test_host_step_matches_oracle(oracle_mod, rows, cols, chunks, grouped):
+    """The host-to-host step (row chunks, amax accumulated across chunks,
+    copies overlapped on three streams) returns the oracle's outputs."""
+    from fp4_quantization_aware_trace_b200 import host_step
+    if rows == 16384:
+        s = inputs.attention_input()
+    else:
+        s = inputs.tiny_site(rows + cols, rows, cols, eps=0.01)
+    offs = np.array([0, rows // 5, rows // 5, rows * 3 // 4, rows], np.int64) if grouped else None
+    G = 4 if grouped else 1
+    h = host_step.HostStep(rows, cols, offs, chunks=chunks)
+    assert len(h.cuts) >= 2
+    xr_h, xt_h, g_h = (t.contiguous().pin_memory() for t in (s.x_roll, s.x_train, s.grad))
+    out_h = h.alloc_host()
+    for _ in range(2):                       # twice: buffers are reused
+        h.run(xr_h, xt_h, g_h, out_h)
+        torch.cuda.synchronize()
+    xr, xt, g = inputs.bits(s.x_roll), inputs.bits(s.x_train), inputs.bits(s.grad)
+    codes, mbits, scales, gscale = oracle_mod.capture(xr, G, offs)
+    out, mask = oracle_mod.guided_fwd(xt, mbits, scales, gscale, G, offs)
+    out_r, mask_r = oracle_mod.rtn_fwd(xt, scales, gscale, G, offs)
+    gin = oracle_mod.fq_bwd(g, mask)
+    ref = dict(codes=codes, mbits=mbits, scales=scales, gscale=gscale, out=out, mask=mask,
+               grad_in=gin, out_rtn=out_r, mask_rtn=mask_r)
+    for k, v in ref.items():
+        got = _u(out_h[k])
+        if k == "gscale":
+            got, v = got.view(np.uint32), v.view(np.uint32)
+        _eq(f"host step {k}", got, v)
