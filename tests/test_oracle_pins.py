@@ -688,3 +688,32 @@ def test_swizzle_scales_is_a_padded_permutation(oracle_mod):
     assert got.size == 384 * 40
     assert np.count_nonzero(got) == rows * scols
     assert np.array_equal(np.sort(got[got != 0]), np.sort(lin.reshape(-1)))
+
+
+def test_mismatch_distance_by_grid_index(oracle_mod):
+    """The ladder distance equals the number of steps between the two values
+    in the sorted list of the 15 signed E2M1 codewords (+0 and -0 one point),
+    on independent rollout / training values, so that opposite signs and long
+    distances occur."""
+    rng = np.random.default_rng(77)
+    xr = rng.standard_normal((16, 256)).astype(np.float32) * np.exp(rng.standard_normal((16, 256)))
+    xt = rng.standard_normal((16, 256)).astype(np.float32) * np.exp(rng.standard_normal((16, 256)))
+    xr_b = inputs.bits(torch.from_numpy(xr).to(torch.bfloat16))
+    xt_b = inputs.bits(torch.from_numpy(xt).to(torch.bfloat16))
+    codes, mbits, scales, gscale = oracle_mod.capture(xr_b)
+    hist = oracle_mod.mismatch_histogram(xt_b, codes, scales, gscale)
+    grid = [float(v) for v, _ in bf.SIGNED_GRID]          # ascending, 15 points
+    assert len(grid) == 15
+
+    def index(c):
+        v = float(Fraction(bf._MAGS[c & 7])) * (-1.0 if c & 8 else 1.0)
+        return grid.index(v + 0.0)                           # -0.0 -> +0.0
+
+    q_roll = oracle_mod.unpack_codes(codes)
+    rules = [oracle_mod.fake_quant_codes(xt_b, scales, gscale, None).reshape(-1),
+             oracle_mod.fake_quant_codes(xt_b, scales, gscale, mbits).reshape(-1),
+             oracle_mod.full_guided_codes(xt_b, codes, scales, gscale).reshape(-1)]
+    for k in range(3):
+        d = np.array([abs(index(int(a)) - index(int(b))) for a, b in zip(rules[k], q_roll)])
+        assert np.array_equal(hist[k], np.bincount(d, minlength=15)), k
+    assert hist[0, 2:].sum() > 0 and np.count_nonzero(hist[0]) > 5   # long distances occur
