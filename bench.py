@@ -355,7 +355,9 @@ def run_trace(args):
             gph = torch.cuda.CUDAGraph()
             cs = torch.cuda.Stream()
             cs.wait_stream(stream)
-            with torch.cuda.graph(gph, stream=cs):
+            # thread-local: other threads' CUDA calls (e.g. a process group's
+            # watchdog) must not invalidate the capture
+            with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
                 step(s=cs)
             torch.cuda.synchronize()
             for _ in range(max(args.warmup, 3)):

@@ -412,7 +412,7 @@ def test_step_in_a_cuda_graph(oracle_mod):
     cs = torch.cuda.Stream()
     cs.wait_stream(torch.cuda.current_stream())
     gph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(gph, stream=cs):
+    with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
         ops.capture(xr, None, cap, ws, cs)
         ops.guided_fq_fwd(xt, cap, out, mask, cs)
         ops.fq_bwd(g, mask, gin, cs)
