@@ -114,6 +114,24 @@ def _load():
         lib.oracle_mx_full_guided_fwd.restype = None
         lib.oracle_mx_fake_quant_codes.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int]
         lib.oracle_mx_fake_quant_codes.restype = None
+        lib.oracle_mx8_scale.argtypes = [ctypes.c_float]
+        lib.oracle_mx8_scale.restype = ctypes.c_uint8
+        lib.oracle_e4m3_bracket.argtypes = [ctypes.c_float, P, P]
+        lib.oracle_e4m3_bracket.restype = None
+        lib.oracle_e4m3_guided_code.argtypes = [ctypes.c_float, ctypes.c_int]
+        lib.oracle_e4m3_guided_code.restype = ctypes.c_int
+        lib.oracle_e4m3_full_guided_code.argtypes = [ctypes.c_float, ctypes.c_int]
+        lib.oracle_e4m3_full_guided_code.restype = ctypes.c_int
+        lib.oracle_mx8_capture.argtypes = [P, i64, i64, P, P, P]
+        lib.oracle_mx8_capture.restype = None
+        lib.oracle_mx8_guided_fwd.argtypes = [P, i64, i64, P, P, P, P]
+        lib.oracle_mx8_guided_fwd.restype = None
+        lib.oracle_mx8_rtn_fwd.argtypes = [P, i64, i64, P, P, P]
+        lib.oracle_mx8_rtn_fwd.restype = None
+        lib.oracle_mx8_full_guided_fwd.argtypes = [P, i64, i64, P, P, P, P]
+        lib.oracle_mx8_full_guided_fwd.restype = None
+        lib.oracle_mx8_fake_quant_codes.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int]
+        lib.oracle_mx8_fake_quant_codes.restype = None
         lib.oracle_swizzled_scale_bytes.argtypes = [i64, i64]
         lib.oracle_swizzled_scale_bytes.restype = i64
         lib.oracle_swizzle_scales.argtypes = [P, i64, i64, P]
@@ -473,3 +491,62 @@ def swizzle_scales(scales) -> np.ndarray:
     out = np.zeros(swizzled_scale_bytes(rows, scols), np.uint8)
     _load().oracle_swizzle_scales(_ptr(lin), rows, scols, _ptr(out))
     return out
+
+
+# -- W4A8: E4M3 activations with MX scales --------------------------------------
+
+def mx8_scale(amax: float) -> int:
+    return int(_load().oracle_mx8_scale(float(amax)))
+
+
+def e4m3_bracket(a: float) -> tuple[int, int]:
+    lo, hi = ctypes.c_int(0), ctypes.c_int(0)
+    _load().oracle_e4m3_bracket(float(a), ctypes.byref(lo), ctypes.byref(hi))
+    return lo.value, hi.value
+
+
+def e4m3_guided_code(a: float, bit: int) -> int:
+    return int(_load().oracle_e4m3_guided_code(float(a), int(bit)))
+
+
+def e4m3_full_guided_code(z: float, roll_code: int) -> int:
+    return int(_load().oracle_e4m3_full_guided_code(float(z), int(roll_code)))
+
+
+def mx8_capture(x_roll):
+    """(codes uint8[N], mbits uint32[N/32], scales uint8[rows, cols/32])."""
+    x = _as_bf16_bits(x_roll)
+    rows, cols = x.shape
+    n = rows * cols
+    codes = np.zeros(n, np.uint8)
+    mbits = np.zeros(n // 32, np.uint32)
+    scales = np.zeros((rows, cols // 32), np.uint8)
+    _load().oracle_mx8_capture(_ptr(x), rows, cols, _ptr(codes), _ptr(mbits), _ptr(scales))
+    return codes, mbits, scales
+
+
+def mx8_guided_fwd(x_train, mbits, scales):
+    return _mx_fwd(_load().oracle_mx8_guided_fwd, x_train,
+                   np.ascontiguousarray(mbits, dtype=np.uint32), scales)
+
+
+def mx8_rtn_fwd(x, scales):
+    return _mx_fwd(_load().oracle_mx8_rtn_fwd, x, None, scales)
+
+
+def mx8_full_guided_fwd(x_train, rcodes, scales):
+    return _mx_fwd(_load().oracle_mx8_full_guided_fwd, x_train,
+                   np.ascontiguousarray(rcodes, dtype=np.uint8), scales)
+
+
+def mx8_fake_quant_codes(x, scales, mbits=None, rcodes=None):
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    sites = np.zeros(rows * cols, np.uint8)
+    mode = 1 if mbits is not None else (2 if rcodes is not None else 0)
+    mb = None if mbits is None else np.ascontiguousarray(mbits, dtype=np.uint32)
+    rc = None if rcodes is None else np.ascontiguousarray(rcodes, dtype=np.uint8)
+    _load().oracle_mx8_fake_quant_codes(_ptr(x), rows, cols, _ptr(mb), _ptr(rc),
+                                        _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
+                                        _ptr(sites), mode)
+    return sites.reshape(rows, cols)

@@ -21,9 +21,10 @@
  * format the post's rollout runs in; the pages name NVFP4 but do not spell
  * it out, so the readings taken here are listed at each step.
  *
- * The MXFP4 variant at the end of the file (the post's results list: the
+ * The MXFP4 variant near the end of the file (the post's results list: the
  * method carries over to MXFP4 W4A4) swaps the scale step for the OCP
- * Microscaling one; the rounding rules on the E2M1 grid are unchanged.
+ * Microscaling one; the rounding rules on the E2M1 grid are unchanged.  The
+ * W4A8 variant after it applies the same rules to E4M3 (FP8) activations.
  *
  * Every floating-point operation below is ONE IEEE-754 binary32 operation
  * with round-to-nearest-even.  Build with -ffp-contract=off and without
@@ -632,4 +633,149 @@ void oracle_swizzle_scales(const uint8_t* lin, int64_t rows, int64_t scols,
       out[tile * 512 + 16 * (rr % 32) + 4 * (rr / 32) + cc] = lin[r * scols + c];
     }
   }
+}
+
+/* ------------------------------------------------------------------ */
+/* W4A8: TRACE on FP8 activations with MX scales (MXFP8)                */
+/*                                                                      */
+/* The results list names the W4A8 setting beside MXFP4 W4A4.  With     */
+/* 8-bit activations the elements are E4M3 (the OCP MX FP8 element that  */
+/* carries mantissa bits) in 32-element blocks with an E8M0 scale        */
+/* X = 2^e, e = floor(log2 max|x|) - 8 (8 is the exponent of E4M3's      */
+/* largest value 448 = 1.75 * 2^8), clamped to [-127, 127] (-127 for an  */
+/* all-zero block).  z = x / X, clipped to [-448, 448]; round to nearest */
+/* E4M3 with ties to the even mantissa; the code is one byte (sign bit 7, */
+/* magnitude 0..0x7E); the cached bit is the lowest bit of the magnitude */
+/* code (its mantissa's last bit); the STE mask is |z| <= 448.  The      */
+/* bracket and the two guided choices are those of the E2M1 path on the  */
+/* E4M3 grid, whose neighbouring codes also alternate that bit.          */
+/* ------------------------------------------------------------------ */
+
+uint8_t oracle_mx8_scale(float amax) {
+  int e = -127;
+  if (amax != 0.0f) {
+    int k;
+    (void)frexpf(amax, &k);
+    e = (k - 1) - 8;
+    if (e < -127) e = -127;
+    if (e > 127) e = 127;
+  }
+  return (uint8_t)(e + 127);
+}
+
+/* The E4M3 codes around a in [0, 448]: the largest with value <= a and the
+ * smallest with value >= a (by scanning the 127 finite magnitudes). */
+void oracle_e4m3_bracket(float a, int* lo, int* hi) {
+  assert(a >= 0.0f && a <= 448.0f);
+  int l = 0, h = 0x7E;
+  for (int c = 0; c <= 0x7E; ++c)
+    if (oracle_e4m3_to_f32((uint8_t)c) <= a) l = c;
+  for (int c = 0x7E; c >= 0; --c)
+    if (oracle_e4m3_to_f32((uint8_t)c) >= a) h = c;
+  *lo = l;
+  *hi = h;
+}
+
+int oracle_e4m3_guided_code(float a, int bit) {
+  int lo, hi;
+  oracle_e4m3_bracket(a, &lo, &hi);
+  if (lo == hi) return lo;
+  return ((lo & 1) == (bit & 1)) ? lo : hi;
+}
+
+/* z unclipped; roll_code: the rollout's E4M3 byte (sign bit 7). */
+int oracle_e4m3_full_guided_code(float z, int roll_code) {
+  float a = fabsf(z);
+  if (a > 448.0f) a = 448.0f;
+  int lo, hi;
+  oracle_e4m3_bracket(a, &lo, &hi);
+  const float s = signbit(z) ? -1.0f : 1.0f;
+  const float q_lo = s * oracle_e4m3_to_f32((uint8_t)lo), q_hi = s * oracle_e4m3_to_f32((uint8_t)hi);
+  const float q_roll = ((roll_code & 0x80) ? -1.0f : 1.0f) *
+                       oracle_e4m3_to_f32((uint8_t)(roll_code & 0x7F));
+  return (fabsf(q_hi - q_roll) < fabsf(q_lo - q_roll)) ? hi : lo;
+}
+
+/* MXFP8 capture: codes uint8[N] (element i = byte i), mbits, E8M0 scales
+ * [rows, cols/32]. */
+void oracle_mx8_capture(const uint16_t* x, int64_t rows, int64_t cols,
+                        uint8_t* codes, uint32_t* mbits, uint8_t* scales) {
+  assert(cols % 32 == 0);
+  const int64_t n = rows * cols;
+  memset(mbits, 0, (size_t)(n / 32) * sizeof(uint32_t));
+  for (int64_t b = 0; b < n / 32; ++b) {
+    float bmax = 0.0f;
+    for (int j = 0; j < 32; ++j) {
+      const float a = fabsf(oracle_bf16_to_f32(x[b * 32 + j]));
+      if (a > bmax) bmax = a;
+    }
+    scales[b] = oracle_mx8_scale(bmax);
+    const float X = oracle_e8m0_to_f32(scales[b]);
+    for (int j = 0; j < 32; ++j) {
+      const int64_t i = b * 32 + j;
+      const float z = oracle_bf16_to_f32(x[i]) / X;
+      float a = fabsf(z);
+      if (a > 448.0f) a = 448.0f;
+      const int c = oracle_f32_to_e4m3(a);
+      codes[i] = (uint8_t)((signbit(z) ? 0x80 : 0) | c);
+      mbits[i / 32] |= (uint32_t)(c & 1) << (i & 31);
+    }
+  }
+}
+
+static void mx8_fake_quant(const uint16_t* x, int64_t rows, int64_t cols,
+                           const uint32_t* mbits, const uint8_t* rcodes,
+                           const uint8_t* scales, uint16_t* out, uint32_t* mask,
+                           uint8_t* sites, int mode) {
+  assert(cols % 32 == 0);
+  const int64_t n = rows * cols;
+  if (mask) memset(mask, 0, (size_t)(n / 32) * sizeof(uint32_t));
+  for (int64_t b = 0; b < n / 32; ++b) {
+    const float X = oracle_e8m0_to_f32(scales[b]);
+    for (int j = 0; j < 32; ++j) {
+      const int64_t i = b * 32 + j;
+      const float xv = oracle_bf16_to_f32(x[i]);
+      assert(isfinite(xv));
+      const float z = xv / X;
+      float a = fabsf(z);
+      if (mask && a <= 448.0f) mask[i / 32] |= 1u << (i & 31);
+      if (a > 448.0f) a = 448.0f;
+      int c;
+      if (mode == FQ_GUIDED)
+        c = oracle_e4m3_guided_code(a, (int)((mbits[i / 32] >> (i & 31)) & 1u));
+      else if (mode == FQ_FULL)
+        c = oracle_e4m3_full_guided_code(z, rcodes[i]);
+      else
+        c = oracle_f32_to_e4m3(a);
+      if (out) {
+        float v = oracle_e4m3_to_f32((uint8_t)c) * X; /* exact: 4 significant bits */
+        if (signbit(z)) v = -v;
+        out[i] = oracle_f32_to_bf16(v);
+      }
+      if (sites) sites[i] = (uint8_t)((signbit(z) ? 0x80 : 0) | c);
+    }
+  }
+}
+
+void oracle_mx8_guided_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                           const uint32_t* mbits, const uint8_t* scales,
+                           uint16_t* out, uint32_t* mask) {
+  mx8_fake_quant(x, rows, cols, mbits, 0, scales, out, mask, 0, FQ_GUIDED);
+}
+
+void oracle_mx8_rtn_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                        const uint8_t* scales, uint16_t* out, uint32_t* mask) {
+  mx8_fake_quant(x, rows, cols, 0, 0, scales, out, mask, 0, FQ_RTN);
+}
+
+void oracle_mx8_full_guided_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                                const uint8_t* rcodes, const uint8_t* scales,
+                                uint16_t* out, uint32_t* mask) {
+  mx8_fake_quant(x, rows, cols, 0, rcodes, scales, out, mask, 0, FQ_FULL);
+}
+
+void oracle_mx8_fake_quant_codes(const uint16_t* x, int64_t rows, int64_t cols,
+                                 const uint32_t* mbits, const uint8_t* rcodes,
+                                 const uint8_t* scales, uint8_t* sites, int mode) {
+  mx8_fake_quant(x, rows, cols, mbits, rcodes, scales, 0, 0, sites, mode);
 }

@@ -238,3 +238,84 @@ def brute_mx_pipeline(x_roll: np.ndarray, x_train: np.ndarray):
             outs["out_full"][i] = deq(brute_full_guided(z, rv)[0], neg, Xq)
     return dict(codes=codes, mbits=mbits, scales=scales.reshape(rows, cols // 32), mask=mask,
                 **{k: v.reshape(rows, cols) for k, v in outs.items()})
+
+
+# ---------------------------------------------------------------------------
+# W4A8: E4M3 (FP8) activations with MX scales
+# ---------------------------------------------------------------------------
+
+def brute_mx8_scale(amax: Fraction) -> int:
+    """The E8M0 byte putting amax / X in [256, 512) (E4M3's top binade), by
+    search over all bytes; the smallest byte when none does (or amax = 0)."""
+    if amax == 0:
+        return 0
+    hits = [b for b in range(255) if 256 <= amax / e8m0_value(b) < 512]
+    assert len(hits) <= 1
+    return hits[0] if hits else 0
+
+
+def brute_e4m3_rtn(a: Fraction) -> int:
+    """Nearest E4M3 magnitude code to clip(a, 448), ties to the even code."""
+    a = min(a, Fraction(448))
+    best = None
+    for v, b in E4M3_TABLE:
+        d = abs(a - v)
+        if best is None or d < best[0] or (d == best[0] and (b & 1) == 0):
+            best = (d, b)
+    return best[1]
+
+
+def brute_e4m3_bracket(a: Fraction) -> tuple[int, int]:
+    a = min(a, Fraction(448))
+    lo = max((t for t in E4M3_TABLE if t[0] <= a), key=lambda t: t[0])[1]
+    hi = min((t for t in E4M3_TABLE if t[0] >= a), key=lambda t: t[0])[1]
+    return lo, hi
+
+
+def brute_mx8_pipeline(x_roll: np.ndarray, x_train: np.ndarray):
+    """MXFP8 capture on x_roll, then guided / RTN / full-guided forwards of
+    x_train, by exhaustive searches over the E4M3 values."""
+    rows, cols = x_roll.shape
+    n = rows * cols
+    xr = [bf16_bits_to_float(int(h)) for h in x_roll.reshape(-1)]
+    xt = [bf16_bits_to_float(int(h)) for h in x_train.reshape(-1)]
+    codes = np.zeros(n, np.uint8)
+    mbits = np.zeros(n // 32, np.uint32)
+    scales = np.zeros(n // 32, np.uint8)
+    outs = {k: np.zeros(n, np.uint16) for k in ("out_guided", "out_rtn", "out_full")}
+    mask = np.zeros(n // 32, np.uint32)
+
+    def deq(code: int, neg: bool, X: Fraction) -> int:
+        v = f32(float(e4m3_value(code) * X))      # exact
+        return float_to_bf16_bits(-v if neg else v)
+
+    for b in range(n // 32):
+        blk = range(32 * b, 32 * b + 32)
+        sb = brute_mx8_scale(max(Fraction(abs(xr[i])) for i in blk))
+        scales[b] = sb
+        Xq = e8m0_value(sb)
+        X = f32(float(Xq))
+        for i in blk:
+            z = f32(xr[i]) / X
+            c = brute_e4m3_rtn(Fraction(float(abs(z))))
+            codes[i] = (0x80 if np.signbit(z) else 0) | c
+            mbits[i // 32] |= (c & 1) << (i & 31)
+        for i in blk:
+            z = f32(xt[i]) / X
+            neg = bool(np.signbit(z))
+            a = Fraction(float(abs(z)))
+            if a <= 448:
+                mask[i // 32] |= 1 << (i & 31)
+            lo, hi = brute_e4m3_bracket(a)
+            bit = (int(mbits[i // 32]) >> (i & 31)) & 1
+            g = lo if lo == hi or (lo & 1) == bit else hi
+            rc = int(codes[i])
+            rv = e4m3_value(rc & 0x7F) * (-1 if rc & 0x80 else 1)
+            s = -1 if neg else 1
+            dl, dh = abs(s * e4m3_value(lo) - rv), abs(s * e4m3_value(hi) - rv)
+            full = hi if dh < dl else lo
+            outs["out_guided"][i] = deq(g, neg, Xq)
+            outs["out_rtn"][i] = deq(brute_e4m3_rtn(a), neg, Xq)
+            outs["out_full"][i] = deq(full, neg, Xq)
+    return dict(codes=codes, mbits=mbits, scales=scales.reshape(rows, cols // 32), mask=mask,
+                **{k: v.reshape(rows, cols) for k, v in outs.items()})

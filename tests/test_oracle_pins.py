@@ -717,3 +717,68 @@ def test_mismatch_distance_by_grid_index(oracle_mod):
         d = np.array([abs(index(int(a)) - index(int(b))) for a, b in zip(rules[k], q_roll)])
         assert np.array_equal(hist[k], np.bincount(d, minlength=15)), k
     assert hist[0, 2:].sum() > 0 and np.count_nonzero(hist[0]) > 5   # long distances occur
+
+
+# --------------------------------------------------------------------------
+# W4A8: E4M3 activations with MX scales (results list: the W4A8 setting)
+# --------------------------------------------------------------------------
+
+def test_mx8_scale_vs_bruteforce(oracle_mod):
+    pats = np.arange(0x7F80, dtype=np.uint32)
+    vals = (pats << 16).view(np.float32)
+    for a in vals[::11].tolist() + [0.0, 2.0 ** -133, 2.0 ** -119, 2.0 ** -118, 3.3e38, 512.0, 511.0,
+                                   256.0, 448.0]:
+        a = float(np.float32(a))
+        assert oracle_mod.mx8_scale(a) == bf.brute_mx8_scale(Fraction(a)), a
+
+
+def test_e4m3_bracket_and_guided_vs_bruteforce(oracle_mod):
+    """On every E4M3 value, every midpoint and +-1 ulp around them, both bits:
+    the bracket and the guided choice against exhaustive search; neighbouring
+    codes alternate their lowest bit, so one member qualifies."""
+    vals = sorted(float(v) for v, _ in bf.E4M3_TABLE)
+    pts = set(vals)
+    for a, b in zip(vals[:-1], vals[1:]):
+        m = np.float32((a + b) / 2)
+        pts.update([float(m), float(np.nextafter(m, np.float32(0))), float(np.nextafter(m, np.float32(1e9)))])
+    pts.update([460.0, 1e6])
+    for a in sorted(pts):
+        a32 = float(np.float32(a))
+        lo, hi = bf.brute_e4m3_bracket(Fraction(a32))
+        assert oracle_mod.e4m3_bracket(min(a32, 448.0)) == (lo, hi), a32
+        for bit in (0, 1):
+            want = lo if lo == hi or (lo & 1) == bit else hi
+            assert oracle_mod.e4m3_guided_code(min(a32, 448.0), bit) == want
+        assert oracle_mod.e4m3_full_guided_code(a32, lo) == lo
+        assert oracle_mod.e4m3_full_guided_code(-a32, 0x80 | hi) == hi
+
+
+@pytest.mark.parametrize("case", range(7))
+def test_mx8_pipeline_vs_bruteforce(oracle_mod, case):
+    xr, xt, _ = _tiny_cases()[case]
+    ref = bf.brute_mx8_pipeline(xr, xt)
+    codes, mbits, scales = oracle_mod.mx8_capture(xr)
+    assert np.array_equal(scales, ref["scales"])
+    assert np.array_equal(codes, ref["codes"])
+    assert np.array_equal(mbits, ref["mbits"])
+    out, mask = oracle_mod.mx8_guided_fwd(xt, mbits, scales)
+    assert np.array_equal(mask, ref["mask"]) and np.array_equal(out, ref["out_guided"])
+    out_r, _ = oracle_mod.mx8_rtn_fwd(xt, scales)
+    assert np.array_equal(out_r, ref["out_rtn"])
+    out_f, _ = oracle_mod.mx8_full_guided_fwd(xt, codes, scales)
+    assert np.array_equal(out_f, ref["out_full"])
+
+
+def test_mx8_identity_and_cache_size(oracle_mod):
+    """Guided on x_roll itself reproduces the rollout codes (all three rules);
+    the W4A8 compact cache is 1 bit + one E8M0 byte per 32 elements = 1.25
+    bits per element against 8.25 for the full FP8 codes."""
+    s = inputs.tiny_site(47, 16, 256, eps=0.02)
+    xr = inputs.bits(s.x_roll)
+    codes, mbits, scales = oracle_mod.mx8_capture(xr)
+    for kw in ({}, {"mbits": mbits}, {"rcodes": codes}):
+        q = oracle_mod.mx8_fake_quant_codes(xr, scales, **kw).reshape(-1)
+        assert np.array_equal(q, codes)
+    n = xr.size
+    assert (mbits.nbytes + scales.nbytes) * 8 / n == 1.25
+    assert (codes.nbytes + scales.nbytes) * 8 / n == 8.25
