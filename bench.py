@@ -523,6 +523,35 @@ def run_trace(args):
              for j in range(2)]
     tl_ms = max_over_ranks(tl_ms, pg, dev)
 
+    # W4A8 (E4M3 activations, MX scales) on the same sites
+    m8c = [ops.mx8_capture(w["xr"], stream=stream) for w in work]
+
+    def mx8_pass(evs):
+        for i, w in enumerate(work):
+            ev = evs[i] if evs is not None else None
+            if ev: ev[0].record(stream)
+            ops.mx8_capture(w["xr"], m8c[i], stream)
+            if ev: ev[1].record(stream)
+            ops.mx8_guided_fq_fwd(w["xt"], m8c[i], w["out"], w["mask"], stream)
+            if ev: ev[2].record(stream)
+            ops.mx8_rtn_fq_fwd(w["xt"], m8c[i].scales, w["out_r"], w["mask_r"], stream)
+            if ev: ev[3].record(stream)
+            ops.mx8_full_guided_fq_fwd(w["xt"], m8c[i], w["out"], w["mask"], stream)
+            if ev: ev[4].record(stream)
+
+    mx8_pass(None)
+    m8_ev = []
+    for k in range(args.steps):
+        flush.fill_((k + 97) & 0xFF)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
+        mx8_pass(evs)
+        m8_ev.append(evs)
+    torch.cuda.synchronize()
+    m8_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in m8_ev for i in range(len(work)))
+             for j in range(4)]
+    m8_ms = max_over_ranks(m8_ms, pg, dev)
+    del m8c
+
     mx_pass(None)  # untimed: first launches
     mx_ev = []
     for k in range(args.steps):
@@ -588,6 +617,16 @@ def run_trace(args):
                        "gbs": round(n * b_k / (ms * 1e-3) / 1e9, 1),
                        "frac_of_hbm": round(n * b_k / (ms * 1e-3) / 1e9 / hbm, 4)}
     next_rows["mxfp4"] = mx_rows
+    m8_rows = {}
+    for j, (nm, kn, b_k) in enumerate([("capture", "k_mx8_capture", 3.15625),
+                                       ("guided_fwd", "k_mx8_fake_quant<1>", 4.28125),
+                                       ("rtn_fwd", "k_mx8_fake_quant<0>", 4.15625),
+                                       ("full_guided_fwd", "k_mx8_fake_quant<2>", 5.15625)]):
+        ms = m8_ms[j] / args.steps
+        m8_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": b_k,
+                       "gbs": round(n * b_k / (ms * 1e-3) / 1e9, 1),
+                       "frac_of_hbm": round(n * b_k / (ms * 1e-3) / 1e9 / hbm, 4)}
+    next_rows["w4a8"] = m8_rows
     next_rows["tiled_scales"] = {
         nm: {"kernel": kn, "us": round(tl_ms[j] / args.steps * 1e3, 2), "bytes_per_elem": b_k,
              "gbs": round(n * b_k / (tl_ms[j] / args.steps * 1e-3) / 1e9, 1),

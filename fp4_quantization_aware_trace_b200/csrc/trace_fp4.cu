@@ -1131,6 +1131,158 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
+// Kernels 10-11: W4A8 -- TRACE on FP8 (E4M3) activations with MX scales (the
+// post's results list names the W4A8 setting).  32-element blocks with an
+// E8M0 scale X = 2^e, e = floor(log2 max|x|) - 8 (448 = 1.75 * 2^8), clamped
+// at -127; z = x * 2^-e exactly as for MXFP4; round to nearest E4M3 (ties to
+// the even mantissa) saturating at 448; one byte per code (sign in bit 7);
+// the cached bit is the lowest bit of the magnitude code; STE mask |z| <= 448.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int mx8_exp(uint32_t amax) {
+  if (amax == 0u) return -127;
+  const int e = (int)(amax >> 7);
+  const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;
+  return max(fl - 8, -127);
+}
+
+// Two fp32 -> two E4M3 bytes (round to nearest even, satfinite), lo in bits
+// 0-7; the sign of each input is kept, also on zeros.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 bytes (lo in bits 0-7) -> f16x2 (exact, signed).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)two;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return h2;
+}
+
+// Grid addend for the E4M3 grid: M = 2^20 * max(2^-6, 2^E) (E the binade
+// of a <= 448), so that a + M keeps 3 fraction bits of a's binade (2^-9
+// steps below 2^-6, E4M3's subnormal spacing).
+__device__ __forceinline__ float grid_magic8(float a) {
+  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0A000000u, 0x46800000u));
+}
+
+// Lowest bit of each of 4 code bytes -> 4 bits.
+__device__ __forceinline__ uint32_t byte_lsbs(uint32_t w) {
+  return ((w & 0x01010101u) * 0x01020408u) >> 24;
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx8_capture(const V8* __restrict__ x, Shape sh, V8* __restrict__ codes,
+                  uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const int e = mx8_exp(max(absmax_block(v0), absmax_block(v1)));
+    const float inv = pow2f(-e);
+    const u64 inv2 = pk(inv, inv);
+    V8 c;
+    uint32_t bits = 0u;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t w = k < 8 ? v0.w[k] : v1.w[k - 8];
+      float zl, zh;
+      upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+      // |z| < 512 from the block's own maximum; the conversion saturates
+      // past 448 and keeps the sign of x
+      const uint32_t two = cvt_e4m3x2(zl, zh);
+      if (k & 1) c.w[k >> 1] |= two << 16; else c.w[k >> 1] = two;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) bits |= byte_lsbs(c.w[k]) << (4 * k);
+    st_block(codes + (b >> 1), c);  // one 32-byte store (a struct copy would split it)
+    mbits[b >> 1] = bits;
+    scales[b >> 1] = (uint8_t)(e + 127);
+  }
+}
+
+// Two elements of the W4A8 fake-quant forward.  side: kGuided -- the cached
+// bits in bits 0 and 1; kFull -- the two rollout code bytes (low first).
+template <int MODE>
+__device__ __forceinline__ uint32_t mx8_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
+                                                uint32_t& m, int pos) {
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+  m |= (le_mask(fabsf(zl), 448.0f) & (1u << pos)) | (le_mask(fabsf(zh), 448.0f) & (2u << pos));
+  const float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);
+  float tl, th;
+  if (MODE == kRtn) {
+    const uint32_t h2 = e4m3x2_to_f16x2(cvt_e4m3x2(al, ah));
+    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+  } else {
+    const u64 MM = pk(grid_magic8(al), grid_magic8(ah));
+    const u64 aa = pk(al, ah);
+    float lol, loh, hil, hih;
+    upk(add_rm2(aa, MM), lol, loh);
+    upk(add_rp2(aa, MM), hil, hih);
+    if (MODE == kGuided) {
+      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+      upk(sub2(pk(sl, sh), MM), tl, th);
+    } else {
+      float fl, fh, cl, ch;
+      upk(sub2(pk(lol, loh), MM), fl, fh);
+      upk(sub2(pk(hil, hih), MM), cl, ch);
+      const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFFFu);
+      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+      tl = rl > fl ? cl : fl;
+      th = rh > fh ? ch : fh;
+    }
+  }
+  float ql, qh;
+  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx8_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
+                     const V8* __restrict__ rcodes, const uint8_t* __restrict__ scales,
+                     V8* __restrict__ out, uint32_t* __restrict__ mask) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const V8 rc = MODE == kFull ? ld_block_stream(rcodes + (b >> 1)) : zero_block();
+    const int e = (int)__ldcs(scales + (b >> 1)) - 127;
+    const float inv = pow2f(-e), X = pow2f(e);
+    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
+    uint32_t m = 0u;
+    V8 o;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
+                          : MODE == kFull ? rc.w[k >> 1] >> (16 * (k & 1)) : 0u;
+      o.w[k] = mx8_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
+    }
+    st_block(out + b, o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
+                          : MODE == kFull ? rc.w[4 + (k >> 1)] >> (16 * (k & 1)) : 0u;
+      o.w[k] = mx8_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
+    }
+    st_block(out + b + 1, o);
+    mask[b >> 1] = m;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Kernel 6: plain copy with the same access pattern (bandwidth yardstick).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -1247,6 +1399,25 @@ int mx_fake_quant_dispatch(int mode, int grid, cudaStream_t s, const uint16_t* x
                   (const uint4*)rcodes, scales, (V8*)out, mask);
   return launch(k_mx_fake_quant<kRtn, SW>, grid, s, (const V8*)x, sh, (const uint32_t*)nullptr,
                 (const uint4*)nullptr, scales, (V8*)out, mask);
+}
+
+template <int MODE>
+int mx8_launch(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* mbits,
+               const uint8_t* rcodes, const uint8_t* scales, uint16_t* out, uint32_t* mask,
+               void* stream) {
+  int st = check_shape(rows, cols, 1, nullptr);
+  if (st) return st;
+  if (rows == 0) return TRACE_OK;
+  if (!x || (MODE == kGuided && !mbits) || (MODE == kFull && !rcodes) || !scales || !out || !mask)
+    return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || (MODE == kGuided && !aligned(mbits, 4)) ||
+      (MODE == kFull && !aligned(rcodes, 32)) || !aligned(out, 32) || !aligned(mask, 4))
+    return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, 1);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  return launch(k_mx8_fake_quant<MODE>, grid, (cudaStream_t)stream, (const V8*)x, sh, mbits,
+                (const V8*)rcodes, scales, (V8*)out, mask);
 }
 
 }  // namespace
@@ -1562,6 +1733,37 @@ int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows, int6
     return TRACE_ERR_SHAPE;
   return mx_fake_quant_launch(rule, x_train, rows, cols, mbits, codes, scales, out, ste_mask,
                               stream, scale_layout == TRACE_SCALES_TILED_128x4);
+}
+
+int trace_mx8_capture(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                      uint32_t* mbits, uint8_t* scales, void* stream) {
+  int st = check_shape(rows, cols, 1, nullptr);
+  if (st) return st;
+  if (rows == 0) return TRACE_OK;
+  if (!x || !codes || !mbits || !scales) return TRACE_ERR_NULL;
+  if (!aligned(x, 32) || !aligned(codes, 32) || !aligned(mbits, 4)) return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, 1);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  return launch(k_mx8_capture, grid, (cudaStream_t)stream, (const V8*)x, sh, (V8*)codes, mbits,
+                scales);
+}
+
+int trace_mx8_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                            const uint32_t* mbits, const uint8_t* scales, uint16_t* out,
+                            uint32_t* ste_mask, void* stream) {
+  return mx8_launch<kGuided>(x_train, rows, cols, mbits, nullptr, scales, out, ste_mask, stream);
+}
+
+int trace_mx8_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,
+                                 const uint8_t* codes, const uint8_t* scales, uint16_t* out,
+                                 uint32_t* ste_mask, void* stream) {
+  return mx8_launch<kFull>(x_train, rows, cols, nullptr, codes, scales, out, ste_mask, stream);
+}
+
+int trace_mx8_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* scales,
+                         uint16_t* out, uint32_t* ste_mask, void* stream) {
+  return mx8_launch<kRtn>(x, rows, cols, nullptr, nullptr, scales, out, ste_mask, stream);
 }
 
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,

@@ -86,6 +86,14 @@ def library() -> ctypes.CDLL:
         lib.trace_mx_fq_fwd_ex.restype = ctypes.c_int
         lib.trace_capture_amax.argtypes = [P, i64, i64, i32, P, P, P]
         lib.trace_capture_amax.restype = ctypes.c_int
+        lib.trace_mx8_capture.argtypes = [P, i64, i64, P, P, P, P]
+        lib.trace_mx8_capture.restype = ctypes.c_int
+        lib.trace_mx8_guided_fq_fwd.argtypes = [P, i64, i64, P, P, P, P, P]
+        lib.trace_mx8_guided_fq_fwd.restype = ctypes.c_int
+        lib.trace_mx8_full_guided_fq_fwd.argtypes = [P, i64, i64, P, P, P, P, P]
+        lib.trace_mx8_full_guided_fq_fwd.restype = ctypes.c_int
+        lib.trace_mx8_rtn_fq_fwd.argtypes = [P, i64, i64, P, P, P, P]
+        lib.trace_mx8_rtn_fq_fwd.restype = ctypes.c_int
         lib.trace_capture_amax_accumulate.argtypes = [P, i64, i64, i32, P, P, P]
         lib.trace_capture_amax_accumulate.restype = ctypes.c_int
         lib.trace_capture_with_amax.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, i32, P]
@@ -369,6 +377,61 @@ def mx_rtn_fq_fwd(x: torch.Tensor, scales: torch.Tensor, out=None, mask=None, st
     """MXFP4 round-to-nearest fake-quant with given E8M0 scales."""
     rows, cols, out, mask = _fq_outputs(x, out, mask)
     trace_mx_rtn_fq_fwd(x, rows, cols, scales, out, mask, stream)
+    return out, mask
+
+
+def trace_mx8_capture(x, rows, cols, codes, mbits, scales, stream=None) -> None:
+    _check(library().trace_mx8_capture(_p(x), rows, cols, _p(codes), _p(mbits), _p(scales),
+                                       _stream(stream)), "trace_mx8_capture")
+
+
+def trace_mx8_guided_fq_fwd(x_train, rows, cols, mbits, scales, out, ste_mask, stream=None) -> None:
+    _check(library().trace_mx8_guided_fq_fwd(_p(x_train), rows, cols, _p(mbits), _p(scales),
+                                             _p(out), _p(ste_mask), _stream(stream)),
+           "trace_mx8_guided_fq_fwd")
+
+
+def trace_mx8_full_guided_fq_fwd(x_train, rows, cols, codes, scales, out, ste_mask,
+                                 stream=None) -> None:
+    _check(library().trace_mx8_full_guided_fq_fwd(_p(x_train), rows, cols, _p(codes), _p(scales),
+                                                  _p(out), _p(ste_mask), _stream(stream)),
+           "trace_mx8_full_guided_fq_fwd")
+
+
+def trace_mx8_rtn_fq_fwd(x, rows, cols, scales, out, ste_mask, stream=None) -> None:
+    _check(library().trace_mx8_rtn_fq_fwd(_p(x), rows, cols, _p(scales), _p(out), _p(ste_mask),
+                                          _stream(stream)), "trace_mx8_rtn_fq_fwd")
+
+
+def mx8_capture(x: torch.Tensor, out: MxCapture | None = None, stream=None) -> MxCapture:
+    """W4A8 rollout capture (E4M3 activations, MX scales): codes are one
+    byte per element."""
+    rows, cols = _bf16_2d(x)
+    n = rows * cols
+    if out is None:
+        out = MxCapture(codes=torch.empty(n, dtype=torch.uint8, device=x.device),
+                        mbits=torch.empty(n // 32, dtype=torch.int32, device=x.device),
+                        scales=torch.empty(rows, cols // 32, dtype=torch.uint8, device=x.device))
+    trace_mx8_capture(x, rows, cols, out.codes, out.mbits, out.scales, stream)
+    return out
+
+
+def mx8_guided_fq_fwd(x_train: torch.Tensor, cache: MxCapture, out=None, mask=None, stream=None):
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    trace_mx8_guided_fq_fwd(x_train, rows, cols, cache.mbits, cache.scales, out, mask, stream)
+    return out, mask
+
+
+def mx8_full_guided_fq_fwd(x_train: torch.Tensor, cache: MxCapture, out=None, mask=None,
+                           stream=None):
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    trace_mx8_full_guided_fq_fwd(x_train, rows, cols, cache.codes, cache.scales, out, mask, stream)
+    return out, mask
+
+
+def mx8_rtn_fq_fwd(x: torch.Tensor, scales: torch.Tensor, out=None, mask=None, stream=None):
+    rows, cols, out, mask = _fq_outputs(x, out, mask)
+    trace_mx8_rtn_fq_fwd(x, rows, cols, scales, out, mask, stream)
     return out, mask
 
 

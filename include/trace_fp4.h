@@ -212,6 +212,39 @@ int trace_mx_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
                         const uint8_t* scales, uint16_t* out,
                         uint32_t* ste_mask, void* stream);
 
+/* ---- W4A8: TRACE on FP8 (E4M3) activations with MX scales --------------
+ * The results list names the W4A8 setting beside MXFP4.  With 8-bit
+ * activations the elements are E4M3 in 32-element blocks with an E8M0 scale
+ * X = 2^e, e = floor(log2 max|x|) - 8 (448 = 1.75 * 2^8 is E4M3's largest
+ * value), clamped at -127 (-127 for an all-zero block); z = x / X, clipped
+ * to [-448, 448]; round to nearest E4M3 with ties to the even mantissa; the
+ * cached bit is the lowest bit of the magnitude code; the guided choice is
+ * the bracket member (on the E4M3 grid, subnormals included) whose lowest
+ * bit equals it; the STE mask is |z| <= 448; out = bf16(q* * X).
+ *   codes : uint8[N], one E4M3 byte per element (sign in bit 7), 32-byte
+ *           aligned.
+ *   mbits : uint32[N/32] (element i = bit i&31 of word i>>5), 4-byte aligned.
+ *   scales: uint8[rows, cols/32] E8M0 bytes, no alignment requirement.
+ *           Capture writes 0..246 (a bf16 maximum stays below 2^128); the
+ *           forwards need 0..246 as well (448 * 2^120 would overflow).
+ *   x / out 32-byte aligned, ste_mask 4-byte aligned.  trace_fq_bwd serves
+ *   this format too.  The compact cache is mbits + scales: 1.25 bits per
+ *   element against 8.25 for the full FP8 codes. */
+int trace_mx8_capture(const uint16_t* x, int64_t rows, int64_t cols,
+                      uint8_t* codes, uint32_t* mbits, uint8_t* scales,
+                      void* stream);
+int trace_mx8_guided_fq_fwd(const uint16_t* x_train, int64_t rows,
+                            int64_t cols, const uint32_t* mbits,
+                            const uint8_t* scales, uint16_t* out,
+                            uint32_t* ste_mask, void* stream);
+int trace_mx8_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows,
+                                 int64_t cols, const uint8_t* codes,
+                                 const uint8_t* scales, uint16_t* out,
+                                 uint32_t* ste_mask, void* stream);
+int trace_mx8_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
+                         const uint8_t* scales, uint16_t* out,
+                         uint32_t* ste_mask, void* stream);
+
 /* ---- Block-scale layout of a block-scaled FP4 GEMM ------------------------
  * The abstract on the thelatestinai.com TRACE page credits NVFP4 with FP4
  * GEMMs that run W4A4 natively.  The rollout's own FP4 GEMM (a tcgen05
