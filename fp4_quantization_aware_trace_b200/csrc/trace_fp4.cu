@@ -1173,6 +1173,7 @@ __device__ __forceinline__ uint32_t byte_lsbs(uint32_t w) {
   return ((w & 0x01010101u) * 0x01020408u) >> 24;
 }
 
+template <bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mx8_capture(const V8* __restrict__ x, Shape sh, V8* __restrict__ codes,
                   uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
@@ -1200,7 +1201,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int k = 0; k < 8; ++k) bits |= byte_lsbs(c.w[k]) << (4 * k);
     st_block(codes + (b >> 1), c);  // one 32-byte store (a struct copy would split it)
     mbits[b >> 1] = bits;
-    scales[b >> 1] = (uint8_t)(e + 127);
+    size_t so = b >> 1;
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
+    }
+    scales[so] = (uint8_t)(e + 127);
   }
 }
 
@@ -1247,7 +1253,7 @@ __device__ __forceinline__ uint32_t mx8_fq_pair(uint32_t w, uint32_t side, u64 i
   return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
 }
 
-template <int MODE>
+template <int MODE, bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mx8_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
                      const V8* __restrict__ rcodes, const uint8_t* __restrict__ scales,
@@ -1259,7 +1265,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
     const V8 rc = MODE == kFull ? ld_block_stream(rcodes + (b >> 1)) : zero_block();
-    const int e = (int)__ldcs(scales + (b >> 1)) - 127;
+    size_t so = b >> 1;
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
+    }
+    const int e = (int)__ldcs(scales + so) - 127;
     const float inv = pow2f(-e), X = pow2f(e);
     const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
     uint32_t m = 0u;
@@ -1404,7 +1415,7 @@ int mx_fake_quant_dispatch(int mode, int grid, cudaStream_t s, const uint16_t* x
 template <int MODE>
 int mx8_launch(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* mbits,
                const uint8_t* rcodes, const uint8_t* scales, uint16_t* out, uint32_t* mask,
-               void* stream) {
+               void* stream, bool tiled = false) {
   int st = check_shape(rows, cols, 1, nullptr);
   if (st) return st;
   if (rows == 0) return TRACE_OK;
@@ -1413,10 +1424,14 @@ int mx8_launch(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* mb
   if (!aligned(x, 32) || (MODE == kGuided && !aligned(mbits, 4)) ||
       (MODE == kFull && !aligned(rcodes, 32)) || !aligned(out, 32) || !aligned(mask, 4))
     return TRACE_ERR_ALIGN;
-  const Shape sh = make_shape(rows, cols, 1);
+  Shape sh = make_shape(rows, cols, 1);
+  sh.sw_ct = (uint32_t)((cols / 32 + 3) / 4);
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
-  return launch(k_mx8_fake_quant<MODE>, grid, (cudaStream_t)stream, (const V8*)x, sh, mbits,
+  if (tiled)
+    return launch(k_mx8_fake_quant<MODE, true>, grid, (cudaStream_t)stream, (const V8*)x, sh,
+                  mbits, (const V8*)rcodes, scales, (V8*)out, mask);
+  return launch(k_mx8_fake_quant<MODE, false>, grid, (cudaStream_t)stream, (const V8*)x, sh, mbits,
                 (const V8*)rcodes, scales, (V8*)out, mask);
 }
 
@@ -1735,18 +1750,52 @@ int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows, int6
                               stream, scale_layout == TRACE_SCALES_TILED_128x4);
 }
 
-int trace_mx8_capture(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
-                      uint32_t* mbits, uint8_t* scales, void* stream) {
+static int mx8_capture_impl(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                            uint32_t* mbits, uint8_t* scales, bool tiled, void* stream) {
   int st = check_shape(rows, cols, 1, nullptr);
   if (st) return st;
   if (rows == 0) return TRACE_OK;
   if (!x || !codes || !mbits || !scales) return TRACE_ERR_NULL;
   if (!aligned(x, 32) || !aligned(codes, 32) || !aligned(mbits, 4)) return TRACE_ERR_ALIGN;
-  const Shape sh = make_shape(rows, cols, 1);
+  Shape sh = make_shape(rows, cols, 1);
+  sh.sw_ct = (uint32_t)((cols / 32 + 3) / 4);
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
-  return launch(k_mx8_capture, grid, (cudaStream_t)stream, (const V8*)x, sh, (V8*)codes, mbits,
-                scales);
+  if (tiled)
+    return launch(k_mx8_capture<true>, grid, (cudaStream_t)stream, (const V8*)x, sh, (V8*)codes,
+                  mbits, scales);
+  return launch(k_mx8_capture<false>, grid, (cudaStream_t)stream, (const V8*)x, sh, (V8*)codes,
+                mbits, scales);
+}
+
+int trace_mx8_capture(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                      uint32_t* mbits, uint8_t* scales, void* stream) {
+  return mx8_capture_impl(x, rows, cols, codes, mbits, scales, false, stream);
+}
+
+int trace_mx8_capture_ex(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,
+                         uint32_t* mbits, uint8_t* scales, int32_t scale_layout, void* stream) {
+  if (scale_layout != TRACE_SCALES_ROW_MAJOR && scale_layout != TRACE_SCALES_TILED_128x4)
+    return TRACE_ERR_SHAPE;
+  return mx8_capture_impl(x, rows, cols, codes, mbits, scales,
+                          scale_layout == TRACE_SCALES_TILED_128x4, stream);
+}
+
+int trace_mx8_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows, int64_t cols,
+                        const uint32_t* mbits, const uint8_t* codes, const uint8_t* scales,
+                        uint16_t* out, uint32_t* ste_mask, int32_t scale_layout, void* stream) {
+  if ((scale_layout != TRACE_SCALES_ROW_MAJOR && scale_layout != TRACE_SCALES_TILED_128x4) ||
+      rule < TRACE_RULE_RTN || rule > TRACE_RULE_FULL)
+    return TRACE_ERR_SHAPE;
+  const bool tiled = scale_layout == TRACE_SCALES_TILED_128x4;
+  if (rule == TRACE_RULE_GUIDED)
+    return mx8_launch<kGuided>(x_train, rows, cols, mbits, nullptr, scales, out, ste_mask, stream,
+                               tiled);
+  if (rule == TRACE_RULE_FULL)
+    return mx8_launch<kFull>(x_train, rows, cols, nullptr, codes, scales, out, ste_mask, stream,
+                             tiled);
+  return mx8_launch<kRtn>(x_train, rows, cols, nullptr, nullptr, scales, out, ste_mask, stream,
+                          tiled);
 }
 
 int trace_mx8_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t cols,

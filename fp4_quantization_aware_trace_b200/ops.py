@@ -94,6 +94,10 @@ def library() -> ctypes.CDLL:
         lib.trace_mx8_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_mx8_rtn_fq_fwd.argtypes = [P, i64, i64, P, P, P, P]
         lib.trace_mx8_rtn_fq_fwd.restype = ctypes.c_int
+        lib.trace_mx8_capture_ex.argtypes = [P, i64, i64, P, P, P, i32, P]
+        lib.trace_mx8_capture_ex.restype = ctypes.c_int
+        lib.trace_mx8_fq_fwd_ex.argtypes = [i32, P, i64, i64, P, P, P, P, P, i32, P]
+        lib.trace_mx8_fq_fwd_ex.restype = ctypes.c_int
         lib.trace_capture_amax_accumulate.argtypes = [P, i64, i64, i32, P, P, P]
         lib.trace_capture_amax_accumulate.restype = ctypes.c_int
         lib.trace_capture_with_amax.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, i32, P]
@@ -556,6 +560,31 @@ def capture_sharded(x: torch.Tensor, offsets: torch.Tensor | None = None, group=
     trace_capture_with_amax(x, rows, cols, G, offsets, amax, cap.codes, cap.mbits, cap.scales,
                             cap.gscale, TRACE_SCALES_ROW_MAJOR, stream)
     return cap
+
+
+def mx8_capture_tiled(x: torch.Tensor, stream=None) -> MxCapture:
+    """W4A8 capture with the E8M0 scales in the 128 x 4 tiled layout."""
+    rows, cols = _bf16_2d(x)
+    n = rows * cols
+    cap = MxCapture(codes=torch.empty(n, dtype=torch.uint8, device=x.device),
+                    mbits=torch.empty(n // 32, dtype=torch.int32, device=x.device),
+                    scales=torch.zeros(trace_scale_bytes(rows, cols, 32, TRACE_SCALES_TILED_128x4),
+                                       dtype=torch.uint8, device=x.device))
+    _check(library().trace_mx8_capture_ex(_p(x), rows, cols, _p(cap.codes), _p(cap.mbits),
+                                          _p(cap.scales), TRACE_SCALES_TILED_128x4,
+                                          _stream(stream)), "trace_mx8_capture_ex")
+    return cap
+
+
+def mx8_fq_fwd_tiled(rule: int, x_train: torch.Tensor, cache: MxCapture, out=None, mask=None,
+                     stream=None):
+    """W4A8 forward (rule TRACE_RULE_*) reading tiled scales."""
+    rows, cols, out, mask = _fq_outputs(x_train, out, mask)
+    _check(library().trace_mx8_fq_fwd_ex(rule, _p(x_train), rows, cols, _p(cache.mbits),
+                                         _p(cache.codes), _p(cache.scales), _p(out), _p(mask),
+                                         TRACE_SCALES_TILED_128x4, _stream(stream)),
+           "trace_mx8_fq_fwd_ex")
+    return out, mask
 
 
 MISMATCH_RULES = ("rtn", "guided_1bit", "full_guided")

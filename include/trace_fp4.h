@@ -292,6 +292,16 @@ int trace_mx_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows,
                        const uint8_t* codes, const uint8_t* scales,
                        uint16_t* out, uint32_t* ste_mask, int32_t scale_layout,
                        void* stream);
+/* The same for the W4A8 calls (E8M0 scales of 32-element blocks, the layout a
+ * block-scaled FP8 GEMM reads too). */
+int trace_mx8_capture_ex(const uint16_t* x, int64_t rows, int64_t cols,
+                         uint8_t* codes, uint32_t* mbits, uint8_t* scales,
+                         int32_t scale_layout, void* stream);
+int trace_mx8_fq_fwd_ex(int32_t rule, const uint16_t* x_train, int64_t rows,
+                        int64_t cols, const uint32_t* mbits,
+                        const uint8_t* codes, const uint8_t* scales,
+                        uint16_t* out, uint32_t* ste_mask, int32_t scale_layout,
+                        void* stream);
 
 /* ---- Capture of a row-sharded tensor -------------------------------------
  * When one tensor's rows are spread over several GPUs, its global scale

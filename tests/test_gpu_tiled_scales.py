@@ -221,3 +221,23 @@ def test_host_step_matches_oracle(oracle_mod, rows, cols, chunks, grouped):
         if k == "gscale":
             got, v = got.view(np.uint32), v.view(np.uint32)
         _eq(f"host step {k}", got, v)
+
+
+@pytest.mark.parametrize("rows,cols", [(3, 64), (129, 160), (300, 2048)])
+def test_w4a8_tiled(oracle_mod, rows, cols):
+    s = inputs.tiny_site(rows * 5 + cols, rows, cols, eps=0.02)
+    xr, xt = s.x_roll.to(DEV), s.x_train.to(DEV)
+    cap = ops.mx8_capture_tiled(xr)
+    got = {r: ops.mx8_fq_fwd_tiled(r, xt, cap) for r in RULES}
+    torch.cuda.synchronize()
+    xrb, xtb = inputs.bits(s.x_roll), inputs.bits(s.x_train)
+    codes, mbits, scales = oracle_mod.mx8_capture(xrb)
+    outs = {ops.TRACE_RULE_GUIDED: oracle_mod.mx8_guided_fwd(xtb, mbits, scales),
+            ops.TRACE_RULE_RTN: oracle_mod.mx8_rtn_fwd(xtb, scales),
+            ops.TRACE_RULE_FULL: oracle_mod.mx8_full_guided_fwd(xtb, codes, scales)}
+    _eq("w4a8 codes", _u(cap.codes), codes)
+    _eq("w4a8 mbits", _u(cap.mbits), mbits)
+    _eq("w4a8 tiled scales", _u(cap.scales), oracle_mod.swizzle_scales(scales))
+    for r in RULES:
+        _eq(f"w4a8 out rule {r}", _u(got[r][0]), outs[r][0])
+        _eq(f"w4a8 mask rule {r}", _u(got[r][1]), outs[r][1])
