@@ -1294,6 +1294,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // ---------------------------------------------------------------------------
+// Self-test kernel: the block-scale rounding (cvt_e4m3, as capture uses it)
+// on fp32 inputs generated from their index, for exhaustive checks.
+// ---------------------------------------------------------------------------
+__global__ void k_selftest_e4m3(uint32_t first_bits, uint32_t count, uint8_t* __restrict__ out) {
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x)
+    out[i] = (uint8_t)cvt_e4m3(__uint_as_float(first_bits + i));
+}
+
+// ---------------------------------------------------------------------------
 // Kernel 6: plain copy with the same access pattern (bandwidth yardstick).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
@@ -1813,6 +1822,18 @@ int trace_mx8_full_guided_fq_fwd(const uint16_t* x_train, int64_t rows, int64_t 
 int trace_mx8_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols, const uint8_t* scales,
                          uint16_t* out, uint32_t* ste_mask, void* stream) {
   return mx8_launch<kRtn>(x, rows, cols, nullptr, nullptr, scales, out, ste_mask, stream);
+}
+
+int trace_selftest_e4m3_sweep(uint32_t first_bits, uint32_t count, uint8_t* out,
+                              void* stream) {
+  if (count == 0) return TRACE_OK;
+  if (!out) return TRACE_ERR_NULL;
+  // positive finite inputs only: the last bit pattern must stay below +inf
+  if (first_bits >= 0x7F800000u || count > 0x7F800000u - first_bits) return TRACE_ERR_SHAPE;
+  const int sms = sm_count();
+  if (sms <= 0) return TRACE_ERR_CUDA;
+  k_selftest_e4m3<<<sms * 8, 256, 0, (cudaStream_t)stream>>>(first_bits, count, out);
+  return cudaGetLastError() == cudaSuccess ? TRACE_OK : TRACE_ERR_CUDA;
 }
 
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,

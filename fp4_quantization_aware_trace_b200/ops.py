@@ -94,6 +94,8 @@ def library() -> ctypes.CDLL:
         lib.trace_mx8_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_mx8_rtn_fq_fwd.argtypes = [P, i64, i64, P, P, P, P]
         lib.trace_mx8_rtn_fq_fwd.restype = ctypes.c_int
+        lib.trace_selftest_e4m3_sweep.argtypes = [ctypes.c_uint32, ctypes.c_uint32, P, P]
+        lib.trace_selftest_e4m3_sweep.restype = ctypes.c_int
         lib.trace_mx8_capture_ex.argtypes = [P, i64, i64, P, P, P, i32, P]
         lib.trace_mx8_capture_ex.restype = ctypes.c_int
         lib.trace_mx8_fq_fwd_ex.argtypes = [i32, P, i64, i64, P, P, P, P, P, i32, P]
@@ -205,6 +207,11 @@ def trace_mismatch_histogram(x_train, rows, cols, num_groups, offsets, codes, sc
     _check(library().trace_mismatch_histogram(_p(x_train), rows, cols, num_groups, _p(offsets),
                                               _p(codes), _p(scales), _p(gscale), _p(hist),
                                               _stream(stream)), "trace_mismatch_histogram")
+
+
+def trace_selftest_e4m3_sweep(first_bits: int, count: int, out, stream=None) -> None:
+    _check(library().trace_selftest_e4m3_sweep(first_bits, count, _p(out), _stream(stream)),
+           "trace_selftest_e4m3_sweep")
 
 
 def trace_copy_bf16(src, dst, numel, stream=None) -> None:

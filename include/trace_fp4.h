@@ -353,6 +353,16 @@ int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
                      const uint8_t* scales, const float* gscale, uint16_t* out,
                      uint32_t* ste_mask, void* stream);
 
+/* Self-test, not a step of the method: the E4M3 rounding that capture applies
+ * to t = bmax / (6 s_g) (round to nearest even, saturating at 448), run on the
+ * fp32 values whose bit patterns are first_bits .. first_bits + count - 1,
+ * written to out[count] (device, no alignment requirement).  The range must
+ * hold positive finite values only (below 0x7F800000), else TRACE_ERR_SHAPE.
+ * It lets a test compare the device conversion with a reference on every
+ * positive finite fp32. */
+int trace_selftest_e4m3_sweep(uint32_t first_bits, uint32_t count, uint8_t* out,
+                              void* stream);
+
 /* Plain bf16 copy (dst = src) with the same load/store path as the kernels
  * above: the measured-bandwidth yardstick for the roofline.  Not part of the
  * method.  32-byte aligned, numel % 16 == 0, no overlap. */

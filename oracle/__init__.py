@@ -132,6 +132,8 @@ def _load():
         lib.oracle_mx8_full_guided_fwd.restype = None
         lib.oracle_mx8_fake_quant_codes.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int]
         lib.oracle_mx8_fake_quant_codes.restype = None
+        lib.oracle_e4m3_sweep.argtypes = [ctypes.c_uint32, ctypes.c_uint32, P]
+        lib.oracle_e4m3_sweep.restype = None
         lib.oracle_swizzled_scale_bytes.argtypes = [i64, i64]
         lib.oracle_swizzled_scale_bytes.restype = i64
         lib.oracle_swizzle_scales.argtypes = [P, i64, i64, P]
@@ -550,3 +552,10 @@ def mx8_fake_quant_codes(x, scales, mbits=None, rcodes=None):
                                         _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
                                         _ptr(sites), mode)
     return sites.reshape(rows, cols)
+
+
+def e4m3_sweep(first_bits: int, count: int) -> np.ndarray:
+    """E4M3 codes of the fp32 values with bit patterns first_bits + i."""
+    out = np.zeros(count, np.uint8)
+    _load().oracle_e4m3_sweep(first_bits, count, _ptr(out))
+    return out

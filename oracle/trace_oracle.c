@@ -779,3 +779,14 @@ void oracle_mx8_fake_quant_codes(const uint16_t* x, int64_t rows, int64_t cols,
                                  const uint8_t* scales, uint8_t* sites, int mode) {
   mx8_fake_quant(x, rows, cols, mbits, rcodes, scales, 0, 0, sites, mode);
 }
+
+/* E4M3 rounding of the fp32 values with bit patterns first .. first+count-1
+ * (positive finite), for the exhaustive comparison with the device. */
+void oracle_e4m3_sweep(uint32_t first, uint32_t count, uint8_t* out) {
+  for (uint32_t i = 0; i < count; ++i) {
+    const uint32_t u = first + i;
+    float t;
+    memcpy(&t, &u, sizeof t);
+    out[i] = oracle_f32_to_e4m3(t);
+  }
+}

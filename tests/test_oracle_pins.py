@@ -782,3 +782,18 @@ def test_mx8_identity_and_cache_size(oracle_mod):
     n = xr.size
     assert (mbits.nbytes + scales.nbytes) * 8 / n == 1.25
     assert (codes.nbytes + scales.nbytes) * 8 / n == 8.25
+
+
+def test_e4m3_encode_vs_torch_dense(oracle_mod):
+    """Every 97th fp32 bit pattern below the saturation tie 464 (11.7 M
+    values, subnormals included) against torch's float8_e4m3fn conversion."""
+    end = 0x43E80000                                  # 464.0
+    idx = np.arange(0, end, 97, dtype=np.uint32)
+    ref = torch.from_numpy(idx.view(np.float32).copy()).to(torch.float8_e4m3fn)
+    ref = ref.view(torch.uint8).numpy()
+    got = np.empty(idx.size, np.uint8)
+    for k0 in range(0, idx.size, 65536):              # contiguous runs, every 97th kept
+        k1 = min(idx.size, k0 + 65536)
+        first = int(idx[k0])
+        got[k0:k1] = oracle_mod.e4m3_sweep(first, int(idx[k1 - 1]) - first + 1)[::97]
+    assert np.array_equal(got, ref)
