@@ -52,7 +52,18 @@ KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<1> 
 LAUNCHES_PER_STEP = 6  # zero + amax + capture, guided, bwd, rtn
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
-CSRC = os.path.join(ROOT, "fp4_quantization_aware_trace_b200", "csrc", "trace_fp4.cu")
+CSRC_DIR = os.path.join(ROOT, "fp4_quantization_aware_trace_b200", "csrc")
+
+
+def source_hash() -> str:
+    """sha256/16 over the CUDA sources (every file of csrc/, by name)."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(CSRC_DIR)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(CSRC_DIR, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()[:16]
 PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 
@@ -95,7 +106,7 @@ def measured_peaks():
 def traffic_from_profiles(kernel_key: str):
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, or
     None when the summary is missing or the source changed since."""
-    src_hash = hashlib.sha256(open(CSRC, "rb").read()).hexdigest()[:16]
+    src_hash = source_hash()
     path = os.path.join(PROFILE_DIR, f"{kernel_key}_attn_in_16384x2048.md")
     if not os.path.exists(path):
         return None

@@ -8,6 +8,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC = os.path.join(PKG, "csrc", "trace_fp4.cu")
+CSRC_DIR = os.path.join(PKG, "csrc")
 HDR = os.path.join(ROOT, "include", "trace_fp4.h")
 LIB = os.path.join(PKG, "libtrace_fp4.so")
 
@@ -29,9 +30,12 @@ def nvcc() -> str:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile csrc/trace_fp4.cu into the package directory; returns the path."""
+    """Compile csrc/trace_fp4.cu (which includes the csrc/*.cuh kernels) into
+    the package directory; returns the path."""
+    deps = [HDR] + [os.path.join(CSRC_DIR, f) for f in os.listdir(CSRC_DIR)
+                    if f.endswith((".cu", ".cuh"))]
     if (not force and os.path.exists(LIB)
-            and os.path.getmtime(LIB) >= max(os.path.getmtime(SRC), os.path.getmtime(HDR))):
+            and os.path.getmtime(LIB) >= max(os.path.getmtime(d) for d in deps)):
         return LIB
     tmp = LIB + f".tmp{os.getpid()}"
     cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", tmp, SRC]

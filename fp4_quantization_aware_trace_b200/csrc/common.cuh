@@ -1,0 +1,296 @@
+// common.cuh -- device helpers shared by every kernel of libtrace_fp4.so:
+// launch constants, programmatic dependent launch, the fast division,
+// 32-byte loads and stores, packed fp32x2 arithmetic, the hardware number
+// format conversions, the exact-quotient and grid-rounding helpers, the group
+// cursor, the shape record and the tiled scale offset.  Included by
+// trace_fp4.cu inside its anonymous namespace (one translation unit).
+#pragma once
+
+typedef unsigned long long u64;
+
+constexpr int kThreads = 256;
+constexpr int kBlkPerThread = 2;
+constexpr int kTileBlks = kThreads * kBlkPerThread;  // 512 blocks = 8192 elements
+constexpr int kCtasPerSm = 4;    // resident CTAs per SM the register budget allows
+constexpr int kGridPerSm = 32;   // CTAs launched per SM: about one tile each
+constexpr int kAmaxTable = 256;  // groups per CTA kept in shared memory
+
+constexpr uint32_t kDMin = 0x12800000u;     // 2^-90: fast paths need d >= 2^-90
+constexpr uint32_t kDMax = 0x71800000u;     // 2^100: capture / round-to-nearest
+constexpr uint32_t kDMaxExactZ = 0x47800000u;  // 2^16: guided (see below)
+// The guided path divides |x| * 2^64: every nonzero bf16 then has a normal
+// quotient and an exactly representable remainder for d in the fast range.
+constexpr float kXs = 0x1p64f;
+constexpr float kSixS = 0x1p64f * 6.0f;
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch (sm_90+): every kernel waits for the
+// previous kernel in the stream to complete before it reads any global
+// memory, then lets the next kernel start launching.  Launched with the
+// programmatic-serialization attribute, a kernel's launch and prologue
+// overlap the tail of the one before it; launched without it, both
+// instructions are no-ops.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Fast unsigned 32-bit division by a runtime constant (Granlund & Montgomery,
+// "Division by invariant integers using multiplication", PLDI 1994, the
+// round-up method with the add-back step): block index -> row.
+// ---------------------------------------------------------------------------
+struct FastDiv {
+  uint32_t d, m, s;  // s = ceil(log2 d); d <= 1 handled separately
+};
+
+FastDiv make_fastdiv(uint32_t d) {
+  FastDiv f{d, 0u, 0u};
+  if (d <= 1) return f;
+  uint32_t l = 0;
+  while ((1ull << l) < d) ++l;
+  f.s = l;
+  f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1ull);
+  return f;
+}
+
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
+  if (f.d <= 1) return n;
+  uint32_t t = __umulhi(n, f.m);
+  return (t + ((n - t) >> 1)) >> (f.s - 1);
+}
+
+// ---------------------------------------------------------------------------
+// Memory access (public PTX ISA: 32-byte vector loads/stores on sm_100)
+// ---------------------------------------------------------------------------
+struct V8 {
+  uint32_t w[8];
+};
+
+// One 16-element bf16 block; read once, not kept in L1.
+__device__ __forceinline__ V8 ld_block_stream(const void* p) {
+  V8 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                 "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void st_block(void* p, const V8& v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+               "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+               "r"(v.w[7])
+               : "memory");
+}
+
+__device__ __forceinline__ V8 zero_block() {
+  V8 v;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v.w[k] = 0u;
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// Packed fp32x2 arithmetic (public PTX ISA, sm_100: mul/fma/add/sub .f32x2)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ u64 pk(float lo, float hi) {
+  u64 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk(u64 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+  u64 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+  u64 r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ u64 add_rm2(u64 a, u64 b) {
+  u64 r;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ u64 add_rp2(u64 a, u64 b) {
+  u64 r;
+  asm("add.rp.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
+  u64 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Number-format helpers (hardware conversions from the public PTX ISA)
+// ---------------------------------------------------------------------------
+
+// Two fp32 -> one byte of two E2M1 codes (round to nearest even, satfinite):
+// lo in bits 0-3, hi in bits 4-7; the sign of each input is kept.
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+      "cvt.u16.u8 %0, b;\n\t}"
+      : "=h"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Byte of two E2M1 codes -> f16x2 (exact): lo code in the low half.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.u8.u32 b, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
+      : "=r"(r)
+      : "r"(byte));
+  return r;
+}
+
+// fp32 >= 0 -> E4M3 byte (round to nearest even, saturating at 448).
+__device__ __forceinline__ uint32_t cvt_e4m3(float t) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
+  return (uint32_t)(r & 0xFFu);
+}
+
+// E4M3 byte -> fp32 (exact, through f16).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)b;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Two fp32 -> bf16x2 (round to nearest even): lo in the low half.
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// max|x| over a block as bf16 bits (integer order = magnitude order).
+__device__ __forceinline__ uint32_t absmax_block(const V8& v) {
+  uint32_t m = __vmaxu2(v.w[0] & 0x7FFF7FFFu, v.w[1] & 0x7FFF7FFFu);
+#pragma unroll
+  for (int k = 2; k < 8; ++k) m = __vmaxu2(m, v.w[k] & 0x7FFF7FFFu);
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Bit j of the result = bit 4j of n (the lowest bit of each nibble).
+__device__ __forceinline__ uint32_t nibble_lsbs(uint32_t n) {
+  uint32_t c = n & 0x11111111u;
+  c = (c | (c >> 3)) & 0x03030303u;
+  c = (c | (c >> 6)) & 0x000F000Fu;
+  return (c | (c >> 12)) & 0xFFu;
+}
+
+// Per-block constants of the fast path.
+struct BlkK {
+  u64 rr;    // (r, r), r = RN(1/d)
+  u64 ndd;   // (-d, -d)
+  u64 sbv2;  // (s_b, s_b), times 2^-64 on the guided path
+  u64 sg2;   // (s_g, s_g)
+};
+
+__device__ __forceinline__ BlkK make_blk(float d, float sbv, float s_g) {
+  BlkK k;
+  const float r = __frcp_rn(d);
+  k.rr = pk(r, r);
+  k.ndd = pk(-d, -d);
+  k.sbv2 = pk(sbv, sbv);
+  k.sg2 = pk(s_g, s_g);
+  return k;
+}
+
+// 0xFFFFFFFF when a <= b (false for NaN), else 0.
+__device__ __forceinline__ uint32_t le_mask(float a, float b) {
+  uint32_t r;
+  asm("set.le.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ bool fast_scale(float d, uint32_t dmax_bits = kDMax) {
+  const uint32_t db = __float_as_uint(d);
+  return db >= kDMin && db <= dmax_bits;
+}
+
+// Correctly rounded quotients of a pair: (lo, hi) / d.
+__device__ __forceinline__ u64 quot2(u64 xx, const BlkK& k) {
+  const u64 q0 = mul2(xx, k.rr);
+  const u64 e = fma2(q0, k.ndd, xx);
+  return fma2(e, k.rr, q0);
+}
+
+// Magic addend of the grid rounding for a = min(|z|, 6) * 2^64:
+// M = 2^86 * max(1, 2^E), E the binade of a / 2^64.
+__device__ __forceinline__ float grid_magic_s(float a_s) {
+  return __uint_as_float(max((__float_as_uint(a_s) & 0x7F800000u) + 0x0B000000u, 0x6A800000u));
+}
+
+// ---------------------------------------------------------------------------
+// Group lookup: offsets[g] <= row < offsets[g+1], cached per thread.
+// ---------------------------------------------------------------------------
+struct GroupCursor {
+  const int64_t* offs;
+  int G;
+  uint32_t lo, hi;  // cached row range of group g
+  int g;
+
+  __device__ void init(const int64_t* o, int G_) {
+    offs = o;
+    G = G_;
+    lo = 1u;
+    hi = 0u;
+    g = 0;
+  }
+  // returns true when the group changed
+  __device__ __forceinline__ bool seek(uint32_t row) {
+    if (G == 1) {
+      if (lo == 0u) return false;
+      g = 0;
+      lo = 0u;
+      hi = 0xFFFFFFFFu;
+      return true;
+    }
+    if (row >= lo && row < hi) return false;
+    int a = 0, b = G;  // last g with offs[g] <= row
+    while (b - a > 1) {
+      const int m = (a + b) >> 1;
+      if ((uint64_t)offs[m] <= row) a = m; else b = m;
+    }
+    g = a;
+    lo = (uint32_t)offs[a];
+    hi = (uint32_t)offs[a + 1];
+    return true;
+  }
+};
+
+struct Shape {
+  uint32_t nblk;    // N / 16
+  uint32_t ntiles;  // ceil(nblk / kTileBlks)
+  FastDiv bpr;      // blocks per row
+  int G;
+  uint32_t sw_ct;   // tiled scale layout: 128 x 4 tiles per row of tiles
+};
+
+// Byte offset of the scale at (row, col) in the tiled layout a block-scaled
+// FP4 GEMM reads: the scale matrix cut into 128-row x 4-column tiles of 512
+// bytes, stored in row-major tile order (ct tiles per row of tiles); inside
+// a tile, row r and column c sit at 16 (r mod 32) + 4 (r div 32) + c.
+__device__ __forceinline__ size_t tiled_scale_offset(uint32_t row, uint32_t col, uint32_t ct) {
+  return ((size_t)(row >> 7) * ct + (col >> 2)) * 512u + ((row & 31u) << 4) +
+         (((row >> 5) & 3u) << 2) + (col & 3u);
+}

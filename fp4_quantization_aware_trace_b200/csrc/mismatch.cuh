@@ -1,0 +1,194 @@
+// mismatch.cuh -- the mismatch-distance histogram kernel (ladder distance of
+// the round-to-nearest, 1-bit guided and full-information guided codes from
+// the rollout's).  Included by trace_fp4.cu inside its anonymous namespace.
+#pragma once
+
+// ---------------------------------------------------------------------------
+// Kernel 7: mismatch diagnostic.  For each element of x_train, with the
+// rollout's scales, the distance on the signed E2M1 ladder (-6 .. -0.5, 0,
+// 0.5 .. 6: 15 points) between the rollout's code and the code each of three
+// training-side rules picks -- round to nearest, 1-bit guided, full-
+// information guided -- counted into 3 x 15 bins (compact-cache paragraph:
+// sites where the two sides disagree are nearly all one codeword apart).
+//
+// The codes of 8 elements travel as 8 nibbles of one 32-bit word, and the
+// three rules, the distances and the counting run on whole words: every
+// per-nibble sum or difference below stays inside 0..15, so no carry or
+// borrow crosses into the next nibble.
+// ---------------------------------------------------------------------------
+constexpr int kHistBins = 15;  // distances 0..14
+constexpr int kHistModes = 3;  // round to nearest, 1-bit guided, full-information guided
+
+// The codes of one block, elements 0-7 in word 0 and 8-15 in word 1: floor
+// and ceiling magnitude codes of clip(|z|) on the grid (equal when it is a
+// codeword) and the round-to-nearest code with the sign of z.
+struct BlockCodes {
+  uint32_t f[2], c[2], r[2];
+};
+
+// One pair on the fast path: as the guided forward, z * 2^64 from |x|, the
+// floor and ceiling by directed rounding on the grid, each scaled back and
+// converted exactly to its code; round to nearest through the hardware
+// conversion (ties to the even code) of min(|z|, 6) with the sign of x.
+__device__ __forceinline__ void codes_pair(uint32_t w, const BlkK& k, uint32_t& fb, uint32_t& cb,
+                                           uint32_t& rb) {
+  const uint32_t wa = w & 0x7FFF7FFFu;
+  const u64 xx = pk(__uint_as_float(wa << 16), __uint_as_float(wa & 0xFFFF0000u));
+  float zl, zh;
+  upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
+  const float al = fminf(zl, kSixS), ah = fminf(zh, kSixS);  // NaN (|x| * 2^64 = inf) -> 6 * 2^64
+  const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
+  const u64 aa = pk(al, ah);
+  const u64 un = pk(0x1p-64f, 0x1p-64f);
+  float fl, fh, cl, ch, rl, rh;
+  upk(mul2(sub2(add_rm2(aa, MM), MM), un), fl, fh);
+  upk(mul2(sub2(add_rp2(aa, MM), MM), un), cl, ch);
+  upk(mul2(aa, un), rl, rh);
+  rl = __uint_as_float(__float_as_uint(rl) | ((w << 16) & 0x80000000u));
+  rh = __uint_as_float(__float_as_uint(rh) | (w & 0x80000000u));
+  fb = cvt_e2m1x2(fl, fh);
+  cb = cvt_e2m1x2(cl, ch);
+  rb = cvt_e2m1x2(rl, rh);
+}
+
+// The same codes on the exact path (d outside the fast range).
+__device__ __noinline__ void codes_block_exact(V8 v, float d, BlockCodes* bc) {
+  uint32_t f[2] = {0u, 0u}, c[2] = {0u, 0u}, r[2] = {0u, 0u};
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t w = v.w[j >> 1];
+    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+    const Exact e = exact_site(xf, d);
+    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
+    const int sh = 4 * (j & 7);
+    f[j >> 3] |= (uint32_t)e.floor << sh;
+    c[j >> 3] |= (uint32_t)(e.exact ? e.floor : e.floor + 1) << sh;
+    r[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << sh;
+  }
+  for (int h = 0; h < 2; ++h) {
+    bc->f[h] = f[h];
+    bc->c[h] = c[h];
+    bc->r[h] = r[h];
+  }
+}
+
+__device__ __forceinline__ BlockCodes block_codes(const V8& v, float sbv, float s_g) {
+  BlockCodes bc;
+  const float d = __fmul_rn(s_g, sbv);
+  if (d == 0.0f) {
+    // zero block: z = +-0, every code is zero with the sign of x
+    bc.f[0] = bc.f[1] = bc.c[0] = bc.c[1] = 0u;
+    bc.r[0] = bc.r[1] = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = v.w[k];
+      bc.r[k >> 2] |= ((((w >> 15) & 1u) << 3) | ((w >> 31) << 7)) << (8 * (k & 3));
+    }
+  } else if (fast_scale(d, kDMaxExactZ)) {
+    const BlkK bk = make_blk(d, 0.0f, 0.0f);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t fb[4], cb[4], rb[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) codes_pair(v.w[4 * h + k], bk, fb[k], cb[k], rb[k]);
+      bc.f[h] = fb[0] | (fb[1] << 8) | (fb[2] << 16) | (fb[3] << 24);
+      bc.c[h] = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
+      bc.r[h] = rb[0] | (rb[1] << 8) | (rb[2] << 16) | (rb[3] << 24);
+    }
+  } else {
+    codes_block_exact(v, d, &bc);
+  }
+  return bc;
+}
+
+// Ladder distances of 8 nibbles: training magnitude codes t against the
+// rollout magnitudes qm (both 0..7); s15 is 0xF on nibbles where the two
+// signs agree.  Same sign: |t - qm|; opposite signs: t + qm.
+__device__ __forceinline__ uint32_t ladder_dist8(uint32_t t, uint32_t qm, uint32_t s15) {
+  const uint32_t diff = t + 0x88888888u - qm;  // 8 + t - qm, in 1..15
+  const uint32_t ge = diff & 0x88888888u;      // t >= qm
+  const uint32_t m15 = ge | (ge - (ge >> 3));  // 0xF where t >= qm
+  // t >= qm: diff - 8;  t < qm: 8 - diff = (7 - diff) + 1
+  const uint32_t ad = (diff ^ 0x77777777u ^ m15) + 0x11111111u - (ge >> 3);
+  return (ad & s15) | ((t + qm) & ~s15);
+}
+
+// Count 8 distances: ones in a register, two and above (rare) in shared
+// memory; zeros are what is left over at the end.
+__device__ __forceinline__ void count8(uint32_t d, uint32_t& ones, uint32_t* bins) {
+  const uint32_t ge2 = (((d >> 1) & 0x77777777u) + 0x77777777u) & 0x88888888u;  // d >= 2
+  ones += __popc(d & 0x11111111u & ~(ge2 >> 3));
+  for (uint32_t g = ge2; g != 0u; g &= g - 1u) {
+    const int j = (__ffs((int)g) - 1) >> 2;
+    // a distance is at most 14; the clamp only keeps the index in bounds
+    atomicAdd(&bins[min((d >> (4 * j)) & 0xFu, 14u)], 1u);
+  }
+}
+
+// The three rules on 8 elements: f, c, r as in BlockCodes, q the rollout's
+// signed codes.
+__device__ __forceinline__ void hist_word(uint32_t f, uint32_t c, uint32_t r, uint32_t q,
+                                          uint32_t (&ones)[kHistModes], uint32_t* bins) {
+  const uint32_t ne = c - f;  // 1 where the bracket holds two codewords
+  const uint32_t qm = q & 0x77777777u;
+  const uint32_t s8 = ~(q ^ r) & 0x88888888u;  // signs of z and q_roll agree
+  const uint32_t s15 = s8 | (s8 - (s8 >> 3));
+  // round to nearest
+  count8(ladder_dist8(r & 0x77777777u, qm, s15), ones[0], bins);
+  // 1-bit guided: the ceiling where the floor's mantissa bit is not q_roll's
+  count8(ladder_dist8(f + ((f ^ q) & ne), qm, s15), ones[1], bins + kHistBins);
+  // full information: the ceiling where q_roll, on z's side, lies above the
+  // floor (8 + qm - f - 1 has bit 3 set exactly when qm > f)
+  const uint32_t up = ((qm + 0x88888888u - f - 0x11111111u) >> 3) & (s8 >> 3) & ne;
+  count8(ladder_dist8(f + up, qm, s15), ones[2], bins + 2 * kHistBins);
+}
+
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mismatch_hist(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+                    const uint4* __restrict__ rcodes, const uint16_t* __restrict__ scales,
+                    const float* __restrict__ gscale, unsigned long long* __restrict__ hist) {
+  __shared__ uint32_t bins[kHistModes * kHistBins];
+  __shared__ uint32_t seen;
+  if (threadIdx.x < kHistModes * kHistBins) bins[threadIdx.x] = 0u;
+  if (threadIdx.x == 0) seen = 0u;
+  __syncthreads();
+  pdl_begin();
+  GroupCursor gc;
+  gc.init(offs, sh.G);
+  float s_g = 1.0f;
+  uint32_t ones[kHistModes] = {0u, 0u, 0u}, n = 0u;
+
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint4 rc = __ldcs(rcodes + (b >> 1));
+    const uint32_t sb2 = __ldcs(scales + (b >> 1));
+    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
+    const BlockCodes k0 = block_codes(v0, e4m3_to_f32(sb2 & 0xFFu), s_g);
+    hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
+    hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);
+    const BlockCodes k1 = block_codes(v1, e4m3_to_f32(sb2 >> 8), s_g);
+    hist_word(k1.f[0], k1.c[0], k1.r[0], rc.z, ones, bins);
+    hist_word(k1.f[1], k1.c[1], k1.r[1], rc.w, ones, bins);
+    n += 32u;
+  }
+#pragma unroll
+  for (int k = 0; k < kHistModes; ++k) ones[k] = __reduce_add_sync(0xFFFFFFFFu, ones[k]);
+  n = __reduce_add_sync(0xFFFFFFFFu, n);
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int k = 0; k < kHistModes; ++k) atomicAdd(&bins[k * kHistBins + 1], ones[k]);
+    atomicAdd(&seen, n);
+  }
+  __syncthreads();
+  if (threadIdx.x < kHistModes * kHistBins) {
+    const int k = threadIdx.x / kHistBins, dist = threadIdx.x % kHistBins;
+    uint32_t v = bins[threadIdx.x];
+    if (dist == 0) {
+      uint32_t other = 0u;
+      for (int j = 1; j < kHistBins; ++j) other += bins[k * kHistBins + j];
+      v = seen - other;
+    }
+    if (v != 0u) atomicAdd(hist + threadIdx.x, (unsigned long long)v);
+  }
+}

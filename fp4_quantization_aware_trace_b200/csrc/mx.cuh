@@ -1,0 +1,324 @@
+// mx.cuh -- the MX-scaled variants: MXFP4 (W4A4, E2M1 elements) and W4A8
+// (E4M3 activations), capture and fake-quant forwards.  Included by
+// trace_fp4.cu inside its anonymous namespace.
+#pragma once
+
+// ---------------------------------------------------------------------------
+// Kernels 8-9: the MXFP4 variant (the post's results list: the method carries
+// over to MXFP4).  OCP Microscaling scales: one E8M0 byte per 32 elements of
+// a row, X = 2^e with e = floor(log2 max|x|) - 2 clamped at -127, and no
+// global scale.  A thread's pair of 16-element blocks is exactly one MX
+// block.  Dividing by a power of two is exact up to the one rounding of the
+// result, so z = x * 2^-e matches z = fl(x / X) with no correction step and
+// no exact path; the E2M1 decisions are those of the NVFP4 kernels.
+// ---------------------------------------------------------------------------
+
+// 2^k as fp32 for k in [-127, 127] (2^-127 is a subnormal).
+__device__ __forceinline__ float pow2f(int k) {
+  return __uint_as_float(k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00800000u >> (-126 - k));
+}
+
+// E8M0 exponent of a block whose max|x| has the bf16 bits amax (sign
+// cleared): floor(log2 amax) - 2, at least -127 (a bf16 amax stays below
+// 2^128, so the top of the range is never reached); -127 for an all-zero
+// block.
+__device__ __forceinline__ int mx_exp(uint32_t amax) {
+  if (amax == 0u) return -127;
+  const int e = (int)(amax >> 7);
+  const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;  // bf16 subnormal: m * 2^-133
+  return max(fl - 2, -127);
+}
+
+// Magic addend of the grid rounding for a = min(|z|, 6) (unscaled):
+// M = 2^22 * max(1, 2^E).
+__device__ __forceinline__ float grid_magic(float a) {
+  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
+}
+
+// Codes of one 16-element block: c0 elements 0-7, c1 elements 8-15.
+__device__ __forceinline__ void mx_codes_block(const V8& v, u64 inv2, uint32_t& c0, uint32_t& c1) {
+  uint32_t c[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w = v.w[k];
+    float zl, zh;
+    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+    // |z| < 8 from the block's own maximum; the conversion saturates past 6
+    // and keeps the sign of x, also on zeros
+    c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+  }
+  c0 = c[0];
+  c1 = c[1];
+}
+
+template <bool SW>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx_capture(const V8* __restrict__ x, Shape sh, uint4* __restrict__ codes,
+                 uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const int e = mx_exp(max(absmax_block(v0), absmax_block(v1)));
+    const float inv = pow2f(-e);
+    const u64 inv2 = pk(inv, inv);
+    uint4 c;
+    mx_codes_block(v0, inv2, c.x, c.y);
+    mx_codes_block(v1, inv2, c.z, c.w);
+    codes[b >> 1] = c;
+    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
+                    (nibble_lsbs(c.w) << 24);
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      scales[tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct)] = (uint8_t)(e + 127);
+    } else {
+      scales[b >> 1] = (uint8_t)(e + 127);
+    }
+  }
+}
+
+// Two elements of the MX fake-quant forward (side as fq_pair).
+template <int MODE>
+__device__ __forceinline__ uint32_t mx_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
+                                               uint32_t& m, int pos) {
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
+  m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
+  const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
+  float tl, th;  // chosen codeword value
+  if (MODE == kRtn) {
+    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
+    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+  } else {
+    const u64 MM = pk(grid_magic(al), grid_magic(ah));
+    const u64 aa = pk(al, ah);
+    float lol, loh, hil, hih;
+    upk(add_rm2(aa, MM), lol, loh);
+    upk(add_rp2(aa, MM), hil, hih);
+    if (MODE == kGuided) {
+      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+      upk(sub2(pk(sl, sh), MM), tl, th);
+    } else {
+      float fl, fh, cl, ch;
+      upk(sub2(pk(lol, loh), MM), fl, fh);
+      upk(sub2(pk(hil, hih), MM), cl, ch);
+      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
+      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+      tl = rl > fl ? cl : fl;
+      th = rh > fh ? ch : fh;
+    }
+  }
+  float ql, qh;
+  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+template <int MODE, bool SW>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
+                    const uint4* __restrict__ rcodes, const uint8_t* __restrict__ scales,
+                    V8* __restrict__ out, uint32_t* __restrict__ mask) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
+    size_t so = b >> 1;
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
+    }
+    const int e = (int)__ldcs(scales + so) - 127;
+    const float inv = pow2f(-e), X = pow2f(e);
+    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
+    uint32_t m = 0u;
+    V8 o;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
+                          : MODE == kFull ? ((k < 4 ? rc.x : rc.y) >> (8 * (k & 3))) : 0u;
+      o.w[k] = mx_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
+    }
+    st_block(out + b, o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
+                          : MODE == kFull ? ((k < 4 ? rc.z : rc.w) >> (8 * (k & 3))) : 0u;
+      o.w[k] = mx_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
+    }
+    st_block(out + b + 1, o);
+    mask[b >> 1] = m;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernels 10-11: W4A8 -- TRACE on FP8 (E4M3) activations with MX scales (the
+// post's results list names the W4A8 setting).  32-element blocks with an
+// E8M0 scale X = 2^e, e = floor(log2 max|x|) - 8 (448 = 1.75 * 2^8), clamped
+// at -127; z = x * 2^-e exactly as for MXFP4; round to nearest E4M3 (ties to
+// the even mantissa) saturating at 448; one byte per code (sign in bit 7);
+// the cached bit is the lowest bit of the magnitude code; STE mask |z| <= 448.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int mx8_exp(uint32_t amax) {
+  if (amax == 0u) return -127;
+  const int e = (int)(amax >> 7);
+  const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;
+  return max(fl - 8, -127);
+}
+
+// Two fp32 -> two E4M3 bytes (round to nearest even, satfinite), lo in bits
+// 0-7; the sign of each input is kept, also on zeros.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 bytes (lo in bits 0-7) -> f16x2 (exact, signed).
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)two;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  return h2;
+}
+
+// Grid addend for the E4M3 grid: M = 2^20 * max(2^-6, 2^E) (E the binade
+// of a <= 448), so that a + M keeps 3 fraction bits of a's binade (2^-9
+// steps below 2^-6, E4M3's subnormal spacing).
+__device__ __forceinline__ float grid_magic8(float a) {
+  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0A000000u, 0x46800000u));
+}
+
+// Lowest bit of each of 4 code bytes -> 4 bits.
+__device__ __forceinline__ uint32_t byte_lsbs(uint32_t w) {
+  return ((w & 0x01010101u) * 0x01020408u) >> 24;
+}
+
+template <bool SW>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx8_capture(const V8* __restrict__ x, Shape sh, V8* __restrict__ codes,
+                  uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const int e = mx8_exp(max(absmax_block(v0), absmax_block(v1)));
+    const float inv = pow2f(-e);
+    const u64 inv2 = pk(inv, inv);
+    V8 c;
+    uint32_t bits = 0u;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t w = k < 8 ? v0.w[k] : v1.w[k - 8];
+      float zl, zh;
+      upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+      // |z| < 512 from the block's own maximum; the conversion saturates
+      // past 448 and keeps the sign of x
+      const uint32_t two = cvt_e4m3x2(zl, zh);
+      if (k & 1) c.w[k >> 1] |= two << 16; else c.w[k >> 1] = two;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) bits |= byte_lsbs(c.w[k]) << (4 * k);
+    st_block(codes + (b >> 1), c);  // one 32-byte store (a struct copy would split it)
+    mbits[b >> 1] = bits;
+    size_t so = b >> 1;
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
+    }
+    scales[so] = (uint8_t)(e + 127);
+  }
+}
+
+// Two elements of the W4A8 fake-quant forward.  side: kGuided -- the cached
+// bits in bits 0 and 1; kFull -- the two rollout code bytes (low first).
+template <int MODE>
+__device__ __forceinline__ uint32_t mx8_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
+                                                uint32_t& m, int pos) {
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+  m |= (le_mask(fabsf(zl), 448.0f) & (1u << pos)) | (le_mask(fabsf(zh), 448.0f) & (2u << pos));
+  const float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);
+  float tl, th;
+  if (MODE == kRtn) {
+    const uint32_t h2 = e4m3x2_to_f16x2(cvt_e4m3x2(al, ah));
+    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+  } else {
+    const u64 MM = pk(grid_magic8(al), grid_magic8(ah));
+    const u64 aa = pk(al, ah);
+    float lol, loh, hil, hih;
+    upk(add_rm2(aa, MM), lol, loh);
+    upk(add_rp2(aa, MM), hil, hih);
+    if (MODE == kGuided) {
+      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+      upk(sub2(pk(sl, sh), MM), tl, th);
+    } else {
+      float fl, fh, cl, ch;
+      upk(sub2(pk(lol, loh), MM), fl, fh);
+      upk(sub2(pk(hil, hih), MM), cl, ch);
+      const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFFFu);
+      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+      tl = rl > fl ? cl : fl;
+      th = rh > fh ? ch : fh;
+    }
+  }
+  float ql, qh;
+  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+template <int MODE, bool SW>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_mx8_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
+                     const V8* __restrict__ rcodes, const uint8_t* __restrict__ scales,
+                     V8* __restrict__ out, uint32_t* __restrict__ mask) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const V8 rc = MODE == kFull ? ld_block_stream(rcodes + (b >> 1)) : zero_block();
+    size_t so = b >> 1;
+    if (SW) {
+      const uint32_t row = fastdiv(b, sh.bpr);
+      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
+    }
+    const int e = (int)__ldcs(scales + so) - 127;
+    const float inv = pow2f(-e), X = pow2f(e);
+    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
+    uint32_t m = 0u;
+    V8 o;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
+                          : MODE == kFull ? rc.w[k >> 1] >> (16 * (k & 1)) : 0u;
+      o.w[k] = mx8_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
+    }
+    st_block(out + b, o);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
+                          : MODE == kFull ? rc.w[4 + (k >> 1)] >> (16 * (k & 1)) : 0u;
+      o.w[k] = mx8_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
+    }
+    st_block(out + b + 1, o);
+    mask[b >> 1] = m;
+  }
+}

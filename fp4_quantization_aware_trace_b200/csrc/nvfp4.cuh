@@ -1,0 +1,439 @@
+// nvfp4.cuh -- the NVFP4 kernels of the path: zeroing of the amax
+// accumulators, the grid amax, rollout capture, the fake-quant forward (round
+// to nearest, 1-bit guided, full-information guided) and the masked
+// straight-through backward, plus their exact per-element path.  Included by
+// trace_fp4.cu inside its anonymous namespace.
+#pragma once
+
+// ---- exact path: the format's steps with an IEEE division -----------------
+
+struct Exact {
+  int rtn;     // round-to-nearest magnitude code of clip(|z|)
+  int floor;   // largest code with value <= clip(|z|)
+  bool exact;  // clip(|z|) is a codeword (bracket collapses)
+  bool in;     // |z| <= 6 (STE mask)
+};
+
+__device__ __forceinline__ Exact exact_site(float xf, float d) {
+  const float z = (d == 0.0f) ? copysignf(0.0f, xf) : __fdiv_rn(xf, d);
+  const float a = fabsf(z);
+  Exact e;
+  e.in = a <= 6.0f;
+  const float c = fminf(a, 6.0f);
+  e.rtn = (c <= 0.25f) ? 0 : (c < 0.75f) ? 1 : (c <= 1.25f) ? 2 : (c < 1.75f) ? 3
+        : (c <= 2.5f) ? 4 : (c < 3.5f) ? 5 : (c <= 5.0f) ? 6 : 7;
+  e.floor = (c < 0.5f) ? 0 : (c < 1.0f) ? 1 : (c < 1.5f) ? 2 : (c < 2.0f) ? 3
+          : (c < 3.0f) ? 4 : (c < 4.0f) ? 5 : (c < 6.0f) ? 6 : 7;
+  const float v = (e.floor == 0) ? 0.0f : (e.floor == 1) ? 0.5f : (e.floor == 2) ? 1.0f
+                : (e.floor == 3) ? 1.5f : (e.floor == 4) ? 2.0f : (e.floor == 5) ? 3.0f
+                : (e.floor == 6) ? 4.0f : 6.0f;
+  e.exact = (c == v);
+  return e;
+}
+
+// E2M1 magnitude (as fp32) of a code 0..7.
+__device__ __forceinline__ float e2m1_value(int c) {
+  return c >= 2 ? __uint_as_float((uint32_t)(c + 252) << 22) : (c == 1 ? 0.5f : 0.0f);
+}
+
+// Capture of one block on the exact path: 16 codes (sign<<3 | rtn).
+__device__ __noinline__ void capture_block_exact(V8 v, float d, uint32_t* code_lo,
+                                                 uint32_t* code_hi) {
+  uint32_t c[2] = {0u, 0u};
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t w = v.w[j >> 1];
+    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+    const Exact e = exact_site(xf, d);
+    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
+    c[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << (4 * (j & 7));
+  }
+  *code_lo = c[0];
+  *code_hi = c[1];
+}
+
+// Fake-quant of one block on the exact path: bf16 outputs and STE mask.
+// mode: 0 round-to-nearest, 1 1-bit guided (bits16), 2 full-information
+// guided (rollout codes c0: elements 0-7, c1: 8-15).
+__device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, float s_g,
+                                                    uint32_t bits16, uint32_t c0, uint32_t c1,
+                                                    int mode, V8* out, uint32_t* mask16) {
+  uint32_t m = 0u;
+  for (int k = 0; k < 8; ++k) out->w[k] = 0u;
+  for (int j = 0; j < 16; ++j) {
+    const uint32_t w = v.w[j >> 1];
+    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+    const Exact e = exact_site(xf, d);
+    int c = e.rtn;
+    if (mode == 1) {
+      const int bit = (int)((bits16 >> j) & 1u);
+      c = e.exact ? e.floor : e.floor + ((e.floor ^ bit) & 1);
+    } else if (mode == 2) {
+      // nearest of floor / ceiling to the rollout value on z's side of zero
+      const uint32_t rc = ((j < 8 ? c0 : c1) >> (4 * (j & 7))) & 0xFu;
+      float q = e2m1_value((int)(rc & 7u));
+      const bool neg_roll = (rc & 8u) != 0u, neg_z = ((w >> ((j & 1) ? 31 : 15)) & 1u) != 0u;
+      if (neg_roll != neg_z) q = -q;
+      const int hi = e.exact ? e.floor : e.floor + 1;
+      c = (q > e2m1_value(e.floor)) ? hi : e.floor;
+    }
+    const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
+        __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
+    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
+    out->w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
+    m |= (uint32_t)e.in << j;
+  }
+  *mask16 = m;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 0: zero the per-group amax accumulators.
+// ---------------------------------------------------------------------------
+__global__ void k_zero_u32(uint32_t* p, int n) {
+  pdl_begin();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1: per-group amax (bits of max|x| as bf16, kept as u32 so that
+// atomicMax orders them as magnitudes).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_amax(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+           uint32_t* __restrict__ amax) {
+  __shared__ uint32_t table[kAmaxTable];
+  __shared__ int g_first_s;
+  pdl_begin();
+  if (blockIdx.x >= sh.ntiles) return;
+
+  GroupCursor gc;
+  gc.init(offs, sh.G);
+  if (threadIdx.x == 0) {
+    gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
+    g_first_s = gc.g;
+  }
+  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
+  __syncthreads();
+  const int g_first = g_first_s;
+  gc.init(offs, sh.G);
+
+  uint32_t run = 0u;
+  int run_g = -1;
+  auto flush = [&](int g, uint32_t val) {
+    if (g < 0 || val == 0u) return;
+    const int slot = g - g_first;
+    if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
+    else atomicMax(&amax[g], val);
+  };
+
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    V8 v[kBlkPerThread];
+    const uint32_t base = t * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
+    }
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b >= sh.nblk) continue;
+      if (sh.G > 1) {
+        gc.seek(fastdiv(b, sh.bpr));
+        if (gc.g != run_g) {
+          flush(run_g, run);
+          run = 0u;
+          run_g = gc.g;
+        }
+      } else {
+        run_g = 0;
+      }
+      run = max(run, absmax_block(v[u]));
+    }
+  }
+  if (sh.G == 1) {
+    for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
+    if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
+  } else {
+    flush(run_g, run);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
+    const uint32_t val = table[i];
+    if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
+  }
+}
+
+// Per-group constants of capture.
+struct GroupK {
+  float s_g;    // amax / 2688, or 1
+  float den6;   // RN(6 * s_g)
+  float r6;     // RN(1 / den6)
+  bool fast6;   // den6 in the range where bmax/den6 may use the FMA quotient
+};
+
+__device__ __forceinline__ GroupK group_consts(uint32_t amax_bits) {
+  GroupK k;
+  const float a = __uint_as_float(amax_bits << 16);
+  k.s_g = amax_bits == 0u ? 1.0f : __fdiv_rn(a, 2688.0f);
+  k.den6 = __fmul_rn(6.0f, k.s_g);
+  k.fast6 = fast_scale(k.den6);
+  k.r6 = k.fast6 ? __frcp_rn(k.den6) : 0.0f;
+  return k;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: capture.  Per 16-element block: E4M3 scale; per element: the
+// round-to-nearest code and its mantissa bit.
+// ---------------------------------------------------------------------------
+// One block: returns its E4M3 scale byte, writes its 16 codes to c0 (elements
+// 0-7) and c1 (8-15).
+__device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk, uint32_t& c0,
+                                                  uint32_t& c1) {
+  // block scale: t = bmax / RN(6 s_g), E4M3 round-to-nearest-even, satfinite
+  const float bmax = __uint_as_float(absmax_block(v) << 16);
+  float tq;
+  if (gk.fast6) {
+    const float q0 = __fmul_rn(bmax, gk.r6);
+    tq = __fmaf_rn(__fmaf_rn(q0, -gk.den6, bmax), gk.r6, q0);
+  } else {
+    tq = __fdiv_rn(bmax, gk.den6);
+  }
+  const uint32_t sb = cvt_e4m3(tq);
+  const float d = __fmul_rn(gk.s_g, e4m3_to_f32(sb));
+  if (d == 0.0f) {
+    // zero block: z = +-0, code = sign only
+    c0 = c1 = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = v.w[k];
+      const uint32_t nib = (((w >> 15) & 1u) << 3) | ((w >> 31) << 7);
+      if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
+    }
+  } else if (fast_scale(d)) {
+    const BlkK bk = make_blk(d, 0.0f, 0.0f);
+    uint32_t c[2] = {0u, 0u};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t w = v.w[k];
+      const float xl = bf16_lo(w), xh = bf16_hi(w);
+      float zl, zh;
+      upk(quot2(pk(xl, xh), bk), zl, zh);
+      // the code carries the sign of x (also for zeros and underflows)
+      zl = __uint_as_float((__float_as_uint(zl) & 0x7FFFFFFFu) | (__float_as_uint(xl) & 0x80000000u));
+      zh = __uint_as_float((__float_as_uint(zh) & 0x7FFFFFFFu) | (w & 0x80000000u));
+      c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+    }
+    c0 = c[0];
+    c1 = c[1];
+  } else {
+    capture_block_exact(v, d, &c0, &c1);
+  }
+  return sb;
+}
+
+// Each thread owns two adjacent blocks: one 16-byte store of codes, one
+// 32-bit store of mantissa bits, one 16-bit store of scales.
+// SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
+template <bool SW>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+              const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
+              uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales,
+              float* __restrict__ gscale) {
+  pdl_begin();
+  // global scales of all groups (any CTA may write them; all write the same)
+  for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
+    gscale[g] = group_consts(amax[g]).s_g;
+
+  GroupCursor gc;
+  gc.init(offs, sh.G);
+  GroupK gk = group_consts(0u);
+
+  // tiles in reverse order: k_amax read the high tiles last, so they are the
+  // most likely to be still in L2
+  for (uint32_t i = blockIdx.x; i < sh.ntiles; i += gridDim.x) {
+    const uint32_t t = sh.ntiles - 1u - i;
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    // both blocks of the pair are in the same row (cols is a multiple of 32)
+    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+    if (gc.seek(row)) gk = group_consts(__ldg(amax + gc.g));
+    uint4 c;
+    const uint32_t s0 = capture_block(v0, gk, c.x, c.y);
+    const uint32_t s1 = capture_block(v1, gk, c.z, c.w);
+    codes[b >> 1] = c;
+    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
+                    (nibble_lsbs(c.w) << 24);
+    const uint16_t sv = (uint16_t)(s0 | (s1 << 8));
+    if (SW)  // the pair's two columns are neighbours inside one tile
+      *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
+    else
+      reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 3/5: fake-quant forward with given scales: bf16 q*·s and the STE
+// mask, q* chosen by round-to-nearest, by the cached mantissa bit, or by the
+// whole rollout code.
+// ---------------------------------------------------------------------------
+// Fake-quant modes: round to nearest (vanilla QAT), 1-bit guided (TRACE's
+// compact cache), full-information guided (the cache keeps the whole code).
+enum FqMode { kRtn = 0, kGuided = 1, kFull = 2 };
+
+// Two elements (one bf16x2 word w) of the fake-quant forward.  `side` carries
+// the guidance of the pair: MODE kGuided -- the cached bits of the two
+// elements in bits 0 and 1; kFull -- the rollout's two 4-bit codes (low
+// nibble first).  Mask bits go to positions pos, pos + 1 of m.
+template <int MODE>
+__device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const BlkK& k,
+                                            uint32_t& m, int pos) {
+  // signed x; only |z| is used below (sign of the output comes from w)
+  const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  float ql, qh;
+  if (MODE != kRtn) {
+    // z * 2^64 (exact; +-inf/NaN only where |x|/d overflows)
+    float zl, zh;
+    upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
+    m |= (le_mask(fabsf(zl), kSixS) & (1u << pos)) | (le_mask(fabsf(zh), kSixS) & (2u << pos));
+    const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
+    const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
+    const u64 aa = pk(al, ah);
+    float lol, loh, hil, hih;
+    upk(add_rm2(aa, MM), lol, loh);
+    upk(add_rp2(aa, MM), hil, hih);
+    if (MODE == kGuided) {
+      // of floor / ceiling, the one whose mantissa bit is the cached bit: the
+      // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
+      // bit of the floor sum is its codeword's mantissa bit
+      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+      const float tl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+      const float th = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+      upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
+    } else {
+      // of floor / ceiling, the one nearest the rollout codeword: the
+      // rollout value reflected to z's side of zero picks the ceiling
+      // exactly when it lies above the floor (no codeword lies between)
+      float fl, fh, cl, ch;
+      upk(sub2(pk(lol, loh), MM), fl, fh);
+      upk(sub2(pk(hil, hih), MM), cl, ch);
+      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
+      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+      upk(mul2(pk(rl, rh), pk(kXs, kXs)), rl, rh);
+      const float tl = rl > fl ? cl : fl;
+      const float th = rh > fh ? ch : fh;
+      upk(mul2(mul2(pk(tl, th), k.sbv2), k.sg2), ql, qh);
+    }
+  } else {
+    float zl, zh;
+    upk(quot2(xx, k), zl, zh);
+    m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
+    const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
+    // round to nearest on the grid (ties to the even code), then dequantise
+    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
+    const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    const float vh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    upk(mul2(mul2(pk(vl, vh), k.sbv2), k.sg2), ql, qh);
+  }
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+// One 16-element block of the fake-quant forward: bf16 outputs and 16 mask
+// bits.  side: kGuided -- the block's 16 cached bits; kFull -- its 16
+// rollout codes (c0: elements 0-7, c1: 8-15).
+template <int MODE>
+__device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, uint32_t c0,
+                                                 uint32_t c1, float sbv, float s_g, V8& o,
+                                                 uint32_t& m) {
+  const float d = __fmul_rn(s_g, sbv);
+  m = 0u;
+  if (d == 0.0f) {
+    // zero block: z = +-0, output +-0, mask set
+#pragma unroll
+    for (int k = 0; k < 8; ++k) o.w[k] = v.w[k] & 0x80008000u;
+    m = 0xFFFFu;
+  } else if (fast_scale(d, MODE != kRtn ? kDMaxExactZ : kDMax)) {
+    const BlkK bk = make_blk(d, MODE != kRtn ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t side = MODE == kGuided ? bits16 >> (2 * k)
+                          : MODE == kFull ? ((k < 4 ? c0 : c1) >> (8 * (k & 3))) : 0u;
+      o.w[k] = fq_pair<MODE>(v.w[k], side, bk, m, 2 * k);
+    }
+  } else {
+    fake_quant_block_exact(v, d, sbv, s_g, bits16, c0, c1, MODE, &o, &m);
+  }
+}
+
+// Each thread owns two adjacent blocks, so their mantissa bits, scales and
+// mask move as one 32-bit / 16-bit / 32-bit access (the full codes as one
+// 16-byte access).
+// MINB: resident CTAs per SM the register budget is cut for.  The
+// full-information forward has a second build at 2 CTAs per SM for large
+// tensors: each thread then walks several tiles, and with the larger register
+// budget it ran 16% faster on B200 at 268M elements (and 13% slower at 33M,
+// where a thread sees one tile).
+template <int MODE, bool SW, int MINB = kCtasPerSm>
+__global__ void __launch_bounds__(kThreads, MINB)
+    k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+                 const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
+                 const uint8_t* __restrict__ scales, const float* __restrict__ gscale,
+                 V8* __restrict__ out, uint32_t* __restrict__ mask) {
+  pdl_begin();
+  GroupCursor gc;
+  gc.init(offs, sh.G);
+  float s_g = 1.0f;
+
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+    const uint32_t sb2 =
+        SW ? __ldcs(reinterpret_cast<const unsigned short*>(
+                 scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
+           : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
+    if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
+    V8 o;
+    uint32_t m0, m1;
+    fake_quant_block<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
+    st_block(out + b, o);
+    // a row holds a whole number of 32-element words, so both blocks of the
+    // pair are in the same row and group
+    fake_quant_block<MODE>(v1, bits >> 16, rc.z, rc.w, e4m3_to_f32(sb2 >> 8), s_g, o, m1);
+    st_block(out + b + 1, o);
+    mask[b >> 1] = m0 | (m1 << 16);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 4: masked straight-through backward.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint32_t* __restrict__ mask,
+              V8* __restrict__ gin) {
+  pdl_begin();
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
+    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // two adjacent blocks
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(g + b), v1 = ld_block_stream(g + b + 1);
+    const uint32_t m = __ldcs(mask + (b >> 1));
+    V8 r0, r1;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      // bits (2k, 2k+1) -> keep masks of the two halves of word k
+      r0.w[k] = v0.w[k] & ((((m >> (2 * k)) & 1u) * 0x0000FFFFu) |
+                           (((m >> (2 * k + 1)) & 1u) * 0xFFFF0000u));
+      r1.w[k] = v1.w[k] & ((((m >> (2 * k + 16)) & 1u) * 0x0000FFFFu) |
+                           (((m >> (2 * k + 17)) & 1u) * 0xFFFF0000u));
+    }
+    st_block(gin + b, r0);
+    st_block(gin + b + 1, r1);
+  }
+}

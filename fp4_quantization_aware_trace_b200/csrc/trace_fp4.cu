@@ -52,6 +52,10 @@
 //     outside [2^-90, 2^100] ([2^-90, 2^16] for the guided forward) go
 //     through an exact per-element path that divides with IEEE
 //     round-to-nearest.
+// File layout: this file holds the host side and the C ABI; the kernels are
+// in csrc/*.cuh, included below inside this file's anonymous namespace (one
+// translation unit): common.cuh (shared device helpers), nvfp4.cuh, mismatch.cuh,
+// mx.cuh, util.cuh.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -61,1268 +65,11 @@
 
 namespace {
 
-typedef unsigned long long u64;
-
-constexpr int kThreads = 256;
-constexpr int kBlkPerThread = 2;
-constexpr int kTileBlks = kThreads * kBlkPerThread;  // 512 blocks = 8192 elements
-constexpr int kCtasPerSm = 4;    // resident CTAs per SM the register budget allows
-constexpr int kGridPerSm = 32;   // CTAs launched per SM: about one tile each
-constexpr int kAmaxTable = 256;  // groups per CTA kept in shared memory
-
-constexpr uint32_t kDMin = 0x12800000u;     // 2^-90: fast paths need d >= 2^-90
-constexpr uint32_t kDMax = 0x71800000u;     // 2^100: capture / round-to-nearest
-constexpr uint32_t kDMaxExactZ = 0x47800000u;  // 2^16: guided (see below)
-// The guided path divides |x| * 2^64: every nonzero bf16 then has a normal
-// quotient and an exactly representable remainder for d in the fast range.
-constexpr float kXs = 0x1p64f;
-constexpr float kSixS = 0x1p64f * 6.0f;
-
-// ---------------------------------------------------------------------------
-// Programmatic dependent launch (sm_90+): every kernel waits for the
-// previous kernel in the stream to complete before it reads any global
-// memory, then lets the next kernel start launching.  Launched with the
-// programmatic-serialization attribute, a kernel's launch and prologue
-// overlap the tail of the one before it; launched without it, both
-// instructions are no-ops.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ void pdl_begin() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
-// ---------------------------------------------------------------------------
-// Fast unsigned 32-bit division by a runtime constant (Granlund & Montgomery,
-// "Division by invariant integers using multiplication", PLDI 1994, the
-// round-up method with the add-back step): block index -> row.
-// ---------------------------------------------------------------------------
-struct FastDiv {
-  uint32_t d, m, s;  // s = ceil(log2 d); d <= 1 handled separately
-};
-
-FastDiv make_fastdiv(uint32_t d) {
-  FastDiv f{d, 0u, 0u};
-  if (d <= 1) return f;
-  uint32_t l = 0;
-  while ((1ull << l) < d) ++l;
-  f.s = l;
-  f.m = (uint32_t)((((1ull << l) - d) << 32) / d + 1ull);
-  return f;
-}
-
-__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv& f) {
-  if (f.d <= 1) return n;
-  uint32_t t = __umulhi(n, f.m);
-  return (t + ((n - t) >> 1)) >> (f.s - 1);
-}
-
-// ---------------------------------------------------------------------------
-// Memory access (public PTX ISA: 32-byte vector loads/stores on sm_100)
-// ---------------------------------------------------------------------------
-struct V8 {
-  uint32_t w[8];
-};
-
-// One 16-element bf16 block; read once, not kept in L1.
-__device__ __forceinline__ V8 ld_block_stream(const void* p) {
-  V8 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
-                 "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
-               : "l"(p));
-  return v;
-}
-
-__device__ __forceinline__ void st_block(void* p, const V8& v) {
-  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
-               "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
-               "r"(v.w[7])
-               : "memory");
-}
-
-__device__ __forceinline__ V8 zero_block() {
-  V8 v;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v.w[k] = 0u;
-  return v;
-}
-
-// ---------------------------------------------------------------------------
-// Packed fp32x2 arithmetic (public PTX ISA, sm_100: mul/fma/add/sub .f32x2)
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ u64 pk(float lo, float hi) {
-  u64 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void upk(u64 v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
-  u64 r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
-  u64 r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ u64 add_rm2(u64 a, u64 b) {
-  u64 r;
-  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ u64 add_rp2(u64 a, u64 b) {
-  u64 r;
-  asm("add.rp.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ u64 sub2(u64 a, u64 b) {
-  u64 r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
-// ---------------------------------------------------------------------------
-// Number-format helpers (hardware conversions from the public PTX ISA)
-// ---------------------------------------------------------------------------
-
-// Two fp32 -> one byte of two E2M1 codes (round to nearest even, satfinite):
-// lo in bits 0-3, hi in bits 4-7; the sign of each input is kept.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint16_t r;
-  asm("{\n\t.reg .b8 b;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
-      "cvt.u16.u8 %0, b;\n\t}"
-      : "=h"(r)
-      : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Byte of two E2M1 codes -> f16x2 (exact): lo code in the low half.
-__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 b;\n\t"
-      "cvt.u8.u32 b, %1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
-      : "=r"(r)
-      : "r"(byte));
-  return r;
-}
-
-// fp32 >= 0 -> E4M3 byte (round to nearest even, saturating at 448).
-__device__ __forceinline__ uint32_t cvt_e4m3(float t) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
-  return (uint32_t)(r & 0xFFu);
-}
-
-// E4M3 byte -> fp32 (exact, through f16).
-__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-  uint32_t h2;
-  uint16_t in = (uint16_t)b;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-}
-
-// Two fp32 -> bf16x2 (round to nearest even): lo in the low half.
-__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-// max|x| over a block as bf16 bits (integer order = magnitude order).
-__device__ __forceinline__ uint32_t absmax_block(const V8& v) {
-  uint32_t m = __vmaxu2(v.w[0] & 0x7FFF7FFFu, v.w[1] & 0x7FFF7FFFu);
-#pragma unroll
-  for (int k = 2; k < 8; ++k) m = __vmaxu2(m, v.w[k] & 0x7FFF7FFFu);
-  return max(m & 0xFFFFu, m >> 16);
-}
-
-// Bit j of the result = bit 4j of n (the lowest bit of each nibble).
-__device__ __forceinline__ uint32_t nibble_lsbs(uint32_t n) {
-  uint32_t c = n & 0x11111111u;
-  c = (c | (c >> 3)) & 0x03030303u;
-  c = (c | (c >> 6)) & 0x000F000Fu;
-  return (c | (c >> 12)) & 0xFFu;
-}
-
-// Per-block constants of the fast path.
-struct BlkK {
-  u64 rr;    // (r, r), r = RN(1/d)
-  u64 ndd;   // (-d, -d)
-  u64 sbv2;  // (s_b, s_b), times 2^-64 on the guided path
-  u64 sg2;   // (s_g, s_g)
-};
-
-__device__ __forceinline__ BlkK make_blk(float d, float sbv, float s_g) {
-  BlkK k;
-  const float r = __frcp_rn(d);
-  k.rr = pk(r, r);
-  k.ndd = pk(-d, -d);
-  k.sbv2 = pk(sbv, sbv);
-  k.sg2 = pk(s_g, s_g);
-  return k;
-}
-
-// 0xFFFFFFFF when a <= b (false for NaN), else 0.
-__device__ __forceinline__ uint32_t le_mask(float a, float b) {
-  uint32_t r;
-  asm("set.le.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
-  return r;
-}
-
-__device__ __forceinline__ bool fast_scale(float d, uint32_t dmax_bits = kDMax) {
-  const uint32_t db = __float_as_uint(d);
-  return db >= kDMin && db <= dmax_bits;
-}
-
-// Correctly rounded quotients of a pair: (lo, hi) / d.
-__device__ __forceinline__ u64 quot2(u64 xx, const BlkK& k) {
-  const u64 q0 = mul2(xx, k.rr);
-  const u64 e = fma2(q0, k.ndd, xx);
-  return fma2(e, k.rr, q0);
-}
-
-// Magic addend of the grid rounding for a = min(|z|, 6) * 2^64:
-// M = 2^86 * max(1, 2^E), E the binade of a / 2^64.
-__device__ __forceinline__ float grid_magic_s(float a_s) {
-  return __uint_as_float(max((__float_as_uint(a_s) & 0x7F800000u) + 0x0B000000u, 0x6A800000u));
-}
-
-// ---- exact path: the format's steps with an IEEE division -----------------
-
-struct Exact {
-  int rtn;     // round-to-nearest magnitude code of clip(|z|)
-  int floor;   // largest code with value <= clip(|z|)
-  bool exact;  // clip(|z|) is a codeword (bracket collapses)
-  bool in;     // |z| <= 6 (STE mask)
-};
-
-__device__ __forceinline__ Exact exact_site(float xf, float d) {
-  const float z = (d == 0.0f) ? copysignf(0.0f, xf) : __fdiv_rn(xf, d);
-  const float a = fabsf(z);
-  Exact e;
-  e.in = a <= 6.0f;
-  const float c = fminf(a, 6.0f);
-  e.rtn = (c <= 0.25f) ? 0 : (c < 0.75f) ? 1 : (c <= 1.25f) ? 2 : (c < 1.75f) ? 3
-        : (c <= 2.5f) ? 4 : (c < 3.5f) ? 5 : (c <= 5.0f) ? 6 : 7;
-  e.floor = (c < 0.5f) ? 0 : (c < 1.0f) ? 1 : (c < 1.5f) ? 2 : (c < 2.0f) ? 3
-          : (c < 3.0f) ? 4 : (c < 4.0f) ? 5 : (c < 6.0f) ? 6 : 7;
-  const float v = (e.floor == 0) ? 0.0f : (e.floor == 1) ? 0.5f : (e.floor == 2) ? 1.0f
-                : (e.floor == 3) ? 1.5f : (e.floor == 4) ? 2.0f : (e.floor == 5) ? 3.0f
-                : (e.floor == 6) ? 4.0f : 6.0f;
-  e.exact = (c == v);
-  return e;
-}
-
-// E2M1 magnitude (as fp32) of a code 0..7.
-__device__ __forceinline__ float e2m1_value(int c) {
-  return c >= 2 ? __uint_as_float((uint32_t)(c + 252) << 22) : (c == 1 ? 0.5f : 0.0f);
-}
-
-// Capture of one block on the exact path: 16 codes (sign<<3 | rtn).
-__device__ __noinline__ void capture_block_exact(V8 v, float d, uint32_t* code_lo,
-                                                 uint32_t* code_hi) {
-  uint32_t c[2] = {0u, 0u};
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t w = v.w[j >> 1];
-    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
-    const Exact e = exact_site(xf, d);
-    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
-    c[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << (4 * (j & 7));
-  }
-  *code_lo = c[0];
-  *code_hi = c[1];
-}
-
-// Fake-quant of one block on the exact path: bf16 outputs and STE mask.
-// mode: 0 round-to-nearest, 1 1-bit guided (bits16), 2 full-information
-// guided (rollout codes c0: elements 0-7, c1: 8-15).
-__device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, float s_g,
-                                                    uint32_t bits16, uint32_t c0, uint32_t c1,
-                                                    int mode, V8* out, uint32_t* mask16) {
-  uint32_t m = 0u;
-  for (int k = 0; k < 8; ++k) out->w[k] = 0u;
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t w = v.w[j >> 1];
-    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
-    const Exact e = exact_site(xf, d);
-    int c = e.rtn;
-    if (mode == 1) {
-      const int bit = (int)((bits16 >> j) & 1u);
-      c = e.exact ? e.floor : e.floor + ((e.floor ^ bit) & 1);
-    } else if (mode == 2) {
-      // nearest of floor / ceiling to the rollout value on z's side of zero
-      const uint32_t rc = ((j < 8 ? c0 : c1) >> (4 * (j & 7))) & 0xFu;
-      float q = e2m1_value((int)(rc & 7u));
-      const bool neg_roll = (rc & 8u) != 0u, neg_z = ((w >> ((j & 1) ? 31 : 15)) & 1u) != 0u;
-      if (neg_roll != neg_z) q = -q;
-      const int hi = e.exact ? e.floor : e.floor + 1;
-      c = (q > e2m1_value(e.floor)) ? hi : e.floor;
-    }
-    const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
-        __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
-    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
-    out->w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
-    m |= (uint32_t)e.in << j;
-  }
-  *mask16 = m;
-}
-
-// ---------------------------------------------------------------------------
-// Group lookup: offsets[g] <= row < offsets[g+1], cached per thread.
-// ---------------------------------------------------------------------------
-struct GroupCursor {
-  const int64_t* offs;
-  int G;
-  uint32_t lo, hi;  // cached row range of group g
-  int g;
-
-  __device__ void init(const int64_t* o, int G_) {
-    offs = o;
-    G = G_;
-    lo = 1u;
-    hi = 0u;
-    g = 0;
-  }
-  // returns true when the group changed
-  __device__ __forceinline__ bool seek(uint32_t row) {
-    if (G == 1) {
-      if (lo == 0u) return false;
-      g = 0;
-      lo = 0u;
-      hi = 0xFFFFFFFFu;
-      return true;
-    }
-    if (row >= lo && row < hi) return false;
-    int a = 0, b = G;  // last g with offs[g] <= row
-    while (b - a > 1) {
-      const int m = (a + b) >> 1;
-      if ((uint64_t)offs[m] <= row) a = m; else b = m;
-    }
-    g = a;
-    lo = (uint32_t)offs[a];
-    hi = (uint32_t)offs[a + 1];
-    return true;
-  }
-};
-
-struct Shape {
-  uint32_t nblk;    // N / 16
-  uint32_t ntiles;  // ceil(nblk / kTileBlks)
-  FastDiv bpr;      // blocks per row
-  int G;
-  uint32_t sw_ct;   // tiled scale layout: 128 x 4 tiles per row of tiles
-};
-
-// Byte offset of the scale at (row, col) in the tiled layout a block-scaled
-// FP4 GEMM reads: the scale matrix cut into 128-row x 4-column tiles of 512
-// bytes, stored in row-major tile order (ct tiles per row of tiles); inside
-// a tile, row r and column c sit at 16 (r mod 32) + 4 (r div 32) + c.
-__device__ __forceinline__ size_t tiled_scale_offset(uint32_t row, uint32_t col, uint32_t ct) {
-  return ((size_t)(row >> 7) * ct + (col >> 2)) * 512u + ((row & 31u) << 4) +
-         (((row >> 5) & 3u) << 2) + (col & 3u);
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 0: zero the per-group amax accumulators.
-// ---------------------------------------------------------------------------
-__global__ void k_zero_u32(uint32_t* p, int n) {
-  pdl_begin();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0u;
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 1: per-group amax (bits of max|x| as bf16, kept as u32 so that
-// atomicMax orders them as magnitudes).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_amax(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-           uint32_t* __restrict__ amax) {
-  __shared__ uint32_t table[kAmaxTable];
-  __shared__ int g_first_s;
-  pdl_begin();
-  if (blockIdx.x >= sh.ntiles) return;
-
-  GroupCursor gc;
-  gc.init(offs, sh.G);
-  if (threadIdx.x == 0) {
-    gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
-    g_first_s = gc.g;
-  }
-  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
-  __syncthreads();
-  const int g_first = g_first_s;
-  gc.init(offs, sh.G);
-
-  uint32_t run = 0u;
-  int run_g = -1;
-  auto flush = [&](int g, uint32_t val) {
-    if (g < 0 || val == 0u) return;
-    const int slot = g - g_first;
-    if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
-    else atomicMax(&amax[g], val);
-  };
-
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    V8 v[kBlkPerThread];
-    const uint32_t base = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
-    }
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      if (b >= sh.nblk) continue;
-      if (sh.G > 1) {
-        gc.seek(fastdiv(b, sh.bpr));
-        if (gc.g != run_g) {
-          flush(run_g, run);
-          run = 0u;
-          run_g = gc.g;
-        }
-      } else {
-        run_g = 0;
-      }
-      run = max(run, absmax_block(v[u]));
-    }
-  }
-  if (sh.G == 1) {
-    for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
-    if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
-  } else {
-    flush(run_g, run);
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
-    const uint32_t val = table[i];
-    if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
-  }
-}
-
-// Per-group constants of capture.
-struct GroupK {
-  float s_g;    // amax / 2688, or 1
-  float den6;   // RN(6 * s_g)
-  float r6;     // RN(1 / den6)
-  bool fast6;   // den6 in the range where bmax/den6 may use the FMA quotient
-};
-
-__device__ __forceinline__ GroupK group_consts(uint32_t amax_bits) {
-  GroupK k;
-  const float a = __uint_as_float(amax_bits << 16);
-  k.s_g = amax_bits == 0u ? 1.0f : __fdiv_rn(a, 2688.0f);
-  k.den6 = __fmul_rn(6.0f, k.s_g);
-  k.fast6 = fast_scale(k.den6);
-  k.r6 = k.fast6 ? __frcp_rn(k.den6) : 0.0f;
-  return k;
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 2: capture.  Per 16-element block: E4M3 scale; per element: the
-// round-to-nearest code and its mantissa bit.
-// ---------------------------------------------------------------------------
-// One block: returns its E4M3 scale byte, writes its 16 codes to c0 (elements
-// 0-7) and c1 (8-15).
-__device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk, uint32_t& c0,
-                                                  uint32_t& c1) {
-  // block scale: t = bmax / RN(6 s_g), E4M3 round-to-nearest-even, satfinite
-  const float bmax = __uint_as_float(absmax_block(v) << 16);
-  float tq;
-  if (gk.fast6) {
-    const float q0 = __fmul_rn(bmax, gk.r6);
-    tq = __fmaf_rn(__fmaf_rn(q0, -gk.den6, bmax), gk.r6, q0);
-  } else {
-    tq = __fdiv_rn(bmax, gk.den6);
-  }
-  const uint32_t sb = cvt_e4m3(tq);
-  const float d = __fmul_rn(gk.s_g, e4m3_to_f32(sb));
-  if (d == 0.0f) {
-    // zero block: z = +-0, code = sign only
-    c0 = c1 = 0u;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t w = v.w[k];
-      const uint32_t nib = (((w >> 15) & 1u) << 3) | ((w >> 31) << 7);
-      if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
-    }
-  } else if (fast_scale(d)) {
-    const BlkK bk = make_blk(d, 0.0f, 0.0f);
-    uint32_t c[2] = {0u, 0u};
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t w = v.w[k];
-      const float xl = bf16_lo(w), xh = bf16_hi(w);
-      float zl, zh;
-      upk(quot2(pk(xl, xh), bk), zl, zh);
-      // the code carries the sign of x (also for zeros and underflows)
-      zl = __uint_as_float((__float_as_uint(zl) & 0x7FFFFFFFu) | (__float_as_uint(xl) & 0x80000000u));
-      zh = __uint_as_float((__float_as_uint(zh) & 0x7FFFFFFFu) | (w & 0x80000000u));
-      c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
-    }
-    c0 = c[0];
-    c1 = c[1];
-  } else {
-    capture_block_exact(v, d, &c0, &c1);
-  }
-  return sb;
-}
-
-// Each thread owns two adjacent blocks: one 16-byte store of codes, one
-// 32-bit store of mantissa bits, one 16-bit store of scales.
-// SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
-template <bool SW>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-              const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
-              uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales,
-              float* __restrict__ gscale) {
-  pdl_begin();
-  // global scales of all groups (any CTA may write them; all write the same)
-  for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
-    gscale[g] = group_consts(amax[g]).s_g;
-
-  GroupCursor gc;
-  gc.init(offs, sh.G);
-  GroupK gk = group_consts(0u);
-
-  // tiles in reverse order: k_amax read the high tiles last, so they are the
-  // most likely to be still in L2
-  for (uint32_t i = blockIdx.x; i < sh.ntiles; i += gridDim.x) {
-    const uint32_t t = sh.ntiles - 1u - i;
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    // both blocks of the pair are in the same row (cols is a multiple of 32)
-    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-    if (gc.seek(row)) gk = group_consts(__ldg(amax + gc.g));
-    uint4 c;
-    const uint32_t s0 = capture_block(v0, gk, c.x, c.y);
-    const uint32_t s1 = capture_block(v1, gk, c.z, c.w);
-    codes[b >> 1] = c;
-    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
-                    (nibble_lsbs(c.w) << 24);
-    const uint16_t sv = (uint16_t)(s0 | (s1 << 8));
-    if (SW)  // the pair's two columns are neighbours inside one tile
-      *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
-    else
-      reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 3/5: fake-quant forward with given scales: bf16 q*·s and the STE
-// mask, q* chosen by round-to-nearest, by the cached mantissa bit, or by the
-// whole rollout code.
-// ---------------------------------------------------------------------------
-// Fake-quant modes: round to nearest (vanilla QAT), 1-bit guided (TRACE's
-// compact cache), full-information guided (the cache keeps the whole code).
-enum FqMode { kRtn = 0, kGuided = 1, kFull = 2 };
-
-// Two elements (one bf16x2 word w) of the fake-quant forward.  `side` carries
-// the guidance of the pair: MODE kGuided -- the cached bits of the two
-// elements in bits 0 and 1; kFull -- the rollout's two 4-bit codes (low
-// nibble first).  Mask bits go to positions pos, pos + 1 of m.
-template <int MODE>
-__device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const BlkK& k,
-                                            uint32_t& m, int pos) {
-  // signed x; only |z| is used below (sign of the output comes from w)
-  const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-  float ql, qh;
-  if (MODE != kRtn) {
-    // z * 2^64 (exact; +-inf/NaN only where |x|/d overflows)
-    float zl, zh;
-    upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
-    m |= (le_mask(fabsf(zl), kSixS) & (1u << pos)) | (le_mask(fabsf(zh), kSixS) & (2u << pos));
-    const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
-    const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
-    const u64 aa = pk(al, ah);
-    float lol, loh, hil, hih;
-    upk(add_rm2(aa, MM), lol, loh);
-    upk(add_rp2(aa, MM), hil, hih);
-    if (MODE == kGuided) {
-      // of floor / ceiling, the one whose mantissa bit is the cached bit: the
-      // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
-      // bit of the floor sum is its codeword's mantissa bit
-      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-      const float tl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
-      const float th = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
-      upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
-    } else {
-      // of floor / ceiling, the one nearest the rollout codeword: the
-      // rollout value reflected to z's side of zero picks the ceiling
-      // exactly when it lies above the floor (no codeword lies between)
-      float fl, fh, cl, ch;
-      upk(sub2(pk(lol, loh), MM), fl, fh);
-      upk(sub2(pk(hil, hih), MM), cl, ch);
-      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
-      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
-      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
-      upk(mul2(pk(rl, rh), pk(kXs, kXs)), rl, rh);
-      const float tl = rl > fl ? cl : fl;
-      const float th = rh > fh ? ch : fh;
-      upk(mul2(mul2(pk(tl, th), k.sbv2), k.sg2), ql, qh);
-    }
-  } else {
-    float zl, zh;
-    upk(quot2(xx, k), zl, zh);
-    m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
-    const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
-    // round to nearest on the grid (ties to the even code), then dequantise
-    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
-    const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    const float vh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-    upk(mul2(mul2(pk(vl, vh), k.sbv2), k.sg2), ql, qh);
-  }
-  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
-}
-
-// One 16-element block of the fake-quant forward: bf16 outputs and 16 mask
-// bits.  side: kGuided -- the block's 16 cached bits; kFull -- its 16
-// rollout codes (c0: elements 0-7, c1: 8-15).
-template <int MODE>
-__device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, uint32_t c0,
-                                                 uint32_t c1, float sbv, float s_g, V8& o,
-                                                 uint32_t& m) {
-  const float d = __fmul_rn(s_g, sbv);
-  m = 0u;
-  if (d == 0.0f) {
-    // zero block: z = +-0, output +-0, mask set
-#pragma unroll
-    for (int k = 0; k < 8; ++k) o.w[k] = v.w[k] & 0x80008000u;
-    m = 0xFFFFu;
-  } else if (fast_scale(d, MODE != kRtn ? kDMaxExactZ : kDMax)) {
-    const BlkK bk = make_blk(d, MODE != kRtn ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits16 >> (2 * k)
-                          : MODE == kFull ? ((k < 4 ? c0 : c1) >> (8 * (k & 3))) : 0u;
-      o.w[k] = fq_pair<MODE>(v.w[k], side, bk, m, 2 * k);
-    }
-  } else {
-    fake_quant_block_exact(v, d, sbv, s_g, bits16, c0, c1, MODE, &o, &m);
-  }
-}
-
-// Each thread owns two adjacent blocks, so their mantissa bits, scales and
-// mask move as one 32-bit / 16-bit / 32-bit access (the full codes as one
-// 16-byte access).
-// MINB: resident CTAs per SM the register budget is cut for.  The
-// full-information forward has a second build at 2 CTAs per SM for large
-// tensors: each thread then walks several tiles, and with the larger register
-// budget it ran 16% faster on B200 at 268M elements (and 13% slower at 33M,
-// where a thread sees one tile).
-template <int MODE, bool SW, int MINB = kCtasPerSm>
-__global__ void __launch_bounds__(kThreads, MINB)
-    k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-                 const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
-                 const uint8_t* __restrict__ scales, const float* __restrict__ gscale,
-                 V8* __restrict__ out, uint32_t* __restrict__ mask) {
-  pdl_begin();
-  GroupCursor gc;
-  gc.init(offs, sh.G);
-  float s_g = 1.0f;
-
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
-    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-    const uint32_t sb2 =
-        SW ? __ldcs(reinterpret_cast<const unsigned short*>(
-                 scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
-           : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
-    if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
-    V8 o;
-    uint32_t m0, m1;
-    fake_quant_block<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
-    st_block(out + b, o);
-    // a row holds a whole number of 32-element words, so both blocks of the
-    // pair are in the same row and group
-    fake_quant_block<MODE>(v1, bits >> 16, rc.z, rc.w, e4m3_to_f32(sb2 >> 8), s_g, o, m1);
-    st_block(out + b + 1, o);
-    mask[b >> 1] = m0 | (m1 << 16);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 4: masked straight-through backward.
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_ste_bwd(const V8* __restrict__ g, Shape sh, const uint32_t* __restrict__ mask,
-              V8* __restrict__ gin) {
-  pdl_begin();
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // two adjacent blocks
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(g + b), v1 = ld_block_stream(g + b + 1);
-    const uint32_t m = __ldcs(mask + (b >> 1));
-    V8 r0, r1;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      // bits (2k, 2k+1) -> keep masks of the two halves of word k
-      r0.w[k] = v0.w[k] & ((((m >> (2 * k)) & 1u) * 0x0000FFFFu) |
-                           (((m >> (2 * k + 1)) & 1u) * 0xFFFF0000u));
-      r1.w[k] = v1.w[k] & ((((m >> (2 * k + 16)) & 1u) * 0x0000FFFFu) |
-                           (((m >> (2 * k + 17)) & 1u) * 0xFFFF0000u));
-    }
-    st_block(gin + b, r0);
-    st_block(gin + b + 1, r1);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 7: mismatch diagnostic.  For each element of x_train, with the
-// rollout's scales, the distance on the signed E2M1 ladder (-6 .. -0.5, 0,
-// 0.5 .. 6: 15 points) between the rollout's code and the code each of three
-// training-side rules picks -- round to nearest, 1-bit guided, full-
-// information guided -- counted into 3 x 15 bins (compact-cache paragraph:
-// sites where the two sides disagree are nearly all one codeword apart).
-//
-// The codes of 8 elements travel as 8 nibbles of one 32-bit word, and the
-// three rules, the distances and the counting run on whole words: every
-// per-nibble sum or difference below stays inside 0..15, so no carry or
-// borrow crosses into the next nibble.
-// ---------------------------------------------------------------------------
-constexpr int kHistBins = 15;  // distances 0..14
-constexpr int kHistModes = 3;  // round to nearest, 1-bit guided, full-information guided
-
-// The codes of one block, elements 0-7 in word 0 and 8-15 in word 1: floor
-// and ceiling magnitude codes of clip(|z|) on the grid (equal when it is a
-// codeword) and the round-to-nearest code with the sign of z.
-struct BlockCodes {
-  uint32_t f[2], c[2], r[2];
-};
-
-// One pair on the fast path: as the guided forward, z * 2^64 from |x|, the
-// floor and ceiling by directed rounding on the grid, each scaled back and
-// converted exactly to its code; round to nearest through the hardware
-// conversion (ties to the even code) of min(|z|, 6) with the sign of x.
-__device__ __forceinline__ void codes_pair(uint32_t w, const BlkK& k, uint32_t& fb, uint32_t& cb,
-                                           uint32_t& rb) {
-  const uint32_t wa = w & 0x7FFF7FFFu;
-  const u64 xx = pk(__uint_as_float(wa << 16), __uint_as_float(wa & 0xFFFF0000u));
-  float zl, zh;
-  upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
-  const float al = fminf(zl, kSixS), ah = fminf(zh, kSixS);  // NaN (|x| * 2^64 = inf) -> 6 * 2^64
-  const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
-  const u64 aa = pk(al, ah);
-  const u64 un = pk(0x1p-64f, 0x1p-64f);
-  float fl, fh, cl, ch, rl, rh;
-  upk(mul2(sub2(add_rm2(aa, MM), MM), un), fl, fh);
-  upk(mul2(sub2(add_rp2(aa, MM), MM), un), cl, ch);
-  upk(mul2(aa, un), rl, rh);
-  rl = __uint_as_float(__float_as_uint(rl) | ((w << 16) & 0x80000000u));
-  rh = __uint_as_float(__float_as_uint(rh) | (w & 0x80000000u));
-  fb = cvt_e2m1x2(fl, fh);
-  cb = cvt_e2m1x2(cl, ch);
-  rb = cvt_e2m1x2(rl, rh);
-}
-
-// The same codes on the exact path (d outside the fast range).
-__device__ __noinline__ void codes_block_exact(V8 v, float d, BlockCodes* bc) {
-  uint32_t f[2] = {0u, 0u}, c[2] = {0u, 0u}, r[2] = {0u, 0u};
-  for (int j = 0; j < 16; ++j) {
-    const uint32_t w = v.w[j >> 1];
-    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
-    const Exact e = exact_site(xf, d);
-    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
-    const int sh = 4 * (j & 7);
-    f[j >> 3] |= (uint32_t)e.floor << sh;
-    c[j >> 3] |= (uint32_t)(e.exact ? e.floor : e.floor + 1) << sh;
-    r[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << sh;
-  }
-  for (int h = 0; h < 2; ++h) {
-    bc->f[h] = f[h];
-    bc->c[h] = c[h];
-    bc->r[h] = r[h];
-  }
-}
-
-__device__ __forceinline__ BlockCodes block_codes(const V8& v, float sbv, float s_g) {
-  BlockCodes bc;
-  const float d = __fmul_rn(s_g, sbv);
-  if (d == 0.0f) {
-    // zero block: z = +-0, every code is zero with the sign of x
-    bc.f[0] = bc.f[1] = bc.c[0] = bc.c[1] = 0u;
-    bc.r[0] = bc.r[1] = 0u;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t w = v.w[k];
-      bc.r[k >> 2] |= ((((w >> 15) & 1u) << 3) | ((w >> 31) << 7)) << (8 * (k & 3));
-    }
-  } else if (fast_scale(d, kDMaxExactZ)) {
-    const BlkK bk = make_blk(d, 0.0f, 0.0f);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t fb[4], cb[4], rb[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) codes_pair(v.w[4 * h + k], bk, fb[k], cb[k], rb[k]);
-      bc.f[h] = fb[0] | (fb[1] << 8) | (fb[2] << 16) | (fb[3] << 24);
-      bc.c[h] = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
-      bc.r[h] = rb[0] | (rb[1] << 8) | (rb[2] << 16) | (rb[3] << 24);
-    }
-  } else {
-    codes_block_exact(v, d, &bc);
-  }
-  return bc;
-}
-
-// Ladder distances of 8 nibbles: training magnitude codes t against the
-// rollout magnitudes qm (both 0..7); s15 is 0xF on nibbles where the two
-// signs agree.  Same sign: |t - qm|; opposite signs: t + qm.
-__device__ __forceinline__ uint32_t ladder_dist8(uint32_t t, uint32_t qm, uint32_t s15) {
-  const uint32_t diff = t + 0x88888888u - qm;  // 8 + t - qm, in 1..15
-  const uint32_t ge = diff & 0x88888888u;      // t >= qm
-  const uint32_t m15 = ge | (ge - (ge >> 3));  // 0xF where t >= qm
-  // t >= qm: diff - 8;  t < qm: 8 - diff = (7 - diff) + 1
-  const uint32_t ad = (diff ^ 0x77777777u ^ m15) + 0x11111111u - (ge >> 3);
-  return (ad & s15) | ((t + qm) & ~s15);
-}
-
-// Count 8 distances: ones in a register, two and above (rare) in shared
-// memory; zeros are what is left over at the end.
-__device__ __forceinline__ void count8(uint32_t d, uint32_t& ones, uint32_t* bins) {
-  const uint32_t ge2 = (((d >> 1) & 0x77777777u) + 0x77777777u) & 0x88888888u;  // d >= 2
-  ones += __popc(d & 0x11111111u & ~(ge2 >> 3));
-  for (uint32_t g = ge2; g != 0u; g &= g - 1u) {
-    const int j = (__ffs((int)g) - 1) >> 2;
-    // a distance is at most 14; the clamp only keeps the index in bounds
-    atomicAdd(&bins[min((d >> (4 * j)) & 0xFu, 14u)], 1u);
-  }
-}
-
-// The three rules on 8 elements: f, c, r as in BlockCodes, q the rollout's
-// signed codes.
-__device__ __forceinline__ void hist_word(uint32_t f, uint32_t c, uint32_t r, uint32_t q,
-                                          uint32_t (&ones)[kHistModes], uint32_t* bins) {
-  const uint32_t ne = c - f;  // 1 where the bracket holds two codewords
-  const uint32_t qm = q & 0x77777777u;
-  const uint32_t s8 = ~(q ^ r) & 0x88888888u;  // signs of z and q_roll agree
-  const uint32_t s15 = s8 | (s8 - (s8 >> 3));
-  // round to nearest
-  count8(ladder_dist8(r & 0x77777777u, qm, s15), ones[0], bins);
-  // 1-bit guided: the ceiling where the floor's mantissa bit is not q_roll's
-  count8(ladder_dist8(f + ((f ^ q) & ne), qm, s15), ones[1], bins + kHistBins);
-  // full information: the ceiling where q_roll, on z's side, lies above the
-  // floor (8 + qm - f - 1 has bit 3 set exactly when qm > f)
-  const uint32_t up = ((qm + 0x88888888u - f - 0x11111111u) >> 3) & (s8 >> 3) & ne;
-  count8(ladder_dist8(f + up, qm, s15), ones[2], bins + 2 * kHistBins);
-}
-
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_mismatch_hist(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-                    const uint4* __restrict__ rcodes, const uint16_t* __restrict__ scales,
-                    const float* __restrict__ gscale, unsigned long long* __restrict__ hist) {
-  __shared__ uint32_t bins[kHistModes * kHistBins];
-  __shared__ uint32_t seen;
-  if (threadIdx.x < kHistModes * kHistBins) bins[threadIdx.x] = 0u;
-  if (threadIdx.x == 0) seen = 0u;
-  __syncthreads();
-  pdl_begin();
-  GroupCursor gc;
-  gc.init(offs, sh.G);
-  float s_g = 1.0f;
-  uint32_t ones[kHistModes] = {0u, 0u, 0u}, n = 0u;
-
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const uint4 rc = __ldcs(rcodes + (b >> 1));
-    const uint32_t sb2 = __ldcs(scales + (b >> 1));
-    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
-    const BlockCodes k0 = block_codes(v0, e4m3_to_f32(sb2 & 0xFFu), s_g);
-    hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
-    hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);
-    const BlockCodes k1 = block_codes(v1, e4m3_to_f32(sb2 >> 8), s_g);
-    hist_word(k1.f[0], k1.c[0], k1.r[0], rc.z, ones, bins);
-    hist_word(k1.f[1], k1.c[1], k1.r[1], rc.w, ones, bins);
-    n += 32u;
-  }
-#pragma unroll
-  for (int k = 0; k < kHistModes; ++k) ones[k] = __reduce_add_sync(0xFFFFFFFFu, ones[k]);
-  n = __reduce_add_sync(0xFFFFFFFFu, n);
-  if ((threadIdx.x & 31) == 0) {
-#pragma unroll
-    for (int k = 0; k < kHistModes; ++k) atomicAdd(&bins[k * kHistBins + 1], ones[k]);
-    atomicAdd(&seen, n);
-  }
-  __syncthreads();
-  if (threadIdx.x < kHistModes * kHistBins) {
-    const int k = threadIdx.x / kHistBins, dist = threadIdx.x % kHistBins;
-    uint32_t v = bins[threadIdx.x];
-    if (dist == 0) {
-      uint32_t other = 0u;
-      for (int j = 1; j < kHistBins; ++j) other += bins[k * kHistBins + j];
-      v = seen - other;
-    }
-    if (v != 0u) atomicAdd(hist + threadIdx.x, (unsigned long long)v);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Kernels 8-9: the MXFP4 variant (the post's results list: the method carries
-// over to MXFP4).  OCP Microscaling scales: one E8M0 byte per 32 elements of
-// a row, X = 2^e with e = floor(log2 max|x|) - 2 clamped at -127, and no
-// global scale.  A thread's pair of 16-element blocks is exactly one MX
-// block.  Dividing by a power of two is exact up to the one rounding of the
-// result, so z = x * 2^-e matches z = fl(x / X) with no correction step and
-// no exact path; the E2M1 decisions are those of the NVFP4 kernels.
-// ---------------------------------------------------------------------------
-
-// 2^k as fp32 for k in [-127, 127] (2^-127 is a subnormal).
-__device__ __forceinline__ float pow2f(int k) {
-  return __uint_as_float(k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00800000u >> (-126 - k));
-}
-
-// E8M0 exponent of a block whose max|x| has the bf16 bits amax (sign
-// cleared): floor(log2 amax) - 2, at least -127 (a bf16 amax stays below
-// 2^128, so the top of the range is never reached); -127 for an all-zero
-// block.
-__device__ __forceinline__ int mx_exp(uint32_t amax) {
-  if (amax == 0u) return -127;
-  const int e = (int)(amax >> 7);
-  const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;  // bf16 subnormal: m * 2^-133
-  return max(fl - 2, -127);
-}
-
-// Magic addend of the grid rounding for a = min(|z|, 6) (unscaled):
-// M = 2^22 * max(1, 2^E).
-__device__ __forceinline__ float grid_magic(float a) {
-  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
-}
-
-// Codes of one 16-element block: c0 elements 0-7, c1 elements 8-15.
-__device__ __forceinline__ void mx_codes_block(const V8& v, u64 inv2, uint32_t& c0, uint32_t& c1) {
-  uint32_t c[2] = {0u, 0u};
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t w = v.w[k];
-    float zl, zh;
-    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
-    // |z| < 8 from the block's own maximum; the conversion saturates past 6
-    // and keeps the sign of x, also on zeros
-    c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
-  }
-  c0 = c[0];
-  c1 = c[1];
-}
-
-template <bool SW>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_mx_capture(const V8* __restrict__ x, Shape sh, uint4* __restrict__ codes,
-                 uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
-  pdl_begin();
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const int e = mx_exp(max(absmax_block(v0), absmax_block(v1)));
-    const float inv = pow2f(-e);
-    const u64 inv2 = pk(inv, inv);
-    uint4 c;
-    mx_codes_block(v0, inv2, c.x, c.y);
-    mx_codes_block(v1, inv2, c.z, c.w);
-    codes[b >> 1] = c;
-    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
-                    (nibble_lsbs(c.w) << 24);
-    if (SW) {
-      const uint32_t row = fastdiv(b, sh.bpr);
-      scales[tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct)] = (uint8_t)(e + 127);
-    } else {
-      scales[b >> 1] = (uint8_t)(e + 127);
-    }
-  }
-}
-
-// Two elements of the MX fake-quant forward (side as fq_pair).
-template <int MODE>
-__device__ __forceinline__ uint32_t mx_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
-                                               uint32_t& m, int pos) {
-  float zl, zh;
-  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
-  m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
-  const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
-  float tl, th;  // chosen codeword value
-  if (MODE == kRtn) {
-    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
-    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-  } else {
-    const u64 MM = pk(grid_magic(al), grid_magic(ah));
-    const u64 aa = pk(al, ah);
-    float lol, loh, hil, hih;
-    upk(add_rm2(aa, MM), lol, loh);
-    upk(add_rp2(aa, MM), hil, hih);
-    if (MODE == kGuided) {
-      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
-      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
-      upk(sub2(pk(sl, sh), MM), tl, th);
-    } else {
-      float fl, fh, cl, ch;
-      upk(sub2(pk(lol, loh), MM), fl, fh);
-      upk(sub2(pk(hil, hih), MM), cl, ch);
-      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
-      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
-      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
-      tl = rl > fl ? cl : fl;
-      th = rh > fh ? ch : fh;
-    }
-  }
-  float ql, qh;
-  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
-  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
-}
-
-template <int MODE, bool SW>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_mx_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
-                    const uint4* __restrict__ rcodes, const uint8_t* __restrict__ scales,
-                    V8* __restrict__ out, uint32_t* __restrict__ mask) {
-  pdl_begin();
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
-    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
-    size_t so = b >> 1;
-    if (SW) {
-      const uint32_t row = fastdiv(b, sh.bpr);
-      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
-    }
-    const int e = (int)__ldcs(scales + so) - 127;
-    const float inv = pow2f(-e), X = pow2f(e);
-    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
-    uint32_t m = 0u;
-    V8 o;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
-                          : MODE == kFull ? ((k < 4 ? rc.x : rc.y) >> (8 * (k & 3))) : 0u;
-      o.w[k] = mx_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
-    }
-    st_block(out + b, o);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
-                          : MODE == kFull ? ((k < 4 ? rc.z : rc.w) >> (8 * (k & 3))) : 0u;
-      o.w[k] = mx_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
-    }
-    st_block(out + b + 1, o);
-    mask[b >> 1] = m;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Kernels 10-11: W4A8 -- TRACE on FP8 (E4M3) activations with MX scales (the
-// post's results list names the W4A8 setting).  32-element blocks with an
-// E8M0 scale X = 2^e, e = floor(log2 max|x|) - 8 (448 = 1.75 * 2^8), clamped
-// at -127; z = x * 2^-e exactly as for MXFP4; round to nearest E4M3 (ties to
-// the even mantissa) saturating at 448; one byte per code (sign in bit 7);
-// the cached bit is the lowest bit of the magnitude code; STE mask |z| <= 448.
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ int mx8_exp(uint32_t amax) {
-  if (amax == 0u) return -127;
-  const int e = (int)(amax >> 7);
-  const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;
-  return max(fl - 8, -127);
-}
-
-// Two fp32 -> two E4M3 bytes (round to nearest even, satfinite), lo in bits
-// 0-7; the sign of each input is kept, also on zeros.
-__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Two E4M3 bytes (lo in bits 0-7) -> f16x2 (exact, signed).
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
-  uint32_t h2;
-  uint16_t in = (uint16_t)two;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  return h2;
-}
-
-// Grid addend for the E4M3 grid: M = 2^20 * max(2^-6, 2^E) (E the binade
-// of a <= 448), so that a + M keeps 3 fraction bits of a's binade (2^-9
-// steps below 2^-6, E4M3's subnormal spacing).
-__device__ __forceinline__ float grid_magic8(float a) {
-  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0A000000u, 0x46800000u));
-}
-
-// Lowest bit of each of 4 code bytes -> 4 bits.
-__device__ __forceinline__ uint32_t byte_lsbs(uint32_t w) {
-  return ((w & 0x01010101u) * 0x01020408u) >> 24;
-}
-
-template <bool SW>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_mx8_capture(const V8* __restrict__ x, Shape sh, V8* __restrict__ codes,
-                  uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales) {
-  pdl_begin();
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const int e = mx8_exp(max(absmax_block(v0), absmax_block(v1)));
-    const float inv = pow2f(-e);
-    const u64 inv2 = pk(inv, inv);
-    V8 c;
-    uint32_t bits = 0u;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const uint32_t w = k < 8 ? v0.w[k] : v1.w[k - 8];
-      float zl, zh;
-      upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
-      // |z| < 512 from the block's own maximum; the conversion saturates
-      // past 448 and keeps the sign of x
-      const uint32_t two = cvt_e4m3x2(zl, zh);
-      if (k & 1) c.w[k >> 1] |= two << 16; else c.w[k >> 1] = two;
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) bits |= byte_lsbs(c.w[k]) << (4 * k);
-    st_block(codes + (b >> 1), c);  // one 32-byte store (a struct copy would split it)
-    mbits[b >> 1] = bits;
-    size_t so = b >> 1;
-    if (SW) {
-      const uint32_t row = fastdiv(b, sh.bpr);
-      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
-    }
-    scales[so] = (uint8_t)(e + 127);
-  }
-}
-
-// Two elements of the W4A8 fake-quant forward.  side: kGuided -- the cached
-// bits in bits 0 and 1; kFull -- the two rollout code bytes (low first).
-template <int MODE>
-__device__ __forceinline__ uint32_t mx8_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
-                                                uint32_t& m, int pos) {
-  float zl, zh;
-  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
-  m |= (le_mask(fabsf(zl), 448.0f) & (1u << pos)) | (le_mask(fabsf(zh), 448.0f) & (2u << pos));
-  const float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);
-  float tl, th;
-  if (MODE == kRtn) {
-    const uint32_t h2 = e4m3x2_to_f16x2(cvt_e4m3x2(al, ah));
-    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-  } else {
-    const u64 MM = pk(grid_magic8(al), grid_magic8(ah));
-    const u64 aa = pk(al, ah);
-    float lol, loh, hil, hih;
-    upk(add_rm2(aa, MM), lol, loh);
-    upk(add_rp2(aa, MM), hil, hih);
-    if (MODE == kGuided) {
-      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
-      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
-      upk(sub2(pk(sl, sh), MM), tl, th);
-    } else {
-      float fl, fh, cl, ch;
-      upk(sub2(pk(lol, loh), MM), fl, fh);
-      upk(sub2(pk(hil, hih), MM), cl, ch);
-      const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFFFu);
-      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
-      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
-      tl = rl > fl ? cl : fl;
-      th = rh > fh ? ch : fh;
-    }
-  }
-  float ql, qh;
-  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
-  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
-}
-
-template <int MODE, bool SW>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_mx8_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
-                     const V8* __restrict__ rcodes, const uint8_t* __restrict__ scales,
-                     V8* __restrict__ out, uint32_t* __restrict__ mask) {
-  pdl_begin();
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
-    const V8 rc = MODE == kFull ? ld_block_stream(rcodes + (b >> 1)) : zero_block();
-    size_t so = b >> 1;
-    if (SW) {
-      const uint32_t row = fastdiv(b, sh.bpr);
-      so = tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct);
-    }
-    const int e = (int)__ldcs(scales + so) - 127;
-    const float inv = pow2f(-e), X = pow2f(e);
-    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
-    uint32_t m = 0u;
-    V8 o;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
-                          : MODE == kFull ? rc.w[k >> 1] >> (16 * (k & 1)) : 0u;
-      o.w[k] = mx8_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
-    }
-    st_block(out + b, o);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
-                          : MODE == kFull ? rc.w[4 + (k >> 1)] >> (16 * (k & 1)) : 0u;
-      o.w[k] = mx8_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
-    }
-    st_block(out + b + 1, o);
-    mask[b >> 1] = m;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Self-test kernel: the block-scale rounding (cvt_e4m3, as capture uses it)
-// on fp32 inputs generated from their index, for exhaustive checks.
-// ---------------------------------------------------------------------------
-__global__ void k_selftest_e4m3(uint32_t first_bits, uint32_t count, uint8_t* __restrict__ out) {
-  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < count; i += gridDim.x * blockDim.x)
-    out[i] = (uint8_t)cvt_e4m3(__uint_as_float(first_bits + i));
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 6: plain copy with the same access pattern (bandwidth yardstick).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_copy(const V8* __restrict__ s, Shape sh, V8* __restrict__ d) {
-  pdl_begin();
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    V8 v[kBlkPerThread];
-    const uint32_t base = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      v[u] = b < sh.nblk ? ld_block_stream(s + b) : zero_block();
-    }
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      if (b < sh.nblk) st_block(d + b, v[u]);
-    }
-  }
-}
+#include "common.cuh"
+#include "nvfp4.cuh"
+#include "mismatch.cuh"
+#include "mx.cuh"
+#include "util.cuh"
 
 // ---------------------------------------------------------------------------
 // Host side
