@@ -59,10 +59,14 @@ class RecordLayout:
 
     @staticmethod
     def of(rows: int, cols: int, num_groups: int = 1) -> "RecordLayout":
-        nb, om, os_, og = ops.trace_cache_record_bytes(rows, cols, num_groups)
-        if nb == 0:
-            raise ops.TraceError(f"invalid record shape [{rows}, {cols}] x {num_groups} groups")
-        return RecordLayout(rows, cols, num_groups, nb, om, os_, og)
+        key = (rows, cols, num_groups)
+        lay = _LAYOUTS.get(key)
+        if lay is None:
+            nb, om, os_, og = ops.trace_cache_record_bytes(rows, cols, num_groups)
+            if nb == 0:
+                raise ops.TraceError(f"invalid record shape [{rows}, {cols}] x {num_groups} groups")
+            lay = _LAYOUTS[key] = RecordLayout(rows, cols, num_groups, nb, om, os_, og)
+        return lay
 
     def view(self, record: torch.Tensor, offsets: torch.Tensor | None = None,
              codes: torch.Tensor | None = None) -> ops.Capture:
@@ -78,6 +82,9 @@ class RecordLayout:
             gscale=record[self.gscale_offset:self.gscale_offset + 4 * self.num_groups].view(
                 torch.float32),
             offsets=offsets)
+
+
+_LAYOUTS: dict = {}  # (rows, cols, groups) -> RecordLayout (pure host arithmetic, cached)
 
 
 @dataclasses.dataclass
@@ -117,7 +124,8 @@ class CacheTier:
         i = self._next.get(lay, 0)
         self._next[lay] = (i + 1) % self.ring
         if i == len(slots):
-            slots.append([torch.empty(lay.nbytes, dtype=torch.uint8, device=self.device), None])
+            rec = torch.empty(lay.nbytes, dtype=torch.uint8, device=self.device)
+            slots.append([rec, None, {}])  # record, event of its last copy, cached views
         return slots[i]
 
     def _workspace(self, G: int, rows: int, cols: int) -> torch.Tensor:
@@ -148,7 +156,12 @@ class CacheTier:
         slot = self._slot(lay)
         if slot[1] is not None:
             stream.wait_event(slot[1])        # the slot's previous copy is done
-        cap = lay.view(slot[0], offsets, codes)
+        views = slot[2]
+        vkey = (id(offsets), id(codes))
+        cap = views.get(vkey)
+        if cap is None or cap.offsets is not offsets or cap.codes is not codes:
+            views.clear()
+            cap = views[vkey] = lay.view(slot[0], offsets, codes)
         ops.capture(x, offsets, cap, self._workspace(G, rows, cols), stream)
         ready = torch.cuda.Event()
         ready.record(stream)
