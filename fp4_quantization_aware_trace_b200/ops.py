@@ -35,6 +35,9 @@ def library() -> ctypes.CDLL:
     """Load libtrace_fp4.so (raises if it is missing: build it with
     ``python -c 'import __graft_entry__ as g; g.build()'``)."""
     global _lib
+    lib = _lib
+    if lib is not None:  # loaded: no lock on the per-call path
+        return lib
     with _lock:
         if _lib is not None:
             return _lib
