@@ -616,9 +616,49 @@ def mismatch_histogram(x_train: torch.Tensor, cache: Capture, hist: torch.Tensor
     return hist
 
 
+_FORWARDS = {
+    ("nvfp4", "guided"): lambda x, c: guided_fq_fwd(x, c),
+    ("nvfp4", "full"): lambda x, c: full_guided_fq_fwd(x, c),
+    ("nvfp4", "rtn"): lambda x, c: rtn_fq_fwd(x, c.scales, c.gscale, c.offsets),
+    ("mxfp4", "guided"): lambda x, c: mx_guided_fq_fwd(x, c),
+    ("mxfp4", "full"): lambda x, c: mx_full_guided_fq_fwd(x, c),
+    ("mxfp4", "rtn"): lambda x, c: mx_rtn_fq_fwd(x, c.scales),
+    ("w4a8", "guided"): lambda x, c: mx8_guided_fq_fwd(x, c),
+    ("w4a8", "full"): lambda x, c: mx8_full_guided_fq_fwd(x, c),
+    ("w4a8", "rtn"): lambda x, c: mx8_rtn_fq_fwd(x, c.scales),
+}
+
+
+class TraceFakeQuant(torch.autograd.Function):
+    """Autograd wrapper: forward = the fake-quant forward of `fmt` ("nvfp4",
+    "mxfp4", "w4a8") with `rule` ("guided": the 1-bit cache, "full": the
+    whole rollout codes, "rtn": round to nearest with the rollout's scales)
+    against a rollout capture of that format; backward = the masked
+    straight-through estimator.  Both run in the library."""
+
+    @staticmethod
+    def forward(ctx, x_train, cache, fmt="nvfp4", rule="guided"):
+        fwd = _FORWARDS.get((fmt, rule))
+        if fwd is None:
+            raise TraceError(f"unknown format / rule {fmt!r} / {rule!r}")
+        out, mask = fwd(x_train, cache)
+        ctx.save_for_backward(mask)
+        return out
+
+    @staticmethod
+    def backward(ctx, grad):
+        (mask,) = ctx.saved_tensors
+        return fq_bwd(grad.contiguous(), mask), None, None, None
+
+
+def trace_fake_quant(x_train: torch.Tensor, cache, fmt: str = "nvfp4", rule: str = "guided"):
+    """Differentiable fake-quant of x_train guided by a rollout capture."""
+    return TraceFakeQuant.apply(x_train, cache, fmt, rule)
+
+
 class GuidedFakeQuant(torch.autograd.Function):
-    """Autograd wrapper: forward = guided fake-quant with the rollout cache,
-    backward = masked straight-through estimator (both in the library)."""
+    """NVFP4 1-bit guided forward with the masked straight-through backward
+    (the common case of TraceFakeQuant)."""
 
     @staticmethod
     def forward(ctx, x_train, cache: Capture):
