@@ -132,6 +132,8 @@ def _load():
         lib.oracle_mx8_full_guided_fwd.restype = None
         lib.oracle_mx8_fake_quant_codes.argtypes = [P, i64, i64, P, P, P, P, ctypes.c_int]
         lib.oracle_mx8_fake_quant_codes.restype = None
+        lib.oracle_mx_mismatch_histogram.argtypes = [P, i64, i64, P, P, P]
+        lib.oracle_mx_mismatch_histogram.restype = None
         lib.oracle_e4m3_sweep.argtypes = [ctypes.c_uint32, ctypes.c_uint32, P]
         lib.oracle_e4m3_sweep.restype = None
         lib.oracle_swizzled_scale_bytes.argtypes = [i64, i64]
@@ -559,3 +561,15 @@ def e4m3_sweep(first_bits: int, count: int) -> np.ndarray:
     out = np.zeros(count, np.uint8)
     _load().oracle_e4m3_sweep(first_bits, count, _ptr(out))
     return out
+
+
+def mx_mismatch_histogram(x_train, rcodes, scales):
+    """uint64[3, 15] as mismatch_histogram, with MXFP4 (E8M0) scales."""
+    x = _as_bf16_bits(x_train)
+    rows, cols = x.shape
+    hist = np.zeros(45, np.uint64)
+    _load().oracle_mx_mismatch_histogram(_ptr(x), rows, cols,
+                                         _ptr(np.ascontiguousarray(rcodes, dtype=np.uint8)),
+                                         _ptr(np.ascontiguousarray(scales, dtype=np.uint8)),
+                                         _ptr(hist))
+    return hist.reshape(3, 15)

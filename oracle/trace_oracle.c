@@ -790,3 +790,28 @@ void oracle_e4m3_sweep(uint32_t first, uint32_t count, uint8_t* out) {
     out[i] = oracle_f32_to_e4m3(t);
   }
 }
+
+/* The mismatch diagnostic of oracle_mismatch_histogram for the MXFP4
+ * variant: z = x / X with the rollout's E8M0 scales, the same three rules
+ * and the same 15-point ladder. */
+void oracle_mx_mismatch_histogram(const uint16_t* x, int64_t rows, int64_t cols,
+                                  const uint8_t* rcodes, const uint8_t* scales,
+                                  uint64_t* hist) {
+  assert(cols % 32 == 0);
+  const int64_t n = rows * cols;
+  for (int64_t b = 0; b < n / 32; ++b) {
+    const float X = oracle_e8m0_to_f32(scales[b]);
+    for (int j = 0; j < 32; ++j) {
+      const int64_t i = b * 32 + j;
+      const float z = oracle_bf16_to_f32(x[i]) / X;
+      float a = fabsf(z);
+      if (a > 6.0f) a = 6.0f;
+      const int rc = (rcodes[i / 2] >> (4 * (i & 1))) & 0xF;
+      const int sz = signbit(z) ? 8 : 0;
+      const int lr = ladder(rc);
+      hist[0 * 15 + abs(ladder(sz | oracle_e2m1_rtn(a)) - lr)] += 1;
+      hist[1 * 15 + abs(ladder(sz | oracle_guided_code(a, rc & 1)) - lr)] += 1;
+      hist[2 * 15 + abs(ladder(sz | oracle_full_guided_code(z, rc)) - lr)] += 1;
+    }
+  }
+}

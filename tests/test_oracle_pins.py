@@ -797,3 +797,30 @@ def test_e4m3_encode_vs_torch_dense(oracle_mod):
         first = int(idx[k0])
         got[k0:k1] = oracle_mod.e4m3_sweep(first, int(idx[k1 - 1]) - first + 1)[::97]
     assert np.array_equal(got, ref)
+
+
+def test_mx_mismatch_histogram_vs_codes(oracle_mod):
+    """The MXFP4 histogram re-bins the per-site codes of the pinned MX entry
+    points by grid index, on independent values (sign flips) and on a
+    drifted pair."""
+    rng = np.random.default_rng(78)
+    grid = [float(v) for v, _ in bf.SIGNED_GRID]
+
+    def index(c):
+        return grid.index(float(Fraction(bf._MAGS[c & 7])) * (-1.0 if c & 8 else 1.0) + 0.0)
+
+    xr = (rng.standard_normal((16, 256)) * np.exp(rng.standard_normal((16, 256)))).astype(np.float32)
+    pairs = [(xr, (rng.standard_normal((16, 256)) * 3).astype(np.float32)),
+             (xr, (xr * (1 + 0.05 * rng.standard_normal((16, 256)))).astype(np.float32))]
+    for a, b in pairs:
+        xr_b = inputs.bits(torch.from_numpy(a).to(torch.bfloat16))
+        xt_b = inputs.bits(torch.from_numpy(b).to(torch.bfloat16))
+        codes, mbits, scales = oracle_mod.mx_capture(xr_b)
+        hist = oracle_mod.mx_mismatch_histogram(xt_b, codes, scales)
+        q_roll = oracle_mod.unpack_codes(codes)
+        rules = [oracle_mod.mx_fake_quant_codes(xt_b, scales).reshape(-1),
+                 oracle_mod.mx_fake_quant_codes(xt_b, scales, mbits=mbits).reshape(-1),
+                 oracle_mod.mx_fake_quant_codes(xt_b, scales, rcodes=codes).reshape(-1)]
+        for k in range(3):
+            d = np.array([abs(index(int(p)) - index(int(q))) for p, q in zip(rules[k], q_roll)])
+            assert np.array_equal(hist[k], np.bincount(d, minlength=15)), k
