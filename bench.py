@@ -490,6 +490,7 @@ def run_trace(args):
     # the MXFP4 variant on the same sites: capture, 1-bit guided, RTN and
     # full-guided forwards, each launch timed on its own
     mxc = [ops.mx_capture(w["xr"], stream=stream) for w in work]
+    mx_hist = torch.zeros(3, 15, dtype=torch.int64, device=dev)
 
     def mx_pass(evs):
         for i, w in enumerate(work):
@@ -503,6 +504,8 @@ def run_trace(args):
             if ev: ev[3].record(stream)
             ops.mx_full_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
             if ev: ev[4].record(stream)
+            ops.mx_mismatch_histogram(w["xt"], mxc[i], mx_hist, stream)
+            if ev: ev[5].record(stream)
 
     # capture and guided forward with the scales in the 128 x 4 tiled layout
     # of a block-scaled FP4 GEMM
@@ -567,12 +570,12 @@ def run_trace(args):
     mx_ev = []
     for k in range(args.steps):
         flush.fill_((k + 53) & 0xFF)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in work]
         mx_pass(evs)
         mx_ev.append(evs)
     torch.cuda.synchronize()
     mx_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in mx_ev for i in range(len(work)))
-             for j in range(4)]
+             for j in range(5)]
     mx_ms = max_over_ranks(mx_ms, pg, dev)
 
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
@@ -622,7 +625,8 @@ def run_trace(args):
     for j, (nm, kn, b_k) in enumerate([("capture", "k_mx_capture", 2.65625),
                                        ("guided_fwd", "k_mx_fake_quant<1>", 4.28125),
                                        ("rtn_fwd", "k_mx_fake_quant<0>", 4.15625),
-                                       ("full_guided_fwd", "k_mx_fake_quant<2>", 4.65625)]):
+                                       ("full_guided_fwd", "k_mx_fake_quant<2>", 4.65625),
+                                       ("mismatch_histogram", "k_mismatch_hist<true>", 2.53125)]):
         ms = mx_ms[j] / args.steps
         mx_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": b_k,
                        "gbs": round(n * b_k / (ms * 1e-3) / 1e9, 1),

@@ -240,6 +240,18 @@ __device__ __forceinline__ float grid_magic_s(float a_s) {
   return __uint_as_float(max((__float_as_uint(a_s) & 0x7F800000u) + 0x0B000000u, 0x6A800000u));
 }
 
+// Power-of-two scales and the unscaled grid addend (MX formats).
+// 2^k as fp32 for k in [-127, 127] (2^-127 is a subnormal).
+__device__ __forceinline__ float pow2f(int k) {
+  return __uint_as_float(k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00800000u >> (-126 - k));
+}
+
+// Magic addend of the grid rounding for a = min(|z|, 6) (unscaled):
+// M = 2^22 * max(1, 2^E).
+__device__ __forceinline__ float grid_magic(float a) {
+  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
+}
+
 // ---------------------------------------------------------------------------
 // Group lookup: offsets[g] <= row < offsets[g+1], cached per thread.
 // ---------------------------------------------------------------------------

@@ -100,6 +100,38 @@ __device__ __forceinline__ BlockCodes block_codes(const V8& v, float sbv, float 
   return bc;
 }
 
+// The same codes for an MX block half: z = |x| * 2^-e is exact, so the grid
+// rounding runs on it directly (no quotient, no exact path).
+__device__ __forceinline__ BlockCodes mx_block_codes(const V8& v, u64 inv2) {
+  BlockCodes bc;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t fb[4], cb[4], rb[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t w = v.w[4 * h + k];
+      const uint32_t wa = w & 0x7FFF7FFFu;
+      float zl, zh;
+      upk(mul2(pk(bf16_lo(wa), bf16_hi(wa)), inv2), zl, zh);  // inf only past 6
+      const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);
+      const u64 MM = pk(grid_magic(al), grid_magic(ah));
+      const u64 aa = pk(al, ah);
+      float fl, fh, cl, ch;
+      upk(sub2(add_rm2(aa, MM), MM), fl, fh);
+      upk(sub2(add_rp2(aa, MM), MM), cl, ch);
+      const float rl = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
+      const float rh = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
+      fb[k] = cvt_e2m1x2(fl, fh);
+      cb[k] = cvt_e2m1x2(cl, ch);
+      rb[k] = cvt_e2m1x2(rl, rh);
+    }
+    bc.f[h] = fb[0] | (fb[1] << 8) | (fb[2] << 16) | (fb[3] << 24);
+    bc.c[h] = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
+    bc.r[h] = rb[0] | (rb[1] << 8) | (rb[2] << 16) | (rb[3] << 24);
+  }
+  return bc;
+}
+
 // Ladder distances of 8 nibbles: training magnitude codes t against the
 // rollout magnitudes qm (both 0..7); s15 is 0xF on nibbles where the two
 // signs agree.  Same sign: |t - qm|; opposite signs: t + qm.
@@ -142,9 +174,12 @@ __device__ __forceinline__ void hist_word(uint32_t f, uint32_t c, uint32_t r, ui
   count8(ladder_dist8(f + up, qm, s15), ones[2], bins + 2 * kHistBins);
 }
 
+// MX: MXFP4 scales (one E8M0 byte per thread's pair of blocks, no groups)
+// instead of E4M3 block scales with global scales.
+template <bool MX>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mismatch_hist(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-                    const uint4* __restrict__ rcodes, const uint16_t* __restrict__ scales,
+                    const uint4* __restrict__ rcodes, const uint8_t* __restrict__ scales,
                     const float* __restrict__ gscale, unsigned long long* __restrict__ hist) {
   __shared__ uint32_t bins[kHistModes * kHistBins];
   __shared__ uint32_t seen;
@@ -162,12 +197,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (b >= sh.nblk) continue;
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     const uint4 rc = __ldcs(rcodes + (b >> 1));
-    const uint32_t sb2 = __ldcs(scales + (b >> 1));
-    if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
-    const BlockCodes k0 = block_codes(v0, e4m3_to_f32(sb2 & 0xFFu), s_g);
+    BlockCodes k0, k1;
+    if (MX) {
+      const float inv = pow2f(127 - (int)__ldcs(scales + (b >> 1)));
+      const u64 inv2 = pk(inv, inv);
+      k0 = mx_block_codes(v0, inv2);
+      k1 = mx_block_codes(v1, inv2);
+    } else {
+      const uint32_t sb2 = __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
+      if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
+      k0 = block_codes(v0, e4m3_to_f32(sb2 & 0xFFu), s_g);
+      k1 = block_codes(v1, e4m3_to_f32(sb2 >> 8), s_g);
+    }
     hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
     hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);
-    const BlockCodes k1 = block_codes(v1, e4m3_to_f32(sb2 >> 8), s_g);
     hist_word(k1.f[0], k1.c[0], k1.r[0], rc.z, ones, bins);
     hist_word(k1.f[1], k1.c[1], k1.r[1], rc.w, ones, bins);
     n += 32u;

@@ -13,11 +13,6 @@
 // no exact path; the E2M1 decisions are those of the NVFP4 kernels.
 // ---------------------------------------------------------------------------
 
-// 2^k as fp32 for k in [-127, 127] (2^-127 is a subnormal).
-__device__ __forceinline__ float pow2f(int k) {
-  return __uint_as_float(k >= -126 ? (uint32_t)(k + 127) << 23 : 0x00800000u >> (-126 - k));
-}
-
 // E8M0 exponent of a block whose max|x| has the bf16 bits amax (sign
 // cleared): floor(log2 amax) - 2, at least -127 (a bf16 amax stays below
 // 2^128, so the top of the range is never reached); -127 for an all-zero
@@ -27,12 +22,6 @@ __device__ __forceinline__ int mx_exp(uint32_t amax) {
   const int e = (int)(amax >> 7);
   const int fl = e != 0 ? e - 127 : (31 - __clz((int)amax)) - 133;  // bf16 subnormal: m * 2^-133
   return max(fl - 2, -127);
-}
-
-// Magic addend of the grid rounding for a = min(|z|, 6) (unscaled):
-// M = 2^22 * max(1, 2^E).
-__device__ __forceinline__ float grid_magic(float a) {
-  return __uint_as_float(max((__float_as_uint(a) & 0x7F800000u) + 0x0B000000u, 0x4A800000u));
 }
 
 // Codes of one 16-element block: c0 elements 0-7, c1 elements 8-15.

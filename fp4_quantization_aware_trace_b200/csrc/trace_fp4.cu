@@ -332,9 +332,27 @@ int trace_mismatch_histogram(const uint16_t* x_train, int64_t rows, int64_t cols
   const Shape sh = make_shape(rows, cols, num_groups);
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
-  return launch(k_mismatch_hist, grid, (cudaStream_t)stream, (const V8*)x_train, sh,
-                num_groups > 1 ? group_row_offsets : nullptr, (const uint4*)codes,
-                (const uint16_t*)scales, gscale, (unsigned long long*)hist);
+  return launch(k_mismatch_hist<false>, grid, (cudaStream_t)stream, (const V8*)x_train, sh,
+                num_groups > 1 ? group_row_offsets : nullptr, (const uint4*)codes, scales, gscale,
+                (unsigned long long*)hist);
+}
+
+int trace_mx_mismatch_histogram(const uint16_t* x_train, int64_t rows, int64_t cols,
+                                const uint8_t* codes, const uint8_t* scales, uint64_t* hist,
+                                void* stream) {
+  int st = check_shape(rows, cols, 1, nullptr);
+  if (st) return st;
+  if (!hist) return TRACE_ERR_NULL;
+  if (!aligned(hist, 8)) return TRACE_ERR_ALIGN;
+  if (rows == 0) return TRACE_OK;
+  if (!x_train || !codes || !scales) return TRACE_ERR_NULL;
+  if (!aligned(x_train, 32) || !aligned(codes, 16)) return TRACE_ERR_ALIGN;
+  const Shape sh = make_shape(rows, cols, 1);
+  int grid;
+  if ((st = grid_for(sh, &grid))) return st;
+  return launch(k_mismatch_hist<true>, grid, (cudaStream_t)stream, (const V8*)x_train, sh,
+                (const int64_t*)nullptr, (const uint4*)codes, scales, (const float*)nullptr,
+                (unsigned long long*)hist);
 }
 
 static int mx_capture_impl(const uint16_t* x, int64_t rows, int64_t cols, uint8_t* codes,

@@ -67,6 +67,8 @@ def library() -> ctypes.CDLL:
         lib.trace_capture_static_ws.restype = ctypes.c_int
         lib.trace_mismatch_histogram.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
         lib.trace_mismatch_histogram.restype = ctypes.c_int
+        lib.trace_mx_mismatch_histogram.argtypes = [P, i64, i64, P, P, P, P]
+        lib.trace_mx_mismatch_histogram.restype = ctypes.c_int
         lib.trace_cache_record_bytes.argtypes = [i64, i64, i32, P, P, P]
         lib.trace_cache_record_bytes.restype = sz
         lib.trace_mx_capture.argtypes = [P, i64, i64, P, P, P, P]
@@ -627,6 +629,19 @@ _FORWARDS = {
     ("w4a8", "full"): lambda x, c: mx8_full_guided_fq_fwd(x, c),
     ("w4a8", "rtn"): lambda x, c: mx8_rtn_fq_fwd(x, c.scales),
 }
+
+
+def mx_mismatch_histogram(x_train: torch.Tensor, cache: MxCapture,
+                          hist: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """mismatch_histogram for the MXFP4 variant (E8M0 scales)."""
+    rows, cols = _bf16_2d(x_train)
+    if hist is None:
+        hist = torch.zeros(len(MISMATCH_RULES), MISMATCH_BINS, dtype=torch.int64,
+                           device=x_train.device)
+    _check(library().trace_mx_mismatch_histogram(_p(x_train), rows, cols, _p(cache.codes),
+                                                 _p(cache.scales), _p(hist), _stream(stream)),
+           "trace_mx_mismatch_histogram")
+    return hist
 
 
 class TraceFakeQuant(torch.autograd.Function):

@@ -181,6 +181,13 @@ int trace_mismatch_histogram(const uint16_t* x_train, int64_t rows,
                              const uint8_t* codes, const uint8_t* scales,
                              const float* gscale, uint64_t* hist,
                              void* stream);
+/* The same diagnostic for the MXFP4 variant: z from the rollout's E8M0
+ * scales (uint8[rows, cols/32], row-major, no alignment requirement); codes
+ * as trace_mx_capture writes them; no groups. */
+int trace_mx_mismatch_histogram(const uint16_t* x_train, int64_t rows,
+                                int64_t cols, const uint8_t* codes,
+                                const uint8_t* scales, uint64_t* hist,
+                                void* stream);
 
 /* ---- MXFP4 variant ------------------------------------------------------
  * The post's results list reports that the method carries over to MXFP4.

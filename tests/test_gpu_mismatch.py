@@ -230,3 +230,57 @@ def test_hist_argument_errors():
                                         P(cap.gscale), P(h) + 4, None) == 3
     torch.cuda.synchronize()
     assert int(h.abs().sum()) == 0
+
+
+# --------------------------------------------------------------------------
+# The MXFP4 variant of the diagnostic
+# --------------------------------------------------------------------------
+
+def _mx_check(oracle_mod, xr, xt):
+    cap = ops.mx_capture(xr.to(DEV).contiguous())
+    got = ops.mx_mismatch_histogram(xt.to(DEV).contiguous(), cap)
+    torch.cuda.synchronize()
+    got = got.cpu().numpy().view(np.uint64)
+    xrb, xtb = inputs.bits(xr), inputs.bits(xt)
+    codes, _, scales = oracle_mod.mx_capture(xrb)
+    ref = oracle_mod.mx_mismatch_histogram(xtb, codes, scales)
+    assert np.array_equal(got, ref), f"\n{got}\nvs\n{ref}"
+    return got
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (37, 96), (513, 2048)])
+def test_mx_hist_small_and_special(oracle_mod, rows, cols):
+    s = inputs.tiny_site(rows * 11 + cols, rows, cols, eps=0.05)
+    _mx_check(oracle_mod, s.x_roll, s.x_train)
+    rng = np.random.default_rng(rows)
+    xt = torch.from_numpy((rng.standard_normal((rows, cols)) * 4).astype(np.float32)).to(torch.bfloat16)
+    _mx_check(oracle_mod, s.x_roll, xt)              # independent: sign flips, long distances
+
+
+def test_mx_hist_exhaustive_sweep(oracle_mod):
+    """Every finite bf16 pattern x cycled rollout codes, one launch per E8M0
+    scale byte across capture's range."""
+    p = np.arange(1 << 16, dtype=np.uint32)
+    p = p[((p >> 7) & 0xFF) != 0xFF].astype(np.uint16)
+    pats = np.concatenate([p, np.zeros((-p.size) % 256, np.uint16)]).reshape(-1, 256)
+    slab, C = pats.shape
+    xd = inputs.from_bits(pats, DEV)
+    idx = np.arange(slab * C, dtype=np.int64)
+    hs = []
+    for sb in range(0, 253, 4):
+        nib = ((idx + sb) % 16).astype(np.uint8)
+        rcodes = (nib[0::2] | (nib[1::2] << 4)).astype(np.uint8)
+        scales = np.full((slab, C // 32), sb, np.uint8)
+        cache = ops.MxCapture(codes=torch.from_numpy(rcodes).to(DEV), mbits=None,
+                              scales=torch.from_numpy(scales).to(DEV))
+        hs.append((sb, ops.mx_mismatch_histogram(xd, cache),
+                   oracle_mod.mx_mismatch_histogram(pats, rcodes, scales)))
+    torch.cuda.synchronize()
+    for sb, hg, hr in hs:
+        assert np.array_equal(hg.cpu().numpy().view(np.uint64), hr), f"scale byte {sb}"
+
+
+def test_mx_hist_cfg2(oracle_mod):
+    s = inputs.attention_input(device=DEV)
+    got = _mx_check(oracle_mod, s.x_roll, s.x_train)
+    assert np.all(got.sum(axis=1) == s.x_roll.numel())
