@@ -25,8 +25,9 @@
  *   codes   : uint8[N/2]; byte k holds element 2k in its low nibble and
  *             element 2k+1 in its high nibble.
  *   mbits   : uint32[N/32]; element i is bit (i & 31) of word (i >> 5).
- *   scales  : uint8[rows, cols/16] E4M3 bytes, row-major (linear, not the
- *             swizzled layout of a block-scaled GEMM).
+ *   scales  : uint8[rows, cols/16] E4M3 bytes, row-major (the _ex calls
+ *             further down also read and write the 128 x 4 tiled layout of a
+ *             block-scaled GEMM).
  *   gscale  : float[G], one per group.
  *   ste_mask: uint32[N/32], same packing as mbits; bit set where |z| <= 6
  *             (z before clipping).
@@ -39,8 +40,18 @@
  * pointer owned by the caller; the library never allocates, frees or
  * synchronises.  All calls are asynchronous on `stream` (a cudaStream_t
  * passed as void*, NULL = the legacy default stream).  The library holds no
- * mutable global state apart from a per-device cache of the SM count, so it
- * may be called from several host threads.
+ * mutable global state apart from a per-device cache of the SM count (and
+ * the static scratch of trace_capture_static_ws, see there), so it may be
+ * called from several host threads.  Every call is capturable into a CUDA
+ * graph (trace_capture_static_ws after its first call on the device).
+ *
+ * Contents, in order: status and version; workspace and record-size queries;
+ * the NVFP4 path (capture, 1-bit guided and full-information guided
+ * forwards); the mismatch diagnostic; the MXFP4 (W4A4) and W4A8 variants;
+ * the tiled scale layout (_ex calls); capture's two passes for sharded or
+ * streamed tensors; the straight-through backward and the round-to-nearest
+ * comparator; the E4M3 self-test and the copy yardstick; capture without a
+ * workspace.
  *
  * Errors: arguments are checked on the host before anything is enqueued; a
  * failed check returns its code and enqueues nothing.  A launch failure
