@@ -108,3 +108,47 @@ def test_scale_bytes_query(lib):
     assert lib.trace_scale_bytes(1, 32, 32, 0) == 1
     for bad in [(4, 48, 16, 0), (4, 64, 8, 0), (4, 64, 16, 2), (-1, 64, 16, 0)]:
         assert lib.trace_scale_bytes(*bad) == 0
+
+
+def test_host_argument_checks_newer_calls(lib):
+    """The checks of the calls beyond the core path return before any CUDA
+    call (fake, never dereferenced pointers; no GPU needed)."""
+    P = ctypes.c_void_p
+    a = P(1 << 20)
+    odd = P((1 << 20) + 2)
+    # full-information guidance
+    assert lib.trace_full_guided_fq_fwd(a, 4, 48, 1, None, a, a, a, a, a, None) == 2
+    assert lib.trace_full_guided_fq_fwd(a, 4, 32, 1, None, None, a, a, a, a, None) == 1
+    assert lib.trace_full_guided_fq_fwd(a, 4, 32, 1, None, odd, a, a, a, a, None) == 3
+    # MXFP4 / W4A8
+    for cap in (lib.trace_mx_capture, lib.trace_mx8_capture):
+        assert cap(a, 4, 48, a, a, a, None) == 2
+        assert cap(None, 4, 32, a, a, a, None) == 1
+        assert cap(odd, 4, 32, a, a, a, None) == 3
+    assert lib.trace_mx8_capture(a, 4, 32, P((1 << 20) + 16), a, a, None) == 3   # codes: 32 B
+    for fwd in (lib.trace_mx_guided_fq_fwd, lib.trace_mx8_guided_fq_fwd):
+        assert fwd(a, 4, 32, None, a, a, a, None) == 1
+        assert fwd(a, 4, 32, a, a, odd, a, None) == 3
+    assert lib.trace_mx_rtn_fq_fwd(a, 4, 32, a, a, None, None) == 1
+    assert lib.trace_mx8_rtn_fq_fwd(a, -1, 32, a, a, a, None) == 2
+    # tiled layout: unknown layout / rule
+    assert lib.trace_capture_ex(a, 4, 32, 1, None, a, a, a, a, a, 256, 7, None) == 2
+    assert lib.trace_fq_fwd_ex(5, a, 4, 32, 1, None, a, a, a, a, a, a, 0, None) == 2
+    assert lib.trace_mx_capture_ex(a, 4, 32, a, a, a, 2, None) == 2
+    assert lib.trace_mx8_fq_fwd_ex(0, a, 4, 32, a, a, a, a, a, 3, None) == 2
+    # histograms
+    assert lib.trace_mismatch_histogram(a, 4, 32, 1, None, a, a, a, None, None) == 1
+    assert lib.trace_mismatch_histogram(a, 4, 32, 1, None, a, a, a, P((1 << 20) + 4), None) == 3
+    assert lib.trace_mx_mismatch_histogram(a, 4, 32, a, a, None, None) == 1
+    assert lib.trace_mx_mismatch_histogram(a, 4, 40, a, a, a, None) == 2
+    # capture's two passes
+    assert lib.trace_capture_amax(a, 4, 48, 1, None, a, None) == 2
+    assert lib.trace_capture_amax(a, 4, 32, 1, None, None, None) == 1
+    assert lib.trace_capture_amax_accumulate(a, 4, 32, 1, None, odd, None) == 3
+    assert lib.trace_capture_with_amax(a, 4, 32, 1, None, a, a, a, a, a, 9, None) == 2
+    assert lib.trace_capture_with_amax(a, 4, 32, 1, None, None, a, a, a, a, 0, None) == 1
+    # no-workspace capture: too many groups
+    assert lib.trace_capture_static_ws(a, 4, 32, 4097, a, a, a, a, a, None) == 4
+    # self-test range: must stay below +inf
+    assert lib.trace_selftest_e4m3_sweep(0x7F800000, 1, a, None) == 2
+    assert lib.trace_selftest_e4m3_sweep(0, 0, None, None) == 0
