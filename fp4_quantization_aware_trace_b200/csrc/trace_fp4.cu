@@ -1,7 +1,10 @@
 // trace_fp4.cu -- B200 (sm_100a) kernels and C ABI for TRACE rollout-guided
 // NVFP4 rounding: rollout capture of the compact cache, the guided QAT
 // fake-quant forward, the masked straight-through backward and the
-// round-to-nearest comparator.
+// round-to-nearest comparator; with them the full-information guided
+// forward, the MXFP4 (W4A4) and W4A8 variants, the 128 x 4 tiled scale
+// layout, capture's two passes for sharded or streamed tensors, and the
+// mismatch-distance histogram.
 //
 // Method: rcap.io post "TRACE: Rollout-Guided Quantization-Aware Training for
 // FP4" (2026-10-06), sections "rollout-guided rounding" and "compact cache"
