@@ -604,6 +604,17 @@ int trace_selftest_e4m3_sweep(uint32_t first_bits, uint32_t count, uint8_t* out,
   return cudaGetLastError() == cudaSuccess ? TRACE_OK : TRACE_ERR_CUDA;
 }
 
+int trace_validate_offsets(const int64_t* group_row_offsets, int32_t num_groups, int64_t rows,
+                           uint32_t* flag, void* stream) {
+  if (num_groups < 1 || rows < 0) return TRACE_ERR_SHAPE;
+  if (!group_row_offsets || !flag) return TRACE_ERR_NULL;
+  if (!aligned(group_row_offsets, 8) || !aligned(flag, 4)) return TRACE_ERR_ALIGN;
+  // one CTA: a debugging aid, not a hot path
+  k_validate_offsets<<<1, 1024, 0, (cudaStream_t)stream>>>(group_row_offsets, num_groups, rows,
+                                                          flag);
+  return cudaGetLastError() == cudaSuccess ? TRACE_OK : TRACE_ERR_CUDA;
+}
+
 int trace_fq_bwd(const uint16_t* grad_out, const uint32_t* ste_mask, int64_t numel,
                  uint16_t* grad_in, void* stream) {
   if (numel < 0 || numel % 32 != 0) return TRACE_ERR_SHAPE;

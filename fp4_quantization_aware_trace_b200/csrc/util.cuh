@@ -33,3 +33,23 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
 }
+
+// Group-offset check, one CTA: flag = 0 when offsets[0] == 0,
+// offsets[G] == rows and offsets never decrease; else 1 + the index of the
+// first offending entry.
+__global__ void __launch_bounds__(1024) k_validate_offsets(const int64_t* __restrict__ offs,
+                                                           int32_t G, int64_t rows,
+                                                           uint32_t* __restrict__ flag) {
+  __shared__ uint32_t first_bad;
+  if (threadIdx.x == 0) first_bad = 0xFFFFFFFFu;
+  __syncthreads();
+  uint32_t bad = 0xFFFFFFFFu;
+  for (int64_t i = threadIdx.x; i <= G; i += blockDim.x) {
+    const int64_t v = offs[i];
+    const bool ok = (i == 0 ? v == 0 : v >= offs[i - 1]) && (i < G || v == rows) && v <= rows;
+    if (!ok && (uint32_t)i < bad) bad = (uint32_t)i;
+  }
+  if (bad != 0xFFFFFFFFu) atomicMin(&first_bad, bad);
+  __syncthreads();
+  if (threadIdx.x == 0) *flag = first_bad == 0xFFFFFFFFu ? 0u : first_bad + 1u;
+}

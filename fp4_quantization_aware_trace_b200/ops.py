@@ -99,6 +99,8 @@ def library() -> ctypes.CDLL:
         lib.trace_mx8_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_mx8_rtn_fq_fwd.argtypes = [P, i64, i64, P, P, P, P]
         lib.trace_mx8_rtn_fq_fwd.restype = ctypes.c_int
+        lib.trace_validate_offsets.argtypes = [P, i32, i64, P, P]
+        lib.trace_validate_offsets.restype = ctypes.c_int
         lib.trace_selftest_e4m3_sweep.argtypes = [ctypes.c_uint32, ctypes.c_uint32, P, P]
         lib.trace_selftest_e4m3_sweep.restype = ctypes.c_int
         lib.trace_mx8_capture_ex.argtypes = [P, i64, i64, P, P, P, i32, P]
@@ -135,11 +137,27 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
 
-def _groups(offsets: torch.Tensor | None) -> int:
+DEBUG = os.environ.get("TRACE_DEBUG", "0") not in ("", "0")
+
+
+def validate_offsets(offsets: torch.Tensor, rows: int, stream=None) -> int:
+    """0 when the device offsets are valid for `rows` rows, else 1 + the
+    first offending index (synchronises the stream)."""
+    flag = torch.empty(1, dtype=torch.int32, device=offsets.device)
+    _check(library().trace_validate_offsets(_p(offsets), int(offsets.numel()) - 1, rows, _p(flag),
+                                            _stream(stream)), "trace_validate_offsets")
+    return int(flag.item())
+
+
+def _groups(offsets: torch.Tensor | None, rows: int | None = None) -> int:
     if offsets is None:
         return 1
     if offsets.dtype != torch.int64:
         raise TraceError("group offsets must be int64")
+    if DEBUG and rows is not None:   # TRACE_DEBUG=1: check the device offsets first
+        bad = validate_offsets(offsets, rows)
+        if bad:
+            raise TraceError(f"group offsets invalid at entry {bad - 1}")
     return int(offsets.numel()) - 1
 
 
@@ -268,7 +286,7 @@ def capture(x: torch.Tensor, offsets: torch.Tensor | None = None, out: Capture |
             workspace: torch.Tensor | None = None, stream=None) -> Capture:
     """Rollout capture of one site (x bf16 [rows, cols]; offsets int64 [G+1])."""
     rows, cols = _bf16_2d(x)
-    G = _groups(offsets)
+    G = _groups(offsets, rows)
     if out is None or workspace is None:
         out, workspace = alloc_capture(rows, cols, G, x.device, offsets)
     trace_capture(x, rows, cols, G, offsets, out.codes, out.mbits, out.scales, out.gscale,

@@ -381,6 +381,15 @@ int trace_rtn_fq_fwd(const uint16_t* x, int64_t rows, int64_t cols,
 int trace_selftest_e4m3_sweep(uint32_t first_bits, uint32_t count, uint8_t* out,
                               void* stream);
 
+/* Check a group-offset array on the device (the calls above take its
+ * contents as a precondition they cannot check on the host): writes to
+ * *flag (device uint32, 4-byte aligned) 0 when offsets[0] == 0,
+ * offsets[G] == rows and the entries never decrease, else 1 + the index of
+ * the first offending entry.  offsets: int64[G+1], 8-byte aligned.  Read the
+ * flag after the stream reaches it. */
+int trace_validate_offsets(const int64_t* group_row_offsets, int32_t num_groups,
+                           int64_t rows, uint32_t* flag, void* stream);
+
 /* Plain bf16 copy (dst = src) with the same load/store path as the kernels
  * above: the measured-bandwidth yardstick for the roofline.  Not part of the
  * method.  32-byte aligned, numel % 16 == 0, no overlap. */

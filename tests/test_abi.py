@@ -152,3 +152,11 @@ def test_host_argument_checks_newer_calls(lib):
     # self-test range: must stay below +inf
     assert lib.trace_selftest_e4m3_sweep(0x7F800000, 1, a, None) == 2
     assert lib.trace_selftest_e4m3_sweep(0, 0, None, None) == 0
+
+
+def test_validate_offsets_argument_checks(lib):
+    P = ctypes.c_void_p
+    a = P(1 << 20)
+    assert lib.trace_validate_offsets(a, 0, 4, a, None) == 2
+    assert lib.trace_validate_offsets(None, 2, 4, a, None) == 1
+    assert lib.trace_validate_offsets(P((1 << 20) + 4), 2, 4, a, None) == 3

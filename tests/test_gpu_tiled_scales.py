@@ -241,3 +241,26 @@ def test_w4a8_tiled(oracle_mod, rows, cols):
     for r in RULES:
         _eq(f"w4a8 out rule {r}", _u(got[r][0]), outs[r][0])
         _eq(f"w4a8 mask rule {r}", _u(got[r][1]), outs[r][1])
+
+
+def test_validate_offsets():
+    ok = torch.tensor([0, 0, 5, 5, 9], dtype=torch.int64, device=DEV)
+    assert ops.validate_offsets(ok, 9) == 0
+    assert ops.validate_offsets(torch.tensor([1, 5, 9], dtype=torch.int64, device=DEV), 9) == 1
+    assert ops.validate_offsets(torch.tensor([0, 6, 5, 9], dtype=torch.int64, device=DEV), 9) == 3
+    assert ops.validate_offsets(torch.tensor([0, 5, 8], dtype=torch.int64, device=DEV), 9) == 3
+    assert ops.validate_offsets(torch.tensor([0, 12, 9], dtype=torch.int64, device=DEV), 9) == 2
+    big = torch.arange(0, 100001, dtype=torch.int64, device=DEV)
+    assert ops.validate_offsets(big, 100000) == 0
+    big[77777] = big[77776] - 1
+    assert ops.validate_offsets(big, 100000) == 77778
+
+
+def test_debug_mode_rejects_bad_offsets(monkeypatch):
+    monkeypatch.setattr(ops, "DEBUG", True)
+    x = torch.zeros(9, 32, dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(ops.TraceError):
+        ops.capture(x, torch.tensor([0, 6, 5, 9], dtype=torch.int64, device=DEV))
+    cap = ops.capture(x, torch.tensor([0, 5, 9], dtype=torch.int64, device=DEV))
+    torch.cuda.synchronize()
+    assert cap.gscale.cpu().tolist() == [1.0, 1.0]
