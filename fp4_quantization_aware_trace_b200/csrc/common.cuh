@@ -145,6 +145,22 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   return r;
 }
 
+// Eight fp32 (four pairs lo, hi) -> one word of eight E2M1 codes (round to
+// nearest even, satfinite), element j in bits 4j..4j+3.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3, float a4,
+                                               float a5, float a6, float a7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+  return r;
+}
+
 // Byte of two E2M1 codes -> f16x2 (exact): lo code in the low half.
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   uint32_t r;
@@ -189,12 +205,18 @@ __device__ __forceinline__ uint32_t absmax_block(const V8& v) {
   return max(m & 0xFFFFu, m >> 16);
 }
 
-// Bit j of the result = bit 4j of n (the lowest bit of each nibble).
-__device__ __forceinline__ uint32_t nibble_lsbs(uint32_t n) {
-  uint32_t c = n & 0x11111111u;
-  c = (c | (c >> 3)) & 0x03030303u;
-  c = (c | (c >> 6)) & 0x000F000Fu;
-  return (c | (c >> 12)) & 0xFFu;
+// Mantissa bits of 32 codes: bit 8k + j of the result = bit 4j of word k
+// (the lowest bit of each nibble).  Per word, the two lowest bits of each
+// byte's nibbles are gathered to bits 8b, 8b + 1 and one multiply moves the
+// field of byte b to bits 24 + 2b; the other partial products fall below
+// bit 24 at distinct even positions (no carries) or above bit 31.
+__device__ __forceinline__ uint32_t nibble_lsbs4(uint4 c) {
+  const uint32_t kGather = (1u << 24) | (1u << 18) | (1u << 12) | (1u << 6);
+  const uint32_t tx = ((c.x & 0x01010101u) | ((c.x >> 3) & 0x02020202u)) * kGather;
+  const uint32_t ty = ((c.y & 0x01010101u) | ((c.y >> 3) & 0x02020202u)) * kGather;
+  const uint32_t tz = ((c.z & 0x01010101u) | ((c.z >> 3) & 0x02020202u)) * kGather;
+  const uint32_t tw = ((c.w & 0x01010101u) | ((c.w >> 3) & 0x02020202u)) * kGather;
+  return __byte_perm(__byte_perm(tx, ty, 0x0073u), __byte_perm(tz, tw, 0x0073u), 0x5410u);
 }
 
 // Per-block constants of the fast path.

@@ -26,18 +26,16 @@ __device__ __forceinline__ int mx_exp(uint32_t amax) {
 
 // Codes of one 16-element block: c0 elements 0-7, c1 elements 8-15.
 __device__ __forceinline__ void mx_codes_block(const V8& v, u64 inv2, uint32_t& c0, uint32_t& c1) {
-  uint32_t c[2] = {0u, 0u};
+  // |z| < 8 from the block's own maximum; the conversion saturates past 6
+  // and keeps the sign of x, also on zeros
+  float z[16];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint32_t w = v.w[k];
-    float zl, zh;
-    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
-    // |z| < 8 from the block's own maximum; the conversion saturates past 6
-    // and keeps the sign of x, also on zeros
-    c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), z[2 * k], z[2 * k + 1]);
   }
-  c0 = c[0];
-  c1 = c[1];
+  c0 = cvt_e2m1x8(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7]);
+  c1 = cvt_e2m1x8(z[8], z[9], z[10], z[11], z[12], z[13], z[14], z[15]);
 }
 
 template <bool SW>
@@ -56,8 +54,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     mx_codes_block(v0, inv2, c.x, c.y);
     mx_codes_block(v1, inv2, c.z, c.w);
     codes[b >> 1] = c;
-    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
-                    (nibble_lsbs(c.w) << 24);
+    mbits[b >> 1] = nibble_lsbs4(c);
     if (SW) {
       const uint32_t row = fastdiv(b, sh.bpr);
       scales[tiled_scale_offset(row, (b - row * sh.bpr.d) >> 1, sh.sw_ct)] = (uint8_t)(e + 127);

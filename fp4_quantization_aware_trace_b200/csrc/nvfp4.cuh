@@ -210,21 +210,24 @@ __device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk,
       if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
     }
   } else if (fast_scale(d)) {
-    const BlkK bk = make_blk(d, 0.0f, 0.0f);
-    uint32_t c[2] = {0u, 0u};
+    // The quotient runs negated: with q0' = RN(x * -r), e = x + q0' d (exact)
+    // and z' = RN(q0' + e * -r), z' = -RN(x / d) by the symmetry of
+    // round-to-nearest, and a zero quotient keeps the opposite of x's sign
+    // (x = +-0 and underflows alike), which the unnegated step loses for
+    // x = -0.  The codes of z' with every sign bit flipped are the codes of
+    // RN(x / d) with x's sign (cvt ... satfinite is odd in its input).
+    const float r = __frcp_rn(d);
+    const u64 nrr = pk(-r, -r), dd = pk(d, d);
+    float z[16];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const uint32_t w = v.w[k];
-      const float xl = bf16_lo(w), xh = bf16_hi(w);
-      float zl, zh;
-      upk(quot2(pk(xl, xh), bk), zl, zh);
-      // the code carries the sign of x (also for zeros and underflows)
-      zl = __uint_as_float((__float_as_uint(zl) & 0x7FFFFFFFu) | (__float_as_uint(xl) & 0x80000000u));
-      zh = __uint_as_float((__float_as_uint(zh) & 0x7FFFFFFFu) | (w & 0x80000000u));
-      c[k >> 2] |= cvt_e2m1x2(zl, zh) << (8 * (k & 3));
+      const u64 xx = pk(bf16_lo(w), bf16_hi(w));
+      const u64 q0 = mul2(xx, nrr);
+      upk(fma2(fma2(q0, dd, xx), nrr, q0), z[2 * k], z[2 * k + 1]);
     }
-    c0 = c[0];
-    c1 = c[1];
+    c0 = cvt_e2m1x8(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7]) ^ 0x88888888u;
+    c1 = cvt_e2m1x8(z[8], z[9], z[10], z[11], z[12], z[13], z[14], z[15]) ^ 0x88888888u;
   } else {
     capture_block_exact(v, d, &c0, &c1);
   }
@@ -263,8 +266,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const uint32_t s0 = capture_block(v0, gk, c.x, c.y);
     const uint32_t s1 = capture_block(v1, gk, c.z, c.w);
     codes[b >> 1] = c;
-    mbits[b >> 1] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) | (nibble_lsbs(c.z) << 16) |
-                    (nibble_lsbs(c.w) << 24);
+    mbits[b >> 1] = nibble_lsbs4(c);
     const uint16_t sv = (uint16_t)(s0 | (s1 << 8));
     if (SW)  // the pair's two columns are neighbours inside one tile
       *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;

@@ -3,7 +3,9 @@ use in place of a per-element division and a codeword table (restated in
 plain C in kernel_math_check.c):
 
   * the FMA-corrected reciprocal quotient equals IEEE x/d for every bf16
-    numerator and fp32 denominator significand (both result binades);
+    numerator and fp32 denominator significand (both result binades), and
+    run negated it equals -(x/d) there and keeps the sign opposite to x's
+    for every finite bf16 x (zeros included) across the denominators' range;
   * rounding a + M down / up (M a power-of-two magic addend per binade)
     gives the E2M1 floor / ceiling of every fp32 a in [0, 6] and the
     mantissa bit of the floor codeword.
@@ -36,6 +38,7 @@ def test_quotient_and_grid_identities_hold_exhaustively(tmp_path):
     r = subprocess.run([_build(tmp_path)], capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "quotient: 0 mismatches" in r.stdout and "grid rounding: 0 mismatches" in r.stdout
+    assert "negated quotient: 0 mismatches of 2147483648 cases, 0 in the sign" in r.stdout
 
 
 def test_negative_control_fails(tmp_path):
@@ -44,3 +47,12 @@ def test_negative_control_fails(tmp_path):
     assert r.returncode == 1
     assert "quotient: 0 mismatches" not in r.stdout
     assert "grid rounding: 0 mismatches" not in r.stdout
+
+
+def test_sign_control_fails(tmp_path):
+    """Negating the unnegated step's result loses the sign of x = -0 (its
+    z is +0): the sign sweep must see it."""
+    r = subprocess.run([_build(tmp_path, "SIGN_CONTROL")], capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 1
+    assert ", 0 in the sign" not in r.stdout
