@@ -133,20 +133,9 @@ __device__ __forceinline__ u64 sub2(u64 a, u64 b) {
 // Number-format helpers (hardware conversions from the public PTX ISA)
 // ---------------------------------------------------------------------------
 
-// Two fp32 -> one byte of two E2M1 codes (round to nearest even, satfinite):
-// lo in bits 0-3, hi in bits 4-7; the sign of each input is kept.
-__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
-  uint16_t r;
-  asm("{\n\t.reg .b8 b;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
-      "cvt.u16.u8 %0, b;\n\t}"
-      : "=h"(r)
-      : "f"(hi), "f"(lo));
-  return r;
-}
-
 // Eight fp32 (four pairs lo, hi) -> one word of eight E2M1 codes (round to
-// nearest even, satfinite), element j in bits 4j..4j+3.
+// nearest even, satfinite; the sign of each input is kept), element j in
+// bits 4j..4j+3.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3, float a4,
                                                float a5, float a6, float a7) {
   uint32_t r;
@@ -158,6 +147,24 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, flo
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(r)
       : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+  return r;
+}
+
+// Eight fp32 from an array (element j in bits 4j..4j+3), as above.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float* a) {
+  return cvt_e2m1x8(a[0], a[1], a[2], a[3], a[4], a[5], a[6], a[7]);
+}
+
+// Two fp32 -> their round-to-nearest E2M1 codeword values (ties to the even
+// code, satfinite) as f16x2, lo in the low half: the encode and the exact
+// decode with the code byte kept in an 8-bit register between them.
+__device__ __forceinline__ uint32_t rtn_e2m1x2_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %1, %2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
   return r;
 }
 

@@ -30,8 +30,7 @@ struct BlockCodes {
 // floor and ceiling by directed rounding on the grid, each scaled back and
 // converted exactly to its code; round to nearest through the hardware
 // conversion (ties to the even code) of min(|z|, 6) with the sign of x.
-__device__ __forceinline__ void codes_pair(uint32_t w, const BlkK& k, uint32_t& fb, uint32_t& cb,
-                                           uint32_t& rb) {
+__device__ __forceinline__ void codes_pair(uint32_t w, const BlkK& k, float* f, float* c, float* r) {
   const uint32_t wa = w & 0x7FFF7FFFu;
   const u64 xx = pk(__uint_as_float(wa << 16), __uint_as_float(wa & 0xFFFF0000u));
   float zl, zh;
@@ -40,15 +39,12 @@ __device__ __forceinline__ void codes_pair(uint32_t w, const BlkK& k, uint32_t& 
   const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
   const u64 aa = pk(al, ah);
   const u64 un = pk(0x1p-64f, 0x1p-64f);
-  float fl, fh, cl, ch, rl, rh;
-  upk(mul2(sub2(add_rm2(aa, MM), MM), un), fl, fh);
-  upk(mul2(sub2(add_rp2(aa, MM), MM), un), cl, ch);
+  float rl, rh;
+  upk(mul2(sub2(add_rm2(aa, MM), MM), un), f[0], f[1]);
+  upk(mul2(sub2(add_rp2(aa, MM), MM), un), c[0], c[1]);
   upk(mul2(aa, un), rl, rh);
-  rl = __uint_as_float(__float_as_uint(rl) | ((w << 16) & 0x80000000u));
-  rh = __uint_as_float(__float_as_uint(rh) | (w & 0x80000000u));
-  fb = cvt_e2m1x2(fl, fh);
-  cb = cvt_e2m1x2(cl, ch);
-  rb = cvt_e2m1x2(rl, rh);
+  r[0] = __uint_as_float(__float_as_uint(rl) | ((w << 16) & 0x80000000u));
+  r[1] = __uint_as_float(__float_as_uint(rh) | (w & 0x80000000u));
 }
 
 // The same codes on the exact path (d outside the fast range).
@@ -87,12 +83,12 @@ __device__ __forceinline__ BlockCodes block_codes(const V8& v, float sbv, float 
     const BlkK bk = make_blk(d, 0.0f, 0.0f);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      uint32_t fb[4], cb[4], rb[4];
+      float f[8], c[8], r[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) codes_pair(v.w[4 * h + k], bk, fb[k], cb[k], rb[k]);
-      bc.f[h] = fb[0] | (fb[1] << 8) | (fb[2] << 16) | (fb[3] << 24);
-      bc.c[h] = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
-      bc.r[h] = rb[0] | (rb[1] << 8) | (rb[2] << 16) | (rb[3] << 24);
+      for (int k = 0; k < 4; ++k) codes_pair(v.w[4 * h + k], bk, f + 2 * k, c + 2 * k, r + 2 * k);
+      bc.f[h] = cvt_e2m1x8(f);
+      bc.c[h] = cvt_e2m1x8(c);
+      bc.r[h] = cvt_e2m1x8(r);
     }
   } else {
     codes_block_exact(v, d, &bc);
@@ -106,7 +102,7 @@ __device__ __forceinline__ BlockCodes mx_block_codes(const V8& v, u64 inv2) {
   BlockCodes bc;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    uint32_t fb[4], cb[4], rb[4];
+    float f[8], c[8], r[8];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const uint32_t w = v.w[4 * h + k];
@@ -116,18 +112,14 @@ __device__ __forceinline__ BlockCodes mx_block_codes(const V8& v, u64 inv2) {
       const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);
       const u64 MM = pk(grid_magic(al), grid_magic(ah));
       const u64 aa = pk(al, ah);
-      float fl, fh, cl, ch;
-      upk(sub2(add_rm2(aa, MM), MM), fl, fh);
-      upk(sub2(add_rp2(aa, MM), MM), cl, ch);
-      const float rl = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
-      const float rh = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
-      fb[k] = cvt_e2m1x2(fl, fh);
-      cb[k] = cvt_e2m1x2(cl, ch);
-      rb[k] = cvt_e2m1x2(rl, rh);
+      upk(sub2(add_rm2(aa, MM), MM), f[2 * k], f[2 * k + 1]);
+      upk(sub2(add_rp2(aa, MM), MM), c[2 * k], c[2 * k + 1]);
+      r[2 * k] = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
+      r[2 * k + 1] = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
     }
-    bc.f[h] = fb[0] | (fb[1] << 8) | (fb[2] << 16) | (fb[3] << 24);
-    bc.c[h] = cb[0] | (cb[1] << 8) | (cb[2] << 16) | (cb[3] << 24);
-    bc.r[h] = rb[0] | (rb[1] << 8) | (rb[2] << 16) | (rb[3] << 24);
+    bc.f[h] = cvt_e2m1x8(f);
+    bc.c[h] = cvt_e2m1x8(c);
+    bc.r[h] = cvt_e2m1x8(r);
   }
   return bc;
 }

@@ -74,7 +74,7 @@ __device__ __forceinline__ uint32_t mx_fq_pair(uint32_t w, uint32_t side, u64 in
   const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
   float tl, th;  // chosen codeword value
   if (MODE == kRtn) {
-    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
+    const uint32_t h2 = rtn_e2m1x2_f16x2(al, ah);
     tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
     th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
   } else {

@@ -336,7 +336,7 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const Blk
     m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
     const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
     // round to nearest on the grid (ties to the even code), then dequantise
-    const uint32_t h2 = e2m1x2_to_f16x2(cvt_e2m1x2(al, ah));
+    const uint32_t h2 = rtn_e2m1x2_f16x2(al, ah);
     const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
     const float vh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
     upk(mul2(mul2(pk(vl, vh), k.sbv2), k.sg2), ql, qh);
