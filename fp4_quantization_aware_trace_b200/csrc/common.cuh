@@ -78,6 +78,18 @@ __device__ __forceinline__ V8 ld_block_stream(const void* p) {
   return v;
 }
 
+// The same block through two 16-byte read-only loads, for the rarely taken
+// out-of-line (exact-path) functions: ptxas 12.9 crashed on the 32-byte load
+// form inside a non-inlined function.
+__device__ __forceinline__ V8 ld_block_ro(const V8* p) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  V8 v;
+  v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
+  v.w[4] = b.x; v.w[5] = b.y; v.w[6] = b.z; v.w[7] = b.w;
+  return v;
+}
+
 __device__ __forceinline__ void st_block(void* p, const V8& v) {
   asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
                "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
@@ -192,6 +204,15 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
   uint16_t in = (uint16_t)b;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+
+// Two E4M3 bytes (b0 | b1 << 8) -> fp32 (exact, through f16x2).
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t b2, float& lo, float& hi) {
+  uint32_t h2;
+  uint16_t in = (uint16_t)b2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
+  lo = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+  hi = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
 }
 
 // Two fp32 -> bf16x2 (round to nearest even): lo in the low half.

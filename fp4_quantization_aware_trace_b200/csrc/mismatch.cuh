@@ -48,7 +48,8 @@ __device__ __forceinline__ void codes_pair(uint32_t w, const BlkK& k, float* f, 
 }
 
 // The same codes on the exact path (d outside the fast range).
-__device__ __noinline__ void codes_block_exact(V8 v, float d, BlockCodes* bc) {
+__device__ __noinline__ BlockCodes codes_block_exact(const V8* src, float d) {
+  const V8 v = ld_block_ro(src);
   uint32_t f[2] = {0u, 0u}, c[2] = {0u, 0u}, r[2] = {0u, 0u};
   for (int j = 0; j < 16; ++j) {
     const uint32_t w = v.w[j >> 1];
@@ -60,14 +61,16 @@ __device__ __noinline__ void codes_block_exact(V8 v, float d, BlockCodes* bc) {
     c[j >> 3] |= (uint32_t)(e.exact ? e.floor : e.floor + 1) << sh;
     r[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << sh;
   }
+  BlockCodes bc;
   for (int h = 0; h < 2; ++h) {
-    bc->f[h] = f[h];
-    bc->c[h] = c[h];
-    bc->r[h] = r[h];
+    bc.f[h] = f[h];
+    bc.c[h] = c[h];
+    bc.r[h] = r[h];
   }
+  return bc;
 }
 
-__device__ __forceinline__ BlockCodes block_codes(const V8& v, float sbv, float s_g) {
+__device__ __forceinline__ BlockCodes block_codes(const V8& v, const V8* src, float sbv, float s_g) {
   BlockCodes bc;
   const float d = __fmul_rn(s_g, sbv);
   if (d == 0.0f) {
@@ -91,7 +94,7 @@ __device__ __forceinline__ BlockCodes block_codes(const V8& v, float sbv, float 
       bc.r[h] = cvt_e2m1x8(r);
     }
   } else {
-    codes_block_exact(v, d, &bc);
+    bc = codes_block_exact(src, d);
   }
   return bc;
 }
@@ -198,8 +201,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     } else {
       const uint32_t sb2 = __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
       if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
-      k0 = block_codes(v0, e4m3_to_f32(sb2 & 0xFFu), s_g);
-      k1 = block_codes(v1, e4m3_to_f32(sb2 >> 8), s_g);
+      k0 = block_codes(v0, x + b, e4m3_to_f32(sb2 & 0xFFu), s_g);
+      k1 = block_codes(v1, x + b + 1, e4m3_to_f32(sb2 >> 8), s_g);
     }
     hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
     hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);

@@ -37,8 +37,13 @@ __device__ __forceinline__ float e2m1_value(int c) {
 }
 
 // Capture of one block on the exact path: 16 codes (sign<<3 | rtn).
-__device__ __noinline__ void capture_block_exact(V8 v, float d, uint32_t* code_lo,
-                                                 uint32_t* code_hi) {
+// The out-of-line exact-path functions read their block back from global
+// memory and return their results by value (or store them themselves):
+// passing the block's registers in or taking the address of the caller's
+// outputs put those locals in local memory on every path, the fast one
+// included.
+__device__ __noinline__ uint2 capture_block_exact(const V8* src, float d) {
+  const V8 v = ld_block_ro(src);
   uint32_t c[2] = {0u, 0u};
   for (int j = 0; j < 16; ++j) {
     const uint32_t w = v.w[j >> 1];
@@ -47,18 +52,19 @@ __device__ __noinline__ void capture_block_exact(V8 v, float d, uint32_t* code_l
     const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
     c[j >> 3] |= ((sg << 3) | (uint32_t)e.rtn) << (4 * (j & 7));
   }
-  *code_lo = c[0];
-  *code_hi = c[1];
+  return make_uint2(c[0], c[1]);
 }
 
 // Fake-quant of one block on the exact path: bf16 outputs and STE mask.
 // mode: 0 round-to-nearest, 1 1-bit guided (bits16), 2 full-information
 // guided (rollout codes c0: elements 0-7, c1: 8-15).
-__device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, float s_g,
+__device__ __noinline__ uint32_t fake_quant_block_exact(const V8* src, float d, float sbv, float s_g,
                                                     uint32_t bits16, uint32_t c0, uint32_t c1,
-                                                    int mode, V8* out, uint32_t* mask16) {
+                                                    int mode, V8* dst) {
+  const V8 v = ld_block_ro(src);
   uint32_t m = 0u;
-  for (int k = 0; k < 8; ++k) out->w[k] = 0u;
+  V8 o;
+  for (int k = 0; k < 8; ++k) o.w[k] = 0u;
   for (int j = 0; j < 16; ++j) {
     const uint32_t w = v.w[j >> 1];
     const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
@@ -79,10 +85,11 @@ __device__ __noinline__ void fake_quant_block_exact(V8 v, float d, float sbv, fl
     const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
         __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
     const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
-    out->w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
+    o.w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
     m |= (uint32_t)e.in << j;
   }
-  *mask16 = m;
+  st_block(dst, o);
+  return m;
 }
 
 // ---------------------------------------------------------------------------
@@ -185,21 +192,49 @@ __device__ __forceinline__ GroupK group_consts(uint32_t amax_bits) {
 // Kernel 2: capture.  Per 16-element block: E4M3 scale; per element: the
 // round-to-nearest code and its mantissa bit.
 // ---------------------------------------------------------------------------
-// One block: returns its E4M3 scale byte, writes its 16 codes to c0 (elements
-// 0-7) and c1 (8-15).
-__device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk, uint32_t& c0,
-                                                  uint32_t& c1) {
-  // block scale: t = bmax / RN(6 s_g), E4M3 round-to-nearest-even, satfinite
-  const float bmax = __uint_as_float(absmax_block(v) << 16);
-  float tq;
+// Scale bytes of a pair of blocks: t = bmax / RN(6 s_g), E4M3
+// round-to-nearest-even, satfinite.  Returns s0 | s1 << 8.
+__device__ __forceinline__ uint32_t pair_scale_bytes(const V8& v0, const V8& v1, const GroupK& gk) {
+  const float b0 = __uint_as_float(absmax_block(v0) << 16);
+  const float b1 = __uint_as_float(absmax_block(v1) << 16);
+  float t0, t1;
   if (gk.fast6) {
-    const float q0 = __fmul_rn(bmax, gk.r6);
-    tq = __fmaf_rn(__fmaf_rn(q0, -gk.den6, bmax), gk.r6, q0);
+    const u64 bb = pk(b0, b1), rr = pk(gk.r6, gk.r6);
+    const u64 q0 = mul2(bb, rr);
+    upk(fma2(fma2(q0, pk(-gk.den6, -gk.den6), bb), rr, q0), t0, t1);
   } else {
-    tq = __fdiv_rn(bmax, gk.den6);
+    t0 = __fdiv_rn(b0, gk.den6);
+    t1 = __fdiv_rn(b1, gk.den6);
   }
-  const uint32_t sb = cvt_e4m3(tq);
-  const float d = __fmul_rn(gk.s_g, e4m3_to_f32(sb));
+  return cvt_e4m3(t0) | (cvt_e4m3(t1) << 8);
+}
+
+// Codes of one block whose scale d is on the fast path: c0 elements 0-7,
+// c1 8-15.
+// The quotient runs negated: with q0' = RN(x * -r), e = x + q0' d (exact)
+// and z' = RN(q0' + e * -r), z' = -RN(x / d) by the symmetry of
+// round-to-nearest, and a zero quotient keeps the opposite of x's sign
+// (x = +-0 and underflows alike), which the unnegated step loses for
+// x = -0.  The codes of z' with every sign bit flipped are the codes of
+// RN(x / d) with x's sign (cvt ... satfinite is odd in its input).
+__device__ __forceinline__ void codes_fast(const V8& v, float d, uint32_t& c0, uint32_t& c1) {
+  const float r = __frcp_rn(d);
+  const u64 nrr = pk(-r, -r), dd = pk(d, d);
+  float z[16];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t w = v.w[k];
+    const u64 xx = pk(bf16_lo(w), bf16_hi(w));
+    const u64 q0 = mul2(xx, nrr);
+    upk(fma2(fma2(q0, dd, xx), nrr, q0), z[2 * k], z[2 * k + 1]);
+  }
+  c0 = cvt_e2m1x8(z) ^ 0x88888888u;
+  c1 = cvt_e2m1x8(z + 8) ^ 0x88888888u;
+}
+
+// Codes of one block with any scale d: zero block, fast path or exact path.
+__device__ __forceinline__ void codes_block(const V8& v, const V8* src, float d, uint32_t& c0,
+                                            uint32_t& c1) {
   if (d == 0.0f) {
     // zero block: z = +-0, code = sign only
     c0 = c1 = 0u;
@@ -210,28 +245,12 @@ __device__ __forceinline__ uint32_t capture_block(const V8& v, const GroupK& gk,
       if (k < 4) c0 |= nib << (8 * k); else c1 |= nib << (8 * (k - 4));
     }
   } else if (fast_scale(d)) {
-    // The quotient runs negated: with q0' = RN(x * -r), e = x + q0' d (exact)
-    // and z' = RN(q0' + e * -r), z' = -RN(x / d) by the symmetry of
-    // round-to-nearest, and a zero quotient keeps the opposite of x's sign
-    // (x = +-0 and underflows alike), which the unnegated step loses for
-    // x = -0.  The codes of z' with every sign bit flipped are the codes of
-    // RN(x / d) with x's sign (cvt ... satfinite is odd in its input).
-    const float r = __frcp_rn(d);
-    const u64 nrr = pk(-r, -r), dd = pk(d, d);
-    float z[16];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t w = v.w[k];
-      const u64 xx = pk(bf16_lo(w), bf16_hi(w));
-      const u64 q0 = mul2(xx, nrr);
-      upk(fma2(fma2(q0, dd, xx), nrr, q0), z[2 * k], z[2 * k + 1]);
-    }
-    c0 = cvt_e2m1x8(z[0], z[1], z[2], z[3], z[4], z[5], z[6], z[7]) ^ 0x88888888u;
-    c1 = cvt_e2m1x8(z[8], z[9], z[10], z[11], z[12], z[13], z[14], z[15]) ^ 0x88888888u;
+    codes_fast(v, d, c0, c1);
   } else {
-    capture_block_exact(v, d, &c0, &c1);
+    const uint2 c = capture_block_exact(src, d);
+    c0 = c.x;
+    c1 = c.y;
   }
-  return sb;
 }
 
 // Each thread owns two adjacent blocks: one 16-byte store of codes, one
@@ -262,12 +281,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     // both blocks of the pair are in the same row (cols is a multiple of 32)
     const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
     if (gc.seek(row)) gk = group_consts(__ldg(amax + gc.g));
+    const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
+    float sb0, sb1;
+    e4m3x2_to_f32(s2, sb0, sb1);
+    const float d0 = __fmul_rn(gk.s_g, sb0), d1 = __fmul_rn(gk.s_g, sb1);
     uint4 c;
-    const uint32_t s0 = capture_block(v0, gk, c.x, c.y);
-    const uint32_t s1 = capture_block(v1, gk, c.z, c.w);
+    if (fast_scale(d0) && fast_scale(d1)) {  // the common case, without per-block branches
+      codes_fast(v0, d0, c.x, c.y);
+      codes_fast(v1, d1, c.z, c.w);
+    } else {
+      codes_block(v0, x + b, d0, c.x, c.y);
+      codes_block(v1, x + b + 1, d1, c.z, c.w);
+    }
     codes[b >> 1] = c;
     mbits[b >> 1] = nibble_lsbs4(c);
-    const uint16_t sv = (uint16_t)(s0 | (s1 << 8));
+    const uint16_t sv = (uint16_t)s2;
     if (SW)  // the pair's two columns are neighbours inside one tile
       *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
     else
@@ -348,27 +376,44 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const Blk
 // bits.  side: kGuided -- the block's 16 cached bits; kFull -- its 16
 // rollout codes (c0: elements 0-7, c1: 8-15).
 template <int MODE>
-__device__ __forceinline__ void fake_quant_block(const V8& v, uint32_t bits16, uint32_t c0,
-                                                 uint32_t c1, float sbv, float s_g, V8& o,
-                                                 uint32_t& m) {
-  const float d = __fmul_rn(s_g, sbv);
+__device__ __forceinline__ void fake_quant_fast(const V8& v, uint32_t bits16, uint32_t c0,
+                                                uint32_t c1, float d, float sbv, float s_g, V8& o,
+                                                uint32_t& m) {
+  const BlkK bk = make_blk(d, MODE != kRtn ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
   m = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t side = MODE == kGuided ? bits16 >> (2 * k)
+                        : MODE == kFull ? ((k < 4 ? c0 : c1) >> (8 * (k & 3))) : 0u;
+    o.w[k] = fq_pair<MODE>(v.w[k], side, bk, m, 2 * k);
+  }
+}
+
+// Upper end of the fast range of the scale d for each mode.
+template <int MODE>
+__host__ __device__ constexpr uint32_t fq_dmax() { return MODE != kRtn ? kDMaxExactZ : kDMax; }
+
+// One block with any scale (zero block, fast path or exact path): stores its
+// output at dst and returns its 16 mask bits.
+template <int MODE>
+__device__ __forceinline__ uint32_t fake_quant_block(const V8& v, const V8* src, uint32_t bits16,
+                                                     uint32_t c0, uint32_t c1, float sbv, float s_g,
+                                                     V8* dst) {
+  const float d = __fmul_rn(s_g, sbv);
+  V8 o;
+  uint32_t m;
   if (d == 0.0f) {
     // zero block: z = +-0, output +-0, mask set
 #pragma unroll
     for (int k = 0; k < 8; ++k) o.w[k] = v.w[k] & 0x80008000u;
     m = 0xFFFFu;
-  } else if (fast_scale(d, MODE != kRtn ? kDMaxExactZ : kDMax)) {
-    const BlkK bk = make_blk(d, MODE != kRtn ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits16 >> (2 * k)
-                          : MODE == kFull ? ((k < 4 ? c0 : c1) >> (8 * (k & 3))) : 0u;
-      o.w[k] = fq_pair<MODE>(v.w[k], side, bk, m, 2 * k);
-    }
+  } else if (fast_scale(d, fq_dmax<MODE>())) {
+    fake_quant_fast<MODE>(v, bits16, c0, c1, d, sbv, s_g, o, m);
   } else {
-    fake_quant_block_exact(v, d, sbv, s_g, bits16, c0, c1, MODE, &o, &m);
+    return fake_quant_block_exact(src, d, sbv, s_g, bits16, c0, c1, MODE, dst);
   }
+  st_block(dst, o);
+  return m;
 }
 
 // Each thread owns two adjacent blocks, so their mantissa bits, scales and
@@ -402,14 +447,23 @@ __global__ void __launch_bounds__(kThreads, MINB)
                  scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
            : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
     if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
-    V8 o;
     uint32_t m0, m1;
-    fake_quant_block<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, e4m3_to_f32(sb2 & 0xFFu), s_g, o, m0);
-    st_block(out + b, o);
+    float sbv0, sbv1;
+    e4m3x2_to_f32(sb2, sbv0, sbv1);
     // a row holds a whole number of 32-element words, so both blocks of the
     // pair are in the same row and group
-    fake_quant_block<MODE>(v1, bits >> 16, rc.z, rc.w, e4m3_to_f32(sb2 >> 8), s_g, o, m1);
-    st_block(out + b + 1, o);
+    const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
+    if (fast_scale(d0, fq_dmax<MODE>()) && fast_scale(d1, fq_dmax<MODE>())) {
+      // the common case, without per-block branches
+      V8 o;
+      fake_quant_fast<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
+      st_block(out + b, o);
+      fake_quant_fast<MODE>(v1, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
+      st_block(out + b + 1, o);
+    } else {
+      m0 = fake_quant_block<MODE>(v0, x + b, bits & 0xFFFFu, rc.x, rc.y, sbv0, s_g, out + b);
+      m1 = fake_quant_block<MODE>(v1, x + b + 1, bits >> 16, rc.z, rc.w, sbv1, s_g, out + b + 1);
+    }
     mask[b >> 1] = m0 | (m1 << 16);
   }
 }

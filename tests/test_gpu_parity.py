@@ -192,6 +192,35 @@ def test_parity_special_values(oracle_mod):
     check_full(oracle_mod, s2)
 
 
+def test_parity_signed_zero_quotients(oracle_mod):
+    """Zeros of both signs, and values whose quotient underflows to zero, in
+    blocks whose scale keeps them on the kernels' fast path (block maxima
+    from 1 to 1e30): every such element's code is the zero with the sign of
+    x, and everything else matches the oracle."""
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((96, 256)).astype(np.float32)
+    x[32:64] *= 1e30                  # d near 2^97: tiny values underflow
+    x[:, 0::4] = np.float32(0.0)
+    x[:, 1::4] = np.float32(-0.0)
+    tiny = np.float32(2.0 ** -133)    # smallest bf16 subnormal
+    x[:, 2::8] = tiny
+    x[:, 6::8] = -tiny
+    x[64:, 3::16] = np.float32(-1e-39)
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    # one group per band of 32 rows, so each band gets its own global scale
+    s = inputs.Site("signed_zeros", xb, (xb.float() * 1.003).to(torch.bfloat16),
+                    torch.from_numpy(rng.standard_normal((96, 256)).astype(np.float32)).to(torch.bfloat16),
+                    torch.tensor([0, 32, 64, 96], dtype=torch.int64))
+    got, _ = check_full(oracle_mod, s)
+    # every block is scaled (no zero-block shortcut)
+    assert np.all(got["scales"] > 0)
+    codes = got["codes"].reshape(-1)
+    nib = np.stack([codes & 0xF, codes >> 4], axis=1).reshape(96, 256)
+    assert np.all(nib[:, 0::4] == 0x0) and np.all(nib[:, 1::4] == 0x8)
+    # the quotient of +-2^-133 by d >= 2^90 underflows: zero code, sign of x
+    assert np.all(nib[32:64, 2::8] == 0x0) and np.all(nib[32:64, 6::8] == 0x8)
+
+
 def test_guided_equals_rollout_rtn_when_same_input(oracle_mod):
     s = inputs.attention_input(seed=4, rows=512)
     s.x_train = s.x_roll.clone()
