@@ -78,9 +78,11 @@ __device__ __forceinline__ V8 ld_block_stream(const void* p) {
   return v;
 }
 
-// The same block through two 16-byte read-only loads, for the rarely taken
-// out-of-line (exact-path) functions: ptxas 12.9 crashed on the 32-byte load
-// form inside a non-inlined function.
+// Block load and store for the rarely taken out-of-line (exact-path)
+// functions, as plain 16-byte accesses: with the 32-byte asm forms inside a
+// non-inlined function, ptxas 12.9 crashed (load) or, depending on the other
+// code in the module, stored wrong data (store; caught by the seeded fuzz
+// parity tests).
 __device__ __forceinline__ V8 ld_block_ro(const V8* p) {
   const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
   const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
@@ -88,6 +90,12 @@ __device__ __forceinline__ V8 ld_block_ro(const V8* p) {
   v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
   v.w[4] = b.x; v.w[5] = b.y; v.w[6] = b.z; v.w[7] = b.w;
   return v;
+}
+
+__device__ __forceinline__ void st_block_plain(V8* p, const V8& v) {
+  uint4* q = reinterpret_cast<uint4*>(p);
+  q[0] = make_uint4(v.w[0], v.w[1], v.w[2], v.w[3]);
+  q[1] = make_uint4(v.w[4], v.w[5], v.w[6], v.w[7]);
 }
 
 __device__ __forceinline__ void st_block(void* p, const V8& v) {
@@ -196,14 +204,6 @@ __device__ __forceinline__ uint32_t cvt_e4m3(float t) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(t));
   return (uint32_t)(r & 0xFFu);
-}
-
-// E4M3 byte -> fp32 (exact, through f16).
-__device__ __forceinline__ float e4m3_to_f32(uint32_t b) {
-  uint32_t h2;
-  uint16_t in = (uint16_t)b;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(in));
-  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }
 
 // Two E4M3 bytes (b0 | b1 << 8) -> fp32 (exact, through f16x2).

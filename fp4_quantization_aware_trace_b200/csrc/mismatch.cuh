@@ -70,9 +70,25 @@ __device__ __noinline__ BlockCodes codes_block_exact(const V8* src, float d) {
   return bc;
 }
 
-__device__ __forceinline__ BlockCodes block_codes(const V8& v, const V8* src, float sbv, float s_g) {
+// Codes of a block whose scale d is on the guided fast path.
+__device__ __forceinline__ BlockCodes block_codes_fast(const V8& v, float d) {
   BlockCodes bc;
-  const float d = __fmul_rn(s_g, sbv);
+  const BlkK bk = make_blk(d, 0.0f, 0.0f);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float f[8], c[8], r[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) codes_pair(v.w[4 * h + k], bk, f + 2 * k, c + 2 * k, r + 2 * k);
+    bc.f[h] = cvt_e2m1x8(f);
+    bc.c[h] = cvt_e2m1x8(c);
+    bc.r[h] = cvt_e2m1x8(r);
+  }
+  return bc;
+}
+
+// Codes of a block with any scale d: zero block, fast path or exact path.
+__device__ __forceinline__ BlockCodes block_codes(const V8& v, const V8* src, float d) {
+  BlockCodes bc;
   if (d == 0.0f) {
     // zero block: z = +-0, every code is zero with the sign of x
     bc.f[0] = bc.f[1] = bc.c[0] = bc.c[1] = 0u;
@@ -83,16 +99,7 @@ __device__ __forceinline__ BlockCodes block_codes(const V8& v, const V8* src, fl
       bc.r[k >> 2] |= ((((w >> 15) & 1u) << 3) | ((w >> 31) << 7)) << (8 * (k & 3));
     }
   } else if (fast_scale(d, kDMaxExactZ)) {
-    const BlkK bk = make_blk(d, 0.0f, 0.0f);
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float f[8], c[8], r[8];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) codes_pair(v.w[4 * h + k], bk, f + 2 * k, c + 2 * k, r + 2 * k);
-      bc.f[h] = cvt_e2m1x8(f);
-      bc.c[h] = cvt_e2m1x8(c);
-      bc.r[h] = cvt_e2m1x8(r);
-    }
+    bc = block_codes_fast(v, d);
   } else {
     bc = codes_block_exact(src, d);
   }
@@ -201,8 +208,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     } else {
       const uint32_t sb2 = __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
       if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
-      k0 = block_codes(v0, x + b, e4m3_to_f32(sb2 & 0xFFu), s_g);
-      k1 = block_codes(v1, x + b + 1, e4m3_to_f32(sb2 >> 8), s_g);
+      float sbv0, sbv1;
+      e4m3x2_to_f32(sb2, sbv0, sbv1);
+      const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
+      if (fast_scale(d0, kDMaxExactZ) && fast_scale(d1, kDMaxExactZ)) {
+        // the common case, without per-block branches
+        k0 = block_codes_fast(v0, d0);
+        k1 = block_codes_fast(v1, d1);
+      } else {
+        k0 = block_codes(v0, x + b, d0);
+        k1 = block_codes(v1, x + b + 1, d1);
+      }
     }
     hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
     hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);

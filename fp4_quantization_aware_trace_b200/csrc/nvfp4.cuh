@@ -88,7 +88,7 @@ __device__ __noinline__ uint32_t fake_quant_block_exact(const V8* src, float d, 
     o.w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
     m |= (uint32_t)e.in << j;
   }
-  st_block(dst, o);
+  st_block_plain(dst, o);
   return m;
 }
 
