@@ -290,6 +290,16 @@ __device__ __forceinline__ float grid_magic_s(float a_s) {
   return __uint_as_float(max((__float_as_uint(a_s) & 0x7F800000u) + 0x0B000000u, 0x6A800000u));
 }
 
+// The same addend for a pair, with the binade scaling as one packed multiply
+// (exact: the masked exponent is a power of two or zero).
+__device__ __forceinline__ u64 grid_magic_s2(float al, float ah) {
+  const u64 e = pk(__uint_as_float(__float_as_uint(al) & 0x7F800000u),
+                   __uint_as_float(__float_as_uint(ah) & 0x7F800000u));
+  float ml, mh;
+  upk(mul2(e, pk(0x1p22f, 0x1p22f)), ml, mh);
+  return pk(fmaxf(ml, 0x1p86f), fmaxf(mh, 0x1p86f));
+}
+
 // Power-of-two scales and the unscaled grid addend (MX formats).
 // 2^k as fp32 for k in [-127, 127] (2^-127 is a subnormal).
 __device__ __forceinline__ float pow2f(int k) {

@@ -328,7 +328,7 @@ __device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const Blk
     upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
     m |= (le_mask(fabsf(zl), kSixS) & (1u << pos)) | (le_mask(fabsf(zh), kSixS) & (2u << pos));
     const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
-    const u64 MM = pk(grid_magic_s(al), grid_magic_s(ah));
+    const u64 MM = MODE == kGuided ? grid_magic_s2(al, ah) : pk(grid_magic_s(al), grid_magic_s(ah));
     const u64 aa = pk(al, ah);
     float lol, loh, hil, hih;
     upk(add_rm2(aa, MM), lol, loh);
