@@ -78,6 +78,10 @@ def parse():
                     help="row chunks of the host-to-host step (copies overlap compute)")
     ap.add_argument("--eager", action="store_true",
                     help="time the step as separate launches instead of a CUDA-graph replay")
+    ap.add_argument("--one-stream", action="store_true",
+                    help="capture the graph on one stream (by default the round-to-nearest "
+                         "comparator runs on a second stream beside the guided forward and "
+                         "backward, which depend on capture only as it does)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline leg")
@@ -334,7 +338,11 @@ def run_trace(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None, dom=None, s=None):
+    def step(ev=None, dom=None, s=None, s2=None):
+        """One step over every site on stream s.  With a second stream s2 the
+        round-to-nearest comparator of each site runs there, ordered after that
+        site's capture (its only input besides x_train), beside the guided
+        forward and the backward; s waits for s2 at the end."""
         s = stream if s is None else s
         for i, w in enumerate(work):
             e = ev[i] if ev else None
@@ -342,15 +350,24 @@ def run_trace(args):
             if e: e[0].record(s)
             ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], s)
             if e: e[1].record(s)
+            if s2 is not None:
+                captured = torch.cuda.Event()
+                captured.record(s)
+                s2.wait_event(captured)
+                ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                               w["mask_r"], s2)
             if d: d[0].record(s)
             ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], s)
             if e: e[2].record(s)
             if d: d[1].record(s)
             ops.fq_bwd(w["g"], w["mask"], w["gin"], s)
             if e: e[3].record(s)
-            ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
-                           w["mask_r"], s)
+            if s2 is None:
+                ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                               w["mask_r"], s)
             if e: e[4].record(s)
+        if s2 is not None:
+            s.wait_stream(s2)
 
     for i in range(max(args.warmup, 3)):
         flush.fill_(i & 0xFF)
@@ -366,10 +383,13 @@ def run_trace(args):
             gph = torch.cuda.CUDAGraph()
             cs = torch.cuda.Stream()
             cs.wait_stream(stream)
+            side = None if args.one_stream else torch.cuda.Stream()
             # thread-local: other threads' CUDA calls (e.g. a process group's
             # watchdog) must not invalidate the capture
             with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
-                step(s=cs)
+                if side is not None:
+                    side.wait_stream(cs)  # fork inside the capture
+                step(s=cs, s2=side)
             torch.cuda.synchronize()
             for _ in range(max(args.warmup, 3)):
                 gph.replay()
@@ -745,7 +765,10 @@ def run_trace(args):
         "config": {"workload": workload, "shapes": shapes, "groups": groups,
                    "step": "capture + guided fwd + STE bwd + RTN fwd",
                    "l2": "flushed before every step (256 MiB write)",
-                   "launch": ("CUDA graph of the whole step, captured once and replayed"
+                   "launch": (("CUDA graph of the whole step, captured once and replayed"
+                               + ("" if args.one_stream else
+                                  "; the RTN comparator on a second stream beside the guided "
+                                  "forward and the backward"))
                               if graph_error is None and not args.eager else
                               "separate launches (programmatic stream serialization)"),
                    "parallelism": f"{world} independent sites, one per GPU (no collective)"},

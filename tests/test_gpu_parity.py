@@ -425,11 +425,14 @@ def test_argument_errors_enqueue_nothing():
     torch.cuda.synchronize()
 
 
-def test_step_in_a_cuda_graph(oracle_mod):
+@pytest.mark.parametrize("forked", [False, True])
+def test_step_in_a_cuda_graph(oracle_mod, forked):
     """The library's launches (with programmatic stream serialization) can be
     captured into a CUDA graph: a captured capture -> guided -> bwd -> RTN step
     replays to the oracle's outputs, also on new inputs copied into the same
-    buffers."""
+    buffers.  Forked: the RTN comparator on a second stream after the
+    capture, beside the guided forward and the backward (the benchmark's
+    graph)."""
     s = inputs.tiny_site(61, 640, 512, eps=0.01)
     xr, xt, g = (t.to(DEV) for t in (s.x_roll, s.x_train, s.grad))
     cap, ws = ops.alloc_capture(640, 512)
@@ -441,11 +444,18 @@ def test_step_in_a_cuda_graph(oracle_mod):
     cs = torch.cuda.Stream()
     cs.wait_stream(torch.cuda.current_stream())
     gph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
     with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
         ops.capture(xr, None, cap, ws, cs)
+        if forked:
+            side.wait_stream(cs)
+            ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, None, out_r, mask_r, side)
         ops.guided_fq_fwd(xt, cap, out, mask, cs)
         ops.fq_bwd(g, mask, gin, cs)
-        ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, None, out_r, mask_r, cs)
+        if forked:
+            cs.wait_stream(side)
+        else:
+            ops.rtn_fq_fwd(xt, cap.scales, cap.gscale, None, out_r, mask_r, cs)
     for seed in (61, 62):
         if seed == 62:
             s = inputs.tiny_site(seed, 640, 512, eps=0.03)
