@@ -82,6 +82,9 @@ def parse():
                     help="capture the graph on one stream (by default the round-to-nearest "
                          "comparator runs on a second stream beside the guided forward and "
                          "backward, which depend on capture only as it does)")
+    ap.add_argument("--lanes", type=int, default=2,
+                    help="independent sites of a multi-site workload run on this many "
+                         "stream pairs inside the graph (1: one after another)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="CPU work budget of the oracle baseline leg")
@@ -338,34 +341,54 @@ def run_trace(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None, dom=None, s=None, s2=None):
-        """One step over every site on stream s.  With a second stream s2 the
-        round-to-nearest comparator of each site runs there, ordered after that
-        site's capture (its only input besides x_train), beside the guided
-        forward and the backward; s waits for s2 at the end."""
+    def one_site(w, e, d, s, s2):
+        """capture -> guided fwd -> STE bwd on stream s; the RTN comparator on
+        s2 after the capture (its only input besides x_train), or on s after
+        the backward when s2 is None.  e / d: optional event lists for the
+        per-kernel breakdown and the dominant kernel."""
+        if e: e[0].record(s)
+        ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], s)
+        if e: e[1].record(s)
+        if s2 is not None:
+            captured = torch.cuda.Event()
+            captured.record(s)
+            s2.wait_event(captured)
+            ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                           w["mask_r"], s2)
+        if d: d[0].record(s)
+        ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], s)
+        if e: e[2].record(s)
+        if d: d[1].record(s)
+        ops.fq_bwd(w["g"], w["mask"], w["gin"], s)
+        if e: e[3].record(s)
+        if s2 is None:
+            ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                           w["mask_r"], s)
+        if e: e[4].record(s)
+
+    def step(ev=None, dom=None, s=None, s2=None, lanes=None):
+        """One step over every site.  Sites run one after another on s, each
+        with its RTN comparator on s2 when given; with lanes (a list of (main,
+        side) stream pairs) site i runs on lanes[i % len] instead, since the
+        sites are independent.  Every stream used joins s at the end."""
         s = stream if s is None else s
+        if lanes:
+            for m, sd in lanes:
+                m.wait_stream(s)  # fork
+                if sd is not None:
+                    sd.wait_stream(s)
+            for i, w in enumerate(work):
+                m, sd = lanes[i % len(lanes)]
+                one_site(w, None, None, m, sd)
+            for m, sd in lanes:
+                s.wait_stream(m)  # join
+                if sd is not None:
+                    s.wait_stream(sd)
+            return
+        if s2 is not None:
+            s2.wait_stream(s)
         for i, w in enumerate(work):
-            e = ev[i] if ev else None
-            d = dom[i] if dom else None
-            if e: e[0].record(s)
-            ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], s)
-            if e: e[1].record(s)
-            if s2 is not None:
-                captured = torch.cuda.Event()
-                captured.record(s)
-                s2.wait_event(captured)
-                ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
-                               w["mask_r"], s2)
-            if d: d[0].record(s)
-            ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], s)
-            if e: e[2].record(s)
-            if d: d[1].record(s)
-            ops.fq_bwd(w["g"], w["mask"], w["gin"], s)
-            if e: e[3].record(s)
-            if s2 is None:
-                ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
-                               w["mask_r"], s)
-            if e: e[4].record(s)
+            one_site(w, ev[i] if ev else None, dom[i] if dom else None, s, s2)
         if s2 is not None:
             s.wait_stream(s2)
 
@@ -384,12 +407,16 @@ def run_trace(args):
             cs = torch.cuda.Stream()
             cs.wait_stream(stream)
             side = None if args.one_stream else torch.cuda.Stream()
+            nl = min(max(args.lanes, 1), len(work))
+            lanes = ([(torch.cuda.Stream(), None if args.one_stream else torch.cuda.Stream())
+                      for _ in range(nl)] if nl > 1 else None)
             # thread-local: other threads' CUDA calls (e.g. a process group's
             # watchdog) must not invalidate the capture
             with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
-                if side is not None:
-                    side.wait_stream(cs)  # fork inside the capture
-                step(s=cs, s2=side)
+                if lanes:
+                    step(s=cs, lanes=lanes)
+                else:
+                    step(s=cs, s2=side)
             torch.cuda.synchronize()
             for _ in range(max(args.warmup, 3)):
                 gph.replay()
@@ -768,7 +795,9 @@ def run_trace(args):
                    "launch": (("CUDA graph of the whole step, captured once and replayed"
                                + ("" if args.one_stream else
                                   "; the RTN comparator on a second stream beside the guided "
-                                  "forward and the backward"))
+                                  "forward and the backward")
+                              + (f"; sites on {min(max(args.lanes, 1), len(work))} stream lanes"
+                                 if min(max(args.lanes, 1), len(work)) > 1 else ""))
                               if graph_error is None and not args.eager else
                               "separate launches (programmatic stream serialization)"),
                    "parallelism": f"{world} independent sites, one per GPU (no collective)"},

@@ -425,6 +425,50 @@ def test_argument_errors_enqueue_nothing():
     torch.cuda.synchronize()
 
 
+def test_two_sites_on_two_lanes_in_a_cuda_graph(oracle_mod):
+    """Two independent sites captured into one graph on two stream lanes
+    (each lane: capture -> guided -> bwd, with the RTN comparator on the
+    lane's side stream), forked from and joined to the capture stream, as
+    the benchmark runs multi-site workloads: every output matches the
+    oracle."""
+    sites = [inputs.tiny_site(71, 384, 256, eps=0.01), inputs.tiny_site(72, 512, 128, eps=0.02)]
+    bufs = []
+    for st in sites:
+        R, C = st.x_roll.shape
+        cap, ws = ops.alloc_capture(R, C)
+        bufs.append(dict(xr=st.x_roll.to(DEV), xt=st.x_train.to(DEV), g=st.grad.to(DEV),
+                         cap=cap, ws=ws, out=torch.empty(R, C, dtype=torch.bfloat16, device=DEV),
+                         mask=torch.empty(R * C // 32, dtype=torch.int32, device=DEV),
+                         gin=torch.empty(R, C, dtype=torch.bfloat16, device=DEV),
+                         out_r=torch.empty(R, C, dtype=torch.bfloat16, device=DEV),
+                         mask_r=torch.empty(R * C // 32, dtype=torch.int32, device=DEV)))
+    cs = torch.cuda.Stream()
+    cs.wait_stream(torch.cuda.current_stream())
+    lanes = [(torch.cuda.Stream(), torch.cuda.Stream()) for _ in sites]
+    gph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
+        for (m, sd), b in zip(lanes, bufs):
+            m.wait_stream(cs)
+            ops.capture(b["xr"], None, b["cap"], b["ws"], m)
+            sd.wait_stream(m)
+            ops.rtn_fq_fwd(b["xt"], b["cap"].scales, b["cap"].gscale, None, b["out_r"], b["mask_r"], sd)
+            ops.guided_fq_fwd(b["xt"], b["cap"], b["out"], b["mask"], m)
+            ops.fq_bwd(b["g"], b["mask"], b["gin"], m)
+        for m, sd in lanes:
+            cs.wait_stream(m)
+            cs.wait_stream(sd)
+    gph.replay()
+    torch.cuda.synchronize()
+    for k, (st, b) in enumerate(zip(sites, bufs)):
+        ref = run_oracle(oracle_mod, st)
+        got = dict(codes=_u(b["cap"].codes), mbits=_u(b["cap"].mbits), scales=_u(b["cap"].scales),
+                   gscale=_u(b["cap"].gscale), out=_u(b["out"]), mask=_u(b["mask"]),
+                   grad_in=_u(b["gin"]), out_rtn=_u(b["out_r"]), mask_rtn=_u(b["mask_r"]))
+        for key in got:
+            _eq(f"lanes.{k}.{key}", got[key], ref[key])
+    del gph
+
+
 @pytest.mark.parametrize("forked", [False, True])
 def test_step_in_a_cuda_graph(oracle_mod, forked):
     """The library's launches (with programmatic stream serialization) can be
