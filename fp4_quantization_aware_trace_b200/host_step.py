@@ -31,6 +31,16 @@ def _row_quantum(cols: int) -> int:
     return 256 // math.gcd(cols, 256)
 
 
+def row_chunks(rows: int, cols: int, chunks: int) -> list[tuple[int, int]]:
+    """Row ranges [a, b) covering 0..rows in about `chunks` pieces, every
+    start a multiple of the row quantum (so each chunk's slices of every
+    array keep the alignment the calls require); no empty range."""
+    q = _row_quantum(cols)
+    per = max(q, -(-rows // max(1, chunks)) // q * q)
+    cuts = list(range(0, rows, per)) + [rows]
+    return [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+
+
 class HostStep:
     """The step for one site of shape [rows, cols] (groups by host int64
     offsets, or None), in `chunks` row chunks."""
@@ -45,10 +55,7 @@ class HostStep:
         self.device = torch.device(device)
         self.offsets_h = None if offsets is None else torch.as_tensor(offsets, dtype=torch.int64)
         self.G = 1 if offsets is None else int(self.offsets_h.numel()) - 1
-        q = _row_quantum(cols)
-        per = max(q, -(-rows // max(1, chunks)) // q * q)
-        cuts = list(range(0, rows, per)) + [rows]
-        self.cuts = [(a, b) for a, b in zip(cuts[:-1], cuts[1:]) if b > a]
+        self.cuts = row_chunks(rows, cols, chunks)
         # chunk-local group offsets (the group ids stay global)
         self.chunk_offs = []
         for a, b in self.cuts:
