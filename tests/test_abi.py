@@ -160,3 +160,25 @@ def test_validate_offsets_argument_checks(lib):
     assert lib.trace_validate_offsets(a, 0, 4, a, None) == 2
     assert lib.trace_validate_offsets(None, 2, 4, a, None) == 1
     assert lib.trace_validate_offsets(P((1 << 20) + 4), 2, 4, a, None) == 3
+
+
+def test_host_argument_checks_check_calls(lib):
+    """The self-test, the offset check and capture without a workspace reject
+    bad arguments before any CUDA call (fake, never dereferenced pointers)."""
+    P = ctypes.c_void_p
+    a = P(1 << 20)
+    odd = P((1 << 20) + 2)
+    # E4M3 self-test: nothing to do, no output, inputs not below +inf
+    assert lib.trace_selftest_e4m3_sweep(0x3F800000, 0, None, None) == 0
+    assert lib.trace_selftest_e4m3_sweep(0x3F800000, 16, None, None) == 1
+    assert lib.trace_selftest_e4m3_sweep(0x7F800000, 1, a, None) == 2
+    assert lib.trace_selftest_e4m3_sweep(0x7F7FFFFF, 2, a, None) == 2
+    # offset check: groups, rows, pointers, alignment
+    assert lib.trace_validate_offsets(a, 0, 16, a, None) == 2
+    assert lib.trace_validate_offsets(a, 1, -1, a, None) == 2
+    assert lib.trace_validate_offsets(None, 2, 16, a, None) == 1
+    assert lib.trace_validate_offsets(a, 2, 16, None, None) == 1
+    assert lib.trace_validate_offsets(P((1 << 20) + 4), 2, 16, a, None) == 3
+    assert lib.trace_validate_offsets(a, 2, 16, odd, None) == 3
+    # capture without a workspace: more groups than its static scratch holds
+    assert lib.trace_capture_static_ws(a, 4, 32, 4097, a, a, a, a, a, None) == 4
