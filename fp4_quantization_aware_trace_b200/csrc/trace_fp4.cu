@@ -667,13 +667,24 @@ int trace_capture_static_ws(const uint16_t* x, int64_t rows, int64_t cols, int32
   if (num_groups > TRACE_STATIC_MAX_GROUPS) return TRACE_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TRACE_ERR_CUDA;
+  // The host-side name of the array is only a stand-in, so the kernels get
+  // the address the runtime reports for the current device.  It is looked up
+  // on the first call on a device and again on every call made outside
+  // stream capture: cudaDeviceReset unloads the module, and the array may
+  // come back at another address.  While the stream is capturing, the
+  // address found by an earlier call is used.
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  bool capturing = true;
+  if (cudaStreamIsCapturing((cudaStream_t)stream, &cs) == cudaSuccess)
+    capturing = cs != cudaStreamCaptureStatusNone;
+  else
+    (void)cudaGetLastError();  // the query failed: treat the stream as capturing
   void* ws = g_capture_scratch_addr[dev];
-  if (ws == nullptr) {
-    // first call on this device: the host-side name of the array is only a
-    // stand-in, so ask the runtime for its address on the current device
-    if (cudaGetSymbolAddress(&ws, g_capture_scratch) != cudaSuccess || ws == nullptr)
+  if (!capturing || ws == nullptr) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_capture_scratch) != cudaSuccess || a == nullptr)
       return TRACE_ERR_CUDA;
-    g_capture_scratch_addr[dev] = ws;
+    g_capture_scratch_addr[dev] = ws = a;
   }
   // the accumulators are zeroed by the capture's first kernel on every call
   return trace_capture(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,

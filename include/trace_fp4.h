@@ -42,8 +42,8 @@
  * passed as void*, NULL = the legacy default stream).  The library holds no
  * mutable global state apart from a per-device cache of the SM count (and
  * the static scratch of trace_capture_static_ws, see there), so it may be
- * called from several host threads.  Every call is capturable into a CUDA
- * graph (trace_capture_static_ws after its first call on the device).
+ * called from several host threads.  Every call that takes its scratch
+ * memory from the caller is capturable into a CUDA graph.
  *
  * Contents, in order: status and version; workspace and record-size queries;
  * the NVFP4 path (capture, 1-bit guided and full-information guided
@@ -354,7 +354,10 @@ int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols,
                             uint32_t* mbits, uint8_t* scales, float* gscale,
                             int32_t scale_layout, void* stream);
 
-/* Masked straight-through-estimator backward:
+/* Masked straight-through-estimator backward: the gradient half of the
+ * listing's straight_through_estimator(x_train, s * q_star) (QAT-forward half
+ * of the post's pseudocode listing), which passes the upstream gradient
+ * through the fake-quant unchanged; masked where the forward clipped:
  * grad_in[i] = mask bit i ? grad_out[i] : +0.0 (bit copy).
  *   grad_out, grad_in: bf16 [numel], 32-byte aligned; may alias.
  *   ste_mask: uint32[numel/32], 16-byte aligned.  numel % 32 == 0. */
@@ -409,7 +412,11 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel,
  *   enqueues nothing.
  *   The first call on each device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  Nothing here calls cudaMalloc or cudaFree.
+ *   before any stream capture.  Every later call made outside stream capture
+ *   looks the address up again, because cudaDeviceReset unloads the module
+ *   and the array may come back at another address: after a reset, make the
+ *   first call outside stream capture too.  Nothing here calls cudaMalloc or
+ *   cudaFree.
  *   Every call on a device shares the one array (its contents are zeroed at
  *   the start of each call): two calls that may run at the same time on the
  *   GPU -- e.g. on streams with no ordering between them -- race on it and

@@ -91,3 +91,25 @@ def test_static_workspace_rejects_too_many_groups():
     torch.cuda.synchronize()
     assert st == 4  # TRACE_ERR_WORKSPACE: nothing enqueued
     assert torch.all(o["gscale"] == -7.0)
+
+
+def test_static_workspace_capture_after_device_reset(tmp_path):
+    """cudaDeviceReset unloads the library's module, so the static array may
+    come back at another device address; a plain C program (its own process,
+    since a reset would also pull the device out from under torch) captures
+    without a workspace before and after a reset and compares every output
+    with trace_capture given a workspace."""
+    import os
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "fp4_quantization_aware_trace_b200")
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    exe = str(tmp_path / "c_static_ws_reset")
+    subprocess.run(["gcc", "-O2", "-std=c11", "-Wall", "-Werror", "-I",
+                    os.path.join(root, "include"), "-I", os.path.join(cuda, "include"),
+                    os.path.join(root, "tests", "c_static_ws_reset.c"), "-L", pkg, "-ltrace_fp4",
+                    "-L", os.path.join(cuda, "lib64"), "-lcudart",
+                    f"-Wl,-rpath,{pkg}:{os.path.join(cuda, 'lib64')}", "-o", exe],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
