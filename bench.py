@@ -1,29 +1,37 @@
 #!/usr/bin/env python
 """Throughput of the TRACE capture + guided NVFP4 fake-quant hot path on B200.
 
-One step = one pass of the whole path over one synthetic activation site:
-  rollout capture of x_roll  (3 launches: zero accumulators, grid amax, quantise
-                              -> FP4 codes + compact cache of mantissa bits and scales)
+One step = one pass of the whole path over every site of the workload:
+  rollout capture of x_roll  (grid amax, then quantise -> FP4 codes + compact
+                              cache of mantissa bits and scales)
   guided fake-quant forward of x_train with that cache (bf16 out + STE mask)
   masked straight-through backward of an upstream gradient
   round-to-nearest fake-quant forward of x_train (the vanilla-QAT comparator)
 
-Workload: the Qwen3-30B-A3B-shaped attention-input site, bf16 [16384, 2048],
-lognormal channel scales, 1% outlier channels x100, 0.5% relative training
-noise (seeded, synthetic).  L2 is flushed (256 MiB write) before every step.
+Default workload (the headline): the later-half layer sweep, all 80 sites --
+layers 20..39 of 40 x {qkv-in, o-in, expert up-in, expert down-in}, each
+[65536, 4096] bf16, lognormal channel scales, 1% outlier channels x100, 0.5%
+relative training noise (seeded, synthetic).  All 80 sites' x_roll, x_train
+and grad (120 GiB) stay resident in HBM; every input is read from HBM once
+per step (far larger than the 126 MB L2, so no flush is needed between
+steps).  The attention-input site [16384, 2048] is measured after it, as a
+secondary line (`secondary`), with L2 flushed before every step.
 
-The reported value is algorithmic bytes / time (GB/s): every input read once
-and every output written once per kernel, x_roll read twice by capture (its
-two passes).  Per-element bytes: capture 4.6875, guided 4.3125, backward
-4.125, RTN 4.1875 (+4 bytes per group).  elem/s and the fraction of the
-measured HBM copy bandwidth are reported beside it.
+The value is algorithmic bytes / time (GB/s): every input read once and every
+output written once per kernel, x_roll read twice by capture (its two
+passes).  Per-element bytes: capture 4.6875, guided 4.3125, backward 4.125,
+RTN 4.1875 (+4 bytes per group).  elem/s is reported beside it, and
+`algo_bytes_over_copy_peak` divides the step's algorithmic GB/s by the
+measured copy bandwidth -- not a DRAM fraction: reads that hit L2 count too.
+The per-kernel `roofline` is the HBM fraction of the dominant kernel.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl trace|reference]
                        [--config 1..5]
---config picks another of the five workloads for the same measurement (a step
-then covers every tensor of the workload; the headline is --config 2, the
-default).  Under torchrun every rank runs its own sites (weak scaling, no
-collective on the data path); rank 0 prints one JSON line.
+--config picks one of the five workloads (1 single activation, 2 attention
+input, 3 MoE experts, 4 KV cache, 5 the layer sweep: default).  --gpus N > 1
+without torchrun starts N ranks itself (torch.distributed.run on 127.0.0.1);
+every rank runs its own draw of the workload (weak scaling, no collective on
+the data path) and rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
@@ -32,6 +40,7 @@ import hashlib
 import json
 import os
 import re
+import socket
 import statistics
 import subprocess
 import sys
@@ -44,15 +53,24 @@ if ROOT not in sys.path:
 import torch  # noqa: E402
 
 METRIC = "capture & guided fake-quant fwd GB/s (elem/s) and % of B200 HBM roofline"
-ROWS, COLS = 16384, 2048
-WORKLOAD = "attn_in [16384 x 2048] bf16, Qwen3-30B-A3B-shaped attention-input site"
+HEADLINE_CONFIG = 5
+SECONDARY_CONFIG = 2
 BYTES_PER_ELEM = {"capture": 4.6875, "guided_fwd": 4.3125, "ste_bwd": 4.125, "rtn_fwd": 4.1875}
+STEP_BYTES_PER_ELEM = sum(BYTES_PER_ELEM.values())
 KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<1> (1-bit guided)",
                 "ste_bwd": "k_ste_bwd", "rtn_fwd": "k_fake_quant<0> (round to nearest)"}
-LAUNCHES_PER_STEP = 6  # zero + amax + capture, guided, bwd, rtn
+# kernels of the library launched per site and step: capture (zeroing of the
+# accumulators, amax pass, quantising pass), guided forward, backward, RTN
+LAUNCHES_PER_SITE = 6
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 * 10 ** 6
 CSRC_DIR = os.path.join(ROOT, "fp4_quantization_aware_trace_b200", "csrc")
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+# row windows of the CPU legs (whole rows; about 80 M elements for the
+# baseline leg, 20 M per step for the reference arm)
+CPU_SAMPLE_ELEMS = 80 * 2 ** 20
+REF_SAMPLE_ELEMS = 20 * 2 ** 20
 
 
 def source_hash() -> str:
@@ -64,10 +82,9 @@ def source_hash() -> str:
             with open(os.path.join(CSRC_DIR, name), "rb") as f:
                 h.update(f.read())
     return h.hexdigest()[:16]
-PROFILE_DIR = os.path.join(ROOT, "profiles")
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -76,6 +93,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-chunks", type=int, default=8,
                     help="row chunks of the host-to-host step (copies overlap compute)")
+    ap.add_argument("--e2e-steps", type=int, default=2,
+                    help="timed end-to-end steps (each covers every site)")
     ap.add_argument("--eager", action="store_true",
                     help="time the step as separate launches instead of a CUDA-graph replay")
     ap.add_argument("--one-stream", action="store_true",
@@ -86,12 +105,18 @@ def parse():
                     help="independent sites of a multi-site workload run on this many "
                          "stream pairs inside the graph (1: one after another)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0,
-                    help="CPU work budget of the oracle baseline leg")
-    ap.add_argument("--config", type=int, default=2, choices=[1, 2, 3, 4, 5],
-                    help="workload: 1 single activation, 2 attention input (default, the "
-                         "headline), 3 MoE experts, 4 KV cache, 5 later-half layer sweep")
-    return ap.parse_args()
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the secondary line (attention-input site) after the headline")
+    ap.add_argument("--next-sites", type=int, default=8,
+                    help="sites of the workload the next-row legs (full guidance, "
+                         "histogram, MXFP4, W4A8, tiled scales, cache tier) run on")
+    ap.add_argument("--plumbing-only", action="store_true",
+                    help="run only the multi-rank plumbing (launch, process group over gloo, "
+                         "max over ranks) on CPU, without any GPU work; prints one JSON line")
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG, choices=[1, 2, 3, 4, 5],
+                    help="workload: 1 single activation, 2 attention input, 3 MoE experts, "
+                         "4 KV cache, 5 later-half layer sweep (default, the headline)")
+    return ap.parse_args(argv)
 
 
 def dist_env():
@@ -99,6 +124,20 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def rank_launch_cmd(argv: list[str], gpus: int, port: int) -> list[str]:
+    """Command that runs this script on `gpus` ranks of one node (one
+    process per GPU) with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1",
+            f"--master-port={port}", os.path.abspath(__file__), *argv]
 
 
 def measured_peaks():
@@ -110,17 +149,17 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def traffic_from_profiles(kernel_key: str):
-    """Per-launch DRAM bytes of a kernel from the committed ncu summary, or
-    None when the summary is missing or the source changed since."""
-    src_hash = source_hash()
-    path = os.path.join(PROFILE_DIR, f"{kernel_key}_attn_in_16384x2048.md")
+def traffic_from_profiles(kernel_key: str, tag: str):
+    """Per-launch DRAM bytes of a kernel from the committed ncu summary
+    `profiles/<kernel_key>_<tag>.md`, or None when the summary is missing or
+    the source changed since."""
+    path = os.path.join(PROFILE_DIR, f"{kernel_key}_{tag}.md")
     if not os.path.exists(path):
         return None
     txt = open(path).read()
     h = re.search(r"source_sha256_16:\s*([0-9a-f]+)", txt)
     t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
-    if not h or not t or h.group(1) != src_hash:
+    if not h or not t or h.group(1) != source_hash():
         return None
     return int(t.group(1))
 
@@ -134,6 +173,7 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
 
     def __enter__(self):
         try:
@@ -147,7 +187,6 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
         if self.proc is not None:
             time.sleep(0.3)
             self.proc.terminate()
@@ -156,7 +195,7 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
                 out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+            self.lines += [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
         if not self.lines:
@@ -189,113 +228,185 @@ def max_over_ranks(values, pg, device):
 
 
 def job_gbs(world: int, n_per_rank: int, bytes_per_elem: float, ms_per_step: float) -> float:
-    """Whole-job algorithmic GB/s: every rank processes its own site of
-    n_per_rank elements per step; the step time is the slowest rank's."""
+    """Whole-job algorithmic GB/s: every rank processes its own draw of the
+    workload (n_per_rank elements per step); the step time is the slowest
+    rank's."""
     return world * n_per_rank * bytes_per_elem / (ms_per_step * 1e-3) / 1e9
 
 
 def site_seed(rank: int) -> int:
-    """Seed of rank r's site: rank 0 is the workload's own seed (1)."""
+    """Seed of rank r's attention-input site: rank 0 is the workload's own seed (1)."""
     return 1 + 1000 * rank
 
 
-def make_site(rank: int, device):
-    from fp4_quantization_aware_trace_b200 import inputs
-    return inputs.attention_input(seed=site_seed(rank), rows=ROWS, cols=COLS, device=device)
+# ---------------------------------------------------------------------------
+# Workloads
+# ---------------------------------------------------------------------------
+
+WORKLOAD_NAMES = {
+    1: "single activation [256 x 2048] bf16, 8 outlier channels x50",
+    2: "attn_in [16384 x 2048] bf16, Qwen3-30B-A3B-shaped attention-input site",
+    3: ("MoE experts: 128 experts x 512 tokens, up-proj input [65536 x 2048] and down-proj "
+        "input [65536 x 768] bf16, one group per expert"),
+    4: "FP4 KV cache: K and V [32768 tokens, 4 heads, 128] bf16 as [131072 x 128]",
+    5: ("later-half layer sweep: all 80 sites (layers 20-39 of 40 x qkv-in, o-in, up-in, "
+        "down-in), each [65536 x 4096] bf16"),
+}
+WORKLOAD_TAGS = {1: "single_256x2048", 2: "attn_in_16384x2048", 3: "moe_experts_g128",
+                 4: "kv_cache_131072x128", 5: "layer_sweep_65536x4096"}
 
 
-def make_workload(cfg: int, rank: int, device):
-    """(workload name, sites) of a configuration; rank r shifts every seed."""
+def workload_shapes(cfg: int) -> list[tuple[int, int]]:
+    """[rows, cols] of every site of a configuration (without drawing it)."""
+    return {1: [(256, 2048)], 2: [(16384, 2048)], 3: [(65536, 2048), (65536, 768)],
+            4: [(131072, 128)] * 2, 5: [(65536, 4096)] * 80}[cfg]
+
+
+def workload_sites(cfg: int, rank: int, device):
+    """The sites of a configuration, generated one at a time (a generator);
+    rank r draws its own copy of the recipe (every seed shifted)."""
     from fp4_quantization_aware_trace_b200 import inputs
     off = 1000 * rank
     if cfg == 1:
-        return ("single activation [256 x 2048] bf16, 8 outlier channels x50",
-                [inputs.single_activation(0 + off, device=device)])
-    if cfg == 2:
-        return WORKLOAD, [make_site(rank, device)]
-    if cfg == 3:
-        return ("MoE experts: 128 experts x 512 tokens, up-proj input [65536 x 2048] and "
-                "down-proj input [65536 x 768] bf16, one group per expert",
-                [inputs.moe_experts(2 + off, cols=2048, device=device, name="expert_up_in"),
-                 inputs.moe_experts(12 + off, cols=768, device=device, name="expert_down_in")])
-    if cfg == 4:
-        return ("FP4 KV cache: K and V [32768 tokens, 4 heads, 128] bf16 as [131072 x 128]",
-                [inputs.kv_cache(3 + off, device=device, which="k"),
-                 inputs.kv_cache(3 + off, device=device, which="v")])
-    sites = [inputs.layer_sweep_site(layer, k, device=device)
-             for layer in (20, 21) for k in range(4)]
-    if rank:
-        sites = [inputs.layer_sweep_site(20 + 2 * rank + layer % 2, k, device=device)
-                 for layer in (20, 21) for k in range(4)]
-    return ("later-half layer sweep: 8 of the 80 sites (layers 20-21 x qkv-in, o-in, up-in, "
-            "down-in), each [65536 x 4096] bf16", sites)
+        yield inputs.single_activation(0 + off, device=device)
+    elif cfg == 2:
+        yield inputs.attention_input(seed=site_seed(rank), device=device)
+    elif cfg == 3:
+        yield inputs.moe_experts(2 + off, cols=2048, device=device, name="expert_up_in")
+        yield inputs.moe_experts(12 + off, cols=768, device=device, name="expert_down_in")
+    elif cfg == 4:
+        yield inputs.kv_cache(3 + off, device=device, which="k")
+        yield inputs.kv_cache(3 + off, device=device, which="v")
+    else:
+        for layer in range(20, 40):
+            for k in range(len(inputs.LAYER_SWEEP_SITES)):
+                yield inputs.layer_sweep_site(layer, k, device=device, seed_offset=off)
 
 
 # ---------------------------------------------------------------------------
 # CPU oracle legs (reported baseline / reference arm)
 # ---------------------------------------------------------------------------
 
-def oracle_step(oracle, xr, xt, g):
-    codes, mbits, scales, gscale = oracle.capture(xr)
-    out, mask = oracle.guided_fwd(xt, mbits, scales, gscale)
-    oracle.fq_bwd(g, mask)
-    oracle.rtn_fwd(xt, scales, gscale)
+def site_sample(site, rows_per_site: int, index: int):
+    """Host copies of a window of whole rows of a site plus the global scale
+    of each of those rows, taken from the whole tensor's per-group amax (so
+    the window is quantised exactly as it is inside the whole tensor).
+    The window starts at a seeded row; the amax is taken with torch on the
+    tensor's own device, the global scale with the oracle."""
+    import numpy as np
 
-
-def cpu_oracle_rate(site, budget_s: float, rows: int | None = None):
-    """Time the oracle, as it stands, on host copies of the workload (or its
-    first `rows` rows); returns (GB/s, elem/s, seconds, sample text)."""
     import oracle
     from fp4_quantization_aware_trace_b200 import inputs
+    R, C = site.x_roll.shape
+    k = min(R, max(1, rows_per_site))
+    a = int(np.random.default_rng(1234 + index).integers(0, R - k + 1))
+    offs = None if site.offsets is None else site.offsets.cpu().numpy()
+    mags = site.x_roll.abs()
+    if offs is None:
+        amax = [float(mags.max())]
+    else:
+        amax = [float(mags[int(offs[g]):int(offs[g + 1])].max()) if offs[g + 1] > offs[g] else 0.0
+                for g in range(len(offs) - 1)]
+    gs = np.array([oracle.global_scale(m) for m in amax], np.float32)
+    if offs is None:
+        rg = np.full(k, gs[0], np.float32)
+    else:
+        rg = np.repeat(gs, np.diff(offs)).astype(np.float32)[a:a + k].copy()
+    xr, xt, g = (inputs.bits(t[a:a + k]) for t in (site.x_roll, site.x_train, site.grad))
+    return {"xr": xr, "xt": xt, "g": g, "rg": rg}
+
+
+def oracle_sample_step(samples, threads: int):
+    """The oracle's whole step on every sample, threaded over row chunks:
+    amax pass, capture, guided forward, backward, round-to-nearest forward."""
+    import oracle.threaded as ot
+    for s in samples:
+        ot.group_amax_mt(s["xr"], threads=threads)
+        codes, mbits, scales = ot.capture_rows_mt(s["xr"], s["rg"], threads)
+        _, mask = ot.fake_quant_rows_mt(s["xt"], s["rg"], scales, mbits, threads)
+        ot.fq_bwd_mt(s["g"], mask, threads)
+        ot.fake_quant_rows_mt(s["xt"], s["rg"], scales, None, threads)
+
+
+def rows_per_site(cfg: int, shapes, budget_elems: int) -> int:
+    n_sites = len(shapes)
+    cols = max(c for _, c in shapes)
+    return max(1, budget_elems // (n_sites * cols))
+
+
+def cpu_baseline_leg(cfg: int, sites, budget_elems: int = CPU_SAMPLE_ELEMS, repeats: int = 2):
+    """The oracle, as it stands, threaded over every core of this process,
+    on a window of rows of every site; returns the cpu_baseline object."""
+    import oracle
+    import oracle.threaded as ot
     oracle.build()
-    xr, xt, g = (inputs.bits(t) for t in (site.x_roll, site.x_train, site.grad))
-    if rows is not None:
-        xr, xt, g = xr[:rows].copy(), xt[:rows].copy(), g[:rows].copy()
-    n = xr.size
-    passes, t0 = 0, time.perf_counter()
-    while True:
-        oracle_step(oracle, xr, xt, g)
-        passes += 1
-        el = time.perf_counter() - t0
-        if el >= budget_s:
-            break
-    per = el / passes
-    bpe = sum(BYTES_PER_ELEM.values())
-    sample = (f"{passes} full step(s) (capture+guided+bwd+rtn) over the first {xr.shape[0]} of "
-              f"{ROWS} rows [{xr.shape[0]} x {COLS}] of the same site, single-threaded C oracle")
-    return n * bpe / per / 1e9, n / per, per, sample
+    shapes = [tuple(s.x_roll.shape) for s in sites]
+    rps = rows_per_site(cfg, shapes, budget_elems)
+    samples = [site_sample(s, rps, i) for i, s in enumerate(sites)]
+    n = sum(s["xr"].size for s in samples)
+    threads = ot.cores()
+    oracle_sample_step(samples[:1], threads)  # untimed: library load, pool start
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle_sample_step(samples, threads)
+    per = (time.perf_counter() - t0) / repeats
+    return {"value": round(n * STEP_BYTES_PER_ELEM / per / 1e9, 4), "unit": "GB/s",
+            "cores": threads, "host_cores": os.cpu_count(), "kind": "oracle",
+            "elem_per_s": round(n / per, 1), "s_per_step": round(per, 3),
+            "sample": (f"{repeats} passes of the whole step (amax, capture, guided fwd, STE bwd, "
+                       f"RTN fwd) over a window of {min(rps, shapes[0][0])} whole rows of each of "
+                       f"the {len(sites)} sites ({n} elements), each window quantised with its "
+                       f"tensor's whole-tensor global scale; the C oracle threaded over row "
+                       f"chunks on {threads} cores")}
 
 
 def run_reference(args):
     world, rank, local = dist_env()
     if rank != 0:
         return
-    site = make_site(0, "cpu")
     import oracle
-    from fp4_quantization_aware_trace_b200 import inputs
+    import oracle.threaded as ot
     oracle.build()
-    sample_rows = 4096
-    xr, xt, g = (inputs.bits(t)[:sample_rows].copy() for t in (site.x_roll, site.x_train, site.grad))
-    n = xr.size
+    # the inputs are drawn where the GPU arm draws them (same values), one
+    # site at a time; only each site's row window is kept, on the host
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
+    else:
+        dev = torch.device("cpu")
+    shapes = workload_shapes(args.config)
+    # the row window per site is fixed by the step budget and the shapes
+    rps = rows_per_site(args.config, shapes, REF_SAMPLE_ELEMS)
+    samples = []
+    for i, site in enumerate(workload_sites(args.config, 0, dev)):
+        samples.append(site_sample(site, rps, i))
+        del site
+    if dev.type == "cuda":
+        torch.cuda.empty_cache()
+    n = sum(s["xr"].size for s in samples)
+    threads = ot.cores()
     for _ in range(args.warmup):
-        oracle_step(oracle, xr, xt, g)
+        oracle_sample_step(samples, threads)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_step(oracle, xr, xt, g)
+        oracle_sample_step(samples, threads)
     el = time.perf_counter() - t0
-    bpe = sum(BYTES_PER_ELEM.values())
-    value = n * bpe * args.steps / el / 1e9
-    sample = f"each step: the first {sample_rows} of {ROWS} rows [{sample_rows} x {COLS}]"
+    value = n * STEP_BYTES_PER_ELEM * args.steps / el / 1e9
+    sample = (f"each step: the oracle's whole step over a window of {min(rps, shapes[0][0])} "
+              f"whole rows of each of the {len(shapes)} sites ({n} elements), each window "
+              f"quantised with its tensor's whole-tensor global scale; threaded over row "
+              f"chunks on {threads} cores")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * el / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "elem_per_s": round(n * args.steps / el, 1),
-        "config": {"workload": WORKLOAD, "rows": sample_rows, "cols": COLS, "groups": 1,
+        "config": {"workload": WORKLOAD_NAMES[args.config], "shapes": [list(s) for s in shapes],
+                   "rows_per_site": min(rps, shapes[0][0]),
                    "step": "capture + guided fwd + STE bwd + RTN fwd", "l2": "n/a (CPU)"},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "host_cores": os.cpu_count(), "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -306,117 +417,157 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
-def run_trace(args):
-    world, rank, local = dist_env()
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    pg = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
-        pg = dist
+def _ev():
+    return torch.cuda.Event(enable_timing=True)
 
+
+def _pair():
+    return (_ev(), _ev())
+
+
+class Workload:
+    """The sites of a configuration resident on the device, with what the
+    step writes: each site keeps its compact cache (mantissa bits, scales,
+    global scales); the FP4 codes and the forward / backward outputs live in
+    one set of buffers per stream lane (sites on one lane run in order)."""
+
+    def __init__(self, cfg: int, rank: int, dev, lanes: int):
+        from fp4_quantization_aware_trace_b200 import ops
+        self.cfg, self.dev = cfg, dev
+        self.sites = []
+        for site in workload_sites(cfg, rank, dev):
+            self.sites.append(site)
+        self.nl = max(1, min(lanes, len(self.sites)))
+        nmax = max(s.x_roll.numel() for s in self.sites)
+        i32, bf = torch.int32, torch.bfloat16
+        self.lane_buf = [dict(codes=torch.empty(nmax // 2, dtype=torch.uint8, device=dev),
+                              out=torch.empty(nmax, dtype=bf, device=dev),
+                              gin=torch.empty(nmax, dtype=bf, device=dev),
+                              out_r=torch.empty(nmax, dtype=bf, device=dev),
+                              mask=torch.empty(nmax // 32, dtype=i32, device=dev),
+                              mask_r=torch.empty(nmax // 32, dtype=i32, device=dev))
+                         for _ in range(self.nl)]
+        self.work = []
+        for i, site in enumerate(self.sites):
+            R, C = site.x_roll.shape
+            n = R * C
+            lb = self.lane_buf[i % self.nl]
+            offs = None if site.offsets is None else site.offsets.to(dev)
+            G = site.num_groups
+            cap = ops.Capture(codes=lb["codes"][:n // 2],
+                              mbits=torch.empty(n // 32, dtype=i32, device=dev),
+                              scales=torch.empty(R, C // 16, dtype=torch.uint8, device=dev),
+                              gscale=torch.empty(G, dtype=torch.float32, device=dev),
+                              offsets=offs)
+            ws = torch.empty(max(ops.trace_capture_workspace_bytes(R, C, G), 256),
+                             dtype=torch.uint8, device=dev)
+            self.work.append(dict(
+                site=site, xr=site.x_roll, xt=site.x_train, g=site.grad, offs=offs, cap=cap, ws=ws,
+                lane=i % self.nl, out=lb["out"][:n].view(R, C), gin=lb["gin"][:n].view(R, C),
+                out_r=lb["out_r"][:n].view(R, C), mask=lb["mask"][:n // 32],
+                mask_r=lb["mask_r"][:n // 32]))
+        self.n = sum(w["xr"].numel() for w in self.work)
+        self.shapes = [list(w["xr"].shape) for w in self.work]
+        self.groups = [w["site"].num_groups for w in self.work]
+        self.resident_bytes = sum(3 * w["xr"].numel() * 2 for w in self.work)
+
+    def large(self) -> bool:
+        """Inputs far beyond L2 (a step streams many times the L2 through
+        it before any input comes round again): no flush between steps."""
+        return self.resident_bytes > 16 * L2_BYTES
+
+
+def one_site(w, e, d, s, s2):
+    """capture -> guided fwd -> STE bwd on stream s; the RTN comparator on s2
+    after the capture (its only input besides x_train), or on s after the
+    backward when s2 is None.  e / d: optional event lists for the
+    per-kernel breakdown and the dominant kernel."""
     from fp4_quantization_aware_trace_b200 import ops
-    ops.library()
+    if e: e[0].record(s)
+    ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], s)
+    if e: e[1].record(s)
+    if s2 is not None:
+        captured = torch.cuda.Event()
+        captured.record(s)
+        s2.wait_event(captured)
+        ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                       w["mask_r"], s2)
+    if d: d[0].record(s)
+    ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], s)
+    if d: d[1].record(s)
+    if e: e[2].record(s)
+    ops.fq_bwd(w["g"], w["mask"], w["gin"], s)
+    if e: e[3].record(s)
+    if s2 is None:
+        ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
+                       w["mask_r"], s)
+    if e: e[4].record(s)
 
-    workload, sites = make_workload(args.config, rank, dev)
-    work = []
-    for site in sites:
-        R, C = site.x_roll.shape
-        offs = None if site.offsets is None else site.offsets.to(dev)
-        cap, ws = ops.alloc_capture(R, C, site.num_groups, dev, offs)
-        w = dict(site=site, xr=site.x_roll.contiguous(), xt=site.x_train.contiguous(),
-                 g=site.grad.contiguous(), offs=offs, cap=cap, ws=ws,
-                 out=torch.empty_like(site.x_train), gin=torch.empty_like(site.grad),
-                 out_r=torch.empty_like(site.x_train),
-                 mask=torch.empty(R * C // 32, dtype=torch.int32, device=dev),
-                 mask_r=torch.empty(R * C // 32, dtype=torch.int32, device=dev))
-        work.append(w)
-    n = sum(w["xr"].numel() for w in work)
-    groups = [w["site"].num_groups for w in work]
-    shapes = [list(w["xr"].shape) for w in work]
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+def run_step(work, stream, ev=None, dom=None, s=None, s2=None, lanes=None):
+    """One step over every site.  Sites run one after another on s, each with
+    its RTN comparator on s2 when given; with lanes (a list of (main, side)
+    stream pairs) site i runs on lanes[i % len] instead -- the sites are
+    independent, and site i's output buffers belong to that lane.  Every
+    stream used joins s at the end."""
+    s = stream if s is None else s
+    if lanes:
+        for m, sd in lanes:
+            m.wait_stream(s)  # fork
+            if sd is not None:
+                sd.wait_stream(s)
+        for w in work:
+            m, sd = lanes[w["lane"] % len(lanes)]
+            one_site(w, None, None, m, sd)
+        for m, sd in lanes:
+            s.wait_stream(m)  # join
+            if sd is not None:
+                s.wait_stream(sd)
+        return
+    if s2 is not None:
+        s2.wait_stream(s)
+    for i, w in enumerate(work):
+        one_site(w, ev[i] if ev else None, dom[i] if dom else None, s, s2)
+    if s2 is not None:
+        s.wait_stream(s2)
+
+
+def measure_step(args, wl: Workload, pg, dev, clk, flush):
+    """Time the step over a resident workload: (1) graph-replayed steps (the
+    value), (2) the same steps as separate launches with events around the
+    dominant kernel (the roofline), (3) an untimed pass with events between
+    every call (the per-kernel breakdown).  Returns a dict of max-over-rank
+    milliseconds."""
+    work = wl.work
     stream = torch.cuda.current_stream()
+    do_flush = not wl.large()
 
-    def one_site(w, e, d, s, s2):
-        """capture -> guided fwd -> STE bwd on stream s; the RTN comparator on
-        s2 after the capture (its only input besides x_train), or on s after
-        the backward when s2 is None.  e / d: optional event lists for the
-        per-kernel breakdown and the dominant kernel."""
-        if e: e[0].record(s)
-        ops.capture(w["xr"], w["offs"], w["cap"], w["ws"], s)
-        if e: e[1].record(s)
-        if s2 is not None:
-            captured = torch.cuda.Event()
-            captured.record(s)
-            s2.wait_event(captured)
-            ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
-                           w["mask_r"], s2)
-        if d: d[0].record(s)
-        ops.guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], s)
-        if e: e[2].record(s)
-        if d: d[1].record(s)
-        ops.fq_bwd(w["g"], w["mask"], w["gin"], s)
-        if e: e[3].record(s)
-        if s2 is None:
-            ops.rtn_fq_fwd(w["xt"], w["cap"].scales, w["cap"].gscale, w["offs"], w["out_r"],
-                           w["mask_r"], s)
-        if e: e[4].record(s)
-
-    def step(ev=None, dom=None, s=None, s2=None, lanes=None):
-        """One step over every site.  Sites run one after another on s, each
-        with its RTN comparator on s2 when given; with lanes (a list of (main,
-        side) stream pairs) site i runs on lanes[i % len] instead, since the
-        sites are independent.  Every stream used joins s at the end."""
-        s = stream if s is None else s
-        if lanes:
-            for m, sd in lanes:
-                m.wait_stream(s)  # fork
-                if sd is not None:
-                    sd.wait_stream(s)
-            for i, w in enumerate(work):
-                m, sd = lanes[i % len(lanes)]
-                one_site(w, None, None, m, sd)
-            for m, sd in lanes:
-                s.wait_stream(m)  # join
-                if sd is not None:
-                    s.wait_stream(sd)
-            return
-        if s2 is not None:
-            s2.wait_stream(s)
-        for i, w in enumerate(work):
-            one_site(w, ev[i] if ev else None, dom[i] if dom else None, s, s2)
-        if s2 is not None:
-            s.wait_stream(s2)
+    def flush_l2(k):
+        if do_flush:
+            flush.fill_(k & 0xFF)
 
     for i in range(max(args.warmup, 3)):
-        flush.fill_(i & 0xFF)
-        step()
+        flush_l2(i)
+        run_step(work, stream)
     torch.cuda.synchronize()
 
-    # the step captured once as a CUDA graph (all sites, every kernel of the
-    # path) and replayed per step: one graph launch instead of 6 launches per
-    # site, and no per-launch submission gap between the kernels
     gph, graph_error = None, None
+    nl = wl.nl
     if not args.eager:
         try:
             gph = torch.cuda.CUDAGraph()
             cs = torch.cuda.Stream()
             cs.wait_stream(stream)
             side = None if args.one_stream else torch.cuda.Stream()
-            nl = min(max(args.lanes, 1), len(work))
             lanes = ([(torch.cuda.Stream(), None if args.one_stream else torch.cuda.Stream())
                       for _ in range(nl)] if nl > 1 else None)
             # thread-local: other threads' CUDA calls (e.g. a process group's
             # watchdog) must not invalidate the capture
             with torch.cuda.graph(gph, stream=cs, capture_error_mode="thread_local"):
                 if lanes:
-                    step(s=cs, lanes=lanes)
+                    run_step(work, stream, s=cs, lanes=lanes)
                 else:
-                    step(s=cs, s2=side)
+                    run_step(work, stream, s=cs, s2=side)
             torch.cuda.synchronize()
             for _ in range(max(args.warmup, 3)):
                 gph.replay()
@@ -424,301 +575,106 @@ def run_trace(args):
         except Exception as exc:  # fall back to separate launches, and say so
             gph, graph_error = None, f"{type(exc).__name__}: {exc}"[:200]
 
-    # timed region: one event pair around every step (nothing between the
-    # kernels, so each launch can overlap the tail of the previous one)
-    step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-    # the dominant kernel (guided forward) is also bracketed inside the timed
-    # steps, for the roofline's achieved bandwidth
-    dom_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in work] for _ in range(args.steps)]
-    # per-kernel breakdown: events between the calls (which can delay the
-    # next launch a little, so these durations are slightly pessimistic)
-    kern_ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
-               for _ in range(args.steps)]
-    eager_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
-    with ClockSampler(local) as clk:
+    K = args.steps
+    step_ev = [_pair() for _ in range(K)]
+    dom_ev = [[_pair() for _ in work] for _ in range(K)]
+    kern_ev = [[[_ev() for _ in range(5)] for _ in work] for _ in range(K)]
+    eager_ev = [_pair() for _ in range(K)]
+    with clk:
         # timed region 1 (the value): the step, graph-replayed (or eager)
         if pg: pg.barrier()
         torch.cuda.synchronize()
-        for k in range(args.steps):
-            flush.fill_((k + 7) & 0xFF)
+        for k in range(K):
+            flush_l2(k + 7)
             step_ev[k][0].record(stream)
             if gph is not None:
                 gph.replay()
             else:
-                step(dom=dom_ev[k])
+                run_step(work, stream, dom=dom_ev[k])
             step_ev[k][1].record(stream)
         torch.cuda.synchronize()
         if pg: pg.barrier()
-        # timed region 2: the same step as separate launches, with the
+        # timed region 2: the same steps as separate launches, with the
         # dominant kernel bracketed by events on its stream (the roofline)
         if gph is not None:
             if pg: pg.barrier()
             torch.cuda.synchronize()
-            for k in range(args.steps):
-                flush.fill_((k + 5) & 0xFF)
+            for k in range(K):
+                flush_l2(k + 5)
                 eager_ev[k][0].record(stream)
-                step(dom=dom_ev[k])
+                run_step(work, stream, dom=dom_ev[k])
                 eager_ev[k][1].record(stream)
             torch.cuda.synchronize()
             if pg: pg.barrier()
-    clocks = clk.summary()
     if gph is not None:
         del gph
-    for k in range(args.steps):          # breakdown pass, outside the timed region
-        flush.fill_((k + 11) & 0xFF)
-        step(kern_ev[k])
+    for k in range(K):  # breakdown pass, outside the timed region
+        flush_l2(k + 11)
+        run_step(work, stream, ev=kern_ev[k])
     torch.cuda.synchronize()
-
-    # the next row built beyond the step: full-information guidance (the
-    # cache keeps the rollout's whole codes), timed alone the same way
-    full_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in work] for _ in range(args.steps)]
-    for w in work:  # untimed: the first launch of a kernel also loads it
-        ops.full_guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], stream)
-    for k in range(args.steps):
-        flush.fill_((k + 13) & 0xFF)
-        for i, w in enumerate(work):
-            full_ev[k][i][0].record(stream)
-            ops.full_guided_fq_fwd(w["xt"], w["cap"], w["out"], w["mask"], stream)
-            full_ev[k][i][1].record(stream)
-    torch.cuda.synchronize()
-    full_ms = max_over_ranks([sum(a.elapsed_time(b) for per in full_ev for a, b in per)], pg, dev)[0]
-
-    # the mismatch diagnostic (ladder distance of RTN / 1-bit guided / full
-    # guided codes from the rollout's), one histogram over all sites
-    hist = torch.zeros(3, 15, dtype=torch.int64, device=dev)
-    hist_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in work] for _ in range(args.steps)]
-    for w in work:  # untimed warm-up launch
-        ops.mismatch_histogram(w["xt"], w["cap"], hist, stream)
-    for k in range(args.steps):
-        flush.fill_((k + 29) & 0xFF)
-        hist.zero_()
-        for i, w in enumerate(work):
-            hist_ev[k][i][0].record(stream)
-            ops.mismatch_histogram(w["xt"], w["cap"], hist, stream)
-            hist_ev[k][i][1].record(stream)
-    torch.cuda.synchronize()
-    hist_ms = max_over_ranks([sum(a.elapsed_time(b) for per in hist_ev for a, b in per)], pg, dev)[0]
-    hist_counts = hist.cpu().tolist()
-
-    # the cache tier: every site's compact cache captured into one record and
-    # copied to pinned host memory on a copy stream while the compute stream
-    # goes on; timed from the first capture to the end of the last copy
-    from fp4_quantization_aware_trace_b200 import cache_tier
-    # one device record per site: a smaller ring throttles the captures to
-    # the copy engine (its back-pressure), which is not what is timed here
-    tier = cache_tier.CacheTier(num_layers=1, keep=1, device=dev, ring=len(work))
-    for i, w in enumerate(work):  # untimed: allocates records and host buffers
-        tier.capture(("site", i), 0, w["xr"], w["offs"], w["cap"].codes, stream)
-    torch.cuda.synchronize()
-    tier_ev = []
-    for k in range(args.steps):
-        # each step starts with an idle copy engine (no backlog from the last)
-        torch.cuda.synchronize()
-        flush.fill_((k + 41) & 0xFF)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
-        ev[0].record(stream)
-        for i, w in enumerate(work):
-            tier.capture(("site", i), 0, w["xr"], w["offs"], w["cap"].codes, stream)
-        ev[1].record(stream)
-        ev[2].record(tier.copy_stream)
-        tier_ev.append(ev)
-    torch.cuda.synchronize()
-    tier_compute_ms = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in tier_ev)], pg, dev)[0]
-    tier_total_ms = max_over_ranks([sum(e[0].elapsed_time(e[2]) for e in tier_ev)], pg, dev)[0]
-    rec_bytes = sum(cache_tier.RecordLayout.of(*w["xr"].shape, w["site"].num_groups).nbytes
-                    for w in work)
-    del tier
-
-    # the MXFP4 variant on the same sites: capture, 1-bit guided, RTN and
-    # full-guided forwards, each launch timed on its own
-    mxc = [ops.mx_capture(w["xr"], stream=stream) for w in work]
-    mx_hist = torch.zeros(3, 15, dtype=torch.int64, device=dev)
-
-    def mx_pass(evs):
-        for i, w in enumerate(work):
-            ev = evs[i] if evs is not None else None
-            if ev: ev[0].record(stream)
-            ops.mx_capture(w["xr"], mxc[i], stream)
-            if ev: ev[1].record(stream)
-            ops.mx_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
-            if ev: ev[2].record(stream)
-            ops.mx_rtn_fq_fwd(w["xt"], mxc[i].scales, w["out_r"], w["mask_r"], stream)
-            if ev: ev[3].record(stream)
-            ops.mx_full_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
-            if ev: ev[4].record(stream)
-            ops.mx_mismatch_histogram(w["xt"], mxc[i], mx_hist, stream)
-            if ev: ev[5].record(stream)
-
-    # capture and guided forward with the scales in the 128 x 4 tiled layout
-    # of a block-scaled FP4 GEMM
-    tcap = [ops.capture_tiled(w["xr"], w["offs"], stream) for w in work]
-    tws = [w["ws"] for w in work]
-
-    def tiled_pass(evs):
-        for i, w in enumerate(work):
-            R, C = w["xr"].shape
-            G = w["site"].num_groups
-            ev = evs[i] if evs is not None else None
-            if ev: ev[0].record(stream)
-            ops.trace_capture_ex(w["xr"], R, C, G, w["offs"], tcap[i].codes, tcap[i].mbits,
-                                 tcap[i].scales, tcap[i].gscale, tws[i], tws[i].numel(),
-                                 ops.TRACE_SCALES_TILED_128x4, stream)
-            if ev: ev[1].record(stream)
-            ops.fq_fwd_tiled(ops.TRACE_RULE_GUIDED, w["xt"], tcap[i], w["out"], w["mask"], stream)
-            if ev: ev[2].record(stream)
-
-    tiled_pass(None)
-    tl_ev = []
-    for k in range(args.steps):
-        flush.fill_((k + 67) & 0xFF)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in work]
-        tiled_pass(evs)
-        tl_ev.append(evs)
-    torch.cuda.synchronize()
-    tl_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in tl_ev for i in range(len(work)))
-             for j in range(2)]
-    tl_ms = max_over_ranks(tl_ms, pg, dev)
-
-    # W4A8 (E4M3 activations, MX scales) on the same sites
-    m8c = [ops.mx8_capture(w["xr"], stream=stream) for w in work]
-
-    def mx8_pass(evs):
-        for i, w in enumerate(work):
-            ev = evs[i] if evs is not None else None
-            if ev: ev[0].record(stream)
-            ops.mx8_capture(w["xr"], m8c[i], stream)
-            if ev: ev[1].record(stream)
-            ops.mx8_guided_fq_fwd(w["xt"], m8c[i], w["out"], w["mask"], stream)
-            if ev: ev[2].record(stream)
-            ops.mx8_rtn_fq_fwd(w["xt"], m8c[i].scales, w["out_r"], w["mask_r"], stream)
-            if ev: ev[3].record(stream)
-            ops.mx8_full_guided_fq_fwd(w["xt"], m8c[i], w["out"], w["mask"], stream)
-            if ev: ev[4].record(stream)
-
-    mx8_pass(None)
-    m8_ev = []
-    for k in range(args.steps):
-        flush.fill_((k + 97) & 0xFF)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in work]
-        mx8_pass(evs)
-        m8_ev.append(evs)
-    torch.cuda.synchronize()
-    m8_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in m8_ev for i in range(len(work)))
-             for j in range(4)]
-    m8_ms = max_over_ranks(m8_ms, pg, dev)
-    del m8c
-
-    mx_pass(None)  # untimed: first launches
-    mx_ev = []
-    for k in range(args.steps):
-        flush.fill_((k + 53) & 0xFF)
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in work]
-        mx_pass(evs)
-        mx_ev.append(evs)
-    torch.cuda.synchronize()
-    mx_ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in mx_ev for i in range(len(work)))
-             for j in range(5)]
-    mx_ms = max_over_ranks(mx_ms, pg, dev)
 
     names = ["capture", "guided_fwd", "ste_bwd", "rtn_fwd"]
+    total = sum(a.elapsed_time(b) for a, b in step_ev)
+    eager = (sum(a.elapsed_time(b) for a, b in eager_ev) if graph_error is None and not args.eager
+             else total)
+    dom = sum(a.elapsed_time(b) for per in dom_ev for a, b in per)
     per_kernel = {nm: 0.0 for nm in names}
-    total_ms = sum(a.elapsed_time(b) for a, b in step_ev)
-    eager_ms = (sum(a.elapsed_time(b) for a, b in eager_ev) if graph_error is None and not args.eager
-                else total_ms)
-    eager_ms = max_over_ranks([eager_ms], pg, dev)[0]
-    dom_ms = sum(a.elapsed_time(b) for per in dom_ev for a, b in per)
     for per in kern_ev:
-        for ev in per:
+        for e in per:
             for i, nm in enumerate(names):
-                per_kernel[nm] += ev[i].elapsed_time(ev[i + 1])
-    t_max = max_over_ranks([total_ms, dom_ms] + [per_kernel[nm] for nm in names], pg, dev)
-    total_ms, dom_ms = t_max[0], t_max[1]
-    per_kernel = {nm: t_max[i + 2] for i, nm in enumerate(names)}
+                per_kernel[nm] += e[i].elapsed_time(e[i + 1])
+    t = max_over_ranks([total, eager, dom] + [per_kernel[nm] for nm in names], pg, dev)
+    launch = (("CUDA graph of the whole step, captured once and replayed"
+               + ("" if args.one_stream else
+                  "; the RTN comparator on a second stream beside the guided forward and the "
+                  "backward")
+               + (f"; sites on {nl} stream lanes" if nl > 1 else ""))
+              if graph_error is None and not args.eager else
+              "separate launches (programmatic stream serialization)")
+    return {"total_ms": t[0], "eager_ms": t[1], "dom_ms": t[2],
+            "per_kernel_ms": {nm: t[3 + i] for i, nm in enumerate(names)},
+            "graph_error": graph_error, "launch": launch, "flushed": do_flush,
+            "timed_passes": 2 if graph_error is None and not args.eager else 1}
 
-    ms_step = total_ms / args.steps
-    bpe = sum(BYTES_PER_ELEM.values())
-    value = job_gbs(world, n, bpe, ms_step)
-    hbm, peak_kind = measured_peaks()
+
+def step_summary(args, wl: Workload, m, world, hbm, peak_kind):
+    """The step's value, per-kernel table and roofline from measure_step."""
+    K = args.steps
+    n = wl.n
+    ms_step = m["total_ms"] / K
+    value = job_gbs(world, n, STEP_BYTES_PER_ELEM, ms_step)
     kern = {}
-    for nm in names:
-        ms = per_kernel[nm] / args.steps
-        kern[nm] = {"kernel": KERNEL_NAMES[nm], "us": round(ms * 1e3, 2),
-                    "gbs": round(n * BYTES_PER_ELEM[nm] / (ms * 1e-3) / 1e9, 1),
-                    "elem_per_s": round(n / (ms * 1e-3), 1)}
-        kern[nm]["frac_of_hbm"] = round(kern[nm]["gbs"] / hbm, 4)
-    fms = full_ms / args.steps
-    next_rows = {"full_guided_fwd": {
-        "kernel": "k_fake_quant<kFull>", "us": round(fms * 1e3, 2),
-        "gbs": round(n * 4.6875 / (fms * 1e-3) / 1e9, 1),
-        "frac_of_hbm": round(n * 4.6875 / (fms * 1e-3) / 1e9 / hbm, 4),
-        "bytes_per_elem": 4.6875}}
-    hms = hist_ms / args.steps
-    tot = max(1, sum(hist_counts[0]))
-    next_rows["mismatch_histogram"] = {
-        "kernel": "k_mismatch_hist", "us": round(hms * 1e3, 2),
-        "gbs": round(n * 2.5625 / (hms * 1e-3) / 1e9, 1),
-        "frac_of_hbm": round(n * 2.5625 / (hms * 1e-3) / 1e9 / hbm, 4),
-        "bytes_per_elem": 2.5625,
-        "rules": list(ops.MISMATCH_RULES),
-        "disagree_frac": [round(1.0 - r[0] / tot, 6) for r in hist_counts],
-        "adjacent_frac_of_disagreements": [round(r[1] / max(1, tot - r[0]), 6) for r in hist_counts],
-        "counts": hist_counts}
-    mx_rows = {}
-    for j, (nm, kn, b_k) in enumerate([("capture", "k_mx_capture", 2.65625),
-                                       ("guided_fwd", "k_mx_fake_quant<1>", 4.28125),
-                                       ("rtn_fwd", "k_mx_fake_quant<0>", 4.15625),
-                                       ("full_guided_fwd", "k_mx_fake_quant<2>", 4.65625),
-                                       ("mismatch_histogram", "k_mismatch_hist<true>", 2.53125)]):
-        ms = mx_ms[j] / args.steps
-        mx_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": b_k,
-                       "gbs": round(n * b_k / (ms * 1e-3) / 1e9, 1),
-                       "frac_of_hbm": round(n * b_k / (ms * 1e-3) / 1e9 / hbm, 4)}
-    next_rows["mxfp4"] = mx_rows
-    m8_rows = {}
-    for j, (nm, kn, b_k) in enumerate([("capture", "k_mx8_capture", 3.15625),
-                                       ("guided_fwd", "k_mx8_fake_quant<1>", 4.28125),
-                                       ("rtn_fwd", "k_mx8_fake_quant<0>", 4.15625),
-                                       ("full_guided_fwd", "k_mx8_fake_quant<2>", 5.15625)]):
-        ms = m8_ms[j] / args.steps
-        m8_rows[nm] = {"kernel": kn, "us": round(ms * 1e3, 2), "bytes_per_elem": b_k,
-                       "gbs": round(n * b_k / (ms * 1e-3) / 1e9, 1),
-                       "frac_of_hbm": round(n * b_k / (ms * 1e-3) / 1e9 / hbm, 4)}
-    next_rows["w4a8"] = m8_rows
-    next_rows["tiled_scales"] = {
-        nm: {"kernel": kn, "us": round(tl_ms[j] / args.steps * 1e3, 2), "bytes_per_elem": b_k,
-             "gbs": round(n * b_k / (tl_ms[j] / args.steps * 1e-3) / 1e9, 1),
-             "frac_of_hbm": round(n * b_k / (tl_ms[j] / args.steps * 1e-3) / 1e9 / hbm, 4)}
-        for j, (nm, kn, b_k) in enumerate([("capture", "k_amax + k_capture<true>", 4.6875),
-                                           ("guided_fwd", "k_fake_quant<1, true>", 4.3125)])}
-    cms, tms = tier_compute_ms / args.steps, tier_total_ms / args.steps
-    next_rows["cache_tier"] = {
-        "what": "capture of every site into one compact record + one D2H copy per site to pinned "
-                "host memory on a copy stream",
-        "record_bytes_per_step": rec_bytes, "ring_slots": len(work),
-        "bits_per_elem": round(8 * rec_bytes / n, 4),
-        "capture_only_us": round(per_kernel["capture"] * 1e3 / args.steps, 2),
-        "compute_stream_us": round(cms * 1e3, 2),
-        "until_last_copy_us": round(tms * 1e3, 2),
-        "d2h_gbs": round(rec_bytes / (tms * 1e-3) / 1e9, 2)}
-    # dominant kernel: the guided forward (the largest single launch of the
-    # step), timed inside the timed steps
+    for nm, ms_tot in m["per_kernel_ms"].items():
+        ms = ms_tot / K
+        gbs = n * BYTES_PER_ELEM[nm] / (ms * 1e-3) / 1e9
+        kern[nm] = {"kernel": KERNEL_NAMES[nm], "us": round(ms * 1e3, 2), "gbs": round(gbs, 1),
+                    "elem_per_s": round(n / (ms * 1e-3), 1), "frac_of_hbm": round(gbs / hbm, 4)}
     dom = "guided_fwd"
-    dom_bytes = n * BYTES_PER_ELEM[dom]
-    dom_us = dom_ms / args.steps * 1e3
+    launches = len(wl.work)
+    dom_bytes = n * BYTES_PER_ELEM[dom] / launches          # per launch (average site)
+    dom_us = m["dom_ms"] / (K * launches) * 1e3              # average launch duration
     achieved = round(dom_bytes / (dom_us * 1e-6) / 1e9, 1)
-    traffic = traffic_from_profiles("k_fake_quant_guided")
+    roofline = {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
+                "us_per_launch": round(dom_us, 2), "launches_timed": K * launches,
+                "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(achieved / hbm, 4),
+                "traffic": traffic_from_profiles("k_fake_quant_guided", WORKLOAD_TAGS[wl.cfg]),
+                "algorithmic_bytes": int(dom_bytes)}
+    return {"value": value, "ms_per_step": ms_step,
+            "elem_per_s": world * n / (ms_step * 1e-3),
+            "algo_bytes_over_copy_peak": value / world / hbm,
+            "kernels": kern, "roofline": roofline,
+            "eager_ms_per_step": m["eager_ms"] / K}
 
-    # --- yardstick: the library's plain copy kernel on the same bytes -------
-    ny = max(w["xr"].numel() for w in work)
+
+def yardstick_leg(args, wl, pg, dev, flush):
+    """The library's plain copy kernel on the largest tensor of the workload."""
+    from fp4_quantization_aware_trace_b200 import ops
+    stream = torch.cuda.current_stream()
+    ny = max(w["xr"].numel() for w in wl.work)
     ysrc = torch.empty(ny, dtype=torch.bfloat16, device=dev).fill_(1.0)
     ydst = torch.empty_like(ysrc)
-    yev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    yev = [_pair() for _ in range(args.steps)]
     for i in range(3):
         flush.fill_(i)
         ops.trace_copy_bf16(ysrc, ydst, ny, stream)
@@ -729,53 +685,287 @@ def run_trace(args):
         yev[k][1].record(stream)
     torch.cuda.synchronize()
     y_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in yev) / args.steps], pg, dev)[0]
-    yardstick = {"kernel": "k_copy", "bytes": 4 * ny, "us": round(y_ms * 1e3, 2),
-                 "gbs": round(4 * ny / (y_ms * 1e-3) / 1e9, 1)}
-    del ysrc, ydst
+    return {"kernel": "k_copy", "bytes": 4 * ny, "us": round(y_ms * 1e3, 2),
+            "gbs": round(4 * ny / (y_ms * 1e-3) / 1e9, 1), "l2": "flushed before each launch"}
 
-    # --- end-to-end through the C ABI with pinned host buffers -------------
-    e2e = None
-    if not args.no_e2e and args.config == 2:
-        # through the public host-to-host API: inputs from pinned host memory,
-        # every output back to it, the copies overlapped with the kernels in
-        # row chunks (host_step.HostStep)
-        from fp4_quantization_aware_trace_b200 import host_step
-        hs = []
-        for w in work:
+
+def next_rows_leg(args, wl: Workload, pg, dev, flush, hbm):
+    """The rows built beyond the step, each timed alone over the first
+    `--next-sites` sites: full-information guidance, the mismatch
+    histogram, the cache tier, MXFP4, W4A8 and the tiled scale layout."""
+    from fp4_quantization_aware_trace_b200 import cache_tier, ops
+    stream = torch.cuda.current_stream()
+    work = wl.work[:max(1, args.next_sites)]
+    K = args.steps
+    n = sum(w["xr"].numel() for w in work)
+    caps = [ops.capture(w["xr"], w["offs"], stream=stream) for w in work]  # own codes per site
+
+    def rate(ms_total, b):
+        ms = ms_total / K
+        gbs = n * b / (ms * 1e-3) / 1e9
+        return {"us": round(ms * 1e3, 2), "bytes_per_elem": b, "gbs": round(gbs, 1),
+                "frac_of_hbm": round(gbs / hbm, 4)}
+
+    def timed(fn, nev, seed):
+        fn(None)  # untimed: first launches
+        evs_all = []
+        for k in range(K):
+            flush.fill_((k + seed) & 0xFF)
+            evs = [[_ev() for _ in range(nev)] for _ in work]
+            fn(evs)
+            evs_all.append(evs)
+        torch.cuda.synchronize()
+        ms = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for evs in evs_all
+                  for i in range(len(work))) for j in range(nev - 1)]
+        return max_over_ranks(ms, pg, dev)
+
+    def full_pass(evs):
+        for i, w in enumerate(work):
+            if evs: evs[i][0].record(stream)
+            ops.full_guided_fq_fwd(w["xt"], caps[i], w["out"], w["mask"], stream)
+            if evs: evs[i][1].record(stream)
+
+    rows = {"sites": len(work)}
+    rows["full_guided_fwd"] = dict(kernel="k_fake_quant<kFull>",
+                                   **rate(timed(full_pass, 2, 13)[0], 4.6875))
+
+    hist = torch.zeros(3, 15, dtype=torch.int64, device=dev)
+
+    def hist_pass(evs):
+        hist.zero_()
+        for i, w in enumerate(work):
+            if evs: evs[i][0].record(stream)
+            ops.mismatch_histogram(w["xt"], caps[i], hist, stream)
+            if evs: evs[i][1].record(stream)
+
+    hr = rate(timed(hist_pass, 2, 29)[0], 2.5625)
+    counts = hist.cpu().tolist()
+    tot = max(1, sum(counts[0]))
+    rows["mismatch_histogram"] = dict(
+        kernel="k_mismatch_hist", **hr, rules=list(ops.MISMATCH_RULES),
+        disagree_frac=[round(1.0 - r[0] / tot, 6) for r in counts],
+        adjacent_frac_of_disagreements=[round(r[1] / max(1, tot - r[0]), 6) for r in counts],
+        counts=counts)
+
+    # the cache tier: every site's compact cache captured into one record and
+    # copied to pinned host memory on a copy stream while the compute stream
+    # goes on; timed from the first capture to the end of the last copy
+    tier = cache_tier.CacheTier(num_layers=1, keep=1, device=dev, ring=len(work))
+    for i, w in enumerate(work):  # untimed: allocates records and host buffers
+        tier.capture(("site", i), 0, w["xr"], w["offs"], caps[i].codes, stream)
+    torch.cuda.synchronize()
+    tier_ev = []
+    for k in range(K):
+        torch.cuda.synchronize()  # each step starts with an idle copy engine
+        flush.fill_((k + 41) & 0xFF)
+        ev = [_ev() for _ in range(3)]
+        ev[0].record(stream)
+        for i, w in enumerate(work):
+            tier.capture(("site", i), 0, w["xr"], w["offs"], caps[i].codes, stream)
+        ev[1].record(stream)
+        ev[2].record(tier.copy_stream)
+        tier_ev.append(ev)
+    torch.cuda.synchronize()
+    t_c, t_t = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in tier_ev),
+                               sum(e[0].elapsed_time(e[2]) for e in tier_ev)], pg, dev)
+    rec_bytes = sum(cache_tier.RecordLayout.of(*w["xr"].shape, w["site"].num_groups).nbytes
+                    for w in work)
+    del tier
+    rows["cache_tier"] = {
+        "what": "capture of every site into one compact record + one D2H copy per site to "
+                "pinned host memory on a copy stream",
+        "record_bytes_per_step": rec_bytes, "ring_slots": len(work),
+        "bits_per_elem": round(8 * rec_bytes / n, 4),
+        "compute_stream_us": round(t_c / K * 1e3, 2),
+        "until_last_copy_us": round(t_t / K * 1e3, 2),
+        "d2h_gbs": round(rec_bytes / (t_t / K * 1e-3) / 1e9, 2)}
+
+    # capture and guided forward with the scales in the 128 x 4 tiled layout
+    tcap = [ops.capture_tiled(w["xr"], w["offs"], stream) for w in work]
+
+    def tiled_pass(evs):
+        for i, w in enumerate(work):
             R, C = w["xr"].shape
+            G = w["site"].num_groups
+            if evs: evs[i][0].record(stream)
+            ops.trace_capture_ex(w["xr"], R, C, G, w["offs"], tcap[i].codes, tcap[i].mbits,
+                                 tcap[i].scales, tcap[i].gscale, w["ws"], w["ws"].numel(),
+                                 ops.TRACE_SCALES_TILED_128x4, stream)
+            if evs: evs[i][1].record(stream)
+            ops.fq_fwd_tiled(ops.TRACE_RULE_GUIDED, w["xt"], tcap[i], w["out"], w["mask"], stream)
+            if evs: evs[i][2].record(stream)
+
+    tl = timed(tiled_pass, 3, 67)
+    rows["tiled_scales"] = {
+        "capture": dict(kernel="k_amax + k_capture<true>", **rate(tl[0], 4.6875)),
+        "guided_fwd": dict(kernel="k_fake_quant<1, true>", **rate(tl[1], 4.3125))}
+    del tcap
+
+    # W4A8 (E4M3 activations, MX scales)
+    m8c = [ops.mx8_capture(w["xr"], stream=stream) for w in work]
+
+    def mx8_pass(evs):
+        for i, w in enumerate(work):
+            if evs: evs[i][0].record(stream)
+            ops.mx8_capture(w["xr"], m8c[i], stream)
+            if evs: evs[i][1].record(stream)
+            ops.mx8_guided_fq_fwd(w["xt"], m8c[i], w["out"], w["mask"], stream)
+            if evs: evs[i][2].record(stream)
+            ops.mx8_rtn_fq_fwd(w["xt"], m8c[i].scales, w["out_r"], w["mask_r"], stream)
+            if evs: evs[i][3].record(stream)
+            ops.mx8_full_guided_fq_fwd(w["xt"], m8c[i], w["out"], w["mask"], stream)
+            if evs: evs[i][4].record(stream)
+
+    m8 = timed(mx8_pass, 5, 97)
+    rows["w4a8"] = {nm: dict(kernel=kn, **rate(m8[j], b)) for j, (nm, kn, b) in enumerate(
+        [("capture", "k_mx8_capture", 3.15625), ("guided_fwd", "k_mx8_fake_quant<1>", 4.28125),
+         ("rtn_fwd", "k_mx8_fake_quant<0>", 4.15625),
+         ("full_guided_fwd", "k_mx8_fake_quant<2>", 5.15625)])}
+    del m8c
+
+    # MXFP4 (W4A4, E8M0 scales, 32-element blocks)
+    mxc = [ops.mx_capture(w["xr"], stream=stream) for w in work]
+    mx_hist = torch.zeros(3, 15, dtype=torch.int64, device=dev)
+
+    def mx_pass(evs):
+        for i, w in enumerate(work):
+            if evs: evs[i][0].record(stream)
+            ops.mx_capture(w["xr"], mxc[i], stream)
+            if evs: evs[i][1].record(stream)
+            ops.mx_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
+            if evs: evs[i][2].record(stream)
+            ops.mx_rtn_fq_fwd(w["xt"], mxc[i].scales, w["out_r"], w["mask_r"], stream)
+            if evs: evs[i][3].record(stream)
+            ops.mx_full_guided_fq_fwd(w["xt"], mxc[i], w["out"], w["mask"], stream)
+            if evs: evs[i][4].record(stream)
+            ops.mx_mismatch_histogram(w["xt"], mxc[i], mx_hist, stream)
+            if evs: evs[i][5].record(stream)
+
+    mx = timed(mx_pass, 6, 53)
+    rows["mxfp4"] = {nm: dict(kernel=kn, **rate(mx[j], b)) for j, (nm, kn, b) in enumerate(
+        [("capture", "k_mx_capture", 2.65625), ("guided_fwd", "k_mx_fake_quant<1>", 4.28125),
+         ("rtn_fwd", "k_mx_fake_quant<0>", 4.15625),
+         ("full_guided_fwd", "k_mx_fake_quant<2>", 4.65625),
+         ("mismatch_histogram", "k_mismatch_hist<true>", 2.53125)])}
+    del mxc, caps
+    torch.cuda.synchronize()
+    return rows
+
+
+def e2e_leg(args, wl: Workload, pg, dev, world):
+    """The step end to end through the public host-to-host API
+    (host_step.HostStep): every site's x_roll, x_train and grad go up from
+    pinned host memory and every output comes back to it, the copies
+    overlapped with the kernels in row chunks.  A pinned input set is filled
+    from the site's resident tensors before its timed segment (untimed); each
+    e2e step covers every site, and the segments' device times add up."""
+    from fp4_quantization_aware_trace_b200 import host_step
+    stream = torch.cuda.current_stream()
+    hs = {}
+    for w in wl.work:
+        R, C = w["xr"].shape
+        key = (R, C, None if w["offs"] is None else tuple(w["offs"].cpu().tolist()))
+        if key not in hs:
             offs_h = None if w["offs"] is None else w["offs"].cpu()
             h = host_step.HostStep(R, C, offs_h, chunks=args.e2e_chunks, device=dev)
-            hs.append((h, [w[k].cpu().pin_memory() for k in ("xr", "xt", "g")], h.alloc_host()))
-        ins = [t for _, i, _ in hs for t in i]
-        outs = [t for _, _, o in hs for t in o.values()]
+            hs[key] = (h, [torch.empty((R, C), dtype=torch.bfloat16, pin_memory=True)
+                           for _ in range(3)], h.alloc_host())
+        w["e2e_key"] = key
 
-        def e2e_step():
-            for h, (xr_h, xt_h, g_h), out_h in hs:
-                h.run(xr_h, xt_h, g_h, out_h, stream)
+    def segment(w, ev):
+        h, ins, outs = hs[w["e2e_key"]]
+        for dst, src in zip(ins, (w["xr"], w["xt"], w["g"])):
+            dst.copy_(src)  # untimed: fill the pinned inputs (synchronous)
+        if ev: ev[0].record(stream)
+        h.run(ins[0], ins[1], ins[2], outs, stream)
+        if ev: ev[1].record(stream)
+        return h, ins, outs
 
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if pg: pg.barrier()
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms = max_over_ranks([e0.elapsed_time(e1)], pg, dev)[0] / args.steps
-        h2d = sum(t.numel() * t.element_size() for t in ins)
-        d2h = sum(t.numel() * t.element_size() for t in outs)
-        e2e = {"value": round(job_gbs(world, n, bpe, e2e_ms), 3), "unit": "GB/s",
-               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "api": f"host_step.HostStep.run, {len(hs[0][0].cuts)} row chunks",
-               "elem_per_s": round(world * n / (e2e_ms * 1e-3), 1)}
+    segment(wl.work[0], None)  # untimed: first launches, host buffers touched
+    torch.cuda.synchronize()
+    steps = max(1, args.e2e_steps)
+    evs = []
+    if pg: pg.barrier()
+    h2d = d2h = 0
+    for _ in range(steps):
+        for w in wl.work:
+            ev = _pair()
+            h, ins, outs = segment(w, ev)
+            evs.append(ev)
+            if _ == 0:
+                h2d += sum(t.numel() * t.element_size() for t in ins)
+                d2h += sum(t.numel() * t.element_size() for t in outs.values())
+    torch.cuda.synchronize()
+    if pg: pg.barrier()
+    ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in evs)], pg, dev)[0] / steps
+    chunks = {len(h.cuts) for h, _, _ in hs.values()}
+    return {"value": round(job_gbs(world, wl.n, STEP_BYTES_PER_ELEM, ms), 3), "unit": "GB/s",
+            "ms_per_step": round(ms, 3), "steps": steps,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "api": f"host_step.HostStep.run per site, {sorted(chunks)} row chunks",
+            "elem_per_s": round(world * wl.n / (ms * 1e-3), 1),
+            "timing": "events around each site's host-to-host step, summed over the sites; "
+                      "the pinned inputs are filled before each segment, outside it"}
 
+
+def run_trace(args):
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the library has no CPU path)")
+    if args.gpus != world:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch one process per GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+        pg = dist
+
+    from fp4_quantization_aware_trace_b200 import ops
+    ops.library()
+    hbm, peak_kind = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    clk = ClockSampler(local)
+
+    wl = Workload(args.config, rank, dev, args.lanes)
+    m = measure_step(args, wl, pg, dev, clk, flush)
+    head = step_summary(args, wl, m, world, hbm, peak_kind)
+    yard = yardstick_leg(args, wl, pg, dev, flush)
+    next_rows = next_rows_leg(args, wl, pg, dev, flush, hbm)
+    e2e = None if args.no_e2e else e2e_leg(args, wl, pg, dev, world)
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.config == 2:
-        gbs, eps, per, sample = cpu_oracle_rate(work[0]["site"], args.cpu_seconds)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
-               "sample": sample, "elem_per_s": round(eps, 1), "s_per_step": round(per, 3)}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_leg(args.config, [w["site"] for w in wl.work])
+    n_sites = len(wl.work)
+    config = {"workload": WORKLOAD_NAMES[args.config], "sites": n_sites, "shapes": wl.shapes
+              if n_sites <= 8 else [wl.shapes[0], f"x{n_sites}"], "groups": sorted(set(wl.groups)),
+              "step": "capture + guided fwd + STE bwd + RTN fwd",
+              "resident_input_bytes": wl.resident_bytes,
+              "l2": ("inputs far larger than L2 (each read from HBM once per step): no flush"
+                     if not m["flushed"] else "flushed before every step (256 MiB write)"),
+              "launch": m["launch"],
+              "parallelism": f"{world} GPU(s), each its own draw of the workload (no collective)"}
+    gpu_launches = LAUNCHES_PER_SITE * n_sites * args.steps * m["timed_passes"]
+    del wl
+    torch.cuda.empty_cache()
+
+    secondary = None
+    if not args.no_secondary and args.config == HEADLINE_CONFIG:
+        wl2 = Workload(SECONDARY_CONFIG, rank, dev, args.lanes)
+        m2 = measure_step(args, wl2, pg, dev, clk, flush)
+        s2 = step_summary(args, wl2, m2, world, hbm, peak_kind)
+        secondary = {"workload": WORKLOAD_NAMES[SECONDARY_CONFIG],
+                     "value": round(s2["value"], 3), "unit": "GB/s",
+                     "ms_per_step": round(s2["ms_per_step"], 5),
+                     "elem_per_s": round(s2["elem_per_s"], 1),
+                     "algo_bytes_over_copy_peak": round(s2["algo_bytes_over_copy_peak"], 4),
+                     "kernels": s2["kernels"], "roofline": s2["roofline"],
+                     "yardstick": yardstick_leg(args, wl2, pg, dev, flush),
+                     "l2": "flushed before every step (256 MiB write)", "launch": m2["launch"]}
+        gpu_launches += LAUNCHES_PER_SITE * len(wl2.work) * args.steps * m2["timed_passes"]
+        del wl2
 
     if pg:
         pg.barrier()
@@ -783,55 +973,73 @@ def run_trace(args):
     if rank != 0:
         return
     line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": round(ms_step, 5),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-        "data": "synthetic",
-        "elem_per_s": round(world * n / (ms_step * 1e-3), 1),
-        "frac_of_hbm": round(value / world / hbm, 4),
-        "config": {"workload": workload, "shapes": shapes, "groups": groups,
-                   "step": "capture + guided fwd + STE bwd + RTN fwd",
-                   "l2": "flushed before every step (256 MiB write)",
-                   "launch": (("CUDA graph of the whole step, captured once and replayed"
-                               + ("" if args.one_stream else
-                                  "; the RTN comparator on a second stream beside the guided "
-                                  "forward and the backward")
-                              + (f"; sites on {min(max(args.lanes, 1), len(work))} stream lanes"
-                                 if min(max(args.lanes, 1), len(work)) > 1 else ""))
-                              if graph_error is None and not args.eager else
-                              "separate launches (programmatic stream serialization)"),
-                   "parallelism": f"{world} independent sites, one per GPU (no collective)"},
-        "kernels": kern,
-        "yardstick": yardstick,
-        "next_rows": next_rows,
-        "roofline": {"bound": "hbm", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
-                     "us_per_launch": round(dom_us, 2),
-                     "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": traffic,
-                     "algorithmic_bytes": int(dom_bytes)},
+        "metric": METRIC, "value": round(head["value"], 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": round(head["ms_per_step"], 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "elem_per_s": round(head["elem_per_s"], 1),
+        "algo_bytes_over_copy_peak": round(head["algo_bytes_over_copy_peak"], 4),
+        "config": config,
+        "kernels": head["kernels"],
+        "roofline": head["roofline"],
+        "yardstick": yard,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        # the graph replays launch the same kernels as separate steps do;
-        # with the graph there is also the eager pass for the roofline
-        "gpu_launches": LAUNCHES_PER_STEP * len(work) * args.steps *
-                        (2 if graph_error is None and not args.eager else 1),
-        "eager_ms_per_step": round(eager_ms / args.steps, 5),
-        "graph_error": graph_error,
+        "gpu_launches": gpu_launches,
+        "eager_ms_per_step": round(head["eager_ms_per_step"], 5),
+        "graph_error": m["graph_error"],
+        "secondary": secondary,
+        "next_rows": next_rows,
         "timing": ("value: events around each step (graph replay) only; roofline: events around "
-                   "the guided forward in a second timed pass of eager steps; kernels: a third, "
-                   "untimed pass with events between the calls"),
-        "clocks": clocks,
+                   "every guided-forward launch in a second timed pass of eager steps, averaged "
+                   "over the launches; kernels: a third, untimed pass with events between the "
+                   "calls"),
+        "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
 
 
-def main():
-    args = parse()
-    if args.impl == "reference":
+def run_plumbing(args):
+    """The multi-rank plumbing alone, on CPU: every rank joins a gloo process
+    group (127.0.0.1), the per-rank values reduce to their max, and rank 0
+    prints what it saw."""
+    import datetime
+    import torch.distributed as dist
+    world, rank, local = dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=60))
+    try:
+        got = max_over_ranks([1.0 + rank, 10.0 - rank], dist if world > 1 else None, "cpu")
+        ranks = [torch.zeros(1) for _ in range(world)]
+        if world > 1:
+            dist.all_gather(ranks, torch.tensor([float(rank)]))
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps({"plumbing": True, "n_gpus": world, "ranks": [int(r) for r in ranks],
+                          "max_over_ranks": got,
+                          "master_addr": os.environ.get("MASTER_ADDR", "")}), flush=True)
+
+
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    args = parse(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        if args.impl == "reference" and not args.plumbing_only:
+            run_reference(args)  # one process: rank 0 alone runs the oracle
+            return 0
+        r = subprocess.run(rank_launch_cmd(argv, args.gpus, _free_port()))
+        return r.returncode
+    if args.plumbing_only:
+        run_plumbing(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_trace(args)
+    return 0
 
 
 if __name__ == "__main__":
-    main()
+    sys.exit(main())

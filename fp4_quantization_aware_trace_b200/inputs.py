@@ -140,12 +140,13 @@ LAYER_SWEEP_SITES = ("qkv_in", "o_in", "up_in", "down_in")
 
 
 def layer_sweep_site(layer: int, site: int, rows: int = 65536, cols: int = 4096,
-                     device="cpu") -> Site:
+                     device="cpu", seed_offset: int = 0) -> Site:
     """One site of the later-half-layer sweep (layers 20..39 of 40, four
     sites per layer, each [65536, 4096]): as the attention-input recipe,
-    seeded per (layer, site)."""
+    seeded per (layer, site); seed_offset gives another draw of the same
+    recipe (one per rank of a multi-GPU run)."""
     assert 0 <= site < len(LAYER_SWEEP_SITES)
-    return lognormal_site(1000 + 4 * layer + site, rows, cols, device=device,
+    return lognormal_site(1000 + 4 * layer + site + seed_offset, rows, cols, device=device,
                           name=f"L{layer}_{LAYER_SWEEP_SITES[site]}")
 
 

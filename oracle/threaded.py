@@ -160,3 +160,30 @@ def fq_bwd_mt(grad_out, mask, threads: int | None = None):
     if not parts:
         return np.zeros(shape, np.uint16)
     return np.concatenate(parts).reshape(shape)
+
+
+def capture_rows_mt(x, row_gscale, threads: int | None = None):
+    """oracle.capture_rows on row chunks (rows whose global scale is given
+    per row): (codes, mbits, scales)."""
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    threads = threads or cores()
+    rg = np.ascontiguousarray(row_gscale, dtype=np.float32)
+    parts = _map(lambda a, b: capture_rows(x[a:b], rg[a:b]), _chunks(rows, 4 * threads), threads)
+    return (np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts]),
+            np.concatenate([p[2] for p in parts]))
+
+
+def fake_quant_rows_mt(x, row_gscale, scales, mbits=None, threads: int | None = None):
+    """oracle.fake_quant_rows on row chunks: (out, mask); guided when mbits
+    is given, round to nearest otherwise."""
+    x = _as_bf16_bits(x)
+    rows, cols = x.shape
+    threads = threads or cores()
+    rg = np.ascontiguousarray(row_gscale, dtype=np.float32)
+    sc = np.ascontiguousarray(scales, dtype=np.uint8).reshape(rows, cols // 16)
+    mb = None if mbits is None else np.ascontiguousarray(mbits, np.uint32).reshape(rows, cols // 32)
+    parts = _map(lambda a, b: fake_quant_rows(x[a:b], rg[a:b], sc[a:b],
+                                              None if mb is None else mb[a:b]),
+                 _chunks(rows, 4 * threads), threads)
+    return np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts])

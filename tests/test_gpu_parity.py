@@ -79,8 +79,24 @@ def run_oracle(oracle_mod, site: inputs.Site):
                 grad_in=gin, out_rtn=out_r, mask_rtn=mask_r, out_full=out_f, mask_full=mask_f)
 
 
-def check_full(oracle_mod, site):
-    got, ref = run_gpu(site), run_oracle(oracle_mod, site)
+def run_oracle_mt(site: inputs.Site):
+    """run_oracle through the threaded driver (row chunks on every core):
+    the same results, for the largest tensors."""
+    import oracle.threaded as ot
+    xr, xt, g = inputs.bits(site.x_roll), inputs.bits(site.x_train), inputs.bits(site.grad)
+    G, offs = site.num_groups, _offs_np(site)
+    codes, mbits, scales, gscale = ot.capture_mt(xr, G, offs)
+    out, mask = ot.guided_fwd_mt(xt, mbits, scales, gscale, G, offs)
+    out_r, mask_r = ot.rtn_fwd_mt(xt, scales, gscale, G, offs)
+    out_f, mask_f = ot.full_guided_fwd_mt(xt, codes, scales, gscale, G, offs)
+    gin = ot.fq_bwd_mt(g, mask)
+    return dict(codes=codes, mbits=mbits, scales=scales, gscale=gscale, out=out, mask=mask,
+                grad_in=gin, out_rtn=out_r, mask_rtn=mask_r, out_full=out_f, mask_full=mask_f)
+
+
+def check_full(oracle_mod, site, threaded: bool = False):
+    got = run_gpu(site)
+    ref = run_oracle_mt(site) if threaded else run_oracle(oracle_mod, site)
     for k in ref:
         _eq(f"{site.name}.{k}", got[k], ref[k])
     return got, ref
@@ -341,15 +357,19 @@ def test_parity_cfg4_kv_cache_full(oracle_mod, which):
 
 
 @pytest.mark.parametrize("cols,name", [(2048, "expert_up_in"), (768, "expert_down_in")])
-def test_parity_cfg3_moe_experts(oracle_mod, cols, name):
+def test_parity_cfg3_moe_experts_full(oracle_mod, cols, name):
     s = inputs.moe_experts(seed=2 if cols == 2048 else 12, cols=cols, device=DEV, name=name)
-    if cols == 768:
-        check_full(oracle_mod, s)
-    else:
-        check_sampled_rows(oracle_mod, s, _sample_rows(s.x_roll.shape[0], 256, 3))
+    check_full(oracle_mod, s, threaded=True)
 
 
-@pytest.mark.parametrize("layer,site", [(20, 0), (31, 2), (39, 3)])
+@pytest.mark.parametrize("layer,site", [(20, 0), (39, 3)])
+def test_parity_cfg5_layer_sweep_full(oracle_mod, layer, site):
+    """Two whole sites of the sweep ([65536, 4096], 268 M elements each),
+    every output compared element by element."""
+    check_full(oracle_mod, inputs.layer_sweep_site(layer, site, device=DEV), threaded=True)
+
+
+@pytest.mark.parametrize("layer,site", [(31, 2), (27, 1)])
 def test_parity_cfg5_layer_sweep_sampled(oracle_mod, layer, site):
     s = inputs.layer_sweep_site(layer, site, device=DEV)
     check_sampled_rows(oracle_mod, s, _sample_rows(s.x_roll.shape[0], 64, layer))
