@@ -59,9 +59,9 @@ BYTES_PER_ELEM = {"capture": 4.6875, "guided_fwd": 4.3125, "ste_bwd": 4.125, "rt
 STEP_BYTES_PER_ELEM = sum(BYTES_PER_ELEM.values())
 KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<1> (1-bit guided)",
                 "ste_bwd": "k_ste_bwd", "rtn_fwd": "k_fake_quant<0> (round to nearest)"}
-# kernels of the library launched per site and step: capture (zeroing of the
-# accumulators, amax pass, quantising pass), guided forward, backward, RTN
-LAUNCHES_PER_SITE = 6
+# kernels of the library launched per site and step: capture (amax pass,
+# quantising pass), guided forward, backward, RTN
+LAUNCHES_PER_SITE = 5
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 * 10 ** 6
@@ -110,6 +110,9 @@ def parse(argv=None):
     ap.add_argument("--next-sites", type=int, default=8,
                     help="sites of the workload the next-row legs (full guidance, "
                          "histogram, MXFP4, W4A8, tiled scales, cache tier) run on")
+    ap.add_argument("--sites", type=int, default=0,
+                    help="run only the first N sites of the workload (0: all; for profiling "
+                         "one site of the layer sweep)")
     ap.add_argument("--plumbing-only", action="store_true",
                     help="run only the multi-rank plumbing (launch, process group over gloo, "
                          "max over ranks) on CPU, without any GPU work; prints one JSON line")
@@ -431,12 +434,14 @@ class Workload:
     global scales); the FP4 codes and the forward / backward outputs live in
     one set of buffers per stream lane (sites on one lane run in order)."""
 
-    def __init__(self, cfg: int, rank: int, dev, lanes: int):
+    def __init__(self, cfg: int, rank: int, dev, lanes: int, max_sites: int = 0):
         from fp4_quantization_aware_trace_b200 import ops
         self.cfg, self.dev = cfg, dev
         self.sites = []
         for site in workload_sites(cfg, rank, dev):
             self.sites.append(site)
+            if max_sites and len(self.sites) >= max_sites:
+                break
         self.nl = max(1, min(lanes, len(self.sites)))
         nmax = max(s.x_roll.numel() for s in self.sites)
         i32, bf = torch.int32, torch.bfloat16
@@ -459,7 +464,7 @@ class Workload:
                               scales=torch.empty(R, C // 16, dtype=torch.uint8, device=dev),
                               gscale=torch.empty(G, dtype=torch.float32, device=dev),
                               offsets=offs)
-            ws = torch.empty(max(ops.trace_capture_workspace_bytes(R, C, G), 256),
+            ws = torch.zeros(max(ops.trace_capture_workspace_bytes(R, C, G), 256),
                              dtype=torch.uint8, device=dev)
             self.work.append(dict(
                 site=site, xr=site.x_roll, xt=site.x_train, g=site.grad, offs=offs, cap=cap, ws=ws,
@@ -929,7 +934,7 @@ def run_trace(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     clk = ClockSampler(local)
 
-    wl = Workload(args.config, rank, dev, args.lanes)
+    wl = Workload(args.config, rank, dev, args.lanes, args.sites)
     m = measure_step(args, wl, pg, dev, clk, flush)
     head = step_summary(args, wl, m, world, hbm, peak_kind)
     yard = yardstick_leg(args, wl, pg, dev, flush)
@@ -939,7 +944,10 @@ def run_trace(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_leg(args.config, [w["site"] for w in wl.work])
     n_sites = len(wl.work)
-    config = {"workload": WORKLOAD_NAMES[args.config], "sites": n_sites, "shapes": wl.shapes
+    name = WORKLOAD_NAMES[args.config]
+    if args.sites and n_sites < len(workload_shapes(args.config)):
+        name = f"the first {n_sites} site(s) of: {name}"
+    config = {"workload": name, "sites": n_sites, "shapes": wl.shapes
               if n_sites <= 8 else [wl.shapes[0], f"x{n_sites}"], "groups": sorted(set(wl.groups)),
               "step": "capture + guided fwd + STE bwd + RTN fwd",
               "resident_input_bytes": wl.resident_bytes,

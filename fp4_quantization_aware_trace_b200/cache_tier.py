@@ -132,7 +132,7 @@ class CacheTier:
         nb = max(ops.trace_capture_workspace_bytes(rows, cols, G), 256)
         ws = self._ws.get(nb)
         if ws is None:
-            ws = self._ws[nb] = torch.empty(nb, dtype=torch.uint8, device=self.device)
+            ws = self._ws[nb] = torch.zeros(nb, dtype=torch.uint8, device=self.device)
         return ws
 
     def capture(self, key: Hashable, layer: int, x: torch.Tensor,

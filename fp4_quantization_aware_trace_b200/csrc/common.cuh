@@ -188,6 +188,20 @@ __device__ __forceinline__ uint32_t rtn_e2m1x2_f16x2(float lo, float hi) {
   return r;
 }
 
+// As rtn_e2m1x2_f16x2, also returning the code byte (lo code in bits 0-3,
+// hi code in bits 4-7) in `code`.
+__device__ __forceinline__ uint32_t rtn_e2m1x2_f16x2_code(float lo, float hi, uint32_t& code) {
+  uint32_t r, c;
+  asm("{\n\t.reg .b8 b;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b, %2, %3;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b;\n\t"
+      "cvt.u32.u8 %1, b;\n\t}"
+      : "=r"(r), "=r"(c)
+      : "f"(hi), "f"(lo));
+  code = c;
+  return r;
+}
+
 // Byte of two E2M1 codes -> f16x2 (exact): lo code in the low half.
 __device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   uint32_t r;

@@ -106,34 +106,6 @@ __device__ __forceinline__ BlockCodes block_codes(const V8& v, const V8* src, fl
   return bc;
 }
 
-// The same codes for an MX block half: z = |x| * 2^-e is exact, so the grid
-// rounding runs on it directly (no quotient, no exact path).
-__device__ __forceinline__ BlockCodes mx_block_codes(const V8& v, u64 inv2) {
-  BlockCodes bc;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    float f[8], c[8], r[8];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const uint32_t w = v.w[4 * h + k];
-      const uint32_t wa = w & 0x7FFF7FFFu;
-      float zl, zh;
-      upk(mul2(pk(bf16_lo(wa), bf16_hi(wa)), inv2), zl, zh);  // inf only past 6
-      const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);
-      const u64 MM = pk(grid_magic(al), grid_magic(ah));
-      const u64 aa = pk(al, ah);
-      upk(sub2(add_rm2(aa, MM), MM), f[2 * k], f[2 * k + 1]);
-      upk(sub2(add_rp2(aa, MM), MM), c[2 * k], c[2 * k + 1]);
-      r[2 * k] = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
-      r[2 * k + 1] = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
-    }
-    bc.f[h] = cvt_e2m1x8(f);
-    bc.c[h] = cvt_e2m1x8(c);
-    bc.r[h] = cvt_e2m1x8(r);
-  }
-  return bc;
-}
-
 // Ladder distances of 8 nibbles: training magnitude codes t against the
 // rollout magnitudes qm (both 0..7); s15 is 0xF on nibbles where the two
 // signs agree.  Same sign: |t - qm|; opposite signs: t + qm.
@@ -176,8 +148,37 @@ __device__ __forceinline__ void hist_word(uint32_t f, uint32_t c, uint32_t r, ui
   count8(ladder_dist8(f + up, qm, s15), ones[2], bins + 2 * kHistBins);
 }
 
+// Floor, ceiling and signed round-to-nearest codes of one site on the exact
+// path, packed as f | c << 4 | r << 8: z = x / d (NVFP4) or x * 2^-e given
+// as inv (MX, exact).  Reads the site's bf16 input at src.
+__device__ __noinline__ uint32_t site_codes_exact(const uint16_t* src, float d, float inv, int mx) {
+  const uint32_t xb = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(src));
+  const float xf = __uint_as_float(xb << 16);
+  const Exact e = mx ? exact_of_z(__fmul_rn(xf, inv)) : exact_site(xf, d);
+  const uint32_t c = (uint32_t)(e.exact ? e.floor : e.floor + 1);
+  const uint32_t r = (((xb >> 15) & 1u) << 3) | (uint32_t)e.rtn;
+  return (uint32_t)e.floor | (c << 4) | (r << 8);
+}
+
+// Bit j (0-31) set where nibble j of the four words differs from zero.
+__device__ __forceinline__ uint32_t nibble_any4(uint4 w) {
+  w.x |= w.x >> 1; w.y |= w.y >> 1; w.z |= w.z >> 1; w.w |= w.w >> 1;
+  return nibble_lsbs4(make_uint4(w.x | (w.x >> 2), w.y | (w.y >> 2), w.z | (w.z >> 2),
+                                 w.w | (w.w >> 2)));
+}
+
 // MX: MXFP4 scales (one E8M0 byte per thread's pair of blocks, no groups)
 // instead of E4M3 block scales with global scales.
+//
+// Where the training side's round-to-nearest code (signed) equals the
+// rollout's, all three rules sit at distance 0: round to nearest by
+// definition, the 1-bit rule because that code's mantissa bit is the cached
+// bit (it keeps the bracket member carrying it), the full rule because the
+// rollout codeword is then in the bracket.  So the pass computes the signed
+// round-to-nearest codes as capture does, and only the sites whose code
+// differs from the rollout's -- rare for a drifted pair -- go through the
+// exact per-site codes and the three rules.  Zero blocks and blocks outside
+// the fast range take the whole-block path.
 template <bool MX>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mismatch_hist(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
@@ -199,32 +200,44 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (b >= sh.nblk) continue;
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     const uint4 rc = __ldcs(rcodes + (b >> 1));
-    BlockCodes k0, k1;
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
+    n += 32u;
+    float d0 = 0.0f, d1 = 0.0f, inv = 0.0f;
+    uint4 r;
     if (MX) {
-      const float inv = pow2f(127 - (int)__ldcs(scales + (b >> 1)));
+      inv = pow2f(127 - (int)__ldcs(scales + (b >> 1)));
       const u64 inv2 = pk(inv, inv);
-      k0 = mx_block_codes(v0, inv2);
-      k1 = mx_block_codes(v1, inv2);
+      mx_codes_block(v0, inv2, r.x, r.y);
+      mx_codes_block(v1, inv2, r.z, r.w);
     } else {
       const uint32_t sb2 = __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
       if (gc.seek(sh.G > 1 ? fastdiv(b, sh.bpr) : 0u)) s_g = __ldg(gscale + gc.g);
       float sbv0, sbv1;
       e4m3x2_to_f32(sb2, sbv0, sbv1);
-      const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
-      if (fast_scale(d0, kDMaxExactZ) && fast_scale(d1, kDMaxExactZ)) {
-        // the common case, without per-block branches
-        k0 = block_codes_fast(v0, d0);
-        k1 = block_codes_fast(v1, d1);
-      } else {
-        k0 = block_codes(v0, x + b, d0);
-        k1 = block_codes(v1, x + b + 1, d1);
+      d0 = __fmul_rn(s_g, sbv0);
+      d1 = __fmul_rn(s_g, sbv1);
+      if (!(fast_scale(d0) && fast_scale(d1))) {
+        // zero block or a scale outside the fast range: whole blocks
+        const BlockCodes k0 = block_codes(v0, x + b, d0), k1 = block_codes(v1, x + b + 1, d1);
+        hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
+        hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);
+        hist_word(k1.f[0], k1.c[0], k1.r[0], rc.z, ones, bins);
+        hist_word(k1.f[1], k1.c[1], k1.r[1], rc.w, ones, bins);
+        continue;
       }
+      codes_fast(v0, d0, r.x, r.y);
+      codes_fast(v1, d1, r.z, r.w);
     }
-    hist_word(k0.f[0], k0.c[0], k0.r[0], rc.x, ones, bins);
-    hist_word(k0.f[1], k0.c[1], k0.r[1], rc.y, ones, bins);
-    hist_word(k1.f[0], k1.c[0], k1.r[0], rc.z, ones, bins);
-    hist_word(k1.f[1], k1.c[1], k1.r[1], rc.w, ones, bins);
-    n += 32u;
+    uint32_t bad = nibble_any4(make_uint4(r.x ^ rc.x, r.y ^ rc.y, r.z ^ rc.z, r.w ^ rc.w));
+    while (bad != 0u) {
+      const int j = __ffs(bad) - 1;
+      bad &= bad - 1u;
+      const uint32_t q = ((j < 8 ? rc.x : j < 16 ? rc.y : j < 24 ? rc.z : rc.w) >> (4 * (j & 7))) & 0xFu;
+      const uint32_t fcr = site_codes_exact(src + j, j < 16 ? d0 : d1, inv, MX ? 1 : 0);
+      // one site in nibble 0; the other seven nibbles are all zero and count
+      // as distance 0
+      hist_word(fcr & 0xFu, (fcr >> 4) & 0xFu, fcr >> 8, q, ones, bins);
+    }
   }
 #pragma unroll
   for (int k = 0; k < kHistModes; ++k) ones[k] = __reduce_add_sync(0xFFFFFFFFu, ones[k]);

@@ -64,46 +64,79 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
-// Two elements of the MX fake-quant forward (side as fq_pair).
-template <int MODE>
-__device__ __forceinline__ uint32_t mx_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
-                                               uint32_t& m, int pos) {
-  float zl, zh;
-  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
-  m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
-  const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
-  float tl, th;  // chosen codeword value
-  if (MODE == kRtn) {
-    const uint32_t h2 = rtn_e2m1x2_f16x2(al, ah);
-    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-  } else {
-    const u64 MM = pk(grid_magic(al), grid_magic(ah));
-    const u64 aa = pk(al, ah);
-    float lol, loh, hil, hih;
-    upk(add_rm2(aa, MM), lol, loh);
-    upk(add_rp2(aa, MM), hil, hih);
-    if (MODE == kGuided) {
-      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
-      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
-      upk(sub2(pk(sl, sh), MM), tl, th);
+// One site of an MX guided forward recomputed one element at a time (mode
+// and side as site_exact): z = x * 2^-e is exact, the rule's code scaled
+// back by X = 2^e.  Reads the site's bf16 input at src, returns its output
+// bits.
+__device__ __noinline__ uint32_t mx_site_fix(const uint16_t* src, float inv, float X, uint32_t side,
+                                             int mode) {
+  const uint32_t xb = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(src));
+  const Exact e = exact_of_z(__fmul_rn(__uint_as_float(xb << 16), inv));
+  const int c = rule_code(e, xb, side, mode);
+  const uint32_t mag = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e2m1_value(c), X)));
+  return (xb & 0x8000u) | mag;
+}
+
+// Round to nearest over one 16-element half of an MX block (scale 2^e given
+// as inv2 = 2^-e and X2 = 2^e): bf16 outputs, mask bits at pos0..pos0+15 of
+// m, and the codes as rtn_block (KIND 0 none, 1 magnitudes, 2 signed with
+// x's sign).
+template <int KIND>
+__device__ __forceinline__ void mx_rtn_block(const V8& v, u64 inv2, u64 X2, V8& o, uint32_t& m,
+                                             int pos0, uint32_t& c0, uint32_t& c1) {
+  c0 = 0u;
+  c1 = 0u;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t w = v.w[p];
+    float zl, zh;
+    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
+    m |= (le_mask(fabsf(zl), 6.0f) & (1u << (pos0 + 2 * p))) |
+         (le_mask(fabsf(zh), 6.0f) & (2u << (pos0 + 2 * p)));
+    float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
+    uint32_t h2;
+    if (KIND == 0) {
+      h2 = rtn_e2m1x2_f16x2(al, ah);
     } else {
-      float fl, fh, cl, ch;
-      upk(sub2(pk(lol, loh), MM), fl, fh);
-      upk(sub2(pk(hil, hih), MM), cl, ch);
-      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
-      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
-      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
-      tl = rl > fl ? cl : fl;
-      th = rh > fh ? ch : fh;
+      if (KIND == 2) {
+        al = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
+        ah = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
+      }
+      uint32_t code;
+      h2 = rtn_e2m1x2_f16x2_code(al, ah, code);
+      if (p < 4) c0 |= code << (8 * p); else c1 |= code << (8 * (p - 4));
     }
+    const float tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    const float th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    float ql, qh;
+    upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+    o.w[p] = cvt_bf16x2(ql, qh) | (w & 0x80008000u);
   }
-  float ql, qh;
-  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
-  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+// One 16-element half of the MX fake-quant forward: round to nearest, then
+// (guided rules) the sites whose rule disagrees with it recomputed and
+// patched in, as fq_block_fast.  src: the half's inputs.
+template <int MODE>
+__device__ __forceinline__ void mx_fq_half(const V8& v, const uint16_t* src, uint32_t bits16,
+                                           uint32_t r0, uint32_t r1, float inv, float X, u64 inv2,
+                                           u64 X2, V8& o, uint32_t& m, int pos0) {
+  uint32_t c0, c1;
+  mx_rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, inv2, X2, o, m, pos0, c0, c1);
+  if (MODE == kRtn) return;
+  uint32_t bad = MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu
+                                 : nibble_any2(c0 ^ r0, c1 ^ r1);
+  while (bad != 0u) {
+    const int j = __ffs(bad) - 1;
+    bad &= bad - 1u;
+    const uint32_t side = MODE == kGuided ? (bits16 >> j) & 1u
+                                          : ((j < 8 ? r0 : r1) >> (4 * (j & 7))) & 0xFu;
+    const uint32_t val = mx_site_fix(src + j, inv, X, side, MODE);
+    const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k == (j >> 1)) o.w[k] = (o.w[k] & keep) | (val << sh);
+  }
 }
 
 template <int MODE, bool SW>
@@ -126,21 +159,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int e = (int)__ldcs(scales + so) - 127;
     const float inv = pow2f(-e), X = pow2f(e);
     const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
     uint32_t m = 0u;
     V8 o;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
-                          : MODE == kFull ? ((k < 4 ? rc.x : rc.y) >> (8 * (k & 3))) : 0u;
-      o.w[k] = mx_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
-    }
+    mx_fq_half<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, inv, X, inv2, X2, o, m, 0);
     st_block(out + b, o);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
-                          : MODE == kFull ? ((k < 4 ? rc.z : rc.w) >> (8 * (k & 3))) : 0u;
-      o.w[k] = mx_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
-    }
+    mx_fq_half<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, inv, X, inv2, X2, o, m, 16);
     st_block(out + b + 1, o);
     mask[b >> 1] = m;
   }
@@ -226,47 +250,90 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
-// Two elements of the W4A8 fake-quant forward.  side: kGuided -- the cached
-// bits in bits 0 and 1; kFull -- the two rollout code bytes (low first).
-template <int MODE>
-__device__ __forceinline__ uint32_t mx8_fq_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2,
-                                                uint32_t& m, int pos) {
-  float zl, zh;
-  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
-  m |= (le_mask(fabsf(zl), 448.0f) & (1u << pos)) | (le_mask(fabsf(zh), 448.0f) & (2u << pos));
-  const float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);
-  float tl, th;
-  if (MODE == kRtn) {
-    const uint32_t h2 = e4m3x2_to_f16x2(cvt_e4m3x2(al, ah));
-    tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+// One site of a W4A8 guided forward recomputed on its own (mode 1: side =
+// the cached bit; mode 2: side = the rollout's code byte): z = x * 2^-e is
+// exact; floor and ceiling on the E4M3 grid by directed rounding with the
+// grid addend; the rule's choice scaled back by X = 2^e.  Reads the site's
+// bf16 input at src, returns its output bits.
+__device__ __noinline__ uint32_t mx8_site_fix(const uint16_t* src, float inv, float X,
+                                              uint32_t side, int mode) {
+  const uint32_t xb = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(src));
+  const float z = __fmul_rn(__uint_as_float(xb << 16), inv);
+  const float a = fminf(fabsf(z), 448.0f);  // NaN (only past 448) -> 448
+  const float M = grid_magic8(a);
+  const float lo = __fadd_rd(a, M), hi = __fadd_ru(a, M);
+  float t;
+  if (mode == 1) {
+    // of floor / ceiling, the one whose mantissa bit is the cached bit
+    const uint32_t lb = __float_as_uint(lo);
+    t = __fsub_rn(__uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hi) - lb))), M);
   } else {
-    const u64 MM = pk(grid_magic8(al), grid_magic8(ah));
-    const u64 aa = pk(al, ah);
-    float lol, loh, hil, hih;
-    upk(add_rm2(aa, MM), lol, loh);
-    upk(add_rp2(aa, MM), hil, hih);
-    if (MODE == kGuided) {
-      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-      const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
-      const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
-      upk(sub2(pk(sl, sh), MM), tl, th);
-    } else {
-      float fl, fh, cl, ch;
-      upk(sub2(pk(lol, loh), MM), fl, fh);
-      upk(sub2(pk(hil, hih), MM), cl, ch);
-      const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFFFu);
-      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
-      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
-      tl = rl > fl ? cl : fl;
-      th = rh > fh ? ch : fh;
-    }
+    // of floor / ceiling, the one nearest the rollout value reflected to
+    // z's side of zero
+    const float f = __fsub_rn(lo, M), c = __fsub_rn(hi, M);
+    const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFu);
+    float r = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    r = __uint_as_float(__float_as_uint(r) ^ ((xb << 16) & 0x80000000u));
+    t = r > f ? c : f;
   }
-  float ql, qh;
-  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
-  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+  const uint32_t mag = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(t, X)));
+  return (xb & 0x8000u) | mag;
+}
+
+// One 16-element half of the W4A8 fake-quant forward: round to nearest on
+// the E4M3 grid (hardware conversion, ties to the even mantissa,
+// saturating at 448) with the STE mask, then, for the guided rules, the
+// sites whose rule disagrees with it recomputed and patched in, as
+// fq_block_fast: the 1-bit rule wherever the code's lowest bit is not the
+// cached bit, the full rule wherever the code (signed with x's sign) is not
+// the rollout's.  bits16: the cached bits; r: the rollout's 16 code bytes
+// of this half (4 words, element j in byte j).  src: the half's inputs.
+template <int MODE>
+__device__ __forceinline__ void mx8_fq_half(const V8& v, const uint16_t* src, uint32_t bits16,
+                                            uint4 r, float inv, float X, u64 inv2, u64 X2, V8& o,
+                                            uint32_t& m, int pos0) {
+  uint32_t bad = 0u;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t w = v.w[p];
+    float zl, zh;
+    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+    m |= (le_mask(fabsf(zl), 448.0f) & (1u << (pos0 + 2 * p))) |
+         (le_mask(fabsf(zh), 448.0f) & (2u << (pos0 + 2 * p)));
+    float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);  // NaN -> 448
+    if (MODE == kFull) {
+      al = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
+      ah = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
+    }
+    const uint32_t two = cvt_e4m3x2(al, ah);
+    if (MODE == kGuided) {
+      // lowest bits of the two codes (compared with the cached bits below)
+      bad |= ((two & 1u) | ((two >> 7) & 2u)) << (2 * p);
+    } else if (MODE == kFull) {
+      const uint32_t rw = (p & 2) ? (p & 4 ? r.w : r.y) : (p & 4 ? r.z : r.x);
+      const uint32_t dx = two ^ ((rw >> (16 * (p & 1))) & 0xFFFFu);
+      bad |= (((dx & 0xFFu) != 0u) | (((dx >> 8) != 0u) << 1)) << (2 * p);
+    }
+    const uint32_t h2 = e4m3x2_to_f16x2(two);
+    const float tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    const float th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    float ql, qh;
+    upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+    o.w[p] = cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+  }
+  if (MODE == kRtn) return;
+  if (MODE == kGuided) bad = (bad ^ bits16) & 0xFFFFu;
+  while (bad != 0u) {
+    const int j = __ffs(bad) - 1;
+    bad &= bad - 1u;
+    const uint32_t rw = j < 4 ? r.x : j < 8 ? r.y : j < 12 ? r.z : r.w;
+    const uint32_t side = MODE == kGuided ? (bits16 >> j) & 1u : (rw >> (8 * (j & 3))) & 0xFFu;
+    const uint32_t val = mx8_site_fix(src + j, inv, X, side, MODE);
+    const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      if (k == (j >> 1)) o.w[k] = (o.w[k] & keep) | (val << sh);
+  }
 }
 
 template <int MODE, bool SW>
@@ -289,21 +356,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int e = (int)__ldcs(scales + so) - 127;
     const float inv = pow2f(-e), X = pow2f(e);
     const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
     uint32_t m = 0u;
     V8 o;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (2 * k)
-                          : MODE == kFull ? rc.w[k >> 1] >> (16 * (k & 1)) : 0u;
-      o.w[k] = mx8_fq_pair<MODE>(v0.w[k], side, inv2, X2, m, 2 * k);
-    }
+    mx8_fq_half<MODE>(v0, src, bits & 0xFFFFu, make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]),
+                      inv, X, inv2, X2, o, m, 0);
     st_block(out + b, o);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t side = MODE == kGuided ? bits >> (16 + 2 * k)
-                          : MODE == kFull ? rc.w[4 + (k >> 1)] >> (16 * (k & 1)) : 0u;
-      o.w[k] = mx8_fq_pair<MODE>(v1.w[k], side, inv2, X2, m, 16 + 2 * k);
-    }
+    mx8_fq_half<MODE>(v1, src + 16, bits >> 16, make_uint4(rc.w[4], rc.w[5], rc.w[6], rc.w[7]),
+                      inv, X, inv2, X2, o, m, 16);
     st_block(out + b + 1, o);
     mask[b >> 1] = m;
   }

@@ -14,8 +14,8 @@ struct Exact {
   bool in;     // |z| <= 6 (STE mask)
 };
 
-__device__ __forceinline__ Exact exact_site(float xf, float d) {
-  const float z = (d == 0.0f) ? copysignf(0.0f, xf) : __fdiv_rn(xf, d);
+// The decisions of a site from its exact quotient z.
+__device__ __forceinline__ Exact exact_of_z(float z) {
   const float a = fabsf(z);
   Exact e;
   e.in = a <= 6.0f;
@@ -29,6 +29,11 @@ __device__ __forceinline__ Exact exact_site(float xf, float d) {
                 : (e.floor == 6) ? 4.0f : 6.0f;
   e.exact = (c == v);
   return e;
+}
+
+// The decisions of a site x with scale d (IEEE division; d = 0 gives +-0).
+__device__ __forceinline__ Exact exact_site(float xf, float d) {
+  return exact_of_z((d == 0.0f) ? copysignf(0.0f, xf) : __fdiv_rn(xf, d));
 }
 
 // E2M1 magnitude (as fp32) of a code 0..7.
@@ -55,9 +60,40 @@ __device__ __noinline__ uint2 capture_block_exact(const V8* src, float d) {
   return make_uint2(c[0], c[1]);
 }
 
+// Output bits (bf16 with x's sign) of one site on the exact path, for
+// `mode` 0 round to nearest, 1 guided by the cached bit `side`, 2 guided by
+// the rollout's signed 4-bit code `side` (full information: of floor and
+// ceiling, the one nearest the rollout value reflected to z's side of zero;
+// no codeword lies between them, so that is the ceiling exactly when the
+// value lies above the floor).  `in` receives the STE mask bit.
+// The code a rule picks at a site with decisions e (mode and side as
+// site_exact below; xb: the site's bf16 bits, for its sign).
+__device__ __forceinline__ int rule_code(const Exact& e, uint32_t xb, uint32_t side, int mode) {
+  int c = e.rtn;
+  if (mode == 1) {
+    c = e.exact ? e.floor : e.floor + ((e.floor ^ (int)(side & 1u)) & 1);
+  } else if (mode == 2) {
+    float q = e2m1_value((int)(side & 7u));
+    if (((side >> 3) & 1u) != ((xb >> 15) & 1u)) q = -q;
+    const int hi = e.exact ? e.floor : e.floor + 1;
+    c = (q > e2m1_value(e.floor)) ? hi : e.floor;
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint32_t site_exact(uint32_t xb, float d, float sbv, float s_g,
+                                               uint32_t side, int mode, bool& in) {
+  const Exact e = exact_site(__uint_as_float(xb << 16), d);
+  const int c = rule_code(e, xb, side, mode);
+  in = e.in;
+  const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
+      __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
+  return (xb & 0x8000u) | mag;
+}
+
 // Fake-quant of one block on the exact path: bf16 outputs and STE mask.
-// mode: 0 round-to-nearest, 1 1-bit guided (bits16), 2 full-information
-// guided (rollout codes c0: elements 0-7, c1: 8-15).
+// mode as site_exact; bits16: the cached bits (mode 1); c0, c1: the rollout
+// codes of elements 0-7 and 8-15 (mode 2).
 __device__ __noinline__ uint32_t fake_quant_block_exact(const V8* src, float d, float sbv, float s_g,
                                                     uint32_t bits16, uint32_t c0, uint32_t c1,
                                                     int mode, V8* dst) {
@@ -67,29 +103,25 @@ __device__ __noinline__ uint32_t fake_quant_block_exact(const V8* src, float d, 
   for (int k = 0; k < 8; ++k) o.w[k] = 0u;
   for (int j = 0; j < 16; ++j) {
     const uint32_t w = v.w[j >> 1];
-    const float xf = (j & 1) ? bf16_hi(w) : bf16_lo(w);
-    const Exact e = exact_site(xf, d);
-    int c = e.rtn;
-    if (mode == 1) {
-      const int bit = (int)((bits16 >> j) & 1u);
-      c = e.exact ? e.floor : e.floor + ((e.floor ^ bit) & 1);
-    } else if (mode == 2) {
-      // nearest of floor / ceiling to the rollout value on z's side of zero
-      const uint32_t rc = ((j < 8 ? c0 : c1) >> (4 * (j & 7))) & 0xFu;
-      float q = e2m1_value((int)(rc & 7u));
-      const bool neg_roll = (rc & 8u) != 0u, neg_z = ((w >> ((j & 1) ? 31 : 15)) & 1u) != 0u;
-      if (neg_roll != neg_z) q = -q;
-      const int hi = e.exact ? e.floor : e.floor + 1;
-      c = (q > e2m1_value(e.floor)) ? hi : e.floor;
-    }
-    const uint32_t mag = (uint32_t)__bfloat16_as_ushort(
-        __float2bfloat16_rn(__fmul_rn(__fmul_rn(e2m1_value(c), sbv), s_g)));
-    const uint32_t sg = (j & 1) ? (w >> 31) : ((w >> 15) & 1u);
-    o.w[j >> 1] |= ((sg << 15) | mag) << (16 * (j & 1));
-    m |= (uint32_t)e.in << j;
+    const uint32_t xb = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+    const uint32_t side = mode == 1 ? (bits16 >> j) & 1u
+                        : ((j < 8 ? c0 : c1) >> (4 * (j & 7))) & 0xFu;
+    bool in;
+    o.w[j >> 1] |= site_exact(xb, d, sbv, s_g, side, mode, in) << (16 * (j & 1));
+    m |= (uint32_t)in << j;
   }
   st_block_plain(dst, o);
   return m;
+}
+
+// One site of a guided forward recomputed on the exact path (the fast pass
+// rounded it to nearest, and the site's rule may choose the other
+// neighbour): reads the site's bf16 input at src, returns its output bits.
+__device__ __noinline__ uint32_t guided_site_fix(const uint16_t* src, float d, float sbv,
+                                                 float s_g, uint32_t side, int mode) {
+  bool in;
+  return site_exact((uint32_t)__ldg(reinterpret_cast<const unsigned short*>(src)), d, sbv, s_g,
+                    side, mode, in);
 }
 
 // ---------------------------------------------------------------------------
@@ -256,16 +288,20 @@ __device__ __forceinline__ void codes_block(const V8& v, const V8* src, float d,
 // Each thread owns two adjacent blocks: one 16-byte store of codes, one
 // 32-bit store of mantissa bits, one 16-bit store of scales.
 // SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
-template <bool SW>
+// RESET: `amax` is the call's workspace (G accumulators, then a ticket
+// counter at amax[G]); the last CTA to finish -- the one that draws ticket
+// gridDim.x - 1, after every other CTA has read the accumulators it needed
+// -- sets the accumulators and the ticket back to zero, so the next capture
+// with the same workspace needs no zeroing launch.  Nothing waits.
+template <bool SW, bool RESET>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-              const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
-              uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales,
-              float* __restrict__ gscale) {
+              uint32_t* amax, uint4* __restrict__ codes, uint32_t* __restrict__ mbits,
+              uint8_t* __restrict__ scales, float* __restrict__ gscale) {
   pdl_begin();
   // global scales of all groups (any CTA may write them; all write the same)
   for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
-    gscale[g] = group_consts(amax[g]).s_g;
+    gscale[g] = group_consts(__ldcg(amax + g)).s_g;
 
   GroupCursor gc;
   gc.init(offs, sh.G);
@@ -280,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
     // both blocks of the pair are in the same row (cols is a multiple of 32)
     const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-    if (gc.seek(row)) gk = group_consts(__ldg(amax + gc.g));
+    if (gc.seek(row)) gk = group_consts(__ldcg(amax + gc.g));
     const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
     float sb0, sb1;
     e4m3x2_to_f32(s2, sb0, sb1);
@@ -301,6 +337,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     else
       reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
   }
+  if (RESET) {
+    __shared__ uint32_t last_s;
+    __syncthreads();  // this CTA's reads of the accumulators are done
+    if (threadIdx.x == 0) {
+      __threadfence();
+      last_s = atomicAdd(amax + sh.G, 1u) == gridDim.x - 1u;
+    }
+    __syncthreads();
+    if (last_s) {
+      __threadfence();
+      for (int g = threadIdx.x; g <= sh.G; g += kThreads) amax[g] = 0u;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -312,86 +361,95 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // compact cache), full-information guided (the cache keeps the whole code).
 enum FqMode { kRtn = 0, kGuided = 1, kFull = 2 };
 
-// Two elements (one bf16x2 word w) of the fake-quant forward.  `side` carries
-// the guidance of the pair: MODE kGuided -- the cached bits of the two
-// elements in bits 0 and 1; kFull -- the rollout's two 4-bit codes (low
-// nibble first).  Mask bits go to positions pos, pos + 1 of m.
-template <int MODE>
-__device__ __forceinline__ uint32_t fq_pair(uint32_t w, uint32_t side, const BlkK& k,
-                                            uint32_t& m, int pos) {
-  // signed x; only |z| is used below (sign of the output comes from w)
-  const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
-  float ql, qh;
-  if (MODE != kRtn) {
-    // z * 2^64 (exact; +-inf/NaN only where |x|/d overflows)
+// Round to nearest over one fast-path block (d in [2^-90, 2^100]): bf16
+// outputs q*s with x's sign, the 16 STE mask bits, and with KIND 1 the 16
+// magnitude codes, with KIND 2 the 16 codes signed with x's sign (c0:
+// elements 0-7, c1: 8-15, element j in nibble j % 8); KIND 0 returns no
+// codes.
+template <int KIND>
+__device__ __forceinline__ void rtn_block(const V8& v, float d, float sbv, float s_g, V8& o,
+                                          uint32_t& m, uint32_t& c0, uint32_t& c1) {
+  const BlkK k = make_blk(d, sbv, s_g);
+  m = 0u;
+  c0 = 0u;
+  c1 = 0u;
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t w = v.w[p];
     float zl, zh;
-    upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
-    m |= (le_mask(fabsf(zl), kSixS) & (1u << pos)) | (le_mask(fabsf(zh), kSixS) & (2u << pos));
-    const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
-    const u64 MM = MODE == kGuided ? grid_magic_s2(al, ah) : pk(grid_magic_s(al), grid_magic_s(ah));
-    const u64 aa = pk(al, ah);
-    float lol, loh, hil, hih;
-    upk(add_rm2(aa, MM), lol, loh);
-    upk(add_rp2(aa, MM), hil, hih);
-    if (MODE == kGuided) {
-      // of floor / ceiling, the one whose mantissa bit is the cached bit: the
-      // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
-      // bit of the floor sum is its codeword's mantissa bit
-      const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
-      const float tl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
-      const float th = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
-      upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
+    upk(quot2(pk(bf16_lo(w), bf16_hi(w)), k), zl, zh);
+    m |= (le_mask(fabsf(zl), 6.0f) & (1u << (2 * p))) | (le_mask(fabsf(zh), 6.0f) & (2u << (2 * p)));
+    float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
+    uint32_t h2;
+    if (KIND == 0) {
+      // round to nearest on the grid (ties to the even code), decoded
+      h2 = rtn_e2m1x2_f16x2(al, ah);
     } else {
-      // of floor / ceiling, the one nearest the rollout codeword: the
-      // rollout value reflected to z's side of zero picks the ceiling
-      // exactly when it lies above the floor (no codeword lies between)
-      float fl, fh, cl, ch;
-      upk(sub2(pk(lol, loh), MM), fl, fh);
-      upk(sub2(pk(hil, hih), MM), cl, ch);
-      const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
-      float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-      float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
-      rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
-      rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
-      upk(mul2(pk(rl, rh), pk(kXs, kXs)), rl, rh);
-      const float tl = rl > fl ? cl : fl;
-      const float th = rh > fh ? ch : fh;
-      upk(mul2(mul2(pk(tl, th), k.sbv2), k.sg2), ql, qh);
+      if (KIND == 2) {
+        al = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
+        ah = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
+      }
+      uint32_t code;
+      h2 = rtn_e2m1x2_f16x2_code(al, ah, code);
+      if (p < 4) c0 |= code << (8 * p); else c1 |= code << (8 * (p - 4));
     }
-  } else {
-    float zl, zh;
-    upk(quot2(xx, k), zl, zh);
-    m |= (le_mask(fabsf(zl), 6.0f) & (1u << pos)) | (le_mask(fabsf(zh), 6.0f) & (2u << pos));
-    const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
-    // round to nearest on the grid (ties to the even code), then dequantise
-    const uint32_t h2 = rtn_e2m1x2_f16x2(al, ah);
     const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
     const float vh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    float ql, qh;
     upk(mul2(mul2(pk(vl, vh), k.sbv2), k.sg2), ql, qh);
+    o.w[p] = cvt_bf16x2(ql, qh) | (w & 0x80008000u);
   }
-  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
 }
 
-// One 16-element block of the fake-quant forward: bf16 outputs and 16 mask
-// bits.  side: kGuided -- the block's 16 cached bits; kFull -- its 16
-// rollout codes (c0: elements 0-7, c1: 8-15).
+// Lowest bit of each of the 16 nibbles of (c0, c1) in bits 0-15 (bit j =
+// nibble j); bits 16-31 are not defined.  Multiply-gather as nibble_lsbs4.
+__device__ __forceinline__ uint32_t nibble_lsbs2(uint32_t c0, uint32_t c1) {
+  const uint32_t kGather = (1u << 24) | (1u << 18) | (1u << 12) | (1u << 6);
+  const uint32_t t0 = ((c0 & 0x01010101u) | ((c0 >> 3) & 0x02020202u)) * kGather;
+  const uint32_t t1 = ((c1 & 0x01010101u) | ((c1 >> 3) & 0x02020202u)) * kGather;
+  return __byte_perm(t0, t1, 0x0073u);
+}
+
+// Bit j (0-15) set where nibble j of (c0, c1) is nonzero.
+__device__ __forceinline__ uint32_t nibble_any2(uint32_t c0, uint32_t c1) {
+  c0 |= c0 >> 1;
+  c1 |= c1 >> 1;
+  return nibble_lsbs2(c0 | (c0 >> 2), c1 | (c1 >> 2)) & 0xFFFFu;
+}
+
+// One fast-path block of the fake-quant forward: bf16 outputs in o, the 16
+// mask bits in m.  The guided rules (MODE kGuided: bits16 = the block's
+// cached bits; kFull: r0, r1 = its rollout codes, elements 0-7 and 8-15)
+// start from round to nearest, which is one of the two codewords around z,
+// and keep it wherever the rule agrees with it: the 1-bit rule wherever its
+// mantissa bit equals the cached bit (the bracket member with that bit, or
+// the collapsed bracket), the full rule wherever its code equals the
+// rollout's (the rollout codeword itself is then in the bracket).  At the
+// other sites -- where the training and rollout sides round differently,
+// rare for a drifted pair -- the site is recomputed on the exact path and
+// patched in.  src: the block's inputs, read there by the patch (o is
+// stored by the caller afterwards, so out may alias x).
 template <int MODE>
-__device__ __forceinline__ void fake_quant_fast(const V8& v, uint32_t bits16, uint32_t c0,
-                                                uint32_t c1, float d, float sbv, float s_g, V8& o,
-                                                uint32_t& m) {
-  const BlkK bk = make_blk(d, MODE != kRtn ? __fmul_rn(sbv, 0x1p-64f) : sbv, s_g);
-  m = 0u;
+__device__ __forceinline__ void fq_block_fast(const V8& v, const uint16_t* src, uint32_t bits16,
+                                              uint32_t r0, uint32_t r1, float d, float sbv,
+                                              float s_g, V8& o, uint32_t& m) {
+  uint32_t c0, c1;
+  rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, d, sbv, s_g, o, m, c0, c1);
+  if (MODE == kRtn) return;
+  uint32_t bad = MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu
+                                 : nibble_any2(c0 ^ r0, c1 ^ r1);
+  while (bad != 0u) {
+    const int j = __ffs(bad) - 1;
+    bad &= bad - 1u;
+    const uint32_t side = MODE == kGuided ? (bits16 >> j) & 1u
+                                          : ((j < 8 ? r0 : r1) >> (4 * (j & 7))) & 0xFu;
+    const uint32_t val = guided_site_fix(src + j, d, sbv, s_g, side, MODE);
+    const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint32_t side = MODE == kGuided ? bits16 >> (2 * k)
-                        : MODE == kFull ? ((k < 4 ? c0 : c1) >> (8 * (k & 3))) : 0u;
-    o.w[k] = fq_pair<MODE>(v.w[k], side, bk, m, 2 * k);
+    for (int k = 0; k < 8; ++k)
+      if (k == (j >> 1)) o.w[k] = (o.w[k] & keep) | (val << sh);
   }
 }
-
-// Upper end of the fast range of the scale d for each mode.
-template <int MODE>
-__host__ __device__ constexpr uint32_t fq_dmax() { return MODE != kRtn ? kDMaxExactZ : kDMax; }
 
 // One block with any scale (zero block, fast path or exact path): stores its
 // output at dst and returns its 16 mask bits.
@@ -407,8 +465,9 @@ __device__ __forceinline__ uint32_t fake_quant_block(const V8& v, const V8* src,
 #pragma unroll
     for (int k = 0; k < 8; ++k) o.w[k] = v.w[k] & 0x80008000u;
     m = 0xFFFFu;
-  } else if (fast_scale(d, fq_dmax<MODE>())) {
-    fake_quant_fast<MODE>(v, bits16, c0, c1, d, sbv, s_g, o, m);
+  } else if (fast_scale(d)) {
+    fq_block_fast<MODE>(v, reinterpret_cast<const uint16_t*>(src), bits16, c0, c1, d, sbv, s_g,
+                        o, m);
   } else {
     return fake_quant_block_exact(src, d, sbv, s_g, bits16, c0, c1, MODE, dst);
   }
@@ -453,12 +512,13 @@ __global__ void __launch_bounds__(kThreads, MINB)
     // a row holds a whole number of 32-element words, so both blocks of the
     // pair are in the same row and group
     const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
-    if (fast_scale(d0, fq_dmax<MODE>()) && fast_scale(d1, fq_dmax<MODE>())) {
+    if (fast_scale(d0) && fast_scale(d1)) {
       // the common case, without per-block branches
       V8 o;
-      fake_quant_fast<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
+      const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
+      fq_block_fast<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
       st_block(out + b, o);
-      fake_quant_fast<MODE>(v1, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
+      fq_block_fast<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
       st_block(out + b + 1, o);
     } else {
       m0 = fake_quant_block<MODE>(v0, x + b, bits & 0xFFFFu, rc.x, rc.y, sbv0, s_g, out + b);

@@ -57,8 +57,8 @@
 //     round-to-nearest.
 // File layout: this file holds the host side and the C ABI; the kernels are
 // in csrc/*.cuh, included below inside this file's anonymous namespace (one
-// translation unit): common.cuh (shared device helpers), nvfp4.cuh, mismatch.cuh,
-// mx.cuh, util.cuh.
+// translation unit): common.cuh (shared device helpers), nvfp4.cuh, mx.cuh,
+// mismatch.cuh, util.cuh.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -70,8 +70,8 @@ namespace {
 
 #include "common.cuh"
 #include "nvfp4.cuh"
-#include "mismatch.cuh"
 #include "mx.cuh"
+#include "mismatch.cuh"
 #include "util.cuh"
 
 // ---------------------------------------------------------------------------
@@ -214,7 +214,8 @@ int trace_abi_version(void) { return TRACE_ABI_VERSION; }
 
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
   if (rows < 0 || cols <= 0 || cols % 32 != 0 || num_groups < 1) return 0;
-  return ((size_t)num_groups * 4u + 255u) / 256u * 256u;
+  // G accumulators and the quantising pass's ticket counter
+  return ((size_t)num_groups * 4u + 4u + 255u) / 256u * 256u;
 }
 
 size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
@@ -232,10 +233,13 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
   return up16(og + 4u * (size_t)num_groups);
 }
 
+// zero_first: zero the workspace with a launch of its own before the amax
+// pass (the static-scratch entry point, whose array other calls share);
+// otherwise the workspace holds zeros on entry, as every capture leaves it.
 static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                         const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
                         uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
-                        bool tiled, void* stream) {
+                        bool tiled, void* stream, bool zero_first = false) {
   int st = check_shape(rows, cols, num_groups, group_row_offsets);
   if (st) return st;
   // with no rows only the global scales are written; the data pointers of
@@ -252,14 +256,18 @@ static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t n
   cudaStream_t s = (cudaStream_t)stream;
   uint32_t* amax = (uint32_t*)workspace;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
-  const int zg = (num_groups + kThreads - 1) / kThreads;
-  if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups))) return st;
+  if (zero_first) {
+    const int zg = (num_groups + 1 + kThreads - 1) / kThreads;
+    if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups + 1))) return st;
+  }
   if (sh.nblk > 0 && (st = launch(k_amax, grid, s, (const V8*)x, sh, offs, amax))) return st;
-  if (tiled)
-    return launch(k_capture<true>, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax,
-                  (uint4*)codes, (uint32_t*)mbits, scales, gscale);
-  return launch(k_capture<false>, grid, s, (const V8*)x, sh, offs, (const uint32_t*)amax,
-                (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+  st = tiled ? launch(k_capture<true, true>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes,
+                      (uint32_t*)mbits, scales, gscale)
+             : launch(k_capture<false, true>, grid, s, (const V8*)x, sh, offs, amax,
+                      (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+  // a failed launch would leave the accumulators set: clear them (best effort)
+  if (st != TRACE_OK) (void)cudaMemsetAsync(workspace, 0, ((size_t)num_groups + 1) * 4u, s);
+  return st;
 }
 
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
@@ -484,11 +492,12 @@ int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols, int32
   if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
+  uint32_t* am = const_cast<uint32_t*>(amax);  // read only: no reset in this variant
   if (scale_layout == TRACE_SCALES_TILED_128x4)
-    return launch(k_capture<true>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes, mbits,
-                  scales, gscale);
-  return launch(k_capture<false>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes, mbits,
-                scales, gscale);
+    return launch(k_capture<true, false>, grid, s, (const V8*)x, sh, offs, am, (uint4*)codes,
+                  mbits, scales, gscale);
+  return launch(k_capture<false, false>, grid, s, (const V8*)x, sh, offs, am, (uint4*)codes,
+                mbits, scales, gscale);
 }
 
 int trace_capture_ex(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
@@ -657,7 +666,9 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* str
 // that trace_capture takes as `workspace` in a fixed array that lives in the
 // library itself, one copy per GPU, for the life of the process.
 // ---------------------------------------------------------------------------
-static __device__ __align__(256) uint32_t g_capture_scratch[TRACE_STATIC_MAX_GROUPS];
+// TRACE_STATIC_MAX_GROUPS accumulators, the quantising pass's ticket counter
+// and padding to a multiple of 256 bytes
+static __device__ __align__(256) uint32_t g_capture_scratch[TRACE_STATIC_MAX_GROUPS + 64];
 
 static void* g_capture_scratch_addr[kMaxDevices];  // per device; benign race (same value)
 
@@ -686,9 +697,10 @@ int trace_capture_static_ws(const uint16_t* x, int64_t rows, int64_t cols, int32
       return TRACE_ERR_CUDA;
     g_capture_scratch_addr[dev] = ws = a;
   }
-  // the accumulators are zeroed by the capture's first kernel on every call
-  return trace_capture(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,
-                       ws, sizeof(g_capture_scratch), stream);
+  // the array is zeroed by the capture's first kernel on every call (and
+  // left zeroed by its last)
+  return capture_impl(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,
+                      ws, sizeof(g_capture_scratch), false, stream, true);
 }
 
 }  // extern "C"

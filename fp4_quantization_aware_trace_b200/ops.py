@@ -277,7 +277,8 @@ def alloc_capture(rows: int, cols: int, num_groups: int = 1, device="cuda",
                   scales=torch.empty(rows, cols // 16, dtype=torch.uint8, device=device),
                   gscale=torch.empty(num_groups, dtype=torch.float32, device=device),
                   offsets=offsets)
-    ws = torch.empty(max(trace_capture_workspace_bytes(rows, cols, num_groups), 256),
+    # zeros before its first use; every capture leaves it zeroed again
+    ws = torch.zeros(max(trace_capture_workspace_bytes(rows, cols, num_groups), 256),
                      dtype=torch.uint8, device=device)
     return cap, ws
 

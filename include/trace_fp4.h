@@ -89,12 +89,12 @@ typedef enum {
 const char* trace_strerror(int status);
 
 /* ABI version of this header (bumped on any incompatible change). */
-#define TRACE_ABI_VERSION 1
+#define TRACE_ABI_VERSION 2
 int trace_abi_version(void);
 
 /* Bytes of device workspace that trace_capture needs for G groups: the
- * per-group amax accumulators (4 bytes each, rounded up to 256).  Returns 0
- * when the shape is invalid. */
+ * per-group amax accumulators (4 bytes each) and a ticket counter, rounded
+ * up to 256.  Returns 0 when the shape is invalid. */
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols,
                                      int32_t num_groups);
 
@@ -124,8 +124,14 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
  *   scales  : out, uint8[N/16], 16-byte aligned.
  *   gscale  : out, float[G], 4-byte aligned.
  *   workspace: device scratch of at least trace_capture_workspace_bytes()
- *             bytes, 256-byte aligned; its contents on entry do not matter.
- * Launches three kernels (zero the accumulators, grid amax, quantise). */
+ *             bytes, 256-byte aligned, holding zeros before its first use
+ *             (e.g. cudaMemsetAsync once, when it is allocated); every call
+ *             leaves it all-zero again, so a workspace can serve any number
+ *             of calls one after another (not two calls that may run at the
+ *             same time).
+ * Launches two kernels: the grid amax (max-accumulated into the workspace),
+ * then the quantising pass, whose last CTA to finish (an atomic ticket in
+ * the workspace; nothing waits) sets the workspace back to zero. */
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
                   int32_t num_groups, const int64_t* group_row_offsets,
                   uint8_t* codes, uint32_t* mbits, uint8_t* scales,
@@ -405,8 +411,9 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel,
  * the library -- e.g. a host program whose device memory is fixed at
  * start-up, or a binding that can only pass along the buffers it was given.
  * Instead of a `workspace` argument, the amax accumulators live in a static
- * array inside the library: TRACE_STATIC_MAX_GROUPS uint32 (16 KiB) per GPU
- * that loads the library, kept until the process exits.
+ * array inside the library: TRACE_STATIC_MAX_GROUPS + 64 uint32 (16.25 KiB:
+ * the accumulators, a ticket counter and padding) per GPU that loads the
+ * library, kept until the process exits.
  *   Arguments and outputs are those of trace_capture without `workspace`.
  *   num_groups > TRACE_STATIC_MAX_GROUPS: returns TRACE_ERR_WORKSPACE and
  *   enqueues nothing.

@@ -101,6 +101,7 @@ int main(int argc, char** argv) {
   CK(cudaMalloc((void**)&d_gs, GROUPS * 4));
   CK(cudaMalloc((void**)&d_offs, sizeof offs));
   CK(cudaMalloc(&d_ws, ws_bytes));
+  CK(cudaMemset(d_ws, 0, ws_bytes)); /* zeros before first use */
   CK(cudaMemcpy(d_xr, xr, n * 2, cudaMemcpyHostToDevice));
   CK(cudaMemcpy(d_xt, xt, n * 2, cudaMemcpyHostToDevice));
   CK(cudaMemcpy(d_g, g, n * 2, cudaMemcpyHostToDevice));

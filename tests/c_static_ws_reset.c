@@ -66,6 +66,7 @@ static int one_round(int e0, int round) {
   CK(cudaMalloc((void**)&x, n * 2));
   CK(cudaMalloc((void**)&offs, sizeof(hoffs)));
   CK(cudaMalloc(&ws, wsb));
+  CK(cudaMemset(ws, 0, wsb)); /* zeros before first use */
   for (int k = 0; k < 2; ++k) {
     CK(cudaMalloc((void**)&codes[k], n / 2));
     CK(cudaMalloc((void**)&mbits[k], n / 8));

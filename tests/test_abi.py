@@ -50,16 +50,17 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_strings(lib):
-    assert lib.trace_abi_version() == 1
+    assert lib.trace_abi_version() == 2
     for st in range(6):
         assert lib.trace_strerror(st)
     assert b"unknown" in lib.trace_strerror(99)
 
 
 def test_workspace_query(lib):
+    # G accumulators and the ticket counter, 4 bytes each, in 256-byte units
     assert ops.trace_capture_workspace_bytes(16, 32, 1) == 256
-    assert ops.trace_capture_workspace_bytes(16, 32, 64) == 256
-    assert ops.trace_capture_workspace_bytes(16, 32, 65) == 512
+    assert ops.trace_capture_workspace_bytes(16, 32, 63) == 256
+    assert ops.trace_capture_workspace_bytes(16, 32, 64) == 512
     assert ops.trace_capture_workspace_bytes(16, 33, 1) == 0
     assert ops.trace_capture_workspace_bytes(16, 32, 0) == 0
 

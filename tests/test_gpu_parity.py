@@ -415,7 +415,7 @@ def test_canaries_untouched():
                                                  gscale=4 * G, out=2 * n, mask=n // 8,
                                                  gin=2 * n).items()}
         v = {k: b[1] for k, b in bufs.items()}
-        ws = torch.empty(ops.trace_capture_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=DEV)
+        ws = torch.zeros(ops.trace_capture_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=DEV)
         xr, xt, g = s.x_roll.to(DEV), s.x_train.to(DEV), s.grad.to(DEV)
         ops.trace_capture(xr, rows, cols, G, o, v["codes"], v["mbits"], v["scales"], v["gscale"],
                           ws, ws.numel())
@@ -535,3 +535,31 @@ def test_step_in_a_cuda_graph(oracle_mod, forked):
         for k in got:
             _eq(f"graph.{seed}.{k}", got[k], ref[k])
     del gph
+
+
+def test_workspace_left_zeroed_and_reused(oracle_mod):
+    """Capture leaves its workspace all-zero (the quantising pass's last CTA
+    resets the accumulators and the ticket), so one workspace serves calls
+    one after another: a tensor with a huge maximum, then ragged groups of
+    small values, then an empty tensor -- each matches the oracle."""
+    cases = []
+    a = inputs.tiny_site(501, 700, 256).x_roll.float()
+    a[13, 7] = 3.0e5
+    cases.append((a.to(torch.bfloat16), None))
+    b = (inputs.tiny_site(502, 300, 128).x_roll.float() * 1e-4).to(torch.bfloat16)
+    cases.append((b, np.array([0, 50, 50, 300], np.int64)))
+    cases.append((torch.zeros(0, 64, dtype=torch.bfloat16), None))
+    G_max = 3
+    ws = torch.zeros(ops.trace_capture_workspace_bytes(1, 32, G_max), dtype=torch.uint8, device=DEV)
+    for x, offs in cases:
+        R, C = x.shape
+        G = 1 if offs is None else len(offs) - 1
+        o = None if offs is None else torch.from_numpy(offs).to(DEV)
+        cap, _ = ops.alloc_capture(R, C, G, DEV, o)
+        ops.capture(x.to(DEV), o, cap, ws)
+        torch.cuda.synchronize()
+        assert int(ws.count_nonzero()) == 0
+        ref = oracle_mod.capture(inputs.bits(x), G, offs)
+        for name, got, want in zip(("codes", "mbits", "scales", "gscale"),
+                                   (cap.codes, cap.mbits, cap.scales, cap.gscale), ref):
+            _eq(name, _u(got), want)

@@ -824,3 +824,46 @@ def test_mx_mismatch_histogram_vs_codes(oracle_mod):
         for k in range(3):
             d = np.array([abs(index(int(p)) - index(int(q))) for p, q in zip(rules[k], q_roll)])
             assert np.array_equal(hist[k], np.bincount(d, minlength=15)), k
+
+
+def _boundary_lattice():
+    """Every codeword and midpoint of [0, 6], +-1..3 ulps around each, and
+    random magnitudes (float32)."""
+    pts = [0.0, 0.25, 0.5, 0.75, 1.0, 1.25, 1.5, 1.75, 2.0, 2.5, 3.0, 3.5, 4.0, 5.0, 6.0]
+    out = set()
+    for p in pts:
+        v = np.float32(p)
+        for k in range(4):
+            out.add(float(v))
+            v = np.nextafter(v, np.float32(7.0))
+        v = np.float32(p)
+        for k in range(3):
+            v = np.nextafter(v, np.float32(-1.0))
+            if v >= 0:
+                out.add(float(v))
+    rng = np.random.default_rng(77)
+    out.update(float(a) for a in rng.uniform(0, 6, 3000).astype(np.float32))
+    out.update(float(a) for a in (rng.uniform(0, 1e-3, 200).astype(np.float32)))
+    return sorted(a for a in out if 0.0 <= a <= 6.0)
+
+
+def test_guided_rules_keep_round_to_nearest_where_it_agrees(oracle_mod):
+    """The guided forwards start from round to nearest and recompute only the
+    sites where a rule may differ.  Pinned here with the oracle's own rules:
+    the 1-bit rule returns the round-to-nearest code wherever that code's
+    mantissa bit equals the cached bit, and the full-information rule returns
+    it wherever the rollout's signed code equals it (both signs, z beyond 6
+    clipped)."""
+    lat = _boundary_lattice()
+    for a in lat:
+        r = oracle_mod.e2m1_rtn(a)
+        assert oracle_mod.guided_code(a, r & 1) == r, a
+        for z in (a, -a, a * 1.5 + 6.0, -(a * 1.5 + 6.0)):
+            zc = min(abs(z), 6.0)
+            rs = (8 if np.signbit(np.float32(z)) else 0) | oracle_mod.e2m1_rtn(np.float32(zc))
+            assert oracle_mod.full_guided_code(z, rs) == rs & 7, z
+    # and the premise is not vacuous: where the bit disagrees, the 1-bit rule
+    # moves off round to nearest at every site that is not a codeword
+    moved = sum(oracle_mod.guided_code(a, 1 - (oracle_mod.e2m1_rtn(a) & 1)) !=
+                oracle_mod.e2m1_rtn(a) for a in lat)
+    assert moved > 0.9 * len(lat)

@@ -38,7 +38,7 @@ def _outs(rows, cols, G):
 def _reference(x, offs, G):
     rows, cols = x.shape
     o = _outs(rows, cols, G)
-    ws = torch.empty(ops.trace_capture_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=DEV)
+    ws = torch.zeros(ops.trace_capture_workspace_bytes(rows, cols, G), dtype=torch.uint8, device=DEV)
     ops.trace_capture(x, rows, cols, G, offs, o["codes"], o["mbits"], o["scales"], o["gscale"],
                       ws, ws.numel())
     return o
