@@ -673,25 +673,38 @@ def step_summary(args, wl: Workload, m, world, hbm, peak_kind):
 
 
 def yardstick_leg(args, wl, pg, dev, flush):
-    """The library's plain copy kernel on the largest tensor of the workload."""
+    """The library's copy kernels on the largest tensor of the workload: the
+    plain one (32-byte loads straight to registers, the kernels' own access
+    pattern) and the one with its reads staged through shared memory by the
+    bulk-copy engine (cp.async.bulk + mbarrier, four 16 KiB tiles in flight
+    per CTA).  Both are checked to have copied every byte."""
     from fp4_quantization_aware_trace_b200 import ops
     stream = torch.cuda.current_stream()
     ny = max(w["xr"].numel() for w in wl.work)
-    ysrc = torch.empty(ny, dtype=torch.bfloat16, device=dev).fill_(1.0)
+    ysrc = torch.randn(ny, device=dev).to(torch.bfloat16)
     ydst = torch.empty_like(ysrc)
-    yev = [_pair() for _ in range(args.steps)]
-    for i in range(3):
-        flush.fill_(i)
-        ops.trace_copy_bf16(ysrc, ydst, ny, stream)
-    for k in range(args.steps):
-        flush.fill_((k + 3) & 0xFF)
-        yev[k][0].record(stream)
-        ops.trace_copy_bf16(ysrc, ydst, ny, stream)
-        yev[k][1].record(stream)
-    torch.cuda.synchronize()
-    y_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in yev) / args.steps], pg, dev)[0]
-    return {"kernel": "k_copy", "bytes": 4 * ny, "us": round(y_ms * 1e3, 2),
-            "gbs": round(4 * ny / (y_ms * 1e-3) / 1e9, 1), "l2": "flushed before each launch"}
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = {}
+    for name, fn in (("k_copy", lambda: ops.trace_copy_bf16(ysrc, ydst, ny, stream)),
+                     ("k_copy_staged", lambda: ops.trace_copy_bf16_staged(ysrc, ydst, ny, err,
+                                                                          stream))):
+        yev = [_pair() for _ in range(args.steps)]
+        for i in range(3):
+            flush.fill_(i)
+            fn()
+        ydst.zero_()
+        for k in range(args.steps):
+            flush.fill_((k + 3) & 0xFF)
+            yev[k][0].record(stream)
+            fn()
+            yev[k][1].record(stream)
+        torch.cuda.synchronize()
+        ok = bool(torch.equal(ydst, ysrc)) and int(err.item()) == 0
+        y_ms = max_over_ranks([sum(a.elapsed_time(b) for a, b in yev) / args.steps], pg, dev)[0]
+        out[name] = {"bytes": 4 * ny, "us": round(y_ms * 1e3, 2),
+                     "gbs": round(4 * ny / (y_ms * 1e-3) / 1e9, 1), "copied_ok": ok}
+    out["l2"] = "flushed before each launch"
+    return out
 
 
 def next_rows_leg(args, wl: Workload, pg, dev, flush, hbm):

@@ -656,6 +656,48 @@ int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel, void* str
 }
 
 
+int trace_copy_bf16_staged(const uint16_t* src, uint16_t* dst, int64_t numel, uint32_t* err,
+                           void* stream) {
+  if (numel < 0 || numel % 16 != 0) return TRACE_ERR_SHAPE;
+  if ((long double)numel / 16 >= 4294967296.0L - (long double)kTileBlks) return TRACE_ERR_SHAPE;
+  if (numel == 0) return TRACE_OK;
+  if (!src || !dst || !err) return TRACE_ERR_NULL;
+  if (!aligned(src, 32) || !aligned(dst, 32) || !aligned(err, 4)) return TRACE_ERR_ALIGN;
+  Shape sh;
+  sh.nblk = (uint32_t)(numel / 16);
+  sh.ntiles = (uint32_t)(((uint64_t)sh.nblk + kTileBlks - 1) / kTileBlks);
+  sh.bpr = make_fastdiv(1);
+  sh.G = 1;
+  sh.sw_ct = 1;
+  const int sms = sm_count();
+  if (sms <= 0) return TRACE_ERR_CUDA;
+  const size_t smem = (size_t)kStages * kTileBytes;  // 64 KiB: two CTAs per SM
+  static bool attr_set[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TRACE_ERR_CUDA;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(k_copy_staged, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return TRACE_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  uint32_t grid = (uint32_t)sms * 2u;
+  if (sh.ntiles < grid) grid = sh.ntiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_copy_staged, (const V8*)src, sh, (V8*)dst, err) == cudaSuccess
+             ? TRACE_OK
+             : TRACE_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------------------
 // Capture without a caller-provided workspace.
 //

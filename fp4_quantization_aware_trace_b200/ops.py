@@ -61,6 +61,8 @@ def library() -> ctypes.CDLL:
         lib.trace_rtn_fq_fwd.restype = ctypes.c_int
         lib.trace_copy_bf16.argtypes = [P, P, i64, P]
         lib.trace_copy_bf16.restype = ctypes.c_int
+        lib.trace_copy_bf16_staged.argtypes = [P, P, i64, P, P]
+        lib.trace_copy_bf16_staged.restype = ctypes.c_int
         lib.trace_full_guided_fq_fwd.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, P]
         lib.trace_full_guided_fq_fwd.restype = ctypes.c_int
         lib.trace_capture_static_ws.argtypes = [P, i64, i64, i32, P, P, P, P, P, P]
@@ -239,6 +241,11 @@ def trace_selftest_e4m3_sweep(first_bits: int, count: int, out, stream=None) -> 
 
 def trace_copy_bf16(src, dst, numel, stream=None) -> None:
     _check(library().trace_copy_bf16(_p(src), _p(dst), numel, _stream(stream)), "trace_copy_bf16")
+
+
+def trace_copy_bf16_staged(src, dst, numel, err, stream=None) -> None:
+    _check(library().trace_copy_bf16_staged(_p(src), _p(dst), numel, _p(err), _stream(stream)),
+           "trace_copy_bf16_staged")
 
 
 # ---------------------------------------------------------------------------

@@ -405,6 +405,18 @@ int trace_validate_offsets(const int64_t* group_row_offsets, int32_t num_groups,
 int trace_copy_bf16(const uint16_t* src, uint16_t* dst, int64_t numel,
                     void* stream);
 
+/* The same copy with the reads staged through shared memory by the bulk-copy
+ * engine (cp.async.bulk global -> shared, an mbarrier per stage, four 16 KiB
+ * tiles in flight per CTA, two CTAs per SM), each thread then storing its
+ * part from registers: the yardstick of a TMA-staged pipeline, measured
+ * beside the plain copy.  Not part of the method.  err: device uint32,
+ * 4-byte aligned, set to 1 if a CTA gave up waiting for a stage (a bounded
+ * wait; never expected) and left alone otherwise -- the caller zeroes it and
+ * reads it after the stream reaches the copy.  Same shape and alignment rules
+ * as trace_copy_bf16. */
+int trace_copy_bf16_staged(const uint16_t* src, uint16_t* dst, int64_t numel,
+                           uint32_t* err, void* stream);
+
 /* Rollout capture for callers that cannot provide a workspace.  The paper
  * has no counterpart: this is a calling convention, not a step of the method.
  * Who needs it: a caller that may not allocate device memory when it calls

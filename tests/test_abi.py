@@ -91,6 +91,12 @@ def test_host_argument_checks(lib):
     # sizes
     assert lib.trace_fq_bwd(a, a, 40, a, None) == 2
     assert lib.trace_copy_bf16(a, a, 12, None) == 2
+    # the staged copy yardstick
+    assert lib.trace_copy_bf16_staged(a, a, 12, a, None) == 2
+    assert lib.trace_copy_bf16_staged(a, a, 16, None, None) == 1
+    assert lib.trace_copy_bf16_staged(a, odd, 16, a, None) == 3
+    assert lib.trace_copy_bf16_staged(a, a, 16, odd, None) == 3
+    assert lib.trace_copy_bf16_staged(a, a, 0, None, None) == 0
 
 
 def test_binding_rejects_host_tensors(lib):

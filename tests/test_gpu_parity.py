@@ -563,3 +563,22 @@ def test_workspace_left_zeroed_and_reused(oracle_mod):
         for name, got, want in zip(("codes", "mbits", "scales", "gscale"),
                                    (cap.codes, cap.mbits, cap.scales, cap.gscale), ref):
             _eq(name, _u(got), want)
+
+
+@pytest.mark.parametrize("numel", [16, 8192 * 16 - 16, 8192 * 16 * 37 + 48])
+def test_copy_yardsticks_copy_every_byte(numel):
+    """The two bandwidth yardsticks (plain, and reads staged through shared
+    memory by the bulk-copy engine) copy every element, ragged last tile
+    included, and the staged one reports no timed-out wait."""
+    src = torch.randn(numel, device=DEV).to(torch.bfloat16)
+    for staged in (False, True):
+        dst = torch.full_like(src, 7.0)
+        if staged:
+            err = torch.zeros(1, dtype=torch.int32, device=DEV)
+            ops.trace_copy_bf16_staged(src, dst, numel, err)
+        else:
+            ops.trace_copy_bf16(src, dst, numel)
+        torch.cuda.synchronize()
+        assert torch.equal(dst.view(torch.int16), src.view(torch.int16)), staged
+        if staged:
+            assert int(err.item()) == 0
