@@ -144,13 +144,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   pdl_begin();
   if (blockIdx.x >= sh.ntiles) return;
 
+  // the first tile's loads go out before the CTA's set-up barrier
+  V8 v[kBlkPerThread];
+  {
+    const uint32_t base = blockIdx.x * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
+    }
+  }
   GroupCursor gc;
   gc.init(offs, sh.G);
-  if (threadIdx.x == 0) {
-    gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
-    g_first_s = gc.g;
+  if (sh.G > 1) {
+    if (threadIdx.x == 0) {
+      gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
+      g_first_s = gc.g;
+    }
+    for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
+  } else if (threadIdx.x == 0) {
+    table[0] = 0u;
+    g_first_s = 0;
   }
-  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
   __syncthreads();
   const int g_first = g_first_s;
   gc.init(offs, sh.G);
@@ -164,14 +179,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     else atomicMax(&amax[g], val);
   };
 
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
-    V8 v[kBlkPerThread];
+  for (uint32_t t = blockIdx.x; t < sh.ntiles;) {
     const uint32_t base = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
-    }
 #pragma unroll
     for (int u = 0; u < kBlkPerThread; ++u) {
       const uint32_t b = base + u * kThreads;
@@ -188,14 +197,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       }
       run = max(run, absmax_block(v[u]));
     }
+    t += gridDim.x;
+    if (t >= sh.ntiles) break;
+    const uint32_t nb = t * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = nb + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
+    }
   }
   if (sh.G == 1) {
-    for (int o = 16; o > 0; o >>= 1) run = max(run, __shfl_xor_sync(0xFFFFFFFFu, run, o));
+    run = __reduce_max_sync(0xFFFFFFFFu, run);
     if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
   } else {
     flush(run_g, run);
   }
   __syncthreads();
+  if (sh.G == 1) {
+    if (threadIdx.x == 0 && table[0]) atomicMax(&amax[0], table[0]);
+    return;
+  }
   for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
     const uint32_t val = table[i];
     if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
