@@ -14,8 +14,9 @@ layers 20..39 of 40 x {qkv-in, o-in, expert up-in, expert down-in}, each
 relative training noise (seeded, synthetic).  All 80 sites' x_roll, x_train
 and grad (120 GiB) stay resident in HBM; every input is read from HBM once
 per step (far larger than the 126 MB L2, so no flush is needed between
-steps).  The attention-input site [16384, 2048] is measured after it, as a
-secondary line (`secondary`), with L2 flushed before every step.
+steps).  The attention-input site [16384, 2048], the MoE expert inputs and
+the KV cache follow as secondary lines (`secondary`), with L2 flushed before
+every step.
 
 The value is algorithmic bytes / time (GB/s): every input read once and every
 output written once per kernel, x_roll read twice by capture (its two
@@ -54,7 +55,7 @@ import torch  # noqa: E402
 
 METRIC = "capture & guided fake-quant fwd GB/s (elem/s) and % of B200 HBM roofline"
 HEADLINE_CONFIG = 5
-SECONDARY_CONFIG = 2
+SECONDARY_CONFIGS = (2, 3, 4)
 BYTES_PER_ELEM = {"capture": 4.6875, "guided_fwd": 4.3125, "ste_bwd": 4.125, "rtn_fwd": 4.1875}
 STEP_BYTES_PER_ELEM = sum(BYTES_PER_ELEM.values())
 KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<1> (1-bit guided)",
@@ -106,7 +107,8 @@ def parse(argv=None):
                          "stream pairs inside the graph (1: one after another)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the secondary line (attention-input site) after the headline")
+                    help="skip the secondary lines (attention input, MoE experts, KV cache) "
+                         "after the headline")
     ap.add_argument("--next-sites", type=int, default=8,
                     help="sites of the workload the next-row legs (full guidance, "
                          "histogram, MXFP4, W4A8, tiled scales, cache tier) run on")
@@ -974,19 +976,24 @@ def run_trace(args):
 
     secondary = None
     if not args.no_secondary and args.config == HEADLINE_CONFIG:
-        wl2 = Workload(SECONDARY_CONFIG, rank, dev, args.lanes)
-        m2 = measure_step(args, wl2, pg, dev, clk, flush)
-        s2 = step_summary(args, wl2, m2, world, hbm, peak_kind)
-        secondary = {"workload": WORKLOAD_NAMES[SECONDARY_CONFIG],
-                     "value": round(s2["value"], 3), "unit": "GB/s",
-                     "ms_per_step": round(s2["ms_per_step"], 5),
-                     "elem_per_s": round(s2["elem_per_s"], 1),
-                     "algo_bytes_over_copy_peak": round(s2["algo_bytes_over_copy_peak"], 4),
-                     "kernels": s2["kernels"], "roofline": s2["roofline"],
-                     "yardstick": yardstick_leg(args, wl2, pg, dev, flush),
-                     "l2": "flushed before every step (256 MiB write)", "launch": m2["launch"]}
-        gpu_launches += LAUNCHES_PER_SITE * len(wl2.work) * args.steps * m2["timed_passes"]
-        del wl2
+        secondary = {}
+        for cfg2 in SECONDARY_CONFIGS:
+            wl2 = Workload(cfg2, rank, dev, args.lanes)
+            m2 = measure_step(args, wl2, pg, dev, clk, flush)
+            s2 = step_summary(args, wl2, m2, world, hbm, peak_kind)
+            secondary[WORKLOAD_TAGS[cfg2]] = {
+                "workload": WORKLOAD_NAMES[cfg2], "shapes": wl2.shapes,
+                "value": round(s2["value"], 3), "unit": "GB/s",
+                "ms_per_step": round(s2["ms_per_step"], 5),
+                "eager_ms_per_step": round(s2["eager_ms_per_step"], 5),
+                "elem_per_s": round(s2["elem_per_s"], 1),
+                "algo_bytes_over_copy_peak": round(s2["algo_bytes_over_copy_peak"], 4),
+                "kernels": s2["kernels"], "roofline": s2["roofline"],
+                "yardstick": yardstick_leg(args, wl2, pg, dev, flush),
+                "l2": "flushed before every step (256 MiB write)", "launch": m2["launch"]}
+            gpu_launches += LAUNCHES_PER_SITE * len(wl2.work) * args.steps * m2["timed_passes"]
+            del wl2
+            torch.cuda.empty_cache()
 
     if pg:
         pg.barrier()
