@@ -160,6 +160,55 @@ __device__ __noinline__ uint32_t site_codes_exact(const uint16_t* src, float d, 
   return (uint32_t)e.floor | (c << 4) | (r << 8);
 }
 
+// Signed round-to-nearest codes of one fast-path block (c0: elements 0-7,
+// c1: 8-15), each with the sign of x: the exact quotient, min(|z|, 6) --
+// which also maps the NaN of an overflowing quotient (a training value far
+// beyond the rollout's scale) to 6 -- and the hardware conversion.
+__device__ __forceinline__ void rtn_codes_signed(const V8& v, float d, uint32_t& c0,
+                                                 uint32_t& c1) {
+  const BlkK k = make_blk(d, 0.0f, 0.0f);
+  float a[16];
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    const uint32_t w = v.w[p];
+    float zl, zh;
+    upk(quot2(pk(bf16_lo(w), bf16_hi(w)), k), zl, zh);
+    a[2 * p] = __uint_as_float(__float_as_uint(fminf(fabsf(zl), 6.0f)) | ((w << 16) & 0x80000000u));
+    a[2 * p + 1] = __uint_as_float(__float_as_uint(fminf(fabsf(zh), 6.0f)) | (w & 0x80000000u));
+  }
+  c0 = cvt_e2m1x8(a);
+  c1 = cvt_e2m1x8(a + 8);
+}
+
+// Floor, ceiling and signed round-to-nearest codes of one pair (word w) as
+// three bytes (lo element in the low nibble), by the grid rounding of
+// codes_pair (NVFP4, constants k) or on z = |x| * 2^-e (MX, inv2).
+__device__ __forceinline__ void pair_codes(uint32_t w, const BlkK& k, uint32_t& f, uint32_t& c,
+                                           uint32_t& r) {
+  float ff[2], cc[2], rr[2];
+  codes_pair(w, k, ff, cc, rr);
+  f = cvt_e2m1x8(ff[0], ff[1], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+  c = cvt_e2m1x8(cc[0], cc[1], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+  r = cvt_e2m1x8(rr[0], rr[1], 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+}
+__device__ __forceinline__ void mx_pair_codes(uint32_t w, u64 inv2, uint32_t& f, uint32_t& c,
+                                              uint32_t& r) {
+  const uint32_t wa = w & 0x7FFF7FFFu;
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(wa), bf16_hi(wa)), inv2), zl, zh);  // inf only past 6
+  const float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);
+  const u64 MM = pk(grid_magic(al), grid_magic(ah));
+  const u64 aa = pk(al, ah);
+  float fl, fh, cl, ch;
+  upk(sub2(add_rm2(aa, MM), MM), fl, fh);
+  upk(sub2(add_rp2(aa, MM), MM), cl, ch);
+  f = cvt_e2m1x8(fl, fh, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+  c = cvt_e2m1x8(cl, ch, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f);
+  r = cvt_e2m1x8(__uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u)),
+                 __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u)), 0.f, 0.f, 0.f, 0.f,
+                 0.f, 0.f);
+}
+
 // Bit j (0-31) set where nibble j of the four words differs from zero.
 __device__ __forceinline__ uint32_t nibble_any4(uint4 w) {
   w.x |= w.x >> 1; w.y |= w.y >> 1; w.z |= w.z >> 1; w.w |= w.w >> 1;
@@ -225,18 +274,35 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         hist_word(k1.f[1], k1.c[1], k1.r[1], rc.w, ones, bins);
         continue;
       }
-      codes_fast(v0, d0, r.x, r.y);
-      codes_fast(v1, d1, r.z, r.w);
+      rtn_codes_signed(v0, d0, r.x, r.y);
+      rtn_codes_signed(v1, d1, r.z, r.w);
     }
-    uint32_t bad = nibble_any4(make_uint4(r.x ^ rc.x, r.y ^ rc.y, r.z ^ rc.z, r.w ^ rc.w));
-    while (bad != 0u) {
-      const int j = __ffs(bad) - 1;
-      bad &= bad - 1u;
-      const uint32_t q = ((j < 8 ? rc.x : j < 16 ? rc.y : j < 24 ? rc.z : rc.w) >> (4 * (j & 7))) & 0xFu;
-      const uint32_t fcr = site_codes_exact(src + j, j < 16 ? d0 : d1, inv, MX ? 1 : 0);
-      // one site in nibble 0; the other seven nibbles are all zero and count
-      // as distance 0
-      hist_word(fcr & 0xFu, (fcr >> 4) & 0xFu, fcr >> 8, q, ones, bins);
+    const uint32_t bad = nibble_any4(make_uint4(r.x ^ rc.x, r.y ^ rc.y, r.z ^ rc.z, r.w ^ rc.w));
+    // the pairs holding such a site, each counted whole: a site of the pair
+    // whose code agrees sits at distance 0 under every rule, which is what
+    // the count leaves to the remainder anyway
+    uint32_t pairs = (bad | (bad >> 1)) & 0x55555555u;
+    while (pairs != 0u) {
+      const int p = (__ffs(pairs) - 1) >> 1;  // 0..15: pair p & 7 of block p >> 3
+      pairs &= pairs - 1u;
+      const uint32_t q = ((p < 4 ? rc.x : p < 8 ? rc.y : p < 12 ? rc.z : rc.w) >> (8 * (p & 3))) & 0xFFu;
+      const uint32_t w = p < 8 ? pick_word(v0, p) : pick_word(v1, p & 7);
+      const float d = p < 8 ? d0 : d1;
+      uint32_t f, c, rr;
+      if (MX) {
+        mx_pair_codes(w, pk(inv, inv), f, c, rr);
+      } else if (fast_scale(d, kDMaxExactZ)) {
+        pair_codes(w, make_blk(d, 0.0f, 0.0f), f, c, rr);
+      } else {
+        const uint32_t lo = site_codes_exact(src + 2 * p, d, inv, 0);
+        const uint32_t hi = site_codes_exact(src + 2 * p + 1, d, inv, 0);
+        f = (lo & 0xFu) | ((hi & 0xFu) << 4);
+        c = ((lo >> 4) & 0xFu) | (hi & 0xF0u);
+        rr = (lo >> 8) | ((hi >> 8) << 4);
+      }
+      // the pair in the lowest byte; the other six nibbles are all zero and
+      // count as distance 0
+      hist_word(f, c, rr, q, ones, bins);
     }
   }
 #pragma unroll

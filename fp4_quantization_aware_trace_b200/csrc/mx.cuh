@@ -64,19 +64,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
-// One site of an MX guided forward recomputed one element at a time (mode
-// and side as site_exact): z = x * 2^-e is exact, the rule's code scaled
-// back by X = 2^e.  Reads the site's bf16 input at src, returns its output
-// bits.
-__device__ __noinline__ uint32_t mx_site_fix(const uint16_t* src, float inv, float X, uint32_t side,
-                                             int mode) {
-  const uint32_t xb = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(src));
-  const Exact e = exact_of_z(__fmul_rn(__uint_as_float(xb << 16), inv));
-  const int c = rule_code(e, xb, side, mode);
-  const uint32_t mag = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(e2m1_value(c), X)));
-  return (xb & 0x8000u) | mag;
-}
-
 // Round to nearest over one 16-element half of an MX block (scale 2^e given
 // as inv2 = 2^-e and X2 = 2^e): bf16 outputs, mask bits at pos0..pos0+15 of
 // m, and the codes as rtn_block (KIND 0 none, 1 magnitudes, 2 signed with
@@ -114,28 +101,59 @@ __device__ __forceinline__ void mx_rtn_block(const V8& v, u64 inv2, u64 X2, V8& 
   }
 }
 
-// One 16-element half of the MX fake-quant forward: round to nearest, then
-// (guided rules) the sites whose rule disagrees with it recomputed and
-// patched in, as fq_block_fast.  src: the half's inputs.
+// Two elements of an MX guided rule: z = x * 2^-e exact, floor and ceiling
+// by directed rounding with the unscaled grid addend, the rule's choice
+// (side as guided_pair), scaled back by X = 2^e.
 template <int MODE>
-__device__ __forceinline__ void mx_fq_half(const V8& v, const uint16_t* src, uint32_t bits16,
-                                           uint32_t r0, uint32_t r1, float inv, float X, u64 inv2,
-                                           u64 X2, V8& o, uint32_t& m, int pos0) {
+__device__ __forceinline__ uint32_t mx_guided_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2) {
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
+  const float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
+  const u64 MM = pk(grid_magic(al), grid_magic(ah));
+  const u64 aa = pk(al, ah);
+  float lol, loh, hil, hih;
+  upk(add_rm2(aa, MM), lol, loh);
+  upk(add_rp2(aa, MM), hil, hih);
+  float tl, th;
+  if (MODE == kGuided) {
+    const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+    const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+    const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+    upk(sub2(pk(sl, sh), MM), tl, th);
+  } else {
+    float fl, fh, cl, ch;
+    upk(sub2(pk(lol, loh), MM), fl, fh);
+    upk(sub2(pk(hil, hih), MM), cl, ch);
+    const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
+    float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+    rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+    tl = rl > fl ? cl : fl;
+    th = rh > fh ? ch : fh;
+  }
+  float ql, qh;
+  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+// One 16-element half of the MX fake-quant forward: round to nearest, then
+// (guided rules) the pairs holding a site where the rule disagrees with it
+// recomputed with the rule's pair routine, as fq_block_fast.
+template <int MODE>
+__device__ __forceinline__ void mx_fq_half(const V8& v, uint32_t bits16, uint32_t r0, uint32_t r1,
+                                           u64 inv2, u64 X2, V8& o, uint32_t& m, int pos0) {
   uint32_t c0, c1;
   mx_rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, inv2, X2, o, m, pos0, c0, c1);
   if (MODE == kRtn) return;
-  uint32_t bad = MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu
-                                 : nibble_any2(c0 ^ r0, c1 ^ r1);
-  while (bad != 0u) {
-    const int j = __ffs(bad) - 1;
-    bad &= bad - 1u;
-    const uint32_t side = MODE == kGuided ? (bits16 >> j) & 1u
-                                          : ((j < 8 ? r0 : r1) >> (4 * (j & 7))) & 0xFu;
-    const uint32_t val = mx_site_fix(src + j, inv, X, side, MODE);
-    const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (k == (j >> 1)) o.w[k] = (o.w[k] & keep) | (val << sh);
+  const uint32_t bad = MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu
+                                       : nibble_any2(c0 ^ r0, c1 ^ r1);
+  uint32_t pairs = (bad | (bad >> 1)) & 0x5555u;
+  while (pairs != 0u) {
+    const int p = (__ffs(pairs) - 1) >> 1;
+    pairs &= pairs - 1u;
+    const uint32_t side = MODE == kGuided ? bits16 >> (2 * p) : (p < 4 ? r0 : r1) >> (8 * (p & 3));
+    put_word(o, p, mx_guided_pair<MODE>(pick_word(v, p), side, inv2, X2));
   }
 }
 
@@ -158,13 +176,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     const int e = (int)__ldcs(scales + so) - 127;
     const float inv = pow2f(-e), X = pow2f(e);
-    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
+    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);  // 2^-e and 2^e
     uint32_t m = 0u;
     V8 o;
-    mx_fq_half<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, inv, X, inv2, X2, o, m, 0);
+    mx_fq_half<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, inv2, X2, o, m, 0);
     st_block(out + b, o);
-    mx_fq_half<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, inv, X, inv2, X2, o, m, 16);
+    mx_fq_half<MODE>(v1, bits >> 16, rc.z, rc.w, inv2, X2, o, m, 16);
     st_block(out + b + 1, o);
     mask[b >> 1] = m;
   }
@@ -250,34 +267,41 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
-// One site of a W4A8 guided forward recomputed on its own (mode 1: side =
-// the cached bit; mode 2: side = the rollout's code byte): z = x * 2^-e is
-// exact; floor and ceiling on the E4M3 grid by directed rounding with the
-// grid addend; the rule's choice scaled back by X = 2^e.  Reads the site's
-// bf16 input at src, returns its output bits.
-__device__ __noinline__ uint32_t mx8_site_fix(const uint16_t* src, float inv, float X,
-                                              uint32_t side, int mode) {
-  const uint32_t xb = (uint32_t)__ldg(reinterpret_cast<const unsigned short*>(src));
-  const float z = __fmul_rn(__uint_as_float(xb << 16), inv);
-  const float a = fminf(fabsf(z), 448.0f);  // NaN (only past 448) -> 448
-  const float M = grid_magic8(a);
-  const float lo = __fadd_rd(a, M), hi = __fadd_ru(a, M);
-  float t;
-  if (mode == 1) {
-    // of floor / ceiling, the one whose mantissa bit is the cached bit
-    const uint32_t lb = __float_as_uint(lo);
-    t = __fsub_rn(__uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hi) - lb))), M);
+// Two elements of a W4A8 guided rule: z = x * 2^-e exact, floor and ceiling
+// on the E4M3 grid by directed rounding with the grid addend, the rule's
+// choice (side: kGuided -- the two cached bits; kFull -- the rollout's two
+// code bytes, low first), scaled back by X = 2^e.
+template <int MODE>
+__device__ __forceinline__ uint32_t mx8_guided_pair(uint32_t w, uint32_t side, u64 inv2, u64 X2) {
+  float zl, zh;
+  upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
+  const float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);
+  const u64 MM = pk(grid_magic8(al), grid_magic8(ah));
+  const u64 aa = pk(al, ah);
+  float lol, loh, hil, hih;
+  upk(add_rm2(aa, MM), lol, loh);
+  upk(add_rp2(aa, MM), hil, hih);
+  float tl, th;
+  if (MODE == kGuided) {
+    const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+    const float sl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+    const float sh = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+    upk(sub2(pk(sl, sh), MM), tl, th);
   } else {
-    // of floor / ceiling, the one nearest the rollout value reflected to
-    // z's side of zero
-    const float f = __fsub_rn(lo, M), c = __fsub_rn(hi, M);
-    const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFu);
-    float r = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
-    r = __uint_as_float(__float_as_uint(r) ^ ((xb << 16) & 0x80000000u));
-    t = r > f ? c : f;
+    float fl, fh, cl, ch;
+    upk(sub2(pk(lol, loh), MM), fl, fh);
+    upk(sub2(pk(hil, hih), MM), cl, ch);
+    const uint32_t h2 = e4m3x2_to_f16x2(side & 0xFFFFu);
+    float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+    rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+    tl = rl > fl ? cl : fl;
+    th = rh > fh ? ch : fh;
   }
-  const uint32_t mag = (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(__fmul_rn(t, X)));
-  return (xb & 0x8000u) | mag;
+  float ql, qh;
+  upk(mul2(pk(tl, th), X2), ql, qh);  // exact
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
 }
 
 // One 16-element half of the W4A8 fake-quant forward: round to nearest on
@@ -286,12 +310,12 @@ __device__ __noinline__ uint32_t mx8_site_fix(const uint16_t* src, float inv, fl
 // sites whose rule disagrees with it recomputed and patched in, as
 // fq_block_fast: the 1-bit rule wherever the code's lowest bit is not the
 // cached bit, the full rule wherever the code (signed with x's sign) is not
-// the rollout's.  bits16: the cached bits; r: the rollout's 16 code bytes
-// of this half (4 words, element j in byte j).  src: the half's inputs.
+// the rollout's; the pairs holding such a site are recomputed with the
+// rule's pair routine.  bits16: the cached bits; r: the rollout's 16 code
+// bytes of this half (4 words, element j in byte j).
 template <int MODE>
-__device__ __forceinline__ void mx8_fq_half(const V8& v, const uint16_t* src, uint32_t bits16,
-                                            uint4 r, float inv, float X, u64 inv2, u64 X2, V8& o,
-                                            uint32_t& m, int pos0) {
+__device__ __forceinline__ void mx8_fq_half(const V8& v, uint32_t bits16, uint4 r, u64 inv2,
+                                            u64 X2, V8& o, uint32_t& m, int pos0) {
   uint32_t bad = 0u;
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
@@ -323,16 +347,13 @@ __device__ __forceinline__ void mx8_fq_half(const V8& v, const uint16_t* src, ui
   }
   if (MODE == kRtn) return;
   if (MODE == kGuided) bad = (bad ^ bits16) & 0xFFFFu;
-  while (bad != 0u) {
-    const int j = __ffs(bad) - 1;
-    bad &= bad - 1u;
-    const uint32_t rw = j < 4 ? r.x : j < 8 ? r.y : j < 12 ? r.z : r.w;
-    const uint32_t side = MODE == kGuided ? (bits16 >> j) & 1u : (rw >> (8 * (j & 3))) & 0xFFu;
-    const uint32_t val = mx8_site_fix(src + j, inv, X, side, MODE);
-    const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (k == (j >> 1)) o.w[k] = (o.w[k] & keep) | (val << sh);
+  uint32_t pairs = (bad | (bad >> 1)) & 0x5555u;
+  while (pairs != 0u) {
+    const int p = (__ffs(pairs) - 1) >> 1;
+    pairs &= pairs - 1u;
+    const uint32_t rw = p < 2 ? r.x : p < 4 ? r.y : p < 6 ? r.z : r.w;
+    const uint32_t side = MODE == kGuided ? bits16 >> (2 * p) : rw >> (16 * (p & 1));
+    put_word(o, p, mx8_guided_pair<MODE>(pick_word(v, p), side, inv2, X2));
   }
 }
 
@@ -355,15 +376,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
     const int e = (int)__ldcs(scales + so) - 127;
     const float inv = pow2f(-e), X = pow2f(e);
-    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
+    const u64 inv2 = pk(inv, inv), X2 = pk(X, X);  // 2^-e and 2^e
     uint32_t m = 0u;
     V8 o;
-    mx8_fq_half<MODE>(v0, src, bits & 0xFFFFu, make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]),
-                      inv, X, inv2, X2, o, m, 0);
+    mx8_fq_half<MODE>(v0, bits & 0xFFFFu, make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]), inv2, X2,
+                      o, m, 0);
     st_block(out + b, o);
-    mx8_fq_half<MODE>(v1, src + 16, bits >> 16, make_uint4(rc.w[4], rc.w[5], rc.w[6], rc.w[7]),
-                      inv, X, inv2, X2, o, m, 16);
+    mx8_fq_half<MODE>(v1, bits >> 16, make_uint4(rc.w[4], rc.w[5], rc.w[6], rc.w[7]), inv2, X2, o,
+                      m, 16);
     st_block(out + b + 1, o);
     mask[b >> 1] = m;
   }

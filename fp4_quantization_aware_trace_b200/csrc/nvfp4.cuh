@@ -382,15 +382,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // compact cache), full-information guided (the cache keeps the whole code).
 enum FqMode { kRtn = 0, kGuided = 1, kFull = 2 };
 
-// Round to nearest over one fast-path block (d in [2^-90, 2^100]): bf16
-// outputs q*s with x's sign, the 16 STE mask bits, and with KIND 1 the 16
+// Round to nearest over one fast-path block (d in [2^-90, 2^100], block
+// constants k): bf16 outputs q*s with x's sign, the 16 STE mask bits, and
+// with KIND 1 the 16
 // magnitude codes, with KIND 2 the 16 codes signed with x's sign (c0:
 // elements 0-7, c1: 8-15, element j in nibble j % 8); KIND 0 returns no
 // codes.
 template <int KIND>
-__device__ __forceinline__ void rtn_block(const V8& v, float d, float sbv, float s_g, V8& o,
-                                          uint32_t& m, uint32_t& c0, uint32_t& c1) {
-  const BlkK k = make_blk(d, sbv, s_g);
+__device__ __forceinline__ void rtn_block(const V8& v, const BlkK& k, V8& o, uint32_t& m,
+                                          uint32_t& c0, uint32_t& c1) {
   m = 0u;
   c0 = 0u;
   c1 = 0u;
@@ -438,6 +438,66 @@ __device__ __forceinline__ uint32_t nibble_any2(uint32_t c0, uint32_t c1) {
   return nibble_lsbs2(c0 | (c0 >> 2), c1 | (c1 >> 2)) & 0xFFFFu;
 }
 
+// Two elements (one bf16x2 word w) of a guided rule, for d in [2^-90, 2^16]:
+// z * 2^64 exact (|x| * 2^64 keeps every nonzero bf16's quotient and
+// remainder normal there, so "z is exactly zero" is decided exactly), floor
+// and ceiling by directed rounding with the grid addend, then the rule's
+// choice.  side: kGuided -- the two cached bits in bits 0 and 1; kFull -- the
+// rollout's two codes (low nibble first).  k: the block's constants with
+// s_b scaled by 2^-64.  Returns the pair's bf16 outputs with x's signs.
+template <int MODE>
+__device__ __forceinline__ uint32_t guided_pair(uint32_t w, uint32_t side, const BlkK& k) {
+  const u64 xx = pk(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  float zl, zh;
+  upk(quot2(mul2(xx, pk(kXs, kXs)), k), zl, zh);
+  const float al = fminf(fabsf(zl), kSixS), ah = fminf(fabsf(zh), kSixS);  // NaN -> 6 * 2^64
+  const u64 MM = MODE == kGuided ? grid_magic_s2(al, ah) : pk(grid_magic_s(al), grid_magic_s(ah));
+  const u64 aa = pk(al, ah);
+  float lol, loh, hil, hih;
+  upk(add_rm2(aa, MM), lol, loh);
+  upk(add_rp2(aa, MM), hil, hih);
+  float ql, qh;
+  if (MODE == kGuided) {
+    // of floor / ceiling, the one whose mantissa bit is the cached bit: the
+    // bits of the two sums differ by 0 (a on the grid) or 1, and the lowest
+    // bit of the floor sum is its codeword's mantissa bit
+    const uint32_t lb = __float_as_uint(lol), hb = __float_as_uint(loh);
+    const float tl = __uint_as_float(lb + ((lb ^ side) & (__float_as_uint(hil) - lb)));
+    const float th = __uint_as_float(hb + ((hb ^ (side >> 1)) & (__float_as_uint(hih) - hb)));
+    upk(mul2(mul2(sub2(pk(tl, th), MM), k.sbv2), k.sg2), ql, qh);
+  } else {
+    // of floor / ceiling, the one nearest the rollout codeword: the rollout
+    // value reflected to z's side of zero picks the ceiling exactly when it
+    // lies above the floor (no codeword lies between)
+    float fl, fh, cl, ch;
+    upk(sub2(pk(lol, loh), MM), fl, fh);
+    upk(sub2(pk(hil, hih), MM), cl, ch);
+    const uint32_t h2 = e2m1x2_to_f16x2(side & 0xFFu);
+    float rl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+    float rh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+    rl = __uint_as_float(__float_as_uint(rl) ^ ((w << 16) & 0x80000000u));
+    rh = __uint_as_float(__float_as_uint(rh) ^ (w & 0x80000000u));
+    upk(mul2(pk(rl, rh), pk(kXs, kXs)), rl, rh);
+    const float tl = rl > fl ? cl : fl;
+    const float th = rh > fh ? ch : fh;
+    upk(mul2(mul2(pk(tl, th), k.sbv2), k.sg2), ql, qh);
+  }
+  return cvt_bf16x2(ql, qh) | (w & 0x80008000u);
+}
+
+// Word p (0-7) of a block, and a block with word p replaced, by selects (no
+// indexed access, which would put the block in local memory).
+__device__ __forceinline__ uint32_t pick_word(const V8& v, int p) {
+  uint32_t w = v.w[0];
+#pragma unroll
+  for (int k = 1; k < 8; ++k) w = (p == k) ? v.w[k] : w;
+  return w;
+}
+__device__ __forceinline__ void put_word(V8& v, int p, uint32_t w) {
+#pragma unroll
+  for (int k = 0; k < 8; ++k) v.w[k] = (p == k) ? w : v.w[k];
+}
+
 // One fast-path block of the fake-quant forward: bf16 outputs in o, the 16
 // mask bits in m.  The guided rules (MODE kGuided: bits16 = the block's
 // cached bits; kFull: r0, r1 = its rollout codes, elements 0-7 and 8-15)
@@ -445,20 +505,36 @@ __device__ __forceinline__ uint32_t nibble_any2(uint32_t c0, uint32_t c1) {
 // and keep it wherever the rule agrees with it: the 1-bit rule wherever its
 // mantissa bit equals the cached bit (the bracket member with that bit, or
 // the collapsed bracket), the full rule wherever its code equals the
-// rollout's (the rollout codeword itself is then in the bracket).  At the
-// other sites -- where the training and rollout sides round differently,
-// rare for a drifted pair -- the site is recomputed on the exact path and
-// patched in.  src: the block's inputs, read there by the patch (o is
-// stored by the caller afterwards, so out may alias x).
+// rollout's (the rollout codeword itself is then in the bracket).  The pairs
+// holding a site where they disagree -- where the training and rollout sides
+// round differently, rare for a drifted pair -- are recomputed with the
+// rule's own pair routine, from registers; for d beyond 2^16 (outside that
+// routine's range) such sites go through the exact per-site path, reading
+// the block's inputs at src (o is stored by the caller afterwards, so out
+// may alias x).
 template <int MODE>
 __device__ __forceinline__ void fq_block_fast(const V8& v, const uint16_t* src, uint32_t bits16,
                                               uint32_t r0, uint32_t r1, float d, float sbv,
                                               float s_g, V8& o, uint32_t& m) {
+  BlkK k = make_blk(d, sbv, s_g);
   uint32_t c0, c1;
-  rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, d, sbv, s_g, o, m, c0, c1);
+  rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, k, o, m, c0, c1);
   if (MODE == kRtn) return;
   uint32_t bad = MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu
                                  : nibble_any2(c0 ^ r0, c1 ^ r1);
+  if (bad == 0u) return;
+  if (fast_scale(d, kDMaxExactZ)) {
+    k.sbv2 = mul2(k.sbv2, pk(0x1p-64f, 0x1p-64f));  // exact
+    uint32_t pairs = (bad | (bad >> 1)) & 0x5555u;
+    while (pairs != 0u) {
+      const int p = (__ffs(pairs) - 1) >> 1;
+      pairs &= pairs - 1u;
+      const uint32_t side = MODE == kGuided ? bits16 >> (2 * p)
+                                            : (p < 4 ? r0 : r1) >> (8 * (p & 3));
+      put_word(o, p, guided_pair<MODE>(pick_word(v, p), side, k));
+    }
+    return;
+  }
   while (bad != 0u) {
     const int j = __ffs(bad) - 1;
     bad &= bad - 1u;
@@ -466,9 +542,8 @@ __device__ __forceinline__ void fq_block_fast(const V8& v, const uint16_t* src, 
                                           : ((j < 8 ? r0 : r1) >> (4 * (j & 7))) & 0xFu;
     const uint32_t val = guided_site_fix(src + j, d, sbv, s_g, side, MODE);
     const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
-#pragma unroll
-    for (int k = 0; k < 8; ++k)
-      if (k == (j >> 1)) o.w[k] = (o.w[k] & keep) | (val << sh);
+    const int p = j >> 1;
+    put_word(o, p, (pick_word(o, p) & keep) | (val << sh));
   }
 }
 
