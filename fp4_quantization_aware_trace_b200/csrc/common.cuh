@@ -239,11 +239,20 @@ __device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// max|x| over a block as bf16 bits (integer order = magnitude order).
+// Per half, max(|a|, |b|) of two bf16 pairs (the sign bit of each half is
+// the xor of the inputs' signs; callers clear it).
+__device__ __forceinline__ uint32_t absmax2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+// max|x| over a block as bf16 bits (integer order = magnitude order): a tree
+// of magnitude maxima over the 8 words, then the larger half.
 __device__ __forceinline__ uint32_t absmax_block(const V8& v) {
-  uint32_t m = __vmaxu2(v.w[0] & 0x7FFF7FFFu, v.w[1] & 0x7FFF7FFFu);
-#pragma unroll
-  for (int k = 2; k < 8; ++k) m = __vmaxu2(m, v.w[k] & 0x7FFF7FFFu);
+  const uint32_t m = absmax2(absmax2(absmax2(v.w[0], v.w[1]), absmax2(v.w[2], v.w[3])),
+                             absmax2(absmax2(v.w[4], v.w[5]), absmax2(v.w[6], v.w[7]))) &
+                     0x7FFF7FFFu;
   return max(m & 0xFFFFu, m >> 16);
 }
 
@@ -277,6 +286,24 @@ __device__ __forceinline__ BlkK make_blk(float d, float sbv, float s_g) {
   k.sbv2 = pk(sbv, sbv);
   k.sg2 = pk(s_g, s_g);
   return k;
+}
+
+// STE mask bit of a quotient z >= 0 as a float, on the FMA pipe: 1.0 where
+// z <= 6, else 0.0 (NaN and infinity included).  z * -2^100 + (6 * 2^100 +
+// 2^79) is rounded once: it is 2^79 at z = 6, at most 0 from the next float
+// past 6 (6 + 2^-21) on, and the saturation maps it (NaN included) to 0 or 1.
+__device__ __forceinline__ float le6_step(float z) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(z), "f"(-0x1p100f), "f"(0x1.800002p102f));
+  return r;
+}
+
+// The same for the W4A8 mask, z <= 448: 448 * 2^100 + 2^85 (448 = 1.75 * 2^8,
+// and 2^85 is the spacing of floats at 448 * 2^100).
+__device__ __forceinline__ float le448_step(float z) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(z), "f"(-0x1p100f), "f"(0x1.c00002p108f));
+  return r;
 }
 
 // 0xFFFFFFFF when a <= b (false for NaN), else 0.

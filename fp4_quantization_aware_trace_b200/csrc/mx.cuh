@@ -71,16 +71,20 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 template <int KIND>
 __device__ __forceinline__ void mx_rtn_block(const V8& v, u64 inv2, u64 X2, V8& o, uint32_t& m,
                                              int pos0, uint32_t& c0, uint32_t& c1) {
+  // z = |x| * 2^-e (the sign is put back on the output); the mask bits are
+  // accumulated on the FMA pipe as rtn_block does
+  u64 mf = pk(0.0f, 0.0f);
+  const u64 four = pk(4.0f, 4.0f);
   c0 = 0u;
   c1 = 0u;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
+  for (int p = 7; p >= 0; --p) {
     const uint32_t w = v.w[p];
     float zl, zh;
-    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);  // exact z (inf only past 6)
-    m |= (le_mask(fabsf(zl), 6.0f) & (1u << (pos0 + 2 * p))) |
-         (le_mask(fabsf(zh), 6.0f) & (2u << (pos0 + 2 * p)));
-    float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);
+    upk(mul2(pk(__uint_as_float((w & 0x7FFFu) << 16), __uint_as_float(w & 0x7FFF0000u)), inv2),
+        zl, zh);  // exact z >= 0 (inf only past 6)
+    mf = fma2(mf, four, pk(le6_step(zl), le6_step(zh)));
+    float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);
     uint32_t h2;
     if (KIND == 0) {
       h2 = rtn_e2m1x2_f16x2(al, ah);
@@ -91,7 +95,7 @@ __device__ __forceinline__ void mx_rtn_block(const V8& v, u64 inv2, u64 X2, V8& 
       }
       uint32_t code;
       h2 = rtn_e2m1x2_f16x2_code(al, ah, code);
-      if (p < 4) c0 |= code << (8 * p); else c1 |= code << (8 * (p - 4));
+      if (p < 4) c0 += code << (8 * p); else c1 += code << (8 * (p - 4));
     }
     const float tl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
     const float th = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
@@ -99,6 +103,9 @@ __device__ __forceinline__ void mx_rtn_block(const V8& v, u64 inv2, u64 X2, V8& 
     upk(mul2(pk(tl, th), X2), ql, qh);  // exact
     o.w[p] = cvt_bf16x2(ql, qh) | (w & 0x80008000u);
   }
+  float ml, mh;
+  upk(mf, ml, mh);
+  m |= __float2uint_rn(__fmaf_rn(mh, 2.0f, ml)) << pos0;
 }
 
 // Two elements of an MX guided rule: z = x * 2^-e exact, floor and ceiling
@@ -317,14 +324,16 @@ template <int MODE>
 __device__ __forceinline__ void mx8_fq_half(const V8& v, uint32_t bits16, uint4 r, u64 inv2,
                                             u64 X2, V8& o, uint32_t& m, int pos0) {
   uint32_t bad = 0u;
+  u64 mf = pk(0.0f, 0.0f);
+  const u64 four = pk(4.0f, 4.0f);
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
+  for (int p = 7; p >= 0; --p) {
     const uint32_t w = v.w[p];
     float zl, zh;
-    upk(mul2(pk(bf16_lo(w), bf16_hi(w)), inv2), zl, zh);
-    m |= (le_mask(fabsf(zl), 448.0f) & (1u << (pos0 + 2 * p))) |
-         (le_mask(fabsf(zh), 448.0f) & (2u << (pos0 + 2 * p)));
-    float al = fminf(fabsf(zl), 448.0f), ah = fminf(fabsf(zh), 448.0f);  // NaN -> 448
+    upk(mul2(pk(__uint_as_float((w & 0x7FFFu) << 16), __uint_as_float(w & 0x7FFF0000u)), inv2),
+        zl, zh);  // exact z >= 0 (inf only past 448)
+    mf = fma2(mf, four, pk(le448_step(zl), le448_step(zh)));
+    float al = fminf(zl, 448.0f), ah = fminf(zh, 448.0f);
     if (MODE == kFull) {
       al = __uint_as_float(__float_as_uint(al) | ((w << 16) & 0x80000000u));
       ah = __uint_as_float(__float_as_uint(ah) | (w & 0x80000000u));
@@ -345,6 +354,9 @@ __device__ __forceinline__ void mx8_fq_half(const V8& v, uint32_t bits16, uint4 
     upk(mul2(pk(tl, th), X2), ql, qh);  // exact
     o.w[p] = cvt_bf16x2(ql, qh) | (w & 0x80008000u);
   }
+  float ml, mh;
+  upk(mf, ml, mh);
+  m |= __float2uint_rn(__fmaf_rn(mh, 2.0f, ml)) << pos0;
   if (MODE == kRtn) return;
   if (MODE == kGuided) bad = (bad ^ bits16) & 0xFFFFu;
   uint32_t pairs = (bad | (bad >> 1)) & 0x5555u;

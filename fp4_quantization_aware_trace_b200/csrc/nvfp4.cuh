@@ -319,14 +319,38 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
               uint32_t* amax, uint4* __restrict__ codes, uint32_t* __restrict__ mbits,
               uint8_t* __restrict__ scales, float* __restrict__ gscale) {
+  __shared__ uint32_t amax_s, last_s;
   pdl_begin();
-  // global scales of all groups (any CTA may write them; all write the same)
-  for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
-    gscale[g] = group_consts(__ldcg(amax + g)).s_g;
-
   GroupCursor gc;
   gc.init(offs, sh.G);
   GroupK gk = group_consts(0u);
+  const bool one = sh.G == 1;
+  if (one) {
+    // a single group: thread 0 reads the accumulator once for the CTA and,
+    // with RESET, then takes its ticket (acquire-release, before this CTA
+    // has written anything); the CTA drawing the last ticket -- every CTA
+    // has read the accumulator by then -- zeroes it and the ticket
+    if (threadIdx.x == 0) {
+      const uint32_t a = __ldcg(amax);
+      amax_s = a;
+      if (blockIdx.x == 0) gscale[0] = group_consts(a).s_g;
+      if (RESET) {
+        uint32_t t;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(amax + 1) : "memory");
+        if (t == gridDim.x - 1u) {
+          amax[0] = 0u;
+          amax[1] = 0u;
+        }
+      }
+    }
+    __syncthreads();
+    gk = group_consts(amax_s);
+    gc.seek(0u);
+  } else {
+    // global scales of all groups (any CTA may write them; all write the same)
+    for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
+      gscale[g] = group_consts(__ldcg(amax + g)).s_g;
+  }
 
   // tiles in reverse order: k_amax read the high tiles last, so they are the
   // most likely to be still in L2
@@ -358,8 +382,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     else
       reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
   }
-  if (RESET) {
-    __shared__ uint32_t last_s;
+  if (RESET && !one) {
+    // groups: the CTAs read the accumulators as their rows change group, so
+    // each takes its ticket at the end, after a fence
     __syncthreads();  // this CTA's reads of the accumulators are done
     if (threadIdx.x == 0) {
       __threadfence();
@@ -391,16 +416,22 @@ enum FqMode { kRtn = 0, kGuided = 1, kFull = 2 };
 template <int KIND>
 __device__ __forceinline__ void rtn_block(const V8& v, const BlkK& k, V8& o, uint32_t& m,
                                           uint32_t& c0, uint32_t& c1) {
-  m = 0u;
+  // the quotient is taken of |x| (the sign is put back on the output), and
+  // the mask bits are accumulated on the FMA pipe as a float, Horner style
+  // from the last pair down: bit 2p of mf.lo, bit 2p of mf.hi (element
+  // 2p + 1) -- exact, every partial sum stays below 2^16
+  u64 mf = pk(0.0f, 0.0f);
+  const u64 four = pk(4.0f, 4.0f);
   c0 = 0u;
   c1 = 0u;
 #pragma unroll
-  for (int p = 0; p < 8; ++p) {
+  for (int p = 7; p >= 0; --p) {
     const uint32_t w = v.w[p];
     float zl, zh;
-    upk(quot2(pk(bf16_lo(w), bf16_hi(w)), k), zl, zh);
-    m |= (le_mask(fabsf(zl), 6.0f) & (1u << (2 * p))) | (le_mask(fabsf(zh), 6.0f) & (2u << (2 * p)));
-    float al = fminf(fabsf(zl), 6.0f), ah = fminf(fabsf(zh), 6.0f);  // NaN -> 6
+    upk(quot2(pk(__uint_as_float((w & 0x7FFFu) << 16), __uint_as_float(w & 0x7FFF0000u)), k),
+        zl, zh);  // z >= 0; NaN where |x| / d overflows
+    mf = fma2(mf, four, pk(le6_step(zl), le6_step(zh)));
+    float al = fminf(zl, 6.0f), ah = fminf(zh, 6.0f);  // NaN -> 6
     uint32_t h2;
     if (KIND == 0) {
       // round to nearest on the grid (ties to the even code), decoded
@@ -412,7 +443,7 @@ __device__ __forceinline__ void rtn_block(const V8& v, const BlkK& k, V8& o, uin
       }
       uint32_t code;
       h2 = rtn_e2m1x2_f16x2_code(al, ah, code);
-      if (p < 4) c0 |= code << (8 * p); else c1 |= code << (8 * (p - 4));
+      if (p < 4) c0 += code << (8 * p); else c1 += code << (8 * (p - 4));
     }
     const float vl = __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
     const float vh = __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
@@ -420,6 +451,9 @@ __device__ __forceinline__ void rtn_block(const V8& v, const BlkK& k, V8& o, uin
     upk(mul2(mul2(pk(vl, vh), k.sbv2), k.sg2), ql, qh);
     o.w[p] = cvt_bf16x2(ql, qh) | (w & 0x80008000u);
   }
+  float ml, mh;
+  upk(mf, ml, mh);
+  m = __float2uint_rn(__fmaf_rn(mh, 2.0f, ml));
 }
 
 // Lowest bit of each of the 16 nibbles of (c0, c1) in bits 0-15 (bit j =
