@@ -546,17 +546,24 @@ __device__ __forceinline__ void put_word(V8& v, int p, uint32_t w) {
 // routine's range) such sites go through the exact per-site path, reading
 // the block's inputs at src (o is stored by the caller afterwards, so out
 // may alias x).
+// The round-to-nearest pass of fq_block_fast alone: outputs and mask, and
+// the returned bits of the sites where the block's rule disagrees with it.
+template <int MODE>
+__device__ __forceinline__ uint32_t fq_block_rtn(const V8& v, uint32_t bits16, uint32_t r0,
+                                                 uint32_t r1, const BlkK& k, V8& o, uint32_t& m) {
+  uint32_t c0, c1;
+  rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, k, o, m, c0, c1);
+  if (MODE == kRtn) return 0u;
+  return MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu : nibble_any2(c0 ^ r0, c1 ^ r1);
+}
+
 template <int MODE>
 __device__ __forceinline__ void fq_block_fast(const V8& v, const uint16_t* src, uint32_t bits16,
                                               uint32_t r0, uint32_t r1, float d, float sbv,
                                               float s_g, V8& o, uint32_t& m) {
   BlkK k = make_blk(d, sbv, s_g);
-  uint32_t c0, c1;
-  rtn_block<MODE == kRtn ? 0 : MODE == kGuided ? 1 : 2>(v, k, o, m, c0, c1);
-  if (MODE == kRtn) return;
-  uint32_t bad = MODE == kGuided ? (nibble_lsbs2(c0, c1) ^ bits16) & 0xFFFFu
-                                 : nibble_any2(c0 ^ r0, c1 ^ r1);
-  if (bad == 0u) return;
+  uint32_t bad = fq_block_rtn<MODE>(v, bits16, r0, r1, k, o, m);
+  if (MODE == kRtn || bad == 0u) return;
   if (fast_scale(d, kDMaxExactZ)) {
     k.sbv2 = mul2(k.sbv2, pk(0x1p-64f, 0x1p-64f));  // exact
     uint32_t pairs = (bad | (bad >> 1)) & 0x5555u;
@@ -578,6 +585,28 @@ __device__ __forceinline__ void fq_block_fast(const V8& v, const uint16_t* src, 
     const uint32_t sh = 16u * (uint32_t)(j & 1), keep = 0xFFFF0000u >> sh;
     const int p = j >> 1;
     put_word(o, p, (pick_word(o, p) & keep) | (val << sh));
+  }
+}
+
+// Pair q (0-15) of a thread's two blocks recomputed with its guided rule
+// and stored over the round-to-nearest word already written at out: the
+// variant for outputs that do not alias the inputs, so the pair's input word
+// is read back from x (a cache hit: the block was just read) instead of kept
+// in registers.  d, sbv: the pair's block; side as guided_pair (MODE kGuided:
+// the pair's two cached bits in bits 0 and 1; kFull: its two rollout codes).
+template <int MODE>
+__device__ __forceinline__ void patch_pair(const uint32_t* xw, uint32_t* ow, int q, float d,
+                                           float sbv, float s_g, uint32_t side) {
+  if (fast_scale(d, kDMaxExactZ)) {
+    ow[q] = guided_pair<MODE>(__ldg(xw + q), side, make_blk(d, __fmul_rn(sbv, 0x1p-64f), s_g));
+  } else {
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(xw + q);
+    const uint32_t lo = guided_site_fix(src, d, sbv, s_g, MODE == kGuided ? side & 1u : side & 0xFu,
+                                        MODE);
+    const uint32_t hi = guided_site_fix(src + 1, d, sbv, s_g,
+                                        MODE == kGuided ? (side >> 1) & 1u : (side >> 4) & 0xFu,
+                                        MODE);
+    ow[q] = lo | (hi << 16);
   }
 }
 
@@ -613,7 +642,10 @@ __device__ __forceinline__ uint32_t fake_quant_block(const V8& v, const V8* src,
 // tensors: each thread then walks several tiles, and with the larger register
 // budget it ran 16% faster on B200 at 268M elements (and 13% slower at 33M,
 // where a thread sees one tile).
-template <int MODE, bool SW, int MINB = kCtasPerSm>
+// SEP: out does not alias x.  The guided rules then write both blocks'
+// round-to-nearest outputs first and recompute the pairs that need it in one
+// loop for the thread's 32 elements, reading their inputs back from x.
+template <int MODE, bool SW, int MINB = kCtasPerSm, bool SEP = false>
 __global__ void __launch_bounds__(kThreads, MINB)
     k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
                  const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
@@ -642,7 +674,27 @@ __global__ void __launch_bounds__(kThreads, MINB)
     // a row holds a whole number of 32-element words, so both blocks of the
     // pair are in the same row and group
     const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
-    if (fast_scale(d0) && fast_scale(d1)) {
+    if (SEP && MODE != kRtn && fast_scale(d0) && fast_scale(d1)) {
+      // the common case for separate output buffers
+      V8 o;
+      const uint32_t bad0 =
+          fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, make_blk(d0, sbv0, s_g), o, m0);
+      st_block(out + b, o);
+      const uint32_t bad1 =
+          fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, make_blk(d1, sbv1, s_g), o, m1);
+      st_block(out + b + 1, o);
+      uint32_t pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
+      uint32_t* ow = reinterpret_cast<uint32_t*>(out + b);
+      while (pairs != 0u) {
+        const int q = (__ffs(pairs) - 1) >> 1;  // pair q & 7 of block q >> 3
+        pairs &= pairs - 1u;
+        const uint32_t side =
+            MODE == kGuided ? bits >> (2 * q)
+                            : (q < 4 ? rc.x : q < 8 ? rc.y : q < 12 ? rc.z : rc.w) >> (8 * (q & 3));
+        patch_pair<MODE>(xw, ow, q, q < 8 ? d0 : d1, q < 8 ? sbv0 : sbv1, s_g, side);
+      }
+    } else if (fast_scale(d0) && fast_scale(d1)) {
       // the common case, without per-block branches
       V8 o;
       const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);

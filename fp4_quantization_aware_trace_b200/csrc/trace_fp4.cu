@@ -139,20 +139,31 @@ int launch(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
                                                                                       : TRACE_ERR_CUDA;
 }
 
+// The guided rules: SEP when out does not overlap x (see k_fake_quant).
+template <int MODE, bool SW>
+int guided_dispatch(bool sep, int grid, cudaStream_t s, const uint16_t* x, const Shape& sh,
+                    const int64_t* o, const uint32_t* mbits, const uint8_t* rcodes,
+                    const uint8_t* scales, const float* gscale, uint16_t* out, uint32_t* mask) {
+  if (sep)
+    return launch(k_fake_quant<MODE, SW, kCtasPerSm, true>, grid, s, (const V8*)x, sh, o, mbits,
+                  (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
+  return launch(k_fake_quant<MODE, SW, kCtasPerSm, false>, grid, s, (const V8*)x, sh, o, mbits,
+                (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
+}
+
 template <bool SW>
 int fake_quant_dispatch(int mode, int grid, cudaStream_t s, const uint16_t* x,
                                const Shape& sh, const int64_t* o, const uint32_t* mbits,
                                const uint8_t* rcodes, const uint8_t* scales, const float* gscale,
                                uint16_t* out, uint32_t* mask) {
+  const size_t bytes = (size_t)sh.nblk * 32u;
+  const bool sep = (uintptr_t)out + bytes <= (uintptr_t)x || (uintptr_t)x + bytes <= (uintptr_t)out;
   if (mode == kGuided)
-    return launch(k_fake_quant<kGuided, SW>, grid, s, (const V8*)x, sh, o, mbits,
-                  (const uint4*)nullptr, scales, gscale, (V8*)out, mask);
-  if (mode == kFull && sh.ntiles >= 4u * (uint32_t)grid)  // at least 4 tiles per CTA
-    return launch(k_fake_quant<kFull, SW, 2>, grid, s, (const V8*)x, sh, o,
-                  (const uint32_t*)nullptr, (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
+    return guided_dispatch<kGuided, SW>(sep, grid, s, x, sh, o, mbits, nullptr, scales, gscale,
+                                        out, mask);
   if (mode == kFull)
-    return launch(k_fake_quant<kFull, SW>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
-                  (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
+    return guided_dispatch<kFull, SW>(sep, grid, s, x, sh, o, nullptr, rcodes, scales, gscale, out,
+                                      mask);
   return launch(k_fake_quant<kRtn, SW>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
                 (const uint4*)nullptr, scales, gscale, (V8*)out, mask);
 }
