@@ -325,23 +325,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   gc.init(offs, sh.G);
   GroupK gk = group_consts(0u);
   const bool one = sh.G == 1;
+  // tiles in reverse order: k_amax read the high tiles last, so they are the
+  // most likely to be still in L2.  The first tile's loads go out before
+  // the CTA's set-up below.
+  uint32_t i = blockIdx.x;
+  auto tile_base = [&](uint32_t k) { return (sh.ntiles - 1u - k) * kTileBlks + 2u * threadIdx.x; };
+  V8 v0 = zero_block(), v1 = zero_block();
+  if (i < sh.ntiles && tile_base(i) < sh.nblk) {
+    v0 = ld_block_stream(x + tile_base(i));
+    v1 = ld_block_stream(x + tile_base(i) + 1);
+  }
+  uint32_t ticket = 0u;
   if (one) {
     // a single group: thread 0 reads the accumulator once for the CTA and,
-    // with RESET, then takes its ticket (acquire-release, before this CTA
-    // has written anything); the CTA drawing the last ticket -- every CTA
-    // has read the accumulator by then -- zeroes it and the ticket
+    // with RESET, then takes its ticket with a release add (ordering that
+    // read before it; the result is looked at only at the end of the CTA).
+    // The CTA that drew the last ticket -- every CTA has read the
+    // accumulator by then -- zeroes it and the ticket after an acquire fence.
     if (threadIdx.x == 0) {
       const uint32_t a = __ldcg(amax);
       amax_s = a;
       if (blockIdx.x == 0) gscale[0] = group_consts(a).s_g;
-      if (RESET) {
-        uint32_t t;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(amax + 1) : "memory");
-        if (t == gridDim.x - 1u) {
-          amax[0] = 0u;
-          amax[1] = 0u;
-        }
-      }
+      if (RESET)
+        asm volatile("atom.release.gpu.global.add.u32 %0, [%1], 1;"
+                     : "=r"(ticket)
+                     : "l"(amax + 1)
+                     : "memory");
     }
     __syncthreads();
     gk = group_consts(amax_s);
@@ -352,35 +361,42 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       gscale[g] = group_consts(__ldcg(amax + g)).s_g;
   }
 
-  // tiles in reverse order: k_amax read the high tiles last, so they are the
-  // most likely to be still in L2
-  for (uint32_t i = blockIdx.x; i < sh.ntiles; i += gridDim.x) {
-    const uint32_t t = sh.ntiles - 1u - i;
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    // both blocks of the pair are in the same row (cols is a multiple of 32)
-    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-    if (gc.seek(row)) gk = group_consts(__ldcg(amax + gc.g));
-    const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
-    float sb0, sb1;
-    e4m3x2_to_f32(s2, sb0, sb1);
-    const float d0 = __fmul_rn(gk.s_g, sb0), d1 = __fmul_rn(gk.s_g, sb1);
-    uint4 c;
-    if (fast_scale(d0) && fast_scale(d1)) {  // the common case, without per-block branches
-      codes_fast(v0, d0, c.x, c.y);
-      codes_fast(v1, d1, c.z, c.w);
-    } else {
-      codes_block(v0, x + b, d0, c.x, c.y);
-      codes_block(v1, x + b + 1, d1, c.z, c.w);
+  for (; i < sh.ntiles; i += gridDim.x) {
+    const uint32_t b = tile_base(i);  // even; nblk is even
+    const uint32_t inext = i + gridDim.x;
+    if (b < sh.nblk) {
+      // both blocks of the pair are in the same row (cols is a multiple of 32)
+      const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+      if (gc.seek(row)) gk = group_consts(__ldcg(amax + gc.g));
+      const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
+      float sb0, sb1;
+      e4m3x2_to_f32(s2, sb0, sb1);
+      const float d0 = __fmul_rn(gk.s_g, sb0), d1 = __fmul_rn(gk.s_g, sb1);
+      uint4 c;
+      if (fast_scale(d0) && fast_scale(d1)) {  // the common case, without per-block branches
+        codes_fast(v0, d0, c.x, c.y);
+        codes_fast(v1, d1, c.z, c.w);
+      } else {
+        codes_block(v0, x + b, d0, c.x, c.y);
+        codes_block(v1, x + b + 1, d1, c.z, c.w);
+      }
+      codes[b >> 1] = c;
+      mbits[b >> 1] = nibble_lsbs4(c);
+      const uint16_t sv = (uint16_t)s2;
+      if (SW)  // the pair's two columns are neighbours inside one tile
+        *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
+      else
+        reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
     }
-    codes[b >> 1] = c;
-    mbits[b >> 1] = nibble_lsbs4(c);
-    const uint16_t sv = (uint16_t)s2;
-    if (SW)  // the pair's two columns are neighbours inside one tile
-      *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
-    else
-      reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
+    if (inext < sh.ntiles && tile_base(inext) < sh.nblk) {
+      v0 = ld_block_stream(x + tile_base(inext));
+      v1 = ld_block_stream(x + tile_base(inext) + 1);
+    }
+  }
+  if (RESET && one && threadIdx.x == 0 && ticket == gridDim.x - 1u) {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    amax[0] = 0u;
+    amax[1] = 0u;
   }
   if (RESET && !one) {
     // groups: the CTAs read the accumulators as their rows change group, so
