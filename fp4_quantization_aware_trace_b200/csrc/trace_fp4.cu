@@ -198,11 +198,19 @@ int mx8_launch(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* mb
   sh.sw_ct = (uint32_t)((cols / 32 + 3) / 4);
   int grid;
   if ((st = grid_for(sh, &grid))) return st;
+  const size_t bytes = (size_t)sh.nblk * 32u;
+  const bool sep = MODE != kRtn && ((uintptr_t)out + bytes <= (uintptr_t)x ||
+                                    (uintptr_t)x + bytes <= (uintptr_t)out);
+  cudaStream_t s = (cudaStream_t)stream;
   if (tiled)
-    return launch(k_mx8_fake_quant<MODE, true>, grid, (cudaStream_t)stream, (const V8*)x, sh,
-                  mbits, (const V8*)rcodes, scales, (V8*)out, mask);
-  return launch(k_mx8_fake_quant<MODE, false>, grid, (cudaStream_t)stream, (const V8*)x, sh, mbits,
-                (const V8*)rcodes, scales, (V8*)out, mask);
+    return sep ? launch(k_mx8_fake_quant<MODE, true, true>, grid, s, (const V8*)x, sh, mbits,
+                        (const V8*)rcodes, scales, (V8*)out, mask)
+               : launch(k_mx8_fake_quant<MODE, true, false>, grid, s, (const V8*)x, sh, mbits,
+                        (const V8*)rcodes, scales, (V8*)out, mask);
+  return sep ? launch(k_mx8_fake_quant<MODE, false, true>, grid, s, (const V8*)x, sh, mbits,
+                      (const V8*)rcodes, scales, (V8*)out, mask)
+             : launch(k_mx8_fake_quant<MODE, false, false>, grid, s, (const V8*)x, sh, mbits,
+                      (const V8*)rcodes, scales, (V8*)out, mask);
 }
 
 }  // namespace

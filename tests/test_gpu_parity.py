@@ -582,3 +582,44 @@ def test_copy_yardsticks_copy_every_byte(numel):
         assert torch.equal(dst.view(torch.int16), src.view(torch.int16)), staged
         if staged:
             assert int(err.item()) == 0
+
+
+@pytest.mark.parametrize("drift", ["drifted", "independent"])
+def test_guided_rules_in_place_and_separate_vs_oracle(oracle_mod, drift):
+    """Every guided rule of every format, written to a separate buffer (the
+    forwards then recompute disagreeing pairs after storing round to
+    nearest) and in place over x_train (they patch each block in registers),
+    against the oracle.  Independent training values make most sites
+    disagree with the rollout, so the recompute paths carry most of the
+    work; drifted ones exercise the common sparse case."""
+    s = inputs.tiny_site(611, 640, 256, eps=0.02)
+    xr = s.x_roll
+    xt = s.x_train if drift == "drifted" else inputs.tiny_site(612, 640, 256).x_roll
+    hr, ht = inputs.bits(xr), inputs.bits(xt)
+    xr_d, xt_d = xr.to(DEV), xt.to(DEV)
+    codes, mbits, scales, gscale = oracle_mod.capture(hr)
+    c4, b4, s4 = oracle_mod.mx_capture(hr)
+    c8, b8, s8 = oracle_mod.mx8_capture(hr)
+    cases = {
+        "nvfp4 guided": (lambda x, o: ops.guided_fq_fwd(x, ops.capture(xr_d), out=o),
+                         oracle_mod.guided_fwd(ht, mbits, scales, gscale)),
+        "nvfp4 full": (lambda x, o: ops.full_guided_fq_fwd(x, ops.capture(xr_d), out=o),
+                       oracle_mod.full_guided_fwd(ht, codes, scales, gscale)),
+        "mxfp4 guided": (lambda x, o: ops.mx_guided_fq_fwd(x, ops.mx_capture(xr_d), out=o),
+                         oracle_mod.mx_guided_fwd(ht, b4, s4)),
+        "mxfp4 full": (lambda x, o: ops.mx_full_guided_fq_fwd(x, ops.mx_capture(xr_d), out=o),
+                       oracle_mod.mx_full_guided_fwd(ht, c4, s4)),
+        "w4a8 guided": (lambda x, o: ops.mx8_guided_fq_fwd(x, ops.mx8_capture(xr_d), out=o),
+                        oracle_mod.mx8_guided_fwd(ht, b8, s8)),
+        "w4a8 full": (lambda x, o: ops.mx8_full_guided_fq_fwd(x, ops.mx8_capture(xr_d), out=o),
+                      oracle_mod.mx8_full_guided_fwd(ht, c8, s8)),
+    }
+    for name, (fn, (ref_out, ref_mask)) in cases.items():
+        sep_out, sep_mask = fn(xt_d, torch.empty_like(xt_d))
+        buf = xt_d.clone()
+        inp_out, inp_mask = fn(buf, buf)
+        torch.cuda.synchronize()
+        _eq(f"{name} separate out", _u(sep_out), ref_out)
+        _eq(f"{name} separate mask", _u(sep_mask), ref_mask)
+        _eq(f"{name} in-place out", _u(buf), ref_out)
+        _eq(f"{name} in-place mask", _u(inp_mask), ref_mask)
