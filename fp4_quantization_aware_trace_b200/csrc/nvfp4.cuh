@@ -309,17 +309,17 @@ __device__ __forceinline__ void codes_block(const V8& v, const V8* src, float d,
 // Each thread owns two adjacent blocks: one 16-byte store of codes, one
 // 32-bit store of mantissa bits, one 16-bit store of scales.
 // SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
-// RESET: `amax` is the call's workspace (G accumulators, then a ticket
-// counter at amax[G]); the last CTA to finish -- the one that draws ticket
-// gridDim.x - 1, after every other CTA has read the accumulators it needed
-// -- sets the accumulators and the ticket back to zero, so the next capture
-// with the same workspace needs no zeroing launch.  Nothing waits.
+// RESET (a single group only): `amax` is the call's workspace (the
+// accumulator, then a ticket counter); the CTA that draws the last ticket --
+// after every CTA has read the accumulator -- sets both back to zero, so the
+// next capture with the same workspace needs no zeroing launch.  Nothing
+// waits.
 template <bool SW, bool RESET>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
               uint32_t* amax, uint4* __restrict__ codes, uint32_t* __restrict__ mbits,
               uint8_t* __restrict__ scales, float* __restrict__ gscale) {
-  __shared__ uint32_t amax_s, last_s;
+  __shared__ uint32_t amax_s;
   pdl_begin();
   GroupCursor gc;
   gc.init(offs, sh.G);
@@ -397,20 +397,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     asm volatile("fence.acq_rel.gpu;" ::: "memory");
     amax[0] = 0u;
     amax[1] = 0u;
-  }
-  if (RESET && !one) {
-    // groups: the CTAs read the accumulators as their rows change group, so
-    // each takes its ticket at the end, after a fence
-    __syncthreads();  // this CTA's reads of the accumulators are done
-    if (threadIdx.x == 0) {
-      __threadfence();
-      last_s = atomicAdd(amax + sh.G, 1u) == gridDim.x - 1u;
-    }
-    __syncthreads();
-    if (last_s) {
-      __threadfence();
-      for (int g = threadIdx.x; g <= sh.G; g += kThreads) amax[g] = 0u;
-    }
   }
 }
 

@@ -254,7 +254,9 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
 
 // zero_first: zero the workspace with a launch of its own before the amax
 // pass (the static-scratch entry point, whose array other calls share);
-// otherwise the workspace holds zeros on entry, as every capture leaves it.
+// otherwise the workspace holds zeros on entry, as every capture leaves it:
+// a single group's quantising pass resets it as it goes (a ticket), and for
+// groups a third launch zeroes it after the quantising pass.
 static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                         const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
                         uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
@@ -275,15 +277,24 @@ static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t n
   cudaStream_t s = (cudaStream_t)stream;
   uint32_t* amax = (uint32_t*)workspace;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
-  if (zero_first) {
-    const int zg = (num_groups + 1 + kThreads - 1) / kThreads;
-    if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups + 1))) return st;
-  }
+  const int zg = (num_groups + 1 + kThreads - 1) / kThreads;
+  if (zero_first &&
+      (st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups + 1)))
+    return st;
   if (sh.nblk > 0 && (st = launch(k_amax, grid, s, (const V8*)x, sh, offs, amax))) return st;
-  st = tiled ? launch(k_capture<true, true>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes,
-                      (uint32_t*)mbits, scales, gscale)
-             : launch(k_capture<false, true>, grid, s, (const V8*)x, sh, offs, amax,
-                      (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+  if (num_groups == 1) {
+    st = tiled ? launch(k_capture<true, true>, grid, s, (const V8*)x, sh, offs, amax,
+                        (uint4*)codes, (uint32_t*)mbits, scales, gscale)
+               : launch(k_capture<false, true>, grid, s, (const V8*)x, sh, offs, amax,
+                        (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+  } else {
+    st = tiled ? launch(k_capture<true, false>, grid, s, (const V8*)x, sh, offs, amax,
+                        (uint4*)codes, (uint32_t*)mbits, scales, gscale)
+               : launch(k_capture<false, false>, grid, s, (const V8*)x, sh, offs, amax,
+                        (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+    if (st == TRACE_OK)
+      st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups + 1);
+  }
   // a failed launch would leave the accumulators set: clear them (best effort)
   if (st != TRACE_OK) (void)cudaMemsetAsync(workspace, 0, ((size_t)num_groups + 1) * 4u, s);
   return st;
