@@ -14,6 +14,7 @@ constexpr int kTileBlks = kThreads * kBlkPerThread;  // 512 blocks = 8192 elemen
 constexpr int kCtasPerSm = 4;    // resident CTAs per SM the register budget allows
 constexpr int kGridPerSm = 32;   // CTAs launched per SM: about one tile each
 constexpr int kAmaxTable = 256;  // groups per CTA kept in shared memory
+constexpr int kAmaxCtasPerSm = 4;  // the amax pass: a persistent grid of this many CTAs per SM
 
 constexpr uint32_t kDMin = 0x12800000u;     // 2^-90: fast paths need d >= 2^-90
 constexpr uint32_t kDMax = 0x71800000u;     // 2^100: capture / round-to-nearest

@@ -124,103 +124,25 @@ __device__ __noinline__ uint32_t guided_site_fix(const uint16_t* src, float d, f
                     side, mode, in);
 }
 
+// Both sites of a pair (bf16x2 word w) on the exact path: output bits with
+// x's signs.  side as guided_pair below (mode 1: the two cached bits in bits
+// 0 and 1; mode 2: the two rollout codes, low nibble first).
+__device__ __noinline__ uint32_t guided_word_exact(uint32_t w, float d, float sbv, float s_g,
+                                                   uint32_t side, int mode) {
+  bool in;
+  const uint32_t lo = site_exact(w & 0xFFFFu, d, sbv, s_g, mode == 1 ? side & 1u : side & 0xFu,
+                                 mode, in);
+  const uint32_t hi = site_exact(w >> 16, d, sbv, s_g,
+                                 mode == 1 ? (side >> 1) & 1u : (side >> 4) & 0xFu, mode, in);
+  return lo | (hi << 16);
+}
+
 // ---------------------------------------------------------------------------
 // Kernel 0: zero the per-group amax accumulators.
 // ---------------------------------------------------------------------------
 __global__ void k_zero_u32(uint32_t* p, int n) {
   pdl_begin();
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) p[i] = 0u;
-}
-
-// ---------------------------------------------------------------------------
-// Kernel 1: per-group amax (bits of max|x| as bf16, kept as u32 so that
-// atomicMax orders them as magnitudes).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, kCtasPerSm)
-    k_amax(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-           uint32_t* __restrict__ amax) {
-  __shared__ uint32_t table[kAmaxTable];
-  __shared__ int g_first_s;
-  pdl_begin();
-  if (blockIdx.x >= sh.ntiles) return;
-
-  // the first tile's loads go out before the CTA's set-up barrier
-  V8 v[kBlkPerThread];
-  {
-    const uint32_t base = blockIdx.x * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
-    }
-  }
-  GroupCursor gc;
-  gc.init(offs, sh.G);
-  if (sh.G > 1) {
-    if (threadIdx.x == 0) {
-      gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
-      g_first_s = gc.g;
-    }
-    for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
-  } else if (threadIdx.x == 0) {
-    table[0] = 0u;
-    g_first_s = 0;
-  }
-  __syncthreads();
-  const int g_first = g_first_s;
-  gc.init(offs, sh.G);
-
-  uint32_t run = 0u;
-  int run_g = -1;
-  auto flush = [&](int g, uint32_t val) {
-    if (g < 0 || val == 0u) return;
-    const int slot = g - g_first;
-    if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
-    else atomicMax(&amax[g], val);
-  };
-
-  for (uint32_t t = blockIdx.x; t < sh.ntiles;) {
-    const uint32_t base = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = base + u * kThreads;
-      if (b >= sh.nblk) continue;
-      if (sh.G > 1) {
-        gc.seek(fastdiv(b, sh.bpr));
-        if (gc.g != run_g) {
-          flush(run_g, run);
-          run = 0u;
-          run_g = gc.g;
-        }
-      } else {
-        run_g = 0;
-      }
-      run = max(run, absmax_block(v[u]));
-    }
-    t += gridDim.x;
-    if (t >= sh.ntiles) break;
-    const uint32_t nb = t * kTileBlks + threadIdx.x;
-#pragma unroll
-    for (int u = 0; u < kBlkPerThread; ++u) {
-      const uint32_t b = nb + u * kThreads;
-      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
-    }
-  }
-  if (sh.G == 1) {
-    run = __reduce_max_sync(0xFFFFFFFFu, run);
-    if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
-  } else {
-    flush(run_g, run);
-  }
-  __syncthreads();
-  if (sh.G == 1) {
-    if (threadIdx.x == 0 && table[0]) atomicMax(&amax[0], table[0]);
-    return;
-  }
-  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
-    const uint32_t val = table[i];
-    if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
-  }
 }
 
 // Per-group constants of capture.
@@ -239,6 +161,133 @@ __device__ __forceinline__ GroupK group_consts(uint32_t amax_bits) {
   k.fast6 = fast_scale(k.den6);
   k.r6 = k.fast6 ? __frcp_rn(k.den6) : 0.0f;
   return k;
+}
+
+// The same constants from s_g (as the amax pass leaves it in gscale).
+__device__ __forceinline__ GroupK group_consts_of_sg(float s_g) {
+  GroupK k;
+  k.s_g = s_g;
+  k.den6 = __fmul_rn(6.0f, s_g);
+  k.fast6 = fast_scale(k.den6);
+  k.r6 = k.fast6 ? __frcp_rn(k.den6) : 0.0f;
+  return k;
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 1: per-group amax (bits of max|x| as bf16, kept as u32 so that
+// atomicMax orders them as magnitudes), max-accumulated into amax[0, G).
+// A persistent grid (a few CTAs per SM), each thread with two tiles' loads in
+// flight.
+// FIN: the amax pass of a capture.  amax[G] is then a ticket counter; the
+// CTA that draws the last ticket -- after every CTA's accumulation is
+// visible -- takes the final amax of each group (reading and zeroing the
+// accumulator in one exchange), writes its s_g to gscale, and zeroes the
+// ticket: the workspace is zero again for the next call, and the quantising
+// pass reads only gscale.
+// ---------------------------------------------------------------------------
+template <bool FIN>
+__global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
+    k_amax(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+           uint32_t* __restrict__ amax, float* __restrict__ gscale) {
+  __shared__ uint32_t table[kAmaxTable];
+  __shared__ int g_first_s;
+  __shared__ uint32_t last_s;
+  pdl_begin();
+
+  // tiles t (A) and t + gridDim.x (B) in flight; the first loads go out
+  // before the CTA's set-up barrier
+  const uint32_t step = gridDim.x;
+  V8 a0, a1, b0, b1;
+  auto load = [&](uint32_t t, V8& v0, V8& v1) {
+    const uint32_t b = t * kTileBlks + threadIdx.x;
+    v0 = (t < sh.ntiles && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
+    v1 = (t < sh.ntiles && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads)
+                                                     : zero_block();
+  };
+  load(blockIdx.x, a0, a1);
+  load(blockIdx.x + step, b0, b1);
+  GroupCursor gc;
+  gc.init(offs, sh.G);
+  if (sh.G > 1) {
+    if (threadIdx.x == 0) {
+      gc.seek(blockIdx.x < sh.ntiles ? fastdiv(blockIdx.x * kTileBlks, sh.bpr) : 0u);
+      g_first_s = gc.g;
+    }
+    for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
+  } else if (threadIdx.x == 0) {
+    table[0] = 0u;
+    g_first_s = 0;
+  }
+  __syncthreads();
+  const int g_first = g_first_s;
+  gc.init(offs, sh.G);
+
+  uint32_t run = 0u;
+  int run_g = sh.G > 1 ? -1 : 0;
+  auto flush = [&](int g, uint32_t val) {
+    if (g < 0 || val == 0u) return;
+    const int slot = g - g_first;
+    if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
+    else atomicMax(&amax[g], val);
+  };
+  auto take = [&](uint32_t t, const V8& v0, const V8& v1) {
+    if (sh.G == 1) {  // blocks past the end were loaded as zeros
+      run = max(run, max(absmax_block(v0), absmax_block(v1)));
+      return;
+    }
+    const uint32_t b = t * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t bu = b + u * kThreads;
+      if (bu >= sh.nblk) continue;
+      gc.seek(fastdiv(bu, sh.bpr));
+      if (gc.g != run_g) {
+        flush(run_g, run);
+        run = 0u;
+        run_g = gc.g;
+      }
+      run = max(run, absmax_block(u == 0 ? v0 : v1));
+    }
+  };
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += 2u * step) {
+    take(t, a0, a1);
+    load(t + 2u * step, a0, a1);
+    if (t + step >= sh.ntiles) break;
+    take(t + step, b0, b1);
+    load(t + 3u * step, b0, b1);
+  }
+  if (sh.G == 1) {
+    run = __reduce_max_sync(0xFFFFFFFFu, run);
+    if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
+  } else {
+    flush(run_g, run);
+  }
+  __syncthreads();
+  if (sh.G == 1) {
+    if (threadIdx.x != 0) return;
+    if (table[0]) atomicMax(&amax[0], table[0]);
+    if (!FIN) return;
+    __threadfence();  // this CTA's maximum before its ticket
+    if (atomicAdd(&amax[1], 1u) != gridDim.x - 1u) return;
+    __threadfence();
+    gscale[0] = group_consts(atomicExch(&amax[0], 0u)).s_g;
+    amax[1] = 0u;
+    return;
+  }
+  for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
+    const uint32_t val = table[i];
+    if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
+  }
+  if (!FIN) return;
+  __threadfence();  // each thread's maxima before the CTA's ticket
+  __syncthreads();
+  if (threadIdx.x == 0) last_s = atomicAdd(&amax[sh.G], 1u) == gridDim.x - 1u;
+  __syncthreads();
+  if (!last_s) return;
+  __threadfence();
+  for (int g = threadIdx.x; g < sh.G; g += kThreads)
+    gscale[g] = group_consts(atomicExch(&amax[g], 0u)).s_g;
+  if (threadIdx.x == 0) amax[sh.G] = 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -309,25 +358,23 @@ __device__ __forceinline__ void codes_block(const V8& v, const V8* src, float d,
 // Each thread owns two adjacent blocks: one 16-byte store of codes, one
 // 32-bit store of mantissa bits, one 16-bit store of scales.
 // SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
-// RESET (a single group only): `amax` is the call's workspace (the
-// accumulator, then a ticket counter); the CTA that draws the last ticket --
-// after every CTA has read the accumulator -- sets both back to zero, so the
-// next capture with the same workspace needs no zeroing launch.  Nothing
-// waits.
-template <bool SW, bool RESET>
+// PRE: the amax pass of the same capture has written gscale, and the group
+// constants are taken from it; otherwise they are computed here from the
+// given per-group amax words, and this pass writes gscale.  Nothing waits on
+// another CTA.
+template <bool SW, bool PRE>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-              uint32_t* amax, uint4* __restrict__ codes, uint32_t* __restrict__ mbits,
-              uint8_t* __restrict__ scales, float* __restrict__ gscale) {
-  __shared__ uint32_t amax_s;
+              const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
+              uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales,
+              float* __restrict__ gscale) {
   pdl_begin();
   GroupCursor gc;
   gc.init(offs, sh.G);
-  GroupK gk = group_consts(0u);
-  const bool one = sh.G == 1;
-  // tiles in reverse order: k_amax read the high tiles last, so they are the
-  // most likely to be still in L2.  The first tile's loads go out before
-  // the CTA's set-up below.
+  GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
+  // tiles in reverse order: the amax pass read the high tiles last, so they
+  // are the most likely to be still in L2.  The first tile's loads go out
+  // before anything else.
   uint32_t i = blockIdx.x;
   auto tile_base = [&](uint32_t k) { return (sh.ntiles - 1u - k) * kTileBlks + 2u * threadIdx.x; };
   V8 v0 = zero_block(), v1 = zero_block();
@@ -335,27 +382,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     v0 = ld_block_stream(x + tile_base(i));
     v1 = ld_block_stream(x + tile_base(i) + 1);
   }
-  uint32_t ticket = 0u;
-  if (one) {
-    // a single group: thread 0 reads the accumulator once for the CTA and,
-    // with RESET, then takes its ticket with a release add (ordering that
-    // read before it; the result is looked at only at the end of the CTA).
-    // The CTA that drew the last ticket -- every CTA has read the
-    // accumulator by then -- zeroes it and the ticket after an acquire fence.
-    if (threadIdx.x == 0) {
-      const uint32_t a = __ldcg(amax);
-      amax_s = a;
-      if (blockIdx.x == 0) gscale[0] = group_consts(a).s_g;
-      if (RESET)
-        asm volatile("atom.release.gpu.global.add.u32 %0, [%1], 1;"
-                     : "=r"(ticket)
-                     : "l"(amax + 1)
-                     : "memory");
-    }
-    __syncthreads();
-    gk = group_consts(amax_s);
-    gc.seek(0u);
-  } else {
+  if (!PRE) {
     // global scales of all groups (any CTA may write them; all write the same)
     for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
       gscale[g] = group_consts(__ldcg(amax + g)).s_g;
@@ -367,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (b < sh.nblk) {
       // both blocks of the pair are in the same row (cols is a multiple of 32)
       const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-      if (gc.seek(row)) gk = group_consts(__ldcg(amax + gc.g));
+      if (gc.seek(row))
+        gk = PRE ? group_consts_of_sg(__ldcg(gscale + gc.g)) : group_consts(__ldcg(amax + gc.g));
       const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
       float sb0, sb1;
       e4m3x2_to_f32(s2, sb0, sb1);
@@ -392,11 +420,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       v0 = ld_block_stream(x + tile_base(inext));
       v1 = ld_block_stream(x + tile_base(inext) + 1);
     }
-  }
-  if (RESET && one && threadIdx.x == 0 && ticket == gridDim.x - 1u) {
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-    amax[0] = 0u;
-    amax[1] = 0u;
   }
 }
 
@@ -612,6 +635,81 @@ __device__ __forceinline__ void patch_pair(const uint32_t* xw, uint32_t* ow, int
   }
 }
 
+// The pairs a guided rule recomputes, queued per CTA for the variant with
+// separate output buffers.  A drifted pair disagrees with round to nearest
+// at well under 1% of the sites, so a thread meets such a pair now and then
+// and a warp, recomputing its threads' pairs in place, would run the pair
+// routine with one or two of its 32 lanes active; from the queue, every
+// lane of a warp recomputes one pair.  An entry: the pair's input word, the
+// block index b of the thread's first block (the pair is word q of the 16
+// words of blocks b and b + 1), q | side << 4 | the block's E4M3 scale byte
+// << 12, and s_g.  The queue is drained every kPatchEvery tiles and at the
+// end of the CTA; a thread that finds it full recomputes its pair at once.
+constexpr int kPatchCap = 512;
+constexpr int kPatchEvery = 4;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Queue the pairs marked in `pend` (bit 2q: pair q of the thread's blocks b
+// and b + 1).  Every lane of the warp calls it, with or without pairs.
+template <int MODE>
+__device__ __forceinline__ void queue_pairs(uint4* pq, uint32_t* pq_n, uint32_t pend,
+                                            const V8* x, V8* out, uint32_t b, uint32_t bits,
+                                            const uint4& rc, uint32_t sb2, float s_g) {
+  const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
+  uint32_t bal = __ballot_sync(0xFFFFFFFFu, pend != 0u);
+  while (bal != 0u) {
+    const int lead = __ffs(bal) - 1;
+    uint32_t base = 0u;
+    if ((int)(threadIdx.x & 31u) == lead) base = atomicAdd(pq_n, (uint32_t)__popc(bal));
+    base = __shfl_sync(0xFFFFFFFFu, base, lead);
+    if (pend != 0u) {
+      const int q = (__ffs(pend) - 1) >> 1;
+      pend &= pend - 1u;
+      const uint32_t pos = base + (uint32_t)__popc(bal & lanemask_lt());
+      const uint32_t side =
+          MODE == kGuided ? (bits >> (2 * q)) & 3u
+                          : ((q < 4 ? rc.x : q < 8 ? rc.y : q < 12 ? rc.z : rc.w) >> (8 * (q & 3))) &
+                                0xFFu;
+      const uint32_t sbyte = (sb2 >> (q < 8 ? 0 : 8)) & 0xFFu;
+      if (pos < (uint32_t)kPatchCap) {
+        pq[pos] = make_uint4(__ldg(xw + q), b, (uint32_t)q | (side << 4) | (sbyte << 12),
+                             __float_as_uint(s_g));
+      } else {
+        float sbv, unused;
+        e4m3x2_to_f32(sbyte, sbv, unused);
+        patch_pair<MODE>(xw, reinterpret_cast<uint32_t*>(out + b), q, __fmul_rn(s_g, sbv), sbv,
+                         s_g, side);
+      }
+    }
+    bal = __ballot_sync(0xFFFFFFFFu, pend != 0u);
+  }
+}
+
+// Recompute the first n queued pairs, one per thread, and store them over
+// the round-to-nearest words at out.  Called by the whole CTA after a
+// barrier that makes the queue and those words visible.
+template <int MODE>
+__device__ __forceinline__ void drain_pairs(const uint4* pq, uint32_t n, V8* out) {
+  for (uint32_t e = threadIdx.x; e < n; e += kThreads) {
+    const uint4 en = pq[e];
+    const int q = (int)(en.z & 15u);
+    const uint32_t side = (en.z >> 4) & 0xFFu;
+    float sbv, unused;
+    e4m3x2_to_f32((en.z >> 12) & 0xFFu, sbv, unused);
+    const float s_g = __uint_as_float(en.w);
+    const float d = __fmul_rn(s_g, sbv);
+    uint32_t* ow = reinterpret_cast<uint32_t*>(out + en.y) + q;
+    *ow = fast_scale(d, kDMaxExactZ)
+              ? guided_pair<MODE>(en.x, side, make_blk(d, __fmul_rn(sbv, 0x1p-64f), s_g))
+              : guided_word_exact(en.x, d, sbv, s_g, side, MODE);
+  }
+}
+
 // One block with any scale (zero block, fast path or exact path): stores its
 // output at dst and returns its 16 mask bits.
 template <int MODE>
@@ -645,70 +743,88 @@ __device__ __forceinline__ uint32_t fake_quant_block(const V8& v, const V8* src,
 // budget it ran 16% faster on B200 at 268M elements (and 13% slower at 33M,
 // where a thread sees one tile).
 // SEP: out does not alias x.  The guided rules then write both blocks'
-// round-to-nearest outputs first and recompute the pairs that need it in one
-// loop for the thread's 32 elements, reading their inputs back from x.
+// round-to-nearest outputs first and queue the pairs that need the rule's
+// own routine (queue_pairs); the CTA recomputes them together.
 template <int MODE, bool SW, int MINB = kCtasPerSm, bool SEP = false>
 __global__ void __launch_bounds__(kThreads, MINB)
     k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
                  const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
                  const uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                  V8* __restrict__ out, uint32_t* __restrict__ mask) {
+  constexpr bool kQueue = SEP && MODE != kRtn;
+  __shared__ uint4 pq[kQueue ? kPatchCap : 1];
+  __shared__ uint32_t pq_n;
   pdl_begin();
+  if (kQueue) {
+    if (threadIdx.x == 0) pq_n = 0u;
+    __syncthreads();
+  }
   GroupCursor gc;
   gc.init(offs, sh.G);
   float s_g = 1.0f;
 
+  // the trip count is the same for every thread of the CTA (the queue's
+  // barriers rely on it)
+  uint32_t it = 0u;
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
-    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-    const uint32_t sb2 =
-        SW ? __ldcs(reinterpret_cast<const unsigned short*>(
-                 scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
-           : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
-    if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
-    uint32_t m0, m1;
-    float sbv0, sbv1;
-    e4m3x2_to_f32(sb2, sbv0, sbv1);
-    // a row holds a whole number of 32-element words, so both blocks of the
-    // pair are in the same row and group
-    const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
-    if (SEP && MODE != kRtn && fast_scale(d0) && fast_scale(d1)) {
-      // the common case for separate output buffers
-      V8 o;
-      const uint32_t bad0 =
-          fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, make_blk(d0, sbv0, s_g), o, m0);
-      st_block(out + b, o);
-      const uint32_t bad1 =
-          fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, make_blk(d1, sbv1, s_g), o, m1);
-      st_block(out + b + 1, o);
-      uint32_t pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
-      const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
-      uint32_t* ow = reinterpret_cast<uint32_t*>(out + b);
-      while (pairs != 0u) {
-        const int q = (__ffs(pairs) - 1) >> 1;  // pair q & 7 of block q >> 3
-        pairs &= pairs - 1u;
-        const uint32_t side =
-            MODE == kGuided ? bits >> (2 * q)
-                            : (q < 4 ? rc.x : q < 8 ? rc.y : q < 12 ? rc.z : rc.w) >> (8 * (q & 3));
-        patch_pair<MODE>(xw, ow, q, q < 8 ? d0 : d1, q < 8 ? sbv0 : sbv1, s_g, side);
+    uint32_t pairs = 0u, bits = 0u, sb2 = 0u;
+    uint4 rc = make_uint4(0u, 0u, 0u, 0u);
+    if (b < sh.nblk) {
+      const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+      if (MODE == kGuided) bits = __ldcs(mbits + (b >> 1));
+      if (MODE == kFull) rc = __ldcs(rcodes + (b >> 1));
+      const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+      sb2 = SW ? __ldcs(reinterpret_cast<const unsigned short*>(
+                     scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
+               : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
+      if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
+      uint32_t m0, m1;
+      float sbv0, sbv1;
+      e4m3x2_to_f32(sb2, sbv0, sbv1);
+      // a row holds a whole number of 32-element words, so both blocks of the
+      // pair are in the same row and group
+      const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
+      if (kQueue && fast_scale(d0) && fast_scale(d1)) {
+        // the common case for separate output buffers
+        V8 o;
+        const uint32_t bad0 =
+            fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, make_blk(d0, sbv0, s_g), o, m0);
+        st_block(out + b, o);
+        const uint32_t bad1 =
+            fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, make_blk(d1, sbv1, s_g), o, m1);
+        st_block(out + b + 1, o);
+        pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
+      } else if (fast_scale(d0) && fast_scale(d1)) {
+        // the common case, without per-block branches
+        V8 o;
+        const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
+        fq_block_fast<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
+        st_block(out + b, o);
+        fq_block_fast<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
+        st_block(out + b + 1, o);
+      } else {
+        m0 = fake_quant_block<MODE>(v0, x + b, bits & 0xFFFFu, rc.x, rc.y, sbv0, s_g, out + b);
+        m1 = fake_quant_block<MODE>(v1, x + b + 1, bits >> 16, rc.z, rc.w, sbv1, s_g,
+                                    out + b + 1);
       }
-    } else if (fast_scale(d0) && fast_scale(d1)) {
-      // the common case, without per-block branches
-      V8 o;
-      const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
-      fq_block_fast<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
-      st_block(out + b, o);
-      fq_block_fast<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
-      st_block(out + b + 1, o);
-    } else {
-      m0 = fake_quant_block<MODE>(v0, x + b, bits & 0xFFFFu, rc.x, rc.y, sbv0, s_g, out + b);
-      m1 = fake_quant_block<MODE>(v1, x + b + 1, bits >> 16, rc.z, rc.w, sbv1, s_g, out + b + 1);
+      mask[b >> 1] = m0 | (m1 << 16);
     }
-    mask[b >> 1] = m0 | (m1 << 16);
+    if (kQueue) {
+      queue_pairs<MODE>(pq, &pq_n, pairs, x, out, b, bits, rc, sb2, s_g);
+      if (++it % kPatchEvery == 0u) {
+        __syncthreads();
+        const uint32_t n = min(pq_n, (uint32_t)kPatchCap);
+        drain_pairs<MODE>(pq, n, out);
+        __syncthreads();  // everyone has read the count and its entries
+        if (threadIdx.x == 0) pq_n = 0u;
+        __syncthreads();
+      }
+    }
+  }
+  if (kQueue) {
+    __syncthreads();
+    drain_pairs<MODE>(pq, min(pq_n, (uint32_t)kPatchCap), out);
   }
 }
 

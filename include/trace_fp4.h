@@ -129,10 +129,10 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
  *             leaves it all-zero again, so a workspace can serve any number
  *             of calls one after another (not two calls that may run at the
  *             same time).
- * Launches the grid amax (max-accumulated into the workspace) and the
- * quantising pass; for one group the CTA of that pass that draws the last
- * ticket (an atomic counter in the workspace; nothing waits) sets the
- * workspace back to zero, for groups a third, one-CTA launch zeroes it. */
+ * Launches the grid amax (max-accumulated into the workspace; the CTA that
+ * draws the last ticket -- an atomic counter in the workspace; nothing waits
+ * -- writes gscale and sets the workspace back to zero) and the quantising
+ * pass, which reads gscale. */
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
                   int32_t num_groups, const int64_t* group_row_offsets,
                   uint8_t* codes, uint32_t* mbits, uint8_t* scales,
