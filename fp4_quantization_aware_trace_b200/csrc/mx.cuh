@@ -376,7 +376,11 @@ __device__ __forceinline__ void mx8_fq_half(const V8& v, uint32_t bits16, uint4 
   }
 }
 
-template <int MODE, bool SW>
+// SEP: out does not alias x; the guided rules then store both halves'
+// round-to-nearest outputs and recompute the pairs that need it in one loop
+// per thread, their inputs and rollout codes read back from memory, as
+// k_fake_quant does.
+template <int MODE, bool SW, bool SEP = false>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_mx8_fake_quant(const V8* __restrict__ x, Shape sh, const uint32_t* __restrict__ mbits,
                      const V8* __restrict__ rcodes, const uint8_t* __restrict__ scales,
@@ -398,12 +402,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const u64 inv2 = pk(inv, inv), X2 = pk(X, X);  // 2^-e and 2^e
     uint32_t m = 0u;
     V8 o;
-    mx8_fq_half<MODE>(v0, bits & 0xFFFFu, make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]), inv2, X2,
-                      o, m, 0);
-    st_block(out + b, o);
-    mx8_fq_half<MODE>(v1, bits >> 16, make_uint4(rc.w[4], rc.w[5], rc.w[6], rc.w[7]), inv2, X2, o,
-                      m, 16);
-    st_block(out + b + 1, o);
+    if (SEP && MODE != kRtn) {
+      const uint32_t bad0 = mx8_rtn_half<MODE>(
+          v0, bits & 0xFFFFu, make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]), inv2, X2, o, m, 0);
+      st_block(out + b, o);
+      const uint32_t bad1 = mx8_rtn_half<MODE>(
+          v1, bits >> 16, make_uint4(rc.w[4], rc.w[5], rc.w[6], rc.w[7]), inv2, X2, o, m, 16);
+      st_block(out + b + 1, o);
+      uint32_t pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
+      const unsigned short* rh = reinterpret_cast<const unsigned short*>(rcodes + (b >> 1));
+      uint32_t* ow = reinterpret_cast<uint32_t*>(out + b);
+      while (pairs != 0u) {
+        const int q = (__ffs(pairs) - 1) >> 1;  // pair q of the thread's 32 elements
+        pairs &= pairs - 1u;
+        const uint32_t side = MODE == kGuided ? bits >> (2 * q) : (uint32_t)__ldg(rh + q);
+        ow[q] = mx8_guided_pair<MODE>(__ldg(xw + q), side, inv2, X2);
+      }
+    } else {
+      mx8_fq_half<MODE>(v0, bits & 0xFFFFu, make_uint4(rc.w[0], rc.w[1], rc.w[2], rc.w[3]), inv2,
+                        X2, o, m, 0);
+      st_block(out + b, o);
+      mx8_fq_half<MODE>(v1, bits >> 16, make_uint4(rc.w[4], rc.w[5], rc.w[6], rc.w[7]), inv2, X2,
+                        o, m, 16);
+      st_block(out + b + 1, o);
+    }
     mask[b >> 1] = m;
   }
 }

@@ -124,19 +124,6 @@ __device__ __noinline__ uint32_t guided_site_fix(const uint16_t* src, float d, f
                     side, mode, in);
 }
 
-// Both sites of a pair (bf16x2 word w) on the exact path: output bits with
-// x's signs.  side as guided_pair below (mode 1: the two cached bits in bits
-// 0 and 1; mode 2: the two rollout codes, low nibble first).
-__device__ __noinline__ uint32_t guided_word_exact(uint32_t w, float d, float sbv, float s_g,
-                                                   uint32_t side, int mode) {
-  bool in;
-  const uint32_t lo = site_exact(w & 0xFFFFu, d, sbv, s_g, mode == 1 ? side & 1u : side & 0xFu,
-                                 mode, in);
-  const uint32_t hi = site_exact(w >> 16, d, sbv, s_g,
-                                 mode == 1 ? (side >> 1) & 1u : (side >> 4) & 0xFu, mode, in);
-  return lo | (hi << 16);
-}
-
 // ---------------------------------------------------------------------------
 // Kernel 0: zero the per-group amax accumulators.
 // ---------------------------------------------------------------------------
@@ -635,81 +622,6 @@ __device__ __forceinline__ void patch_pair(const uint32_t* xw, uint32_t* ow, int
   }
 }
 
-// The pairs a guided rule recomputes, queued per CTA for the variant with
-// separate output buffers.  A drifted pair disagrees with round to nearest
-// at well under 1% of the sites, so a thread meets such a pair now and then
-// and a warp, recomputing its threads' pairs in place, would run the pair
-// routine with one or two of its 32 lanes active; from the queue, every
-// lane of a warp recomputes one pair.  An entry: the pair's input word, the
-// block index b of the thread's first block (the pair is word q of the 16
-// words of blocks b and b + 1), q | side << 4 | the block's E4M3 scale byte
-// << 12, and s_g.  The queue is drained every kPatchEvery tiles and at the
-// end of the CTA; a thread that finds it full recomputes its pair at once.
-constexpr int kPatchCap = 512;
-constexpr int kPatchEvery = 4;
-
-__device__ __forceinline__ uint32_t lanemask_lt() {
-  uint32_t m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
-}
-
-// Queue the pairs marked in `pend` (bit 2q: pair q of the thread's blocks b
-// and b + 1).  Every lane of the warp calls it, with or without pairs.
-template <int MODE>
-__device__ __forceinline__ void queue_pairs(uint4* pq, uint32_t* pq_n, uint32_t pend,
-                                            const V8* x, V8* out, uint32_t b, uint32_t bits,
-                                            const uint4& rc, uint32_t sb2, float s_g) {
-  const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
-  uint32_t bal = __ballot_sync(0xFFFFFFFFu, pend != 0u);
-  while (bal != 0u) {
-    const int lead = __ffs(bal) - 1;
-    uint32_t base = 0u;
-    if ((int)(threadIdx.x & 31u) == lead) base = atomicAdd(pq_n, (uint32_t)__popc(bal));
-    base = __shfl_sync(0xFFFFFFFFu, base, lead);
-    if (pend != 0u) {
-      const int q = (__ffs(pend) - 1) >> 1;
-      pend &= pend - 1u;
-      const uint32_t pos = base + (uint32_t)__popc(bal & lanemask_lt());
-      const uint32_t side =
-          MODE == kGuided ? (bits >> (2 * q)) & 3u
-                          : ((q < 4 ? rc.x : q < 8 ? rc.y : q < 12 ? rc.z : rc.w) >> (8 * (q & 3))) &
-                                0xFFu;
-      const uint32_t sbyte = (sb2 >> (q < 8 ? 0 : 8)) & 0xFFu;
-      if (pos < (uint32_t)kPatchCap) {
-        pq[pos] = make_uint4(__ldg(xw + q), b, (uint32_t)q | (side << 4) | (sbyte << 12),
-                             __float_as_uint(s_g));
-      } else {
-        float sbv, unused;
-        e4m3x2_to_f32(sbyte, sbv, unused);
-        patch_pair<MODE>(xw, reinterpret_cast<uint32_t*>(out + b), q, __fmul_rn(s_g, sbv), sbv,
-                         s_g, side);
-      }
-    }
-    bal = __ballot_sync(0xFFFFFFFFu, pend != 0u);
-  }
-}
-
-// Recompute the first n queued pairs, one per thread, and store them over
-// the round-to-nearest words at out.  Called by the whole CTA after a
-// barrier that makes the queue and those words visible.
-template <int MODE>
-__device__ __forceinline__ void drain_pairs(const uint4* pq, uint32_t n, V8* out) {
-  for (uint32_t e = threadIdx.x; e < n; e += kThreads) {
-    const uint4 en = pq[e];
-    const int q = (int)(en.z & 15u);
-    const uint32_t side = (en.z >> 4) & 0xFFu;
-    float sbv, unused;
-    e4m3x2_to_f32((en.z >> 12) & 0xFFu, sbv, unused);
-    const float s_g = __uint_as_float(en.w);
-    const float d = __fmul_rn(s_g, sbv);
-    uint32_t* ow = reinterpret_cast<uint32_t*>(out + en.y) + q;
-    *ow = fast_scale(d, kDMaxExactZ)
-              ? guided_pair<MODE>(en.x, side, make_blk(d, __fmul_rn(sbv, 0x1p-64f), s_g))
-              : guided_word_exact(en.x, d, sbv, s_g, side, MODE);
-  }
-}
-
 // One block with any scale (zero block, fast path or exact path): stores its
 // output at dst and returns its 16 mask bits.
 template <int MODE>
@@ -743,88 +655,70 @@ __device__ __forceinline__ uint32_t fake_quant_block(const V8& v, const V8* src,
 // budget it ran 16% faster on B200 at 268M elements (and 13% slower at 33M,
 // where a thread sees one tile).
 // SEP: out does not alias x.  The guided rules then write both blocks'
-// round-to-nearest outputs first and queue the pairs that need the rule's
-// own routine (queue_pairs); the CTA recomputes them together.
+// round-to-nearest outputs first and recompute the pairs that need it in one
+// loop for the thread's 32 elements, reading their inputs back from x.
 template <int MODE, bool SW, int MINB = kCtasPerSm, bool SEP = false>
 __global__ void __launch_bounds__(kThreads, MINB)
     k_fake_quant(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
                  const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
                  const uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                  V8* __restrict__ out, uint32_t* __restrict__ mask) {
-  constexpr bool kQueue = SEP && MODE != kRtn;
-  __shared__ uint4 pq[kQueue ? kPatchCap : 1];
-  __shared__ uint32_t pq_n;
   pdl_begin();
-  if (kQueue) {
-    if (threadIdx.x == 0) pq_n = 0u;
-    __syncthreads();
-  }
   GroupCursor gc;
   gc.init(offs, sh.G);
   float s_g = 1.0f;
 
-  // the trip count is the same for every thread of the CTA (the queue's
-  // barriers rely on it)
-  uint32_t it = 0u;
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    uint32_t pairs = 0u, bits = 0u, sb2 = 0u;
-    uint4 rc = make_uint4(0u, 0u, 0u, 0u);
-    if (b < sh.nblk) {
-      const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
-      if (MODE == kGuided) bits = __ldcs(mbits + (b >> 1));
-      if (MODE == kFull) rc = __ldcs(rcodes + (b >> 1));
-      const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-      sb2 = SW ? __ldcs(reinterpret_cast<const unsigned short*>(
-                     scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
-               : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
-      if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
-      uint32_t m0, m1;
-      float sbv0, sbv1;
-      e4m3x2_to_f32(sb2, sbv0, sbv1);
-      // a row holds a whole number of 32-element words, so both blocks of the
-      // pair are in the same row and group
-      const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
-      if (kQueue && fast_scale(d0) && fast_scale(d1)) {
-        // the common case for separate output buffers
-        V8 o;
-        const uint32_t bad0 =
-            fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, make_blk(d0, sbv0, s_g), o, m0);
-        st_block(out + b, o);
-        const uint32_t bad1 =
-            fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, make_blk(d1, sbv1, s_g), o, m1);
-        st_block(out + b + 1, o);
-        pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
-      } else if (fast_scale(d0) && fast_scale(d1)) {
-        // the common case, without per-block branches
-        V8 o;
-        const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
-        fq_block_fast<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
-        st_block(out + b, o);
-        fq_block_fast<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
-        st_block(out + b + 1, o);
-      } else {
-        m0 = fake_quant_block<MODE>(v0, x + b, bits & 0xFFFFu, rc.x, rc.y, sbv0, s_g, out + b);
-        m1 = fake_quant_block<MODE>(v1, x + b + 1, bits >> 16, rc.z, rc.w, sbv1, s_g,
-                                    out + b + 1);
+    if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+    const uint32_t sb2 =
+        SW ? __ldcs(reinterpret_cast<const unsigned short*>(
+                 scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
+           : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
+    if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
+    uint32_t m0, m1;
+    float sbv0, sbv1;
+    e4m3x2_to_f32(sb2, sbv0, sbv1);
+    // a row holds a whole number of 32-element words, so both blocks of the
+    // pair are in the same row and group
+    const float d0 = __fmul_rn(s_g, sbv0), d1 = __fmul_rn(s_g, sbv1);
+    if (SEP && MODE != kRtn && fast_scale(d0) && fast_scale(d1)) {
+      // the common case for separate output buffers
+      V8 o;
+      const uint32_t bad0 =
+          fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, make_blk(d0, sbv0, s_g), o, m0);
+      st_block(out + b, o);
+      const uint32_t bad1 =
+          fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, make_blk(d1, sbv1, s_g), o, m1);
+      st_block(out + b + 1, o);
+      uint32_t pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
+      const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
+      uint32_t* ow = reinterpret_cast<uint32_t*>(out + b);
+      while (pairs != 0u) {
+        const int q = (__ffs(pairs) - 1) >> 1;  // pair q & 7 of block q >> 3
+        pairs &= pairs - 1u;
+        const uint32_t side =
+            MODE == kGuided ? bits >> (2 * q)
+                            : (q < 4 ? rc.x : q < 8 ? rc.y : q < 12 ? rc.z : rc.w) >> (8 * (q & 3));
+        patch_pair<MODE>(xw, ow, q, q < 8 ? d0 : d1, q < 8 ? sbv0 : sbv1, s_g, side);
       }
-      mask[b >> 1] = m0 | (m1 << 16);
+    } else if (fast_scale(d0) && fast_scale(d1)) {
+      // the common case, without per-block branches
+      V8 o;
+      const uint16_t* src = reinterpret_cast<const uint16_t*>(x + b);
+      fq_block_fast<MODE>(v0, src, bits & 0xFFFFu, rc.x, rc.y, d0, sbv0, s_g, o, m0);
+      st_block(out + b, o);
+      fq_block_fast<MODE>(v1, src + 16, bits >> 16, rc.z, rc.w, d1, sbv1, s_g, o, m1);
+      st_block(out + b + 1, o);
+    } else {
+      m0 = fake_quant_block<MODE>(v0, x + b, bits & 0xFFFFu, rc.x, rc.y, sbv0, s_g, out + b);
+      m1 = fake_quant_block<MODE>(v1, x + b + 1, bits >> 16, rc.z, rc.w, sbv1, s_g, out + b + 1);
     }
-    if (kQueue) {
-      queue_pairs<MODE>(pq, &pq_n, pairs, x, out, b, bits, rc, sb2, s_g);
-      if (++it % kPatchEvery == 0u) {
-        __syncthreads();
-        const uint32_t n = min(pq_n, (uint32_t)kPatchCap);
-        drain_pairs<MODE>(pq, n, out);
-        __syncthreads();  // everyone has read the count and its entries
-        if (threadIdx.x == 0) pq_n = 0u;
-        __syncthreads();
-      }
-    }
-  }
-  if (kQueue) {
-    __syncthreads();
-    drain_pairs<MODE>(pq, min(pq_n, (uint32_t)kPatchCap), out);
+    mask[b >> 1] = m0 | (m1 << 16);
   }
 }
 

@@ -625,17 +625,16 @@ def test_guided_rules_in_place_and_separate_vs_oracle(oracle_mod, drift):
         _eq(f"{name} in-place mask", _u(inp_mask), ref_mask)
 
 
-def test_guided_recompute_queue_at_many_tiles_per_cta(oracle_mod):
-    """The guided forwards with separate outputs queue the pairs they
-    recompute per CTA and drain the queue every few tiles.  A [40960, 8192]
-    tensor gives every CTA eight or nine tiles (two drains inside the walk
-    and one at its end); its rows 1024-3071 carry training values drawn
-    independently of the rollout's, so that CTAs whose tiles fall there
-    overflow the queue and recompute directly.  The whole tensor of both
-    guided rules against the threaded oracle."""
+def test_guided_separate_outputs_many_tiles_per_cta(oracle_mod):
+    """The guided forwards with separate outputs store round to nearest and
+    then recompute the pairs where the rule disagrees.  A [40960, 8192]
+    tensor gives every CTA eight or nine tiles; its rows 1024-3071 carry
+    training values drawn independently of the rollout's, so that most
+    pairs there are recomputed, while the other rows drift slightly.  The
+    whole tensor of both guided rules against the threaded oracle."""
     import oracle.threaded as ot
     R, C = 40960, 8192
-    s = inputs.lognormal_site(7301, R, C, device=DEV, name="queue")
+    s = inputs.lognormal_site(7301, R, C, device=DEV, name="sep_many_tiles")
     other = inputs.lognormal_site(7302, 2048, C, device=DEV, name="other")
     xt = s.x_train.clone()
     xt[1024:3072] = other.x_roll
@@ -646,12 +645,12 @@ def test_guided_recompute_queue_at_many_tiles_per_cta(oracle_mod):
     hr, ht = inputs.bits(s.x_roll), inputs.bits(xt)
     del s, other, xt
     codes, mbits, scales, gscale = ot.capture_mt(hr)
-    _eq("queue.codes", _u(cap.codes), codes)
-    _eq("queue.mbits", _u(cap.mbits), mbits)
+    _eq("sep_many_tiles.codes", _u(cap.codes), codes)
+    _eq("sep_many_tiles.mbits", _u(cap.mbits), mbits)
     ref_out, ref_mask = ot.guided_fwd_mt(ht, mbits, scales, gscale)
-    _eq("queue.out", _u(out), ref_out)
-    _eq("queue.mask", _u(mask), ref_mask)
+    _eq("sep_many_tiles.out", _u(out), ref_out)
+    _eq("sep_many_tiles.mask", _u(mask), ref_mask)
     del ref_out, ref_mask
     ref_out, ref_mask = ot.full_guided_fwd_mt(ht, codes, scales, gscale)
-    _eq("queue.out_full", _u(out_f), ref_out)
-    _eq("queue.mask_full", _u(mask_f), ref_mask)
+    _eq("sep_many_tiles.out_full", _u(out_f), ref_out)
+    _eq("sep_many_tiles.mask_full", _u(mask_f), ref_mask)
