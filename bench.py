@@ -2,8 +2,9 @@
 """Throughput of the TRACE capture + guided NVFP4 fake-quant hot path on B200.
 
 One step = one pass of the whole path over every site of the workload:
-  rollout capture of x_roll  (grid amax, then quantise -> FP4 codes + compact
-                              cache of mantissa bits and scales)
+  rollout capture of x_roll  (grid amax, grid barrier, then quantise -> FP4
+                              codes + compact cache of mantissa bits and
+                              scales; one cooperative launch)
   guided fake-quant forward of x_train with that cache (bf16 out + STE mask)
   masked straight-through backward of an upstream gradient
   round-to-nearest fake-quant forward of x_train (the vanilla-QAT comparator)
@@ -19,8 +20,8 @@ the KV cache follow as secondary lines (`secondary`), with L2 flushed before
 every step.
 
 The value is algorithmic bytes / time (GB/s): every input read once and every
-output written once per kernel, x_roll read twice by capture (its two
-passes).  Per-element bytes: capture 4.6875, guided 4.3125, backward 4.125,
+output written once per kernel, x_roll read twice by capture (its amax and
+quantising phases).  Per-element bytes: capture 4.6875, guided 4.3125, backward 4.125,
 RTN 4.1875 (+4 bytes per group).  elem/s is reported beside it, and
 `algo_bytes_over_copy_peak` divides the step's algorithmic GB/s by the
 measured copy bandwidth -- not a DRAM fraction: reads that hit L2 count too.
@@ -58,11 +59,12 @@ HEADLINE_CONFIG = 5
 SECONDARY_CONFIGS = (2, 3, 4)
 BYTES_PER_ELEM = {"capture": 4.6875, "guided_fwd": 4.3125, "ste_bwd": 4.125, "rtn_fwd": 4.1875}
 STEP_BYTES_PER_ELEM = sum(BYTES_PER_ELEM.values())
-KERNEL_NAMES = {"capture": "k_amax + k_capture", "guided_fwd": "k_fake_quant<1> (1-bit guided)",
+KERNEL_NAMES = {"capture": "k_capture_coop (amax, grid barrier, quantise)",
+                "guided_fwd": "k_fake_quant<1> (1-bit guided)",
                 "ste_bwd": "k_ste_bwd", "rtn_fwd": "k_fake_quant<0> (round to nearest)"}
-# kernels of the library launched per site and step: capture (amax pass,
-# quantising pass), guided forward, backward, RTN
-LAUNCHES_PER_SITE = 5
+# kernels of the library launched per site and step: capture (one
+# cooperative launch), guided forward, backward, RTN
+LAUNCHES_PER_SITE = 4
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 * 10 ** 6
@@ -817,7 +819,7 @@ def next_rows_leg(args, wl: Workload, pg, dev, flush, hbm):
 
     tl = timed(tiled_pass, 3, 67)
     rows["tiled_scales"] = {
-        "capture": dict(kernel="k_amax + k_capture<true>", **rate(tl[0], 4.6875)),
+        "capture": dict(kernel="k_capture_coop<true>", **rate(tl[0], 4.6875)),
         "guided_fwd": dict(kernel="k_fake_quant<1, true>", **rate(tl[1], 4.3125))}
     del tcap
 

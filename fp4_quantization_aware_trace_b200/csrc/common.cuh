@@ -14,7 +14,10 @@ constexpr int kTileBlks = kThreads * kBlkPerThread;  // 512 blocks = 8192 elemen
 constexpr int kCtasPerSm = 4;    // resident CTAs per SM the register budget allows
 constexpr int kGridPerSm = 32;   // CTAs launched per SM: about one tile each
 constexpr int kAmaxTable = 256;  // groups per CTA kept in shared memory
-constexpr int kAmaxCtasPerSm = 4;  // the amax pass: a persistent grid of this many CTAs per SM
+// Polls of the one-launch capture's grid barrier before it gives up (with a
+// 256 ns sleep between polls: about a second).  The launch is cooperative,
+// so every CTA is resident and the barrier completes long before.
+constexpr uint32_t kBarrierPolls = 1u << 22;
 
 constexpr uint32_t kDMin = 0x12800000u;     // 2^-90: fast paths need d >= 2^-90
 constexpr uint32_t kDMax = 0x71800000u;     // 2^100: capture / round-to-nearest
@@ -32,6 +35,17 @@ constexpr float kSixS = 0x1p64f * 6.0f;
 // overlap the tail of the one before it; launched without it, both
 // instructions are no-ops.
 // ---------------------------------------------------------------------------
+// Acquire load / release store at GPU scope (the grid barrier of the
+// one-launch capture).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void pdl_begin() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");

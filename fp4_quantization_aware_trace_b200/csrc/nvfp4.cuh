@@ -162,42 +162,33 @@ __device__ __forceinline__ GroupK group_consts_of_sg(float s_g) {
 
 // ---------------------------------------------------------------------------
 // Kernel 1: per-group amax (bits of max|x| as bf16, kept as u32 so that
-// atomicMax orders them as magnitudes), max-accumulated into amax[0, G).
-// A persistent grid (a few CTAs per SM), each thread with two tiles' loads in
-// flight.
-// FIN: the amax pass of a capture.  amax[G] is then a ticket counter; the
-// CTA that draws the last ticket -- after every CTA's accumulation is
-// visible -- takes the final amax of each group (reading and zeroing the
-// accumulator in one exchange), writes its s_g to gscale, and zeroes the
-// ticket: the workspace is zero again for the next call, and the quantising
-// pass reads only gscale.
+// atomicMax orders them as magnitudes), max-accumulated into amax[0, G):
+// the first pass of a capture whose tensor is split into row shards or
+// chunks (the one-launch capture below reduces inside its own grid).
 // ---------------------------------------------------------------------------
-template <bool FIN>
-__global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_amax(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
-           uint32_t* __restrict__ amax, float* __restrict__ gscale) {
+           uint32_t* __restrict__ amax) {
   __shared__ uint32_t table[kAmaxTable];
   __shared__ int g_first_s;
-  __shared__ uint32_t last_s;
   pdl_begin();
+  if (blockIdx.x >= sh.ntiles) return;
 
-  // tiles t (A) and t + gridDim.x (B) in flight; the first loads go out
-  // before the CTA's set-up barrier
-  const uint32_t step = gridDim.x;
-  V8 a0, a1, b0, b1;
-  auto load = [&](uint32_t t, V8& v0, V8& v1) {
-    const uint32_t b = t * kTileBlks + threadIdx.x;
-    v0 = (t < sh.ntiles && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
-    v1 = (t < sh.ntiles && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads)
-                                                     : zero_block();
-  };
-  load(blockIdx.x, a0, a1);
-  load(blockIdx.x + step, b0, b1);
+  // the first tile's loads go out before the CTA's set-up barrier
+  V8 v[kBlkPerThread];
+  {
+    const uint32_t base = blockIdx.x * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
+    }
+  }
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (sh.G > 1) {
     if (threadIdx.x == 0) {
-      gc.seek(blockIdx.x < sh.ntiles ? fastdiv(blockIdx.x * kTileBlks, sh.bpr) : 0u);
+      gc.seek(fastdiv(blockIdx.x * kTileBlks, sh.bpr));
       g_first_s = gc.g;
     }
     for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
@@ -210,38 +201,40 @@ __global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
   gc.init(offs, sh.G);
 
   uint32_t run = 0u;
-  int run_g = sh.G > 1 ? -1 : 0;
+  int run_g = -1;
   auto flush = [&](int g, uint32_t val) {
     if (g < 0 || val == 0u) return;
     const int slot = g - g_first;
     if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
     else atomicMax(&amax[g], val);
   };
-  auto take = [&](uint32_t t, const V8& v0, const V8& v1) {
-    if (sh.G == 1) {  // blocks past the end were loaded as zeros
-      run = max(run, max(absmax_block(v0), absmax_block(v1)));
-      return;
-    }
-    const uint32_t b = t * kTileBlks + threadIdx.x;
+
+  for (uint32_t t = blockIdx.x; t < sh.ntiles;) {
+    const uint32_t base = t * kTileBlks + threadIdx.x;
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const uint32_t bu = b + u * kThreads;
-      if (bu >= sh.nblk) continue;
-      gc.seek(fastdiv(bu, sh.bpr));
-      if (gc.g != run_g) {
-        flush(run_g, run);
-        run = 0u;
-        run_g = gc.g;
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = base + u * kThreads;
+      if (b >= sh.nblk) continue;
+      if (sh.G > 1) {
+        gc.seek(fastdiv(b, sh.bpr));
+        if (gc.g != run_g) {
+          flush(run_g, run);
+          run = 0u;
+          run_g = gc.g;
+        }
+      } else {
+        run_g = 0;
       }
-      run = max(run, absmax_block(u == 0 ? v0 : v1));
+      run = max(run, absmax_block(v[u]));
     }
-  };
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += 2u * step) {
-    take(t, a0, a1);
-    load(t + 2u * step, a0, a1);
-    if (t + step >= sh.ntiles) break;
-    take(t + step, b0, b1);
-    load(t + 3u * step, b0, b1);
+    t += gridDim.x;
+    if (t >= sh.ntiles) break;
+    const uint32_t nb = t * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < kBlkPerThread; ++u) {
+      const uint32_t b = nb + u * kThreads;
+      v[u] = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
+    }
   }
   if (sh.G == 1) {
     run = __reduce_max_sync(0xFFFFFFFFu, run);
@@ -251,30 +244,13 @@ __global__ void __launch_bounds__(kThreads, kAmaxCtasPerSm)
   }
   __syncthreads();
   if (sh.G == 1) {
-    if (threadIdx.x != 0) return;
-    if (table[0]) atomicMax(&amax[0], table[0]);
-    if (!FIN) return;
-    __threadfence();  // this CTA's maximum before its ticket
-    if (atomicAdd(&amax[1], 1u) != gridDim.x - 1u) return;
-    __threadfence();
-    gscale[0] = group_consts(atomicExch(&amax[0], 0u)).s_g;
-    amax[1] = 0u;
+    if (threadIdx.x == 0 && table[0]) atomicMax(&amax[0], table[0]);
     return;
   }
   for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
     const uint32_t val = table[i];
     if (val && g_first + i < sh.G) atomicMax(&amax[g_first + i], val);
   }
-  if (!FIN) return;
-  __threadfence();  // each thread's maxima before the CTA's ticket
-  __syncthreads();
-  if (threadIdx.x == 0) last_s = atomicAdd(&amax[sh.G], 1u) == gridDim.x - 1u;
-  __syncthreads();
-  if (!last_s) return;
-  __threadfence();
-  for (int g = threadIdx.x; g < sh.G; g += kThreads)
-    gscale[g] = group_consts(atomicExch(&amax[g], 0u)).s_g;
-  if (threadIdx.x == 0) amax[sh.G] = 0u;
 }
 
 // ---------------------------------------------------------------------------
@@ -345,11 +321,10 @@ __device__ __forceinline__ void codes_block(const V8& v, const V8* src, float d,
 // Each thread owns two adjacent blocks: one 16-byte store of codes, one
 // 32-bit store of mantissa bits, one 16-bit store of scales.
 // SW: scales in the tiled layout of a block-scaled GEMM instead of row-major.
-// PRE: the amax pass of the same capture has written gscale, and the group
-// constants are taken from it; otherwise they are computed here from the
-// given per-group amax words, and this pass writes gscale.  Nothing waits on
-// another CTA.
-template <bool SW, bool PRE>
+// The quantising pass given the per-group amax words (of a sharded or
+// chunk-streamed tensor): the group constants are computed from them, and
+// this pass writes gscale.
+template <bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
               const uint32_t* __restrict__ amax, uint4* __restrict__ codes,
@@ -359,9 +334,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   GroupCursor gc;
   gc.init(offs, sh.G);
   GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
-  // tiles in reverse order: the amax pass read the high tiles last, so they
-  // are the most likely to be still in L2.  The first tile's loads go out
-  // before anything else.
+  // tiles in reverse order: an amax pass just before read the high tiles
+  // last, so they are the most likely to be still in L2.  The first tile's
+  // loads go out before anything else.
   uint32_t i = blockIdx.x;
   auto tile_base = [&](uint32_t k) { return (sh.ntiles - 1u - k) * kTileBlks + 2u * threadIdx.x; };
   V8 v0 = zero_block(), v1 = zero_block();
@@ -369,11 +344,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     v0 = ld_block_stream(x + tile_base(i));
     v1 = ld_block_stream(x + tile_base(i) + 1);
   }
-  if (!PRE) {
-    // global scales of all groups (any CTA may write them; all write the same)
-    for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
-      gscale[g] = group_consts(__ldcg(amax + g)).s_g;
-  }
+  // global scales of all groups (any CTA may write them; all write the same)
+  for (int g = blockIdx.x * kThreads + threadIdx.x; g < sh.G; g += gridDim.x * kThreads)
+    gscale[g] = group_consts(__ldcg(amax + g)).s_g;
 
   for (; i < sh.ntiles; i += gridDim.x) {
     const uint32_t b = tile_base(i);  // even; nblk is even
@@ -381,8 +354,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (b < sh.nblk) {
       // both blocks of the pair are in the same row (cols is a multiple of 32)
       const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
-      if (gc.seek(row))
-        gk = PRE ? group_consts_of_sg(__ldcg(gscale + gc.g)) : group_consts(__ldcg(amax + gc.g));
+      if (gc.seek(row)) gk = group_consts(__ldcg(amax + gc.g));
       const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
       float sb0, sb1;
       e4m3x2_to_f32(s2, sb0, sb1);
@@ -406,6 +378,190 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     if (inext < sh.ntiles && tile_base(inext) < sh.nblk) {
       v0 = ld_block_stream(x + tile_base(inext));
       v1 = ld_block_stream(x + tile_base(inext) + 1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2': capture in one launch.  A cooperative grid (every CTA resident
+// at once, at most a few per SM): each CTA reduces the amax of its tiles
+// into the accumulators, the CTAs meet at a grid barrier, and each CTA then
+// quantises the same tiles in reverse order, so that it starts on what it
+// read last (in L2 on tensors that fit there).  The barrier's last arriving
+// CTA takes each group's final amax, zeroes its accumulator, writes s_g to
+// gscale and releases the others, which read their constants from gscale.
+// Workspace (u32): [0] arrival count (zero between calls), [1] generation
+// (counts calls), [2] error flag (set if a CTA gave up waiting), [3] unused,
+// [4, 4 + G) the accumulators (zero between calls).
+// ---------------------------------------------------------------------------
+template <bool SW>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    k_capture_coop(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
+                   uint32_t* __restrict__ ws, uint4* __restrict__ codes,
+                   uint32_t* __restrict__ mbits, uint8_t* __restrict__ scales,
+                   float* __restrict__ gscale) {
+  __shared__ uint32_t table[kAmaxTable];
+  __shared__ int g_first_s;
+  __shared__ uint32_t gen_s, last_s, ok_s;
+  uint32_t* const cnt = ws;
+  uint32_t* const gen = ws + 1;
+  uint32_t* const err = ws + 2;
+  uint32_t* const acc = ws + 4;
+  const uint32_t step = gridDim.x;
+
+  // ---- phase 1: amax of this CTA's tiles (t = blockIdx.x + k * step), two
+  // tiles in flight per thread; the first loads go out before the set-up
+  V8 a0, a1, b0, b1;
+  auto load = [&](uint32_t t, V8& v0, V8& v1) {
+    const uint32_t b = t * kTileBlks + threadIdx.x;
+    v0 = (t < sh.ntiles && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
+    v1 = (t < sh.ntiles && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads)
+                                                     : zero_block();
+  };
+  load(blockIdx.x, a0, a1);
+  load(blockIdx.x + step, b0, b1);
+  GroupCursor gc;
+  gc.init(offs, sh.G);
+  if (threadIdx.x == 0) gen_s = ld_acquire_gpu(gen);  // before this CTA's arrival
+  if (sh.G > 1) {
+    if (threadIdx.x == 0) {
+      gc.seek(blockIdx.x < sh.ntiles ? fastdiv(blockIdx.x * kTileBlks, sh.bpr) : 0u);
+      g_first_s = gc.g;
+    }
+    for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
+  } else if (threadIdx.x == 0) {
+    table[0] = 0u;
+    g_first_s = 0;
+  }
+  __syncthreads();
+  const int g_first = g_first_s;
+  gc.init(offs, sh.G);
+  uint32_t run = 0u;
+  int run_g = sh.G > 1 ? -1 : 0;
+  auto flush = [&](int g, uint32_t val) {
+    if (g < 0 || val == 0u) return;
+    const int slot = g - g_first;
+    if (slot >= 0 && slot < kAmaxTable) atomicMax(&table[slot], val);
+    else atomicMax(&acc[g], val);
+  };
+  auto take = [&](uint32_t t, const V8& v0, const V8& v1) {
+    if (sh.G == 1) {  // blocks past the end were loaded as zeros
+      run = max(run, max(absmax_block(v0), absmax_block(v1)));
+      return;
+    }
+    const uint32_t b = t * kTileBlks + threadIdx.x;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t bu = b + u * kThreads;
+      if (bu >= sh.nblk) continue;
+      gc.seek(fastdiv(bu, sh.bpr));
+      if (gc.g != run_g) {
+        flush(run_g, run);
+        run = 0u;
+        run_g = gc.g;
+      }
+      run = max(run, absmax_block(u == 0 ? v0 : v1));
+    }
+  };
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += 2u * step) {
+    take(t, a0, a1);
+    load(t + 2u * step, a0, a1);
+    if (t + step >= sh.ntiles) break;
+    take(t + step, b0, b1);
+    load(t + 3u * step, b0, b1);
+  }
+  if (sh.G == 1) {
+    run = __reduce_max_sync(0xFFFFFFFFu, run);
+    if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
+  } else {
+    flush(run_g, run);
+  }
+  __syncthreads();
+  if (sh.G == 1) {
+    if (threadIdx.x == 0 && table[0]) atomicMax(&acc[0], table[0]);
+  } else {
+    for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
+      const uint32_t val = table[i];
+      if (val && g_first + i < sh.G) atomicMax(&acc[g_first + i], val);
+    }
+  }
+
+  // ---- grid barrier
+  __threadfence();  // this thread's maxima before the CTA's arrival
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    last_s = atomicAdd(cnt, 1u) == step - 1u;
+    ok_s = 1u;
+  }
+  __syncthreads();
+  if (last_s) {
+    __threadfence();
+#pragma unroll 4
+    for (int g = threadIdx.x; g < sh.G; g += kThreads) {
+      const uint32_t a = __ldcg(acc + g);
+      acc[g] = 0u;
+      gscale[g] = group_consts(a).s_g;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      *cnt = 0u;
+      __threadfence();  // the global scales and the reset before the release
+      st_release_gpu(gen, gen_s + 1u);
+    }
+  } else if (threadIdx.x == 0) {
+    uint32_t polls = 0u;
+    while (ld_acquire_gpu(gen) == gen_s) {
+      if (++polls >= kBarrierPolls) {
+        atomicExch(err, 1u);
+        ok_s = 0u;
+        break;
+      }
+      __nanosleep(256);
+    }
+  }
+  __syncthreads();
+  if (!ok_s) return;
+
+  // ---- phase 2: quantise the same tiles, last first; two adjacent blocks
+  // per thread
+  const uint32_t ntile_cta =
+      blockIdx.x < sh.ntiles ? (sh.ntiles - 1u - blockIdx.x) / step + 1u : 0u;
+  gc.init(offs, sh.G);
+  GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
+  auto tile_base = [&](uint32_t k) { return (blockIdx.x + k * step) * kTileBlks + 2u * threadIdx.x; };
+  V8 v0 = zero_block(), v1 = zero_block();
+  if (ntile_cta > 0u && tile_base(ntile_cta - 1u) < sh.nblk) {
+    v0 = ld_block_stream(x + tile_base(ntile_cta - 1u));
+    v1 = ld_block_stream(x + tile_base(ntile_cta - 1u) + 1);
+  }
+  for (uint32_t k = ntile_cta; k-- > 0u;) {
+    const uint32_t b = tile_base(k);  // even; nblk is even
+    if (b < sh.nblk) {
+      const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+      if (gc.seek(row)) gk = group_consts_of_sg(__ldcg(gscale + gc.g));
+      const uint32_t s2 = pair_scale_bytes(v0, v1, gk);
+      float sb0, sb1;
+      e4m3x2_to_f32(s2, sb0, sb1);
+      const float d0 = __fmul_rn(gk.s_g, sb0), d1 = __fmul_rn(gk.s_g, sb1);
+      uint4 c;
+      if (fast_scale(d0) && fast_scale(d1)) {
+        codes_fast(v0, d0, c.x, c.y);
+        codes_fast(v1, d1, c.z, c.w);
+      } else {
+        codes_block(v0, x + b, d0, c.x, c.y);
+        codes_block(v1, x + b + 1, d1, c.z, c.w);
+      }
+      codes[b >> 1] = c;
+      mbits[b >> 1] = nibble_lsbs4(c);
+      const uint16_t sv = (uint16_t)s2;
+      if (SW)
+        *reinterpret_cast<uint16_t*>(scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)) = sv;
+      else
+        reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
+    }
+    if (k > 0u && tile_base(k - 1u) < sh.nblk) {
+      v0 = ld_block_stream(x + tile_base(k - 1u));
+      v1 = ld_block_stream(x + tile_base(k - 1u) + 1);
     }
   }
 }

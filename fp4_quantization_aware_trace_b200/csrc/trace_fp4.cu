@@ -111,17 +111,6 @@ Shape make_shape(int64_t rows, int64_t cols, int32_t G) {
   return sh;
 }
 
-// The amax pass: a persistent grid (each CTA walks many tiles), at least
-// one CTA (the capture's amax pass writes the constants even for no rows).
-int amax_grid_for(const Shape& sh, int* grid) {
-  const int sms = sm_count();
-  if (sms <= 0) return TRACE_ERR_CUDA;
-  uint32_t g = (uint32_t)sms * kAmaxCtasPerSm;
-  if (sh.ntiles < g) g = sh.ntiles;
-  *grid = (int)(g > 0 ? g : 1);
-  return TRACE_OK;
-}
-
 int grid_for(const Shape& sh, int* grid) {
   const int sms = sm_count();
   if (sms <= 0) return TRACE_ERR_CUDA;
@@ -224,6 +213,49 @@ int mx8_launch(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* mb
                       (const V8*)rcodes, scales, (V8*)out, mask);
 }
 
+// A cooperative launch (every CTA resident at once; the one-launch capture's
+// grid barrier relies on it).
+template <typename... KArgs, typename... Args>
+int launch_coop(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? TRACE_OK
+                                                                                      : TRACE_ERR_CUDA;
+}
+
+// Grid of the one-launch capture: as many CTAs as can be resident at once
+// (the occupancy of that kernel on this device, queried once), at most one
+// per tile, at least one.
+int g_coop_per_sm[kMaxDevices][2];  // 0 = not queried yet (benign race: same value)
+
+template <bool SW>
+int coop_grid_for(const Shape& sh, int* grid) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TRACE_ERR_CUDA;
+  int per_sm = g_coop_per_sm[dev][SW ? 1 : 0];
+  if (per_sm <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_capture_coop<SW>, kThreads, 0) !=
+            cudaSuccess ||
+        per_sm <= 0)
+      return TRACE_ERR_CUDA;
+    g_coop_per_sm[dev][SW ? 1 : 0] = per_sm;
+  }
+  const int sms = sm_count();
+  if (sms <= 0) return TRACE_ERR_CUDA;
+  uint32_t g = (uint32_t)sms * (uint32_t)per_sm;
+  if (sh.ntiles < g) g = sh.ntiles;
+  *grid = (int)(g > 0 ? g : 1);
+  return TRACE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -244,8 +276,9 @@ int trace_abi_version(void) { return TRACE_ABI_VERSION; }
 
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
   if (rows < 0 || cols <= 0 || cols % 32 != 0 || num_groups < 1) return 0;
-  // G accumulators and the amax pass's ticket counter
-  return ((size_t)num_groups * 4u + 4u + 255u) / 256u * 256u;
+  // an arrival count, a generation, an error flag, one unused word, then
+  // the G accumulators
+  return ((size_t)num_groups * 4u + 16u + 255u) / 256u * 256u;
 }
 
 size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
@@ -263,10 +296,10 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
   return up16(og + 4u * (size_t)num_groups);
 }
 
-// zero_first: zero the accumulators and the ticket with a launch of their
-// own before the amax pass (the static-scratch entry point, whose array
-// other calls share); otherwise they hold zeros on entry, as every capture
-// leaves them: the amax pass's last CTA resets them (a ticket).
+// One cooperative launch (k_capture_coop).  zero_first: zero the workspace
+// with a launch of its own first (the static-scratch entry point, whose
+// array other calls share); otherwise it is as the previous call left it
+// (zeros before the first): the arrival count and the accumulators zero.
 static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
                         const int64_t* group_row_offsets, uint8_t* codes, uint32_t* mbits,
                         uint8_t* scales, float* gscale, void* workspace, size_t workspace_bytes,
@@ -282,25 +315,18 @@ static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t n
     return TRACE_ERR_ALIGN;
   if (workspace_bytes < trace_capture_workspace_bytes(rows, cols, num_groups)) return TRACE_ERR_WORKSPACE;
   const Shape sh = make_shape(rows, cols, num_groups);
-  int grid, agrid;
-  if ((st = grid_for(sh, &grid)) || (st = amax_grid_for(sh, &agrid))) return st;
+  int grid;
+  if ((st = tiled ? coop_grid_for<true>(sh, &grid) : coop_grid_for<false>(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
-  uint32_t* acc = (uint32_t*)workspace;
+  uint32_t* ws = (uint32_t*)workspace;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
-  const int zg = (num_groups + 1 + kThreads - 1) / kThreads;
-  if (zero_first && (st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, acc, (int)num_groups + 1)))
-    return st;
-  st = launch(k_amax<true>, agrid, s, (const V8*)x, sh, offs, acc, gscale);
-  if (st == TRACE_OK && sh.nblk > 0) {
-    const uint32_t* no_amax = nullptr;
-    st = tiled ? launch(k_capture<true, true>, grid, s, (const V8*)x, sh, offs, no_amax,
-                        (uint4*)codes, (uint32_t*)mbits, scales, gscale)
-               : launch(k_capture<false, true>, grid, s, (const V8*)x, sh, offs, no_amax,
-                        (uint4*)codes, (uint32_t*)mbits, scales, gscale);
-  }
-  // a failed launch could leave the accumulators set: clear them (best effort)
-  if (st != TRACE_OK) (void)cudaMemsetAsync(workspace, 0, ((size_t)num_groups + 1) * 4u, s);
-  return st;
+  const int zn = (int)num_groups + 4;
+  const int zg = (zn + kThreads - 1) / kThreads;
+  if (zero_first && (st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, ws, zn))) return st;
+  return tiled ? launch_coop(k_capture_coop<true>, grid, s, (const V8*)x, sh, offs, ws,
+                             (uint4*)codes, (uint32_t*)mbits, scales, gscale)
+               : launch_coop(k_capture_coop<false>, grid, s, (const V8*)x, sh, offs, ws,
+                             (uint4*)codes, (uint32_t*)mbits, scales, gscale);
 }
 
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
@@ -485,13 +511,13 @@ int trace_capture_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t nu
   if (!aligned(x, 32) || !aligned(amax, 4)) return TRACE_ERR_ALIGN;
   const Shape sh = make_shape(rows, cols, num_groups);
   int grid;
-  if ((st = amax_grid_for(sh, &grid))) return st;
+  if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int zg = (num_groups + kThreads - 1) / kThreads;
   if ((st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, amax, (int)num_groups))) return st;
   if (sh.nblk == 0) return TRACE_OK;
-  return launch(k_amax<false>, grid, s, (const V8*)x, sh,
-                num_groups > 1 ? group_row_offsets : nullptr, amax, (float*)nullptr);
+  return launch(k_amax, grid, s, (const V8*)x, sh, num_groups > 1 ? group_row_offsets : nullptr,
+                amax);
 }
 
 int trace_capture_amax_accumulate(const uint16_t* x, int64_t rows, int64_t cols,
@@ -504,9 +530,9 @@ int trace_capture_amax_accumulate(const uint16_t* x, int64_t rows, int64_t cols,
   const Shape sh = make_shape(rows, cols, num_groups);
   if (sh.nblk == 0) return TRACE_OK;
   int grid;
-  if ((st = amax_grid_for(sh, &grid))) return st;
-  return launch(k_amax<false>, grid, (cudaStream_t)stream, (const V8*)x, sh,
-                num_groups > 1 ? group_row_offsets : nullptr, amax, (float*)nullptr);
+  if ((st = grid_for(sh, &grid))) return st;
+  return launch(k_amax, grid, (cudaStream_t)stream, (const V8*)x, sh,
+                num_groups > 1 ? group_row_offsets : nullptr, amax);
 }
 
 int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
@@ -526,10 +552,10 @@ int trace_capture_with_amax(const uint16_t* x, int64_t rows, int64_t cols, int32
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
   if (scale_layout == TRACE_SCALES_TILED_128x4)
-    return launch(k_capture<true, false>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes,
-                  mbits, scales, gscale);
-  return launch(k_capture<false, false>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes,
-                mbits, scales, gscale);
+    return launch(k_capture<true>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes, mbits,
+                  scales, gscale);
+  return launch(k_capture<false>, grid, s, (const V8*)x, sh, offs, amax, (uint4*)codes, mbits,
+                scales, gscale);
 }
 
 int trace_capture_ex(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,
@@ -740,7 +766,7 @@ int trace_copy_bf16_staged(const uint16_t* src, uint16_t* dst, int64_t numel, ui
 // that trace_capture takes as `workspace` in a fixed array that lives in the
 // library itself, one copy per GPU, for the life of the process.
 // ---------------------------------------------------------------------------
-// TRACE_STATIC_MAX_GROUPS accumulators, the amax pass's ticket counter and
+// TRACE_STATIC_MAX_GROUPS accumulators, the four words before them and
 // padding to a multiple of 256 bytes
 static __device__ __align__(256) uint32_t g_capture_scratch[TRACE_STATIC_MAX_GROUPS + 64];
 
@@ -771,8 +797,7 @@ int trace_capture_static_ws(const uint16_t* x, int64_t rows, int64_t cols, int32
       return TRACE_ERR_CUDA;
     g_capture_scratch_addr[dev] = ws = a;
   }
-  // the accumulators are zeroed by the capture's first kernel on every call
-  // (and left zeroed by the amax pass)
+  // the array is zeroed by the capture's first kernel on every call
   return capture_impl(x, rows, cols, num_groups, group_row_offsets, codes, mbits, scales, gscale,
                       ws, sizeof(g_capture_scratch), false, stream, true);
 }

@@ -92,9 +92,9 @@ const char* trace_strerror(int status);
 #define TRACE_ABI_VERSION 2
 int trace_abi_version(void);
 
-/* Bytes of device workspace that trace_capture needs for G groups: the
- * per-group amax accumulators (4 bytes each) and a ticket counter, rounded
- * up to 256.  Returns 0 when the shape is invalid. */
+/* Bytes of device workspace that trace_capture needs for G groups: four
+ * words of grid-barrier state, then the per-group amax accumulators (4 bytes
+ * each), rounded up to 256.  Returns 0 when the shape is invalid. */
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols,
                                      int32_t num_groups);
 
@@ -126,13 +126,19 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
  *   workspace: device scratch of at least trace_capture_workspace_bytes()
  *             bytes, 256-byte aligned, holding zeros before its first use
  *             (e.g. cudaMemsetAsync once, when it is allocated); every call
- *             leaves it all-zero again, so a workspace can serve any number
- *             of calls one after another (not two calls that may run at the
- *             same time).
- * Launches the grid amax (max-accumulated into the workspace; the CTA that
- * draws the last ticket -- an atomic counter in the workspace; nothing waits
- * -- writes gscale and sets the workspace back to zero) and the quantising
- * pass, which reads gscale. */
+ *             leaves it ready for the next, so a workspace can serve any
+ *             number of calls one after another (not two calls that may run
+ *             at the same time).  Words: [0] an arrival count and [4, 4+G)
+ *             the accumulators, both zero again after every call; [1] counts
+ *             calls; [2] is set to nonzero if a CTA ever gave up waiting at
+ *             the grid barrier (about a second; with the cooperative launch
+ *             every CTA is resident, so it is not expected), in which case
+ *             that call's outputs are not valid; [3] is unused.
+ * One cooperative launch (every CTA resident at once, a few per SM): each
+ * CTA max-accumulates the amax of its tiles into the workspace, the CTAs
+ * meet at a grid barrier whose last arriving CTA writes gscale and zeroes
+ * the accumulators, and each CTA then quantises its own tiles, last read
+ * first (from L2 where the tensor fits there). */
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
                   int32_t num_groups, const int64_t* group_row_offsets,
                   uint8_t* codes, uint32_t* mbits, uint8_t* scales,
@@ -425,7 +431,7 @@ int trace_copy_bf16_staged(const uint16_t* src, uint16_t* dst, int64_t numel,
  * start-up, or a binding that can only pass along the buffers it was given.
  * Instead of a `workspace` argument, the amax accumulators live in a static
  * array inside the library: TRACE_STATIC_MAX_GROUPS + 64 uint32 (16.25 KiB:
- * the accumulators, a ticket counter and padding) per GPU that loads the
+ * the accumulators, the barrier's state and padding) per GPU that loads the
  * library, kept until the process exits.
  *   Arguments and outputs are those of trace_capture without `workspace`.
  *   num_groups > TRACE_STATIC_MAX_GROUPS: returns TRACE_ERR_WORKSPACE and

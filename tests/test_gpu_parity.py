@@ -538,10 +538,12 @@ def test_step_in_a_cuda_graph(oracle_mod, forked):
 
 
 def test_workspace_left_zeroed_and_reused(oracle_mod):
-    """Capture leaves its workspace all-zero (the quantising pass's last CTA
-    resets the accumulators and the ticket), so one workspace serves calls
-    one after another: a tensor with a huge maximum, then ragged groups of
-    small values, then an empty tensor -- each matches the oracle."""
+    """Capture leaves its workspace ready for the next call -- the arrival
+    count and the accumulators zero (the grid barrier's last CTA resets
+    them), the error flag clear, the call count advanced by one -- so one
+    workspace serves calls one after another: a tensor with a huge maximum,
+    then ragged groups of small values, then an empty tensor -- each matches
+    the oracle."""
     cases = []
     a = inputs.tiny_site(501, 700, 256).x_roll.float()
     a[13, 7] = 3.0e5
@@ -551,14 +553,16 @@ def test_workspace_left_zeroed_and_reused(oracle_mod):
     cases.append((torch.zeros(0, 64, dtype=torch.bfloat16), None))
     G_max = 3
     ws = torch.zeros(ops.trace_capture_workspace_bytes(1, 32, G_max), dtype=torch.uint8, device=DEV)
-    for x, offs in cases:
+    for k, (x, offs) in enumerate(cases):
         R, C = x.shape
         G = 1 if offs is None else len(offs) - 1
         o = None if offs is None else torch.from_numpy(offs).to(DEV)
         cap, _ = ops.alloc_capture(R, C, G, DEV, o)
         ops.capture(x.to(DEV), o, cap, ws)
         torch.cuda.synchronize()
-        assert int(ws.count_nonzero()) == 0
+        w = ws.view(torch.int32).cpu()
+        assert int(w[0]) == 0 and int(w[2]) == 0 and int(w[1]) == k + 1
+        assert int(w[3:].count_nonzero()) == 0
         ref = oracle_mod.capture(inputs.bits(x), G, offs)
         for name, got, want in zip(("codes", "mbits", "scales", "gscale"),
                                    (cap.codes, cap.mbits, cap.scales, cap.gscale), ref):
