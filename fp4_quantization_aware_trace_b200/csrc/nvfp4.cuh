@@ -384,7 +384,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // ---------------------------------------------------------------------------
 // Kernel 2': capture in one launch.  A cooperative grid (every CTA resident
-// at once, at most a few per SM): each CTA reduces the amax of its tiles
+// at once, at most a few per SM): each CTA reduces the amax of its tiles --
+// one contiguous range of tiles per CTA, so that a CTA meets few groups --
 // into the accumulators, the CTAs meet at a grid barrier, and each CTA then
 // quantises the same tiles in reverse order, so that it starts on what it
 // read last (in L2 on tensors that fit there).  The barrier's last arriving
@@ -407,25 +408,27 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint32_t* const gen = ws + 1;
   uint32_t* const err = ws + 2;
   uint32_t* const acc = ws + 4;
-  const uint32_t step = gridDim.x;
+  // this CTA's tiles: [t0, t1), nonempty when there are tiles (the grid has
+  // at most one CTA per tile)
+  const uint32_t t0 = (uint32_t)((uint64_t)blockIdx.x * sh.ntiles / gridDim.x);
+  const uint32_t t1 = (uint32_t)((uint64_t)(blockIdx.x + 1u) * sh.ntiles / gridDim.x);
 
-  // ---- phase 1: amax of this CTA's tiles (t = blockIdx.x + k * step), two
-  // tiles in flight per thread; the first loads go out before the set-up
+  // ---- phase 1: amax of the CTA's tiles, two in flight per thread; the
+  // first loads go out before the set-up
   V8 a0, a1, b0, b1;
   auto load = [&](uint32_t t, V8& v0, V8& v1) {
     const uint32_t b = t * kTileBlks + threadIdx.x;
-    v0 = (t < sh.ntiles && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
-    v1 = (t < sh.ntiles && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads)
-                                                     : zero_block();
+    v0 = (t < t1 && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
+    v1 = (t < t1 && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads) : zero_block();
   };
-  load(blockIdx.x, a0, a1);
-  load(blockIdx.x + step, b0, b1);
+  load(t0, a0, a1);
+  load(t0 + 1u, b0, b1);
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (threadIdx.x == 0) gen_s = ld_acquire_gpu(gen);  // before this CTA's arrival
   if (sh.G > 1) {
     if (threadIdx.x == 0) {
-      gc.seek(blockIdx.x < sh.ntiles ? fastdiv(blockIdx.x * kTileBlks, sh.bpr) : 0u);
+      gc.seek(t0 < t1 ? fastdiv(t0 * kTileBlks, sh.bpr) : 0u);
       g_first_s = gc.g;
     }
     for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) table[i] = 0u;
@@ -463,12 +466,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       run = max(run, absmax_block(u == 0 ? v0 : v1));
     }
   };
-  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += 2u * step) {
+  for (uint32_t t = t0; t < t1; t += 2u) {
     take(t, a0, a1);
-    load(t + 2u * step, a0, a1);
-    if (t + step >= sh.ntiles) break;
-    take(t + step, b0, b1);
-    load(t + 3u * step, b0, b1);
+    load(t + 2u, a0, a1);
+    if (t + 1u >= t1) break;
+    take(t + 1u, b0, b1);
+    load(t + 3u, b0, b1);
   }
   if (sh.G == 1) {
     run = __reduce_max_sync(0xFFFFFFFFu, run);
@@ -490,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __threadfence();  // this thread's maxima before the CTA's arrival
   __syncthreads();
   if (threadIdx.x == 0) {
-    last_s = atomicAdd(cnt, 1u) == step - 1u;
+    last_s = atomicAdd(cnt, 1u) == gridDim.x - 1u;
     ok_s = 1u;
   }
   __syncthreads();
@@ -524,11 +527,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   // ---- phase 2: quantise the same tiles, last first; two adjacent blocks
   // per thread
-  const uint32_t ntile_cta =
-      blockIdx.x < sh.ntiles ? (sh.ntiles - 1u - blockIdx.x) / step + 1u : 0u;
+  const uint32_t ntile_cta = t1 - t0;
   gc.init(offs, sh.G);
   GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
-  auto tile_base = [&](uint32_t k) { return (blockIdx.x + k * step) * kTileBlks + 2u * threadIdx.x; };
+  auto tile_base = [&](uint32_t k) { return (t0 + k) * kTileBlks + 2u * threadIdx.x; };
   V8 v0 = zero_block(), v1 = zero_block();
   if (ntile_cta > 0u && tile_base(ntile_cta - 1u) < sh.nblk) {
     v0 = ld_block_stream(x + tile_base(ntile_cta - 1u));
