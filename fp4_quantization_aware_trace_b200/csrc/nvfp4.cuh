@@ -764,11 +764,18 @@ __device__ __forceinline__ void fq_block_fast(const V8& v, const uint16_t* src, 
 // is read back from x (a cache hit: the block was just read) instead of kept
 // in registers.  d, sbv: the pair's block; side as guided_pair (MODE kGuided:
 // the pair's two cached bits in bits 0 and 1; kFull: its two rollout codes).
+// r: RN(1/d), as the round-to-nearest pass took it.
 template <int MODE>
 __device__ __forceinline__ void patch_pair(const uint32_t* xw, uint32_t* ow, int q, float d,
-                                           float sbv, float s_g, uint32_t side) {
+                                           float r, float sbv, float s_g, uint32_t side) {
   if (fast_scale(d, kDMaxExactZ)) {
-    ow[q] = guided_pair<MODE>(__ldg(xw + q), side, make_blk(d, __fmul_rn(sbv, 0x1p-64f), s_g));
+    BlkK k;
+    k.rr = pk(r, r);
+    k.ndd = pk(-d, -d);
+    const float sbs = __fmul_rn(sbv, 0x1p-64f);  // exact
+    k.sbv2 = pk(sbs, sbs);
+    k.sg2 = pk(s_g, s_g);
+    ow[q] = guided_pair<MODE>(__ldg(xw + q), side, k);
   } else {
     const uint16_t* src = reinterpret_cast<const uint16_t*>(xw + q);
     const uint32_t lo = guided_site_fix(src, d, sbv, s_g, MODE == kGuided ? side & 1u : side & 0xFu,
@@ -847,12 +854,15 @@ __global__ void __launch_bounds__(kThreads, MINB)
     if (SEP && MODE != kRtn && fast_scale(d0) && fast_scale(d1)) {
       // the common case for separate output buffers
       V8 o;
-      const uint32_t bad0 =
-          fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, make_blk(d0, sbv0, s_g), o, m0);
+      const BlkK k0 = make_blk(d0, sbv0, s_g);
+      const uint32_t bad0 = fq_block_rtn<MODE>(v0, bits & 0xFFFFu, rc.x, rc.y, k0, o, m0);
       st_block(out + b, o);
-      const uint32_t bad1 =
-          fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, make_blk(d1, sbv1, s_g), o, m1);
+      const BlkK k1 = make_blk(d1, sbv1, s_g);
+      const uint32_t bad1 = fq_block_rtn<MODE>(v1, bits >> 16, rc.z, rc.w, k1, o, m1);
       st_block(out + b + 1, o);
+      float r0, r1, unused;
+      upk(k0.rr, r0, unused);
+      upk(k1.rr, r1, unused);
       uint32_t pairs = ((bad0 | (bad0 >> 1)) & 0x5555u) | (((bad1 | (bad1 >> 1)) & 0x5555u) << 16);
       const uint32_t* xw = reinterpret_cast<const uint32_t*>(x + b);
       uint32_t* ow = reinterpret_cast<uint32_t*>(out + b);
@@ -862,7 +872,8 @@ __global__ void __launch_bounds__(kThreads, MINB)
         const uint32_t side =
             MODE == kGuided ? bits >> (2 * q)
                             : (q < 4 ? rc.x : q < 8 ? rc.y : q < 12 ? rc.z : rc.w) >> (8 * (q & 3));
-        patch_pair<MODE>(xw, ow, q, q < 8 ? d0 : d1, q < 8 ? sbv0 : sbv1, s_g, side);
+        patch_pair<MODE>(xw, ow, q, q < 8 ? d0 : d1, q < 8 ? r0 : r1, q < 8 ? sbv0 : sbv1, s_g,
+                         side);
       }
     } else if (fast_scale(d0) && fast_scale(d1)) {
       // the common case, without per-block branches
