@@ -489,6 +489,16 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
 
+  // phase 2's first tile (the last one read) is loaded before the barrier,
+  // so that the wait covers its latency; x is not written by this kernel
+  const uint32_t ntile_cta = t1 - t0;
+  auto tile_base = [&](uint32_t k) { return (t0 + k) * kTileBlks + 2u * threadIdx.x; };
+  V8 v0 = zero_block(), v1 = zero_block();
+  if (ntile_cta > 0u && tile_base(ntile_cta - 1u) < sh.nblk) {
+    v0 = ld_block_stream(x + tile_base(ntile_cta - 1u));
+    v1 = ld_block_stream(x + tile_base(ntile_cta - 1u) + 1);
+  }
+
   // ---- grid barrier
   __threadfence();  // this thread's maxima before the CTA's arrival
   __syncthreads();
@@ -527,15 +537,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   // ---- phase 2: quantise the same tiles, last first; two adjacent blocks
   // per thread
-  const uint32_t ntile_cta = t1 - t0;
   gc.init(offs, sh.G);
   GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
-  auto tile_base = [&](uint32_t k) { return (t0 + k) * kTileBlks + 2u * threadIdx.x; };
-  V8 v0 = zero_block(), v1 = zero_block();
-  if (ntile_cta > 0u && tile_base(ntile_cta - 1u) < sh.nblk) {
-    v0 = ld_block_stream(x + tile_base(ntile_cta - 1u));
-    v1 = ld_block_stream(x + tile_base(ntile_cta - 1u) + 1);
-  }
   for (uint32_t k = ntile_cta; k-- > 0u;) {
     const uint32_t b = tile_base(k);  // even; nblk is even
     if (b < sh.nblk) {
