@@ -831,83 +831,22 @@ __global__ void __launch_bounds__(kThreads, MINB)
                  const uint32_t* __restrict__ mbits, const uint4* __restrict__ rcodes,
                  const uint8_t* __restrict__ scales, const float* __restrict__ gscale,
                  V8* __restrict__ out, uint32_t* __restrict__ mask) {
-  // A persistent grid (a few CTAs per SM) walks the tiles t = blockIdx.x +
-  // k * gridDim.x.  x (and the rollout codes) of the next two tiles are in
-  // flight into shared memory (cp.async, two stages per warp) while a tile
-  // is computed, and the small per-thread inputs (cached bits, scales) are
-  // loaded into registers a tile ahead, so that loads and arithmetic
-  // overlap inside every CTA instead of only across CTAs.  A warp copies its
-  // own 2 KiB of x with 512-byte contiguous copies; chunk c (16 bytes) of
-  // the warp's region sits at (c % 4) * 32 + c / 4, so that lane l finds
-  // its four chunks 4l .. 4l + 3 at l, 32 + l, 64 + l, 96 + l (no bank
-  // conflicts when they are read).
-  constexpr int kXChunks = 128;
-  constexpr int kWarpChunks = kXChunks + (MODE == kFull ? 32 : 0);
-  __shared__ uint4 stage[2][(kThreads / 32) * kWarpChunks];
   pdl_begin();
   GroupCursor gc;
   gc.init(offs, sh.G);
   float s_g = 1.0f;
-  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-  uint4* const wst0 = &stage[0][warp * kWarpChunks];
-  uint4* const wst1 = &stage[1][warp * kWarpChunks];
 
-  // x (and the rollout codes) of tile t into a stage: one commit group per
-  // tile, empty past the end
-  auto issue = [&](uint32_t t, uint4* wst) {
-    if (t < sh.ntiles) {
-      const uint32_t wb = t * kTileBlks + 64u * warp;  // the warp's first block
-      const char* src = reinterpret_cast<const char*>(x + wb);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint32_t c = 32u * j + lane;
-        if (wb + (c >> 1) < sh.nblk) cp_async16(wst + ((c & 3u) * 32u + (c >> 2)), src + 16u * c);
-      }
-      if (MODE == kFull && wb + 2u * lane < sh.nblk)
-        cp_async16(wst + kXChunks + lane, rcodes + ((wb >> 1) + lane));
-    }
-    cp_async_commit();
-  };
-  // cached bits and scale bytes of tile t
-  auto load_side = [&](uint32_t t, uint32_t& bits, uint32_t& sb2) {
-    const uint32_t b = t * kTileBlks + 2u * threadIdx.x;
-    if (t >= sh.ntiles || b >= sh.nblk) return;
-    if (MODE == kGuided) bits = __ldcs(mbits + (b >> 1));
-    if (SW) {
-      const uint32_t row = fastdiv(b, sh.bpr);
-      sb2 = __ldcs(reinterpret_cast<const unsigned short*>(
-          scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)));
-    } else {
-      sb2 = __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
-    }
-  };
-
-  uint32_t t = blockIdx.x;
-  issue(t, wst0);
-  issue(t + gridDim.x, wst1);
-  uint32_t nbits = 0u, nsb2 = 0u;
-  load_side(t, nbits, nsb2);
-  for (uint32_t k = 0u; t < sh.ntiles; t += gridDim.x, ++k) {
-    uint4* const wst = (k & 1u) ? wst1 : wst0;
+  for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
-    const uint32_t bits = nbits, sb2 = nsb2;
-    load_side(t + gridDim.x, nbits, nsb2);
-    cp_async_wait<1>();  // this thread's copies of tile t
-    __syncwarp();        // ... and the rest of the warp's
-    V8 v0, v1;
-    {
-      const uint4 u0 = wst[lane], u1 = wst[32u + lane], u2 = wst[64u + lane],
-                  u3 = wst[96u + lane];
-      v0.w[0] = u0.x; v0.w[1] = u0.y; v0.w[2] = u0.z; v0.w[3] = u0.w;
-      v0.w[4] = u1.x; v0.w[5] = u1.y; v0.w[6] = u1.z; v0.w[7] = u1.w;
-      v1.w[0] = u2.x; v1.w[1] = u2.y; v1.w[2] = u2.z; v1.w[3] = u2.w;
-      v1.w[4] = u3.x; v1.w[5] = u3.y; v1.w[6] = u3.z; v1.w[7] = u3.w;
-    }
-    const uint4 rc = MODE == kFull ? wst[kXChunks + lane] : make_uint4(0u, 0u, 0u, 0u);
-    __syncwarp();  // the warp has read the stage before it is refilled
-    issue(t + 2u * gridDim.x, wst);
     if (b >= sh.nblk) continue;
+    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
+    const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
+    const uint32_t sb2 =
+        SW ? __ldcs(reinterpret_cast<const unsigned short*>(
+                 scales + tiled_scale_offset(row, b - row * sh.bpr.d, sh.sw_ct)))
+           : __ldcs(reinterpret_cast<const unsigned short*>(scales) + (b >> 1));
     if (gc.seek(row)) s_g = __ldg(gscale + gc.g);
     uint32_t m0, m1;
     float sbv0, sbv1;
@@ -953,7 +892,6 @@ __global__ void __launch_bounds__(kThreads, MINB)
     }
     mask[b >> 1] = m0 | (m1 << 16);
   }
-  cp_async_wait<0>();  // no copy may land in this CTA's shared memory after it exits
 }
 
 // ---------------------------------------------------------------------------

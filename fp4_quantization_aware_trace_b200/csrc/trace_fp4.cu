@@ -111,17 +111,6 @@ Shape make_shape(int64_t rows, int64_t cols, int32_t G) {
   return sh;
 }
 
-// The persistent grid of k_fake_quant: kCtasPerSm CTAs per SM, at most one
-// per tile.
-int fq_grid_for(const Shape& sh, int* grid) {
-  const int sms = sm_count();
-  if (sms <= 0) return TRACE_ERR_CUDA;
-  uint32_t g = (uint32_t)sms * kCtasPerSm;
-  if (sh.ntiles < g) g = sh.ntiles;
-  *grid = (int)(g > 0 ? g : 1);
-  return TRACE_OK;
-}
-
 int grid_for(const Shape& sh, int* grid) {
   const int sms = sm_count();
   if (sms <= 0) return TRACE_ERR_CUDA;
@@ -150,33 +139,16 @@ int launch(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
                                                                                       : TRACE_ERR_CUDA;
 }
 
-// k_fake_quant keeps two stages of its tiles in shared memory (32 or 40 KiB
-// per CTA): ask once per build for the largest shared-memory carve-out, so
-// that kCtasPerSm of them fit on an SM.
-template <int MODE, bool SW, bool SEP>
-int fq_launch(int grid, cudaStream_t s, const uint16_t* x, const Shape& sh, const int64_t* o,
-              const uint32_t* mbits, const uint8_t* rcodes, const uint8_t* scales,
-              const float* gscale, uint16_t* out, uint32_t* mask) {
-  static bool carveout_set = false;  // benign race: the same attribute
-  auto* kernel = k_fake_quant<MODE, SW, kCtasPerSm, SEP>;
-  if (!carveout_set) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared) != cudaSuccess)
-      return TRACE_ERR_CUDA;
-    carveout_set = true;
-  }
-  return launch(kernel, grid, s, (const V8*)x, sh, o, mbits, (const uint4*)rcodes, scales, gscale,
-                (V8*)out, mask);
-}
-
 // The guided rules: SEP when out does not overlap x (see k_fake_quant).
 template <int MODE, bool SW>
 int guided_dispatch(bool sep, int grid, cudaStream_t s, const uint16_t* x, const Shape& sh,
                     const int64_t* o, const uint32_t* mbits, const uint8_t* rcodes,
                     const uint8_t* scales, const float* gscale, uint16_t* out, uint32_t* mask) {
   if (sep)
-    return fq_launch<MODE, SW, true>(grid, s, x, sh, o, mbits, rcodes, scales, gscale, out, mask);
-  return fq_launch<MODE, SW, false>(grid, s, x, sh, o, mbits, rcodes, scales, gscale, out, mask);
+    return launch(k_fake_quant<MODE, SW, kCtasPerSm, true>, grid, s, (const V8*)x, sh, o, mbits,
+                  (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
+  return launch(k_fake_quant<MODE, SW, kCtasPerSm, false>, grid, s, (const V8*)x, sh, o, mbits,
+                (const uint4*)rcodes, scales, gscale, (V8*)out, mask);
 }
 
 template <bool SW>
@@ -192,8 +164,8 @@ int fake_quant_dispatch(int mode, int grid, cudaStream_t s, const uint16_t* x,
   if (mode == kFull)
     return guided_dispatch<kFull, SW>(sep, grid, s, x, sh, o, nullptr, rcodes, scales, gscale, out,
                                       mask);
-  return fq_launch<kRtn, SW, false>(grid, s, x, sh, o, nullptr, nullptr, scales, gscale, out,
-                                    mask);
+  return launch(k_fake_quant<kRtn, SW>, grid, s, (const V8*)x, sh, o, (const uint32_t*)nullptr,
+                (const uint4*)nullptr, scales, gscale, (V8*)out, mask);
 }
 
 template <bool SW>
@@ -383,7 +355,7 @@ static int fake_quant_launch(int mode, const uint16_t* x, int64_t rows, int64_t 
   const Shape sh = make_shape(rows, cols, G);
   if (sh.nblk == 0) return TRACE_OK;
   int grid;
-  if ((st = fq_grid_for(sh, &grid))) return st;
+  if ((st = grid_for(sh, &grid))) return st;
   cudaStream_t s = (cudaStream_t)stream;
   const int64_t* o = G > 1 ? offs : nullptr;
   return tiled ? fake_quant_dispatch<true>(mode, grid, s, x, sh, o, mbits, rcodes, scales, gscale,
