@@ -413,9 +413,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const uint32_t t0 = (uint32_t)((uint64_t)blockIdx.x * sh.ntiles / gridDim.x);
   const uint32_t t1 = (uint32_t)((uint64_t)(blockIdx.x + 1u) * sh.ntiles / gridDim.x);
 
-  // ---- phase 1: amax of the CTA's tiles, two in flight per thread; the
-  // first loads go out before the set-up
-  V8 a0, a1, b0, b1;
+  // ---- phase 1: amax of the CTA's tiles, three in flight per thread (the
+  // quantising phase sets the register budget, so they cost no occupancy);
+  // the first loads go out before the set-up
+  V8 a0, a1, b0, b1, c0, c1;
   auto load = [&](uint32_t t, V8& v0, V8& v1) {
     const uint32_t b = t * kTileBlks + threadIdx.x;
     v0 = (t < t1 && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
@@ -423,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   };
   load(t0, a0, a1);
   load(t0 + 1u, b0, b1);
+  load(t0 + 2u, c0, c1);
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (threadIdx.x == 0) gen_s = ld_acquire_gpu(gen);  // before this CTA's arrival
@@ -466,12 +468,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       run = max(run, absmax_block(u == 0 ? v0 : v1));
     }
   };
-  for (uint32_t t = t0; t < t1; t += 2u) {
+  for (uint32_t t = t0; t < t1; t += 3u) {
     take(t, a0, a1);
-    load(t + 2u, a0, a1);
+    load(t + 3u, a0, a1);
     if (t + 1u >= t1) break;
     take(t + 1u, b0, b1);
-    load(t + 3u, b0, b1);
+    load(t + 4u, b0, b1);
+    if (t + 2u >= t1) break;
+    take(t + 2u, c0, c1);
+    load(t + 5u, c0, c1);
   }
   if (sh.G == 1) {
     run = __reduce_max_sync(0xFFFFFFFFu, run);
