@@ -93,6 +93,17 @@ __device__ __forceinline__ V8 ld_block_stream(const void* p) {
   return v;
 }
 
+// The same load kept in L1: for the guided forwards with separate outputs,
+// which read words of the block back for the pairs they recompute.
+__device__ __forceinline__ V8 ld_block_l1(const void* p) {
+  V8 v;
+  asm volatile("ld.global.nc.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]),
+                 "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+               : "l"(p));
+  return v;
+}
+
 // Block load and store for the rarely taken out-of-line (exact-path)
 // functions, as plain 16-byte accesses: with the 32-byte asm forms inside a
 // non-inlined function, ptxas 12.9 crashed (load) or, depending on the other

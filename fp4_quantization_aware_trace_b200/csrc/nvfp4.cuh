@@ -844,7 +844,11 @@ __global__ void __launch_bounds__(kThreads, MINB)
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
     if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    // with separate outputs the guided rules read words of x back (the
+    // pairs they recompute): keep the blocks in L1 for that
+    constexpr bool kKeepL1 = SEP && MODE != kRtn;
+    const V8 v0 = kKeepL1 ? ld_block_l1(x + b) : ld_block_stream(x + b);
+    const V8 v1 = kKeepL1 ? ld_block_l1(x + b + 1) : ld_block_stream(x + b + 1);
     const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
     const uint4 rc = MODE == kFull ? __ldcs(rcodes + (b >> 1)) : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
