@@ -389,9 +389,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   for (uint32_t t = blockIdx.x; t < sh.ntiles; t += gridDim.x) {
     const uint32_t b = t * kTileBlks + 2u * threadIdx.x;  // even; nblk is even
     if (b >= sh.nblk) continue;
-    const V8 v0 = ld_block_stream(x + b), v1 = ld_block_stream(x + b + 1);
+    // with separate outputs the guided rules read words of x (and halfwords
+    // of the rollout codes) back for the pairs they recompute: keep them in L1
+    constexpr bool kKeepL1 = SEP && MODE != kRtn;
+    const V8 v0 = kKeepL1 ? ld_block_l1(x + b) : ld_block_stream(x + b);
+    const V8 v1 = kKeepL1 ? ld_block_l1(x + b + 1) : ld_block_stream(x + b + 1);
     const uint32_t bits = MODE == kGuided ? __ldcs(mbits + (b >> 1)) : 0u;
-    const V8 rc = MODE == kFull ? ld_block_stream(rcodes + (b >> 1)) : zero_block();
+    const V8 rc = MODE != kFull ? zero_block()
+                  : kKeepL1     ? ld_block_l1(rcodes + (b >> 1))
+                                : ld_block_stream(rcodes + (b >> 1));
     size_t so = b >> 1;
     if (SW) {
       const uint32_t row = fastdiv(b, sh.bpr);
