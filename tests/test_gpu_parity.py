@@ -12,6 +12,8 @@ tensor.
 """
 from __future__ import annotations
 
+import time
+
 import numpy as np
 import pytest
 import torch
@@ -658,3 +660,35 @@ def test_guided_separate_outputs_many_tiles_per_cta(oracle_mod):
     ref_out, ref_mask = ot.full_guided_fwd_mt(ht, codes, scales, gscale)
     _eq("sep_many_tiles.out_full", _u(out_f), ref_out)
     _eq("sep_many_tiles.mask_full", _u(mask_f), ref_mask)
+
+
+def test_capture_grid_barrier_gives_up_and_flags(oracle_mod):
+    """The one-launch capture's grid barrier waits a bounded time.  A
+    workspace whose arrival count starts far from zero never lets any CTA
+    see itself arrive last, so nobody releases the barrier: every CTA gives
+    up after its polls (about a second), sets the workspace's error flag and
+    returns.  The call itself succeeds, the GPU stays usable, and a capture
+    with a clean workspace right after matches the oracle."""
+    x = inputs.tiny_site(901, 512, 256).x_roll
+    R, C = x.shape
+    ws = torch.zeros(ops.trace_capture_workspace_bytes(R, C, 1), dtype=torch.uint8, device=DEV)
+    w = ws.view(torch.int32)
+    w[0] = 1 << 30  # the arrival count: no CTA draws gridDim.x - 1
+    cap, _ = ops.alloc_capture(R, C, 1, DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    ops.capture(x.to(DEV), None, cap, ws)
+    torch.cuda.synchronize()
+    waited = time.perf_counter() - t0
+    print(f"grid barrier gave up after {waited:.2f} s")
+    assert int(w[2].item()) == 1, "the barrier did not report giving up"
+    assert waited < 30.0
+    ws.zero_()
+    cap, _ = ops.alloc_capture(R, C, 1, DEV)
+    ops.capture(x.to(DEV), None, cap, ws)
+    torch.cuda.synchronize()
+    assert int(w[2].item()) == 0
+    ref = oracle_mod.capture(inputs.bits(x), 1, None)
+    for name, got, want in zip(("codes", "mbits", "scales", "gscale"),
+                               (cap.codes, cap.mbits, cap.scales, cap.gscale), ref):
+        _eq(name, _u(got), want)
