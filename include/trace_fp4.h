@@ -131,7 +131,7 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
  *             at the same time).  Words: [0] an arrival count and [4, 4+G)
  *             the accumulators, both zero again after every call; [1] counts
  *             calls; [2] is set to nonzero if a CTA ever gave up waiting at
- *             the grid barrier (about a second; with the cooperative launch
+ *             the grid barrier (about two seconds; with the cooperative launch
  *             every CTA is resident, so it is not expected), in which case
  *             that call's outputs are not valid; [3] is unused.
  * One cooperative launch (every CTA resident at once, a few per SM): each

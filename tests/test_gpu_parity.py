@@ -666,7 +666,7 @@ def test_capture_grid_barrier_gives_up_and_flags(oracle_mod):
     """The one-launch capture's grid barrier waits a bounded time.  A
     workspace whose arrival count starts far from zero never lets any CTA
     see itself arrive last, so nobody releases the barrier: every CTA gives
-    up after its polls (about a second), sets the workspace's error flag and
+    up after its polls (about two seconds on B200), sets the workspace's error flag and
     returns.  The call itself succeeds, the GPU stays usable, and a capture
     with a clean workspace right after matches the oracle."""
     x = inputs.tiny_site(901, 512, 256).x_roll
