@@ -268,6 +268,7 @@ const char* trace_strerror(int status) {
     case TRACE_ERR_ALIGN: return "a pointer is not aligned as the call requires";
     case TRACE_ERR_WORKSPACE: return "workspace smaller than trace_capture_workspace_bytes()";
     case TRACE_ERR_CUDA: return "a CUDA runtime call or kernel launch failed";
+    case TRACE_ERR_TIMEOUT: return "a capture gave up waiting at its grid barrier";
     default: return "unknown status";
   }
 }
@@ -327,6 +328,20 @@ static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t n
                              (uint4*)codes, (uint32_t*)mbits, scales, gscale)
                : launch_coop(k_capture_coop<false>, grid, s, (const V8*)x, sh, offs, ws,
                              (uint4*)codes, (uint32_t*)mbits, scales, gscale);
+}
+
+int trace_capture_status(void* workspace, void* stream) {
+  if (!workspace) return TRACE_ERR_NULL;
+  if (!aligned(workspace, 4)) return TRACE_ERR_ALIGN;
+  cudaStream_t s = (cudaStream_t)stream;
+  uint32_t* flag = (uint32_t*)workspace + 2;
+  uint32_t h = 0u;
+  if (cudaMemcpyAsync(&h, flag, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return TRACE_ERR_CUDA;
+  if (h == 0u) return TRACE_OK;
+  if (cudaMemsetAsync(flag, 0, sizeof(h), s) != cudaSuccess) return TRACE_ERR_CUDA;
+  return TRACE_ERR_TIMEOUT;
 }
 
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols, int32_t num_groups,

@@ -25,6 +25,7 @@ _lock = threading.Lock()
 _lib = None
 
 TRACE_OK = 0
+TRACE_ERR_TIMEOUT = 6
 
 
 class TraceError(RuntimeError):
@@ -113,6 +114,8 @@ def library() -> ctypes.CDLL:
         lib.trace_capture_amax_accumulate.restype = ctypes.c_int
         lib.trace_capture_with_amax.argtypes = [P, i64, i64, i32, P, P, P, P, P, P, i32, P]
         lib.trace_capture_with_amax.restype = ctypes.c_int
+        lib.trace_capture_status.argtypes = [P, P]
+        lib.trace_capture_status.restype = ctypes.c_int
         _lib = lib
         return lib
 
@@ -301,6 +304,16 @@ def capture(x: torch.Tensor, offsets: torch.Tensor | None = None, out: Capture |
                   workspace, workspace.numel(), stream)
     return out
 
+
+def capture_status(workspace: torch.Tensor, stream=None) -> bool:
+    """True when no capture that used `workspace` has given up waiting at
+    its grid barrier since the last check (trace_capture_status: waits for
+    the stream, reads and clears the workspace's error word)."""
+    st = library().trace_capture_status(_p(workspace), _stream(stream))
+    if st == TRACE_ERR_TIMEOUT:
+        return False
+    _check(st, "trace_capture_status")
+    return True
 
 def guided_fq_fwd(x_train: torch.Tensor, cache: Capture, out: torch.Tensor | None = None,
                   mask: torch.Tensor | None = None, stream=None):

@@ -82,7 +82,9 @@ typedef enum {
   TRACE_ERR_SHAPE = 2,     /* rows < 0, cols <= 0, cols % 32, G < 1, size limit */
   TRACE_ERR_ALIGN = 3,     /* a pointer is not aligned as the call requires */
   TRACE_ERR_WORKSPACE = 4, /* workspace smaller than the query returned */
-  TRACE_ERR_CUDA = 5       /* a CUDA runtime call or launch failed */
+  TRACE_ERR_CUDA = 5,      /* a CUDA runtime call or launch failed */
+  TRACE_ERR_TIMEOUT = 6    /* a capture gave up waiting at its grid barrier
+                              (reported by trace_capture_status) */
 } trace_status;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -144,6 +146,16 @@ int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
                   uint8_t* codes, uint32_t* mbits, uint8_t* scales,
                   float* gscale, void* workspace, size_t workspace_bytes,
                   void* stream);
+
+/* Whether a capture that used `workspace` gave up waiting at its grid
+ * barrier: the one device-side wait of the path.  Capture is asynchronous,
+ * so it cannot return this itself; this call waits for the work queued on
+ * `stream` to finish, reads the workspace's error word (word 2), clears it
+ * and returns TRACE_ERR_TIMEOUT if it was set (the outputs of the capture(s)
+ * since the last check are then not valid), else TRACE_OK.  workspace:
+ * device, as given to trace_capture, 4-byte aligned; NULL returns
+ * TRACE_ERR_NULL.  Not for use during stream capture (it synchronises). */
+int trace_capture_status(void* workspace, void* stream);
 
 /* Guided QAT fake-quant forward (the QAT-forward half of the listing):
  * z = clip(x_train / (s_g*s_b), -6, 6) with the ROLLOUT's scales; of the two

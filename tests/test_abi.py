@@ -51,7 +51,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_version_and_strings(lib):
     assert lib.trace_abi_version() == 2
-    for st in range(6):
+    for st in range(7):
         assert lib.trace_strerror(st)
     assert b"unknown" in lib.trace_strerror(99)
 
@@ -156,6 +156,9 @@ def test_host_argument_checks_newer_calls(lib):
     assert lib.trace_capture_amax_accumulate(a, 4, 32, 1, None, odd, None) == 3
     assert lib.trace_capture_with_amax(a, 4, 32, 1, None, a, a, a, a, a, 9, None) == 2
     assert lib.trace_capture_with_amax(a, 4, 32, 1, None, None, a, a, a, a, 0, None) == 1
+    # capture status: NULL / misaligned workspace
+    assert lib.trace_capture_status(None, None) == 1
+    assert lib.trace_capture_status(P((1 << 20) + 2), None) == 3
     # no-workspace capture: too many groups
     assert lib.trace_capture_static_ws(a, 4, 32, 4097, a, a, a, a, a, None) == 4
     # self-test range: must stay below +inf

@@ -683,11 +683,13 @@ def test_capture_grid_barrier_gives_up_and_flags(oracle_mod):
     print(f"grid barrier gave up after {waited:.2f} s")
     assert int(w[2].item()) == 1, "the barrier did not report giving up"
     assert waited < 30.0
+    assert ops.capture_status(ws) is False  # TRACE_ERR_TIMEOUT, and the word is cleared
+    assert int(w[2].item()) == 0
     ws.zero_()
     cap, _ = ops.alloc_capture(R, C, 1, DEV)
     ops.capture(x.to(DEV), None, cap, ws)
     torch.cuda.synchronize()
-    assert int(w[2].item()) == 0
+    assert int(w[2].item()) == 0 and ops.capture_status(ws) is True
     ref = oracle_mod.capture(inputs.bits(x), 1, None)
     for name, got, want in zip(("codes", "mbits", "scales", "gscale"),
                                (cap.codes, cap.mbits, cap.scales, cap.gscale), ref):
