@@ -332,13 +332,6 @@ __device__ __forceinline__ float le448_step(float z) {
   return r;
 }
 
-// 0xFFFFFFFF when a <= b (false for NaN), else 0.
-__device__ __forceinline__ uint32_t le_mask(float a, float b) {
-  uint32_t r;
-  asm("set.le.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
-  return r;
-}
-
 __device__ __forceinline__ bool fast_scale(float d, uint32_t dmax_bits = kDMax) {
   const uint32_t db = __float_as_uint(d);
   return db >= kDMin && db <= dmax_bits;
