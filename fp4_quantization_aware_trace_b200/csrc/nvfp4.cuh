@@ -404,6 +404,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __shared__ uint32_t table[kAmaxTable];
   __shared__ int g_first_s;
   __shared__ uint32_t gen_s, last_s, ok_s;
+  pdl_begin();
   uint32_t* const cnt = ws;
   uint32_t* const gen = ws + 1;
   uint32_t* const err = ws + 2;

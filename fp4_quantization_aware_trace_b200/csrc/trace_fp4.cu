@@ -214,7 +214,11 @@ int mx8_launch(const uint16_t* x, int64_t rows, int64_t cols, const uint32_t* mb
 }
 
 // A cooperative launch (every CTA resident at once; the one-launch capture's
-// grid barrier relies on it).
+// grid barrier relies on it), with programmatic stream serialization as the
+// other launches: the grid may be launched while the previous kernel
+// drains (it waits for it before touching memory).  Every kernel of the
+// library triggers its dependents at its start, so when this grid is
+// launched every CTA of the previous kernel has already started.
 template <typename... KArgs, typename... Args>
 int launch_coop(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args) {
   cudaLaunchConfig_t cfg = {};
@@ -222,11 +226,13 @@ int launch_coop(void (*kernel)(KArgs...), int grid, cudaStream_t s, Args... args
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) == cudaSuccess ? TRACE_OK
                                                                                       : TRACE_ERR_CUDA;
 }
