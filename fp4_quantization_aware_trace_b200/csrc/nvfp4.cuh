@@ -384,27 +384,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // ---------------------------------------------------------------------------
 // Kernel 2': capture in one launch.  A cooperative grid (every CTA resident
-// at once, at most a few per SM): each CTA reduces the amax of its tiles
-// into the accumulators, the CTAs meet at a grid barrier, and the CTAs then
-// quantise the tiles, the last read first (in L2 on tensors that fit there).
-// The barrier's last arriving CTA takes each group's final amax, zeroes its
-// accumulator, writes s_g to gscale and releases the others, which read
-// their constants from gscale.
-// Which CTA takes which tile: with groups, one contiguous range of tiles per
-// CTA in both phases, so that a CTA meets few groups.  With one group (no
-// such constraint), the CTAs finish each phase together however DRAM serves
-// them: in the amax phase each CTA takes tiles blockIdx.x + k * gridDim.x for
-// k < 3 and then claims tiles from a counter; the quantising phase claims
-// tiles from another counter, highest tile first.
+// at once, at most a few per SM): each CTA reduces the amax of its tiles --
+// one contiguous range of tiles per CTA, so that a CTA meets few groups --
+// into the accumulators, the CTAs meet at a grid barrier, and each CTA then
+// quantises the same tiles in reverse order, so that it starts on what it
+// read last (in L2 on tensors that fit there).  The barrier's last arriving
+// CTA takes each group's final amax, zeroes its accumulator, writes s_g to
+// gscale and releases the others, which read their constants from gscale.
 // Workspace (u32): [0] arrival count (zero between calls), [1] generation
-// (counts calls), [2] error flag (set if a CTA gave up waiting), [3] the amax
-// phase's tile counter (zero between calls), [4], [5] the quantising phase's
-// tile counters, one per parity of the generation (a call uses the one the
-// call before reset), [6], [7] unused, [8, 8 + G) the accumulators (zero
-// between calls).
+// (counts calls), [2] error flag (set if a CTA gave up waiting), [3] unused,
+// [4, 4 + G) the accumulators (zero between calls).
 // ---------------------------------------------------------------------------
-constexpr int kWsHeader = 8;
-
 template <bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture_coop(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
@@ -413,41 +403,33 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
                    float* __restrict__ gscale) {
   __shared__ uint32_t table[kAmaxTable];
   __shared__ int g_first_s;
-  __shared__ uint32_t gen_s, last_s, ok_s, first2_s;
-  __shared__ uint32_t q_s[2];
+  __shared__ uint32_t gen_s, last_s, ok_s;
   pdl_begin();
   uint32_t* const cnt = ws;
   uint32_t* const gen = ws + 1;
   uint32_t* const err = ws + 2;
-  uint32_t* const ctr1 = ws + 3;
-  uint32_t* const acc = ws + kWsHeader;
-  const bool one = sh.G == 1;
-  const uint32_t grid = gridDim.x;
-  // groups: this CTA's tiles [t0, t1), nonempty when there are tiles (the
-  // grid has at most one CTA per tile); one group: every tile is open to
-  // every CTA
-  const uint32_t t0 = one ? 0u : (uint32_t)((uint64_t)blockIdx.x * sh.ntiles / grid);
-  const uint32_t t1 = one ? sh.ntiles : (uint32_t)((uint64_t)(blockIdx.x + 1u) * sh.ntiles / grid);
+  uint32_t* const acc = ws + 4;
+  // this CTA's tiles: [t0, t1), nonempty when there are tiles (the grid has
+  // at most one CTA per tile)
+  const uint32_t t0 = (uint32_t)((uint64_t)blockIdx.x * sh.ntiles / gridDim.x);
+  const uint32_t t1 = (uint32_t)((uint64_t)(blockIdx.x + 1u) * sh.ntiles / gridDim.x);
 
-  // ---- phase 1: amax, three tiles in flight per thread (the quantising
-  // phase sets the register budget, so they cost no occupancy); the first
-  // loads go out before the set-up
+  // ---- phase 1: amax of the CTA's tiles, three in flight per thread (the
+  // quantising phase sets the register budget, so they cost no occupancy);
+  // the first loads go out before the set-up
   V8 a0, a1, b0, b1, c0, c1;
   auto load = [&](uint32_t t, V8& v0, V8& v1) {
     const uint32_t b = t * kTileBlks + threadIdx.x;
-    v0 = (t >= t0 && t < t1 && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
-    v1 = (t >= t0 && t < t1 && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads)
-                                                       : zero_block();
+    v0 = (t < t1 && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
+    v1 = (t < t1 && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads) : zero_block();
   };
-  uint32_t ta = one ? blockIdx.x : t0, tb = one ? ta + grid : t0 + 1u,
-           tc = one ? ta + 2u * grid : t0 + 2u;
-  load(ta, a0, a1);
-  load(tb, b0, b1);
-  load(tc, c0, c1);
+  load(t0, a0, a1);
+  load(t0 + 1u, b0, b1);
+  load(t0 + 2u, c0, c1);
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (threadIdx.x == 0) gen_s = ld_acquire_gpu(gen);  // before this CTA's arrival
-  if (!one) {
+  if (sh.G > 1) {
     if (threadIdx.x == 0) {
       gc.seek(t0 < t1 ? fastdiv(t0 * kTileBlks, sh.bpr) : 0u);
       g_first_s = gc.g;
@@ -459,11 +441,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   __syncthreads();
   const int g_first = g_first_s;
-  // the quantising phase's counter of this call: the call before reset it
-  uint32_t* const ctr2 = ws + 4 + (gen_s & 1u);
   gc.init(offs, sh.G);
   uint32_t run = 0u;
-  int run_g = one ? 0 : -1;
+  int run_g = sh.G > 1 ? -1 : 0;
   auto flush = [&](int g, uint32_t val) {
     if (g < 0 || val == 0u) return;
     const int slot = g - g_first;
@@ -471,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     else atomicMax(&acc[g], val);
   };
   auto take = [&](uint32_t t, const V8& v0, const V8& v1) {
-    if (one) {  // blocks past the end were loaded as zeros
+    if (sh.G == 1) {  // blocks past the end were loaded as zeros
       run = max(run, max(absmax_block(v0), absmax_block(v1)));
       return;
     }
@@ -489,60 +469,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       run = max(run, absmax_block(u == 0 ? v0 : v1));
     }
   };
-  if (one) {
-    // after its three first tiles a CTA claims tile 3 * gridDim.x + c, c
-    // from the counter; thread 0 holds one claim ahead, whose result it
-    // reads only after a tile's work, and a barrier hands each claim to the
-    // CTA (two slots, alternating).  Claims rise, so the first tile at or
-    // past the end ends the phase for the CTA.
-    uint32_t pend = 0u;
-    if (threadIdx.x == 0) pend = atomicAdd(ctr1, 1u);
-    const uint32_t base = 3u * grid;
-    int slot = 0;
-    auto next = [&]() {
-      if (threadIdx.x == 0) {
-        q_s[slot] = base + pend;
-        pend = atomicAdd(ctr1, 1u);
-      }
-      __syncthreads();
-      const uint32_t t = q_s[slot];
-      slot ^= 1;
-      return t;
-    };
-    for (;;) {
-      if (ta >= sh.ntiles) break;
-      take(ta, a0, a1);
-      ta = next();
-      load(ta, a0, a1);
-      if (tb >= sh.ntiles) break;
-      take(tb, b0, b1);
-      tb = next();
-      load(tb, b0, b1);
-      if (tc >= sh.ntiles) break;
-      take(tc, c0, c1);
-      tc = next();
-      load(tc, c0, c1);
-    }
-  } else {
-    for (uint32_t t = t0; t < t1; t += 3u) {
-      take(t, a0, a1);
-      load(t + 3u, a0, a1);
-      if (t + 1u >= t1) break;
-      take(t + 1u, b0, b1);
-      load(t + 4u, b0, b1);
-      if (t + 2u >= t1) break;
-      take(t + 2u, c0, c1);
-      load(t + 5u, c0, c1);
-    }
+  for (uint32_t t = t0; t < t1; t += 3u) {
+    take(t, a0, a1);
+    load(t + 3u, a0, a1);
+    if (t + 1u >= t1) break;
+    take(t + 1u, b0, b1);
+    load(t + 4u, b0, b1);
+    if (t + 2u >= t1) break;
+    take(t + 2u, c0, c1);
+    load(t + 5u, c0, c1);
   }
-  if (one) {
+  if (sh.G == 1) {
     run = __reduce_max_sync(0xFFFFFFFFu, run);
     if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
   } else {
     flush(run_g, run);
   }
   __syncthreads();
-  if (one) {
+  if (sh.G == 1) {
     if (threadIdx.x == 0 && table[0]) atomicMax(&acc[0], table[0]);
   } else {
     for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
@@ -551,29 +495,21 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
 
-  // the quantising phase's first tile is known (and loaded) before the
-  // barrier, so that the wait covers its latency; x is not written by this
-  // kernel.  One group: tile ntiles - 1 - c for a claim c; groups: the last
-  // tile of the CTA's range.
-  uint32_t pend2 = 0u;
-  if (one && threadIdx.x == 0) {
-    first2_s = atomicAdd(ctr2, 1u);
-    pend2 = atomicAdd(ctr2, 1u);
+  // phase 2's first tile (the last one read) is loaded before the barrier,
+  // so that the wait covers its latency; x is not written by this kernel
+  const uint32_t ntile_cta = t1 - t0;
+  auto tile_base = [&](uint32_t k) { return (t0 + k) * kTileBlks + 2u * threadIdx.x; };
+  V8 v0 = zero_block(), v1 = zero_block();
+  if (ntile_cta > 0u && tile_base(ntile_cta - 1u) < sh.nblk) {
+    v0 = ld_block_stream(x + tile_base(ntile_cta - 1u));
+    v1 = ld_block_stream(x + tile_base(ntile_cta - 1u) + 1);
   }
-  auto tile2 = [&](uint32_t c) { return c < sh.ntiles ? sh.ntiles - 1u - c : 0xFFFFFFFFu; };
 
   // ---- grid barrier
-  __threadfence();  // this thread's maxima and claims before the CTA's arrival
+  __threadfence();  // this thread's maxima before the CTA's arrival
   __syncthreads();
-  uint32_t t2 = one ? tile2(first2_s) : (t0 < t1 ? t1 - 1u : 0xFFFFFFFFu);
-  auto tile_base = [&](uint32_t t) { return t * kTileBlks + 2u * threadIdx.x; };
-  V8 v0 = zero_block(), v1 = zero_block();
-  if (t2 != 0xFFFFFFFFu && tile_base(t2) < sh.nblk) {
-    v0 = ld_block_stream(x + tile_base(t2));
-    v1 = ld_block_stream(x + tile_base(t2) + 1);
-  }
   if (threadIdx.x == 0) {
-    last_s = atomicAdd(cnt, 1u) == grid - 1u;
+    last_s = atomicAdd(cnt, 1u) == gridDim.x - 1u;
     ok_s = 1u;
   }
   __syncthreads();
@@ -588,9 +524,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncthreads();
     if (threadIdx.x == 0) {
       *cnt = 0u;
-      *ctr1 = 0u;                        // every CTA has made its last claim
-      ws[4 + ((gen_s + 1u) & 1u)] = 0u;  // the next call's counter (the call before used it)
-      __threadfence();  // the global scales and the resets before the release
+      __threadfence();  // the global scales and the reset before the release
       st_release_gpu(gen, gen_s + 1u);
     }
   } else if (threadIdx.x == 0) {
@@ -607,12 +541,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
   if (!ok_s) return;
 
-  // ---- phase 2: quantise, two adjacent blocks per thread
+  // ---- phase 2: quantise the same tiles, last first; two adjacent blocks
+  // per thread
   gc.init(offs, sh.G);
   GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
-  int slot2 = 0;
-  while (t2 != 0xFFFFFFFFu) {
-    const uint32_t b = tile_base(t2);  // even; nblk is even
+  for (uint32_t k = ntile_cta; k-- > 0u;) {
+    const uint32_t b = tile_base(k);  // even; nblk is even
     if (b < sh.nblk) {
       const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
       if (gc.seek(row)) gk = group_consts_of_sg(__ldcg(gscale + gc.g));
@@ -636,20 +570,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       else
         reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
     }
-    if (one) {
-      if (threadIdx.x == 0) {
-        q_s[slot2] = pend2;
-        pend2 = atomicAdd(ctr2, 1u);
-      }
-      __syncthreads();
-      t2 = tile2(q_s[slot2]);
-      slot2 ^= 1;
-    } else {
-      t2 = t2 > t0 ? t2 - 1u : 0xFFFFFFFFu;
-    }
-    if (t2 != 0xFFFFFFFFu && tile_base(t2) < sh.nblk) {
-      v0 = ld_block_stream(x + tile_base(t2));
-      v1 = ld_block_stream(x + tile_base(t2) + 1);
+    if (k > 0u && tile_base(k - 1u) < sh.nblk) {
+      v0 = ld_block_stream(x + tile_base(k - 1u));
+      v1 = ld_block_stream(x + tile_base(k - 1u) + 1);
     }
   }
 }
