@@ -384,31 +384,17 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
 // ---------------------------------------------------------------------------
 // Kernel 2': capture in one launch.  A cooperative grid (every CTA resident
-// at once, at most a few per SM): the CTAs reduce the amax of their tiles
-// into the accumulators, meet at a grid barrier, and quantise the tiles, the
-// last read first (in L2 on tensors that fit there).  The barrier's last
-// arriving CTA takes each group's final amax, zeroes its accumulator, writes
-// s_g to gscale and releases the others, which read their constants from
-// gscale.
-// Who takes which tile: with groups, one contiguous range of tiles per CTA in
-// both phases, so that a CTA meets few groups.  With one group the warps
-// take tiles themselves, so that they finish each phase together however
-// DRAM serves them: a warp walks a tile as 8 steps of 64 blocks (two
-// adjacent blocks per lane); in the amax phase warp w of the grid takes
-// tile w first and then tiles claimed from a counter, in the quantising
-// phase every tile is claimed from a second counter, highest tile first.
-// Lane 0 holds the next claim while the warp walks the current tile, so no
-// claim is waited for and no CTA barrier is involved.
+// at once, at most a few per SM): each CTA reduces the amax of its tiles --
+// one contiguous range of tiles per CTA, so that a CTA meets few groups --
+// into the accumulators, the CTAs meet at a grid barrier, and each CTA then
+// quantises the same tiles in reverse order, so that it starts on what it
+// read last (in L2 on tensors that fit there).  The barrier's last arriving
+// CTA takes each group's final amax, zeroes its accumulator, writes s_g to
+// gscale and releases the others, which read their constants from gscale.
 // Workspace (u32): [0] arrival count (zero between calls), [1] generation
-// (counts calls), [2] error flag (set if a CTA gave up waiting), [3] the amax
-// phase's tile counter (zero between calls), [4], [5] the quantising phase's
-// tile counters, one per parity of the generation (a call uses the one the
-// call before reset), [6], [7] unused, [8, 8 + G) the accumulators (zero
-// between calls).
+// (counts calls), [2] error flag (set if a CTA gave up waiting), [3] unused,
+// [4, 4 + G) the accumulators (zero between calls).
 // ---------------------------------------------------------------------------
-constexpr int kWsHeader = 8;
-constexpr uint32_t kNoTile = 0xFFFFFFFFu;
-
 template <bool SW>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     k_capture_coop(const V8* __restrict__ x, Shape sh, const int64_t* __restrict__ offs,
@@ -422,58 +408,28 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   uint32_t* const cnt = ws;
   uint32_t* const gen = ws + 1;
   uint32_t* const err = ws + 2;
-  uint32_t* const ctr1 = ws + 3;
-  uint32_t* const acc = ws + kWsHeader;
-  const bool one = sh.G == 1;
-  const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t nwarps = gridDim.x * (kThreads / 32);
-  const uint32_t gw = blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);  // warp of the grid
-  // groups: this CTA's tiles [t0, t1), nonempty when there are tiles (the
-  // grid has at most one CTA per tile)
-  const uint32_t t0 = one ? 0u : (uint32_t)((uint64_t)blockIdx.x * sh.ntiles / gridDim.x);
-  const uint32_t t1 = one ? sh.ntiles : (uint32_t)((uint64_t)(blockIdx.x + 1u) * sh.ntiles / gridDim.x);
+  uint32_t* const acc = ws + 4;
+  // this CTA's tiles: [t0, t1), nonempty when there are tiles (the grid has
+  // at most one CTA per tile)
+  const uint32_t t0 = (uint32_t)((uint64_t)blockIdx.x * sh.ntiles / gridDim.x);
+  const uint32_t t1 = (uint32_t)((uint64_t)(blockIdx.x + 1u) * sh.ntiles / gridDim.x);
 
-  // ---- phase 1: amax
-  // One group, a warp's walk: step j (0-7) of tile t covers blocks
-  // t * 512 + 64 j + 2 lane and the one after.  `ticket` (lane 0): the
-  // claim for the tile after the current one, issued when the current one
-  // was entered and read when it is left.
-  uint32_t w_tile = gw < sh.ntiles ? gw : kNoTile, w_step = 0u, ticket = 0u;
-  if (one && w_tile != kNoTile && lane == 0u) ticket = atomicAdd(ctr1, 1u);
-  auto walk_load = [&](V8& v0, V8& v1) -> bool {  // the warp's next step, loaded
-    if (w_tile == kNoTile) return false;
-    const uint32_t b = w_tile * kTileBlks + 64u * w_step + 2u * lane;
-    v0 = b < sh.nblk ? ld_block_stream(x + b) : zero_block();
-    v1 = b + 1u < sh.nblk ? ld_block_stream(x + b + 1) : zero_block();
-    if (++w_step == 8u) {
-      w_step = 0u;
-      const uint32_t c = __shfl_sync(0xFFFFFFFFu, ticket, 0);
-      w_tile = nwarps + c < sh.ntiles ? nwarps + c : kNoTile;
-      if (w_tile != kNoTile && lane == 0u) ticket = atomicAdd(ctr1, 1u);
-    }
-    return true;
-  };
-  // groups: the CTA's range, three tiles in flight per thread
+  // ---- phase 1: amax of the CTA's tiles, three in flight per thread (the
+  // quantising phase sets the register budget, so they cost no occupancy);
+  // the first loads go out before the set-up
   V8 a0, a1, b0, b1, c0, c1;
   auto load = [&](uint32_t t, V8& v0, V8& v1) {
     const uint32_t b = t * kTileBlks + threadIdx.x;
     v0 = (t < t1 && b < sh.nblk) ? ld_block_stream(x + b) : zero_block();
     v1 = (t < t1 && b + kThreads < sh.nblk) ? ld_block_stream(x + b + kThreads) : zero_block();
   };
-  bool ha = false, hb = false, hc = false;
-  if (one) {
-    ha = walk_load(a0, a1);
-    hb = walk_load(b0, b1);
-    hc = walk_load(c0, c1);
-  } else {
-    load(t0, a0, a1);
-    load(t0 + 1u, b0, b1);
-    load(t0 + 2u, c0, c1);
-  }
+  load(t0, a0, a1);
+  load(t0 + 1u, b0, b1);
+  load(t0 + 2u, c0, c1);
   GroupCursor gc;
   gc.init(offs, sh.G);
   if (threadIdx.x == 0) gen_s = ld_acquire_gpu(gen);  // before this CTA's arrival
-  if (!one) {
+  if (sh.G > 1) {
     if (threadIdx.x == 0) {
       gc.seek(t0 < t1 ? fastdiv(t0 * kTileBlks, sh.bpr) : 0u);
       g_first_s = gc.g;
@@ -485,11 +441,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
   __syncthreads();
   const int g_first = g_first_s;
-  // the quantising phase's counter of this call: the call before reset it
-  uint32_t* const ctr2 = ws + 4 + (gen_s & 1u);
   gc.init(offs, sh.G);
   uint32_t run = 0u;
-  int run_g = one ? 0 : -1;
+  int run_g = sh.G > 1 ? -1 : 0;
   auto flush = [&](int g, uint32_t val) {
     if (g < 0 || val == 0u) return;
     const int slot = g - g_first;
@@ -497,6 +451,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     else atomicMax(&acc[g], val);
   };
   auto take = [&](uint32_t t, const V8& v0, const V8& v1) {
+    if (sh.G == 1) {  // blocks past the end were loaded as zeros
+      run = max(run, max(absmax_block(v0), absmax_block(v1)));
+      return;
+    }
     const uint32_t b = t * kTileBlks + threadIdx.x;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -511,40 +469,24 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       run = max(run, absmax_block(u == 0 ? v0 : v1));
     }
   };
-  if (one) {
-    // steps come out in the order they were loaded; once the walk has
-    // ended every later load reports it too
-    for (;;) {
-      if (!ha) break;
-      run = max(run, max(absmax_block(a0), absmax_block(a1)));
-      ha = walk_load(a0, a1);
-      if (!hb) break;
-      run = max(run, max(absmax_block(b0), absmax_block(b1)));
-      hb = walk_load(b0, b1);
-      if (!hc) break;
-      run = max(run, max(absmax_block(c0), absmax_block(c1)));
-      hc = walk_load(c0, c1);
-    }
-  } else {
-    for (uint32_t t = t0; t < t1; t += 3u) {
-      take(t, a0, a1);
-      load(t + 3u, a0, a1);
-      if (t + 1u >= t1) break;
-      take(t + 1u, b0, b1);
-      load(t + 4u, b0, b1);
-      if (t + 2u >= t1) break;
-      take(t + 2u, c0, c1);
-      load(t + 5u, c0, c1);
-    }
+  for (uint32_t t = t0; t < t1; t += 3u) {
+    take(t, a0, a1);
+    load(t + 3u, a0, a1);
+    if (t + 1u >= t1) break;
+    take(t + 1u, b0, b1);
+    load(t + 4u, b0, b1);
+    if (t + 2u >= t1) break;
+    take(t + 2u, c0, c1);
+    load(t + 5u, c0, c1);
   }
-  if (one) {
+  if (sh.G == 1) {
     run = __reduce_max_sync(0xFFFFFFFFu, run);
     if ((threadIdx.x & 31) == 0 && run) atomicMax(&table[0], run);
   } else {
     flush(run_g, run);
   }
   __syncthreads();
-  if (one) {
+  if (sh.G == 1) {
     if (threadIdx.x == 0 && table[0]) atomicMax(&acc[0], table[0]);
   } else {
     for (int i = threadIdx.x; i < kAmaxTable; i += kThreads) {
@@ -553,46 +495,18 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     }
   }
 
-  // ---- the quantising phase's first step is known (and loaded) before the
-  // barrier, so that the wait covers its latency; x is not written by this
-  // kernel.  One group: a warp walks tiles ntiles - 1 - c for its claims c,
-  // each from step 7 down to 0; groups: the CTA's range, last tile first.
-  uint32_t q_tile = kNoTile, q_step = 7u;
-  if (one) {
-    uint32_t c = 0u;
-    if (lane == 0u) c = atomicAdd(ctr2, 1u);
-    c = __shfl_sync(0xFFFFFFFFu, c, 0);
-    q_tile = c < sh.ntiles ? sh.ntiles - 1u - c : kNoTile;
-    if (q_tile != kNoTile && lane == 0u) ticket = atomicAdd(ctr2, 1u);
-  } else {
-    q_tile = t0 < t1 ? t1 - 1u : kNoTile;
-  }
-  // block of the current phase-2 step
-  auto q_block = [&]() {
-    return one ? q_tile * kTileBlks + 64u * q_step + 2u * lane
-               : q_tile * kTileBlks + 2u * threadIdx.x;
-  };
-  // move to the next phase-2 step (warp- or CTA-uniform)
-  auto q_advance = [&]() {
-    if (one) {
-      if (q_step-- == 0u) {
-        q_step = 7u;
-        const uint32_t c = __shfl_sync(0xFFFFFFFFu, ticket, 0);
-        q_tile = c < sh.ntiles ? sh.ntiles - 1u - c : kNoTile;
-        if (q_tile != kNoTile && lane == 0u) ticket = atomicAdd(ctr2, 1u);
-      }
-    } else {
-      q_tile = q_tile > t0 ? q_tile - 1u : kNoTile;
-    }
-  };
+  // phase 2's first tile (the last one read) is loaded before the barrier,
+  // so that the wait covers its latency; x is not written by this kernel
+  const uint32_t ntile_cta = t1 - t0;
+  auto tile_base = [&](uint32_t k) { return (t0 + k) * kTileBlks + 2u * threadIdx.x; };
   V8 v0 = zero_block(), v1 = zero_block();
-  if (q_tile != kNoTile && q_block() < sh.nblk) {
-    v0 = ld_block_stream(x + q_block());
-    v1 = ld_block_stream(x + q_block() + 1);
+  if (ntile_cta > 0u && tile_base(ntile_cta - 1u) < sh.nblk) {
+    v0 = ld_block_stream(x + tile_base(ntile_cta - 1u));
+    v1 = ld_block_stream(x + tile_base(ntile_cta - 1u) + 1);
   }
 
   // ---- grid barrier
-  __threadfence();  // this thread's maxima and claims before the CTA's arrival
+  __threadfence();  // this thread's maxima before the CTA's arrival
   __syncthreads();
   if (threadIdx.x == 0) {
     last_s = atomicAdd(cnt, 1u) == gridDim.x - 1u;
@@ -610,9 +524,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     __syncthreads();
     if (threadIdx.x == 0) {
       *cnt = 0u;
-      *ctr1 = 0u;                        // every warp has made its last claim
-      ws[4 + ((gen_s + 1u) & 1u)] = 0u;  // the next call's counter (the call before used it)
-      __threadfence();  // the global scales and the resets before the release
+      __threadfence();  // the global scales and the reset before the release
       st_release_gpu(gen, gen_s + 1u);
     }
   } else if (threadIdx.x == 0) {
@@ -629,11 +541,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __syncthreads();
   if (!ok_s) return;
 
-  // ---- phase 2: quantise, two adjacent blocks per thread
+  // ---- phase 2: quantise the same tiles, last first; two adjacent blocks
+  // per thread
   gc.init(offs, sh.G);
   GroupK gk = {1.0f, 6.0f, 0.0f, false};  // set at the first block (seek)
-  while (q_tile != kNoTile) {
-    const uint32_t b = q_block();  // even; nblk is even
+  for (uint32_t k = ntile_cta; k-- > 0u;) {
+    const uint32_t b = tile_base(k);  // even; nblk is even
     if (b < sh.nblk) {
       const uint32_t row = (SW || sh.G > 1) ? fastdiv(b, sh.bpr) : 0u;
       if (gc.seek(row)) gk = group_consts_of_sg(__ldcg(gscale + gc.g));
@@ -657,10 +570,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       else
         reinterpret_cast<uint16_t*>(scales)[b >> 1] = sv;
     }
-    q_advance();
-    if (q_tile != kNoTile && q_block() < sh.nblk) {
-      v0 = ld_block_stream(x + q_block());
-      v1 = ld_block_stream(x + q_block() + 1);
+    if (k > 0u && tile_base(k - 1u) < sh.nblk) {
+      v0 = ld_block_stream(x + tile_base(k - 1u));
+      v1 = ld_block_stream(x + tile_base(k - 1u) + 1);
     }
   }
 }

@@ -283,9 +283,9 @@ int trace_abi_version(void) { return TRACE_ABI_VERSION; }
 
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols, int32_t num_groups) {
   if (rows < 0 || cols <= 0 || cols % 32 != 0 || num_groups < 1) return 0;
-  // eight words of the one-launch capture's state (arrival count,
-  // generation, error flag, tile counters), then the G accumulators
-  return ((size_t)num_groups * 4u + 4u * (size_t)kWsHeader + 255u) / 256u * 256u;
+  // an arrival count, a generation, an error flag, one unused word, then
+  // the G accumulators
+  return ((size_t)num_groups * 4u + 16u + 255u) / 256u * 256u;
 }
 
 size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
@@ -327,7 +327,7 @@ static int capture_impl(const uint16_t* x, int64_t rows, int64_t cols, int32_t n
   cudaStream_t s = (cudaStream_t)stream;
   uint32_t* ws = (uint32_t*)workspace;
   const int64_t* offs = num_groups > 1 ? group_row_offsets : nullptr;
-  const int zn = (int)num_groups + kWsHeader;
+  const int zn = (int)num_groups + 4;
   const int zg = (zn + kThreads - 1) / kThreads;
   if (zero_first && (st = launch(k_zero_u32, zg < 1024 ? zg : 1024, s, ws, zn))) return st;
   return tiled ? launch_coop(k_capture_coop<true>, grid, s, (const V8*)x, sh, offs, ws,
@@ -787,7 +787,7 @@ int trace_copy_bf16_staged(const uint16_t* src, uint16_t* dst, int64_t numel, ui
 // that trace_capture takes as `workspace` in a fixed array that lives in the
 // library itself, one copy per GPU, for the life of the process.
 // ---------------------------------------------------------------------------
-// TRACE_STATIC_MAX_GROUPS accumulators, the eight words before them and
+// TRACE_STATIC_MAX_GROUPS accumulators, the four words before them and
 // padding to a multiple of 256 bytes
 static __device__ __align__(256) uint32_t g_capture_scratch[TRACE_STATIC_MAX_GROUPS + 64];
 

@@ -94,10 +94,9 @@ const char* trace_strerror(int status);
 #define TRACE_ABI_VERSION 2
 int trace_abi_version(void);
 
-/* Bytes of device workspace that trace_capture needs for G groups: eight
- * words of state (grid barrier, tile counters), then the per-group amax
- * accumulators (4 bytes each), rounded up to 256.  Returns 0 when the shape
- * is invalid. */
+/* Bytes of device workspace that trace_capture needs for G groups: four
+ * words of grid-barrier state, then the per-group amax accumulators (4 bytes
+ * each), rounded up to 256.  Returns 0 when the shape is invalid. */
 size_t trace_capture_workspace_bytes(int64_t rows, int64_t cols,
                                      int32_t num_groups);
 
@@ -131,21 +130,17 @@ size_t trace_cache_record_bytes(int64_t rows, int64_t cols, int32_t num_groups,
  *             (e.g. cudaMemsetAsync once, when it is allocated); every call
  *             leaves it ready for the next, so a workspace can serve any
  *             number of calls one after another (not two calls that may run
- *             at the same time).  Words: [0] an arrival count, [3] a tile
- *             counter and [8, 8+G) the accumulators, all zero again after
- *             every call; [1] counts calls; [2] is set to nonzero if a CTA
- *             ever gave up waiting at the grid barrier (about two seconds;
- *             with the cooperative launch every CTA is resident, so it is not
- *             expected), in which case that call's outputs are not valid;
- *             [4], [5] tile counters that alternate between calls; [6], [7]
- *             unused.
- * One cooperative launch (every CTA resident at once, a few per SM): the
- * CTAs max-accumulate the amax of their tiles into the workspace, meet at a
- * grid barrier whose last arriving CTA writes gscale and zeroes the
- * accumulators, and quantise the tiles, the last read first (from L2 where
- * the tensor fits there).  With one group the CTAs take tiles from counters
- * in the workspace, so that they finish each phase together; with groups
- * each CTA keeps one contiguous range of tiles. */
+ *             at the same time).  Words: [0] an arrival count and [4, 4+G)
+ *             the accumulators, both zero again after every call; [1] counts
+ *             calls; [2] is set to nonzero if a CTA ever gave up waiting at
+ *             the grid barrier (about two seconds; with the cooperative launch
+ *             every CTA is resident, so it is not expected), in which case
+ *             that call's outputs are not valid; [3] is unused.
+ * One cooperative launch (every CTA resident at once, a few per SM): each
+ * CTA max-accumulates the amax of its tiles into the workspace, the CTAs
+ * meet at a grid barrier whose last arriving CTA writes gscale and zeroes
+ * the accumulators, and each CTA then quantises its own tiles, last read
+ * first (from L2 where the tensor fits there). */
 int trace_capture(const uint16_t* x, int64_t rows, int64_t cols,
                   int32_t num_groups, const int64_t* group_row_offsets,
                   uint8_t* codes, uint32_t* mbits, uint8_t* scales,

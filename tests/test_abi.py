@@ -57,11 +57,11 @@ def test_version_and_strings(lib):
 
 
 def test_workspace_query(lib):
-    # eight words of state and G accumulators, 4 bytes each, in 256-byte
-    # units
+    # four words of barrier state and G accumulators, 4 bytes each, in
+    # 256-byte units
     assert ops.trace_capture_workspace_bytes(16, 32, 1) == 256
-    assert ops.trace_capture_workspace_bytes(16, 32, 56) == 256
-    assert ops.trace_capture_workspace_bytes(16, 32, 57) == 512
+    assert ops.trace_capture_workspace_bytes(16, 32, 60) == 256
+    assert ops.trace_capture_workspace_bytes(16, 32, 61) == 512
     assert ops.trace_capture_workspace_bytes(16, 32, 4096) == 16640
     assert ops.trace_capture_workspace_bytes(16, 33, 1) == 0
     assert ops.trace_capture_workspace_bytes(16, 32, 0) == 0
